@@ -1,0 +1,598 @@
+/*
+ * oracle.c -- float64 CPU oracle for per-row L2 normalisation.
+ *
+ * TEST INFRASTRUCTURE ONLY (see oracle.h): loaded by the tests, the smoke
+ * check and the benchmark's CPU-baseline leg, never by the product path.
+ *
+ * Build: gcc -O2 -ffp-contract=off -fno-fast-math -fPIC -shared -pthread
+ * (oracle/build.py).  No FMA contraction, no fast-math: each line below is
+ * one IEEE double operation in the order written.
+ */
+#include "oracle.h"
+
+#include <math.h>
+#include <pthread.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* bf16: 1 sign bit, 8 exponent bits (bias 127), 7 fraction bits.  A finite
+ * non-zero bf16 is m * 2^q with q = E - 7 in the binade [2^E, 2^(E+1)) for
+ * E >= -126, and q = -133 below 2^-126 (subnormals).  Rounding a double to
+ * bf16 is: count the quanta of its binade, round that count to the nearest
+ * integer with ties to even (rint under the default rounding mode), and
+ * rebuild.  Results at or above 2^128 overflow to infinity.                 */
+
+uint16_t or_bf16_rne(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v))
+        return (uint16_t)(sign | 0x7FC0u);
+    double a = fabs(v);
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7F80u);
+    if (a == 0.0)
+        return sign;
+
+    int e;
+    (void)frexp(a, &e);             /* a in [2^(e-1), 2^e) */
+    int E = e - 1;
+    int q = (E >= -126) ? E - 7 : -133;
+    double n = rint(ldexp(a, -q)); /* quanta, ties to even; exact scaling */
+    if (n == 0.0)
+        return sign;
+    double r = ldexp(n, q);        /* the rounded magnitude, exact */
+    if (r >= ldexp(1.0, 128))
+        return (uint16_t)(sign | 0x7F80u);
+    if (r < ldexp(1.0, -126))
+        return (uint16_t)(sign | (uint16_t)n); /* subnormal: n < 128 quanta */
+
+    int e2;
+    (void)frexp(r, &e2);
+    int E2 = e2 - 1;
+    unsigned frac = (unsigned)(ldexp(r, 7 - E2) - 128.0);
+    return (uint16_t)(sign | (unsigned)((E2 + 127) << 7) | frac);
+}
+
+double or_bf16_value(uint16_t bits)
+{
+    int s = bits >> 15;
+    int e = (bits >> 7) & 0xFF;
+    int m = bits & 0x7F;
+    double v;
+    if (e == 0xFF)
+        v = m ? NAN : INFINITY;
+    else if (e == 0)
+        v = ldexp((double)m, -133);
+    else
+        v = ldexp((double)(128 + m), e - 127 - 7);
+    return s ? -v : v;
+}
+
+static double round_bf16(double v) { return or_bf16_value(or_bf16_rne(v)); }
+
+/* ------------------------------------------------------------------------ */
+/* Row helpers.                                                              */
+
+static double sum_sq(const double *x, int64_t C)
+{
+    double S = 0.0;
+    for (int64_t j = 0; j < C; ++j)
+        S += x[j] * x[j];
+    return S;
+}
+
+/* The row norm.  [DS] eq. W_eff divides by the row length; the sum carries
+ * eps inside the square root as [TF] states for its rows. */
+static double row_norm(double S, double eps, unsigned flags)
+{
+    if (flags & OR_EPS_ZERO)
+        return sqrt(S);
+    if (flags & OR_EPS_OUTSIDE)
+        return sqrt(S) + eps;
+    return sqrt(S + eps);
+}
+
+/* [DS] "What DragonScale changes", eq. W_eff = diag(g) r W / ||W||_row. */
+void or_wn_forward_row(const double *w, int64_t C, double g, double rho,
+                       double eps, unsigned flags, double *out)
+{
+    double n = row_norm(sum_sq(w, C), eps, flags);
+    for (int64_t j = 0; j < C; ++j)
+        out[j] = g * rho * w[j] / n;
+}
+
+/* Chain rule on the forward above, L = sum_j gy_j out_j:
+ *   dL/dg   = rho sum_j gy_j w_j / n                       = rho D / n
+ *   dL/dw_k = g rho (gy_k / n - w_k D / n^3)               (dn/dw_k = w_k / n)
+ *           = (g rho / n) (gy_k - w_k D / (S + eps)).
+ * [DS] eq. dL/dW prints the eps = 0 form (g r/||W||)(I - w^ w^T) dL/dW_eff. */
+void or_wn_backward_row(const double *w, const double *gy, int64_t C, double g,
+                        double rho, double eps, unsigned flags, double *grad_w,
+                        double *grad_g)
+{
+    double S = sum_sq(w, C);
+    double D = 0.0;
+    for (int64_t j = 0; j < C; ++j)
+        D += w[j] * gy[j];
+    double e = (flags & OR_EPS_ZERO) ? 0.0 : eps;
+    double n = sqrt(S + e);
+    double n2 = (flags & OR_BWD_PRINTED) ? S : S + e;
+    if (grad_g)
+        *grad_g = rho * D / n;
+    for (int64_t j = 0; j < C; ++j)
+        grad_w[j] = (g * rho / n) * (gy[j] - w[j] * D / n2);
+}
+
+/* [DS] "Optimizer": after the step each row is rescaled back to its radius. */
+void or_row_renorm_row(const double *w, int64_t C, double rho, double eps,
+                       unsigned flags, double *out)
+{
+    double n = row_norm(sum_sq(w, C), eps, flags);
+    for (int64_t j = 0; j < C; ++j)
+        out[j] = rho * w[j] / n;
+}
+
+/* [TF] tf_l2_rows.  The sum of two bf16 values is rounded once, from its f64
+ * value: when f64 cannot hold the sum exactly the smaller term is below
+ * 2^-45 of the larger, far from any bf16 halfway point, so the f64 detour
+ * cannot move the result across one. */
+void or_l2_row(const double *x, const double *r, int64_t C, double eps,
+               unsigned flags, double *s, uint16_t *y, double *y_exact)
+{
+    for (int64_t j = 0; j < C; ++j) {
+        if (!r)
+            s[j] = x[j];
+        else if (flags & OR_DROP_SUM_ROUND)
+            s[j] = x[j] + r[j];
+        else
+            s[j] = round_bf16(x[j] + r[j]);
+    }
+    double n = row_norm(sum_sq(s, C), eps, flags);
+    for (int64_t j = 0; j < C; ++j) {
+        double v = s[j] / n;
+        y[j] = or_bf16_rne(v);
+        if (y_exact)
+            y_exact[j] = v;
+    }
+}
+
+/* [TF] tf_slerp_rows: a normalised lerp between two unit rows. */
+void or_slerp_row(const double *res, const double *out, const double *alpha,
+                  int64_t C, double eps, unsigned flags, double *tmp,
+                  uint16_t *h, double *h_exact)
+{
+    double *a = tmp, *b = tmp + C, *t = tmp + 2 * C;
+    double na = row_norm(sum_sq(res, C), eps, flags);
+    double nb = row_norm(sum_sq(out, C), eps, flags);
+    for (int64_t j = 0; j < C; ++j) {
+        a[j] = res[j] / na;
+        if (!(flags & OR_DROP_SLERP_A))
+            a[j] = round_bf16(a[j]);
+        b[j] = out[j] / nb;
+        if (!(flags & OR_DROP_SLERP_B))
+            b[j] = round_bf16(b[j]);
+    }
+    for (int64_t j = 0; j < C; ++j)
+        t[j] = a[j] + fabs(alpha[j]) * (b[j] - a[j]);
+    double nt = row_norm(sum_sq(t, C), eps, flags);
+    for (int64_t j = 0; j < C; ++j) {
+        double v = t[j] / nt;
+        h[j] = or_bf16_rne(v);
+        if (h_exact)
+            h_exact[j] = v;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Interval forms.                                                           */
+
+static double dmin(double a, double b) { return a < b ? a : b; }
+static double dmax(double a, double b) { return a > b ? a : b; }
+
+/* bf16 bits of both ends of [v - delta|v|, v + delta|v|] (rounding is
+ * monotone, so every value inside rounds between them). */
+static void round_ends(double v, double delta, uint16_t *lo, uint16_t *hi)
+{
+    double w = delta * fabs(v);
+    *lo = or_bf16_rne(v - w);
+    *hi = or_bf16_rne(v + w);
+}
+
+void or_l2_row_interval(const double *x, const double *r, int64_t C,
+                        double eps, double delta, unsigned flags, double *s,
+                        uint16_t *lo, uint16_t *hi)
+{
+    for (int64_t j = 0; j < C; ++j) {
+        if (!r)
+            s[j] = x[j];
+        else if (flags & OR_DROP_SUM_ROUND)
+            s[j] = x[j] + r[j];
+        else
+            s[j] = round_bf16(x[j] + r[j]);
+    }
+    double n = row_norm(sum_sq(s, C), eps, flags);
+    for (int64_t j = 0; j < C; ++j)
+        round_ends(s[j] / n, delta, &lo[j], &hi[j]);
+}
+
+/* Interval of x / sqrt(S + eps) over x in [xl, xh], norm in [nl, nh] > 0. */
+static void quotient_ends(double xl, double xh, double nl, double nh,
+                          double delta, double *ql, double *qh)
+{
+    double c0 = xl / nl, c1 = xl / nh, c2 = xh / nl, c3 = xh / nh;
+    double a = dmin(dmin(c0, c1), dmin(c2, c3));
+    double b = dmax(dmax(c0, c1), dmax(c2, c3));
+    *ql = a - delta * fabs(a);
+    *qh = b + delta * fabs(b);
+}
+
+void or_slerp_row_interval(const double *res, const double *out,
+                           const double *alpha, int64_t C, double eps,
+                           double delta, unsigned flags, double *tmp,
+                           uint16_t *lo, uint16_t *hi)
+{
+    double *tl = tmp, *th = tmp + C;
+    double na = row_norm(sum_sq(res, C), eps, flags);
+    double nb = row_norm(sum_sq(out, C), eps, flags);
+    double Sl = 0.0, Sh = 0.0;
+    for (int64_t j = 0; j < C; ++j) {
+        /* a = bf16(l2(res)), b = bf16(l2(out)): both roundings of the ends */
+        double va = res[j] / na, vb = out[j] / nb;
+        double al = va - delta * fabs(va), ah = va + delta * fabs(va);
+        double bl = vb - delta * fabs(vb), bh = vb + delta * fabs(vb);
+        if (!(flags & OR_DROP_SLERP_A)) {
+            al = round_bf16(al);
+            ah = round_bf16(ah);
+        }
+        if (!(flags & OR_DROP_SLERP_B)) {
+            bl = round_bf16(bl);
+            bh = round_bf16(bh);
+        }
+        /* t = a + m (b - a) is affine in a and b: extremes at the corners */
+        double m = fabs(alpha[j]);
+        double t0 = al + m * (bl - al), t1 = al + m * (bh - al);
+        double t2 = ah + m * (bl - ah), t3 = ah + m * (bh - ah);
+        double lo_t = dmin(dmin(t0, t1), dmin(t2, t3));
+        double hi_t = dmax(dmax(t0, t1), dmax(t2, t3));
+        /* fp32 steps: the difference b - a (exact whenever float can hold
+         * it), then a + m (b - a) rounded once (a fused multiply-add) */
+        double dmag = dmax(dmax(fabs(bl - al), fabs(bh - al)),
+                           dmax(fabs(bl - ah), fabs(bh - ah)));
+        int d_exact = (double)(float)(bl - al) == bl - al &&
+                      (double)(float)(bh - al) == bh - al &&
+                      (double)(float)(bl - ah) == bl - ah &&
+                      (double)(float)(bh - ah) == bh - ah;
+        double dslack = d_exact ? 0.0 : delta * m * dmag;
+        tl[j] = lo_t - delta * fabs(lo_t) - dslack;
+        th[j] = hi_t + delta * fabs(hi_t) + dslack;
+        double ql = tl[j] * tl[j], qh = th[j] * th[j];
+        Sl += (tl[j] > 0.0 || th[j] < 0.0) ? dmin(ql, qh) : 0.0;
+        Sh += dmax(ql, qh);
+    }
+    double nl = row_norm(Sl * (1.0 - delta), eps, flags);
+    double nh = row_norm(Sh * (1.0 + delta), eps, flags);
+    if (!(nl > 0.0) || !isfinite(nh)) {
+        /* degenerate norm (zero row at eps = 0, non-finite input): the point
+         * form decides; both ends carry its bits */
+        or_slerp_row(res, out, alpha, C, eps, flags, tmp, lo, NULL);
+        memcpy(hi, lo, sizeof(uint16_t) * (size_t)C);
+        return;
+    }
+    for (int64_t j = 0; j < C; ++j) {
+        double ql, qh;
+        quotient_ends(tl[j], th[j], nl, nh, delta, &ql, &qh);
+        lo[j] = or_bf16_rne(ql);
+        hi[j] = or_bf16_rne(qh);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Matrix drivers.  Each worker owns a contiguous range of rows and its own
+ * scratch rows; inputs are widened to double exactly before the row call.   */
+
+enum { OP_FWD, OP_BWD, OP_RENORM, OP_L2, OP_SLERP, OP_L2_IV, OP_SLERP_IV };
+
+typedef struct {
+    int op;
+    int64_t r0, r1, C, ld, ld2;
+    const float *w;
+    const float *g;
+    const void *gy;
+    int gy_bf16;
+    const uint16_t *x, *r;
+    const float *alpha;
+    double rho, eps, delta;
+    unsigned flags;
+    double *out_d;   /* dense [R, C] doubles */
+    double *out_g;   /* [R] */
+    uint16_t *out_h; /* dense [R, C] bf16 bits */
+    uint16_t *out_h2; /* dense [R, C] bf16 bits (interval upper ends) */
+    int status;
+} job_t;
+
+static void *run_job(void *arg)
+{
+    job_t *jb = (job_t *)arg;
+    int64_t C = jb->C;
+    double *buf = (double *)malloc(sizeof(double) * (size_t)(6 * C));
+    if (!buf) {
+        jb->status = -1;
+        return NULL;
+    }
+    double *u = buf, *v = buf + C, *tmp = buf + 2 * C, *al = buf + 5 * C;
+    if (jb->op == OP_SLERP || jb->op == OP_SLERP_IV)
+        for (int64_t j = 0; j < C; ++j)
+            al[j] = (double)jb->alpha[j];
+
+    for (int64_t row = jb->r0; row < jb->r1; ++row) {
+        size_t o = (size_t)row * (size_t)C;
+        switch (jb->op) {
+        case OP_FWD:
+        case OP_RENORM: {
+            const float *wr = jb->w + row * jb->ld;
+            for (int64_t j = 0; j < C; ++j)
+                u[j] = (double)wr[j];
+            if (jb->op == OP_FWD)
+                or_wn_forward_row(u, C, jb->g ? (double)jb->g[row] : 1.0,
+                                  jb->rho, jb->eps, jb->flags, jb->out_d + o);
+            else
+                or_row_renorm_row(u, C, jb->rho, jb->eps, jb->flags,
+                                  jb->out_d + o);
+            break;
+        }
+        case OP_BWD: {
+            const float *wr = jb->w + row * jb->ld;
+            for (int64_t j = 0; j < C; ++j)
+                u[j] = (double)wr[j];
+            if (jb->gy_bf16) {
+                const uint16_t *gr = (const uint16_t *)jb->gy + row * jb->ld2;
+                for (int64_t j = 0; j < C; ++j)
+                    v[j] = or_bf16_value(gr[j]);
+            } else {
+                const float *gr = (const float *)jb->gy + row * jb->ld2;
+                for (int64_t j = 0; j < C; ++j)
+                    v[j] = (double)gr[j];
+            }
+            double gg = 0.0;
+            or_wn_backward_row(u, v, C, jb->g ? (double)jb->g[row] : 1.0,
+                               jb->rho, jb->eps, jb->flags, jb->out_d + o, &gg);
+            if (jb->out_g)
+                jb->out_g[row] = gg;
+            break;
+        }
+        case OP_L2:
+        case OP_L2_IV: {
+            const uint16_t *xr = jb->x + row * jb->ld;
+            for (int64_t j = 0; j < C; ++j)
+                u[j] = or_bf16_value(xr[j]);
+            const double *rp = NULL;
+            if (jb->r) {
+                const uint16_t *rr = jb->r + row * jb->ld;
+                for (int64_t j = 0; j < C; ++j)
+                    v[j] = or_bf16_value(rr[j]);
+                rp = v;
+            }
+            if (jb->op == OP_L2)
+                or_l2_row(u, rp, C, jb->eps, jb->flags, tmp, jb->out_h + o,
+                          jb->out_d ? jb->out_d + o : NULL);
+            else
+                or_l2_row_interval(u, rp, C, jb->eps, jb->delta, jb->flags,
+                                   tmp, jb->out_h + o, jb->out_h2 + o);
+            break;
+        }
+        case OP_SLERP:
+        case OP_SLERP_IV: {
+            const uint16_t *xr = jb->x + row * jb->ld;
+            const uint16_t *rr = jb->r + row * jb->ld;
+            for (int64_t j = 0; j < C; ++j) {
+                u[j] = or_bf16_value(xr[j]);
+                v[j] = or_bf16_value(rr[j]);
+            }
+            if (jb->op == OP_SLERP)
+                or_slerp_row(u, v, al, C, jb->eps, jb->flags, tmp,
+                             jb->out_h + o, jb->out_d ? jb->out_d + o : NULL);
+            else
+                or_slerp_row_interval(u, v, al, C, jb->eps, jb->delta,
+                                      jb->flags, tmp, jb->out_h + o,
+                                      jb->out_h2 + o);
+            break;
+        }
+        }
+    }
+    free(buf);
+    jb->status = 0;
+    return NULL;
+}
+
+static int run_rows(const job_t *proto, int64_t R, int nthreads)
+{
+    if (R <= 0)
+        return 0;
+    if (nthreads < 1)
+        nthreads = 1;
+    if ((int64_t)nthreads > R)
+        nthreads = (int)R;
+    job_t *jobs = (job_t *)calloc((size_t)nthreads, sizeof(job_t));
+    pthread_t *tid = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    int *started = (int *)calloc((size_t)nthreads, sizeof(int));
+    if (!jobs || !tid || !started) {
+        free(jobs);
+        free(tid);
+        free(started);
+        return -1;
+    }
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = *proto;
+        jobs[t].r0 = R * t / nthreads;
+        jobs[t].r1 = R * (t + 1) / nthreads;
+        jobs[t].status = -1;
+    }
+    for (int t = 1; t < nthreads; ++t)
+        started[t] = pthread_create(&tid[t], NULL, run_job, &jobs[t]) == 0;
+    run_job(&jobs[0]);
+    int rc = jobs[0].status;
+    for (int t = 1; t < nthreads; ++t) {
+        if (started[t])
+            pthread_join(tid[t], NULL);
+        else
+            run_job(&jobs[t]);
+        if (jobs[t].status != 0)
+            rc = -1;
+    }
+    free(jobs);
+    free(tid);
+    free(started);
+    return rc;
+}
+
+static int bad_shape(int64_t R, int64_t C, int64_t ld)
+{
+    return R < 0 || C < 1 || ld < C;
+}
+
+int or_wn_forward(const float *w, int64_t R, int64_t C, int64_t ld,
+                  const float *g, double rho, double eps, unsigned flags,
+                  double *out, int nthreads)
+{
+    if (bad_shape(R, C, ld) || (R > 0 && (!w || !out)))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_FWD;
+    jb.C = C;
+    jb.ld = ld;
+    jb.w = w;
+    jb.g = g;
+    jb.rho = rho;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_d = out;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_wn_backward(const float *w, int64_t R, int64_t C, int64_t ld,
+                   const void *gy, int gy_is_bf16, int64_t ld_gy,
+                   const float *g, double rho, double eps, unsigned flags,
+                   double *grad_w, double *grad_g, int nthreads)
+{
+    if (bad_shape(R, C, ld) || ld_gy < C || (R > 0 && (!w || !gy || !grad_w)))
+        return -1;
+    if (flags & ~(OR_EPS_ZERO | OR_BWD_PRINTED))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_BWD;
+    jb.C = C;
+    jb.ld = ld;
+    jb.ld2 = ld_gy;
+    jb.w = w;
+    jb.g = g;
+    jb.gy = gy;
+    jb.gy_bf16 = gy_is_bf16;
+    jb.rho = rho;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_d = grad_w;
+    jb.out_g = grad_g;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_row_renorm(const float *w, int64_t R, int64_t C, int64_t ld, double rho,
+                  double eps, unsigned flags, double *out, int nthreads)
+{
+    if (bad_shape(R, C, ld) || (R > 0 && (!w || !out)))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_RENORM;
+    jb.C = C;
+    jb.ld = ld;
+    jb.w = w;
+    jb.rho = rho;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_d = out;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_l2_rows(const uint16_t *x, const uint16_t *r, int64_t R, int64_t C,
+               int64_t ld, double eps, unsigned flags, uint16_t *y,
+               double *y_exact, int nthreads)
+{
+    if (bad_shape(R, C, ld) || (R > 0 && (!x || !y)))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_L2;
+    jb.C = C;
+    jb.ld = ld;
+    jb.x = x;
+    jb.r = r;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_h = y;
+    jb.out_d = y_exact;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_slerp_rows(const uint16_t *res, const uint16_t *out, const float *alpha,
+                  int64_t R, int64_t C, int64_t ld, double eps, unsigned flags,
+                  uint16_t *h, double *h_exact, int nthreads)
+{
+    if (bad_shape(R, C, ld) || (R > 0 && (!res || !out || !alpha || !h)))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_SLERP;
+    jb.C = C;
+    jb.ld = ld;
+    jb.x = res;
+    jb.r = out;
+    jb.alpha = alpha;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_h = h;
+    jb.out_d = h_exact;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_l2_rows_interval(const uint16_t *x, const uint16_t *r, int64_t R,
+                        int64_t C, int64_t ld, double eps, double delta,
+                        unsigned flags, uint16_t *lo, uint16_t *hi,
+                        int nthreads)
+{
+    if (bad_shape(R, C, ld) || !(delta >= 0.0) || (R > 0 && (!x || !lo || !hi)))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_L2_IV;
+    jb.C = C;
+    jb.ld = ld;
+    jb.x = x;
+    jb.r = r;
+    jb.eps = eps;
+    jb.delta = delta;
+    jb.flags = flags;
+    jb.out_h = lo;
+    jb.out_h2 = hi;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_slerp_rows_interval(const uint16_t *res, const uint16_t *out,
+                           const float *alpha, int64_t R, int64_t C,
+                           int64_t ld, double eps, double delta,
+                           unsigned flags, uint16_t *lo, uint16_t *hi,
+                           int nthreads)
+{
+    if (bad_shape(R, C, ld) || !(delta >= 0.0) ||
+        (R > 0 && (!res || !out || !alpha || !lo || !hi)))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_SLERP_IV;
+    jb.C = C;
+    jb.ld = ld;
+    jb.x = res;
+    jb.r = out;
+    jb.alpha = alpha;
+    jb.eps = eps;
+    jb.delta = delta;
+    jb.flags = flags;
+    jb.out_h = lo;
+    jb.out_h2 = hi;
+    return run_rows(&jb, R, nthreads);
+}

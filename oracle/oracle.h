@@ -1,0 +1,143 @@
+/*
+ * oracle.h -- float64 CPU oracle for per-row L2 normalisation.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path (the
+ * CUDA library under l2_row_b200/) never calls it, shares no code, header,
+ * table or constant with it, and must fail loudly when its own extension is
+ * missing instead of falling back here.
+ *
+ * Every function is the plain definition of the operation, written one row
+ * at a time, left to right, in double precision, with the bf16 rounding
+ * points the sources state applied explicitly (f64 -> bf16 directly, round to
+ * nearest, ties to even; never through float).
+ *
+ * Sources:
+ *   [DS]  DragonScale package description (PyPI), sections "What DragonScale
+ *         changes" (eq. W_eff, eq. dL/dW), "Patching options" (options table:
+ *         mode, method) and "Optimizer" (rescale after the step).
+ *   [TF]  TensorFold pull request #1260 (Dory native CUDA family),
+ *         Conversation, the norms.cu commit describing tf_l2_rows and
+ *         tf_slerp_rows.
+ *
+ * Parity pins live in tests/ (closed forms, invariants, central finite
+ * differences, exact-rational fixtures under tests/golden/, negative controls).
+ */
+#ifndef L2ROW_ORACLE_H
+#define L2ROW_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Variant flags.  0 = the definition.  Every other bit plants one deliberate
+ * deviation so that tests can show the checker is sharp (negative controls). */
+#define OR_DROP_SUM_ROUND 0x01u /* l2_rows: use x + r unrounded instead of bf16(x + r)   */
+#define OR_DROP_SLERP_A   0x02u /* slerp: use l2(res) unrounded instead of bf16(l2(res)) */
+#define OR_DROP_SLERP_B   0x04u /* slerp: use l2(out) unrounded instead of bf16(l2(out)) */
+#define OR_EPS_OUTSIDE    0x08u /* norm = sqrt(S) + eps instead of sqrt(S + eps)         */
+#define OR_EPS_ZERO       0x10u /* norm = sqrt(S), eps ignored                           */
+#define OR_BWD_PRINTED    0x20u /* backward: project with S instead of S + eps (the
+                                   eps-free form of the printed dL/dW)                   */
+
+/* bf16 helpers.  or_bf16_rne rounds a double straight to bf16 bits. */
+uint16_t or_bf16_rne(double v);
+double   or_bf16_value(uint16_t bits);
+
+/* ---- one row, all values already exact doubles -------------------------- */
+
+/* [DS] eq. W_eff: out_j = g * rho * w_j / sqrt(sum_k w_k^2 + eps). */
+void or_wn_forward_row(const double *w, int64_t C, double g, double rho,
+                       double eps, unsigned flags, double *out);
+
+/* Exact derivative of or_wn_forward_row for L = sum_j gy_j * out_j:
+ *   D = sum w_j gy_j, n = sqrt(S + eps),
+ *   grad_g   = rho * D / n,
+ *   grad_w_j = (g rho / n) * (gy_j - w_j * D / (S + eps)).
+ * At eps = 0 this is [DS] eq. dL/dW. */
+void or_wn_backward_row(const double *w, const double *gy, int64_t C, double g,
+                        double rho, double eps, unsigned flags, double *grad_w,
+                        double *grad_g);
+
+/* [DS] "Optimizer": rescale the row back to its radius, out_j = rho w_j / n. */
+void or_row_renorm_row(const double *w, int64_t C, double rho, double eps,
+                       unsigned flags, double *out);
+
+/* [TF] tf_l2_rows: s = x or bf16(x + r); y = bf16(s / sqrt(sum s^2 + eps)).
+ * r may be NULL.  s_tmp holds C doubles.  y_exact (may be NULL) receives the
+ * value before the final rounding. */
+void or_l2_row(const double *x, const double *r, int64_t C, double eps,
+               unsigned flags, double *s_tmp, uint16_t *y, double *y_exact);
+
+/* [TF] tf_slerp_rows: a = bf16(l2(res)), b = bf16(l2(out)),
+ * t_j = a_j + |alpha_j| (b_j - a_j), h = bf16(t / sqrt(sum t^2 + eps)).
+ * tmp holds 3*C doubles.  h_exact may be NULL. */
+void or_slerp_row(const double *res, const double *out, const double *alpha,
+                  int64_t C, double eps, unsigned flags, double *tmp,
+                  uint16_t *h, double *h_exact);
+
+/* ---- interval forms ----------------------------------------------------- *
+ * [TF] checks each output against "float64's value at the bf16 rounding
+ * points as a range over the fp32 run's spread".  These forms take the same
+ * steps as the point forms but carry an interval: every fp32 evaluation of a
+ * step may be off by a relative `delta`; at each bf16 rounding point both
+ * roundings of the interval's ends are kept.  Output: the lowest and highest
+ * bf16 results (bits) an fp32 evaluation within `delta` can produce.  The
+ * slerp lerp is taken as fp32 steps: the difference b - a, then a + m(b - a)
+ * rounded once (fused multiply-add).  With delta = 0 both equal the point
+ * form.  tmp: l2 needs C doubles, slerp 3*C. */
+void or_l2_row_interval(const double *x, const double *r, int64_t C,
+                        double eps, double delta, unsigned flags, double *tmp,
+                        uint16_t *lo, uint16_t *hi);
+void or_slerp_row_interval(const double *res, const double *out,
+                           const double *alpha, int64_t C, double eps,
+                           double delta, unsigned flags, double *tmp,
+                           uint16_t *lo, uint16_t *hi);
+
+/* ---- matrices: row-major with leading dimension ld (elements) ----------- *
+ * Outputs are dense [R, C].  nthreads <= 1 runs on the calling thread;
+ * otherwise rows are split into nthreads contiguous ranges (each row is still
+ * computed by one thread in the same order, so results do not depend on it).
+ * Return 0 on success, -1 on a bad argument or allocation failure. */
+
+/* g may be NULL (mode "unit": g = 1). */
+int or_wn_forward(const float *w, int64_t R, int64_t C, int64_t ld,
+                  const float *g, double rho, double eps, unsigned flags,
+                  double *out, int nthreads);
+
+/* gy is float32 (gy_is_bf16 = 0) or bf16 bits (gy_is_bf16 = 1), leading
+ * dimension ld_gy.  grad_g may be NULL. */
+int or_wn_backward(const float *w, int64_t R, int64_t C, int64_t ld,
+                   const void *gy, int gy_is_bf16, int64_t ld_gy,
+                   const float *g, double rho, double eps, unsigned flags,
+                   double *grad_w, double *grad_g, int nthreads);
+
+int or_row_renorm(const float *w, int64_t R, int64_t C, int64_t ld, double rho,
+                  double eps, unsigned flags, double *out, int nthreads);
+
+/* x, r: bf16 bits; r may be NULL.  y_exact may be NULL. */
+int or_l2_rows(const uint16_t *x, const uint16_t *r, int64_t R, int64_t C,
+               int64_t ld, double eps, unsigned flags, uint16_t *y,
+               double *y_exact, int nthreads);
+
+int or_slerp_rows(const uint16_t *res, const uint16_t *out, const float *alpha,
+                  int64_t R, int64_t C, int64_t ld, double eps, unsigned flags,
+                  uint16_t *h, double *h_exact, int nthreads);
+
+int or_l2_rows_interval(const uint16_t *x, const uint16_t *r, int64_t R,
+                        int64_t C, int64_t ld, double eps, double delta,
+                        unsigned flags, uint16_t *lo, uint16_t *hi,
+                        int nthreads);
+int or_slerp_rows_interval(const uint16_t *res, const uint16_t *out,
+                           const float *alpha, int64_t R, int64_t C,
+                           int64_t ld, double eps, double delta,
+                           unsigned flags, uint16_t *lo, uint16_t *hi,
+                           int nthreads);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* L2ROW_ORACLE_H */

@@ -1,0 +1,203 @@
+"""numpy front end of liboracle.so (ctypes).  Test infrastructure only.
+
+Arrays are passed as 2-D numpy views (row stride = leading dimension); bf16
+tensors travel as their uint16 bit patterns.  Outputs are dense [R, C].
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+
+import numpy as np
+
+from . import build as _build
+
+OR_DROP_SUM_ROUND = 0x01
+OR_DROP_SLERP_A = 0x02
+OR_DROP_SLERP_B = 0x04
+OR_EPS_OUTSIDE = 0x08
+OR_EPS_ZERO = 0x10
+OR_BWD_PRINTED = 0x20
+
+_lib = None
+
+
+def lib() -> ct.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ct.CDLL(_build.build())
+        i64, dbl, uns, vp, i32 = ct.c_int64, ct.c_double, ct.c_uint, ct.c_void_p, ct.c_int
+        _lib.or_bf16_rne.argtypes = [dbl]
+        _lib.or_bf16_rne.restype = ct.c_uint16
+        _lib.or_bf16_value.argtypes = [ct.c_uint16]
+        _lib.or_bf16_value.restype = dbl
+        _lib.or_wn_forward.argtypes = [vp, i64, i64, i64, vp, dbl, dbl, uns, vp, i32]
+        _lib.or_wn_backward.argtypes = [vp, i64, i64, i64, vp, i32, i64, vp, dbl, dbl, uns, vp, vp, i32]
+        _lib.or_row_renorm.argtypes = [vp, i64, i64, i64, dbl, dbl, uns, vp, i32]
+        _lib.or_l2_rows.argtypes = [vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
+        _lib.or_slerp_rows.argtypes = [vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
+        _lib.or_wn_backward_row.argtypes = [vp, vp, i64, dbl, dbl, dbl, uns, vp, vp]
+        _lib.or_wn_forward_row.argtypes = [vp, i64, dbl, dbl, dbl, uns, vp]
+        _lib.or_l2_rows_interval.argtypes = [vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
+        _lib.or_slerp_rows_interval.argtypes = [vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
+        for f in ("or_wn_forward", "or_wn_backward", "or_row_renorm", "or_l2_rows", "or_slerp_rows",
+                  "or_l2_rows_interval", "or_slerp_rows_interval"):
+            getattr(_lib, f).restype = i32
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _rows(a: np.ndarray, dtype) -> tuple[np.ndarray, int]:
+    """Check a 2-D row-major view with unit column stride; return (a, ld)."""
+    if a.dtype != dtype or a.ndim != 2:
+        raise TypeError(f"expected 2-D {np.dtype(dtype)}, got {a.dtype} {a.shape}")
+    if a.shape[0] == 0:
+        return a, a.shape[1]
+    if a.strides[1] != a.itemsize or a.strides[0] % a.itemsize:
+        a = np.ascontiguousarray(a)
+    return a, a.strides[0] // a.itemsize if a.shape[0] > 1 else a.shape[1]
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ct.c_void_p)
+
+
+def _check(rc: int, name: str) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle {name} rejected its arguments")
+
+
+def bf16_rne(v: float) -> int:
+    return int(lib().or_bf16_rne(float(v)))
+
+
+def bf16_value(bits: int) -> float:
+    return float(lib().or_bf16_value(int(bits) & 0xFFFF))
+
+
+def wn_forward(w, g=None, *, rho=1.0, eps=1e-6, flags=0, nthreads=1):
+    """f64 W_eff [R, C] for fp32 rows w [R, C] (g fp32 [R] or None)."""
+    w, ld = _rows(w, np.float32)
+    R, C = w.shape
+    out = np.empty((R, C), np.float64)
+    g = None if g is None else np.ascontiguousarray(g, np.float32)
+    _check(lib().or_wn_forward(_p(w), R, C, ld, _p(g), rho, eps, flags, _p(out), nthreads), "wn_forward")
+    return out
+
+
+def wn_backward(w, gy, g=None, *, rho=1.0, eps=1e-6, flags=0, nthreads=1):
+    """f64 (grad_w [R, C], grad_g [R]); gy fp32 or bf16 bits (uint16)."""
+    w, ld = _rows(w, np.float32)
+    is_bf16 = gy.dtype == np.uint16
+    gy, ldg = _rows(gy, np.uint16 if is_bf16 else np.float32)
+    R, C = w.shape
+    if gy.shape != (R, C):
+        raise ValueError("gy shape")
+    gw = np.empty((R, C), np.float64)
+    gg = np.empty((R,), np.float64)
+    g = None if g is None else np.ascontiguousarray(g, np.float32)
+    _check(lib().or_wn_backward(_p(w), R, C, ld, _p(gy), int(is_bf16), ldg, _p(g), rho, eps, flags,
+                                _p(gw), _p(gg), nthreads), "wn_backward")
+    return gw, gg
+
+
+def row_renorm(w, *, rho=1.0, eps=1e-6, flags=0, nthreads=1):
+    w, ld = _rows(w, np.float32)
+    R, C = w.shape
+    out = np.empty((R, C), np.float64)
+    _check(lib().or_row_renorm(_p(w), R, C, ld, rho, eps, flags, _p(out), nthreads), "row_renorm")
+    return out
+
+
+def l2_rows(x, r=None, *, eps=1e-6, flags=0, nthreads=1, exact=False):
+    """bf16 bits y [R, C] (uint16); with exact=True also the f64 value before rounding."""
+    x, ld = _rows(x, np.uint16)
+    R, C = x.shape
+    if r is not None:
+        r, ldr = _rows(r, np.uint16)
+        if r.shape != x.shape:
+            raise ValueError("r shape")
+        if ldr != ld:
+            x, r = np.ascontiguousarray(x), np.ascontiguousarray(r)
+            ld = C
+    y = np.empty((R, C), np.uint16)
+    ye = np.empty((R, C), np.float64) if exact else None
+    _check(lib().or_l2_rows(_p(x), _p(r), R, C, ld, eps, flags, _p(y), _p(ye), nthreads), "l2_rows")
+    return (y, ye) if exact else y
+
+
+def slerp_rows(res, out, alpha, *, eps=1e-6, flags=0, nthreads=1, exact=False):
+    res, ld = _rows(res, np.uint16)
+    out, ldo = _rows(out, np.uint16)
+    if out.shape != res.shape:
+        raise ValueError("out shape")
+    if ldo != ld:
+        res, out = np.ascontiguousarray(res), np.ascontiguousarray(out)
+        ld = res.shape[1]
+    R, C = res.shape
+    alpha = np.ascontiguousarray(alpha, np.float32)
+    if alpha.shape != (C,):
+        raise ValueError("alpha shape")
+    h = np.empty((R, C), np.uint16)
+    he = np.empty((R, C), np.float64) if exact else None
+    _check(lib().or_slerp_rows(_p(res), _p(out), _p(alpha), R, C, ld, eps, flags, _p(h), _p(he), nthreads),
+           "slerp_rows")
+    return (h, he) if exact else h
+
+
+def l2_rows_interval(x, r=None, *, eps=1e-6, delta=1e-5, flags=0, nthreads=1):
+    """(lo, hi) bf16 bits: the outputs any fp32 evaluation within relative
+    `delta` per step can produce (TensorFold's range over the fp32 spread)."""
+    x, ld = _rows(x, np.uint16)
+    R, C = x.shape
+    if r is not None:
+        r, ldr = _rows(r, np.uint16)
+        if ldr != ld:
+            x, r = np.ascontiguousarray(x), np.ascontiguousarray(r)
+            ld = C
+    lo = np.empty((R, C), np.uint16)
+    hi = np.empty((R, C), np.uint16)
+    _check(lib().or_l2_rows_interval(_p(x), _p(r), R, C, ld, eps, delta, flags, _p(lo), _p(hi), nthreads),
+           "l2_rows_interval")
+    return lo, hi
+
+
+def slerp_rows_interval(res, out, alpha, *, eps=1e-6, delta=1e-5, flags=0, nthreads=1):
+    res, ld = _rows(res, np.uint16)
+    out, ldo = _rows(out, np.uint16)
+    if ldo != ld:
+        res, out = np.ascontiguousarray(res), np.ascontiguousarray(out)
+        ld = res.shape[1]
+    R, C = res.shape
+    alpha = np.ascontiguousarray(alpha, np.float32)
+    lo = np.empty((R, C), np.uint16)
+    hi = np.empty((R, C), np.uint16)
+    _check(lib().or_slerp_rows_interval(_p(res), _p(out), _p(alpha), R, C, ld, eps, delta, flags, _p(lo), _p(hi),
+                                        nthreads), "slerp_rows_interval")
+    return lo, hi
+
+
+def wn_forward_row64(w, g=1.0, *, rho=1.0, eps=1e-6, flags=0):
+    """One row with f64 inputs (for finite differences)."""
+    w = np.ascontiguousarray(w, np.float64)
+    out = np.empty_like(w)
+    lib().or_wn_forward_row(_p(w), w.size, float(g), rho, eps, flags, _p(out))
+    return out
+
+
+def wn_backward_row64(w, gy, g=1.0, *, rho=1.0, eps=1e-6, flags=0):
+    w = np.ascontiguousarray(w, np.float64)
+    gy = np.ascontiguousarray(gy, np.float64)
+    gw = np.empty_like(w)
+    gg = ct.c_double()
+    lib().or_wn_backward_row(_p(w), _p(gy), w.size, float(g), rho, eps, flags, _p(gw), ct.byref(gg))
+    return gw, gg.value
+
+
+__all__ = [n for n in dir() if not n.startswith("_") and n not in ("annotations", "ct", "os", "np")]
