@@ -1,0 +1,508 @@
+#!/usr/bin/env python
+"""Benchmark of the per-row L2 normalisation hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+
+  1. ds_wn_forward   every weight of a 12-layer d_model-768 decoder plus its
+                     tied embedding (85 segments, 114,944 rows, 100,073,472
+                     fp32 elements) -> bf16 W_eff, one call
+  2. ds_l2_rows      activation rows X [16384, 4096] bf16
+  3. ds_wn_backward  the same 85 segments, bf16 GY -> fp32 grad_w, grad_g
+  4. ds_l2_rows      X + R (fused residual add)
+  5. ds_row_renorm   the 85 segments in place
+  6. ds_slerp_rows   res = X, out = R, alpha [4096]
+
+Every call reads more than the 126 MB L2 and consecutive calls touch
+disjoint buffers (>= 268 MB of other traffic between two uses of one
+buffer), so inputs come from HBM without an explicit flush.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  `value` is algorithmic bytes moved by all
+ranks per second (GB/s); per-kernel GB/s and rows/s, the roofline of the
+dominant kernel, the end-to-end figure through the C ABI from pinned host
+buffers, and the float64 CPU oracle timed on a bounded sample ride along.
+Under torchrun every rank runs the same step on its own seeded data (weak
+scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes as ct
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "achieved HBM GB/s (fraction of B200 peak) and rows/s per kernel, fwd+bwd"
+EPS = 1e-6
+ACT_ROWS, ACT_COLS = 16384, 4096
+WORKLOAD = ("whole-model weights: 85 segments (12 layers x {q,k,v,o,gate,up,down} + tied embedding "
+            "[32000,768]), 100,073,472 fp32 elements, fwd (bf16 W_eff) + bwd (bf16 GY) + renorm; "
+            "activation rows [16384,4096] bf16: l2, l2 + residual, slerp")
+CALLS = ("wn_forward", "l2_rows", "wn_backward", "l2_rows_residual", "row_renorm", "slerp_rows")
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------ bookkeeping --
+
+def step_bytes(weights, act_rows=ACT_ROWS, act_cols=ACT_COLS) -> dict[str, int]:
+    """Algorithmic bytes per call: every input read once, every output
+    written once (per-row gains and grad_g 4 B per row)."""
+    E = sum(s.w.size for s in weights)
+    R = sum(s.rows for s in weights)
+    A = act_rows * act_cols
+    return {
+        "wn_forward": E * (4 + 2) + R * 4,
+        "wn_backward": E * (4 + 2 + 4) + R * (4 + 4),
+        "row_renorm": E * (4 + 4),
+        "l2_rows": A * (2 + 2),
+        "l2_rows_residual": A * (2 + 2 + 2),
+        "slerp_rows": A * (2 + 2 + 2) + act_cols * 4,
+    }
+
+
+def step_rows(weights, act_rows=ACT_ROWS) -> dict[str, int]:
+    R = sum(s.rows for s in weights)
+    return {"wn_forward": R, "wn_backward": R, "row_renorm": R,
+            "l2_rows": act_rows, "l2_rows_residual": act_rows, "slerp_rows": act_rows}
+
+
+def measured_peaks() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_source_digest() -> str:
+    h = hashlib.sha256()
+    for rel in ("l2_row_b200/csrc/ds_kernels.cu", "l2_row_b200/csrc/ds_device.cuh", "l2_row_b200/csrc/ds_internal.h"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str) -> float | None:
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec["kernels"][kernel]
+        if rec.get("source_digest") != kernel_source_digest():
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples: list[tuple[int, int]] = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            pass
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM)
+                rs = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+        return False
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        mhz = [m for m, _ in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= r
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+# ------------------------------------------------------------- our arm -----
+
+class Step:
+    """Device buffers, prebuilt C segment tables and the six calls of a step."""
+
+    def __init__(self, seed: int):
+        import torch
+
+        from l2_row_b200 import ds
+        from l2_row_b200 import workloads as wl
+
+        self.torch, self.ds = torch, ds
+        self.model = wl.whole_model(seed)
+        self.act = wl.activations(seed, ACT_ROWS, ACT_COLS).acts[0]
+        dev = "cuda"
+
+        def f32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+
+        def bf16(b):
+            return torch.from_numpy(np.ascontiguousarray(b, np.uint16).view(np.int16)).to(dev).view(torch.bfloat16)
+
+        # one flat buffer per tensor kind keeps the H2D copies of the e2e leg few and large
+        segs = self.model.weights
+        n_el = sum(s.w.size for s in segs)
+        n_rows = sum(s.rows for s in segs)
+        self.w = torch.empty(n_el, dtype=torch.float32, device=dev)
+        self.gy = torch.empty(n_el, dtype=torch.bfloat16, device=dev)
+        self.gain = torch.empty(n_rows, dtype=torch.float32, device=dev)
+        self.weff = torch.empty(n_el, dtype=torch.bfloat16, device=dev)
+        self.grad_w = torch.empty(n_el, dtype=torch.float32, device=dev)
+        self.grad_g = torch.empty(n_rows, dtype=torch.float32, device=dev)
+        self.host_w = np.concatenate([s.w.ravel() for s in segs])
+        self.host_gy = np.concatenate([s.gy.ravel() for s in segs])
+        self.host_gain = np.concatenate([s.g for s in segs])
+        self.w.copy_(f32(self.host_w))
+        self.gy.copy_(bf16(self.host_gy))
+        self.gain.copy_(f32(self.host_gain))
+        fwd, bwd, ren = [], [], []
+        eo = ro = 0
+        for s in segs:
+            R, C = s.rows, s.cols
+            sl = slice(eo, eo + R * C)
+            w = self.w[sl].view(R, C)
+            gain = self.gain[ro:ro + R]
+            fwd.append(ds.WSeg(w=w, gain=gain, w_eff=self.weff[sl].view(R, C)).to_c())
+            bwd.append(ds.WSeg(w=w, gain=gain, gy=self.gy[sl].view(R, C), grad_w=self.grad_w[sl].view(R, C),
+                               grad_g=self.grad_g[ro:ro + R]).to_c())
+            ren.append(ds.WSeg(w=w).to_c())
+            eo += R * C
+            ro += R
+        self.x = bf16(self.act.x)
+        self.r = bf16(self.act.r)
+        self.alpha = f32(self.act.alpha)
+        self.y = torch.empty_like(self.x)
+        self.y2 = torch.empty_like(self.x)
+        self.h = torch.empty_like(self.x)
+        self.tables = {
+            "wn_forward": (ds.ds_wseg * len(fwd))(*fwd),
+            "wn_backward": (ds.ds_wseg * len(bwd))(*bwd),
+            "row_renorm": (ds.ds_wseg * len(ren))(*ren),
+            "l2_rows": (ds.ds_aseg * 1)(ds.ASeg(x=self.x, y=self.y).to_c()),
+            "l2_rows_residual": (ds.ds_aseg * 1)(ds.ASeg(x=self.x, r=self.r, y=self.y2).to_c()),
+            "slerp_rows": (ds.ds_aseg * 1)(ds.ASeg(x=self.x, r=self.r, y=self.h, alpha=self.alpha).to_c()),
+        }
+        self.nseg = len(segs)
+        lib = ds.lib()
+        eps = ct.c_float(EPS)
+        t = self.tables
+        self.calls = {
+            "wn_forward": lambda s: lib.ds_wn_forward(t["wn_forward"], self.nseg, ds.DS_BF16, eps, s),
+            "l2_rows": lambda s: lib.ds_l2_rows(t["l2_rows"], 1, eps, s),
+            "wn_backward": lambda s: lib.ds_wn_backward(t["wn_backward"], self.nseg, ds.DS_BF16, eps, s),
+            "l2_rows_residual": lambda s: lib.ds_l2_rows(t["l2_rows_residual"], 1, eps, s),
+            "row_renorm": lambda s: lib.ds_row_renorm(t["row_renorm"], self.nseg, eps, s),
+            "slerp_rows": lambda s: lib.ds_slerp_rows(t["slerp_rows"], 1, eps, s),
+        }
+
+    def run(self, stream_ptr: int, events=None) -> None:
+        for i, name in enumerate(CALLS):
+            if events is not None:
+                events[i].record()
+            st = self.calls[name](stream_ptr)
+            if st != 0:
+                raise self.ds.DSError(st, name)
+        if events is not None:
+            events[len(CALLS)].record()
+
+
+def run_ours(args, rank: int, world: int, local_rank: int) -> None:
+    import torch
+
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist_mod
+
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local_rank))
+        dist = dist_mod
+
+    from l2_row_b200 import ds
+
+    step = Step(seed=rank)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    bytes_per = step_bytes(step.model.weights)
+    rows_per = step_rows(step.model.weights)
+    step_total = sum(bytes_per.values())
+
+    for _ in range(max(3, args.warmup)):
+        step.run(sp)
+    torch.cuda.synchronize()
+    if ds.ds_get_device_status(sp) != ds.DS_OK:
+        raise RuntimeError("device error during warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(CALLS) + 1)] for _ in range(K)]
+    n0 = ds.ds_launch_count()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        for k in range(K):
+            step.run(sp, evs[k])
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    launches = ds.ds_launch_count() - n0
+    if ds.ds_get_device_status(sp) != ds.DS_OK:
+        raise RuntimeError("device error in the timed region")
+
+    total_ms = evs[0][0].elapsed_time(evs[-1][-1])
+    per_call = {name: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K)] for i, name in enumerate(CALLS)}
+    if dist:
+        t = torch.tensor([total_ms] + [statistics.fmean(v) for v in per_call.values()], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t[0])
+        call_ms = {name: float(t[i + 1]) for i, name in enumerate(CALLS)}
+    else:
+        call_ms = {name: statistics.fmean(v) for name, v in per_call.items()}
+
+    ms_per_step = total_ms / K
+    value = world * step_total / (ms_per_step * 1e-3) / 1e9
+
+    peak, peak_src = measured_peaks()
+    kernels = {}
+    for name in CALLS:
+        t_s = call_ms[name] * 1e-3
+        gbs = bytes_per[name] / t_s / 1e9
+        kernels[name] = {"us": round(call_ms[name] * 1e3, 2), "bytes": bytes_per[name], "gb_s": round(gbs, 1),
+                         "frac_of_peak": round(gbs / peak, 4), "rows_s": round(rows_per[name] / t_s, 1)}
+    fb_t = (call_ms["wn_forward"] + call_ms["wn_backward"]) * 1e-3
+    fwd_bwd = {"gb_s": round((bytes_per["wn_forward"] + bytes_per["wn_backward"]) / fb_t / 1e9, 1),
+               "rows_s": round(rows_per["wn_forward"] / fb_t, 1),
+               "frac_of_peak": round((bytes_per["wn_forward"] + bytes_per["wn_backward"]) / fb_t / 1e9 / peak, 4)}
+    dom = max(CALLS, key=lambda n: call_ms[n])
+    ach = bytes_per[dom] / (call_ms[dom] * 1e-3) / 1e9
+    traffic = recorded_traffic(dom)
+    roofline = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "traffic": traffic, "kernel": f"ds_{dom}",
+                "algorithmic_bytes": bytes_per[dom], "peak_source": peak_src}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(step, args.e2e_steps, step_total, sp, world, dist)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(step)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, host-generated)",
+        "config": {"workload": WORKLOAD, "eps": EPS, "bytes_per_step": step_total,
+                   "l2": "no flush: every call reads > 126 MB and consecutive calls touch disjoint buffers",
+                   "parallelism": f"replicas x{world} (rows are independent; no collective)"},
+        "kernels": kernels, "fwd_bwd": fwd_bwd, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
+        "gpu_launches": launches, "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def measure_e2e(step: Step, steps: int, step_total: int, sp: int, world: int, dist) -> dict:
+    """The same step through the C ABI starting from pinned host buffers:
+    every step copies its inputs host -> device, runs the six calls and
+    copies every output back."""
+    import torch
+
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    h_in = [(step.w, pin(step.host_w)), (step.gy, pin(step.host_gy.view(np.int16)).view(torch.bfloat16)),
+            (step.gain, pin(step.host_gain)),
+            (step.x, pin(step.act.x.view(np.int16)).view(torch.bfloat16)),
+            (step.r, pin(step.act.r.view(np.int16)).view(torch.bfloat16)), (step.alpha, pin(step.act.alpha))]
+    outs = [step.weff, step.grad_w, step.grad_g, step.w, step.y, step.y2, step.h]
+    h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    h2d = sum(d.numel() * d.element_size() for d, _ in h_in)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+
+    def one():
+        for d, h in h_in:
+            d.copy_(h, non_blocking=True)
+        step.run(sp)
+        for o, h in zip(outs, h_out):
+            h.copy_(o, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+    return {"value": round(world * step_total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3)}
+
+
+# ------------------------------------------------------- the CPU oracle ----
+
+def oracle_sample(model_weights, act, frac: float):
+    """A bounded slice of the step: the first `frac` of every weight
+    segment's rows and of the activation rows."""
+    from l2_row_b200 import workloads as wl
+
+    segs = []
+    for s in model_weights:
+        n = max(1, int(round(s.rows * frac)))
+        segs.append(wl.WeightSeg(s.name, s.w[:n], s.g[:n], s.gy[:n]))
+    n = max(1, int(round(act.rows * frac)))
+    a = wl.ActRows(act.name, act.x[:n], act.r[:n], act.alpha)
+    return segs, a
+
+
+def time_oracle_step(segs, a, nthreads: int) -> tuple[float, int]:
+    """Run the six operations of a step on the oracle; (seconds, bytes)."""
+    import oracle
+
+    t0 = time.perf_counter()
+    for s in segs:
+        oracle.wn_forward(s.w, s.g, eps=EPS, nthreads=nthreads)
+    oracle.l2_rows(a.x, None, eps=EPS, nthreads=nthreads)
+    for s in segs:
+        oracle.wn_backward(s.w, s.gy, s.g, eps=EPS, nthreads=nthreads)
+    oracle.l2_rows(a.x, a.r, eps=EPS, nthreads=nthreads)
+    for s in segs:
+        oracle.row_renorm(s.w, eps=EPS, nthreads=nthreads)
+    oracle.slerp_rows(a.x, a.r, a.alpha, eps=EPS, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    b = step_bytes(segs, a.rows, a.cols)
+    return dt, sum(b.values())
+
+
+def cpu_baseline(step: Step, frac: float = 1 / 4) -> dict:
+    import oracle
+
+    cores = oracle.default_threads()
+    segs, a = oracle_sample(step.model.weights, step.act, frac)
+    dt, nbytes = time_oracle_step(segs, a, cores)
+    return {"value": round(nbytes / dt / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"first 1/{round(1 / frac)} of every segment's rows and of the activation rows "
+                      f"({nbytes / 1e6:.0f} MB algorithmic), all six calls, {dt:.1f} s wall"}
+
+
+def run_reference(args, rank: int, world: int) -> None:
+    """The reference arm: the float64 oracle as it stands, on the host cores,
+    same metric and workload, each step a bounded sample of it."""
+    if rank != 0:
+        return
+    import oracle
+    from l2_row_b200 import workloads as wl
+
+    model = wl.whole_model(0)
+    act = wl.activations(0, ACT_ROWS, ACT_COLS).acts[0]
+    cores = oracle.default_threads()
+    frac = 1 / 256
+    segs, a = oracle_sample(model.weights, act, frac)
+    for _ in range(max(1, args.warmup)):
+        time_oracle_step(segs, a, cores)
+    total, nbytes = 0.0, 0
+    for _ in range(args.steps):
+        dt, b = time_oracle_step(segs, a, cores)
+        total += dt
+        nbytes += b
+    value = nbytes / total / 1e9
+    sample = (f"first 1/256 of every segment's rows and of the activation rows per step "
+              f"({nbytes / args.steps / 1e6:.1f} MB algorithmic per step)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, host-generated)",
+        "config": {"workload": WORKLOAD, "eps": EPS, "sample": sample},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

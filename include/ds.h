@@ -1,0 +1,189 @@
+/*
+ * ds.h -- C ABI of libds: per-row L2 normalisation of weight and activation
+ * rows on NVIDIA B200 (sm_100a).
+ *
+ * Five operations, each over a table of segments (matrices), so that every
+ * weight of a model is handled by one call:
+ *
+ *   ds_wn_forward   W_eff[r,:] = g_r * rho * w[r,:] / sqrt(sum_j w[r,j]^2 + eps)
+ *                   DragonScale package description, "What DragonScale
+ *                   changes", eq. W_eff (unit rows times one gain per row,
+ *                   radius rho: 1 for linears/convs, sqrt(dim) for embeddings).
+ *   ds_wn_backward  the exact gradient of ds_wn_forward:
+ *                   grad_g_r = rho * (w_r . GY_r) / n_r,
+ *                   grad_w_r = (g_r rho / n_r) * (GY_r - w_r (w_r . GY_r) / n_r^2),
+ *                   n_r = sqrt(sum w_r^2 + eps); same section, eq. dL/dW
+ *                   (printed there at eps = 0: the gradient tangent to the row).
+ *   ds_row_renorm   w[r,:] <- rho * w[r,:] / n_r in place; DragonScale,
+ *                   "Optimizer" (method "rescale": after the step each row is
+ *                   rescaled back to its radius).
+ *   ds_l2_rows      y = bf16(s / sqrt(sum s^2 + eps)), s = x or s = bf16(x + r);
+ *                   TensorFold PR #1260, Conversation, the norms.cu commit
+ *                   (tf_l2_rows: a loop's entry l2(state + input), or its exit).
+ *   ds_slerp_rows   a = bf16(l2(x)), b = bf16(l2(r)),
+ *                   t_j = a_j + |alpha_j| (b_j - a_j)  (fp32, one rounding),
+ *                   y = bf16(t / sqrt(sum t^2 + eps)); same commit (tf_slerp_rows,
+ *                   the normalised-lerp residual).
+ *
+ * Numerics: every row reduction accumulates in fp32 in an order fixed by the
+ * row length and the operation alone, so a row's bits never depend on the
+ * row count, the segment table or the launch.  bf16 results are rounded to
+ * nearest even.  Rows whose fp32 sum of squares overflows (or, at eps = 0,
+ * falls below 2^-100) are recomputed with an exact power-of-two rescaling.
+ *
+ * Memory: all pointers are DEVICE pointers owned by the caller (the segment
+ * tables themselves are HOST memory, read only during the call).  The library
+ * allocates nothing, keeps no per-call state and may be called from several
+ * host threads.  Matrices are row-major with leading dimension ld (elements)
+ * >= cols; every row start must be 16-byte aligned (base pointer 16-byte
+ * aligned, ld * element size a multiple of 16), and each buffer must be
+ * readable up to the 16-byte boundary that follows its last element (any
+ * cudaMalloc or PyTorch allocation is).  Elements past cols in a row are never
+ * written.
+ *
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ * default stream) and never synchronise, except ds_get_device_status.
+ * Arguments are validated on the host before anything is launched; a failed
+ * call launches nothing.  Kernels never trap: a bounded device-side wait that
+ * runs out records DS_ERR_DEVICE_TIMEOUT, read by ds_get_device_status.
+ */
+#ifndef DS_H
+#define DS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DS_OK = 0,
+    DS_ERR_INVALID_ARG = 1,       /* NULL pointer, bad shape, bad eps, bad dtype value */
+    DS_ERR_ALIGNMENT = 2,         /* a row start not 16-byte aligned                    */
+    DS_ERR_UNSUPPORTED_DTYPE = 3, /* dtype not allowed for this call                    */
+    DS_ERR_TOO_MANY_SEGMENTS = 4, /* nseg above DS_MAX_SEGMENTS                         */
+    DS_ERR_CUDA = 5,              /* a CUDA runtime call failed (see ds_last_error)     */
+    DS_ERR_DEVICE_TIMEOUT = 6,    /* a bounded device-side wait ran out                 */
+    DS_ERR_OVERLAP = 7            /* an output overlaps an input or another output      */
+} ds_status;
+
+typedef enum { DS_F32 = 0, DS_BF16 = 1 } ds_dtype;
+
+typedef void *ds_stream; /* cudaStream_t */
+
+#define DS_MAX_SEGMENTS 65536
+
+/* One weight matrix (Linear, Embedding, or a Conv flattened to [out, in*k...]).
+ * Which fields a call reads:
+ *   forward:  w, gain, w_eff (written), rows, cols, ld, ld_out, radius
+ *   backward: w, gain, gy, grad_w (written), grad_g (written if gain != NULL),
+ *             rows, cols, ld, ld_out, radius
+ *   renorm:   w (read and written in place), rows, cols, ld, radius          */
+typedef struct {
+    float *w;          /* fp32 [rows, ld] master rows                                */
+    const float *gain; /* fp32 [rows], or NULL: mode "unit" (g = 1, no grad_g)       */
+    void *w_eff;       /* forward output [rows, ld_out], dtype per call               */
+    const void *gy;    /* backward input dL/dW_eff [rows, ld_out], dtype per call     */
+    float *grad_w;     /* backward output fp32 [rows, ld], overwritten                */
+    float *grad_g;     /* backward output fp32 [rows], overwritten (gain != NULL)     */
+    int64_t rows;      /* >= 0                                                        */
+    int64_t cols;      /* >= 1, <= 2^31 - 1                                           */
+    int64_t ld;        /* leading dimension of w and grad_w, >= cols                  */
+    int64_t ld_out;    /* leading dimension of w_eff and gy, >= cols                  */
+    float radius;      /* rho: 1 for linears and convs, sqrt(cols) for embeddings     */
+} ds_wseg;
+
+/* One activation matrix; x, r and y share the leading dimension ld.
+ *   l2_rows:    x bf16 (required), r bf16 residual or NULL, y bf16 output
+ *               (y may be exactly x or exactly r; partial overlap is refused)
+ *   slerp_rows: x = res (required), r = out (required), alpha fp32 [cols]
+ *               (|alpha_j| is the lerp weight), y = output (may alias x or r) */
+typedef struct {
+    const void *x;
+    const void *r;
+    void *y;
+    const float *alpha;
+    int64_t rows; /* >= 0 */
+    int64_t cols; /* >= 1, <= 2^31 - 1 */
+    int64_t ld;   /* >= cols */
+} ds_aseg;
+
+/* out_dtype: DS_BF16 or DS_F32 for every segment's w_eff. */
+ds_status ds_wn_forward(const ds_wseg *segs, int nseg, ds_dtype out_dtype,
+                        float eps, ds_stream stream);
+
+/* gy_dtype: DS_BF16 or DS_F32 for every segment's gy.  w, gy and gain are
+ * read-only; grad_w and grad_g must not overlap any input. */
+ds_status ds_wn_backward(const ds_wseg *segs, int nseg, ds_dtype gy_dtype,
+                         float eps, ds_stream stream);
+
+ds_status ds_row_renorm(const ds_wseg *segs, int nseg, float eps,
+                        ds_stream stream);
+
+ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps,
+                     ds_stream stream);
+
+ds_status ds_slerp_rows(const ds_aseg *segs, int nseg, float eps,
+                        ds_stream stream);
+
+/* Static description of a status code. */
+const char *ds_status_string(ds_status status);
+
+/* Detail of the last failed call on this host thread ("" if none). */
+const char *ds_last_error(void);
+
+/* Synchronises `stream`, then returns and clears the device error word of
+ * the current device (DS_OK, or DS_ERR_DEVICE_TIMEOUT after a bounded wait
+ * ran out), or DS_ERR_CUDA if the synchronisation itself failed. */
+ds_status ds_get_device_status(ds_stream stream);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t ds_launch_count(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int ds_version(void);
+
+/* ---- planning introspection (host only, no GPU needed) ------------------ */
+
+typedef enum {
+    DS_OP_WN_FORWARD = 0,
+    DS_OP_WN_BACKWARD = 1,
+    DS_OP_ROW_RENORM = 2,
+    DS_OP_L2_ROWS = 3,
+    DS_OP_SLERP_ROWS = 4
+} ds_op;
+
+typedef enum {
+    DS_PATH_AUTO = 0,     /* chosen from the row length                       */
+    DS_PATH_WARP = 1,     /* one warp per row, row in registers               */
+    DS_PATH_CTA = 2,      /* 64..256 threads of a CTA per row, in registers   */
+    DS_PATH_CLUSTER = 3,  /* a cluster of 2..8 CTAs per row, DSMEM reduction  */
+    DS_PATH_TWO_PASS = 4  /* a cluster streams the row twice through shared
+                             memory with bulk (TMA) copies                    */
+} ds_path;
+
+/* The row class a call would use for rows of `cols` elements: path, threads
+ * per row inside a CTA (warp/CTA paths) and CTAs per row (cluster/two-pass).
+ * Depends on (op, cols) and the forced path only -- never on the row count. */
+ds_status ds_row_class(ds_op op, int64_t cols, int *path, int *group_threads,
+                       int *cluster_ctas);
+
+/* ---- test knobs (process-wide; not for production use) ------------------ */
+
+/* Force every call onto one path where the row fits it (DS_PATH_AUTO
+ * restores automatic choice).  DS_PATH_TWO_PASS fits every row. */
+ds_status ds_debug_force_path(ds_path path);
+
+/* Bound, in nanoseconds, of every device-side wait (default 2e9). */
+ds_status ds_debug_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Launches one CTA that waits on a shared-memory barrier nothing will ever
+ * complete, bounded by limit_ns, so that the timeout path runs: afterwards
+ * ds_get_device_status returns DS_ERR_DEVICE_TIMEOUT.  No copy is in flight. */
+ds_status ds_debug_wait_timeout_selftest(uint64_t limit_ns, ds_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DS_H */

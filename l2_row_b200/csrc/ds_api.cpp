@@ -1,0 +1,505 @@
+// ds_api.cpp -- the C ABI of libds: argument validation, row-class planning,
+// segment-table packing into kernel parameter blocks, and launches.
+//
+// Planning: every segment's row class depends on (operation, cols) only.
+// Segments of one class go into as few launches as the parameter block
+// allows (kSegPerLaunch segments each); a segment with more rows than a grid
+// can hold is split by rows (rows are independent).  Nothing is allocated.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "ds.h"
+#include "ds_internal.h"
+
+namespace {
+
+using ds::AParams;
+using ds::ASegK;
+using ds::RowClass;
+using ds::WParams;
+using ds::WSegK;
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_force_path{DS_PATH_AUTO};
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+constexpr int64_t kMaxCols = 0x7fffffff;
+constexpr int64_t kMaxGrid = 0x7fffffff;
+
+ds_status fail(ds_status s, const std::string &msg)
+{
+    g_last_error = msg;
+    return s;
+}
+
+std::string where(const char *what, int seg)
+{
+    char buf[96];
+    std::snprintf(buf, sizeof(buf), "segment %d: %s", seg, what);
+    return buf;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+RowClass classify(ds_op op, int64_t cols, int forced)
+{
+    const int64_t E = ds::elems_per_unit(op);
+    const int64_t nu = (cols + E - 1) / E;
+    const int64_t kmax = ds::kmax_of(op);
+    auto group_of = [&]() -> int {
+        for (int G = 32; G <= ds::kCta; G *= 2)
+            if ((nu + G - 1) / G <= kmax)
+                return G;
+        return 0;
+    };
+    auto cluster_of = [&]() -> int {
+        for (int CL = 2; CL <= ds::kMaxCluster; CL *= 2)
+            if ((nu + CL - 1) / CL <= ds::kCta * kmax)
+                return CL;
+        return 0;
+    };
+    switch (forced) {
+    case DS_PATH_WARP:
+        if (nu <= 32 * kmax)
+            return {DS_PATH_WARP, 32, 1};
+        break;
+    case DS_PATH_CTA:
+        if (nu <= ds::kCta * kmax)
+            return {DS_PATH_CTA, std::max(group_of(), 64), 1};
+        break;
+    case DS_PATH_CLUSTER:
+        if (const int CL = cluster_of())
+            return {DS_PATH_CLUSTER, 0, CL};
+        break;
+    case DS_PATH_TWO_PASS:
+        return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster};
+    default:
+        break;
+    }
+    if (const int G = group_of())
+        return {G == 32 ? DS_PATH_WARP : DS_PATH_CTA, G, 1};
+    if (const int CL = cluster_of())
+        return {DS_PATH_CLUSTER, 0, CL};
+    return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster};
+}
+
+// Work units of `rows` rows: CTAs (several rows each) or clusters (one row).
+int64_t units_for(const RowClass &rc, int64_t rows)
+{
+    if (rc.path == DS_PATH_WARP || rc.path == DS_PATH_CTA) {
+        const int64_t rpu = ds::kCta / rc.group;
+        return (rows + rpu - 1) / rpu;
+    }
+    return rows;
+}
+
+// ----------------------------------------------------------- overlap check --
+
+struct Span {
+    uintptr_t lo, hi;
+    int seg;
+    int role;   // 0 = read, 1 = written
+    int alias;  // allowed exact-alias key within a segment (-1: none)
+};
+
+// Byte span of a row-major matrix: through the end of its last row.
+Span span_of(const void *p, int64_t rows, int64_t cols, int64_t ld, int esize, int seg, int role, int alias)
+{
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+    const uintptr_t n = static_cast<uintptr_t>(((rows - 1) * ld + cols) * esize);
+    return {lo, lo + n, seg, role, alias};
+}
+
+ds_status check_overlaps(std::vector<Span> &spans)
+{
+    std::sort(spans.begin(), spans.end(), [](const Span &a, const Span &b) { return a.lo < b.lo; });
+    for (size_t i = 0; i < spans.size(); ++i) {
+        for (size_t j = i + 1; j < spans.size() && spans[j].lo < spans[i].hi; ++j) {
+            const Span &a = spans[i], &b = spans[j];
+            if (a.role == 0 && b.role == 0)
+                continue;
+            const bool exact = a.lo == b.lo && a.hi == b.hi && a.seg == b.seg && a.alias >= 0 &&
+                               a.alias == b.alias;
+            if (!exact)
+                return fail(DS_ERR_OVERLAP, where("an output overlaps another buffer of the call", b.seg));
+        }
+    }
+    return DS_OK;
+}
+
+ds_status check_common(int nseg, const void *segs, float eps, void *)
+{
+    if (nseg < 0)
+        return fail(DS_ERR_INVALID_ARG, "nseg < 0");
+    if (nseg > DS_MAX_SEGMENTS)
+        return fail(DS_ERR_TOO_MANY_SEGMENTS, "nseg above DS_MAX_SEGMENTS");
+    if (nseg > 0 && !segs)
+        return fail(DS_ERR_INVALID_ARG, "segs is NULL");
+    if (!(eps >= 0.f) || !std::isfinite(eps))
+        return fail(DS_ERR_INVALID_ARG, "eps must be finite and >= 0");
+    return DS_OK;
+}
+
+ds_status check_shape(int64_t rows, int64_t cols, int64_t ld, int i)
+{
+    if (rows < 0)
+        return fail(DS_ERR_INVALID_ARG, where("rows < 0", i));
+    if (cols < 1 || cols > kMaxCols)
+        return fail(DS_ERR_INVALID_ARG, where("cols outside [1, 2^31 - 1]", i));
+    if (ld < cols)
+        return fail(DS_ERR_INVALID_ARG, where("leading dimension < cols", i));
+    if (rows > 0 && ld > (int64_t(1) << 40))
+        return fail(DS_ERR_INVALID_ARG, where("leading dimension too large", i));
+    if (rows > (int64_t(1) << 40))
+        return fail(DS_ERR_INVALID_ARG, where("rows too large", i));
+    return DS_OK;
+}
+
+ds_status check_matrix(const void *p, int64_t rows, int64_t ld, int esize, const char *name, int i)
+{
+    if (rows == 0)
+        return DS_OK;
+    if (!p)
+        return fail(DS_ERR_INVALID_ARG, where((std::string(name) + " is NULL").c_str(), i));
+    if (!aligned(p, 16) || (ld * esize) % 16 != 0)
+        return fail(DS_ERR_ALIGNMENT, where((std::string(name) + " rows are not 16-byte aligned").c_str(), i));
+    return DS_OK;
+}
+
+// ------------------------------------------------------------- launching --
+
+// Splits, packs and launches.  `make(i, r0, nrows)` returns the device
+// segment for rows [r0, r0 + nrows) of segment i.
+template <class P, class SegK, class Make, class Launch>
+ds_status launch_all(ds_op op, int nseg, const int64_t *rows, const int64_t *cols, float eps, Make make,
+                     Launch launch, void *stream)
+{
+    const int forced = g_force_path.load(std::memory_order_relaxed);
+    std::vector<RowClass> cls(static_cast<size_t>(nseg));
+    std::vector<char> done(static_cast<size_t>(nseg), 0);
+    for (int i = 0; i < nseg; ++i)
+        cls[i] = classify(op, cols[i], forced);
+
+    static thread_local P params; // ~12 KB: kept off the stack
+    for (int first = 0; first < nseg; ++first) {
+        if (done[first] || rows[first] == 0)
+            continue;
+        const RowClass rc = cls[first];
+        const int64_t unit_cap = kMaxGrid / std::max(1, rc.cluster);
+        int n = 0;
+        int64_t units = 0;
+        auto flush = [&]() -> ds_status {
+            if (n == 0)
+                return DS_OK;
+            params.nseg = n;
+            params.unit_start[n] = units;
+            params.eps = eps;
+            params.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+            const int e = launch(rc, params, units, stream);
+            if (e != 0) {
+                char buf[160];
+                std::snprintf(buf, sizeof(buf), "kernel launch failed (cudaError %d)", e);
+                return fail(DS_ERR_CUDA, buf);
+            }
+            g_launches.fetch_add(1, std::memory_order_relaxed);
+            n = 0;
+            units = 0;
+            return DS_OK;
+        };
+        for (int i = first; i < nseg; ++i) {
+            if (done[i] || rows[i] == 0 || !ds::same_launch(cls[i], rc))
+                continue;
+            done[i] = 1;
+            const RowClass ci = cls[i];
+            // rows per piece so that one piece never exceeds a grid
+            const int64_t rows_per_unit = (ci.path == DS_PATH_WARP || ci.path == DS_PATH_CTA) ? ds::kCta / ci.group : 1;
+            for (int64_t r0 = 0; r0 < rows[i];) {
+                int64_t room = unit_cap - units;
+                if (n == ds::kSegPerLaunch || room <= 0) {
+                    if (ds_status s = flush())
+                        return s;
+                    room = unit_cap;
+                }
+                const int64_t nr = std::min(rows[i] - r0, room * rows_per_unit);
+                params.seg[n] = make(i, r0, nr);
+                params.seg[n].group = ci.group;
+                params.unit_start[n] = units;
+                units += units_for(ci, nr);
+                ++n;
+                r0 += nr;
+            }
+        }
+        if (ds_status s = flush())
+            return s;
+    }
+    return DS_OK;
+}
+
+WSegK wseg_rows(const ds_wseg &s, int64_t r0, int64_t nr, int out_esize, int gy_esize)
+{
+    WSegK k{};
+    k.w = s.w ? s.w + r0 * s.ld : nullptr;
+    k.gain = s.gain ? s.gain + r0 : nullptr;
+    k.out = s.w_eff ? static_cast<char *>(s.w_eff) + r0 * s.ld_out * out_esize : nullptr;
+    k.gy = s.gy ? static_cast<const char *>(s.gy) + r0 * s.ld_out * gy_esize : nullptr;
+    k.grad_w = s.grad_w ? s.grad_w + r0 * s.ld : nullptr;
+    k.grad_g = s.grad_g ? s.grad_g + r0 : nullptr;
+    k.rows = nr;
+    k.ld = s.ld;
+    k.ld_out = s.ld_out;
+    k.cols = static_cast<int32_t>(s.cols);
+    k.nu = static_cast<int32_t>((s.cols + 3) / 4);
+    k.radius = s.radius;
+    return k;
+}
+
+ASegK aseg_rows(const ds_aseg &s, int64_t r0, int64_t nr)
+{
+    ASegK k{};
+    k.x = s.x ? static_cast<const uint16_t *>(s.x) + r0 * s.ld : nullptr;
+    k.r = s.r ? static_cast<const uint16_t *>(s.r) + r0 * s.ld : nullptr;
+    k.y = s.y ? static_cast<uint16_t *>(s.y) + r0 * s.ld : nullptr;
+    k.alpha = s.alpha;
+    k.rows = nr;
+    k.ld = s.ld;
+    k.cols = static_cast<int32_t>(s.cols);
+    k.nu = static_cast<int32_t>((s.cols + 7) / 8);
+    return k;
+}
+
+enum WOp { W_FWD, W_BWD, W_RENORM };
+
+ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float eps, void *stream)
+{
+    g_last_error.clear();
+    if (ds_status s = check_common(nseg, segs, eps, stream))
+        return s;
+    if (wop != W_RENORM && dt != DS_F32 && dt != DS_BF16)
+        return fail(DS_ERR_UNSUPPORTED_DTYPE, "dtype must be DS_F32 or DS_BF16");
+    const int esize = dt == DS_BF16 ? 2 : 4;
+    std::vector<Span> spans;
+    std::vector<int64_t> rows(static_cast<size_t>(nseg)), cols(static_cast<size_t>(nseg));
+    for (int i = 0; i < nseg; ++i) {
+        const ds_wseg &s = segs[i];
+        if (ds_status st = check_shape(s.rows, s.cols, s.ld, i))
+            return st;
+        if (wop != W_RENORM && s.ld_out < s.cols)
+            return fail(DS_ERR_INVALID_ARG, where("ld_out < cols", i));
+        if (!std::isfinite(s.radius))
+            return fail(DS_ERR_INVALID_ARG, where("radius is not finite", i));
+        rows[i] = s.rows;
+        cols[i] = s.cols;
+        if (s.rows == 0)
+            continue;
+        if (ds_status st = check_matrix(s.w, s.rows, s.ld, 4, "w", i))
+            return st;
+        if (wop != W_RENORM && s.gain && !aligned(s.gain, 4))
+            return fail(DS_ERR_ALIGNMENT, where("gain is not 4-byte aligned", i));
+        if (wop == W_FWD) {
+            if (ds_status st = check_matrix(s.w_eff, s.rows, s.ld_out, esize, "w_eff", i))
+                return st;
+            spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 0, -1));
+            if (s.gain)
+                spans.push_back(span_of(s.gain, 1, s.rows, s.rows, 4, i, 0, -1));
+            spans.push_back(span_of(s.w_eff, s.rows, s.cols, s.ld_out, esize, i, 1, -1));
+        } else if (wop == W_BWD) {
+            if (ds_status st = check_matrix(s.gy, s.rows, s.ld_out, esize, "gy", i))
+                return st;
+            if (ds_status st = check_matrix(s.grad_w, s.rows, s.ld, 4, "grad_w", i))
+                return st;
+            if (s.gain && !s.grad_g)
+                return fail(DS_ERR_INVALID_ARG, where("grad_g is NULL while gain is set", i));
+            if (s.gain && !aligned(s.grad_g, 4))
+                return fail(DS_ERR_ALIGNMENT, where("grad_g is not 4-byte aligned", i));
+            spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 0, -1));
+            spans.push_back(span_of(s.gy, s.rows, s.cols, s.ld_out, esize, i, 0, -1));
+            spans.push_back(span_of(s.grad_w, s.rows, s.cols, s.ld, 4, i, 1, -1));
+            if (s.gain) {
+                spans.push_back(span_of(s.gain, 1, s.rows, s.rows, 4, i, 0, -1));
+                spans.push_back(span_of(s.grad_g, 1, s.rows, s.rows, 4, i, 1, -1));
+            }
+        } else {
+            spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 1, -1));
+        }
+    }
+    if (ds_status st = check_overlaps(spans))
+        return st;
+
+    const ds_op op = wop == W_FWD ? DS_OP_WN_FORWARD : wop == W_BWD ? DS_OP_WN_BACKWARD : DS_OP_ROW_RENORM;
+    auto make = [&](int i, int64_t r0, int64_t nr) {
+        WSegK k = wseg_rows(segs[i], r0, nr, esize, esize);
+        if (wop == W_RENORM)
+            k.out = k.w ? const_cast<float *>(k.w) : nullptr;
+        return k;
+    };
+    const bool bf16 = dt == DS_BF16;
+    auto launch = [&](const RowClass &rc, const WParams &p, int64_t units, void *st) -> int {
+        switch (wop) {
+        case W_FWD: return ds::launch_wn_forward(rc, p, units, bf16, st);
+        case W_BWD: return ds::launch_wn_backward(rc, p, units, bf16, st);
+        default: return ds::launch_row_renorm(rc, p, units, st);
+        }
+    };
+    return launch_all<WParams, WSegK>(op, nseg, rows.data(), cols.data(), eps, make, launch, stream);
+}
+
+ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *stream)
+{
+    g_last_error.clear();
+    if (ds_status s = check_common(nseg, segs, eps, stream))
+        return s;
+    std::vector<Span> spans;
+    std::vector<int64_t> rows(static_cast<size_t>(nseg)), cols(static_cast<size_t>(nseg));
+    for (int i = 0; i < nseg; ++i) {
+        const ds_aseg &s = segs[i];
+        if (ds_status st = check_shape(s.rows, s.cols, s.ld, i))
+            return st;
+        rows[i] = s.rows;
+        cols[i] = s.cols;
+        if (s.rows == 0)
+            continue;
+        if (ds_status st = check_matrix(s.x, s.rows, s.ld, 2, "x", i))
+            return st;
+        if (ds_status st = check_matrix(s.y, s.rows, s.ld, 2, "y", i))
+            return st;
+        if (slerp || s.r)
+            if (ds_status st = check_matrix(s.r, s.rows, s.ld, 2, slerp ? "r (out)" : "r", i))
+                return st;
+        if (slerp) {
+            if (!s.alpha)
+                return fail(DS_ERR_INVALID_ARG, where("alpha is NULL", i));
+            if (!aligned(s.alpha, 16))
+                return fail(DS_ERR_ALIGNMENT, where("alpha is not 16-byte aligned", i));
+            spans.push_back(span_of(s.alpha, 1, s.cols, s.cols, 4, i, 0, -1));
+        }
+        // y may be exactly x or exactly r (alias key = segment + 1)
+        spans.push_back(span_of(s.x, s.rows, s.cols, s.ld, 2, i, 0, i));
+        if (s.r)
+            spans.push_back(span_of(s.r, s.rows, s.cols, s.ld, 2, i, 0, i));
+        spans.push_back(span_of(s.y, s.rows, s.cols, s.ld, 2, i, 1, i));
+    }
+    if (ds_status st = check_overlaps(spans))
+        return st;
+    auto make = [&](int i, int64_t r0, int64_t nr) { return aseg_rows(segs[i], r0, nr); };
+    auto launch = [&](const RowClass &rc, const AParams &p, int64_t units, void *st) -> int {
+        return slerp ? ds::launch_slerp_rows(rc, p, units, st) : ds::launch_l2_rows(rc, p, units, st);
+    };
+    return launch_all<AParams, ASegK>(slerp ? DS_OP_SLERP_ROWS : DS_OP_L2_ROWS, nseg, rows.data(), cols.data(), eps,
+                                      make, launch, stream);
+}
+
+} // namespace
+
+extern "C" {
+
+ds_status ds_wn_forward(const ds_wseg *segs, int nseg, ds_dtype out_dtype, float eps, ds_stream stream)
+{
+    return run_weight(W_FWD, segs, nseg, out_dtype, eps, stream);
+}
+
+ds_status ds_wn_backward(const ds_wseg *segs, int nseg, ds_dtype gy_dtype, float eps, ds_stream stream)
+{
+    return run_weight(W_BWD, segs, nseg, gy_dtype, eps, stream);
+}
+
+ds_status ds_row_renorm(const ds_wseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_weight(W_RENORM, segs, nseg, DS_F32, eps, stream);
+}
+
+ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_act(false, segs, nseg, eps, stream);
+}
+
+ds_status ds_slerp_rows(const ds_aseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_act(true, segs, nseg, eps, stream);
+}
+
+const char *ds_status_string(ds_status status)
+{
+    switch (status) {
+    case DS_OK: return "ok";
+    case DS_ERR_INVALID_ARG: return "invalid argument";
+    case DS_ERR_ALIGNMENT: return "row start not 16-byte aligned";
+    case DS_ERR_UNSUPPORTED_DTYPE: return "unsupported dtype";
+    case DS_ERR_TOO_MANY_SEGMENTS: return "too many segments";
+    case DS_ERR_CUDA: return "CUDA error";
+    case DS_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case DS_ERR_OVERLAP: return "output overlaps another buffer";
+    }
+    return "unknown status";
+}
+
+const char *ds_last_error(void) { return g_last_error.c_str(); }
+
+ds_status ds_get_device_status(ds_stream stream)
+{
+    uint32_t code = 0, site = 0;
+    const int e = ds::read_and_clear_device_error(&code, &site, stream);
+    if (e != 0) {
+        char buf[96];
+        std::snprintf(buf, sizeof(buf), "device status read failed (cudaError %d)", e);
+        return fail(DS_ERR_CUDA, buf);
+    }
+    if (code == 0)
+        return DS_OK;
+    char buf[96];
+    std::snprintf(buf, sizeof(buf), "device error %u at site %u", code, site);
+    return fail(code == DS_ERR_DEVICE_TIMEOUT ? DS_ERR_DEVICE_TIMEOUT : DS_ERR_CUDA, buf);
+}
+
+uint64_t ds_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ds_version(void) { return 100; }
+
+ds_status ds_row_class(ds_op op, int64_t cols, int *path, int *group_threads, int *cluster_ctas)
+{
+    if (op < DS_OP_WN_FORWARD || op > DS_OP_SLERP_ROWS)
+        return fail(DS_ERR_INVALID_ARG, "unknown op");
+    if (cols < 1 || cols > kMaxCols)
+        return fail(DS_ERR_INVALID_ARG, "cols outside [1, 2^31 - 1]");
+    const RowClass rc = classify(op, cols, g_force_path.load(std::memory_order_relaxed));
+    if (path)
+        *path = rc.path;
+    if (group_threads)
+        *group_threads = rc.group;
+    if (cluster_ctas)
+        *cluster_ctas = rc.cluster;
+    return DS_OK;
+}
+
+ds_status ds_debug_force_path(ds_path path)
+{
+    if (path < DS_PATH_AUTO || path > DS_PATH_TWO_PASS)
+        return fail(DS_ERR_INVALID_ARG, "unknown path");
+    g_force_path.store(path, std::memory_order_relaxed);
+    return DS_OK;
+}
+
+ds_status ds_debug_set_wait_limit_ns(uint64_t limit_ns)
+{
+    g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    return DS_OK;
+}
+
+ds_status ds_debug_wait_timeout_selftest(uint64_t limit_ns, ds_stream stream)
+{
+    if (limit_ns > 10ull * 1000 * 1000 * 1000)
+        return fail(DS_ERR_INVALID_ARG, "limit above 10 s");
+    const int e = ds::launch_wait_selftest(limit_ns, stream);
+    if (e != 0)
+        return fail(DS_ERR_CUDA, "self-test launch failed");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return DS_OK;
+}
+
+} // extern "C"

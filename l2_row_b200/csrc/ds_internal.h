@@ -1,0 +1,116 @@
+// ds_internal.h -- structures shared by the host planner (ds_api.cpp) and the
+// sm_100a kernels (ds_kernels.cu).  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+
+#include "ds.h"
+
+#ifdef __CUDACC__
+#define DS_HD __host__ __device__
+#else
+#define DS_HD
+#endif
+
+namespace ds {
+
+// Every kernel runs 256-thread CTAs.
+constexpr int kCta = 256;
+constexpr int kWarps = kCta / 32;
+// Register paths hold at most kmax_of(op) 16-byte units of each input per
+// thread: 8 for one input (forward, renorm), 4 where two inputs are held
+// (backward: w and GY; l2 with residual; slerp: res and out).
+constexpr int kKmaxMax = 8;
+DS_HD constexpr int kmax_of(ds_op op) { return (op == DS_OP_WN_FORWARD || op == DS_OP_ROW_RENORM) ? 8 : 4; }
+// Largest cluster (portable limit).
+constexpr int kMaxCluster = 8;
+// Segments per launch (kernel parameter block); larger tables are split.
+constexpr int kSegPerLaunch = 128;
+// Two-pass path: units per thread per chunk, chunk size, pipeline stages.
+constexpr int kStreamK = 4;
+constexpr int kChunkUnits = kCta * kStreamK;
+constexpr int kStages = 4;
+
+// Row length in 16-byte units: weight ops work on quads of fp32 (w is fp32),
+// activation ops on octets of bf16.
+DS_HD constexpr int elems_per_unit(ds_op op) { return op <= DS_OP_ROW_RENORM ? 4 : 8; }
+
+struct RowClass {
+    int path;    // ds_path (never DS_PATH_AUTO)
+    int group;   // threads per row for WARP/CTA paths (32..256)
+    int cluster; // CTAs per row for CLUSTER/TWO_PASS paths (1 otherwise)
+};
+
+// Launch shape: every WARP/CTA-path segment of a call shares one group-kernel
+// launch (each segment carries its own threads-per-row); CLUSTER and TWO_PASS
+// segments share a launch per cluster size.
+inline bool same_launch(const RowClass &a, const RowClass &b)
+{
+    const bool ga = a.path == DS_PATH_WARP || a.path == DS_PATH_CTA;
+    const bool gb = b.path == DS_PATH_WARP || b.path == DS_PATH_CTA;
+    if (ga || gb)
+        return ga && gb;
+    return a.path == b.path && a.cluster == b.cluster;
+}
+
+// Device copy of one weight segment.
+struct WSegK {
+    const float *w;
+    const float *gain;
+    void *out;        // forward: w_eff; renorm: w
+    const void *gy;
+    float *grad_w;
+    float *grad_g;
+    int64_t rows;
+    int64_t ld;
+    int64_t ld_out;
+    int32_t cols;
+    int32_t nu;       // units per row
+    float radius;
+    int32_t group;    // threads per row on the group path (32..256)
+};
+
+// Device copy of one activation segment (bf16 carried as raw 16-bit words).
+struct ASegK {
+    const uint16_t *x;
+    const uint16_t *r;
+    uint16_t *y;
+    const float *alpha;
+    int64_t rows;
+    int64_t ld;
+    int32_t cols;
+    int32_t nu;
+    int32_t group;    // threads per row on the group path (32..256)
+    int32_t pad_;
+};
+
+template <class Seg>
+struct LaunchParams {
+    Seg seg[kSegPerLaunch];
+    int64_t unit_start[kSegPerLaunch + 1]; // prefix sums of work units
+    int32_t nseg;
+    float eps;
+    uint64_t wait_limit_ns;                // bound of every device-side wait
+};
+
+using WParams = LaunchParams<WSegK>;
+using AParams = LaunchParams<ASegK>;
+
+// Error word written by kernels (see ds_get_device_status).
+enum DeviceErrorSite : uint32_t {
+    kSiteStreamWait = 1,
+    kSiteStreamDrain = 2,
+    kSiteSelftest = 3,
+};
+
+// Launchers (ds_kernels.cu).  `units` = grid size in rows-groups (WARP/CTA)
+// or rows (CLUSTER/TWO_PASS); return cudaError_t as int.
+int launch_wn_forward(const RowClass &rc, const WParams &p, int64_t units, bool out_bf16, void *stream);
+int launch_wn_backward(const RowClass &rc, const WParams &p, int64_t units, bool gy_bf16, void *stream);
+int launch_row_renorm(const RowClass &rc, const WParams &p, int64_t units, void *stream);
+int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
+int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
+int launch_wait_selftest(uint64_t limit_ns, void *stream);
+int read_and_clear_device_error(uint32_t *code, uint32_t *site, void *stream);
+
+} // namespace ds

@@ -1,0 +1,278 @@
+"""Thin ctypes binding of libds (include/ds.h): argument marshalling only.
+
+Every step of the computation runs in the CUDA kernels of libds.so.  If the
+library has not been built (``python -m l2_row_b200.build``) importing this
+module raises: there is no CPU fallback.
+
+The five calls keep their C names and take lists of segments:
+
+    ds_wn_forward(segs, out_dtype, eps, stream=None)
+    ds_wn_backward(segs, gy_dtype, eps, stream=None)
+    ds_row_renorm(segs, eps, stream=None)
+    ds_l2_rows(segs, eps, stream=None)
+    ds_slerp_rows(segs, eps, stream=None)
+
+A segment is a ``WSeg`` / ``ASeg`` of CUDA tensors (2-D, unit column stride,
+row stride = leading dimension) or a raw ``ds_wseg`` / ``ds_aseg`` structure.
+``stream`` defaults to torch's current CUDA stream.  A failing call raises
+``DSError`` carrying the status code and the library's message.
+"""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+from dataclasses import dataclass
+from typing import Any, Sequence
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libds.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libds.so is not built ({LIB_PATH}); run `python -m l2_row_b200.build`")
+
+_lib = ct.CDLL(LIB_PATH)
+
+DS_OK, DS_ERR_INVALID_ARG, DS_ERR_ALIGNMENT, DS_ERR_UNSUPPORTED_DTYPE = 0, 1, 2, 3
+DS_ERR_TOO_MANY_SEGMENTS, DS_ERR_CUDA, DS_ERR_DEVICE_TIMEOUT, DS_ERR_OVERLAP = 4, 5, 6, 7
+DS_F32, DS_BF16 = 0, 1
+DS_OP_WN_FORWARD, DS_OP_WN_BACKWARD, DS_OP_ROW_RENORM, DS_OP_L2_ROWS, DS_OP_SLERP_ROWS = range(5)
+DS_PATH_AUTO, DS_PATH_WARP, DS_PATH_CTA, DS_PATH_CLUSTER, DS_PATH_TWO_PASS = range(5)
+DS_MAX_SEGMENTS = 65536
+PATH_NAMES = {DS_PATH_WARP: "warp", DS_PATH_CTA: "cta", DS_PATH_CLUSTER: "cluster", DS_PATH_TWO_PASS: "two_pass"}
+
+
+class ds_wseg(ct.Structure):
+    _fields_ = [("w", ct.c_void_p), ("gain", ct.c_void_p), ("w_eff", ct.c_void_p), ("gy", ct.c_void_p),
+                ("grad_w", ct.c_void_p), ("grad_g", ct.c_void_p), ("rows", ct.c_int64), ("cols", ct.c_int64),
+                ("ld", ct.c_int64), ("ld_out", ct.c_int64), ("radius", ct.c_float)]
+
+
+class ds_aseg(ct.Structure):
+    _fields_ = [("x", ct.c_void_p), ("r", ct.c_void_p), ("y", ct.c_void_p), ("alpha", ct.c_void_p),
+                ("rows", ct.c_int64), ("cols", ct.c_int64), ("ld", ct.c_int64)]
+
+
+_st = ct.c_int
+_lib.ds_wn_forward.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_wn_backward.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_row_renorm.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_l2_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_slerp_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_void_p]
+for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_l2_rows", "ds_slerp_rows",
+           "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
+           "ds_debug_wait_timeout_selftest"):
+    getattr(_lib, _f).restype = _st
+_lib.ds_status_string.argtypes = [ct.c_int]
+_lib.ds_status_string.restype = ct.c_char_p
+_lib.ds_last_error.argtypes = []
+_lib.ds_last_error.restype = ct.c_char_p
+_lib.ds_get_device_status.argtypes = [ct.c_void_p]
+_lib.ds_launch_count.argtypes = []
+_lib.ds_launch_count.restype = ct.c_uint64
+_lib.ds_version.argtypes = []
+_lib.ds_version.restype = ct.c_int
+_lib.ds_row_class.argtypes = [ct.c_int, ct.c_int64, ct.POINTER(ct.c_int), ct.POINTER(ct.c_int),
+                              ct.POINTER(ct.c_int)]
+_lib.ds_debug_force_path.argtypes = [ct.c_int]
+_lib.ds_debug_set_wait_limit_ns.argtypes = [ct.c_uint64]
+_lib.ds_debug_wait_timeout_selftest.argtypes = [ct.c_uint64, ct.c_void_p]
+
+#: every symbol include/ds.h declares
+EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_l2_rows", "ds_slerp_rows",
+           "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
+           "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest")
+
+
+def lib() -> ct.CDLL:
+    """The loaded libds.so (for direct C-ABI calls)."""
+    return _lib
+
+
+class DSError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.ds_status_string(status).decode()
+        detail = _lib.ds_last_error().decode()
+        super().__init__(f"{where}: {msg}" + (f" ({detail})" if detail else ""))
+
+
+def _check(status: int, where: str) -> None:
+    if status != DS_OK:
+        raise DSError(status, where)
+
+
+def _stream_ptr(stream) -> int | None:
+    if stream is None:
+        import torch
+
+        if not torch.cuda.is_available():
+            return None
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(dt) -> int:
+    if isinstance(dt, int):
+        return dt
+    s = str(dt).replace("torch.", "")
+    if s in ("bf16", "bfloat16"):
+        return DS_BF16
+    if s in ("f32", "float32", "float"):
+        return DS_F32
+    raise ValueError(f"unsupported dtype {dt!r}")
+
+
+# ------------------------------------------------------------ tensor views --
+
+def _mat(t, name: str, rows: int, cols: int) -> tuple[int, int]:
+    """(data_ptr, leading dimension) of a 2-D row-major view; (0, cols) for None."""
+    if t is None:
+        return 0, cols
+    if t.dim() != 2 or tuple(t.shape) != (rows, cols):
+        raise ValueError(f"{name}: expected shape ({rows}, {cols}), got {tuple(t.shape)}")
+    if t.stride(1) != 1 and cols > 1:
+        raise ValueError(f"{name}: columns must be contiguous")
+    return t.data_ptr(), (t.stride(0) if rows > 1 else max(t.stride(0), cols))
+
+
+def _vec(t) -> int:
+    if t is None:
+        return 0
+    if t.dim() != 1 or (t.numel() > 1 and t.stride(0) != 1):
+        raise ValueError("per-row vectors must be contiguous 1-D tensors")
+    return t.data_ptr()
+
+
+@dataclass
+class WSeg:
+    """One weight matrix.  w: fp32 [R, C]; gain: fp32 [R] or None; w_eff:
+    forward output [R, C]; gy, grad_w, grad_g: backward input/outputs."""
+
+    w: Any
+    gain: Any = None
+    w_eff: Any = None
+    gy: Any = None
+    grad_w: Any = None
+    grad_g: Any = None
+    radius: float = 1.0
+
+    def to_c(self) -> ds_wseg:
+        R, C = (int(self.w.shape[0]), int(self.w.shape[1]))
+        w, ld = _mat(self.w, "w", R, C)
+        weff, ld_out = _mat(self.w_eff, "w_eff", R, C)
+        gy, ld_gy = _mat(self.gy, "gy", R, C)
+        gw, ld_gw = _mat(self.grad_w, "grad_w", R, C)
+        if self.w_eff is not None and self.gy is not None and ld_out != ld_gy:
+            raise ValueError("w_eff and gy must share a leading dimension")
+        if self.grad_w is not None and ld_gw != ld:
+            raise ValueError("grad_w must share w's leading dimension")
+        return ds_wseg(w, _vec(self.gain), weff, gy, gw, _vec(self.grad_g), R, C, ld,
+                       ld_out if self.w_eff is not None else ld_gy, float(self.radius))
+
+
+@dataclass
+class ASeg:
+    """One activation matrix: x (slerp: res), r (slerp: out; l2: residual or
+    None), y output, alpha fp32 [C] (slerp only).  bf16 [R, C], shared ld."""
+
+    x: Any
+    y: Any
+    r: Any = None
+    alpha: Any = None
+
+    def to_c(self) -> ds_aseg:
+        R, C = (int(self.x.shape[0]), int(self.x.shape[1]))
+        x, ld = _mat(self.x, "x", R, C)
+        y, ldy = _mat(self.y, "y", R, C)
+        r, ldr = _mat(self.r, "r", R, C)
+        if ldy != ld or (self.r is not None and ldr != ld):
+            raise ValueError("x, r and y must share a leading dimension")
+        return ds_aseg(x, r, y, _vec(self.alpha), R, C, ld)
+
+
+def _table(segs, cls):
+    items = [s if isinstance(s, cls) else s.to_c() for s in segs]
+    arr = (cls * max(1, len(items)))(*items)
+    return arr, len(items)
+
+
+def ds_wn_forward(segs: Sequence, out_dtype="bf16", eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_wseg)
+    _check(_lib.ds_wn_forward(arr, n, _dtype_code(out_dtype), eps, _stream_ptr(stream)), "ds_wn_forward")
+
+
+def ds_wn_backward(segs: Sequence, gy_dtype="bf16", eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_wseg)
+    _check(_lib.ds_wn_backward(arr, n, _dtype_code(gy_dtype), eps, _stream_ptr(stream)), "ds_wn_backward")
+
+
+def ds_row_renorm(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_wseg)
+    _check(_lib.ds_row_renorm(arr, n, eps, _stream_ptr(stream)), "ds_row_renorm")
+
+
+def ds_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_aseg)
+    _check(_lib.ds_l2_rows(arr, n, eps, _stream_ptr(stream)), "ds_l2_rows")
+
+
+def ds_slerp_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_aseg)
+    _check(_lib.ds_slerp_rows(arr, n, eps, _stream_ptr(stream)), "ds_slerp_rows")
+
+
+def ds_get_device_status(stream=None) -> int:
+    """Synchronise the stream; return (and clear) the device error word."""
+    return int(_lib.ds_get_device_status(_stream_ptr(stream)))
+
+
+def ds_launch_count() -> int:
+    return int(_lib.ds_launch_count())
+
+
+def ds_version() -> int:
+    return int(_lib.ds_version())
+
+
+def ds_status_string(status: int) -> str:
+    return _lib.ds_status_string(status).decode()
+
+
+def ds_last_error() -> str:
+    return _lib.ds_last_error().decode()
+
+
+def ds_row_class(op: int, cols: int) -> tuple[int, int, int]:
+    """(path, threads per row, CTAs per row) the library picks for this row length."""
+    p, g, c = ct.c_int(), ct.c_int(), ct.c_int()
+    _check(_lib.ds_row_class(op, cols, ct.byref(p), ct.byref(g), ct.byref(c)), "ds_row_class")
+    return p.value, g.value, c.value
+
+
+def ds_debug_force_path(path: int) -> None:
+    _check(_lib.ds_debug_force_path(path), "ds_debug_force_path")
+
+
+def ds_debug_set_wait_limit_ns(limit_ns: int) -> None:
+    _check(_lib.ds_debug_set_wait_limit_ns(limit_ns), "ds_debug_set_wait_limit_ns")
+
+
+def ds_debug_wait_timeout_selftest(limit_ns: int, stream=None) -> None:
+    _check(_lib.ds_debug_wait_timeout_selftest(limit_ns, _stream_ptr(stream)), "ds_debug_wait_timeout_selftest")
+
+
+class force_path:
+    """Context manager: run the enclosed calls on one path (tests)."""
+
+    def __init__(self, path: int):
+        self.path = path
+
+    def __enter__(self):
+        ds_debug_force_path(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        ds_debug_force_path(DS_PATH_AUTO)
+        return False

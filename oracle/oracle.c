@@ -69,6 +69,12 @@ double or_bf16_value(uint16_t bits)
     return s ? -v : v;
 }
 
+void or_bf16_rne_array(const double *src, int64_t n, uint16_t *dst)
+{
+    for (int64_t i = 0; i < n; ++i)
+        dst[i] = or_bf16_rne(src[i]);
+}
+
 static double round_bf16(double v) { return or_bf16_value(or_bf16_rne(v)); }
 
 /* ------------------------------------------------------------------------ */

@@ -45,6 +45,8 @@ extern "C" {
 /* bf16 helpers.  or_bf16_rne rounds a double straight to bf16 bits. */
 uint16_t or_bf16_rne(double v);
 double   or_bf16_value(uint16_t bits);
+/* or_bf16_rne over an array (dst[i] = or_bf16_rne(src[i])). */
+void     or_bf16_rne_array(const double *src, int64_t n, uint16_t *dst);
 
 /* ---- one row, all values already exact doubles -------------------------- */
 

@@ -31,6 +31,8 @@ def lib() -> ct.CDLL:
         _lib.or_bf16_rne.restype = ct.c_uint16
         _lib.or_bf16_value.argtypes = [ct.c_uint16]
         _lib.or_bf16_value.restype = dbl
+        _lib.or_bf16_rne_array.argtypes = [vp, i64, vp]
+        _lib.or_bf16_rne_array.restype = None
         _lib.or_wn_forward.argtypes = [vp, i64, i64, i64, vp, dbl, dbl, uns, vp, i32]
         _lib.or_wn_backward.argtypes = [vp, i64, i64, i64, vp, i32, i64, vp, dbl, dbl, uns, vp, vp, i32]
         _lib.or_row_renorm.argtypes = [vp, i64, i64, i64, dbl, dbl, uns, vp, i32]
@@ -75,6 +77,14 @@ def _check(rc: int, name: str) -> None:
 
 def bf16_rne(v: float) -> int:
     return int(lib().or_bf16_rne(float(v)))
+
+
+def bf16_rne_array(a) -> np.ndarray:
+    """Round every double of `a` straight to bf16 bits (same shape, uint16)."""
+    src = np.ascontiguousarray(a, np.float64)
+    dst = np.empty(src.shape, np.uint16)
+    lib().or_bf16_rne_array(_p(src), src.size, _p(dst))
+    return dst
 
 
 def bf16_value(bits: int) -> float:

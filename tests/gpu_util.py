@@ -1,0 +1,220 @@
+"""GPU-side helpers for the parity tests: move seeded host inputs to the
+device, run the five calls through the C ABI (l2_row_b200.ds), and compare
+the results with the oracle by the rules in tests/checks.py."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from l2_row_b200 import ds
+from l2_row_b200 import workloads as wl
+from tests.checks import (SPREAD, bf16_interval_violations, bf16_ulp_violations, rel_violations)
+
+DEV = "cuda"
+CANARY_F32 = np.float32(-7.0e33)
+CANARY_BF16 = 0x7BAD
+
+
+# --------------------------------------------------------------- transfers --
+
+def dev_f32(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(DEV)
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(bits, np.uint16).view(np.int16))
+    return t.to(DEV).view(torch.bfloat16)
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def host_f32(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy()
+
+
+def padded(rows: int, cols: int, ld: int, dtype, canary) -> tuple[torch.Tensor, torch.Tensor]:
+    """A [rows, cols] view with leading dimension ld inside a buffer that has
+    one guard row before and after, every unused element set to `canary`.
+    Returns (view, whole buffer)."""
+    if dtype == torch.bfloat16:
+        buf = torch.full(((rows + 2) * ld,), canary, dtype=torch.int16, device=DEV).view(torch.bfloat16)
+    else:
+        buf = torch.full(((rows + 2) * ld,), float(canary), dtype=dtype, device=DEV)
+    view = buf[ld:ld + rows * ld].view(rows, ld)[:, :cols] if rows else buf[:0].view(0, cols)
+    return view, buf
+
+
+def guards_intact(buf: torch.Tensor, rows: int, cols: int, ld: int, canary) -> bool:
+    """Everything outside the [rows, cols] window still holds the canary."""
+    if buf.dtype == torch.bfloat16:
+        h = buf.view(torch.int16).cpu().numpy().view(np.uint16)
+    else:
+        h = buf.cpu().numpy()
+    mask = np.ones(h.shape, bool)
+    for r in range(rows):
+        mask[(r + 1) * ld:(r + 1) * ld + cols] = False
+    return bool(np.all(h[mask] == canary))
+
+
+def copy_into(view: torch.Tensor, src: torch.Tensor) -> None:
+    view.copy_(src)
+
+
+# ---------------------------------------------------------------- running --
+
+def run_forward(segs, out_dtype: str, eps: float, stream=None):
+    """segs: list of WeightSeg (host).  Returns list of output tensors."""
+    outs, cs = [], []
+    for s in segs:
+        w = dev_f32(s.w)
+        g = dev_f32(s.g) if s.g is not None else None
+        o = torch.empty(s.w.shape, dtype=torch.bfloat16 if out_dtype == "bf16" else torch.float32, device=DEV)
+        cs.append(ds.WSeg(w=w, gain=g, w_eff=o, radius=s.radius))
+        outs.append(o)
+    ds.ds_wn_forward(cs, out_dtype, eps, stream)
+    torch.cuda.synchronize()
+    return outs
+
+
+def run_backward(segs, gy_dtype: str, eps: float):
+    res, cs = [], []
+    for s in segs:
+        w = dev_f32(s.w)
+        g = dev_f32(s.g) if s.g is not None else None
+        gy = dev_bf16(s.gy) if gy_dtype == "bf16" else dev_f32(s.gy)
+        gw = torch.empty(s.w.shape, dtype=torch.float32, device=DEV)
+        gg = torch.empty(s.w.shape[0], dtype=torch.float32, device=DEV) if g is not None else None
+        cs.append(ds.WSeg(w=w, gain=g, gy=gy, grad_w=gw, grad_g=gg, radius=s.radius))
+        res.append((gw, gg))
+    ds.ds_wn_backward(cs, gy_dtype, eps)
+    torch.cuda.synchronize()
+    return res
+
+
+def run_renorm(segs, eps: float):
+    ws, cs = [], []
+    for s in segs:
+        w = dev_f32(s.w)
+        cs.append(ds.WSeg(w=w, radius=s.radius))
+        ws.append(w)
+    ds.ds_row_renorm(cs, eps)
+    torch.cuda.synchronize()
+    return ws
+
+
+def run_l2(acts, eps: float, residual: bool = True):
+    ys, cs = [], []
+    for a in acts:
+        x = dev_bf16(a.x)
+        r = dev_bf16(a.r) if (residual and a.r is not None) else None
+        y = torch.empty_like(x)
+        cs.append(ds.ASeg(x=x, r=r, y=y))
+        ys.append(y)
+    ds.ds_l2_rows(cs, eps)
+    torch.cuda.synchronize()
+    return ys
+
+
+def run_slerp(acts, eps: float):
+    hs, cs = [], []
+    for a in acts:
+        x, o = dev_bf16(a.x), dev_bf16(a.r)
+        h = torch.empty_like(x)
+        cs.append(ds.ASeg(x=x, r=o, y=h, alpha=dev_f32(a.alpha)))
+        hs.append(h)
+    ds.ds_slerp_rows(cs, eps)
+    torch.cuda.synchronize()
+    return hs
+
+
+# ------------------------------------------------------------ comparisons --
+
+def assert_bf16_rows(got_bits, ref_bits, lo=None, hi=None, what=""):
+    """1-ulp rule against the oracle's bits; where an interval is given, an
+    element outside 1 ulp must lie inside it (a legitimate fp32 outcome at a
+    slerp rounding point), and every element must lie inside it."""
+    bad = bf16_ulp_violations(got_bits, ref_bits)
+    if lo is not None:
+        outside = bf16_interval_violations(got_bits, lo, hi)
+        assert not outside.any(), f"{what}: {int(outside.sum())} outputs outside the fp32-spread interval " \
+                                  f"(first at {np.argwhere(outside)[0].tolist()})"
+        bad &= outside
+    assert not bad.any(), f"{what}: {int(bad.sum())} outputs beyond 1 bf16 ulp (first at {np.argwhere(bad)[0].tolist()})"
+
+
+def check_forward(seg, got: torch.Tensor, eps: float, out_dtype: str, rows=None, what="wn_forward"):
+    w = seg.w if rows is None else seg.w[rows]
+    g = None if seg.g is None else (seg.g if rows is None else seg.g[rows])
+    ref = oracle.wn_forward(w, g, rho=seg.radius, eps=eps, nthreads=oracle.default_threads())
+    got_h = got if rows is None else got[torch.as_tensor(rows, device=got.device)]
+    if out_dtype == "bf16":
+        gb = host_bits(got_h)
+        ref_bits = oracle.bf16_rne_array(ref)
+        lo = oracle.bf16_rne_array(ref - SPREAD * np.abs(ref))
+        hi = oracle.bf16_rne_array(ref + SPREAD * np.abs(ref))
+        assert_bf16_rows(gb, ref_bits, lo, hi, what)
+    else:
+        bad = rel_violations(host_f32(got_h), ref, 2e-6)
+        assert not bad.any(), f"{what}: {int(bad.sum())} fp32 outputs beyond 2e-6 relative"
+
+
+def check_backward(seg, gw: torch.Tensor, gg, eps: float, rows=None, what="wn_backward"):
+    sel = slice(None) if rows is None else rows
+    w, gy = seg.w[sel], seg.gy[sel]
+    g = None if seg.g is None else seg.g[sel]
+    ref_w, ref_g = oracle.wn_backward(w, gy, g, rho=seg.radius, eps=eps, nthreads=oracle.default_threads())
+    idx = None if rows is None else torch.as_tensor(rows, device=gw.device)
+    got_w = host_f32(gw if idx is None else gw[idx])
+    gy64 = (wl.bf16_bits_to_f32(gy) if gy.dtype == np.uint16 else gy).astype(np.float64)
+    w64 = w.astype(np.float64)
+    n = np.sqrt(np.einsum("ij,ij->i", w64, w64) + eps)
+    gabs = np.ones(len(w64)) if g is None else np.abs(g.astype(np.float64))
+    rms = np.sqrt(np.mean(gy64 ** 2, axis=1))
+    floor = (gabs * seg.radius / n * rms)[:, None]
+    bad = rel_violations(got_w, ref_w, 1e-5, floor)
+    assert not bad.any(), f"{what}: {int(bad.sum())} grad_w entries beyond tolerance " \
+                          f"(first at {np.argwhere(bad)[0].tolist()})"
+    if g is not None:
+        got_g = host_f32(gg if idx is None else gg[idx])
+        fl = seg.radius * np.linalg.norm(gy64, axis=1)
+        badg = rel_violations(got_g, ref_g, 1e-5, fl)
+        assert not badg.any(), f"{what}: {int(badg.sum())} grad_g entries beyond tolerance"
+
+
+def check_renorm(seg, got: torch.Tensor, eps: float, rows=None, what="row_renorm"):
+    w = seg.w if rows is None else seg.w[rows]
+    ref = oracle.row_renorm(w, rho=seg.radius, eps=eps, nthreads=oracle.default_threads())
+    got_h = host_f32(got if rows is None else got[torch.as_tensor(rows, device=got.device)])
+    bad = rel_violations(got_h, ref, 2e-6)
+    assert not bad.any(), f"{what}: {int(bad.sum())} fp32 outputs beyond 2e-6 relative"
+
+
+def check_l2(act, got: torch.Tensor, eps: float, residual=True, rows=None, what="l2_rows", flags=0):
+    sel = slice(None) if rows is None else rows
+    x = act.x[sel]
+    r = act.r[sel] if (residual and act.r is not None) else None
+    nt = oracle.default_threads()
+    ref = oracle.l2_rows(x, r, eps=eps, flags=flags, nthreads=nt)
+    lo, hi = oracle.l2_rows_interval(x, r, eps=eps, delta=SPREAD, flags=flags, nthreads=nt)
+    gb = host_bits(got if rows is None else got[torch.as_tensor(rows, device=got.device)])
+    assert_bf16_rows(gb, ref, lo, hi, what)
+
+
+def check_slerp(act, got: torch.Tensor, eps: float, rows=None, what="slerp_rows", flags=0):
+    sel = slice(None) if rows is None else rows
+    x, o = act.x[sel], act.r[sel]
+    nt = oracle.default_threads()
+    ref = oracle.slerp_rows(x, o, act.alpha, eps=eps, flags=flags, nthreads=nt)
+    lo, hi = oracle.slerp_rows_interval(x, o, act.alpha, eps=eps, delta=SPREAD, flags=flags, nthreads=nt)
+    gb = host_bits(got if rows is None else got[torch.as_tensor(rows, device=got.device)])
+    assert_bf16_rows(gb, ref, lo, hi, what)
+
+
+def sample_rows(n: int, k: int, seed: int, must=()) -> np.ndarray:
+    """Sorted unique sample of k rows plus the first, the last and `must`."""
+    rng = np.random.default_rng(seed)
+    pick = set(rng.choice(n, size=min(k, n), replace=False).tolist()) | {0, n - 1} | set(int(m) for m in must)
+    return np.array(sorted(pick), np.int64)

@@ -1,0 +1,229 @@
+"""The C ABI without a GPU: the library loads, exports every symbol
+include/ds.h declares, plans row classes from (op, cols) alone, and rejects
+bad arguments on the host before any launch (no kernel runs here)."""
+from __future__ import annotations
+
+import ctypes as ct
+import os
+import re
+
+import pytest
+
+from l2_row_b200 import ds
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions() -> set[str]:
+    src = open(os.path.join(ROOT, "include", "ds.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(ds_[a-z_0-9]+)\s*\(", src))
+
+
+def test_every_declared_symbol_is_exported():
+    decl = declared_functions()
+    assert decl == set(ds.EXPORTS)
+    for name in decl:
+        assert hasattr(ds.lib(), name), name
+
+
+def test_status_strings_and_version():
+    for code in range(8):
+        assert ds.ds_status_string(code) not in ("", "unknown status")
+    assert ds.ds_status_string(99) == "unknown status"
+    assert ds.ds_version() >= 100
+
+
+# ------------------------------------------------------------- row classes --
+
+W_OPS = (ds.DS_OP_WN_FORWARD, ds.DS_OP_WN_BACKWARD, ds.DS_OP_ROW_RENORM)
+A_OPS = (ds.DS_OP_L2_ROWS, ds.DS_OP_SLERP_ROWS)
+
+
+@pytest.mark.parametrize("op,cols,want", [
+    (ds.DS_OP_WN_FORWARD, 768, (ds.DS_PATH_WARP, 32, 1)),     # 192 quads, 6 per lane
+    (ds.DS_OP_WN_FORWARD, 2048, (ds.DS_PATH_CTA, 64, 1)),
+    (ds.DS_OP_WN_BACKWARD, 768, (ds.DS_PATH_CTA, 64, 1)),     # two inputs: 4 units per thread
+    (ds.DS_OP_WN_BACKWARD, 2048, (ds.DS_PATH_CTA, 128, 1)),
+    (ds.DS_OP_ROW_RENORM, 128, (ds.DS_PATH_WARP, 32, 1)),
+    (ds.DS_OP_L2_ROWS, 4096, (ds.DS_PATH_CTA, 128, 1)),
+    (ds.DS_OP_SLERP_ROWS, 7168, (ds.DS_PATH_CTA, 256, 1)),
+    (ds.DS_OP_L2_ROWS, 16384, (ds.DS_PATH_CLUSTER, 0, 2)),
+    (ds.DS_OP_WN_FORWARD, 14336, (ds.DS_PATH_CLUSTER, 0, 2)),
+    (ds.DS_OP_WN_BACKWARD, 14336, (ds.DS_PATH_CLUSTER, 0, 4)),
+    (ds.DS_OP_WN_FORWARD, 131072, (ds.DS_PATH_TWO_PASS, 0, 8)),
+    (ds.DS_OP_SLERP_ROWS, 262144, (ds.DS_PATH_TWO_PASS, 0, 8)),
+])
+def test_row_class_for_workload_shapes(op, cols, want):
+    assert ds.ds_row_class(op, cols) == want
+
+
+def test_row_class_is_monotone_and_fits():
+    order = {ds.DS_PATH_WARP: 0, ds.DS_PATH_CTA: 1, ds.DS_PATH_CLUSTER: 2, ds.DS_PATH_TWO_PASS: 3}
+    for op in W_OPS + A_OPS:
+        e = 4 if op in W_OPS else 8
+        kmax = 8 if op in (ds.DS_OP_WN_FORWARD, ds.DS_OP_ROW_RENORM) else 4
+        prev = (0, 0, 0)
+        for cols in sorted(set(list(range(1, 600, 7)) + [2 ** k + d for k in range(9, 19) for d in (-1, 0, 1)])):
+            path, g, cl = ds.ds_row_class(op, cols)
+            nu = -(-cols // e)
+            if path in (ds.DS_PATH_WARP, ds.DS_PATH_CTA):
+                assert -(-nu // g) <= kmax and g in (32, 64, 128, 256)
+            elif path == ds.DS_PATH_CLUSTER:
+                assert -(-nu // cl) <= 256 * kmax and cl in (2, 4, 8)
+            key = (order[path], g, cl)
+            assert key >= prev, (op, cols)
+            prev = key
+
+
+def test_forced_paths():
+    with ds.force_path(ds.DS_PATH_TWO_PASS):
+        assert ds.ds_row_class(ds.DS_OP_L2_ROWS, 128)[0] == ds.DS_PATH_TWO_PASS
+    with ds.force_path(ds.DS_PATH_CLUSTER):
+        assert ds.ds_row_class(ds.DS_OP_WN_FORWARD, 768) == (ds.DS_PATH_CLUSTER, 0, 2)
+    with ds.force_path(ds.DS_PATH_WARP):  # does not fit: automatic choice
+        assert ds.ds_row_class(ds.DS_OP_L2_ROWS, 4096)[0] == ds.DS_PATH_CTA
+    with ds.force_path(ds.DS_PATH_CTA):
+        assert ds.ds_row_class(ds.DS_OP_WN_FORWARD, 128) == (ds.DS_PATH_CTA, 64, 1)
+    assert ds.ds_row_class(ds.DS_OP_L2_ROWS, 128)[0] == ds.DS_PATH_WARP
+    with pytest.raises(ds.DSError):
+        ds.ds_debug_force_path(9)
+
+
+# ------------------------------------------------------ host-side validation --
+# Fake, never dereferenced device addresses: every call below fails on the
+# host before anything is launched.
+
+BASE = 0x7F0000000000
+
+
+def wseg(**kw):
+    d = dict(w=BASE, gain=0, w_eff=BASE + (1 << 30), gy=BASE + (2 << 30), grad_w=BASE + (3 << 30),
+             grad_g=0, rows=4, cols=8, ld=8, ld_out=8, radius=1.0)
+    d.update(kw)
+    return ds.ds_wseg(**d)
+
+
+def aseg(**kw):
+    d = dict(x=BASE, r=0, y=BASE + (1 << 30), alpha=BASE + (2 << 30), rows=4, cols=8, ld=8)
+    d.update(kw)
+    return ds.ds_aseg(**d)
+
+
+def call_w(fn, segs, dt=ds.DS_BF16, eps=1e-6):
+    arr = (ds.ds_wseg * max(1, len(segs)))(*segs)
+    if fn == "ds_row_renorm":
+        return getattr(ds.lib(), fn)(arr, len(segs), ct.c_float(eps), None)
+    return getattr(ds.lib(), fn)(arr, len(segs), dt, ct.c_float(eps), None)
+
+
+def call_a(fn, segs, eps=1e-6):
+    arr = (ds.ds_aseg * max(1, len(segs)))(*segs)
+    return getattr(ds.lib(), fn)(arr, len(segs), ct.c_float(eps), None)
+
+
+@pytest.mark.parametrize("fn", ["ds_wn_forward", "ds_wn_backward", "ds_row_renorm"])
+def test_weight_validation(fn):
+    E = ds
+    before = ds.ds_launch_count()
+    assert call_w(fn, [wseg(rows=-1)]) == E.DS_ERR_INVALID_ARG
+    assert call_w(fn, [wseg(cols=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_w(fn, [wseg(ld=4)]) == E.DS_ERR_INVALID_ARG
+    assert call_w(fn, [wseg(w=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_w(fn, [wseg(w=BASE + 4)]) == E.DS_ERR_ALIGNMENT
+    assert call_w(fn, [wseg(ld=10, cols=8)]) == E.DS_ERR_ALIGNMENT          # 40-byte rows
+    assert call_w(fn, [wseg()], eps=-1.0) == E.DS_ERR_INVALID_ARG
+    assert call_w(fn, [wseg()], eps=float("nan")) == E.DS_ERR_INVALID_ARG
+    assert call_w(fn, [wseg()], eps=float("inf")) == E.DS_ERR_INVALID_ARG
+    assert call_w(fn, [wseg(radius=float("nan"))]) == E.DS_ERR_INVALID_ARG
+    arr = (ds.ds_wseg * 1)(wseg())
+    if fn == "ds_row_renorm":
+        assert getattr(ds.lib(), fn)(None, 1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
+        assert getattr(ds.lib(), fn)(arr, -1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
+        assert getattr(ds.lib(), fn)(arr, E.DS_MAX_SEGMENTS + 1, ct.c_float(1e-6), None) == \
+            E.DS_ERR_TOO_MANY_SEGMENTS
+    else:
+        assert call_w(fn, [wseg()], dt=7) == E.DS_ERR_UNSUPPORTED_DTYPE
+        assert call_w(fn, [wseg(ld_out=4)]) == E.DS_ERR_INVALID_ARG
+    # empty work launches nothing and succeeds without touching the device
+    assert call_w(fn, []) == E.DS_OK
+    assert call_w(fn, [wseg(rows=0, w=0, w_eff=0, gy=0, grad_w=0)]) == E.DS_OK
+    assert ds.ds_launch_count() == before
+    assert "segment 0" in ds.ds_last_error() or ds.ds_last_error() == ""
+
+
+def test_weight_specific_validation():
+    E = ds
+    assert call_w("ds_wn_forward", [wseg(w_eff=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_w("ds_wn_forward", [wseg(w_eff=BASE + (1 << 30) + 8)]) == E.DS_ERR_ALIGNMENT
+    assert call_w("ds_wn_backward", [wseg(gy=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_w("ds_wn_backward", [wseg(grad_w=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_w("ds_wn_backward", [wseg(gain=BASE + (4 << 30), grad_g=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_w("ds_wn_backward", [wseg(gain=BASE + (4 << 30) + 2, grad_g=BASE + (5 << 30))]) == \
+        E.DS_ERR_ALIGNMENT
+    # bf16 W_eff rows need ld_out % 8 == 0; fp32 rows need ld_out % 4 == 0
+    assert call_w("ds_wn_forward", [wseg(ld_out=12, ld=12)]) == E.DS_ERR_ALIGNMENT
+    assert ds.ds_last_error().startswith("segment 0")
+
+
+def test_weight_overlap_rejected():
+    E = ds
+    # W_eff over w
+    assert call_w("ds_wn_forward", [wseg(w_eff=BASE + 16)], dt=ds.DS_F32) == E.DS_ERR_OVERLAP
+    # grad_w over gy, even exactly
+    assert call_w("ds_wn_backward", [wseg(grad_w=BASE + (2 << 30))], dt=ds.DS_F32) == E.DS_ERR_OVERLAP
+    # two segments writing the same rows
+    a = wseg()
+    b = wseg(w=BASE + (8 << 30))
+    assert call_w("ds_wn_forward", [a, b]) == E.DS_ERR_OVERLAP
+    # renorm of two overlapping segments
+    assert call_w("ds_row_renorm", [wseg(), wseg(w=BASE + 64)]) == E.DS_ERR_OVERLAP
+    # backward grad_g overlapping the gain vector
+    assert call_w("ds_wn_backward", [wseg(gain=BASE + (4 << 30), grad_g=BASE + (4 << 30) + 4)]) == \
+        E.DS_ERR_OVERLAP
+
+
+@pytest.mark.parametrize("fn", ["ds_l2_rows", "ds_slerp_rows"])
+def test_activation_validation(fn):
+    E = ds
+    slerp = fn == "ds_slerp_rows"
+    r = BASE + (3 << 30)
+    good = dict(r=r) if slerp else {}
+    assert call_a(fn, [aseg(rows=-1, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_a(fn, [aseg(cols=0, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_a(fn, [aseg(ld=7, cols=8, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_a(fn, [aseg(ld=12, cols=8, **good)]) == E.DS_ERR_ALIGNMENT   # 24-byte bf16 rows
+    assert call_a(fn, [aseg(x=0, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_a(fn, [aseg(y=0, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_a(fn, [aseg(x=BASE + 2, **good)]) == E.DS_ERR_ALIGNMENT
+    assert call_a(fn, [aseg(**good)], eps=-1e-6) == E.DS_ERR_INVALID_ARG
+    # partial overlap of y with x is refused (exact aliasing is allowed: tested on the GPU)
+    assert call_a(fn, [aseg(y=BASE + 16, **good)]) == E.DS_ERR_OVERLAP
+    assert call_a(fn, [aseg(**good), aseg(x=BASE + (6 << 30), y=BASE + (1 << 30) + 16, **good)]) == \
+        E.DS_ERR_OVERLAP
+    if slerp:
+        assert call_a(fn, [aseg()]) == E.DS_ERR_INVALID_ARG                # out is required
+        assert call_a(fn, [aseg(r=r, alpha=0)]) == E.DS_ERR_INVALID_ARG
+        assert call_a(fn, [aseg(r=r, alpha=BASE + (2 << 30) + 4)]) == E.DS_ERR_ALIGNMENT
+    else:
+        assert call_a(fn, [aseg(r=BASE + 2)]) == E.DS_ERR_ALIGNMENT
+    assert call_a(fn, []) == E.DS_OK
+    assert call_a(fn, [aseg(rows=0, x=0, y=0, alpha=0)]) == E.DS_OK
+
+
+def test_binding_marshals_tensors_and_rejects_bad_views():
+    import torch
+
+    w = torch.zeros(4, 8)
+    seg = ds.WSeg(w=w, w_eff=torch.zeros(4, 8, dtype=torch.bfloat16))
+    c = seg.to_c()
+    assert (c.rows, c.cols, c.ld, c.ld_out) == (4, 8, 8, 8)
+    wide = torch.zeros(4, 16)
+    c = ds.WSeg(w=wide[:, :8], w_eff=torch.zeros(4, 8)).to_c()
+    assert (c.ld, c.cols) == (16, 8)
+    with pytest.raises(ValueError):
+        ds.WSeg(w=w, w_eff=torch.zeros(3, 8)).to_c()
+    with pytest.raises(ValueError):
+        ds.WSeg(w=w.t().contiguous().t(), w_eff=torch.zeros(4, 8)).to_c()
+    a = ds.ASeg(x=torch.zeros(2, 16, dtype=torch.bfloat16), y=torch.zeros(2, 16, dtype=torch.bfloat16)).to_c()
+    assert (a.rows, a.cols, a.ld, a.r) == (2, 16, 16, None)

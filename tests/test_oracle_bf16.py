@@ -122,3 +122,11 @@ def test_matches_torch_for_float32_values():
                                     (2.0 / 3.0, 0x3F2B), (2 ** -0.5, 0x3F35)])
 def test_hand_values(v, bits):
     assert oracle.bf16_rne(v) == bits
+
+
+def test_array_rounding_matches_scalar():
+    rng = np.random.default_rng(9)
+    v = np.concatenate([rng.standard_normal(3000) * np.exp2(rng.integers(-140, 130, 3000)),
+                        [0.0, -0.0, np.inf, -np.inf, 1e300]])
+    arr = oracle.bf16_rne_array(v)
+    assert [int(b) for b in arr] == [oracle.bf16_rne(float(x)) for x in v]

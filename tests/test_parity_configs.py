@@ -1,0 +1,141 @@
+"""GPU parity at the workloads' full sizes, in the launch configuration the
+benchmark times (one call per operation over the whole segment table), on
+sampled rows the oracle computes one by one:
+
+* MLP pair: up [2048,768] + down [768,2048] (compared in full);
+* activation rows [16384,4096] with 1% of rows scaled by 1e3;
+* the whole 12-layer d_model-768 decoder: 85 weight segments in one call;
+* wide rows: weights [14336,4096], [4096,14336]; activations [8192,7168], [4096,16384];
+* rows past the single-pass limit: [6,131072] fp32 weights, [4,262144] bf16 activations.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from l2_row_b200 import ds
+from l2_row_b200 import workloads as wl
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+def test_mlp_pair_full():
+    wk = wl.mlp_pair(0)
+    outs = gu.run_forward(wk.weights, "bf16", wk.eps)
+    grads = gu.run_backward(wk.weights, "bf16", wk.eps)
+    ws = gu.run_renorm(wk.weights, wk.eps)
+    for s, o, (gw, gg), w in zip(wk.weights, outs, grads, ws):
+        gu.check_forward(s, o, wk.eps, "bf16", what=f"{s.name} forward")
+        gu.check_backward(s, gw, gg, wk.eps, what=f"{s.name} backward")
+        gu.check_renorm(s, w, wk.eps, what=f"{s.name} renorm")
+
+
+@pytest.fixture(scope="module")
+def activations():
+    return wl.activations(0)
+
+
+def test_activation_rows_sampled(activations):
+    a = activations.acts[0]
+    # every spiked row (x or r scaled by 1e3) plus a random sample
+    scale = np.abs(wl.bf16_bits_to_f32(a.x)).max(axis=1) + np.abs(wl.bf16_bits_to_f32(a.r)).max(axis=1)
+    spiked = np.nonzero(scale > 100)[0]
+    assert len(spiked) >= 300
+    rows = gu.sample_rows(a.rows, 512, 1, must=spiked)
+    (y0,) = gu.run_l2([a], activations.eps, residual=False)
+    gu.check_l2(a, y0, activations.eps, residual=False, rows=rows, what="l2 without residual")
+    (y1,) = gu.run_l2([a], activations.eps, residual=True)
+    gu.check_l2(a, y1, activations.eps, residual=True, rows=rows, what="l2 with residual")
+    (h,) = gu.run_slerp([a], activations.eps)
+    gu.check_slerp(a, h, activations.eps, rows=rows, what="slerp")
+
+
+@pytest.fixture(scope="module")
+def whole_model():
+    return wl.whole_model(0)
+
+
+def test_whole_model_one_call(whole_model):
+    wk = whole_model
+    assert len(wk.weights) == 85
+    assert sum(s.rows for s in wk.weights) == 114944
+    assert sum(s.w.size for s in wk.weights) == 100073472
+    before = ds.ds_launch_count()
+    outs = gu.run_forward(wk.weights, "bf16", wk.eps)
+    launches = ds.ds_launch_count() - before
+    assert launches == 1, launches            # 768- and 2048-wide rows share the group-kernel launch
+    grads = gu.run_backward(wk.weights, "bf16", wk.eps)
+    ws = gu.run_renorm(wk.weights, wk.eps)
+    for i, (s, o, (gw, gg), w) in enumerate(zip(wk.weights, outs, grads, ws)):
+        rows = gu.sample_rows(s.rows, 6 if s.rows < 30000 else 64, 100 + i)
+        gu.check_forward(s, o, wk.eps, "bf16", rows=rows, what=f"{s.name} forward")
+        gu.check_backward(s, gw, gg, wk.eps, rows=rows, what=f"{s.name} backward")
+        gu.check_renorm(s, w, wk.eps, rows=rows, what=f"{s.name} renorm")
+
+
+@pytest.fixture(scope="module")
+def wide():
+    return wl.wide(0)
+
+
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
+def test_wide_weights(wide, out_dtype):
+    for i, s in enumerate(wide.weights):
+        rows = gu.sample_rows(s.rows, 48, 200 + i)
+        (o,) = gu.run_forward([s], out_dtype, wide.eps)
+        gu.check_forward(s, o, wide.eps, out_dtype, rows=rows, what=f"{s.name} forward {out_dtype}")
+        del o
+        if out_dtype == "bf16":
+            (gw, gg), = gu.run_backward([s], "bf16", wide.eps)
+            gu.check_backward(s, gw, gg, wide.eps, rows=rows, what=f"{s.name} backward")
+            del gw, gg
+            (w,) = gu.run_renorm([s], wide.eps)
+            gu.check_renorm(s, w, wide.eps, rows=rows, what=f"{s.name} renorm")
+        torch.cuda.empty_cache()
+
+
+def test_wide_activations(wide):
+    for i, a in enumerate(wide.acts):
+        rows = gu.sample_rows(a.rows, 48, 300 + i)
+        for res in (False, True):
+            (y,) = gu.run_l2([a], wide.eps, residual=res)
+            gu.check_l2(a, y, wide.eps, residual=res, rows=rows, what=f"{a.name} l2 residual={res}")
+        (h,) = gu.run_slerp([a], wide.eps)
+        gu.check_slerp(a, h, wide.eps, rows=rows, what=f"{a.name} slerp")
+
+
+def test_wide_forced_two_pass(wide):
+    """The streaming path on the wide shapes agrees with the oracle too."""
+    with ds.force_path(ds.DS_PATH_TWO_PASS):
+        s = wide.weights[1]
+        rows = gu.sample_rows(s.rows, 24, 400)
+        (o,) = gu.run_forward([s], "bf16", wide.eps)
+        gu.check_forward(s, o, wide.eps, "bf16", rows=rows, what="two-pass forward")
+        (gw, gg), = gu.run_backward([s], "bf16", wide.eps)
+        gu.check_backward(s, gw, gg, wide.eps, rows=rows, what="two-pass backward")
+        a = wide.acts[1]
+        rows = gu.sample_rows(a.rows, 24, 401)
+        (y,) = gu.run_l2([a], wide.eps)
+        gu.check_l2(a, y, wide.eps, rows=rows, what="two-pass l2")
+        (h,) = gu.run_slerp([a], wide.eps)
+        gu.check_slerp(a, h, wide.eps, rows=rows, what="two-pass slerp")
+
+
+def test_long_rows_two_pass():
+    wk = wl.long_rows(0)
+    s, a = wk.weights[0], wk.acts[0]
+    assert ds.ds_row_class(ds.DS_OP_WN_FORWARD, s.cols)[0] == ds.DS_PATH_TWO_PASS
+    assert ds.ds_row_class(ds.DS_OP_SLERP_ROWS, a.cols)[0] == ds.DS_PATH_TWO_PASS
+    (o,) = gu.run_forward([s], "bf16", wk.eps)
+    gu.check_forward(s, o, wk.eps, "bf16", what="long forward")
+    (gw, gg), = gu.run_backward([s], "bf16", wk.eps)
+    gu.check_backward(s, gw, gg, wk.eps, what="long backward")
+    (w,) = gu.run_renorm([s], wk.eps)
+    gu.check_renorm(s, w, wk.eps, what="long renorm")
+    for res in (False, True):
+        (y,) = gu.run_l2([a], wk.eps, residual=res)
+        gu.check_l2(a, y, wk.eps, residual=res, what=f"long l2 residual={res}")
+    (h,) = gu.run_slerp([a], wk.eps)
+    gu.check_slerp(a, h, wk.eps, what="long slerp")
