@@ -359,14 +359,27 @@ __device__ __forceinline__ int rescale_exponent(float S, float eps, Red &red, Ge
     return m;
 }
 
+// The row's factor as two parts: result = (entry * pre) * inv.  pre is 1
+// except for rows of subnormals at eps = 0 (m > 100), where 2^m / n would
+// pass FLT_MAX: 2^(m-100) then rides on the entries (both parts are exact
+// powers of two times the rounded inverse, so the product rounds once, as
+// 2^m / n would).
+struct RowScale {
+    float inv;
+    float pre;
+};
+
 template <class Red, class Gen>
-__device__ __forceinline__ float row_inv(float S, float eps, Red &red, Gen &&gen)
+__device__ __forceinline__ RowScale row_scale(float S, float eps, Red &red, Gen &&gen)
 {
     float Ss = S;
     const int m = rescale_exponent(S, eps, red, gen, Ss);
     if (m == 0)
-        return 1.0f / sqrtf(S + eps);
-    return scalbnf(1.0f / sqrtf(Ss + scalbnf(eps, 2 * m)), m);
+        return {1.0f / sqrtf(S + eps), 1.f};
+    const float inv = 1.0f / sqrtf(Ss + scalbnf(eps, 2 * m));
+    if (m > 100)
+        return {scalbnf(inv, 100), scalbnf(1.f, m - 100)};
+    return {scalbnf(inv, m), 1.f};
 }
 
 // ------------------------------------------------ mbarrier + bulk copies --

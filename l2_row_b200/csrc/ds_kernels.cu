@@ -105,9 +105,9 @@ __device__ __forceinline__ void store_octet(uint16_t *row, int u, int cols, uint
     }
 }
 
-__device__ __forceinline__ float4 scale4(float4 v, float s)
+__device__ __forceinline__ float4 scale4(float4 v, float pre, float s)
 {
-    return make_float4(v.x * s, v.y * s, v.z * s, v.w * s);
+    return make_float4((v.x * pre) * s, (v.y * pre) * s, (v.z * pre) * s, (v.w * pre) * s);
 }
 
 __device__ __forceinline__ void acc_sq4(float &acc, float4 v)
@@ -167,13 +167,15 @@ __device__ __forceinline__ uint4 add_bf16x8(uint4 a, uint4 b)
     return s;
 }
 
-__device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float s)
+// bf16(v * pre * s) for the 8 entries (see RowScale for `pre`).
+__device__ __forceinline__ uint4 scale_bf16x8(uint4 v, RowScale r)
 {
+    const float p = r.pre, s = r.inv;
     uint4 o;
-    o.x = pack_bf2(bf_lo(v.x) * s, bf_hi(v.x) * s);
-    o.y = pack_bf2(bf_lo(v.y) * s, bf_hi(v.y) * s);
-    o.z = pack_bf2(bf_lo(v.z) * s, bf_hi(v.z) * s);
-    o.w = pack_bf2(bf_lo(v.w) * s, bf_hi(v.w) * s);
+    o.x = pack_bf2((bf_lo(v.x) * p) * s, (bf_hi(v.x) * p) * s);
+    o.y = pack_bf2((bf_lo(v.y) * p) * s, (bf_hi(v.y) * p) * s);
+    o.z = pack_bf2((bf_lo(v.z) * p) * s, (bf_hi(v.z) * p) * s);
+    o.w = pack_bf2((bf_lo(v.w) * p) * s, (bf_hi(v.w) * p) * s);
     return o;
 }
 
@@ -193,8 +195,10 @@ __device__ __forceinline__ void alpha8(const float *alpha, int u, int cols, floa
     m[7] = fabsf(b.w);
 }
 
-// The lerp t = a + |alpha| (b - a): the difference, then one fused rounding.
-__device__ __forceinline__ float lerp_t(float a, float b, float m) { return fmaf(m, b - a, a); }
+// The lerp t = a + |alpha| (b - a): the difference, then one fused rounding
+// (exact at |alpha| = 0; at |alpha| = 1 the definition gives b, taken as is,
+// since b - a itself may round when a and b are far apart in magnitude).
+__device__ __forceinline__ float lerp_t(float a, float b, float m) { return m == 1.f ? b : fmaf(m, b - a, a); }
 
 // ===================================================== register-row bodies ==
 //
@@ -220,12 +224,12 @@ __device__ __forceinline__ void wn_scale_row(const WSegK &sg, int64_t row, bool 
     for (int k = 0; k < KMAX; ++k)
         acc_sq4(acc[0], x[k]);
     red.sum(acc);
-    const float inv = row_inv(acc[0], eps, red, [&](auto f) {
+    const RowScale rs = row_scale(acc[0], eps, red, [&](auto f) {
 #pragma unroll
         for (int k = 0; k < KMAX; ++k)
             each4(x[k], f);
     });
-    const float sc = (g * sg.radius) * inv;
+    const float sc = (g * sg.radius) * rs.inv;
     if (!active)
         return;
     void *out = RENORM ? static_cast<void *>(const_cast<float *>(sg.w) + row * sg.ld)
@@ -235,7 +239,7 @@ __device__ __forceinline__ void wn_scale_row(const WSegK &sg, int64_t row, bool 
     for (int k = 0; k < KMAX; ++k) {
         const int u = ubeg + lane + k * stride;
         if (u < uend)
-            store_quad<OUT_BF16>(out, u, sg.cols, scale4(x[k], sc));
+            store_quad<OUT_BF16>(out, u, sg.cols, scale4(x[k], rs.pre, sc));
     }
 }
 
@@ -345,7 +349,7 @@ __device__ __forceinline__ void l2_row(const ASegK &sg, int64_t row, bool active
     for (int k = 0; k < KMAX; ++k)
         acc_sq8(acc[0], s[k]);
     red.sum(acc);
-    const float inv = row_inv(acc[0], eps, red, [&](auto f) {
+    const RowScale rs = row_scale(acc[0], eps, red, [&](auto f) {
 #pragma unroll
         for (int k = 0; k < KMAX; ++k)
             each8(s[k], f);
@@ -357,7 +361,7 @@ __device__ __forceinline__ void l2_row(const ASegK &sg, int64_t row, bool active
     for (int k = 0; k < KMAX; ++k) {
         const int u = ubeg + lane + k * stride;
         if (u < uend)
-            store_octet(y, u, sg.cols, scale_bf16x8(s[k], inv));
+            store_octet(y, u, sg.cols, scale_bf16x8(s[k], rs));
     }
 }
 
@@ -382,12 +386,12 @@ __device__ __forceinline__ void slerp_row(const ASegK &sg, int64_t row, bool act
         acc_sq8(acc[1], b[k]);
     }
     red.sum(acc);
-    const float inv_a = row_inv(acc[0], eps, red, [&](auto f) {
+    const RowScale ra = row_scale(acc[0], eps, red, [&](auto f) {
 #pragma unroll
         for (int k = 0; k < KMAX; ++k)
             each8(a[k], f);
     });
-    const float inv_b = row_inv(acc[1], eps, red, [&](auto f) {
+    const RowScale rb = row_scale(acc[1], eps, red, [&](auto f) {
 #pragma unroll
         for (int k = 0; k < KMAX; ++k)
             each8(b[k], f);
@@ -395,8 +399,8 @@ __device__ __forceinline__ void slerp_row(const ASegK &sg, int64_t row, bool act
     // the rounding points a = bf16(l2(res)), b = bf16(l2(out))
 #pragma unroll
     for (int k = 0; k < KMAX; ++k) {
-        a[k] = scale_bf16x8(a[k], inv_a);
-        b[k] = scale_bf16x8(b[k], inv_b);
+        a[k] = scale_bf16x8(a[k], ra);
+        b[k] = scale_bf16x8(b[k], rb);
     }
     auto each_t = [&](auto f) {
 #pragma unroll
@@ -412,7 +416,7 @@ __device__ __forceinline__ void slerp_row(const ASegK &sg, int64_t row, bool act
     float at[1] = {0.f};
     each_t([&](float t) { at[0] = fmaf(t, t, at[0]); });
     red.sum(at);
-    const float inv_t = row_inv(at[0], eps, red, each_t);
+    const RowScale rt = row_scale(at[0], eps, red, each_t);
     if (!active)
         return;
     uint16_t *y = sg.y + row * sg.ld;
@@ -425,7 +429,7 @@ __device__ __forceinline__ void slerp_row(const ASegK &sg, int64_t row, bool act
             float h[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                h[e] = lerp_t(bf_get(a[k], e), bf_get(b[k], e), m[e]) * inv_t;
+                h[e] = (lerp_t(bf_get(a[k], e), bf_get(b[k], e), m[e]) * rt.pre) * rt.inv;
             store_octet(y, u, sg.cols,
                         make_uint4(pack_bf2(h[0], h[1]), pack_bf2(h[2], h[3]), pack_bf2(h[4], h[5]),
                                    pack_bf2(h[6], h[7])));
@@ -538,7 +542,7 @@ struct SScale {
     const WSegK &sg;
     int64_t row;
     float eps;
-    float acc = 0.f, sc = 0.f;
+    float acc = 0.f, sc = 0.f, pre = 1.f;
 
     __device__ SScale(const WSegK &s, int64_t r, float e) : sg(s), row(r), eps(e) {}
     __device__ int unit_bytes(int) const { return 16; }
@@ -556,7 +560,7 @@ struct SScale {
             void *out = RENORM ? static_cast<void *>(const_cast<float *>(sg.w) + row * sg.ld)
                                : static_cast<void *>(static_cast<char *>(sg.out) +
                                                      row * sg.ld_out * (OUT_BF16 ? 2 : 4));
-            store_quad<OUT_BF16>(out, u, c.cols, scale4(v, sc));
+            store_quad<OUT_BF16>(out, u, c.cols, scale4(v, pre, sc));
         }
     }
 
@@ -566,12 +570,13 @@ struct SScale {
         float a[1] = {acc};
         red.sum(a);
         const float *w = sg.w + row * sg.ld;
-        const float inv = row_inv(a[0], eps, red, [&](auto f) {
+        const RowScale rs = row_scale(a[0], eps, red, [&](auto f) {
             for (int ul = threadIdx.x; ul < c.len; ul += kCta)
                 each4(quad_f32(w, c.ubeg + ul, c.cols), f);
         });
         const float g = (!RENORM && sg.gain) ? __ldg(sg.gain + row) : 1.f;
-        sc = (g * sg.radius) * inv;
+        sc = (g * sg.radius) * rs.inv;
+        pre = rs.pre;
     }
     __device__ void finish(bool, bool) {}
 };
@@ -673,7 +678,8 @@ struct SL2 {
     const ASegK &sg;
     int64_t row;
     float eps;
-    float acc = 0.f, inv = 0.f;
+    float acc = 0.f;
+    RowScale rs{0.f, 1.f};
 
     __device__ SL2(const ASegK &s, int64_t r, float e) : sg(s), row(r), eps(e) {}
     __device__ int unit_bytes(int a) const { return (a == 0 || sg.r) ? 16 : 0; }
@@ -698,7 +704,7 @@ struct SL2 {
         if (pass == 0)
             acc_sq8(acc, s);
         else if (store)
-            store_octet(sg.y + row * sg.ld, u, c.cols, scale_bf16x8(s, inv));
+            store_octet(sg.y + row * sg.ld, u, c.cols, scale_bf16x8(s, rs));
     }
 
     template <class Red>
@@ -708,7 +714,7 @@ struct SL2 {
         red.sum(a);
         const uint16_t *x = sg.x + row * sg.ld;
         const uint16_t *r = sg.r ? sg.r + row * sg.ld : nullptr;
-        inv = row_inv(a[0], eps, red, [&](auto f) {
+        rs = row_scale(a[0], eps, red, [&](auto f) {
             for (int ul = threadIdx.x; ul < c.len; ul += kCta) {
                 const int u = c.ubeg + ul;
                 uint4 s = ld16(x + 8 * u);
@@ -729,7 +735,7 @@ struct SSlerp {
     int64_t row;
     float eps;
     float acc[2] = {0.f, 0.f};
-    float inv_a = 0.f, inv_b = 0.f, inv_t = 0.f;
+    RowScale ra{0.f, 1.f}, rb{0.f, 1.f}, rt{0.f, 1.f};
 
     __device__ SSlerp(const ASegK &s, int64_t r, float e) : sg(s), row(r), eps(e) {}
     __device__ int unit_bytes(int) const { return 16; }
@@ -739,10 +745,10 @@ struct SSlerp {
     }
 
     template <class F>
-    __device__ __forceinline__ void each_t(uint4 ra, uint4 rb, int u, int cols, F &&f) const
+    __device__ __forceinline__ void each_t(uint4 xa, uint4 xb, int u, int cols, F &&f) const
     {
-        const uint4 a = scale_bf16x8(ra, inv_a);
-        const uint4 b = scale_bf16x8(rb, inv_b);
+        const uint4 a = scale_bf16x8(xa, ra);
+        const uint4 b = scale_bf16x8(xb, rb);
         float m[8];
         alpha8(sg.alpha, u, cols, m);
 #pragma unroll
@@ -753,22 +759,22 @@ struct SSlerp {
     __device__ __forceinline__ void consume(int pass, const unsigned char *const *st, int j, int u,
                                             const StreamCtx &c, bool store)
     {
-        uint4 ra = *reinterpret_cast<const uint4 *>(st[0] + 16 * j);
-        uint4 rb = *reinterpret_cast<const uint4 *>(st[1] + 16 * j);
+        uint4 xa = *reinterpret_cast<const uint4 *>(st[0] + 16 * j);
+        uint4 xb = *reinterpret_cast<const uint4 *>(st[1] + 16 * j);
         const int valid = c.cols - 8 * u;
         if (valid < 8) {
-            ra = mask_octet(ra, valid);
-            rb = mask_octet(rb, valid);
+            xa = mask_octet(xa, valid);
+            xb = mask_octet(xb, valid);
         }
         if (pass == 0) {
-            acc_sq8(acc[0], ra);
-            acc_sq8(acc[1], rb);
+            acc_sq8(acc[0], xa);
+            acc_sq8(acc[1], xb);
         } else if (pass == 1) {
-            each_t(ra, rb, u, c.cols, [&](float t) { acc[0] = fmaf(t, t, acc[0]); });
+            each_t(xa, xb, u, c.cols, [&](float t) { acc[0] = fmaf(t, t, acc[0]); });
         } else if (store) {
             float h[8];
             int e = 0;
-            each_t(ra, rb, u, c.cols, [&](float t) { h[e++] = t * inv_t; });
+            each_t(xa, xb, u, c.cols, [&](float t) { h[e++] = (t * rt.pre) * rt.inv; });
             store_octet(sg.y + row * sg.ld, u, c.cols,
                         make_uint4(pack_bf2(h[0], h[1]), pack_bf2(h[2], h[3]), pack_bf2(h[4], h[5]),
                                    pack_bf2(h[6], h[7])));
@@ -782,11 +788,11 @@ struct SSlerp {
         const uint16_t *orow = sg.r + row * sg.ld;
         if (pass == 0) {
             red.sum(acc);
-            inv_a = row_inv(acc[0], eps, red, [&](auto f) {
+            ra = row_scale(acc[0], eps, red, [&](auto f) {
                 for (int ul = threadIdx.x; ul < c.len; ul += kCta)
                     each8(octet(xr, c.ubeg + ul, c.cols), f);
             });
-            inv_b = row_inv(acc[1], eps, red, [&](auto f) {
+            rb = row_scale(acc[1], eps, red, [&](auto f) {
                 for (int ul = threadIdx.x; ul < c.len; ul += kCta)
                     each8(octet(orow, c.ubeg + ul, c.cols), f);
             });
@@ -794,7 +800,7 @@ struct SSlerp {
         } else {
             float a[1] = {acc[0]};
             red.sum(a);
-            inv_t = row_inv(a[0], eps, red, [&](auto f) {
+            rt = row_scale(a[0], eps, red, [&](auto f) {
                 for (int ul = threadIdx.x; ul < c.len; ul += kCta) {
                     const int u = c.ubeg + ul;
                     each_t(octet(xr, u, c.cols), octet(orow, u, c.cols), u, c.cols, f);

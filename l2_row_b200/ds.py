@@ -132,6 +132,8 @@ def _mat(t, name: str, rows: int, cols: int) -> tuple[int, int]:
         return 0, cols
     if t.dim() != 2 or tuple(t.shape) != (rows, cols):
         raise ValueError(f"{name}: expected shape ({rows}, {cols}), got {tuple(t.shape)}")
+    if rows == 0:
+        return t.data_ptr(), cols
     if t.stride(1) != 1 and cols > 1:
         raise ValueError(f"{name}: columns must be contiguous")
     return t.data_ptr(), (t.stride(0) if rows > 1 else max(t.stride(0), cols))

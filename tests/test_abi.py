@@ -227,3 +227,11 @@ def test_binding_marshals_tensors_and_rejects_bad_views():
         ds.WSeg(w=w.t().contiguous().t(), w_eff=torch.zeros(4, 8)).to_c()
     a = ds.ASeg(x=torch.zeros(2, 16, dtype=torch.bfloat16), y=torch.zeros(2, 16, dtype=torch.bfloat16)).to_c()
     assert (a.rows, a.cols, a.ld, a.r) == (2, 16, 16, None)
+
+
+def test_binding_accepts_empty_tensors_with_any_strides():
+    import torch
+
+    w = torch.zeros(64, 0).t()          # shape (0, 64), stride (1, 0)
+    c = ds.WSeg(w=w, w_eff=torch.zeros(0, 64)).to_c()
+    assert (c.rows, c.cols) == (0, 64)

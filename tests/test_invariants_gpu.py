@@ -148,7 +148,9 @@ def test_power_of_two_scale_invariance_eps0(path):
 
 def test_extreme_magnitudes_match_oracle():
     """Rows whose fp32 sum of squares overflows (|x| ~ 1e30) or, at eps = 0,
-    underflows (|x| ~ 1e-30) still match the float64 oracle."""
+    underflows (|x| ~ 1e-30, and rows of fp32 subnormals ~ 1e-42) still match
+    the float64 oracle.  (The backward of a subnormal row overflows fp32
+    legitimately -- 1/n > FLT_MAX -- so it is checked at 1e-30 and above.)"""
     rng = np.random.default_rng(7)
     for scale, eps in ((1e30, 1e-6), (3e37, 0.0), (1e-30, 0.0), (1e-42, 0.0)):
         x = wl.to_bf16_bits((rng.standard_normal((8, 1000)) * scale).astype(np.float32))
@@ -159,8 +161,9 @@ def test_extreme_magnitudes_match_oracle():
         s = wl.WeightSeg("w", w, wl.gains(rng, 8), rng.standard_normal((8, 1000)).astype(np.float32))
         (o,) = gu.run_forward([s], "f32", eps)
         gu.check_forward(s, o, eps, "f32", what=f"forward scale={scale}")
-        (gw, gg), = gu.run_backward([s], "f32", eps)
-        gu.check_backward(s, gw, gg, eps, what=f"backward scale={scale}")
+        if scale >= 1e-30:
+            (gw, gg), = gu.run_backward([s], "f32", eps)
+            gu.check_backward(s, gw, gg, eps, what=f"backward scale={scale}")
 
 
 def test_degenerate_rows():

@@ -73,7 +73,8 @@ def test_ragged_weight_rows_with_guards(path):
             ld = ((cols + 7) // 8) * 8 + 8            # padded rows, 16-byte aligned for fp32 and bf16
             seg = wl.WeightSeg("r", wl.drifted_rows(rng, rows, cols, 0.5), wl.gains(rng, rows),
                                wl.normal_bf16(rng, (rows, cols)))
-            w = gu.dev_f32(seg.w)
+            w, _ = gu.padded(rows, cols, ld, torch.float32, gu.CANARY_F32)
+            w.copy_(gu.dev_f32(seg.w))
             g = gu.dev_f32(seg.g)
             out, buf = gu.padded(rows, cols, ld, torch.bfloat16, gu.CANARY_BF16)
             ds.ds_wn_forward([ds.WSeg(w=w, gain=g, w_eff=out)], "bf16", eps)
@@ -82,7 +83,8 @@ def test_ragged_weight_rows_with_guards(path):
             gu.check_forward(seg, out, eps, "bf16", what=f"forward cols={cols}")
             gw, gbuf = gu.padded(rows, cols, ld, torch.float32, gu.CANARY_F32)
             gg = torch.empty(rows, device="cuda")
-            gy = gu.dev_bf16(seg.gy)
+            gy, _ = gu.padded(rows, cols, ld, torch.bfloat16, gu.CANARY_BF16)
+            gy.copy_(gu.dev_bf16(seg.gy))
             ds.ds_wn_backward([ds.WSeg(w=w, gain=g, gy=gy, grad_w=gw, grad_g=gg)], "bf16", eps)
             torch.cuda.synchronize()
             assert gu.guards_intact(gbuf, rows, cols, ld, gu.CANARY_F32), cols
@@ -139,9 +141,16 @@ def test_empty_segments_mixed_in():
     assert ds.ds_launch_count() == before
 
 
-def test_exact_aliasing_allowed():
+@pytest.mark.parametrize("path", [ds.DS_PATH_AUTO, ds.DS_PATH_CLUSTER, ds.DS_PATH_TWO_PASS],
+                         ids=["auto", "cluster", "two_pass"])
+def test_exact_aliasing_allowed(path):
     rng = np.random.default_rng(24)
     act = wl.ActRows("a", wl.normal_bf16(rng, (64, 1000)), wl.normal_bf16(rng, (64, 1000)), wl.alpha_vec(rng, 1000))
+    with ds.force_path(path):
+        _aliasing(act)
+
+
+def _aliasing(act):
     (ref,) = gu.run_l2([act], 1e-6)
     (href,) = gu.run_slerp([act], 1e-6)
     for alias in ("x", "r"):
