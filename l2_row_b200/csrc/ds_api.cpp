@@ -14,6 +14,8 @@
 #include <string>
 #include <vector>
 
+#include <cuda_runtime.h>
+
 #include "ds.h"
 #include "ds_internal.h"
 
@@ -48,13 +50,28 @@ std::string where(const char *what, int seg)
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Bytes a row stages in shared memory on the warp-per-row path, for the
+// widest layout of the operation (fp32 GY; a residual present), so that the
+// path -- and with it the row's arithmetic -- depends on (op, cols) only.
+int64_t tile_row_bytes_worst(ds_op op, int64_t cols)
+{
+    const int64_t q = (cols + 3) / 4 * 16, o = (cols + 7) / 8 * 16;
+    switch (op) {
+    case DS_OP_WN_FORWARD:
+    case DS_OP_ROW_RENORM: return q;
+    case DS_OP_WN_BACKWARD: return 2 * q;
+    default: return 2 * o;
+    }
+}
+
 RowClass classify(ds_op op, int64_t cols, int forced)
 {
     const int64_t E = ds::elems_per_unit(op);
     const int64_t nu = (cols + E - 1) / E;
     const int64_t kmax = ds::kmax_of(op);
+    const bool tile = tile_row_bytes_worst(op, cols) <= ds::kTileSlotBytes;
     auto group_of = [&]() -> int {
-        for (int G = 32; G <= ds::kCta; G *= 2)
+        for (int G = 64; G <= ds::kCta; G *= 2)
             if ((nu + G - 1) / G <= kmax)
                 return G;
         return 0;
@@ -67,37 +84,77 @@ RowClass classify(ds_op op, int64_t cols, int forced)
     };
     switch (forced) {
     case DS_PATH_WARP:
-        if (nu <= 32 * kmax)
-            return {DS_PATH_WARP, 32, 1};
+        if (tile)
+            return {DS_PATH_WARP, 32, 1, 0};
         break;
     case DS_PATH_CTA:
-        if (nu <= ds::kCta * kmax)
-            return {DS_PATH_CTA, std::max(group_of(), 64), 1};
+        if (const int G = group_of())
+            return {DS_PATH_CTA, G, 1, 0};
         break;
     case DS_PATH_CLUSTER:
         if (const int CL = cluster_of())
-            return {DS_PATH_CLUSTER, 0, CL};
+            return {DS_PATH_CLUSTER, 0, CL, 0};
         break;
     case DS_PATH_TWO_PASS:
-        return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster};
+        return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0};
     default:
         break;
     }
+    if (tile)
+        return {DS_PATH_WARP, 32, 1, 0};
     if (const int G = group_of())
-        return {G == 32 ? DS_PATH_WARP : DS_PATH_CTA, G, 1};
+        return {DS_PATH_CTA, G, 1, 0};
     if (const int CL = cluster_of())
-        return {DS_PATH_CLUSTER, 0, CL};
-    return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster};
+        return {DS_PATH_CLUSTER, 0, CL, 0};
+    return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0};
 }
 
-// Work units of `rows` rows: CTAs (several rows each) or clusters (one row).
+// Rows per shared-memory slot on the warp-per-row path for the actual
+// layout (staged arrays of this segment), at most kTileMaxRowsPerSlot.
+int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r)
+{
+    const int64_t q = (cols + 3) / 4, o = (cols + 7) / 8;
+    int64_t bytes = 0;
+    switch (op) {
+    case DS_OP_WN_FORWARD:
+    case DS_OP_ROW_RENORM: bytes = q * 16; break;
+    case DS_OP_WN_BACKWARD: bytes = q * 16 + (q * gy_esize * 4 + 15) / 16 * 16; break;
+    case DS_OP_L2_ROWS: bytes = o * 16 * (has_r ? 2 : 1); break;
+    default: bytes = o * 32; break;
+    }
+    return static_cast<int>(std::min<int64_t>(ds::kTileMaxRowsPerSlot, ds::kTileSlotBytes / bytes));
+}
+
+int sm_count()
+{
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Rows per work unit: a shared-memory slot (warp-per-row path), a CTA
+// (register group path), or one row (a cluster per row).
+int64_t rows_per_unit(const RowClass &rc)
+{
+    if (rc.path == DS_PATH_WARP)
+        return rc.rps;
+    if (rc.path == DS_PATH_CTA)
+        return ds::kCta / rc.group;
+    return 1;
+}
+
 int64_t units_for(const RowClass &rc, int64_t rows)
 {
-    if (rc.path == DS_PATH_WARP || rc.path == DS_PATH_CTA) {
-        const int64_t rpu = ds::kCta / rc.group;
-        return (rows + rpu - 1) / rpu;
-    }
-    return rows;
+    const int64_t rpu = rows_per_unit(rc);
+    return (rows + rpu - 1) / rpu;
 }
 
 // ----------------------------------------------------------- overlap check --
@@ -178,14 +235,10 @@ ds_status check_matrix(const void *p, int64_t rows, int64_t ld, int esize, const
 // Splits, packs and launches.  `make(i, r0, nrows)` returns the device
 // segment for rows [r0, r0 + nrows) of segment i.
 template <class P, class SegK, class Make, class Launch>
-ds_status launch_all(ds_op op, int nseg, const int64_t *rows, const int64_t *cols, float eps, Make make,
+ds_status launch_all(int nseg, const int64_t *rows, const std::vector<RowClass> &cls, float eps, Make make,
                      Launch launch, void *stream)
 {
-    const int forced = g_force_path.load(std::memory_order_relaxed);
-    std::vector<RowClass> cls(static_cast<size_t>(nseg));
     std::vector<char> done(static_cast<size_t>(nseg), 0);
-    for (int i = 0; i < nseg; ++i)
-        cls[i] = classify(op, cols[i], forced);
 
     static thread_local P params; // ~12 KB: kept off the stack
     for (int first = 0; first < nseg; ++first) {
@@ -219,7 +272,7 @@ ds_status launch_all(ds_op op, int nseg, const int64_t *rows, const int64_t *col
             done[i] = 1;
             const RowClass ci = cls[i];
             // rows per piece so that one piece never exceeds a grid
-            const int64_t rows_per_unit = (ci.path == DS_PATH_WARP || ci.path == DS_PATH_CTA) ? ds::kCta / ci.group : 1;
+            const int64_t rpu = rows_per_unit(ci);
             for (int64_t r0 = 0; r0 < rows[i];) {
                 int64_t room = unit_cap - units;
                 if (n == ds::kSegPerLaunch || room <= 0) {
@@ -227,9 +280,9 @@ ds_status launch_all(ds_op op, int nseg, const int64_t *rows, const int64_t *col
                         return s;
                     room = unit_cap;
                 }
-                const int64_t nr = std::min(rows[i] - r0, room * rows_per_unit);
+                const int64_t nr = std::min(rows[i] - r0, room * rpu);
                 params.seg[n] = make(i, r0, nr);
-                params.seg[n].group = ci.group;
+                params.seg[n].group = ci.path == DS_PATH_WARP ? ci.rps : ci.group;
                 params.unit_start[n] = units;
                 units += units_for(ci, nr);
                 ++n;
@@ -333,6 +386,13 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         return st;
 
     const ds_op op = wop == W_FWD ? DS_OP_WN_FORWARD : wop == W_BWD ? DS_OP_WN_BACKWARD : DS_OP_ROW_RENORM;
+    const int forced = g_force_path.load(std::memory_order_relaxed);
+    std::vector<RowClass> cls(static_cast<size_t>(nseg));
+    for (int i = 0; i < nseg; ++i) {
+        cls[i] = classify(op, cols[i], forced);
+        if (cls[i].path == DS_PATH_WARP)
+            cls[i].rps = tile_rows_per_slot(op, cols[i], esize, true);
+    }
     auto make = [&](int i, int64_t r0, int64_t nr) {
         WSegK k = wseg_rows(segs[i], r0, nr, esize, esize);
         if (wop == W_RENORM)
@@ -341,13 +401,18 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
     };
     const bool bf16 = dt == DS_BF16;
     auto launch = [&](const RowClass &rc, const WParams &p, int64_t units, void *st) -> int {
+        if (rc.path == DS_PATH_WARP) {
+            const int tag = wop == W_FWD ? (bf16 ? 0 : 1) : wop == W_BWD ? (bf16 ? 2 : 3) : 4;
+            const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
+            return ds::launch_tile(tag, &p, grid, ds::kTileSlotBytes, ds::kMaxTileSlots, st);
+        }
         switch (wop) {
         case W_FWD: return ds::launch_wn_forward(rc, p, units, bf16, st);
         case W_BWD: return ds::launch_wn_backward(rc, p, units, bf16, st);
         default: return ds::launch_row_renorm(rc, p, units, st);
         }
     };
-    return launch_all<WParams, WSegK>(op, nseg, rows.data(), cols.data(), eps, make, launch, stream);
+    return launch_all<WParams, WSegK>(nseg, rows.data(), cls, eps, make, launch, stream);
 }
 
 ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *stream)
@@ -387,12 +452,23 @@ ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *st
     }
     if (ds_status st = check_overlaps(spans))
         return st;
+    const ds_op op = slerp ? DS_OP_SLERP_ROWS : DS_OP_L2_ROWS;
+    const int forced = g_force_path.load(std::memory_order_relaxed);
+    std::vector<RowClass> cls(static_cast<size_t>(nseg));
+    for (int i = 0; i < nseg; ++i) {
+        cls[i] = classify(op, cols[i], forced);
+        if (cls[i].path == DS_PATH_WARP)
+            cls[i].rps = tile_rows_per_slot(op, cols[i], 2, segs[i].r != nullptr);
+    }
     auto make = [&](int i, int64_t r0, int64_t nr) { return aseg_rows(segs[i], r0, nr); };
     auto launch = [&](const RowClass &rc, const AParams &p, int64_t units, void *st) -> int {
+        if (rc.path == DS_PATH_WARP) {
+            const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
+            return ds::launch_tile(slerp ? 6 : 5, &p, grid, ds::kTileSlotBytes, ds::kMaxTileSlots, st);
+        }
         return slerp ? ds::launch_slerp_rows(rc, p, units, st) : ds::launch_l2_rows(rc, p, units, st);
     };
-    return launch_all<AParams, ASegK>(slerp ? DS_OP_SLERP_ROWS : DS_OP_L2_ROWS, nseg, rows.data(), cols.data(), eps,
-                                      make, launch, stream);
+    return launch_all<AParams, ASegK>(nseg, rows.data(), cls, eps, make, launch, stream);
 }
 
 } // namespace

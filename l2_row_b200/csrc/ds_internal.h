@@ -26,6 +26,10 @@ DS_HD constexpr int kmax_of(ds_op op) { return (op == DS_OP_WN_FORWARD || op == 
 constexpr int kMaxCluster = 8;
 // Segments per launch (kernel parameter block); larger tables are split.
 constexpr int kSegPerLaunch = 128;
+// Warp-per-row (tile) path: ring of shared-memory slots filled by bulk copies.
+constexpr int kTileSlotBytes = 16384;  // rows whose staged input fits a slot
+constexpr int kMaxTileSlots = 13;      // 13 x 16 KB = 208 KB of the 227 KB per CTA
+constexpr int kTileMaxRowsPerSlot = 64;
 // Two-pass path: units per thread per chunk, chunk size, pipeline stages.
 constexpr int kStreamK = 4;
 constexpr int kChunkUnits = kCta * kStreamK;
@@ -37,20 +41,20 @@ DS_HD constexpr int elems_per_unit(ds_op op) { return op <= DS_OP_ROW_RENORM ? 4
 
 struct RowClass {
     int path;    // ds_path (never DS_PATH_AUTO)
-    int group;   // threads per row for WARP/CTA paths (32..256)
+    int group;   // threads per row: 32 on the WARP path, 64..256 on the CTA path
     int cluster; // CTAs per row for CLUSTER/TWO_PASS paths (1 otherwise)
+    int rps;     // WARP path: rows per shared-memory slot for this segment
 };
 
-// Launch shape: every WARP/CTA-path segment of a call shares one group-kernel
-// launch (each segment carries its own threads-per-row); CLUSTER and TWO_PASS
-// segments share a launch per cluster size.
+// Launch shape: all WARP-path segments of a call share one launch of the
+// warp-per-row kernel; all CTA-path segments one launch of the register
+// group kernel (each segment carries its own threads-per-row); CLUSTER and
+// TWO_PASS segments a launch per cluster size.
 inline bool same_launch(const RowClass &a, const RowClass &b)
 {
-    const bool ga = a.path == DS_PATH_WARP || a.path == DS_PATH_CTA;
-    const bool gb = b.path == DS_PATH_WARP || b.path == DS_PATH_CTA;
-    if (ga || gb)
-        return ga && gb;
-    return a.path == b.path && a.cluster == b.cluster;
+    if (a.path == DS_PATH_CLUSTER || a.path == DS_PATH_TWO_PASS)
+        return a.path == b.path && a.cluster == b.cluster;
+    return a.path == b.path;
 }
 
 // Device copy of one weight segment.
@@ -101,6 +105,7 @@ enum DeviceErrorSite : uint32_t {
     kSiteStreamWait = 1,
     kSiteStreamDrain = 2,
     kSiteSelftest = 3,
+    kSiteTileWait = 4,
 };
 
 // Launchers (ds_kernels.cu).  `units` = grid size in rows-groups (WARP/CTA)
@@ -111,6 +116,11 @@ int launch_row_renorm(const RowClass &rc, const WParams &p, int64_t units, void 
 int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_wait_selftest(uint64_t limit_ns, void *stream);
+// Warp-per-row path (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,
+// 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp; params is a
+// WParams (tags 0-4) or AParams (5-6) whose segments carry rows per slot in
+// `group` and whose unit_start counts slots.
+int launch_tile(int tag, const void *params, int grid, int slot_bytes, int nslots, void *stream);
 int read_and_clear_device_error(uint32_t *code, uint32_t *site, void *stream);
 
 } // namespace ds

@@ -1,0 +1,685 @@
+// ds_tile.cu -- the warp-per-row path: a persistent, bulk-copy (TMA) fed
+// kernel for every row that fits a shared-memory slot (<= 16 KB of input).
+//
+// One CTA per SM.  The last warp is the producer: it walks the CTA's slots
+// (slot = a run of consecutive rows of one segment, at most kTileSlotBytes of
+// input) in order, waits until the slot's ring position is free, and fills
+// it with one cp.async.bulk per array (or per row when rows are padded)
+// completing on that position's "full" mbarrier.  Each of the other warps
+// owns one ring position: slot j of the CTA goes to position and warp
+// j % kMaxTileSlots, which waits on "full", normalises its rows out of shared
+// memory, stores the results straight to global memory, and arrives on
+// "empty".  Because a position is consumed by one warp, in order, no barrier
+// is ever waited on more than one phase ahead of its current phase.  Every
+// wait is bounded.
+//
+// Per row a warp sums in a fixed order -- each lane its units u = lane,
+// lane + 32, ... in order, two packed fp32 accumulators (even and odd
+// elements) added at the end, then an xor butterfly over the lanes -- so a
+// row's bits depend on its length and the operation only.
+#include <cuda_runtime.h>
+
+#include "ds_device.cuh"
+
+namespace ds {
+
+// ds_kernels.cu's tags, repeated (the two files share this numbering).
+enum TileTag { tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp };
+
+namespace {
+
+constexpr int kConsumerWarps = kMaxTileSlots;
+constexpr int kTileThreads = (kConsumerWarps + 1) * 32;
+
+struct SlotHdr {
+    int32_t seg;
+    int32_t nrows;
+    int64_t row0;
+};
+
+// ------------------------------------------------------------- helpers --
+
+__device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
+__device__ __forceinline__ float2 lo2(uint32_t w) { return f2(bf_lo(w), bf_hi(w)); }
+
+__device__ __forceinline__ uint32_t pk(float2 v) { return pack_bf2(v.x, v.y); }
+
+__device__ __forceinline__ float warp_sum1(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max1(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ void sq2(float2 &acc, float2 v) { acc = __ffma2_rn(v, v, acc); }
+
+template <class F>
+__device__ __forceinline__ void each4_(float4 v, F &&f)
+{
+    f(v.x);
+    f(v.y);
+    f(v.z);
+    f(v.w);
+}
+
+__device__ __forceinline__ float2 fneg2(float2 v) { return f2(-v.x, -v.y); }
+
+// Factor of a row from its warp-summed S (see RowScale).  The rescale path
+// re-sums with exactly the fast path's structure -- the same pairs, in the
+// same order, into two packed accumulators -- so that a row scaled by 2^k
+// gives the same bits whichever path it takes.  `gen(f)` calls f(pair) on
+// every pair the lane summed, in order.
+template <class Gen>
+__device__ __forceinline__ RowScale tile_scale(float S, float eps, Gen &&gen)
+{
+    if (!needs_rescale(S, eps))
+        return {1.0f / sqrtf(S + eps), 1.f};
+    float M = 0.f;
+    gen([&](float2 v) { M = fmaxf(M, fmaxf(fabsf(v.x), fabsf(v.y))); });
+    M = warp_max1(M);
+    if (!(M > 0.f && M < __int_as_float(0x7f800000)))
+        return {1.0f / sqrtf(S + eps), 1.f};
+    const int m = 48 - ilogbf(M);
+    float2 acc = f2(0.f, 0.f);
+    gen([&](float2 v) {
+        const float2 u = f2(scalbnf(v.x, m), scalbnf(v.y, m));
+        acc = __ffma2_rn(u, u, acc);
+    });
+    const float Ss = warp_sum1(acc.x + acc.y);
+    const float inv = 1.0f / sqrtf(Ss + scalbnf(eps, 2 * m));
+    if (m > 100)
+        return {scalbnf(inv, 100), scalbnf(1.f, m - 100)};
+    return {scalbnf(inv, m), 1.f};
+}
+
+// |alpha| for the 8 elements of unit u, as four pairs (0 past cols).
+__device__ __forceinline__ void alpha_pairs(const float *alpha, int u, int cols, float2 (&m)[4])
+{
+    const int e0 = 8 * u;
+    const float4 a = e0 < cols ? __ldg(reinterpret_cast<const float4 *>(alpha + e0)) : make_float4(0, 0, 0, 0);
+    const float4 b = e0 + 4 < cols ? __ldg(reinterpret_cast<const float4 *>(alpha + e0 + 4)) : make_float4(0, 0, 0, 0);
+    m[0] = f2(fabsf(a.x), fabsf(a.y));
+    m[1] = f2(fabsf(a.z), fabsf(a.w));
+    m[2] = f2(fabsf(b.x), fabsf(b.y));
+    m[3] = f2(fabsf(b.z), fabsf(b.w));
+}
+
+// ------------------------------------------------------- layout per op ---
+//
+// Arrays staged per row and their bytes per 16-byte unit of the row.
+
+template <int T>
+struct TileLayout {
+    static constexpr int kArrays = (T == tFwdBf16 || T == tFwdF32 || T == tRenorm) ? 1 : 2;
+    // bytes per unit of array a
+    static __device__ __forceinline__ int ub(int a, bool has_r)
+    {
+        if (a == 0)
+            return 16;
+        if (T == tBwdBf16)
+            return 8;
+        if (T == tL2)
+            return has_r ? 16 : 0;
+        return 16;
+    }
+};
+
+// Source row pointers of array a.
+template <int T>
+__device__ __forceinline__ const char *tile_src(const WSegK &sg, int a, int64_t row)
+{
+    if (a == 0)
+        return reinterpret_cast<const char *>(sg.w + row * sg.ld);
+    return static_cast<const char *>(sg.gy) + row * sg.ld_out * (T == tBwdBf16 ? 2 : 4);
+}
+
+template <int T>
+__device__ __forceinline__ const char *tile_src(const ASegK &sg, int a, int64_t row)
+{
+    return reinterpret_cast<const char *>((a == 0 ? sg.x : sg.r) + row * sg.ld);
+}
+
+__device__ __forceinline__ bool seg_has_r(const WSegK &) { return true; }
+__device__ __forceinline__ bool seg_has_r(const ASegK &s) { return s.r != nullptr; }
+
+// Row pitch in global memory (bytes) of array a.
+template <int T>
+__device__ __forceinline__ int64_t tile_src_pitch(const WSegK &sg, int a)
+{
+    return a == 0 ? sg.ld * 4 : sg.ld_out * (T == tBwdBf16 ? 2 : 4);
+}
+
+template <int T>
+__device__ __forceinline__ int64_t tile_src_pitch(const ASegK &sg, int)
+{
+    return sg.ld * 2;
+}
+
+// ============================================================ row bodies ==
+//
+// `s0`, `s1`: this row's units of array 0 and 1 in shared memory (unit
+// stride 16 or 8 bytes).  nfull = units with every element valid; `tail` =
+// valid elements of unit nfull (0 if none), handled by lane nfull % 32 after
+// its full units, so every lane's units are summed in increasing order.
+
+template <bool OUT_BF16, bool RENORM>
+__device__ __forceinline__ void tile_scale_row(const WSegK &sg, int64_t row, float g, const unsigned char *s0,
+                                               int lane, int nfull, int tail, float eps, bool store)
+{
+    const float4 *w = reinterpret_cast<const float4 *>(s0);
+    float2 acc = f2(0.f, 0.f);
+#pragma unroll 4
+    for (int u = lane; u < nfull; u += 32) {
+        const float4 v = w[u];
+        sq2(acc, f2(v.x, v.y));
+        sq2(acc, f2(v.z, v.w));
+    }
+    const bool tl = tail && lane == (nfull & 31);
+    float4 vt = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tl) {
+        vt = mask_quad(w[nfull], tail);
+        sq2(acc, f2(vt.x, vt.y));
+        sq2(acc, f2(vt.z, vt.w));
+    }
+    const float S = warp_sum1(acc.x + acc.y);
+    const RowScale rs = tile_scale(S, eps, [&](auto f) {
+        for (int u = lane; u < nfull; u += 32) {
+            const float4 v = w[u];
+            f(f2(v.x, v.y));
+            f(f2(v.z, v.w));
+        }
+        if (tl) {
+            f(f2(vt.x, vt.y));
+            f(f2(vt.z, vt.w));
+        }
+    });
+    if (!store)
+        return;
+    const float sc = (g * sg.radius) * rs.inv;
+    const float2 sc2 = f2(sc, sc), pre2 = f2(rs.pre, rs.pre);
+    char *out = RENORM ? reinterpret_cast<char *>(const_cast<float *>(sg.w) + row * sg.ld)
+                       : static_cast<char *>(sg.out) + row * sg.ld_out * (OUT_BF16 ? 2 : 4);
+    const bool plain = rs.pre == 1.f;
+#pragma unroll 4
+    for (int u = lane; u < nfull; u += 32) {
+        const float4 v = w[u];
+        float2 a = f2(v.x, v.y), b = f2(v.z, v.w);
+        if (!plain) {
+            a = __fmul2_rn(a, pre2);
+            b = __fmul2_rn(b, pre2);
+        }
+        a = __fmul2_rn(a, sc2);
+        b = __fmul2_rn(b, sc2);
+        if constexpr (OUT_BF16)
+            st8(out + 8 * u, make_uint2(pk(a), pk(b)));
+        else
+            st16(out + 16 * u, make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
+                                          __float_as_uint(b.y)));
+    }
+    if (tl) {
+        const float4 y = make_float4((vt.x * rs.pre) * sc, (vt.y * rs.pre) * sc, (vt.z * rs.pre) * sc,
+                                     (vt.w * rs.pre) * sc);
+        if constexpr (OUT_BF16) {
+            uint16_t *o = reinterpret_cast<uint16_t *>(out) + 4 * nfull;
+            const float e[4] = {y.x, y.y, y.z, y.w};
+            for (int i = 0; i < tail; ++i) {
+                __nv_bfloat16 h = __float2bfloat16_rn(e[i]);
+                o[i] = *reinterpret_cast<uint16_t *>(&h);
+            }
+        } else {
+            float *o = reinterpret_cast<float *>(out) + 4 * nfull;
+            o[0] = y.x;
+            if (tail > 1) o[1] = y.y;
+            if (tail > 2) o[2] = y.z;
+        }
+    }
+}
+
+template <bool GY_BF16>
+__device__ __forceinline__ float4 gy_unit(const unsigned char *s1, int u)
+{
+    if constexpr (GY_BF16) {
+        const uint2 r = *reinterpret_cast<const uint2 *>(s1 + 8 * u);
+        return make_float4(bf_lo(r.x), bf_hi(r.x), bf_lo(r.y), bf_hi(r.y));
+    } else {
+        return *reinterpret_cast<const float4 *>(s1 + 16 * u);
+    }
+}
+
+template <bool GY_BF16>
+__device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, float g, const unsigned char *s0,
+                                                  const unsigned char *s1, int lane, int nfull, int tail,
+                                                  float eps, bool store)
+{
+    const float4 *w = reinterpret_cast<const float4 *>(s0);
+    float2 as = f2(0.f, 0.f), ad = f2(0.f, 0.f);
+#pragma unroll 4
+    for (int u = lane; u < nfull; u += 32) {
+        const float4 x = w[u];
+        const float4 d = gy_unit<GY_BF16>(s1, u);
+        sq2(as, f2(x.x, x.y));
+        sq2(as, f2(x.z, x.w));
+        ad = __ffma2_rn(f2(x.x, x.y), f2(d.x, d.y), ad);
+        ad = __ffma2_rn(f2(x.z, x.w), f2(d.z, d.w), ad);
+    }
+    const bool tl = tail && lane == (nfull & 31);
+    float4 xt = make_float4(0.f, 0.f, 0.f, 0.f), dt = xt;
+    if (tl) {
+        xt = mask_quad(w[nfull], tail);
+        dt = mask_quad(gy_unit<GY_BF16>(s1, nfull), tail);
+        sq2(as, f2(xt.x, xt.y));
+        sq2(as, f2(xt.z, xt.w));
+        ad = __ffma2_rn(f2(xt.x, xt.y), f2(dt.x, dt.y), ad);
+        ad = __ffma2_rn(f2(xt.z, xt.w), f2(dt.z, dt.w), ad);
+    }
+    float S = warp_sum1(as.x + as.y);
+    float D = warp_sum1(ad.x + ad.y);
+    // Rows needing the rescale: w scaled by 2^m (exact), S and D re-summed,
+    // 2^m carried into the row constants (as the register paths do).
+    int m = 0;
+    if (needs_rescale(S, eps)) {
+        float M = 0.f;
+        for (int u = lane; u < nfull; u += 32)
+            each4_(w[u], [&](float v) { M = fmaxf(M, fabsf(v)); });
+        if (tl)
+            each4_(xt, [&](float v) { M = fmaxf(M, fabsf(v)); });
+        M = warp_max1(M);
+        if (M > 0.f && M < __int_as_float(0x7f800000)) {
+            m = 48 - ilogbf(M);
+            float2 bs = f2(0.f, 0.f), bd = f2(0.f, 0.f);
+            auto add = [&](float4 x, float4 d) {
+                const float2 p = f2(scalbnf(x.x, m), scalbnf(x.y, m)), q = f2(scalbnf(x.z, m), scalbnf(x.w, m));
+                sq2(bs, p);
+                sq2(bs, q);
+                bd = __ffma2_rn(p, f2(d.x, d.y), bd);
+                bd = __ffma2_rn(q, f2(d.z, d.w), bd);
+            };
+            for (int u = lane; u < nfull; u += 32)
+                add(w[u], gy_unit<GY_BF16>(s1, u));
+            if (tl)
+                add(xt, dt);
+            S = warp_sum1(bs.x + bs.y);
+            D = warp_sum1(bd.x + bd.y);
+        }
+    }
+    if (!store)
+        return;
+    const float n2 = S + (m == 0 ? eps : scalbnf(eps, 2 * m));
+    const float inv = 1.0f / sqrtf(n2);
+    const float q = m == 0 ? D / n2 : scalbnf(D / n2, m);
+    const float pre = (g * sg.radius) * (m == 0 ? inv : scalbnf(inv, m));
+    if (lane == 0 && sg.gain)
+        sg.grad_g[row] = sg.radius * D * inv;
+    const float2 nq = f2(-q, -q), pre2 = f2(pre, pre);
+    char *out = reinterpret_cast<char *>(sg.grad_w + row * sg.ld);
+#pragma unroll 4
+    for (int u = lane; u < nfull; u += 32) {
+        const float4 x = w[u];
+        const float4 d = gy_unit<GY_BF16>(s1, u);
+        const float2 a = __fmul2_rn(__ffma2_rn(f2(x.x, x.y), nq, f2(d.x, d.y)), pre2);
+        const float2 b = __fmul2_rn(__ffma2_rn(f2(x.z, x.w), nq, f2(d.z, d.w)), pre2);
+        st16(out + 16 * u,
+             make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x), __float_as_uint(b.y)));
+    }
+    if (tl) {
+        float *o = reinterpret_cast<float *>(out) + 4 * nfull;
+        o[0] = pre * fmaf(xt.x, -q, dt.x);
+        if (tail > 1) o[1] = pre * fmaf(xt.y, -q, dt.y);
+        if (tail > 2) o[2] = pre * fmaf(xt.z, -q, dt.z);
+    }
+}
+
+// Octet helpers: 8 bf16 as four packed pairs.
+__device__ __forceinline__ void sq8(float2 &acc, uint4 v)
+{
+    sq2(acc, lo2(v.x));
+    sq2(acc, lo2(v.y));
+    sq2(acc, lo2(v.z));
+    sq2(acc, lo2(v.w));
+}
+
+template <class F>
+__device__ __forceinline__ void pairs8(uint4 v, F &&f)
+{
+    f(lo2(v.x));
+    f(lo2(v.y));
+    f(lo2(v.z));
+    f(lo2(v.w));
+}
+
+__device__ __forceinline__ uint4 scale8(uint4 v, RowScale r)
+{
+    const float2 s = f2(r.inv, r.inv);
+    if (r.pre == 1.f)
+        return make_uint4(pk(__fmul2_rn(lo2(v.x), s)), pk(__fmul2_rn(lo2(v.y), s)), pk(__fmul2_rn(lo2(v.z), s)),
+                          pk(__fmul2_rn(lo2(v.w), s)));
+    const float2 p = f2(r.pre, r.pre);
+    return make_uint4(pk(__fmul2_rn(__fmul2_rn(lo2(v.x), p), s)), pk(__fmul2_rn(__fmul2_rn(lo2(v.y), p), s)),
+                      pk(__fmul2_rn(__fmul2_rn(lo2(v.z), p), s)), pk(__fmul2_rn(__fmul2_rn(lo2(v.w), p), s)));
+}
+
+__device__ __forceinline__ uint32_t add_bf2(uint32_t a, uint32_t b)
+{
+    return pk(__fadd2_rn(lo2(a), lo2(b)));
+}
+
+__device__ __forceinline__ void store_tail8(uint16_t *o, uint4 v, int valid)
+{
+    for (int e = 0; e < valid; ++e) {
+        const uint32_t w = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
+        o[e] = static_cast<uint16_t>((e & 1) ? (w >> 16) : (w & 0xFFFFu));
+    }
+}
+
+// l2 rows.  With a residual, pass 1 writes s = bf16(x + r) back over x in the
+// slot, so pass 2 reads s directly.
+__device__ __forceinline__ void tile_l2_row(const ASegK &sg, int64_t row, unsigned char *s0, const unsigned char *s1,
+                                            int lane, int nfull, int tail, float eps, bool store)
+{
+    uint4 *x = reinterpret_cast<uint4 *>(s0);
+    const uint4 *r = reinterpret_cast<const uint4 *>(s1);
+    const bool has_r = sg.r != nullptr;
+    float2 acc = f2(0.f, 0.f);
+    const int nunits = nfull + (tail ? 1 : 0);
+#pragma unroll 4
+    for (int u = lane; u < nunits; u += 32) {
+        uint4 s = x[u];
+        if (has_r) {
+            const uint4 b = r[u];
+            s = make_uint4(add_bf2(s.x, b.x), add_bf2(s.y, b.y), add_bf2(s.z, b.z), add_bf2(s.w, b.w));
+        }
+        if (u == nfull)
+            s = mask_octet(s, tail);
+        if (has_r || u == nfull)
+            x[u] = s;
+        sq8(acc, s);
+    }
+    const float S = warp_sum1(acc.x + acc.y);
+    __syncwarp();
+    const RowScale rs = tile_scale(S, eps, [&](auto f) {
+        for (int u = lane; u < nunits; u += 32)
+            pairs8(x[u], f);
+    });
+    if (!store)
+        return;
+    uint16_t *y = sg.y + row * sg.ld;
+#pragma unroll 4
+    for (int u = lane; u < nfull; u += 32)
+        st16(y + 8 * u, scale8(x[u], rs));
+    if (tail && lane == (nfull & 31))
+        store_tail8(y + 8 * nfull, scale8(x[nfull], rs), tail);
+}
+
+// slerp rows: pass 1 sums res^2 and out^2; pass 2 writes a = bf16(l2(res)) and
+// b = bf16(l2(out)) back into the slot and sums t^2; pass 3 writes h.
+__device__ __forceinline__ float2 lerp2(float2 a, float2 b, float2 m)
+{
+    return __ffma2_rn(m, __fadd2_rn(b, fneg2(a)), a);
+}
+
+__device__ __forceinline__ void tile_slerp_row(const ASegK &sg, int64_t row, unsigned char *s0, unsigned char *s1,
+                                               int lane, int nfull, int tail, float eps, bool store)
+{
+    uint4 *xa = reinterpret_cast<uint4 *>(s0);
+    uint4 *xb = reinterpret_cast<uint4 *>(s1);
+    const int nunits = nfull + (tail ? 1 : 0);
+    float2 aa = f2(0.f, 0.f), ab = f2(0.f, 0.f);
+#pragma unroll 4
+    for (int u = lane; u < nunits; u += 32) {
+        uint4 p = xa[u], q = xb[u];
+        if (u == nfull) {
+            p = mask_octet(p, tail);
+            q = mask_octet(q, tail);
+            xa[u] = p;
+            xb[u] = q;
+        }
+        sq8(aa, p);
+        sq8(ab, q);
+    }
+    const float Sa = warp_sum1(aa.x + aa.y);
+    const float Sb = warp_sum1(ab.x + ab.y);
+    __syncwarp();
+    const RowScale ra = tile_scale(Sa, eps, [&](auto f) {
+        for (int u = lane; u < nunits; u += 32)
+            pairs8(xa[u], f);
+    });
+    const RowScale rb = tile_scale(Sb, eps, [&](auto f) {
+        for (int u = lane; u < nunits; u += 32)
+            pairs8(xb[u], f);
+    });
+    float2 at = f2(0.f, 0.f);
+#pragma unroll 2
+    for (int u = lane; u < nunits; u += 32) {
+        const uint4 a = scale8(xa[u], ra), b = scale8(xb[u], rb);
+        xa[u] = a;
+        xb[u] = b;
+        float2 m[4];
+        alpha_pairs(sg.alpha, u, sg.cols, m);
+        sq2(at, lerp2(lo2(a.x), lo2(b.x), m[0]));
+        sq2(at, lerp2(lo2(a.y), lo2(b.y), m[1]));
+        sq2(at, lerp2(lo2(a.z), lo2(b.z), m[2]));
+        sq2(at, lerp2(lo2(a.w), lo2(b.w), m[3]));
+    }
+    const float St = warp_sum1(at.x + at.y);
+    __syncwarp();
+    auto each_t = [&](auto f) {
+        for (int u = lane; u < nunits; u += 32) {
+            const uint4 a = xa[u], b = xb[u];
+            float2 m[4];
+            alpha_pairs(sg.alpha, u, sg.cols, m);
+            f(lerp2(lo2(a.x), lo2(b.x), m[0]));
+            f(lerp2(lo2(a.y), lo2(b.y), m[1]));
+            f(lerp2(lo2(a.z), lo2(b.z), m[2]));
+            f(lerp2(lo2(a.w), lo2(b.w), m[3]));
+        }
+    };
+    const RowScale rt = tile_scale(St, eps, each_t);
+    if (!store)
+        return;
+    uint16_t *y = sg.y + row * sg.ld;
+    const float2 s = f2(rt.inv, rt.inv), p = f2(rt.pre, rt.pre);
+#pragma unroll 2
+    for (int u = lane; u < nunits; u += 32) {
+        const uint4 a = xa[u], b = xb[u];
+        float2 m[4];
+        alpha_pairs(sg.alpha, u, sg.cols, m);
+        float2 t0 = lerp2(lo2(a.x), lo2(b.x), m[0]), t1 = lerp2(lo2(a.y), lo2(b.y), m[1]);
+        float2 t2 = lerp2(lo2(a.z), lo2(b.z), m[2]), t3 = lerp2(lo2(a.w), lo2(b.w), m[3]);
+        if (rt.pre != 1.f) {
+            t0 = __fmul2_rn(t0, p);
+            t1 = __fmul2_rn(t1, p);
+            t2 = __fmul2_rn(t2, p);
+            t3 = __fmul2_rn(t3, p);
+        }
+        const uint4 h = make_uint4(pk(__fmul2_rn(t0, s)), pk(__fmul2_rn(t1, s)), pk(__fmul2_rn(t2, s)),
+                                   pk(__fmul2_rn(t3, s)));
+        if (u < nfull)
+            st16(y + 8 * u, h);
+        else
+            store_tail8(y + 8 * nfull, h, tail);
+    }
+}
+
+// =============================================================== kernel ==
+
+template <int T>
+using TParams = typename std::conditional<(T <= tRenorm), WParams, AParams>::type;
+
+template <int T>
+__global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant__ TParams<T> p, int slot_bytes)
+{
+    constexpr int nslots = kMaxTileSlots; // one ring position per consumer warp
+    extern __shared__ __align__(128) unsigned char ring[];
+    __shared__ __align__(8) uint64_t full[kMaxTileSlots];
+    __shared__ __align__(8) uint64_t empty[kMaxTileSlots];
+    __shared__ SlotHdr hdr[kMaxTileSlots];
+    __shared__ volatile int abort_flag; // set by the first wait that runs out
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t total = p.unit_start[p.nseg];
+    // this CTA's slots: blockIdx.x, blockIdx.x + gridDim.x, ...
+    const int64_t mine = total > blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < nslots; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        abort_flag = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    using Layout = TileLayout<T>;
+    bool ok = true;
+
+    if (warp == kConsumerWarps) {
+        // ------------------------------------------------------ producer --
+        if (lane == 0) {
+            for (int64_t j = 0; j < mine; ++j) {
+                const int s = static_cast<int>(j % nslots);
+                if (j >= nslots && (abort_flag ||
+                    !mbar_wait_bounded(&empty[s], static_cast<uint32_t>((j / nslots - 1) & 1), p.wait_limit_ns))) {
+                    ok = false;
+                    abort_flag = 1;
+                    break;
+                }
+                const int64_t slot = blockIdx.x + j * gridDim.x;
+                const int si = find_segment(p, slot);
+                const auto &sg = p.seg[si];
+                const int rps = sg.group; // rows per slot for this segment
+                const int64_t row0 = (slot - p.unit_start[si]) * rps;
+                const int nrows = static_cast<int>(sg.rows - row0 < rps ? sg.rows - row0 : rps);
+                hdr[s] = SlotHdr{si, nrows, row0};
+                const bool has_r = seg_has_r(sg);
+                unsigned char *dst = ring + static_cast<size_t>(s) * slot_bytes;
+                uint32_t bytes = 0, pitch[2], off[2];
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    const int u = a < Layout::kArrays ? Layout::ub(a, has_r) : 0;
+                    pitch[a] = (static_cast<uint32_t>(sg.nu) * u + 15u) & ~15u;
+                    off[a] = a == 0 ? 0u : pitch[0] * rps;
+                    bytes += pitch[a] * nrows;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&full[s], bytes);
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    if (!pitch[a])
+                        continue;
+                    const char *src = tile_src<T>(sg, a, row0);
+                    const int64_t src_pitch = tile_src_pitch<T>(sg, a);
+                    if (src_pitch == static_cast<int64_t>(pitch[a])) {
+                        bulk_g2s(dst + off[a], src, pitch[a] * nrows, &full[s]);
+                    } else {
+                        for (int r = 0; r < nrows; ++r)
+                            bulk_g2s(dst + off[a] + r * pitch[a], src + r * src_pitch, pitch[a], &full[s]);
+                    }
+                }
+            }
+        }
+    } else {
+        // ------------------------------------------------------ consumers --
+        // position `warp`; its i-th use holds slot warp + i * nslots
+        const int s = warp;
+        uint32_t phase = 0;
+        for (int64_t j = warp; j < mine; j += nslots, phase ^= 1u) {
+            bool got = !abort_flag && mbar_wait_bounded(&full[s], phase, p.wait_limit_ns);
+            got = __all_sync(0xffffffffu, got);
+            if (!got) {
+                ok = false;
+                abort_flag = 1;
+                break; // nothing more arrives; the stores of this warp stop here
+            }
+            const SlotHdr h = hdr[s];
+            const auto &sg = p.seg[h.seg];
+            const bool has_r = seg_has_r(sg);
+            const int rps = sg.group;
+            unsigned char *base = ring + static_cast<size_t>(s) * slot_bytes;
+            const int u0 = Layout::ub(0, has_r), u1 = Layout::kArrays > 1 ? Layout::ub(1, has_r) : 0;
+            const int pitch0 = (sg.nu * u0 + 15) & ~15;
+            const int pitch1 = (sg.nu * u1 + 15) & ~15;
+            unsigned char *a1 = base + pitch0 * rps;
+            constexpr int E = (T <= tRenorm) ? 4 : 8;
+            const int nfull = sg.cols / E, tail = sg.cols % E;
+            float g_lane = 1.f;
+            for (int r = 0; r < h.nrows; ++r) {
+                const int64_t row = h.row0 + r;
+                unsigned char *s0 = base + r * pitch0;
+                unsigned char *s1 = a1 + r * pitch1;
+                if constexpr (T == tFwdBf16 || T == tFwdF32 || T == tBwdBf16 || T == tBwdF32) {
+                    // gains of the next 32 rows, one per lane
+                    if ((r & 31) == 0)
+                        g_lane = (sg.gain && r + lane < h.nrows) ? __ldg(sg.gain + row + lane) : 1.f;
+                }
+                const float g = __shfl_sync(0xffffffffu, g_lane, r & 31);
+                if constexpr (T == tFwdBf16)
+                    tile_scale_row<true, false>(sg, row, g, s0, lane, nfull, tail, p.eps, got);
+                else if constexpr (T == tFwdF32)
+                    tile_scale_row<false, false>(sg, row, g, s0, lane, nfull, tail, p.eps, got);
+                else if constexpr (T == tRenorm)
+                    tile_scale_row<false, true>(sg, row, 1.f, s0, lane, nfull, tail, p.eps, got);
+                else if constexpr (T == tBwdBf16)
+                    tile_backward_row<true>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, got);
+                else if constexpr (T == tBwdF32)
+                    tile_backward_row<false>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, got);
+                else if constexpr (T == tL2)
+                    tile_l2_row(sg, row, s0, s1, lane, nfull, tail, p.eps, got);
+                else
+                    tile_slerp_row(sg, row, s0, s1, lane, nfull, tail, p.eps, got);
+            }
+            // the slot may hold this warp's generic-proxy writes (s, a, b):
+            // order them before the next bulk copy into it, then release it
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[s]);
+        }
+    }
+    if (!ok)
+        raise_device_error(DS_ERR_DEVICE_TIMEOUT, kSiteTileWait);
+}
+
+} // namespace
+
+template <int T>
+static cudaError_t launch_tile_t(const TParams<T> &p, int grid, int slot_bytes, int nslots, void *stream)
+{
+    if (nslots != kMaxTileSlots)
+        return cudaErrorInvalidValue;
+    const int smem = slot_bytes * nslots;
+    static int attr_smem = 0; // benign race: idempotent
+    if (attr_smem < smem) {
+        cudaError_t e = cudaFuncSetAttribute(k_tile<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess)
+            return e;
+        attr_smem = smem;
+    }
+    k_tile<T><<<grid, kTileThreads, smem, static_cast<cudaStream_t>(stream)>>>(p, slot_bytes);
+    return cudaGetLastError();
+}
+
+int launch_tile(int tag, const void *params, int grid, int slot_bytes, int nslots, void *stream)
+{
+    switch (tag) {
+    case tFwdBf16: return launch_tile_t<tFwdBf16>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
+    case tFwdF32: return launch_tile_t<tFwdF32>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
+    case tBwdBf16: return launch_tile_t<tBwdBf16>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
+    case tBwdF32: return launch_tile_t<tBwdF32>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
+    case tRenorm: return launch_tile_t<tRenorm>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
+    case tL2: return launch_tile_t<tL2>(*static_cast<const AParams *>(params), grid, slot_bytes, nslots, stream);
+    case tSlerp: return launch_tile_t<tSlerp>(*static_cast<const AParams *>(params), grid, slot_bytes, nslots, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+} // namespace ds

@@ -41,12 +41,13 @@ A_OPS = (ds.DS_OP_L2_ROWS, ds.DS_OP_SLERP_ROWS)
 
 
 @pytest.mark.parametrize("op,cols,want", [
-    (ds.DS_OP_WN_FORWARD, 768, (ds.DS_PATH_WARP, 32, 1)),     # 192 quads, 6 per lane
-    (ds.DS_OP_WN_FORWARD, 2048, (ds.DS_PATH_CTA, 64, 1)),
-    (ds.DS_OP_WN_BACKWARD, 768, (ds.DS_PATH_CTA, 64, 1)),     # two inputs: 4 units per thread
-    (ds.DS_OP_WN_BACKWARD, 2048, (ds.DS_PATH_CTA, 128, 1)),
+    (ds.DS_OP_WN_FORWARD, 768, (ds.DS_PATH_WARP, 32, 1)),     # staged rows <= 16 KB: warp per row
+    (ds.DS_OP_WN_FORWARD, 2048, (ds.DS_PATH_WARP, 32, 1)),
+    (ds.DS_OP_WN_BACKWARD, 768, (ds.DS_PATH_WARP, 32, 1)),
+    (ds.DS_OP_WN_BACKWARD, 2048, (ds.DS_PATH_WARP, 32, 1)),   # w + fp32 GY = 16 KB
+    (ds.DS_OP_WN_BACKWARD, 2049, (ds.DS_PATH_CTA, 256, 1)),  # 513 quads, 4 per thread at most
     (ds.DS_OP_ROW_RENORM, 128, (ds.DS_PATH_WARP, 32, 1)),
-    (ds.DS_OP_L2_ROWS, 4096, (ds.DS_PATH_CTA, 128, 1)),
+    (ds.DS_OP_L2_ROWS, 4096, (ds.DS_PATH_WARP, 32, 1)),       # x + r = 16 KB
     (ds.DS_OP_SLERP_ROWS, 7168, (ds.DS_PATH_CTA, 256, 1)),
     (ds.DS_OP_L2_ROWS, 16384, (ds.DS_PATH_CLUSTER, 0, 2)),
     (ds.DS_OP_WN_FORWARD, 14336, (ds.DS_PATH_CLUSTER, 0, 2)),
@@ -67,8 +68,13 @@ def test_row_class_is_monotone_and_fits():
         for cols in sorted(set(list(range(1, 600, 7)) + [2 ** k + d for k in range(9, 19) for d in (-1, 0, 1)])):
             path, g, cl = ds.ds_row_class(op, cols)
             nu = -(-cols // e)
-            if path in (ds.DS_PATH_WARP, ds.DS_PATH_CTA):
-                assert -(-nu // g) <= kmax and g in (32, 64, 128, 256)
+            staged = {ds.DS_OP_WN_FORWARD: 16, ds.DS_OP_ROW_RENORM: 16, ds.DS_OP_WN_BACKWARD: 32}.get(op, 32) * nu
+            if path == ds.DS_PATH_WARP:
+                assert staged <= 16384 and g == 32
+            else:
+                assert staged > 16384
+            if path == ds.DS_PATH_CTA:
+                assert -(-nu // g) <= kmax and g in (64, 128, 256)
             elif path == ds.DS_PATH_CLUSTER:
                 assert -(-nu // cl) <= 256 * kmax and cl in (2, 4, 8)
             key = (order[path], g, cl)
@@ -82,7 +88,7 @@ def test_forced_paths():
     with ds.force_path(ds.DS_PATH_CLUSTER):
         assert ds.ds_row_class(ds.DS_OP_WN_FORWARD, 768) == (ds.DS_PATH_CLUSTER, 0, 2)
     with ds.force_path(ds.DS_PATH_WARP):  # does not fit: automatic choice
-        assert ds.ds_row_class(ds.DS_OP_L2_ROWS, 4096)[0] == ds.DS_PATH_CTA
+        assert ds.ds_row_class(ds.DS_OP_L2_ROWS, 8192)[0] == ds.DS_PATH_CTA
     with ds.force_path(ds.DS_PATH_CTA):
         assert ds.ds_row_class(ds.DS_OP_WN_FORWARD, 128) == (ds.DS_PATH_CTA, 64, 1)
     assert ds.ds_row_class(ds.DS_OP_L2_ROWS, 128)[0] == ds.DS_PATH_WARP

@@ -7,7 +7,9 @@ controls, and the bounded-wait error path.
   free scale direction of DragonScale's "Why scales drift"), also through the
   overflow/underflow rescaling path.
 * l2 with an all-zero residual equals l2 without one; slerp with alpha = 0
-  (|alpha| = 1) equals l2 of bf16(l2(res)) (of bf16(l2(out))).
+  equals l2 of bf16(l2(res)) (the lerp's multiply-add adds an exact zero);
+  at |alpha| = 1 the GPU's b - a may round in fp32, so that end is checked
+  against the oracle (where t = b exactly).
 * Controls: oracle variants that drop one rounding point must fail the check.
 """
 from __future__ import annotations
@@ -117,10 +119,10 @@ def test_slerp_endpoints(path):
         sign = torch.where(torch.arange(C, device="cuda") % 2 == 0, 1.0, -1.0)
         h1 = slerp(sign)
         ref0 = l2(l2(x))
-        ref1 = l2(l2(o))
         torch.cuda.synchronize()
     assert torch.equal(bits(h0), bits(ref0))
-    assert torch.equal(bits(h1), bits(ref1))
+    ends = wl.ActRows("a", a.x, a.r, sign.cpu().numpy().astype(np.float32))
+    gu.check_slerp(ends, h1, 1e-6, what="slerp |alpha| = 1")
 
 
 @pytest.mark.parametrize("path", PATHS, ids=PATH_IDS)
