@@ -234,6 +234,22 @@ ds_status check_matrix(const void *p, int64_t rows, int64_t ld, int esize, const
 
 // Splits, packs and launches.  `make(i, r0, nrows)` returns the device
 // segment for rows [r0, r0 + nrows) of segment i.
+// Slerp launches whose segments all use one alpha vector of at most
+// kTileAlphaCache columns let the staged kernel keep |alpha| in shared memory.
+inline void shared_alpha(WParams &p, int) { p.alpha_shared = nullptr; p.alpha_cols = 0; }
+inline void shared_alpha(AParams &p, int n)
+{
+    p.alpha_shared = nullptr;
+    p.alpha_cols = 0;
+    if (n == 0 || !p.seg[0].alpha || p.seg[0].cols > ds::kTileAlphaCache)
+        return;
+    for (int i = 1; i < n; ++i)
+        if (p.seg[i].alpha != p.seg[0].alpha || p.seg[i].cols != p.seg[0].cols)
+            return;
+    p.alpha_shared = p.seg[0].alpha;
+    p.alpha_cols = p.seg[0].cols;
+}
+
 template <class P, class SegK, class Make, class Launch>
 ds_status launch_all(int nseg, const int64_t *rows, const std::vector<RowClass> &cls, float eps, Make make,
                      Launch launch, void *stream)
@@ -255,6 +271,7 @@ ds_status launch_all(int nseg, const int64_t *rows, const std::vector<RowClass> 
             params.unit_start[n] = units;
             params.eps = eps;
             params.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+            shared_alpha(params, n);
             const int e = launch(rc, params, units, stream);
             if (e != 0) {
                 char buf[160];

@@ -30,6 +30,7 @@ constexpr int kSegPerLaunch = 128;
 constexpr int kTileSlotBytes = 16384;  // rows whose staged input fits a slot
 constexpr int kMaxTileSlots = 13;      // 13 x 16 KB = 208 KB of the 227 KB per CTA
 constexpr int kTileMaxRowsPerSlot = 64;
+constexpr int kTileAlphaCache = 4096;  // slerp: |alpha| staged in shared memory up to this many columns
 // Two-pass path: units per thread per chunk, chunk size, pipeline stages.
 constexpr int kStreamK = 4;
 constexpr int kChunkUnits = kCta * kStreamK;
@@ -95,6 +96,9 @@ struct LaunchParams {
     int32_t nseg;
     float eps;
     uint64_t wait_limit_ns;                // bound of every device-side wait
+    const float *alpha_shared;             // slerp: alpha of every segment (or NULL if they differ)
+    int32_t alpha_cols;                    //        its length
+    int32_t pad_;
 };
 
 using WParams = LaunchParams<WSegK>;

@@ -427,7 +427,8 @@ __device__ __forceinline__ float2 lerp2(float2 a, float2 b, float2 m)
 }
 
 __device__ __forceinline__ void tile_slerp_row(const ASegK &sg, int64_t row, unsigned char *s0, unsigned char *s1,
-                                               int lane, int nfull, int tail, float eps, bool store)
+                                               int lane, int nfull, int tail, float eps, bool store,
+                                               const float *abs_alpha)
 {
     uint4 *xa = reinterpret_cast<uint4 *>(s0);
     uint4 *xb = reinterpret_cast<uint4 *>(s1);
@@ -447,7 +448,6 @@ __device__ __forceinline__ void tile_slerp_row(const ASegK &sg, int64_t row, uns
     }
     const float Sa = warp_sum1(aa.x + aa.y);
     const float Sb = warp_sum1(ab.x + ab.y);
-    __syncwarp();
     const RowScale ra = tile_scale(Sa, eps, [&](auto f) {
         for (int u = lane; u < nunits; u += 32)
             pairs8(xa[u], f);
@@ -456,49 +456,58 @@ __device__ __forceinline__ void tile_slerp_row(const ASegK &sg, int64_t row, uns
         for (int u = lane; u < nunits; u += 32)
             pairs8(xb[u], f);
     });
+    // pass 2: a = bf16(l2(res)), b = bf16(l2(out)), t = a + |alpha| (b - a);
+    // t (fp32) replaces res (its first 4) and out (its last 4) in the slot
+    float4 *ta = reinterpret_cast<float4 *>(s0);
+    float4 *tb = reinterpret_cast<float4 *>(s1);
     float2 at = f2(0.f, 0.f);
 #pragma unroll 2
     for (int u = lane; u < nunits; u += 32) {
         const uint4 a = scale8(xa[u], ra), b = scale8(xb[u], rb);
-        xa[u] = a;
-        xb[u] = b;
         float2 m[4];
-        alpha_pairs(sg.alpha, u, sg.cols, m);
-        sq2(at, lerp2(lo2(a.x), lo2(b.x), m[0]));
-        sq2(at, lerp2(lo2(a.y), lo2(b.y), m[1]));
-        sq2(at, lerp2(lo2(a.z), lo2(b.z), m[2]));
-        sq2(at, lerp2(lo2(a.w), lo2(b.w), m[3]));
+        if (abs_alpha) {
+            const float4 m0 = *reinterpret_cast<const float4 *>(abs_alpha + 8 * u);
+            const float4 m1 = *reinterpret_cast<const float4 *>(abs_alpha + 8 * u + 4);
+            m[0] = f2(m0.x, m0.y);
+            m[1] = f2(m0.z, m0.w);
+            m[2] = f2(m1.x, m1.y);
+            m[3] = f2(m1.z, m1.w);
+        } else {
+            alpha_pairs(sg.alpha, u, sg.cols, m);
+        }
+        const float2 t0 = lerp2(lo2(a.x), lo2(b.x), m[0]), t1 = lerp2(lo2(a.y), lo2(b.y), m[1]);
+        const float2 t2 = lerp2(lo2(a.z), lo2(b.z), m[2]), t3 = lerp2(lo2(a.w), lo2(b.w), m[3]);
+        sq2(at, t0);
+        sq2(at, t1);
+        sq2(at, t2);
+        sq2(at, t3);
+        ta[u] = make_float4(t0.x, t0.y, t1.x, t1.y);
+        tb[u] = make_float4(t2.x, t2.y, t3.x, t3.y);
     }
     const float St = warp_sum1(at.x + at.y);
-    __syncwarp();
-    auto each_t = [&](auto f) {
+    const RowScale rt = tile_scale(St, eps, [&](auto f) {
         for (int u = lane; u < nunits; u += 32) {
-            const uint4 a = xa[u], b = xb[u];
-            float2 m[4];
-            alpha_pairs(sg.alpha, u, sg.cols, m);
-            f(lerp2(lo2(a.x), lo2(b.x), m[0]));
-            f(lerp2(lo2(a.y), lo2(b.y), m[1]));
-            f(lerp2(lo2(a.z), lo2(b.z), m[2]));
-            f(lerp2(lo2(a.w), lo2(b.w), m[3]));
+            const float4 p = ta[u], q = tb[u];
+            f(f2(p.x, p.y));
+            f(f2(p.z, p.w));
+            f(f2(q.x, q.y));
+            f(f2(q.z, q.w));
         }
-    };
-    const RowScale rt = tile_scale(St, eps, each_t);
+    });
     if (!store)
         return;
     uint16_t *y = sg.y + row * sg.ld;
-    const float2 s = f2(rt.inv, rt.inv), p = f2(rt.pre, rt.pre);
-#pragma unroll 2
+    const float2 s = f2(rt.inv, rt.inv), pr = f2(rt.pre, rt.pre);
+    const bool plain = rt.pre == 1.f;
+#pragma unroll 4
     for (int u = lane; u < nunits; u += 32) {
-        const uint4 a = xa[u], b = xb[u];
-        float2 m[4];
-        alpha_pairs(sg.alpha, u, sg.cols, m);
-        float2 t0 = lerp2(lo2(a.x), lo2(b.x), m[0]), t1 = lerp2(lo2(a.y), lo2(b.y), m[1]);
-        float2 t2 = lerp2(lo2(a.z), lo2(b.z), m[2]), t3 = lerp2(lo2(a.w), lo2(b.w), m[3]);
-        if (rt.pre != 1.f) {
-            t0 = __fmul2_rn(t0, p);
-            t1 = __fmul2_rn(t1, p);
-            t2 = __fmul2_rn(t2, p);
-            t3 = __fmul2_rn(t3, p);
+        const float4 p = ta[u], q = tb[u];
+        float2 t0 = f2(p.x, p.y), t1 = f2(p.z, p.w), t2 = f2(q.x, q.y), t3 = f2(q.z, q.w);
+        if (!plain) {
+            t0 = __fmul2_rn(t0, pr);
+            t1 = __fmul2_rn(t1, pr);
+            t2 = __fmul2_rn(t2, pr);
+            t3 = __fmul2_rn(t3, pr);
         }
         const uint4 h = make_uint4(pk(__fmul2_rn(t0, s)), pk(__fmul2_rn(t1, s)), pk(__fmul2_rn(t2, s)),
                                    pk(__fmul2_rn(t3, s)));
@@ -523,6 +532,8 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
     __shared__ __align__(8) uint64_t empty[kMaxTileSlots];
     __shared__ SlotHdr hdr[kMaxTileSlots];
     __shared__ volatile int abort_flag; // set by the first wait that runs out
+    // slerp: |alpha| of the launch's (single) alpha vector
+    __shared__ __align__(16) float s_alpha[T == tSlerp ? kTileAlphaCache : 4];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t total = p.unit_start[p.nseg];
@@ -537,6 +548,11 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
         abort_flag = 0;
         mbar_init_fence();
     }
+    if constexpr (T == tSlerp) {
+        if (p.alpha_shared)
+            for (int i = threadIdx.x; i < p.alpha_cols; i += blockDim.x)
+                s_alpha[i] = fabsf(__ldg(p.alpha_shared + i));
+    }
     __syncthreads();
 
     using Layout = TileLayout<T>;
@@ -545,6 +561,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
     if (warp == kConsumerWarps) {
         // ------------------------------------------------------ producer --
         if (lane == 0) {
+            int si = 0;
             for (int64_t j = 0; j < mine; ++j) {
                 const int s = static_cast<int>(j % nslots);
                 if (j >= nslots && (abort_flag ||
@@ -554,7 +571,8 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
                     break;
                 }
                 const int64_t slot = blockIdx.x + j * gridDim.x;
-                const int si = find_segment(p, slot);
+                while (si + 1 < p.nseg && p.unit_start[si + 1] <= slot) // slots increase: walk forward
+                    ++si;
                 const auto &sg = p.seg[si];
                 const int rps = sg.group; // rows per slot for this segment
                 const int64_t row0 = (slot - p.unit_start[si]) * rps;
@@ -635,7 +653,8 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
                 else if constexpr (T == tL2)
                     tile_l2_row(sg, row, s0, s1, lane, nfull, tail, p.eps, got);
                 else
-                    tile_slerp_row(sg, row, s0, s1, lane, nfull, tail, p.eps, got);
+                    tile_slerp_row(sg, row, s0, s1, lane, nfull, tail, p.eps, got,
+                                   p.alpha_shared ? s_alpha : nullptr);
             }
             // the slot may hold this warp's generic-proxy writes (s, a, b):
             // order them before the next bulk copy into it, then release it
