@@ -421,7 +421,7 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         if (rc.path == DS_PATH_WARP) {
             const int tag = wop == W_FWD ? (bf16 ? 0 : 1) : wop == W_BWD ? (bf16 ? 2 : 3) : 4;
             const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
-            return ds::launch_tile(tag, &p, grid, ds::kTileSlotBytes, ds::kMaxTileSlots, st);
+            return ds::launch_tile(tag, &p, grid, ds::kTileSlotBytes, st);
         }
         switch (wop) {
         case W_FWD: return ds::launch_wn_forward(rc, p, units, bf16, st);
@@ -481,7 +481,7 @@ ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *st
     auto launch = [&](const RowClass &rc, const AParams &p, int64_t units, void *st) -> int {
         if (rc.path == DS_PATH_WARP) {
             const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
-            return ds::launch_tile(slerp ? 6 : 5, &p, grid, ds::kTileSlotBytes, ds::kMaxTileSlots, st);
+            return ds::launch_tile(slerp ? 6 : 5, &p, grid, ds::kTileSlotBytes, st);
         }
         return slerp ? ds::launch_slerp_rows(rc, p, units, st) : ds::launch_l2_rows(rc, p, units, st);
     };

@@ -28,7 +28,7 @@ constexpr int kMaxCluster = 8;
 constexpr int kSegPerLaunch = 128;
 // Warp-per-row (tile) path: ring of shared-memory slots filled by bulk copies.
 constexpr int kTileSlotBytes = 16384;  // rows whose staged input fits a slot
-constexpr int kMaxTileSlots = 13;      // 13 x 16 KB = 208 KB of the 227 KB per CTA
+constexpr int kMaxTileSlots = 13;      // 13 x 16 KB = 208 KB of the 227 KB per CTA (12 for activations)
 constexpr int kTileMaxRowsPerSlot = 64;
 constexpr int kTileAlphaCache = 4096;  // slerp: |alpha| staged in shared memory up to this many columns
 // Two-pass path: units per thread per chunk, chunk size, pipeline stages.
@@ -124,7 +124,7 @@ int launch_wait_selftest(uint64_t limit_ns, void *stream);
 // 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp; params is a
 // WParams (tags 0-4) or AParams (5-6) whose segments carry rows per slot in
 // `group` and whose unit_start counts slots.
-int launch_tile(int tag, const void *params, int grid, int slot_bytes, int nslots, void *stream);
+int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream);
 int read_and_clear_device_error(uint32_t *code, uint32_t *site, void *stream);
 
 } // namespace ds

@@ -5,13 +5,13 @@
 // (slot = a run of consecutive rows of one segment, at most kTileSlotBytes of
 // input) in order, waits until the slot's ring position is free, and fills
 // it with one cp.async.bulk per array (or per row when rows are padded)
-// completing on that position's "full" mbarrier.  Each of the other warps
-// owns one ring position: slot j of the CTA goes to position and warp
-// j % kMaxTileSlots, which waits on "full", normalises its rows out of shared
-// memory, stores the results straight to global memory, and arrives on
-// "empty".  Because a position is consumed by one warp, in order, no barrier
-// is ever waited on more than one phase ahead of its current phase.  Every
-// wait is bounded.
+// completing on that position's "full" mbarrier.  The other warps own the
+// ring positions -- one warp each for the weight calls, a pair for the
+// activation calls: slot j of the CTA goes to position j % positions, whose
+// warp(s) wait on "full", normalise its rows out of shared memory, store the
+// results straight to global memory, and arrive on "empty".  Because a
+// position is consumed by its own warps, in order, no barrier is ever waited
+// on more than one phase ahead of its current phase.  Every wait is bounded.
 //
 // Per row a warp sums in a fixed order -- each lane its units u = lane,
 // lane + 32, ... in order, two packed fp32 accumulators (even and odd
@@ -28,8 +28,6 @@ enum TileTag { tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp };
 
 namespace {
 
-constexpr int kConsumerWarps = kMaxTileSlots;
-constexpr int kTileThreads = (kConsumerWarps + 1) * 32;
 
 struct SlotHdr {
     int32_t seg;
@@ -73,19 +71,82 @@ __device__ __forceinline__ void each4_(float4 v, F &&f)
 
 __device__ __forceinline__ float2 fneg2(float2 v) { return f2(-v.x, -v.y); }
 
-// Factor of a row from its warp-summed S (see RowScale).  The rescale path
+__device__ __forceinline__ void named_sync(int id, int nthreads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// The threads that normalise one row: one warp (weight calls) or the pair of
+// warps that share a ring position (activation calls).  A sum comes back to
+// every thread with the same bits: the xor butterfly in each warp, then, for
+// a pair, warp 0's partial plus warp 1's through shared memory and the
+// position's named barrier.  Two alternating slots make back-to-back
+// reductions safe with one barrier each (both warps of a pair always run the
+// same sequence of reductions).
+template <int WP>
+struct Team {
+    static constexpr int G = 32 * WP; // threads per row
+    int t;                            // this thread's index in the team
+    int bar;                          // named barrier (pairs)
+    float *red;                       // [2 slots][2 warps][2 values] of the position
+    int slot = 0;
+
+    template <int N>
+    __device__ __forceinline__ void sum(float (&v)[N])
+    {
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            v[i] = warp_sum1(v[i]);
+        if constexpr (WP > 1) {
+            static_assert(N <= 2, "two values at most");
+            float *r = red + slot * 4;
+            if ((t & 31) == 0)
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+                    r[(t >> 5) * 2 + i] = v[i];
+            named_sync(bar, G);
+#pragma unroll
+            for (int i = 0; i < N; ++i)
+                v[i] = r[i] + r[2 + i];
+            slot ^= 1;
+        }
+    }
+
+    __device__ __forceinline__ float sum1(float v)
+    {
+        float a[1] = {v};
+        sum(a);
+        return a[0];
+    }
+
+    __device__ __forceinline__ float max(float v)
+    {
+        v = warp_max1(v);
+        if constexpr (WP > 1) {
+            float *r = red + slot * 4;
+            if ((t & 31) == 0)
+                r[(t >> 5) * 2] = v;
+            named_sync(bar, G);
+            v = fmaxf(r[0], r[2]);
+            slot ^= 1;
+        }
+        return v;
+    }
+};
+
+// Factor of a row from its team-summed S (see RowScale).  The rescale path
 // re-sums with exactly the fast path's structure -- the same pairs, in the
 // same order, into two packed accumulators -- so that a row scaled by 2^k
 // gives the same bits whichever path it takes.  `gen(f)` calls f(pair) on
-// every pair the lane summed, in order.
-template <class Gen>
-__device__ __forceinline__ RowScale tile_scale(float S, float eps, Gen &&gen)
+// every pair the thread summed, in order.  The branch is uniform over the team.
+template <class Red, class Gen>
+__device__ __forceinline__ RowScale tile_scale(Red &red, float S, float eps, Gen &&gen)
 {
     if (!needs_rescale(S, eps))
         return {1.0f / sqrtf(S + eps), 1.f};
     float M = 0.f;
     gen([&](float2 v) { M = fmaxf(M, fmaxf(fabsf(v.x), fabsf(v.y))); });
-    M = warp_max1(M);
+    M = red.max(M);
     if (!(M > 0.f && M < __int_as_float(0x7f800000)))
         return {1.0f / sqrtf(S + eps), 1.f};
     const int m = 48 - ilogbf(M);
@@ -94,7 +155,7 @@ __device__ __forceinline__ RowScale tile_scale(float S, float eps, Gen &&gen)
         const float2 u = f2(scalbnf(v.x, m), scalbnf(v.y, m));
         acc = __ffma2_rn(u, u, acc);
     });
-    const float Ss = warp_sum1(acc.x + acc.y);
+    const float Ss = red.sum1(acc.x + acc.y);
     const float inv = 1.0f / sqrtf(Ss + scalbnf(eps, 2 * m));
     if (m > 100)
         return {scalbnf(inv, 100), scalbnf(1.f, m - 100)};
@@ -190,8 +251,9 @@ __device__ __forceinline__ void tile_scale_row(const WSegK &sg, int64_t row, flo
         sq2(acc, f2(vt.x, vt.y));
         sq2(acc, f2(vt.z, vt.w));
     }
+    Team<1> tm{lane, 0, nullptr};
     const float S = warp_sum1(acc.x + acc.y);
-    const RowScale rs = tile_scale(S, eps, [&](auto f) {
+    const RowScale rs = tile_scale(tm, S, eps, [&](auto f) {
         for (int u = lane; u < nfull; u += 32) {
             const float4 v = w[u];
             f(f2(v.x, v.y));
@@ -380,113 +442,164 @@ __device__ __forceinline__ void store_tail8(uint16_t *o, uint4 v, int valid)
     }
 }
 
-// l2 rows.  With a residual, pass 1 writes s = bf16(x + r) back over x in the
-// slot, so pass 2 reads s directly.
-__device__ __forceinline__ void tile_l2_row(const ASegK &sg, int64_t row, unsigned char *s0, const unsigned char *s1,
-                                            int lane, int nfull, int tail, float eps, bool store)
+// l2 rows (a pair of warps per row).  With a residual, pass 1 writes
+// s = bf16(x + r) back over x in the slot (each thread its own units), so
+// pass 2 reads s directly.  Full units run in the loops; the ragged last
+// unit (if any) once, by its owner.
+template <bool HAS_R>
+__device__ __forceinline__ uint4 l2_unit_s(const uint4 *x, const uint4 *r, int u)
 {
+    uint4 s = x[u];
+    if constexpr (HAS_R) {
+        const uint4 b = r[u];
+        s = make_uint4(add_bf2(s.x, b.x), add_bf2(s.y, b.y), add_bf2(s.z, b.z), add_bf2(s.w, b.w));
+    }
+    return s;
+}
+
+template <int WP, bool HAS_R>
+__device__ __forceinline__ void tile_l2_row(Team<WP> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
+                                            const unsigned char *s1, int nfull, int tail, float eps, bool store)
+{
+    constexpr int G = Team<WP>::G;
+    const int t = tm.t;
+    const bool tl = tail && t == nfull % G;
     uint4 *x = reinterpret_cast<uint4 *>(s0);
     const uint4 *r = reinterpret_cast<const uint4 *>(s1);
-    const bool has_r = sg.r != nullptr;
     float2 acc = f2(0.f, 0.f);
-    const int nunits = nfull + (tail ? 1 : 0);
 #pragma unroll 4
-    for (int u = lane; u < nunits; u += 32) {
-        uint4 s = x[u];
-        if (has_r) {
-            const uint4 b = r[u];
-            s = make_uint4(add_bf2(s.x, b.x), add_bf2(s.y, b.y), add_bf2(s.z, b.z), add_bf2(s.w, b.w));
-        }
-        if (u == nfull)
-            s = mask_octet(s, tail);
-        if (has_r || u == nfull)
+    for (int u = t; u < nfull; u += G) {
+        const uint4 s = l2_unit_s<HAS_R>(x, r, u);
+        if constexpr (HAS_R)
             x[u] = s;
         sq8(acc, s);
     }
-    const float S = warp_sum1(acc.x + acc.y);
-    __syncwarp();
-    const RowScale rs = tile_scale(S, eps, [&](auto f) {
-        for (int u = lane; u < nunits; u += 32)
+    if (tl) {
+        const uint4 s = mask_octet(l2_unit_s<HAS_R>(x, r, nfull), tail);
+        x[nfull] = s;
+        sq8(acc, s);
+    }
+    const float S = tm.sum1(acc.x + acc.y);
+    const int nunits = nfull + (tail ? 1 : 0);
+    const RowScale rs = tile_scale(tm, S, eps, [&](auto f) {
+        for (int u = t; u < nunits; u += G)
             pairs8(x[u], f);
     });
     if (!store)
         return;
     uint16_t *y = sg.y + row * sg.ld;
 #pragma unroll 4
-    for (int u = lane; u < nfull; u += 32)
+    for (int u = t; u < nfull; u += G)
         st16(y + 8 * u, scale8(x[u], rs));
-    if (tail && lane == (nfull & 31))
+    if (tl)
         store_tail8(y + 8 * nfull, scale8(x[nfull], rs), tail);
 }
 
-// slerp rows: pass 1 sums res^2 and out^2; pass 2 writes a = bf16(l2(res)) and
-// b = bf16(l2(out)) back into the slot and sums t^2; pass 3 writes h.
+// slerp rows (a pair of warps per row).  Pass 1 sums res^2 and out^2.
+// Pass 2 forms a = bf16(l2(res)), b = bf16(l2(out)) and the lerp
+// t = a + |alpha| (b - a) in fp32, sums t^2, and writes t over the row's
+// inputs in the slot (t's first four of each unit over res, the last four
+// over out; each thread its own units).  Pass 3 scales t and stores h.  The
+// full units run in the loops; the ragged last unit (if any) once, by its
+// owner, after them.
 __device__ __forceinline__ float2 lerp2(float2 a, float2 b, float2 m)
 {
     return __ffma2_rn(m, __fadd2_rn(b, fneg2(a)), a);
 }
 
-__device__ __forceinline__ void tile_slerp_row(const ASegK &sg, int64_t row, unsigned char *s0, unsigned char *s1,
-                                               int lane, int nfull, int tail, float eps, bool store,
+template <bool CACHED>
+__device__ __forceinline__ void abs_alpha8(const float *abs_alpha, const float *alpha, int u, int cols, float2 (&m)[4])
+{
+    if constexpr (CACHED) {
+        const float4 m0 = *reinterpret_cast<const float4 *>(abs_alpha + 8 * u);
+        const float4 m1 = *reinterpret_cast<const float4 *>(abs_alpha + 8 * u + 4);
+        m[0] = f2(m0.x, m0.y);
+        m[1] = f2(m0.z, m0.w);
+        m[2] = f2(m1.x, m1.y);
+        m[3] = f2(m1.z, m1.w);
+    } else {
+        alpha_pairs(alpha, u, cols, m);
+    }
+}
+
+template <bool CACHED>
+__device__ __forceinline__ void slerp_unit_t(uint4 p, uint4 q, RowScale ra, RowScale rb, const float *abs_alpha,
+                                             const float *alpha, int u, int cols, float2 &at, float4 &ta, float4 &tb)
+{
+    const uint4 a = scale8(p, ra), b = scale8(q, rb);
+    float2 m[4];
+    abs_alpha8<CACHED>(abs_alpha, alpha, u, cols, m);
+    const float2 t0 = lerp2(lo2(a.x), lo2(b.x), m[0]), t1 = lerp2(lo2(a.y), lo2(b.y), m[1]);
+    const float2 t2 = lerp2(lo2(a.z), lo2(b.z), m[2]), t3 = lerp2(lo2(a.w), lo2(b.w), m[3]);
+    sq2(at, t0);
+    sq2(at, t1);
+    sq2(at, t2);
+    sq2(at, t3);
+    ta = make_float4(t0.x, t0.y, t1.x, t1.y);
+    tb = make_float4(t2.x, t2.y, t3.x, t3.y);
+}
+
+__device__ __forceinline__ uint4 slerp_unit_h(float4 p, float4 q, float2 s)
+{
+    return make_uint4(pk(__fmul2_rn(f2(p.x, p.y), s)), pk(__fmul2_rn(f2(p.z, p.w), s)),
+                      pk(__fmul2_rn(f2(q.x, q.y), s)), pk(__fmul2_rn(f2(q.z, q.w), s)));
+}
+
+template <int WP, bool CACHED>
+__device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
+                                               unsigned char *s1, int nfull, int tail, float eps, bool store,
                                                const float *abs_alpha)
 {
+    constexpr int G = Team<WP>::G;
+    const int t = tm.t;
+    const bool tl = tail && t == nfull % G; // owner of the ragged last unit
     uint4 *xa = reinterpret_cast<uint4 *>(s0);
     uint4 *xb = reinterpret_cast<uint4 *>(s1);
-    const int nunits = nfull + (tail ? 1 : 0);
+    float4 *ta = reinterpret_cast<float4 *>(s0);
+    float4 *tb = reinterpret_cast<float4 *>(s1);
+    // pass 1
     float2 aa = f2(0.f, 0.f), ab = f2(0.f, 0.f);
 #pragma unroll 4
-    for (int u = lane; u < nunits; u += 32) {
-        uint4 p = xa[u], q = xb[u];
-        if (u == nfull) {
-            p = mask_octet(p, tail);
-            q = mask_octet(q, tail);
-            xa[u] = p;
-            xb[u] = q;
-        }
+    for (int u = t; u < nfull; u += G) {
+        sq8(aa, xa[u]);
+        sq8(ab, xb[u]);
+    }
+    if (tl) {
+        const uint4 p = mask_octet(xa[nfull], tail), q = mask_octet(xb[nfull], tail);
+        xa[nfull] = p;
+        xb[nfull] = q;
         sq8(aa, p);
         sq8(ab, q);
     }
-    const float Sa = warp_sum1(aa.x + aa.y);
-    const float Sb = warp_sum1(ab.x + ab.y);
-    const RowScale ra = tile_scale(Sa, eps, [&](auto f) {
-        for (int u = lane; u < nunits; u += 32)
+    float sab[2] = {aa.x + aa.y, ab.x + ab.y};
+    tm.sum(sab);
+    const int nunits = nfull + (tail ? 1 : 0);
+    const RowScale ra = tile_scale(tm, sab[0], eps, [&](auto f) {
+        for (int u = t; u < nunits; u += G)
             pairs8(xa[u], f);
     });
-    const RowScale rb = tile_scale(Sb, eps, [&](auto f) {
-        for (int u = lane; u < nunits; u += 32)
+    const RowScale rb = tile_scale(tm, sab[1], eps, [&](auto f) {
+        for (int u = t; u < nunits; u += G)
             pairs8(xb[u], f);
     });
-    // pass 2: a = bf16(l2(res)), b = bf16(l2(out)), t = a + |alpha| (b - a);
-    // t (fp32) replaces res (its first 4) and out (its last 4) in the slot
-    float4 *ta = reinterpret_cast<float4 *>(s0);
-    float4 *tb = reinterpret_cast<float4 *>(s1);
+    // pass 2
     float2 at = f2(0.f, 0.f);
-#pragma unroll 2
-    for (int u = lane; u < nunits; u += 32) {
-        const uint4 a = scale8(xa[u], ra), b = scale8(xb[u], rb);
-        float2 m[4];
-        if (abs_alpha) {
-            const float4 m0 = *reinterpret_cast<const float4 *>(abs_alpha + 8 * u);
-            const float4 m1 = *reinterpret_cast<const float4 *>(abs_alpha + 8 * u + 4);
-            m[0] = f2(m0.x, m0.y);
-            m[1] = f2(m0.z, m0.w);
-            m[2] = f2(m1.x, m1.y);
-            m[3] = f2(m1.z, m1.w);
-        } else {
-            alpha_pairs(sg.alpha, u, sg.cols, m);
-        }
-        const float2 t0 = lerp2(lo2(a.x), lo2(b.x), m[0]), t1 = lerp2(lo2(a.y), lo2(b.y), m[1]);
-        const float2 t2 = lerp2(lo2(a.z), lo2(b.z), m[2]), t3 = lerp2(lo2(a.w), lo2(b.w), m[3]);
-        sq2(at, t0);
-        sq2(at, t1);
-        sq2(at, t2);
-        sq2(at, t3);
-        ta[u] = make_float4(t0.x, t0.y, t1.x, t1.y);
-        tb[u] = make_float4(t2.x, t2.y, t3.x, t3.y);
+#pragma unroll 4
+    for (int u = t; u < nfull; u += G) {
+        float4 p, q;
+        slerp_unit_t<CACHED>(xa[u], xb[u], ra, rb, abs_alpha, sg.alpha, u, sg.cols, at, p, q);
+        ta[u] = p;
+        tb[u] = q;
     }
-    const float St = warp_sum1(at.x + at.y);
-    const RowScale rt = tile_scale(St, eps, [&](auto f) {
-        for (int u = lane; u < nunits; u += 32) {
+    if (tl) {
+        float4 p, q;
+        slerp_unit_t<CACHED>(xa[nfull], xb[nfull], ra, rb, abs_alpha, sg.alpha, nfull, sg.cols, at, p, q);
+        ta[nfull] = p;
+        tb[nfull] = q;
+    }
+    const float St = tm.sum1(at.x + at.y);
+    const RowScale rt = tile_scale(tm, St, eps, [&](auto f) {
+        for (int u = t; u < nunits; u += G) {
             const float4 p = ta[u], q = tb[u];
             f(f2(p.x, p.y));
             f(f2(p.z, p.w));
@@ -496,25 +609,27 @@ __device__ __forceinline__ void tile_slerp_row(const ASegK &sg, int64_t row, uns
     });
     if (!store)
         return;
+    // pass 3
     uint16_t *y = sg.y + row * sg.ld;
-    const float2 s = f2(rt.inv, rt.inv), pr = f2(rt.pre, rt.pre);
-    const bool plain = rt.pre == 1.f;
+    const float2 s = f2(rt.inv, rt.inv);
+    if (rt.pre == 1.f) {
 #pragma unroll 4
-    for (int u = lane; u < nunits; u += 32) {
-        const float4 p = ta[u], q = tb[u];
-        float2 t0 = f2(p.x, p.y), t1 = f2(p.z, p.w), t2 = f2(q.x, q.y), t3 = f2(q.z, q.w);
-        if (!plain) {
-            t0 = __fmul2_rn(t0, pr);
-            t1 = __fmul2_rn(t1, pr);
-            t2 = __fmul2_rn(t2, pr);
-            t3 = __fmul2_rn(t3, pr);
+        for (int u = t; u < nfull; u += G)
+            st16(y + 8 * u, slerp_unit_h(ta[u], tb[u], s));
+    } else {
+        const float2 pr = f2(rt.pre, rt.pre);
+        for (int u = t; u < nfull; u += G) {
+            const float4 p = ta[u], q = tb[u];
+            const float4 pp = make_float4(p.x * pr.x, p.y * pr.x, p.z * pr.x, p.w * pr.x);
+            const float4 qq = make_float4(q.x * pr.x, q.y * pr.x, q.z * pr.x, q.w * pr.x);
+            st16(y + 8 * u, slerp_unit_h(pp, qq, s));
         }
-        const uint4 h = make_uint4(pk(__fmul2_rn(t0, s)), pk(__fmul2_rn(t1, s)), pk(__fmul2_rn(t2, s)),
-                                   pk(__fmul2_rn(t3, s)));
-        if (u < nfull)
-            st16(y + 8 * u, h);
-        else
-            store_tail8(y + 8 * nfull, h, tail);
+    }
+    if (tl) {
+        float4 p = ta[nfull], q = tb[nfull];
+        p = make_float4(p.x * rt.pre, p.y * rt.pre, p.z * rt.pre, p.w * rt.pre);
+        q = make_float4(q.x * rt.pre, q.y * rt.pre, q.z * rt.pre, q.w * rt.pre);
+        store_tail8(y + 8 * nfull, slerp_unit_h(p, q, s), tail);
     }
 }
 
@@ -523,15 +638,32 @@ __device__ __forceinline__ void tile_slerp_row(const ASegK &sg, int64_t row, uns
 template <int T>
 using TParams = typename std::conditional<(T <= tRenorm), WParams, AParams>::type;
 
+// Ring shape per operation: the weight calls give each 16 KB ring position
+// one consumer warp (13 positions); the activation calls, whose 16 KB rows
+// are one per position and carry more work per byte, give each position a
+// pair of warps that reduce every row together (12 positions).
 template <int T>
-__global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant__ TParams<T> p, int slot_bytes)
+struct TileCfg {
+    static constexpr int kWP = (T == tL2 || T == tSlerp) ? 2 : 1;
+    static constexpr int kSlots = kWP == 2 ? 12 : 13;
+    static constexpr int kConsumers = kWP * kSlots;
+    static constexpr int kThreads = (kConsumers + 1) * 32;
+};
+
+template <int T>
+__global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
+    k_tile(const __grid_constant__ TParams<T> p, int slot_bytes)
 {
-    constexpr int nslots = kMaxTileSlots; // one ring position per consumer warp
+    using Cfg = TileCfg<T>;
+    constexpr int WP = Cfg::kWP;
+    constexpr int nslots = Cfg::kSlots;
     extern __shared__ __align__(128) unsigned char ring[];
-    __shared__ __align__(8) uint64_t full[kMaxTileSlots];
-    __shared__ __align__(8) uint64_t empty[kMaxTileSlots];
-    __shared__ SlotHdr hdr[kMaxTileSlots];
-    __shared__ volatile int abort_flag; // set by the first wait that runs out
+    __shared__ __align__(8) uint64_t full[nslots];
+    __shared__ __align__(8) uint64_t empty[nslots];
+    __shared__ SlotHdr hdr[nslots];
+    __shared__ float red[nslots * 8];          // pair reductions: [position][2 slots][2 warps][2]
+    __shared__ int vote[nslots * 4];           // pair agreement on a wait: [position][2 phases][2 warps]
+    __shared__ volatile int abort_flag;        // set by the first wait that runs out
     // slerp: |alpha| of the launch's (single) alpha vector
     __shared__ __align__(16) float s_alpha[T == tSlerp ? kTileAlphaCache : 4];
 
@@ -543,7 +675,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
     if (threadIdx.x == 0) {
         for (int s = 0; s < nslots; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], WP);
         }
         abort_flag = 0;
         mbar_init_fence();
@@ -558,7 +690,7 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
     using Layout = TileLayout<T>;
     bool ok = true;
 
-    if (warp == kConsumerWarps) {
+    if (warp == Cfg::kConsumers) {
         // ------------------------------------------------------ producer --
         if (lane == 0) {
             int si = 0;
@@ -607,18 +739,32 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
         }
     } else {
         // ------------------------------------------------------ consumers --
-        // position `warp`; its i-th use holds slot warp + i * nslots
-        const int s = warp;
+        // ring position `s` (its warp, or its pair of warps); its i-th use
+        // holds slot s + i * nslots
+        const int s = warp / WP, half = warp % WP;
+        Team<WP> tm{half * 32 + lane, 1 + s, red + s * 8};
         uint32_t phase = 0;
-        for (int64_t j = warp; j < mine; j += nslots, phase ^= 1u) {
+        bool store = true;
+        for (int64_t j = s; j < mine; j += nslots, phase ^= 1u) {
             bool got = !abort_flag && mbar_wait_bounded(&full[s], phase, p.wait_limit_ns);
             got = __all_sync(0xffffffffu, got);
+            if constexpr (WP > 1) {
+                // both warps of the pair take the same decision (their row
+                // barriers need each other)
+                int *v = vote + s * 4 + phase * 2;
+                if (lane == 0)
+                    v[half] = got;
+                named_sync(tm.bar, Team<WP>::G);
+                got = v[0] && v[1];
+            }
             if (!got) {
+                // nothing more will arrive: store nothing from here on, but
+                // keep releasing positions so that every wait ends
                 ok = false;
                 abort_flag = 1;
-                break; // nothing more arrives; the stores of this warp stop here
+                store = false;
             }
-            const SlotHdr h = hdr[s];
+            const SlotHdr h = got ? hdr[s] : SlotHdr{0, 0, 0};
             const auto &sg = p.seg[h.seg];
             const bool has_r = seg_has_r(sg);
             const int rps = sg.group;
@@ -641,22 +787,27 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
                 }
                 const float g = __shfl_sync(0xffffffffu, g_lane, r & 31);
                 if constexpr (T == tFwdBf16)
-                    tile_scale_row<true, false>(sg, row, g, s0, lane, nfull, tail, p.eps, got);
+                    tile_scale_row<true, false>(sg, row, g, s0, lane, nfull, tail, p.eps, store);
                 else if constexpr (T == tFwdF32)
-                    tile_scale_row<false, false>(sg, row, g, s0, lane, nfull, tail, p.eps, got);
+                    tile_scale_row<false, false>(sg, row, g, s0, lane, nfull, tail, p.eps, store);
                 else if constexpr (T == tRenorm)
-                    tile_scale_row<false, true>(sg, row, 1.f, s0, lane, nfull, tail, p.eps, got);
+                    tile_scale_row<false, true>(sg, row, 1.f, s0, lane, nfull, tail, p.eps, store);
                 else if constexpr (T == tBwdBf16)
-                    tile_backward_row<true>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, got);
+                    tile_backward_row<true>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, store);
                 else if constexpr (T == tBwdF32)
-                    tile_backward_row<false>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, got);
-                else if constexpr (T == tL2)
-                    tile_l2_row(sg, row, s0, s1, lane, nfull, tail, p.eps, got);
+                    tile_backward_row<false>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, store);
+                else if constexpr (T == tL2) {
+                    if (has_r)
+                        tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
+                    else
+                        tile_l2_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
+                }
+                else if (p.alpha_shared)
+                    tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha);
                 else
-                    tile_slerp_row(sg, row, s0, s1, lane, nfull, tail, p.eps, got,
-                                   p.alpha_shared ? s_alpha : nullptr);
+                    tile_slerp_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr);
             }
-            // the slot may hold this warp's generic-proxy writes (s, a, b):
+            // the slot may hold this warp's generic-proxy writes (s, t):
             // order them before the next bulk copy into it, then release it
             fence_proxy_async_smem();
             __syncwarp();
@@ -671,11 +822,9 @@ __global__ void __launch_bounds__(kTileThreads, 1) k_tile(const __grid_constant_
 } // namespace
 
 template <int T>
-static cudaError_t launch_tile_t(const TParams<T> &p, int grid, int slot_bytes, int nslots, void *stream)
+static cudaError_t launch_tile_t(const TParams<T> &p, int grid, int slot_bytes, void *stream)
 {
-    if (nslots != kMaxTileSlots)
-        return cudaErrorInvalidValue;
-    const int smem = slot_bytes * nslots;
+    const int smem = slot_bytes * TileCfg<T>::kSlots;
     static int attr_smem = 0; // benign race: idempotent
     if (attr_smem < smem) {
         cudaError_t e = cudaFuncSetAttribute(k_tile<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -683,20 +832,20 @@ static cudaError_t launch_tile_t(const TParams<T> &p, int grid, int slot_bytes, 
             return e;
         attr_smem = smem;
     }
-    k_tile<T><<<grid, kTileThreads, smem, static_cast<cudaStream_t>(stream)>>>(p, slot_bytes);
+    k_tile<T><<<grid, TileCfg<T>::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(p, slot_bytes);
     return cudaGetLastError();
 }
 
-int launch_tile(int tag, const void *params, int grid, int slot_bytes, int nslots, void *stream)
+int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream)
 {
     switch (tag) {
-    case tFwdBf16: return launch_tile_t<tFwdBf16>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
-    case tFwdF32: return launch_tile_t<tFwdF32>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
-    case tBwdBf16: return launch_tile_t<tBwdBf16>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
-    case tBwdF32: return launch_tile_t<tBwdF32>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
-    case tRenorm: return launch_tile_t<tRenorm>(*static_cast<const WParams *>(params), grid, slot_bytes, nslots, stream);
-    case tL2: return launch_tile_t<tL2>(*static_cast<const AParams *>(params), grid, slot_bytes, nslots, stream);
-    case tSlerp: return launch_tile_t<tSlerp>(*static_cast<const AParams *>(params), grid, slot_bytes, nslots, stream);
+    case tFwdBf16: return launch_tile_t<tFwdBf16>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
+    case tFwdF32: return launch_tile_t<tFwdF32>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
+    case tBwdBf16: return launch_tile_t<tBwdBf16>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
+    case tBwdF32: return launch_tile_t<tBwdF32>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
+    case tRenorm: return launch_tile_t<tRenorm>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
+    case tL2: return launch_tile_t<tL2>(*static_cast<const AParams *>(params), grid, slot_bytes, stream);
+    case tSlerp: return launch_tile_t<tSlerp>(*static_cast<const AParams *>(params), grid, slot_bytes, stream);
     default: return cudaErrorInvalidValue;
     }
 }
