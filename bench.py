@@ -88,6 +88,25 @@ def step_rows(weights, act_rows=ACT_ROWS) -> dict[str, int]:
             "l2_rows": act_rows, "l2_rows_residual": act_rows, "slerp_rows": act_rows}
 
 
+def max_over_ranks(dist, values: list[float], device) -> list[float]:
+    """Element-wise maximum of per-rank timings (ms).  Every rank calls it at
+    the same point with the same number of values; without a process group
+    the values come back unchanged."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_gbs(world: int, bytes_per_rank: int, ms_per_step: float) -> float:
+    """Aggregate GB/s over all ranks: each rank processes its own copy of the
+    step's bytes (weak scaling) in at most the slowest rank's time."""
+    return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 def measured_peaks() -> tuple[float, str]:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -99,7 +118,8 @@ def measured_peaks() -> tuple[float, str]:
 
 def kernel_source_digest() -> str:
     h = hashlib.sha256()
-    for rel in ("l2_row_b200/csrc/ds_kernels.cu", "l2_row_b200/csrc/ds_device.cuh", "l2_row_b200/csrc/ds_internal.h"):
+    for rel in ("l2_row_b200/csrc/ds_kernels.cu", "l2_row_b200/csrc/ds_tile.cu", "l2_row_b200/csrc/ds_api.cpp",
+                "l2_row_b200/csrc/ds_device.cuh", "l2_row_b200/csrc/ds_internal.h"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -314,16 +334,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
 
     total_ms = evs[0][0].elapsed_time(evs[-1][-1])
     per_call = {name: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K)] for i, name in enumerate(CALLS)}
-    if dist:
-        t = torch.tensor([total_ms] + [statistics.fmean(v) for v in per_call.values()], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t[0])
-        call_ms = {name: float(t[i + 1]) for i, name in enumerate(CALLS)}
-    else:
-        call_ms = {name: statistics.fmean(v) for name, v in per_call.items()}
+    t = max_over_ranks(dist, [total_ms] + [statistics.fmean(per_call[n]) for n in CALLS], "cuda")
+    total_ms = t[0]
+    call_ms = {name: t[i + 1] for i, name in enumerate(CALLS)}
 
     ms_per_step = total_ms / K
-    value = world * step_total / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gbs(world, step_total, ms_per_step)
 
     peak, peak_src = measured_peaks()
     kernels = {}
@@ -402,12 +418,8 @@ def measure_e2e(step: Step, steps: int, step_total: int, sp: int, world: int, di
         one()
     b.record()
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / steps
-    if dist:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
-    return {"value": round(world * step_total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+    ms = max_over_ranks(dist, [a.elapsed_time(b) / steps], "cuda")[0]
+    return {"value": round(whole_job_gbs(world, step_total, ms), 2), "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3)}
 
 

@@ -28,7 +28,7 @@ constexpr int kMaxCluster = 8;
 constexpr int kSegPerLaunch = 128;
 // Warp-per-row (tile) path: ring of shared-memory slots filled by bulk copies.
 constexpr int kTileSlotBytes = 16384;  // rows whose staged input fits a slot
-constexpr int kMaxTileSlots = 13;      // 13 x 16 KB = 208 KB of the 227 KB per CTA (12 for activations)
+constexpr int kMaxTileSlots = 13;      // 13 x 16 KB = 208 KB of the 227 KB per CTA
 constexpr int kTileMaxRowsPerSlot = 64;
 constexpr int kTileAlphaCache = 4096;  // slerp: |alpha| staged in shared memory up to this many columns
 // Two-pass path: units per thread per chunk, chunk size, pipeline stages.

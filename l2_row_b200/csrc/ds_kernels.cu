@@ -179,12 +179,15 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, RowScale r)
     return o;
 }
 
-// |alpha| for the 8 elements of unit u (0 past cols; never read past cols).
+// |alpha| for the 8 elements of unit u, 0 past cols.  The float4 holding the
+// last valid element may extend past cols (it never leaves that 16-byte
+// block, so the read stays inside the allocation); whatever it holds there
+// is dropped, so a NaN beyond the vector cannot reach the row's sums.
 __device__ __forceinline__ void alpha8(const float *alpha, int u, int cols, float (&m)[8])
 {
     const int e0 = 8 * u;
-    float4 a = e0 < cols ? ld16_cached(alpha + e0) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 b = e0 + 4 < cols ? ld16_cached(alpha + e0 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 a = e0 < cols ? ld16_cached(alpha + e0) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 b = e0 + 4 < cols ? ld16_cached(alpha + e0 + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
     m[0] = fabsf(a.x);
     m[1] = fabsf(a.y);
     m[2] = fabsf(a.z);
@@ -193,6 +196,11 @@ __device__ __forceinline__ void alpha8(const float *alpha, int u, int cols, floa
     m[5] = fabsf(b.y);
     m[6] = fabsf(b.z);
     m[7] = fabsf(b.w);
+    if (e0 + 8 > cols) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            m[i] = e0 + i < cols ? m[i] : 0.f;
+    }
 }
 
 // The lerp t = a + |alpha| (b - a): the difference, then one fused rounding

@@ -76,19 +76,38 @@ __device__ __forceinline__ void named_sync(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// The threads that normalise one row: one warp (weight calls) or the pair of
-// warps that share a ring position (activation calls).  A sum comes back to
-// every thread with the same bits: the xor butterfly in each warp, then, for
-// a pair, warp 0's partial plus warp 1's through shared memory and the
-// position's named barrier.  Two alternating slots make back-to-back
-// reductions safe with one barrier each (both warps of a pair always run the
-// same sequence of reductions).
+// The threads that normalise one row: one warp (weight calls) or the team
+// of WP warps that share a group of ring positions (activation calls).  A
+// sum comes back to every thread with the same bits: the xor butterfly in
+// each warp, then the warps' partials through shared memory and the group's
+// named barrier, added as a balanced tree in warp order ((w0 + w1) + (w2 +
+// w3) ...).  Two alternating slots make back-to-back reductions safe with one
+// barrier each (all warps of a team run the same sequence of reductions).
+template <int N>
+__device__ __forceinline__ float tree_sum(const float *r, int i)
+{
+    if constexpr (N == 1)
+        return r[i];
+    else
+        return tree_sum<N / 2>(r, i) + tree_sum<N / 2>(r + N, i);
+}
+
+template <int N>
+__device__ __forceinline__ float tree_max(const float *r)
+{
+    if constexpr (N == 1)
+        return r[0];
+    else
+        return fmaxf(tree_max<N / 2>(r), tree_max<N / 2>(r + N));
+}
+
 template <int WP>
 struct Team {
     static constexpr int G = 32 * WP; // threads per row
+    static constexpr int kRed = 4 * WP; // floats of `red`: [2 slots][WP warps][2 values]
     int t;                            // this thread's index in the team
-    int bar;                          // named barrier (pairs)
-    float *red;                       // [2 slots][2 warps][2 values] of the position
+    int bar;                          // named barrier (teams of several warps)
+    float *red;
     int slot = 0;
 
     template <int N>
@@ -99,7 +118,7 @@ struct Team {
             v[i] = warp_sum1(v[i]);
         if constexpr (WP > 1) {
             static_assert(N <= 2, "two values at most");
-            float *r = red + slot * 4;
+            float *r = red + slot * 2 * WP;
             if ((t & 31) == 0)
 #pragma unroll
                 for (int i = 0; i < N; ++i)
@@ -107,7 +126,7 @@ struct Team {
             named_sync(bar, G);
 #pragma unroll
             for (int i = 0; i < N; ++i)
-                v[i] = r[i] + r[2 + i];
+                v[i] = tree_sum<WP>(r, i);
             slot ^= 1;
         }
     }
@@ -123,11 +142,11 @@ struct Team {
     {
         v = warp_max1(v);
         if constexpr (WP > 1) {
-            float *r = red + slot * 4;
+            float *r = red + slot * 2 * WP;
             if ((t & 31) == 0)
                 r[(t >> 5) * 2] = v;
             named_sync(bar, G);
-            v = fmaxf(r[0], r[2]);
+            v = tree_max<WP>(r);
             slot ^= 1;
         }
         return v;
@@ -162,7 +181,9 @@ __device__ __forceinline__ RowScale tile_scale(Red &red, float S, float eps, Gen
     return {scalbnf(inv, m), 1.f};
 }
 
-// |alpha| for the 8 elements of unit u, as four pairs (0 past cols).
+// |alpha| for the 8 elements of unit u, as four pairs, 0 past cols (the
+// float4 holding the last valid element may extend past cols inside its
+// 16-byte block; what it holds there is dropped).
 __device__ __forceinline__ void alpha_pairs(const float *alpha, int u, int cols, float2 (&m)[4])
 {
     const int e0 = 8 * u;
@@ -172,6 +193,11 @@ __device__ __forceinline__ void alpha_pairs(const float *alpha, int u, int cols,
     m[1] = f2(fabsf(a.z), fabsf(a.w));
     m[2] = f2(fabsf(b.x), fabsf(b.y));
     m[3] = f2(fabsf(b.z), fabsf(b.w));
+    if (e0 + 8 > cols) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            m[i] = f2(e0 + 2 * i < cols ? m[i].x : 0.f, e0 + 2 * i + 1 < cols ? m[i].y : 0.f);
+    }
 }
 
 // ------------------------------------------------------- layout per op ---
@@ -401,12 +427,36 @@ __device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, 
 }
 
 // Octet helpers: 8 bf16 as four packed pairs.
-__device__ __forceinline__ void sq8(float2 &acc, uint4 v)
+//
+// Squares of a bf16 pair into the (even, odd) accumulators with one fused
+// multiply-add per element taken straight from the packed halves: the
+// product of two bf16 is exact in fp32, so each step rounds exactly as the
+// fp32 fma of the widened values would (the same bits as sq2(acc, lo2(w))).
+__device__ __forceinline__ void sq_bf2(float2 &acc, uint32_t w)
+{
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, l, l, %0;\n\tfma.rn.f32.bf16 %1, h, h, %1;\n\t}"
+        : "+f"(acc.x), "+f"(acc.y)
+        : "r"(w));
+}
+
+// The same sums through widened pairs (packed fp32 fma): the l2 rows use
+// this form (with a residual the widened pairs also serve the sum x + r);
+// slerp's two-array pass 1 is faster with sq8.
+__device__ __forceinline__ void sq8w(float2 &acc, uint4 v)
 {
     sq2(acc, lo2(v.x));
     sq2(acc, lo2(v.y));
     sq2(acc, lo2(v.z));
     sq2(acc, lo2(v.w));
+}
+
+__device__ __forceinline__ void sq8(float2 &acc, uint4 v)
+{
+    sq_bf2(acc, v.x);
+    sq_bf2(acc, v.y);
+    sq_bf2(acc, v.z);
+    sq_bf2(acc, v.w);
 }
 
 template <class F>
@@ -429,6 +479,10 @@ __device__ __forceinline__ uint4 scale8(uint4 v, RowScale r)
                       pk(__fmul2_rn(__fmul2_rn(lo2(v.z), p), s)), pk(__fmul2_rn(__fmul2_rn(lo2(v.w), p), s)));
 }
 
+// bf16(x + r) for a pair: the fp32 sum, rounded to nearest even.  The fp32
+// sum of two bf16 is exact unless their exponents are more than 16 apart,
+// and then its error lies far from any bf16 halfway point, so this is the
+// exact sum rounded once.
 __device__ __forceinline__ uint32_t add_bf2(uint32_t a, uint32_t b)
 {
     return pk(__fadd2_rn(lo2(a), lo2(b)));
@@ -472,12 +526,12 @@ __device__ __forceinline__ void tile_l2_row(Team<WP> &tm, const ASegK &sg, int64
         const uint4 s = l2_unit_s<HAS_R>(x, r, u);
         if constexpr (HAS_R)
             x[u] = s;
-        sq8(acc, s);
+        sq8w(acc, s);
     }
     if (tl) {
         const uint4 s = mask_octet(l2_unit_s<HAS_R>(x, r, nfull), tail);
         x[nfull] = s;
-        sq8(acc, s);
+        sq8w(acc, s);
     }
     const float S = tm.sum1(acc.x + acc.y);
     const int nunits = nfull + (tail ? 1 : 0);
@@ -511,8 +565,8 @@ template <bool CACHED>
 __device__ __forceinline__ void abs_alpha8(const float *abs_alpha, const float *alpha, int u, int cols, float2 (&m)[4])
 {
     if constexpr (CACHED) {
-        const float4 m0 = *reinterpret_cast<const float4 *>(abs_alpha + 8 * u);
-        const float4 m1 = *reinterpret_cast<const float4 *>(abs_alpha + 8 * u + 4);
+        const float4 m0 = *reinterpret_cast<const float4 *>(abs_alpha + 4 * u);
+        const float4 m1 = *reinterpret_cast<const float4 *>(abs_alpha + kTileAlphaCache / 2 + 4 * u);
         m[0] = f2(m0.x, m0.y);
         m[1] = f2(m0.z, m0.w);
         m[2] = f2(m1.x, m1.y);
@@ -559,7 +613,7 @@ __device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, in
     float4 *tb = reinterpret_cast<float4 *>(s1);
     // pass 1
     float2 aa = f2(0.f, 0.f), ab = f2(0.f, 0.f);
-#pragma unroll 4
+#pragma unroll 2
     for (int u = t; u < nfull; u += G) {
         sq8(aa, xa[u]);
         sq8(ab, xb[u]);
@@ -638,16 +692,19 @@ __device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, in
 template <int T>
 using TParams = typename std::conditional<(T <= tRenorm), WParams, AParams>::type;
 
-// Ring shape per operation: the weight calls give each 16 KB ring position
-// one consumer warp (13 positions); the activation calls, whose 16 KB rows
-// are one per position and carry more work per byte, give each position a
-// pair of warps that reduce every row together (12 positions).
+// Ring shape per operation: 13 ring positions of 16 KB.  The weight calls
+// give each position one consumer warp.  The activation calls, one 16 KB
+// row per position and more work per byte, give each position a pair of
+// warps that reduce every row together (27 warps; slerp's |alpha| cache
+// brings shared memory to ~225 KB of the 227 KB a CTA may hold).
 template <int T>
 struct TileCfg {
     static constexpr int kWP = (T == tL2 || T == tSlerp) ? 2 : 1;
-    static constexpr int kSlots = kWP == 2 ? 12 : 13;
-    static constexpr int kConsumers = kWP * kSlots;
+    static constexpr int kGroups = 13;
+    static constexpr int kSlots = kGroups; // one position per team
+    static constexpr int kConsumers = kWP * kGroups;
     static constexpr int kThreads = (kConsumers + 1) * 32;
+    static_assert(kSlots <= kMaxTileSlots && kConsumers + 1 <= 32, "ring shape");
 };
 
 template <int T>
@@ -661,9 +718,9 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
     __shared__ __align__(8) uint64_t full[nslots];
     __shared__ __align__(8) uint64_t empty[nslots];
     __shared__ SlotHdr hdr[nslots];
-    __shared__ float red[nslots * 8];          // pair reductions: [position][2 slots][2 warps][2]
-    __shared__ int vote[nslots * 4];           // pair agreement on a wait: [position][2 phases][2 warps]
-    __shared__ volatile int abort_flag;        // set by the first wait that runs out
+    __shared__ float red[Cfg::kGroups * Team<WP>::kRed]; // team reductions
+    __shared__ int vote[Cfg::kGroups * 2 * WP];           // team agreement on a wait: [team][2][warp]
+    __shared__ volatile int abort_flag;                    // set by the first wait that runs out
     // slerp: |alpha| of the launch's (single) alpha vector
     __shared__ __align__(16) float s_alpha[T == tSlerp ? kTileAlphaCache : 4];
 
@@ -675,15 +732,23 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < nslots; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], WP);
+            mbar_init(&empty[s], WP); // every warp of the owning team arrives
         }
         abort_flag = 0;
         mbar_init_fence();
     }
     if constexpr (T == tSlerp) {
-        if (p.alpha_shared)
-            for (int i = threadIdx.x; i < p.alpha_cols; i += blockDim.x)
-                s_alpha[i] = fabsf(__ldg(p.alpha_shared + i));
+        // |alpha| split by halves of each 8-element unit: unit u's first four
+        // at [4u], its last four at [half + 4u], so that a warp reading one
+        // float4 per lane touches consecutive 16-byte words (no bank conflict)
+        if (p.alpha_shared) {
+            const int nu = (p.alpha_cols + 7) / 8, half = kTileAlphaCache / 2;
+            for (int i = threadIdx.x; i < 8 * nu; i += blockDim.x) {
+                const int u = i >> 3, e = i & 7;
+                const float v = i < p.alpha_cols ? fabsf(__ldg(p.alpha_shared + i)) : 0.f;
+                s_alpha[(e < 4 ? 0 : half) + 4 * u + (e & 3)] = v;
+            }
+        }
     }
     __syncthreads();
 
@@ -739,23 +804,29 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
         }
     } else {
         // ------------------------------------------------------ consumers --
-        // ring position `s` (its warp, or its pair of warps); its i-th use
-        // holds slot s + i * nslots
-        const int s = warp / WP, half = warp % WP;
-        Team<WP> tm{half * 32 + lane, 1 + s, red + s * 8};
-        uint32_t phase = 0;
+        // team q (one warp, or WP warps) owns ring positions q, q + kGroups,
+        // ...; the CTA's slot j sits at position j % nslots, so the team
+        // takes slots j = q, q + kGroups, ... in order
+        constexpr int NG = Cfg::kGroups;
+        const int q = warp / WP, wi = warp % WP;
+        Team<WP> tm{wi * 32 + lane, 1 + q, red + q * Team<WP>::kRed};
         bool store = true;
-        for (int64_t j = s; j < mine; j += nslots, phase ^= 1u) {
+        int vb = 0;
+        for (int64_t j = q; j < mine; j += NG, vb ^= 1) {
+            const int s = static_cast<int>(j % nslots);
+            const uint32_t phase = static_cast<uint32_t>((j / nslots) & 1);
             bool got = !abort_flag && mbar_wait_bounded(&full[s], phase, p.wait_limit_ns);
             got = __all_sync(0xffffffffu, got);
             if constexpr (WP > 1) {
-                // both warps of the pair take the same decision (their row
+                // all warps of the team take the same decision (their row
                 // barriers need each other)
-                int *v = vote + s * 4 + phase * 2;
+                int *v = vote + (q * 2 + vb) * WP;
                 if (lane == 0)
-                    v[half] = got;
+                    v[wi] = got;
                 named_sync(tm.bar, Team<WP>::G);
-                got = v[0] && v[1];
+#pragma unroll
+                for (int w = 0; w < WP; ++w)
+                    got = got && v[w];
             }
             if (!got) {
                 // nothing more will arrive: store nothing from here on, but
@@ -775,6 +846,17 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
             unsigned char *a1 = base + pitch0 * rps;
             constexpr int E = (T <= tRenorm) ? 4 : 8;
             const int nfull = sg.cols / E, tail = sg.cols % E;
+            // hand the position back: the slot may hold this warp's
+            // generic-proxy writes (s, t, masked tails), so order them
+            // before the next bulk copy into it
+            bool released = false;
+            auto release = [&]() {
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&empty[s]);
+                released = true;
+            };
             float g_lane = 1.f;
             for (int r = 0; r < h.nrows; ++r) {
                 const int64_t row = h.row0 + r;
@@ -801,18 +883,14 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
                         tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
                     else
                         tile_l2_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
-                }
-                else if (p.alpha_shared)
+                } else if (p.alpha_shared) {
                     tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha);
-                else
+                } else {
                     tile_slerp_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr);
+                }
             }
-            // the slot may hold this warp's generic-proxy writes (s, t):
-            // order them before the next bulk copy into it, then release it
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&empty[s]);
+            if (!released)
+                release();
         }
     }
     if (!ok)

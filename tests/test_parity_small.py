@@ -118,7 +118,10 @@ def test_ragged_activation_rows_with_guards(path):
             assert gu.guards_intact(ybuf, rows, cols, ld, gu.CANARY_BF16), cols
             gu.check_l2(act, y, eps, what=f"l2 cols={cols}")
             h, hbuf = gu.padded(rows, cols, ld, torch.bfloat16, gu.CANARY_BF16)
-            ds.ds_slerp_rows([ds.ASeg(x=xs[0], r=rs[0], y=h, alpha=gu.dev_f32(act.alpha))], eps)
+            # alpha's storage continues with NaN past cols: none of it may reach a row
+            abuf = torch.full((cols + 8,), float("nan"), dtype=torch.float32, device="cuda")
+            abuf[:cols].copy_(gu.dev_f32(act.alpha))
+            ds.ds_slerp_rows([ds.ASeg(x=xs[0], r=rs[0], y=h, alpha=abuf[:cols])], eps)
             torch.cuda.synchronize()
             assert gu.guards_intact(hbuf, rows, cols, ld, gu.CANARY_BF16), cols
             gu.check_slerp(act, h, eps, what=f"slerp cols={cols}")
