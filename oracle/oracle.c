@@ -130,6 +130,35 @@ void or_wn_backward_row(const double *w, const double *gy, int64_t C, double g,
         grad_w[j] = (g * rho / n) * (gy[j] - w[j] * D / n2);
 }
 
+/* [DS] "Optimizer", method "rescale", before the step: the part of the
+ * gradient that would change the row's length -- its component along the
+ * row -- is removed:  D = sum_j w_j G_j,  out_j = G_j - w_j * D / (S + eps).
+ * At eps = 0 this is the orthogonal projection onto the row's complement. */
+void or_grad_project_row(const double *w, const double *G, int64_t C,
+                         double eps, unsigned flags, double *out)
+{
+    double S = sum_sq(w, C);
+    double D = 0.0;
+    for (int64_t j = 0; j < C; ++j)
+        D += w[j] * G[j];
+    double n2 = (flags & OR_EPS_ZERO) ? S : S + eps;
+    for (int64_t j = 0; j < C; ++j)
+        out[j] = G[j] - w[j] * D / n2;
+}
+
+/* [DS] "Optimizer", after the step: the same component removed from the
+ * momentum, and the row rescaled back to its radius, both from the row as
+ * the step left it (the rescale does not change its direction):
+ *   m_out_j = m_j - w_j * (sum_k w_k m_k) / (S + eps),
+ *   w_out_j = rho * w_j / sqrt(S + eps). */
+void or_renorm_momentum_row(const double *w, const double *m, int64_t C,
+                            double rho, double eps, unsigned flags,
+                            double *w_out, double *m_out)
+{
+    or_grad_project_row(w, m, C, eps, flags, m_out);
+    or_row_renorm_row(w, C, rho, eps, flags, w_out);
+}
+
 /* [DS] "Optimizer": after the step each row is rescaled back to its radius. */
 void or_row_renorm_row(const double *w, int64_t C, double rho, double eps,
                        unsigned flags, double *out)
@@ -297,7 +326,7 @@ void or_slerp_row_interval(const double *res, const double *out,
 /* Matrix drivers.  Each worker owns a contiguous range of rows and its own
  * scratch rows; inputs are widened to double exactly before the row call.   */
 
-enum { OP_FWD, OP_BWD, OP_RENORM, OP_L2, OP_SLERP, OP_L2_IV, OP_SLERP_IV };
+enum { OP_FWD, OP_BWD, OP_RENORM, OP_L2, OP_SLERP, OP_L2_IV, OP_SLERP_IV, OP_PROJECT, OP_MOMENTUM };
 
 typedef struct {
     int op;
@@ -312,6 +341,7 @@ typedef struct {
     unsigned flags;
     double *out_d;   /* dense [R, C] doubles */
     double *out_g;   /* [R] */
+    double *out_d2;  /* dense [R, C] doubles (second output) */
     uint16_t *out_h; /* dense [R, C] bf16 bits */
     uint16_t *out_h2; /* dense [R, C] bf16 bits (interval upper ends) */
     int status;
@@ -365,6 +395,21 @@ static void *run_job(void *arg)
                                jb->rho, jb->eps, jb->flags, jb->out_d + o, &gg);
             if (jb->out_g)
                 jb->out_g[row] = gg;
+            break;
+        }
+        case OP_PROJECT:
+        case OP_MOMENTUM: {
+            const float *wr = jb->w + row * jb->ld;
+            const float *gr = (const float *)jb->gy + row * jb->ld2;
+            for (int64_t j = 0; j < C; ++j) {
+                u[j] = (double)wr[j];
+                v[j] = (double)gr[j];
+            }
+            if (jb->op == OP_PROJECT)
+                or_grad_project_row(u, v, C, jb->eps, jb->flags, jb->out_d + o);
+            else
+                or_renorm_momentum_row(u, v, C, jb->rho, jb->eps, jb->flags,
+                                       jb->out_d2 + o, jb->out_d + o);
             break;
         }
         case OP_L2:
@@ -499,6 +544,52 @@ int or_wn_backward(const float *w, int64_t R, int64_t C, int64_t ld,
     jb.flags = flags;
     jb.out_d = grad_w;
     jb.out_g = grad_g;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_grad_project(const float *w, int64_t R, int64_t C, int64_t ld,
+                    const float *G, int64_t ld_g, double eps, unsigned flags,
+                    double *out, int nthreads)
+{
+    if (bad_shape(R, C, ld) || ld_g < C || (R > 0 && (!w || !G || !out)))
+        return -1;
+    if (flags & ~OR_EPS_ZERO)
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_PROJECT;
+    jb.C = C;
+    jb.ld = ld;
+    jb.ld2 = ld_g;
+    jb.w = w;
+    jb.gy = G;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_d = out;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_renorm_momentum(const float *w, int64_t R, int64_t C, int64_t ld,
+                       const float *m, int64_t ld_m, double rho, double eps,
+                       unsigned flags, double *w_out, double *m_out,
+                       int nthreads)
+{
+    if (bad_shape(R, C, ld) || ld_m < C ||
+        (R > 0 && (!w || !m || !w_out || !m_out)))
+        return -1;
+    if (flags & ~OR_EPS_ZERO)
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_MOMENTUM;
+    jb.C = C;
+    jb.ld = ld;
+    jb.ld2 = ld_m;
+    jb.w = w;
+    jb.gy = m;
+    jb.rho = rho;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_d = m_out;
+    jb.out_d2 = w_out;
     return run_rows(&jb, R, nthreads);
 }
 

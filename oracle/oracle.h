@@ -63,6 +63,18 @@ void or_wn_backward_row(const double *w, const double *gy, int64_t C, double g,
                         double rho, double eps, unsigned flags, double *grad_w,
                         double *grad_g);
 
+/* [DS] "Optimizer" (method "rescale"), before the step: the gradient's
+ * component along the row removed, out_j = G_j - w_j * (w . G) / (S + eps). */
+void or_grad_project_row(const double *w, const double *G, int64_t C,
+                         double eps, unsigned flags, double *out);
+
+/* [DS] "Optimizer", after the step: the same component removed from the
+ * momentum m, and the row rescaled back to its radius:
+ *   m_out_j = m_j - w_j (w . m) / (S + eps),  w_out_j = rho w_j / sqrt(S + eps). */
+void or_renorm_momentum_row(const double *w, const double *m, int64_t C,
+                            double rho, double eps, unsigned flags,
+                            double *w_out, double *m_out);
+
 /* [DS] "Optimizer": rescale the row back to its radius, out_j = rho w_j / n. */
 void or_row_renorm_row(const double *w, int64_t C, double rho, double eps,
                        unsigned flags, double *out);
@@ -118,6 +130,16 @@ int or_wn_backward(const float *w, int64_t R, int64_t C, int64_t ld,
 
 int or_row_renorm(const float *w, int64_t R, int64_t C, int64_t ld, double rho,
                   double eps, unsigned flags, double *out, int nthreads);
+
+/* G, m: float32 [R, C], leading dimension ld_g / ld_m.  flags: 0 or
+ * OR_EPS_ZERO. */
+int or_grad_project(const float *w, int64_t R, int64_t C, int64_t ld,
+                    const float *G, int64_t ld_g, double eps, unsigned flags,
+                    double *out, int nthreads);
+int or_renorm_momentum(const float *w, int64_t R, int64_t C, int64_t ld,
+                       const float *m, int64_t ld_m, double rho, double eps,
+                       unsigned flags, double *w_out, double *m_out,
+                       int nthreads);
 
 /* x, r: bf16 bits; r may be NULL.  y_exact may be NULL. */
 int or_l2_rows(const uint16_t *x, const uint16_t *r, int64_t R, int64_t C,

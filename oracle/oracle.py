@@ -36,6 +36,10 @@ def lib() -> ct.CDLL:
         _lib.or_wn_forward.argtypes = [vp, i64, i64, i64, vp, dbl, dbl, uns, vp, i32]
         _lib.or_wn_backward.argtypes = [vp, i64, i64, i64, vp, i32, i64, vp, dbl, dbl, uns, vp, vp, i32]
         _lib.or_row_renorm.argtypes = [vp, i64, i64, i64, dbl, dbl, uns, vp, i32]
+        _lib.or_grad_project.argtypes = [vp, i64, i64, i64, vp, i64, dbl, uns, vp, i32]
+        _lib.or_renorm_momentum.argtypes = [vp, i64, i64, i64, vp, i64, dbl, dbl, uns, vp, vp, i32]
+        _lib.or_grad_project_row.argtypes = [vp, vp, i64, dbl, uns, vp]
+        _lib.or_grad_project_row.restype = None
         _lib.or_l2_rows.argtypes = [vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
         _lib.or_slerp_rows.argtypes = [vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
         _lib.or_wn_backward_row.argtypes = [vp, vp, i64, dbl, dbl, dbl, uns, vp, vp]
@@ -191,6 +195,42 @@ def slerp_rows_interval(res, out, alpha, *, eps=1e-6, delta=1e-5, flags=0, nthre
     _check(lib().or_slerp_rows_interval(_p(res), _p(out), _p(alpha), R, C, ld, eps, delta, flags, _p(lo), _p(hi),
                                         nthreads), "slerp_rows_interval")
     return lo, hi
+
+
+def grad_project(w, G, *, eps=1e-6, flags=0, nthreads=1):
+    """f64 G - w (w . G) / (S + eps) [R, C] for fp32 rows w and gradient G."""
+    w, ld = _rows(w, np.float32)
+    G, ldg = _rows(G, np.float32)
+    R, C = w.shape
+    if G.shape != (R, C):
+        raise ValueError("G shape")
+    out = np.empty((R, C), np.float64)
+    _check(lib().or_grad_project(_p(w), R, C, ld, _p(G), ldg, eps, flags, _p(out), nthreads), "grad_project")
+    return out
+
+
+def renorm_momentum(w, m, *, rho=1.0, eps=1e-6, flags=0, nthreads=1):
+    """f64 (w_out, m_out) [R, C]: m's component along the row removed and
+    the row rescaled to its radius."""
+    w, ld = _rows(w, np.float32)
+    m, ldm = _rows(m, np.float32)
+    R, C = w.shape
+    if m.shape != (R, C):
+        raise ValueError("m shape")
+    wo = np.empty((R, C), np.float64)
+    mo = np.empty((R, C), np.float64)
+    _check(lib().or_renorm_momentum(_p(w), R, C, ld, _p(m), ldm, rho, eps, flags, _p(wo), _p(mo), nthreads),
+           "renorm_momentum")
+    return wo, mo
+
+
+def grad_project_row64(w, G, *, eps=1e-6, flags=0):
+    """One row with f64 inputs."""
+    w = np.ascontiguousarray(w, np.float64)
+    G = np.ascontiguousarray(G, np.float64)
+    out = np.empty_like(w)
+    lib().or_grad_project_row(_p(w), _p(G), w.size, eps, flags, _p(out))
+    return out
 
 
 def wn_forward_row64(w, g=1.0, *, rho=1.0, eps=1e-6, flags=0):

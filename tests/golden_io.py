@@ -40,3 +40,12 @@ def act_cases():
         out.append(dict(op=op, x=_vec(x), r=None if r == "-" else _vec(r), alpha=None if a == "-" else _vec(a),
                         eps=Fraction(eps), bits=[int(b, 16) for b in bits.split(",")]))
     return out
+
+
+def optim_cases():
+    """(w, eps, rho, G, projected G, renormed w) as Fractions."""
+    out = []
+    for f in read_lines("optim_exact.txt"):
+        w, eps, rho, G, P, rn = f
+        out.append(dict(w=_vec(w), eps=Fraction(eps), rho=Fraction(rho), G=_vec(G), P=_vec(P), renorm=_vec(rn)))
+    return out
