@@ -17,6 +17,14 @@ disjoint buffers (>= 268 MB of other traffic between two uses of one
 buffer), so inputs come from HBM without an explicit flush.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config step|mlp_pair|wide]
+
+`--config` selects another workload for a per-call report (default: the
+step above).  mlp_pair = up [2048,768] + down [768,2048] (fwd, bwd, renorm;
+L2-resident, so each timed step uses the next of 16 buffer copies and a
+CUDA-graph replay of the calls is timed as well).  wide = weights
+[14336,4096], [4096,14336] (fwd, bwd) and activation rows [8192,7168],
+[4096,16384] (l2, l2 + residual, slerp).
 
 Prints one JSON line (rank 0).  `value` is algorithmic bytes moved by all
 ranks per second (GB/s); per-kernel GB/s and rows/s, the roofline of the
@@ -36,6 +44,7 @@ import statistics
 import sys
 import threading
 import time
+import types
 
 import numpy as np
 
@@ -49,7 +58,13 @@ ACT_ROWS, ACT_COLS = 16384, 4096
 WORKLOAD = ("whole-model weights: 85 segments (12 layers x {q,k,v,o,gate,up,down} + tied embedding "
             "[32000,768]), 100,073,472 fp32 elements, fwd (bf16 W_eff) + bwd (bf16 GY) + renorm; "
             "activation rows [16384,4096] bf16: l2, l2 + residual, slerp")
-CALLS = ("wn_forward", "l2_rows", "wn_backward", "l2_rows_residual", "row_renorm", "slerp_rows")
+WORKLOADS = {
+    "step": WORKLOAD,
+    "mlp_pair": "MLP pair: up [2048,768] + down [768,2048] fp32 rows, one segment table, fwd (bf16 W_eff) + "
+                "bwd (bf16 GY) + renorm; 16 rotating buffer copies",
+    "wide": "wide rows: weights [14336,4096] and [4096,14336] fp32 (fwd bf16 W_eff, bwd bf16 GY), activation "
+            "rows [8192,7168] and [4096,16384] bf16 (l2, l2 + residual, slerp)",
+}
 
 
 def parse_args():
@@ -61,31 +76,63 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--config", choices=tuple(WORKLOADS), default="step")
     return p.parse_args()
 
 
 # ------------------------------------------------------------ bookkeeping --
 
-def step_bytes(weights, act_rows=ACT_ROWS, act_cols=ACT_COLS) -> dict[str, int]:
-    """Algorithmic bytes per call: every input read once, every output
+def call_bytes(kind: str, segs=None, act=None) -> int:
+    """Algorithmic bytes of one call: every input read once, every output
     written once (per-row gains and grad_g 4 B per row)."""
-    E = sum(s.w.size for s in weights)
-    R = sum(s.rows for s in weights)
-    A = act_rows * act_cols
-    return {
-        "wn_forward": E * (4 + 2) + R * 4,
-        "wn_backward": E * (4 + 2 + 4) + R * (4 + 4),
-        "row_renorm": E * (4 + 4),
-        "l2_rows": A * (2 + 2),
-        "l2_rows_residual": A * (2 + 2 + 2),
-        "slerp_rows": A * (2 + 2 + 2) + act_cols * 4,
-    }
+    if act is not None:
+        A = act.rows * act.cols
+        return {"l2": A * (2 + 2), "l2res": A * (2 + 2 + 2), "slerp": A * (2 + 2 + 2) + act.cols * 4}[kind]
+    E = sum(s.w.size for s in segs)
+    R = sum(s.rows for s in segs)
+    return {"fwd": E * (4 + 2) + R * 4, "bwd": E * (4 + 2 + 4) + R * (4 + 4), "renorm": E * (4 + 4)}[kind]
 
 
-def step_rows(weights, act_rows=ACT_ROWS) -> dict[str, int]:
-    R = sum(s.rows for s in weights)
-    return {"wn_forward": R, "wn_backward": R, "row_renorm": R,
-            "l2_rows": act_rows, "l2_rows_residual": act_rows, "slerp_rows": act_rows}
+def call_rows(kind: str, segs=None, act=None) -> int:
+    return act.rows if act is not None else sum(s.rows for s in segs)
+
+
+def step_bytes(weights, act_rows=ACT_ROWS, act_cols=ACT_COLS) -> dict[str, int]:
+    """Bytes of the six calls of the default step for these weights and
+    activation-row shape."""
+    act = types.SimpleNamespace(rows=act_rows, cols=act_cols)
+    return {"wn_forward": call_bytes("fwd", weights), "l2_rows": call_bytes("l2", act=act),
+            "wn_backward": call_bytes("bwd", weights), "l2_rows_residual": call_bytes("l2res", act=act),
+            "row_renorm": call_bytes("renorm", weights), "slerp_rows": call_bytes("slerp", act=act)}
+
+
+def plan(config: str, seed: int):
+    """(weight groups, activation groups, calls, buffer copies) of a workload.
+    A call is (name, kind, group); kinds fwd/bwd/renorm take a weight group
+    (a segment table), l2/l2res/slerp an activation group."""
+    from l2_row_b200 import workloads as wl
+
+    if config == "step":
+        wg = {"model": wl.whole_model(seed).weights}
+        ag = {"x": wl.activations(seed, ACT_ROWS, ACT_COLS).acts[0]}
+        calls = [("wn_forward", "fwd", "model"), ("l2_rows", "l2", "x"), ("wn_backward", "bwd", "model"),
+                 ("l2_rows_residual", "l2res", "x"), ("row_renorm", "renorm", "model"), ("slerp_rows", "slerp", "x")]
+        return wg, ag, calls, 1
+    if config == "mlp_pair":
+        wg = {"mlp": wl.mlp_pair(seed).weights}
+        calls = [("wn_forward", "fwd", "mlp"), ("wn_backward", "bwd", "mlp"), ("row_renorm", "renorm", "mlp")]
+        return wg, {}, calls, 16
+    if config == "wide":
+        w = wl.wide(seed)
+        wg = {s.name[2:]: [s] for s in w.weights}
+        ag = {a.name[2:]: a for a in w.acts}
+        calls = []
+        for g in wg:
+            calls += [(f"wn_forward_{g}", "fwd", g), (f"wn_backward_{g}", "bwd", g)]
+        for g in ag:
+            calls += [(f"l2_rows_{g}", "l2", g), (f"l2_rows_residual_{g}", "l2res", g), (f"slerp_rows_{g}", "slerp", g)]
+        return wg, ag, calls, 1
+    raise ValueError(config)
 
 
 def max_over_ranks(dist, values: list[float], device) -> list[float]:
@@ -201,17 +248,16 @@ class ClockSampler:
 # ------------------------------------------------------------- our arm -----
 
 class Step:
-    """Device buffers, prebuilt C segment tables and the six calls of a step."""
+    """Device buffers, prebuilt C segment tables and the calls of one step of
+    a workload (see `plan`), in `copies` independent buffer sets."""
 
-    def __init__(self, seed: int):
+    def __init__(self, seed: int, config: str = "step"):
         import torch
 
         from l2_row_b200 import ds
-        from l2_row_b200 import workloads as wl
 
         self.torch, self.ds = torch, ds
-        self.model = wl.whole_model(seed)
-        self.act = wl.activations(seed, ACT_ROWS, ACT_COLS).acts[0]
+        self.wg, self.ag, self.plan, self.copies = plan(config, seed)
         dev = "cuda"
 
         def f32(a):
@@ -220,71 +266,124 @@ class Step:
         def bf16(b):
             return torch.from_numpy(np.ascontiguousarray(b, np.uint16).view(np.int16)).to(dev).view(torch.bfloat16)
 
-        # one flat buffer per tensor kind keeps the H2D copies of the e2e leg few and large
-        segs = self.model.weights
-        n_el = sum(s.w.size for s in segs)
-        n_rows = sum(s.rows for s in segs)
-        self.w = torch.empty(n_el, dtype=torch.float32, device=dev)
-        self.gy = torch.empty(n_el, dtype=torch.bfloat16, device=dev)
-        self.gain = torch.empty(n_rows, dtype=torch.float32, device=dev)
-        self.weff = torch.empty(n_el, dtype=torch.bfloat16, device=dev)
-        self.grad_w = torch.empty(n_el, dtype=torch.float32, device=dev)
-        self.grad_g = torch.empty(n_rows, dtype=torch.float32, device=dev)
-        self.host_w = np.concatenate([s.w.ravel() for s in segs])
-        self.host_gy = np.concatenate([s.gy.ravel() for s in segs])
-        self.host_gain = np.concatenate([s.g for s in segs])
-        self.w.copy_(f32(self.host_w))
-        self.gy.copy_(bf16(self.host_gy))
-        self.gain.copy_(f32(self.host_gain))
-        fwd, bwd, ren = [], [], []
-        eo = ro = 0
-        for s in segs:
-            R, C = s.rows, s.cols
-            sl = slice(eo, eo + R * C)
-            w = self.w[sl].view(R, C)
-            gain = self.gain[ro:ro + R]
-            fwd.append(ds.WSeg(w=w, gain=gain, w_eff=self.weff[sl].view(R, C)).to_c())
-            bwd.append(ds.WSeg(w=w, gain=gain, gy=self.gy[sl].view(R, C), grad_w=self.grad_w[sl].view(R, C),
-                               grad_g=self.grad_g[ro:ro + R]).to_c())
-            ren.append(ds.WSeg(w=w).to_c())
-            eo += R * C
-            ro += R
-        self.x = bf16(self.act.x)
-        self.r = bf16(self.act.r)
-        self.alpha = f32(self.act.alpha)
-        self.y = torch.empty_like(self.x)
-        self.y2 = torch.empty_like(self.x)
-        self.h = torch.empty_like(self.x)
-        self.tables = {
-            "wn_forward": (ds.ds_wseg * len(fwd))(*fwd),
-            "wn_backward": (ds.ds_wseg * len(bwd))(*bwd),
-            "row_renorm": (ds.ds_wseg * len(ren))(*ren),
-            "l2_rows": (ds.ds_aseg * 1)(ds.ASeg(x=self.x, y=self.y).to_c()),
-            "l2_rows_residual": (ds.ds_aseg * 1)(ds.ASeg(x=self.x, r=self.r, y=self.y2).to_c()),
-            "slerp_rows": (ds.ds_aseg * 1)(ds.ASeg(x=self.x, r=self.r, y=self.h, alpha=self.alpha).to_c()),
-        }
-        self.nseg = len(segs)
+        # per weight group: one flat buffer per tensor kind (few, large H2D copies in the e2e leg)
+        self.wbuf, self.abuf = {}, {}
+        self.inputs, self.outputs = [], []   # (device tensor, host array) / device tensors of copy 0
+        for name, segs in self.wg.items():
+            host = {"w": np.concatenate([s.w.ravel() for s in segs]),
+                    "gy": np.concatenate([s.gy.ravel() for s in segs]),
+                    "gain": np.concatenate([s.g for s in segs])}
+            n_el, n_rows = host["w"].size, host["gain"].size
+            copies = []
+            for c in range(self.copies):
+                b = {"w": f32(host["w"]), "gy": bf16(host["gy"]), "gain": f32(host["gain"]),
+                     "weff": torch.empty(n_el, dtype=torch.bfloat16, device=dev),
+                     "grad_w": torch.empty(n_el, dtype=torch.float32, device=dev),
+                     "grad_g": torch.empty(n_rows, dtype=torch.float32, device=dev)}
+                copies.append(b)
+            self.wbuf[name] = copies
+            b0 = copies[0]
+            self.inputs += [(b0["w"], host["w"]), (b0["gy"], host["gy"].view(np.int16)), (b0["gain"], host["gain"])]
+            self.outputs += [b0["weff"], b0["grad_w"], b0["grad_g"], b0["w"]]
+        for name, a in self.ag.items():
+            copies = []
+            for c in range(self.copies):
+                x = bf16(a.x)
+                copies.append({"x": x, "r": bf16(a.r), "alpha": f32(a.alpha), "y": torch.empty_like(x),
+                               "y2": torch.empty_like(x), "h": torch.empty_like(x)})
+            self.abuf[name] = copies
+            b0 = copies[0]
+            self.inputs += [(b0["x"], a.x.view(np.int16)), (b0["r"], a.r.view(np.int16)), (b0["alpha"], a.alpha)]
+            self.outputs += [b0["y"], b0["y2"], b0["h"]]
+
+        self.names = [c[0] for c in self.plan]
+        self.bytes = {}
+        self.rows = {}
+        for name, kind, g in self.plan:
+            segs, act = (self.wg[g], None) if g in self.wg else (None, self.ag[g])
+            self.bytes[name] = call_bytes(kind, segs, act)
+            self.rows[name] = call_rows(kind, segs, act)
+
         lib = ds.lib()
         eps = ct.c_float(EPS)
-        t = self.tables
-        self.calls = {
-            "wn_forward": lambda s: lib.ds_wn_forward(t["wn_forward"], self.nseg, ds.DS_BF16, eps, s),
-            "l2_rows": lambda s: lib.ds_l2_rows(t["l2_rows"], 1, eps, s),
-            "wn_backward": lambda s: lib.ds_wn_backward(t["wn_backward"], self.nseg, ds.DS_BF16, eps, s),
-            "l2_rows_residual": lambda s: lib.ds_l2_rows(t["l2_rows_residual"], 1, eps, s),
-            "row_renorm": lambda s: lib.ds_row_renorm(t["row_renorm"], self.nseg, eps, s),
-            "slerp_rows": lambda s: lib.ds_slerp_rows(t["slerp_rows"], 1, eps, s),
-        }
+        self.tables = []
+        self.calls = []   # [copy][call] -> fn(stream)
+        for c in range(self.copies):
+            fns = []
+            for name, kind, g in self.plan:
+                if g in self.wg:
+                    b, segs = self.wbuf[g][c], self.wg[g]
+                    rows = []
+                    eo = ro = 0
+                    for sgm in segs:
+                        R, C = sgm.rows, sgm.cols
+                        sl = slice(eo, eo + R * C)
+                        w = b["w"][sl].view(R, C)
+                        gain = b["gain"][ro:ro + R]
+                        if kind == "fwd":
+                            rows.append(ds.WSeg(w=w, gain=gain, w_eff=b["weff"][sl].view(R, C)).to_c())
+                        elif kind == "bwd":
+                            rows.append(ds.WSeg(w=w, gain=gain, gy=b["gy"][sl].view(R, C),
+                                                grad_w=b["grad_w"][sl].view(R, C),
+                                                grad_g=b["grad_g"][ro:ro + R]).to_c())
+                        else:
+                            rows.append(ds.WSeg(w=w).to_c())
+                        eo += R * C
+                        ro += R
+                    tab = (ds.ds_wseg * len(rows))(*rows)
+                    n = len(rows)
+                    fn = {"fwd": lambda s, t=tab, n=n: lib.ds_wn_forward(t, n, ds.DS_BF16, eps, s),
+                          "bwd": lambda s, t=tab, n=n: lib.ds_wn_backward(t, n, ds.DS_BF16, eps, s),
+                          "renorm": lambda s, t=tab, n=n: lib.ds_row_renorm(t, n, eps, s)}[kind]
+                else:
+                    b = self.abuf[g][c]
+                    if kind == "l2":
+                        seg = ds.ASeg(x=b["x"], y=b["y"])
+                    elif kind == "l2res":
+                        seg = ds.ASeg(x=b["x"], r=b["r"], y=b["y2"])
+                    else:
+                        seg = ds.ASeg(x=b["x"], r=b["r"], y=b["h"], alpha=b["alpha"])
+                    tab = (ds.ds_aseg * 1)(seg.to_c())
+                    fn = (lambda s, t=tab: lib.ds_slerp_rows(t, 1, eps, s)) if kind == "slerp" else \
+                         (lambda s, t=tab: lib.ds_l2_rows(t, 1, eps, s))
+                self.tables.append(tab)
+                fns.append(fn)
+            self.calls.append(fns)
 
-    def run(self, stream_ptr: int, events=None) -> None:
-        for i, name in enumerate(CALLS):
+    def run(self, stream_ptr: int, events=None, k: int = 0) -> None:
+        fns = self.calls[k % self.copies]
+        for i, name in enumerate(self.names):
             if events is not None:
                 events[i].record()
-            st = self.calls[name](stream_ptr)
+            st = fns[i](stream_ptr)
             if st != 0:
                 raise self.ds.DSError(st, name)
         if events is not None:
-            events[len(CALLS)].record()
+            events[len(self.names)].record()
+
+
+def graph_replay_ms(step: Step, reps: int = 20) -> float:
+    """Per-step time of the calls replayed from one CUDA graph that holds one
+    step on each buffer copy (launch-bound workloads)."""
+    import torch
+
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g, stream=side):
+        for k in range(step.copies):
+            step.run(side.cuda_stream, None, k)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / (reps * step.copies)
+    del g
+    return ms
 
 
 def run_ours(args, rank: int, world: int, local_rank: int) -> None:
@@ -303,28 +402,28 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
 
     from l2_row_b200 import ds
 
-    step = Step(seed=rank)
+    step = Step(seed=rank, config=args.config)
+    names = step.names
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
-    bytes_per = step_bytes(step.model.weights)
-    rows_per = step_rows(step.model.weights)
+    bytes_per, rows_per = step.bytes, step.rows
     step_total = sum(bytes_per.values())
 
-    for _ in range(max(3, args.warmup)):
-        step.run(sp)
+    for k in range(max(3, args.warmup)):
+        step.run(sp, None, k)
     torch.cuda.synchronize()
     if ds.ds_get_device_status(sp) != ds.DS_OK:
         raise RuntimeError("device error during warm-up")
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(CALLS) + 1)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(K)]
     n0 = ds.ds_launch_count()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(torch.cuda.current_device()) as clocks:
         for k in range(K):
-            step.run(sp, evs[k])
+            step.run(sp, evs[k], k)
         torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -333,38 +432,48 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         raise RuntimeError("device error in the timed region")
 
     total_ms = evs[0][0].elapsed_time(evs[-1][-1])
-    per_call = {name: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K)] for i, name in enumerate(CALLS)}
-    t = max_over_ranks(dist, [total_ms] + [statistics.fmean(per_call[n]) for n in CALLS], "cuda")
+    per_call = {name: [evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K)] for i, name in enumerate(names)}
+    t = max_over_ranks(dist, [total_ms] + [statistics.fmean(per_call[n]) for n in names], "cuda")
     total_ms = t[0]
-    call_ms = {name: t[i + 1] for i, name in enumerate(CALLS)}
+    call_ms = {name: t[i + 1] for i, name in enumerate(names)}
 
     ms_per_step = total_ms / K
     value = whole_job_gbs(world, step_total, ms_per_step)
 
     peak, peak_src = measured_peaks()
     kernels = {}
-    for name in CALLS:
+    for name in names:
         t_s = call_ms[name] * 1e-3
         gbs = bytes_per[name] / t_s / 1e9
         kernels[name] = {"us": round(call_ms[name] * 1e3, 2), "bytes": bytes_per[name], "gb_s": round(gbs, 1),
                          "frac_of_peak": round(gbs / peak, 4), "rows_s": round(rows_per[name] / t_s, 1)}
-    fb_t = (call_ms["wn_forward"] + call_ms["wn_backward"]) * 1e-3
-    fwd_bwd = {"gb_s": round((bytes_per["wn_forward"] + bytes_per["wn_backward"]) / fb_t / 1e9, 1),
-               "rows_s": round(rows_per["wn_forward"] / fb_t, 1),
-               "frac_of_peak": round((bytes_per["wn_forward"] + bytes_per["wn_backward"]) / fb_t / 1e9 / peak, 4)}
-    dom = max(CALLS, key=lambda n: call_ms[n])
+    fwd_bwd = None
+    fw = [n for n, k, _ in step.plan if k == "fwd"]
+    bw = [n for n, k, _ in step.plan if k == "bwd"]
+    if fw and bw:
+        fb_t = sum(call_ms[n] for n in fw + bw) * 1e-3
+        fb_b = sum(bytes_per[n] for n in fw + bw)
+        fwd_bwd = {"gb_s": round(fb_b / fb_t / 1e9, 1), "rows_s": round(sum(rows_per[n] for n in fw) / fb_t, 1),
+                   "frac_of_peak": round(fb_b / fb_t / 1e9 / peak, 4)}
+    dom = max(names, key=lambda n: call_ms[n])
     ach = bytes_per[dom] / (call_ms[dom] * 1e-3) / 1e9
-    traffic = recorded_traffic(dom)
+    traffic = recorded_traffic(dom) if args.config == "step" else None
     roofline = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(ach / peak, 4), "traffic": traffic, "kernel": f"ds_{dom}",
                 "algorithmic_bytes": bytes_per[dom], "peak_source": peak_src}
+
+    graph = None
+    if step.copies > 1:
+        gms = graph_replay_ms(step)
+        graph = {"ms_per_step": round(gms, 5), "gb_s": round(step_total / (gms * 1e-3) / 1e9, 1),
+                 "calls_per_replay": step.copies * len(names)}
 
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(step, args.e2e_steps, step_total, sp, world, dist)
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "step":
         cpu = cpu_baseline(step)
 
     if dist:
@@ -372,31 +481,36 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
         dist.destroy_process_group()
     if rank != 0:
         return
+    l2_note = ("no flush: every call reads > 126 MB and consecutive calls touch disjoint buffers"
+               if step.copies == 1 else
+               f"no flush: each step uses the next of {step.copies} buffer copies "
+               f"({step.copies * step_total / 1e6:.0f} MB > 126 MB L2)")
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded, host-generated)",
-        "config": {"workload": WORKLOAD, "eps": EPS, "bytes_per_step": step_total,
-                   "l2": "no flush: every call reads > 126 MB and consecutive calls touch disjoint buffers",
+        "config": {"workload": WORKLOADS[args.config], "eps": EPS, "bytes_per_step": step_total, "l2": l2_note,
                    "parallelism": f"replicas x{world} (rows are independent; no collective)"},
         "kernels": kernels, "fwd_bwd": fwd_bwd, "roofline": roofline, "e2e": e2e, "cpu_baseline": cpu,
         "gpu_launches": launches, "clocks": clocks.summary(),
     }
+    if graph:
+        line["graph"] = graph
     print(json.dumps(line), flush=True)
 
 
 def measure_e2e(step: Step, steps: int, step_total: int, sp: int, world: int, dist) -> dict:
     """The same step through the C ABI starting from pinned host buffers:
-    every step copies its inputs host -> device, runs the six calls and
-    copies every output back."""
+    every step copies its inputs host -> device, runs the calls and copies
+    every output back."""
     import torch
 
-    pin = lambda a: torch.from_numpy(a).pin_memory()
-    h_in = [(step.w, pin(step.host_w)), (step.gy, pin(step.host_gy.view(np.int16)).view(torch.bfloat16)),
-            (step.gain, pin(step.host_gain)),
-            (step.x, pin(step.act.x.view(np.int16)).view(torch.bfloat16)),
-            (step.r, pin(step.act.r.view(np.int16)).view(torch.bfloat16)), (step.alpha, pin(step.act.alpha))]
-    outs = [step.weff, step.grad_w, step.grad_g, step.w, step.y, step.y2, step.h]
+    def pin(d, a):
+        h = torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+        return h.view(torch.bfloat16) if d.dtype == torch.bfloat16 else h
+
+    h_in = [(d, pin(d, a)) for d, a in step.inputs]
+    outs = step.outputs
     h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
     h2d = sum(d.numel() * d.element_size() for d, _ in h_in)
     d2h = sum(o.numel() * o.element_size() for o in outs)
@@ -458,15 +572,22 @@ def time_oracle_step(segs, a, nthreads: int) -> tuple[float, int]:
     return dt, sum(b.values())
 
 
-def cpu_baseline(step: Step, frac: float = 1 / 4) -> dict:
+def cpu_baseline(step: Step, min_seconds: float = 10.0, max_reps: int = 20) -> dict:
+    """The oracle on the host cores over the whole step's inputs, repeated
+    until at least `min_seconds` of work (bounded by `max_reps`)."""
     import oracle
 
     cores = oracle.default_threads()
-    segs, a = oracle_sample(step.model.weights, step.act, frac)
-    dt, nbytes = time_oracle_step(segs, a, cores)
-    return {"value": round(nbytes / dt / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"first 1/{round(1 / frac)} of every segment's rows and of the activation rows "
-                      f"({nbytes / 1e6:.0f} MB algorithmic), all six calls, {dt:.1f} s wall"}
+    segs, a = oracle_sample(step.wg["model"], step.ag["x"], 1.0)
+    total, nbytes, reps = 0.0, 0, 0
+    while reps < max_reps and (reps == 0 or total < min_seconds):
+        dt, b = time_oracle_step(segs, a, cores)
+        total += dt
+        nbytes += b
+        reps += 1
+    return {"value": round(nbytes / total / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"the whole step (all six calls on every weight segment and all activation rows, "
+                      f"{nbytes / reps / 1e6:.0f} MB algorithmic) x {reps}, {total:.1f} s wall"}
 
 
 def run_reference(args, rank: int, world: int) -> None:
@@ -480,7 +601,7 @@ def run_reference(args, rank: int, world: int) -> None:
     model = wl.whole_model(0)
     act = wl.activations(0, ACT_ROWS, ACT_COLS).acts[0]
     cores = oracle.default_threads()
-    frac = 1 / 256
+    frac = 1 / 16
     segs, a = oracle_sample(model.weights, act, frac)
     for _ in range(max(1, args.warmup)):
         time_oracle_step(segs, a, cores)
@@ -490,7 +611,7 @@ def run_reference(args, rank: int, world: int) -> None:
         total += dt
         nbytes += b
     value = nbytes / total / 1e9
-    sample = (f"first 1/256 of every segment's rows and of the activation rows per step "
+    sample = (f"first 1/16 of every segment's rows and of the activation rows per step "
               f"({nbytes / args.steps / 1e6:.1f} MB algorithmic per step)")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
