@@ -17,14 +17,15 @@ disjoint buffers (>= 268 MB of other traffic between two uses of one
 buffer), so inputs come from HBM without an explicit flush.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config step|mlp_pair|wide]
+                    [--config step|mlp_pair|wide|optimizer]
 
 `--config` selects another workload for a per-call report (default: the
 step above).  mlp_pair = up [2048,768] + down [768,2048] (fwd, bwd, renorm;
 L2-resident, so each timed step uses the next of 16 buffer copies and a
 CUDA-graph replay of the calls is timed as well).  wide = weights
 [14336,4096], [4096,14336] (fwd, bwd) and activation rows [8192,7168],
-[4096,16384] (l2, l2 + residual, slerp).
+[4096,16384] (l2, l2 + residual, slerp).  optimizer = ds_grad_project and
+ds_renorm_momentum over the whole-model weights.
 
 Prints one JSON line (rank 0).  `value` is algorithmic bytes moved by all
 ranks per second (GB/s); per-kernel GB/s and rows/s, the roofline of the
@@ -64,6 +65,9 @@ WORKLOADS = {
                 "bwd (bf16 GY) + renorm; 16 rotating buffer copies",
     "wide": "wide rows: weights [14336,4096] and [4096,14336] fp32 (fwd bf16 W_eff, bwd bf16 GY), activation "
             "rows [8192,7168] and [4096,16384] bf16 (l2, l2 + residual, slerp)",
+    "optimizer": "optimizer companions of method rescale on the whole-model weights (85 segments, 100,073,472 "
+                 "fp32 elements): gradient projection before the step, momentum projection + renorm after it "
+                 "(fp32 gradient and momentum, in place)",
 }
 
 
@@ -90,7 +94,8 @@ def call_bytes(kind: str, segs=None, act=None) -> int:
         return {"l2": A * (2 + 2), "l2res": A * (2 + 2 + 2), "slerp": A * (2 + 2 + 2) + act.cols * 4}[kind]
     E = sum(s.w.size for s in segs)
     R = sum(s.rows for s in segs)
-    return {"fwd": E * (4 + 2) + R * 4, "bwd": E * (4 + 2 + 4) + R * (4 + 4), "renorm": E * (4 + 4)}[kind]
+    return {"fwd": E * (4 + 2) + R * 4, "bwd": E * (4 + 2 + 4) + R * (4 + 4), "renorm": E * (4 + 4),
+            "project": E * (4 + 4 + 4), "momentum": E * (4 + 4 + 4 + 4)}[kind]
 
 
 def call_rows(kind: str, segs=None, act=None) -> int:
@@ -132,6 +137,10 @@ def plan(config: str, seed: int):
         for g in ag:
             calls += [(f"l2_rows_{g}", "l2", g), (f"l2_rows_residual_{g}", "l2res", g), (f"slerp_rows_{g}", "slerp", g)]
         return wg, ag, calls, 1
+    if config == "optimizer":
+        wg = {"model": wl.with_fp32_state(wl.whole_model(seed).weights, seed + 1)}
+        calls = [("grad_project", "project", "model"), ("renorm_momentum", "momentum", "model")]
+        return wg, {}, calls, 1
     raise ValueError(config)
 
 
@@ -266,25 +275,43 @@ class Step:
         def bf16(b):
             return torch.from_numpy(np.ascontiguousarray(b, np.uint16).view(np.int16)).to(dev).view(torch.bfloat16)
 
-        # per weight group: one flat buffer per tensor kind (few, large H2D copies in the e2e leg)
+        # per weight group: one flat buffer per tensor kind the plan uses
+        # (few, large H2D copies in the e2e leg)
         self.wbuf, self.abuf = {}, {}
         self.inputs, self.outputs = [], []   # (device tensor, host array) / device tensors of copy 0
         for name, segs in self.wg.items():
+            kinds = {k for _, k, g in self.plan if g == name}
+            state = bool(kinds & {"project", "momentum"})   # gy holds the fp32 gradient / momentum
             host = {"w": np.concatenate([s.w.ravel() for s in segs]),
                     "gy": np.concatenate([s.gy.ravel() for s in segs]),
                     "gain": np.concatenate([s.g for s in segs])}
             n_el, n_rows = host["w"].size, host["gain"].size
             copies = []
             for c in range(self.copies):
-                b = {"w": f32(host["w"]), "gy": bf16(host["gy"]), "gain": f32(host["gain"]),
-                     "weff": torch.empty(n_el, dtype=torch.bfloat16, device=dev),
-                     "grad_w": torch.empty(n_el, dtype=torch.float32, device=dev),
-                     "grad_g": torch.empty(n_rows, dtype=torch.float32, device=dev)}
+                b = {"w": f32(host["w"])}
+                if kinds & {"fwd", "bwd"}:
+                    b["gain"] = f32(host["gain"])
+                if "fwd" in kinds:
+                    b["weff"] = torch.empty(n_el, dtype=torch.bfloat16, device=dev)
+                if "bwd" in kinds:
+                    b["gy"] = bf16(host["gy"])
+                    b["grad_w"] = torch.empty(n_el, dtype=torch.float32, device=dev)
+                    b["grad_g"] = torch.empty(n_rows, dtype=torch.float32, device=dev)
+                if state:
+                    b["state"] = f32(host["gy"])
                 copies.append(b)
             self.wbuf[name] = copies
             b0 = copies[0]
-            self.inputs += [(b0["w"], host["w"]), (b0["gy"], host["gy"].view(np.int16)), (b0["gain"], host["gain"])]
-            self.outputs += [b0["weff"], b0["grad_w"], b0["grad_g"], b0["w"]]
+            self.inputs.append((b0["w"], host["w"]))
+            if "gain" in b0:
+                self.inputs.append((b0["gain"], host["gain"]))
+            if "gy" in b0:
+                self.inputs.append((b0["gy"], host["gy"].view(np.int16)))
+            if "state" in b0:
+                self.inputs.append((b0["state"], host["gy"]))
+            self.outputs += [b0[k] for k in ("weff", "grad_w", "grad_g", "state") if k in b0]
+            if kinds & {"renorm", "momentum"}:
+                self.outputs.append(b0["w"])
         for name, a in self.ag.items():
             copies = []
             for c in range(self.copies):
@@ -319,13 +346,15 @@ class Step:
                         R, C = sgm.rows, sgm.cols
                         sl = slice(eo, eo + R * C)
                         w = b["w"][sl].view(R, C)
-                        gain = b["gain"][ro:ro + R]
+                        gain = b["gain"][ro:ro + R] if "gain" in b else None
                         if kind == "fwd":
                             rows.append(ds.WSeg(w=w, gain=gain, w_eff=b["weff"][sl].view(R, C)).to_c())
                         elif kind == "bwd":
                             rows.append(ds.WSeg(w=w, gain=gain, gy=b["gy"][sl].view(R, C),
                                                 grad_w=b["grad_w"][sl].view(R, C),
                                                 grad_g=b["grad_g"][ro:ro + R]).to_c())
+                        elif kind in ("project", "momentum"):
+                            rows.append(ds.WSeg(w=w, grad_w=b["state"][sl].view(R, C), radius=sgm.radius).to_c())
                         else:
                             rows.append(ds.WSeg(w=w).to_c())
                         eo += R * C
@@ -334,7 +363,9 @@ class Step:
                     n = len(rows)
                     fn = {"fwd": lambda s, t=tab, n=n: lib.ds_wn_forward(t, n, ds.DS_BF16, eps, s),
                           "bwd": lambda s, t=tab, n=n: lib.ds_wn_backward(t, n, ds.DS_BF16, eps, s),
-                          "renorm": lambda s, t=tab, n=n: lib.ds_row_renorm(t, n, eps, s)}[kind]
+                          "renorm": lambda s, t=tab, n=n: lib.ds_row_renorm(t, n, eps, s),
+                          "project": lambda s, t=tab, n=n: lib.ds_grad_project(t, n, eps, s),
+                          "momentum": lambda s, t=tab, n=n: lib.ds_renorm_momentum(t, n, eps, s)}[kind]
                 else:
                     b = self.abuf[g][c]
                     if kind == "l2":

@@ -2,7 +2,7 @@
  * ds.h -- C ABI of libds: per-row L2 normalisation of weight and activation
  * rows on NVIDIA B200 (sm_100a).
  *
- * Five operations, each over a table of segments (matrices), so that every
+ * Seven operations, each over a table of segments (matrices), so that every
  * weight of a model is handled by one call:
  *
  *   ds_wn_forward   W_eff[r,:] = g_r * rho * w[r,:] / sqrt(sum_j w[r,j]^2 + eps)
@@ -17,6 +17,16 @@
  *   ds_row_renorm   w[r,:] <- rho * w[r,:] / n_r in place; DragonScale,
  *                   "Optimizer" (method "rescale": after the step each row is
  *                   rescaled back to its radius).
+ *   ds_grad_project G[r,:] <- G[r,:] - w[r,:] (w_r . G_r) / n_r^2 in place;
+ *                   DragonScale, "Optimizer" (method "rescale": before each
+ *                   step the part of each gradient that would change a row's
+ *                   length is removed).
+ *   ds_renorm_momentum  m[r,:] <- m[r,:] - w[r,:] (w_r . m_r) / n_r^2 and
+ *                   w[r,:] <- rho * w[r,:] / n_r, both in place and both from
+ *                   the row as the step left it; same section (after the step
+ *                   the same part is removed from the momentum -- Adam's
+ *                   exp_avg, SGD's or Muon's momentum_buffer -- and each row
+ *                   is rescaled back to its radius).
  *   ds_l2_rows      y = bf16(s / sqrt(sum s^2 + eps)), s = x or s = bf16(x + r);
  *                   TensorFold PR #1260, Conversation, the norms.cu commit
  *                   (tf_l2_rows: a loop's entry l2(state + input), or its exit).
@@ -78,7 +88,13 @@ typedef void *ds_stream; /* cudaStream_t */
  *   forward:  w, gain, w_eff (written), rows, cols, ld, ld_out, radius
  *   backward: w, gain, gy, grad_w (written), grad_g (written if gain != NULL),
  *             rows, cols, ld, ld_out, radius
- *   renorm:   w (read and written in place), rows, cols, ld, radius          */
+ *   renorm:   w (read and written in place), rows, cols, ld, radius
+ *   grad_project:    w (read), grad_w = the gradient G (read and written in
+ *                    place), rows, cols, ld
+ *   renorm_momentum: w (read and written in place), grad_w = the momentum
+ *                    buffer m (read and written in place), rows, cols, ld,
+ *                    radius
+ * (gain, w_eff, gy, grad_g and ld_out are ignored by the last three.)       */
 typedef struct {
     float *w;          /* fp32 [rows, ld] master rows                                */
     const float *gain; /* fp32 [rows], or NULL: mode "unit" (g = 1, no grad_g)       */
@@ -120,6 +136,19 @@ ds_status ds_wn_backward(const ds_wseg *segs, int nseg, ds_dtype gy_dtype,
 ds_status ds_row_renorm(const ds_wseg *segs, int nseg, float eps,
                         ds_stream stream);
 
+/* grad_w holds the fp32 gradient G [rows, ld]; it is overwritten with its
+ * component orthogonal to the row (at eps = 0 exactly; with eps the removed
+ * part is scaled by S/(S+eps), S = sum w^2).  w is read-only and must not
+ * overlap G. */
+ds_status ds_grad_project(const ds_wseg *segs, int nseg, float eps,
+                          ds_stream stream);
+
+/* grad_w holds the fp32 momentum m [rows, ld].  One pass per row: S = sum w^2
+ * and D = w . m from the row as the optimizer step left it, then
+ * m <- m - w D/(S+eps) and w <- rho w/sqrt(S+eps).  w and m must not overlap. */
+ds_status ds_renorm_momentum(const ds_wseg *segs, int nseg, float eps,
+                             ds_stream stream);
+
 ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps,
                      ds_stream stream);
 
@@ -150,12 +179,16 @@ typedef enum {
     DS_OP_WN_BACKWARD = 1,
     DS_OP_ROW_RENORM = 2,
     DS_OP_L2_ROWS = 3,
-    DS_OP_SLERP_ROWS = 4
+    DS_OP_SLERP_ROWS = 4,
+    DS_OP_GRAD_PROJECT = 5,
+    DS_OP_RENORM_MOMENTUM = 6
 } ds_op;
 
 typedef enum {
     DS_PATH_AUTO = 0,     /* chosen from the row length                       */
-    DS_PATH_WARP = 1,     /* one warp per row, row in registers               */
+    DS_PATH_WARP = 1,     /* staged: rows of <= 16 KB of input in shared-memory
+                             slots filled by bulk copies, one warp (weights)
+                             or a pair of warps (activations) per row         */
     DS_PATH_CTA = 2,      /* 64..256 threads of a CTA per row, in registers   */
     DS_PATH_CLUSTER = 3,  /* a cluster of 2..8 CTAs per row, DSMEM reduction  */
     DS_PATH_TWO_PASS = 4  /* a cluster streams the row twice through shared

@@ -59,7 +59,9 @@ int64_t tile_row_bytes_worst(ds_op op, int64_t cols)
     switch (op) {
     case DS_OP_WN_FORWARD:
     case DS_OP_ROW_RENORM: return q;
-    case DS_OP_WN_BACKWARD: return 2 * q;
+    case DS_OP_WN_BACKWARD:
+    case DS_OP_GRAD_PROJECT:
+    case DS_OP_RENORM_MOMENTUM: return 2 * q;
     default: return 2 * o;
     }
 }
@@ -119,6 +121,8 @@ int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r)
     case DS_OP_WN_FORWARD:
     case DS_OP_ROW_RENORM: bytes = q * 16; break;
     case DS_OP_WN_BACKWARD: bytes = q * 16 + (q * gy_esize * 4 + 15) / 16 * 16; break;
+    case DS_OP_GRAD_PROJECT:
+    case DS_OP_RENORM_MOMENTUM: bytes = 2 * q * 16; break;
     case DS_OP_L2_ROWS: bytes = o * 16 * (has_r ? 2 : 1); break;
     default: bytes = o * 32; break;
     }
@@ -344,14 +348,15 @@ ASegK aseg_rows(const ds_aseg &s, int64_t r0, int64_t nr)
     return k;
 }
 
-enum WOp { W_FWD, W_BWD, W_RENORM };
+enum WOp { W_FWD, W_BWD, W_RENORM, W_PROJECT, W_MOMENTUM };
 
 ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float eps, void *stream)
 {
     g_last_error.clear();
     if (ds_status s = check_common(nseg, segs, eps, stream))
         return s;
-    if (wop != W_RENORM && dt != DS_F32 && dt != DS_BF16)
+    const bool fwd_bwd = wop == W_FWD || wop == W_BWD;
+    if (fwd_bwd && dt != DS_F32 && dt != DS_BF16)
         return fail(DS_ERR_UNSUPPORTED_DTYPE, "dtype must be DS_F32 or DS_BF16");
     const int esize = dt == DS_BF16 ? 2 : 4;
     std::vector<Span> spans;
@@ -360,7 +365,7 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         const ds_wseg &s = segs[i];
         if (ds_status st = check_shape(s.rows, s.cols, s.ld, i))
             return st;
-        if (wop != W_RENORM && s.ld_out < s.cols)
+        if (fwd_bwd && s.ld_out < s.cols)
             return fail(DS_ERR_INVALID_ARG, where("ld_out < cols", i));
         if (!std::isfinite(s.radius))
             return fail(DS_ERR_INVALID_ARG, where("radius is not finite", i));
@@ -370,7 +375,7 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
             continue;
         if (ds_status st = check_matrix(s.w, s.rows, s.ld, 4, "w", i))
             return st;
-        if (wop != W_RENORM && s.gain && !aligned(s.gain, 4))
+        if (fwd_bwd && s.gain && !aligned(s.gain, 4))
             return fail(DS_ERR_ALIGNMENT, where("gain is not 4-byte aligned", i));
         if (wop == W_FWD) {
             if (ds_status st = check_matrix(s.w_eff, s.rows, s.ld_out, esize, "w_eff", i))
@@ -395,6 +400,14 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
                 spans.push_back(span_of(s.gain, 1, s.rows, s.rows, 4, i, 0, -1));
                 spans.push_back(span_of(s.grad_g, 1, s.rows, s.rows, 4, i, 1, -1));
             }
+        } else if (wop == W_PROJECT || wop == W_MOMENTUM) {
+            if (ds_status st = check_matrix(s.grad_w, s.rows, s.ld, 4,
+                                            wop == W_PROJECT ? "grad_w (the gradient)" : "grad_w (the momentum)", i))
+                return st;
+            // the gradient / momentum is updated in place; w is read (project)
+            // or updated in place (momentum); the two must not overlap
+            spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, wop == W_MOMENTUM ? 1 : 0, -1));
+            spans.push_back(span_of(s.grad_w, s.rows, s.cols, s.ld, 4, i, 1, -1));
         } else {
             spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 1, -1));
         }
@@ -402,7 +415,10 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
     if (ds_status st = check_overlaps(spans))
         return st;
 
-    const ds_op op = wop == W_FWD ? DS_OP_WN_FORWARD : wop == W_BWD ? DS_OP_WN_BACKWARD : DS_OP_ROW_RENORM;
+    const ds_op op = wop == W_FWD ? DS_OP_WN_FORWARD
+                   : wop == W_BWD ? DS_OP_WN_BACKWARD
+                   : wop == W_RENORM ? DS_OP_ROW_RENORM
+                   : wop == W_PROJECT ? DS_OP_GRAD_PROJECT : DS_OP_RENORM_MOMENTUM;
     const int forced = g_force_path.load(std::memory_order_relaxed);
     std::vector<RowClass> cls(static_cast<size_t>(nseg));
     for (int i = 0; i < nseg; ++i) {
@@ -414,18 +430,33 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         WSegK k = wseg_rows(segs[i], r0, nr, esize, esize);
         if (wop == W_RENORM)
             k.out = k.w ? const_cast<float *>(k.w) : nullptr;
+        if (wop == W_PROJECT || wop == W_MOMENTUM) {
+            // the kernels read the gradient / momentum as their second input
+            // (fp32, the rows' ld) and write it back in place; momentum also
+            // writes the rescaled rows over w
+            k.gy = k.grad_w;
+            k.ld_out = k.ld;
+            k.gain = nullptr;
+            k.grad_g = nullptr;
+            k.out = (wop == W_MOMENTUM && k.w) ? const_cast<float *>(k.w) : nullptr;
+        }
         return k;
     };
     const bool bf16 = dt == DS_BF16;
     auto launch = [&](const RowClass &rc, const WParams &p, int64_t units, void *st) -> int {
         if (rc.path == DS_PATH_WARP) {
-            const int tag = wop == W_FWD ? (bf16 ? 0 : 1) : wop == W_BWD ? (bf16 ? 2 : 3) : 4;
+            const int tag = wop == W_FWD ? (bf16 ? 0 : 1)
+                          : wop == W_BWD ? (bf16 ? 2 : 3)
+                          : wop == W_RENORM ? 4
+                          : wop == W_PROJECT ? 7 : 8;
             const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
             return ds::launch_tile(tag, &p, grid, ds::kTileSlotBytes, st);
         }
         switch (wop) {
         case W_FWD: return ds::launch_wn_forward(rc, p, units, bf16, st);
         case W_BWD: return ds::launch_wn_backward(rc, p, units, bf16, st);
+        case W_PROJECT: return ds::launch_grad_project(rc, p, units, st);
+        case W_MOMENTUM: return ds::launch_renorm_momentum(rc, p, units, st);
         default: return ds::launch_row_renorm(rc, p, units, st);
         }
     };
@@ -507,6 +538,16 @@ ds_status ds_row_renorm(const ds_wseg *segs, int nseg, float eps, ds_stream stre
     return run_weight(W_RENORM, segs, nseg, DS_F32, eps, stream);
 }
 
+ds_status ds_grad_project(const ds_wseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_weight(W_PROJECT, segs, nseg, DS_F32, eps, stream);
+}
+
+ds_status ds_renorm_momentum(const ds_wseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_weight(W_MOMENTUM, segs, nseg, DS_F32, eps, stream);
+}
+
 ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps, ds_stream stream)
 {
     return run_act(false, segs, nseg, eps, stream);
@@ -556,7 +597,7 @@ int ds_version(void) { return 100; }
 
 ds_status ds_row_class(ds_op op, int64_t cols, int *path, int *group_threads, int *cluster_ctas)
 {
-    if (op < DS_OP_WN_FORWARD || op > DS_OP_SLERP_ROWS)
+    if (op < DS_OP_WN_FORWARD || op > DS_OP_RENORM_MOMENTUM)
         return fail(DS_ERR_INVALID_ARG, "unknown op");
     if (cols < 1 || cols > kMaxCols)
         return fail(DS_ERR_INVALID_ARG, "cols outside [1, 2^31 - 1]");

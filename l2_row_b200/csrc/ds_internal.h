@@ -38,7 +38,11 @@ constexpr int kStages = 4;
 
 // Row length in 16-byte units: weight ops work on quads of fp32 (w is fp32),
 // activation ops on octets of bf16.
-DS_HD constexpr int elems_per_unit(ds_op op) { return op <= DS_OP_ROW_RENORM ? 4 : 8; }
+DS_HD constexpr bool is_weight_op(ds_op op)
+{
+    return op <= DS_OP_ROW_RENORM || op == DS_OP_GRAD_PROJECT || op == DS_OP_RENORM_MOMENTUM;
+}
+DS_HD constexpr int elems_per_unit(ds_op op) { return is_weight_op(op) ? 4 : 8; }
 
 struct RowClass {
     int path;    // ds_path (never DS_PATH_AUTO)
@@ -117,6 +121,8 @@ enum DeviceErrorSite : uint32_t {
 int launch_wn_forward(const RowClass &rc, const WParams &p, int64_t units, bool out_bf16, void *stream);
 int launch_wn_backward(const RowClass &rc, const WParams &p, int64_t units, bool gy_bf16, void *stream);
 int launch_row_renorm(const RowClass &rc, const WParams &p, int64_t units, void *stream);
+int launch_grad_project(const RowClass &rc, const WParams &p, int64_t units, void *stream);
+int launch_renorm_momentum(const RowClass &rc, const WParams &p, int64_t units, void *stream);
 int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_wait_selftest(uint64_t limit_ns, void *stream);

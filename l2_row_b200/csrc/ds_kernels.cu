@@ -251,7 +251,17 @@ __device__ __forceinline__ void wn_scale_row(const WSegK &sg, int64_t row, bool 
     }
 }
 
-template <int KMAX, bool GY_BF16, class Red>
+// Epilogues of the two-reduction row body (S = sum w^2, D = w . d):
+//   kModeGrad      ds_wn_backward: grad_w = (g rho / n)(d - w D/n^2), grad_g = rho D / n
+//   kModeProject   ds_grad_project: d <- d - w D/n^2 (d = the gradient, in place)
+//   kModeMomentum  ds_renorm_momentum: d <- d - w D/n^2 (d = the momentum) and
+//                  w <- rho w / n, both in place
+// With the power-of-two rescale (factor 2^m on w) the projection uses the
+// scaled row and the scaled quotient, xs * (Ds / n2s) = w * D / n^2, which
+// stays finite where the unscaled quotient D / n^2 would overflow.
+enum BwdMode { kModeGrad = 0, kModeProject = 1, kModeMomentum = 2 };
+
+template <int KMAX, bool GY_BF16, int MODE, class Red>
 __device__ __forceinline__ void wn_backward_row(const WSegK &sg, int64_t row, bool active, bool leader, int lane,
                                                 int stride, int ubeg, int uend, float eps, Red &red)
 {
@@ -301,6 +311,32 @@ __device__ __forceinline__ void wn_backward_row(const WSegK &sg, int64_t row, bo
     }
     const float n2 = acc[0] + (m == 0 ? eps : scalbnf(eps, 2 * m));
     const float inv = 1.0f / sqrtf(n2);
+    if constexpr (MODE != kModeGrad) {
+        const float qs = acc[1] / n2;          // D / (S + eps) times 2^-m
+        const float sc = sg.radius * inv;      // rho / n times 2^-m
+        if (!active)
+            return;
+        float *dd = sg.grad_w + row * sg.ld;
+        float *wo = static_cast<float *>(sg.out) + row * sg.ld;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            const int u = ubeg + lane + k * stride;
+            if (u < uend) {
+                const float4 xs = m == 0 ? x[k]
+                                         : make_float4(scalbnf(x[k].x, m), scalbnf(x[k].y, m), scalbnf(x[k].z, m),
+                                                       scalbnf(x[k].w, m));
+                float4 y;
+                y.x = fmaf(-xs.x, qs, d[k].x);
+                y.y = fmaf(-xs.y, qs, d[k].y);
+                y.z = fmaf(-xs.z, qs, d[k].z);
+                y.w = fmaf(-xs.w, qs, d[k].w);
+                store_quad<false>(dd, u, sg.cols, y);
+                if constexpr (MODE == kModeMomentum)
+                    store_quad<false>(wo, u, sg.cols, make_float4(xs.x * sc, xs.y * sc, xs.z * sc, xs.w * sc));
+            }
+        }
+        return;
+    }
     const float q = m == 0 ? acc[1] / n2 : scalbnf(acc[1] / n2, m);  // D / (S + eps)
     const float pre = (g * sg.radius) * (m == 0 ? inv : scalbnf(inv, m));
     if (!active)
@@ -448,11 +484,11 @@ __device__ __forceinline__ void slerp_row(const ASegK &sg, int64_t row, bool act
 // ================================================================ kernels ==
 
 // Operation tags: one kernel template per shape, dispatching on the tag.
-enum OpTag { kFwdBf16, kFwdF32, kBwdBf16, kBwdF32, kRenorm, kL2, kSlerp };
+enum OpTag { kFwdBf16, kFwdF32, kBwdBf16, kBwdF32, kRenorm, kL2, kSlerp, kProject, kMomentum };
 
 template <int T>
 struct IsWeight {
-    static constexpr bool value = T <= kRenorm;
+    static constexpr bool value = T <= kRenorm || T >= kProject;
 };
 
 template <int T>
@@ -460,6 +496,8 @@ struct OpOf {
     static constexpr ds_op value = (T == kFwdBf16 || T == kFwdF32) ? DS_OP_WN_FORWARD
                                  : (T == kBwdBf16 || T == kBwdF32) ? DS_OP_WN_BACKWARD
                                  : T == kRenorm ? DS_OP_ROW_RENORM
+                                 : T == kProject ? DS_OP_GRAD_PROJECT
+                                 : T == kMomentum ? DS_OP_RENORM_MOMENTUM
                                  : T == kL2 ? DS_OP_L2_ROWS : DS_OP_SLERP_ROWS;
 };
 
@@ -476,9 +514,13 @@ __device__ __forceinline__ void run_row(const P &p, int si, int64_t row, bool ac
     else if constexpr (T == kRenorm)
         wn_scale_row<K, false, true>(sg, row, active, lane, stride, ubeg, uend, p.eps, red);
     else if constexpr (T == kBwdBf16)
-        wn_backward_row<K, true>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
+        wn_backward_row<K, true, kModeGrad>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
     else if constexpr (T == kBwdF32)
-        wn_backward_row<K, false>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
+        wn_backward_row<K, false, kModeGrad>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
+    else if constexpr (T == kProject)
+        wn_backward_row<K, false, kModeProject>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
+    else if constexpr (T == kMomentum)
+        wn_backward_row<K, false, kModeMomentum>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
     else if constexpr (T == kL2)
         l2_row<K>(sg, row, active, lane, stride, ubeg, uend, p.eps, red);
     else
@@ -589,7 +631,7 @@ struct SScale {
     __device__ void finish(bool, bool) {}
 };
 
-template <bool GY_BF16>
+template <bool GY_BF16, int MODE>
 struct SBackward {
     static constexpr int kPasses = 2;
     static constexpr int kArrays = 2;
@@ -597,7 +639,8 @@ struct SBackward {
     int64_t row;
     float eps;
     float acc[2] = {0.f, 0.f};
-    float pre = 0.f, q = 0.f, gg = 0.f;
+    float pre = 0.f, q = 0.f, gg = 0.f, sc = 0.f;
+    int msh = 0; // power-of-two rescale of w (projection modes)
 
     __device__ SBackward(const WSegK &s, int64_t r, float e) : sg(s), row(r), eps(e) {}
     __device__ int unit_bytes(int a) const { return a == 0 ? 16 : (GY_BF16 ? 8 : 16); }
@@ -627,12 +670,26 @@ struct SBackward {
             acc_sq4(acc[0], x);
             acc_dot4(acc[1], x, d);
         } else if (store) {
-            float4 y;
-            y.x = pre * fmaf(-x.x, q, d.x);
-            y.y = pre * fmaf(-x.y, q, d.y);
-            y.z = pre * fmaf(-x.z, q, d.z);
-            y.w = pre * fmaf(-x.w, q, d.w);
-            store_quad<false>(sg.grad_w + row * sg.ld, u, c.cols, y);
+            if constexpr (MODE == kModeGrad) {
+                float4 y;
+                y.x = pre * fmaf(-x.x, q, d.x);
+                y.y = pre * fmaf(-x.y, q, d.y);
+                y.z = pre * fmaf(-x.z, q, d.z);
+                y.w = pre * fmaf(-x.w, q, d.w);
+                store_quad<false>(sg.grad_w + row * sg.ld, u, c.cols, y);
+            } else {
+                if (msh != 0)
+                    x = make_float4(scalbnf(x.x, msh), scalbnf(x.y, msh), scalbnf(x.z, msh), scalbnf(x.w, msh));
+                float4 y;
+                y.x = fmaf(-x.x, q, d.x);
+                y.y = fmaf(-x.y, q, d.y);
+                y.z = fmaf(-x.z, q, d.z);
+                y.w = fmaf(-x.w, q, d.w);
+                store_quad<false>(sg.grad_w + row * sg.ld, u, c.cols, y);
+                if constexpr (MODE == kModeMomentum)
+                    store_quad<false>(static_cast<float *>(sg.out) + row * sg.ld, u, c.cols,
+                                      make_float4(x.x * sc, x.y * sc, x.z * sc, x.w * sc));
+            }
         }
     }
 
@@ -665,9 +722,15 @@ struct SBackward {
                 acc[1] = a2[1];
             }
         }
-        const float g = sg.gain ? __ldg(sg.gain + row) : 1.f;
         const float n2 = acc[0] + (m == 0 ? eps : scalbnf(eps, 2 * m));
         const float inv = 1.0f / sqrtf(n2);
+        if constexpr (MODE != kModeGrad) {
+            msh = m;
+            q = acc[1] / n2;        // times 2^-m; applied to the scaled row
+            sc = sg.radius * inv;   // rho / n times 2^-m
+            return;
+        }
+        const float g = sg.gain ? __ldg(sg.gain + row) : 1.f;
         q = m == 0 ? acc[1] / n2 : scalbnf(acc[1] / n2, m);
         pre = (g * sg.radius) * (m == 0 ? inv : scalbnf(inv, m));
         gg = sg.radius * acc[1] * inv;
@@ -675,7 +738,7 @@ struct SBackward {
 
     __device__ void finish(bool leader, bool store)
     {
-        if (leader && store && sg.gain)
+        if (MODE == kModeGrad && leader && store && sg.gain)
             sg.grad_g[row] = gg;
     }
 };
@@ -824,8 +887,10 @@ struct StreamOp;
 template <> struct StreamOp<kFwdBf16> { using type = SScale<true, false>; };
 template <> struct StreamOp<kFwdF32> { using type = SScale<false, false>; };
 template <> struct StreamOp<kRenorm> { using type = SScale<false, true>; };
-template <> struct StreamOp<kBwdBf16> { using type = SBackward<true>; };
-template <> struct StreamOp<kBwdF32> { using type = SBackward<false>; };
+template <> struct StreamOp<kBwdBf16> { using type = SBackward<true, kModeGrad>; };
+template <> struct StreamOp<kBwdF32> { using type = SBackward<false, kModeGrad>; };
+template <> struct StreamOp<kProject> { using type = SBackward<false, kModeProject>; };
+template <> struct StreamOp<kMomentum> { using type = SBackward<false, kModeMomentum>; };
 template <> struct StreamOp<kL2> { using type = SL2; };
 template <> struct StreamOp<kSlerp> { using type = SSlerp; };
 
@@ -833,7 +898,7 @@ template <int T>
 constexpr int stream_stage_bytes()
 {
     // widest layout of the operation's arrays per stage
-    return T == kBwdF32 ? 2 * 16 * kChunkUnits
+    return (T == kBwdF32 || T == kProject || T == kMomentum) ? 2 * 16 * kChunkUnits
          : T == kBwdBf16 ? (16 + 8) * kChunkUnits
          : (T == kL2 || T == kSlerp) ? 2 * 16 * kChunkUnits
          : 16 * kChunkUnits;
@@ -1025,6 +1090,16 @@ int launch_wn_backward(const RowClass &rc, const WParams &p, int64_t units, bool
 int launch_row_renorm(const RowClass &rc, const WParams &p, int64_t units, void *stream)
 {
     return launch_op<kRenorm>(rc, p, units, stream);
+}
+
+int launch_grad_project(const RowClass &rc, const WParams &p, int64_t units, void *stream)
+{
+    return launch_op<kProject>(rc, p, units, stream);
+}
+
+int launch_renorm_momentum(const RowClass &rc, const WParams &p, int64_t units, void *stream)
+{
+    return launch_op<kMomentum>(rc, p, units, stream);
 }
 
 int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream)

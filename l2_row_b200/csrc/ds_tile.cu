@@ -24,7 +24,9 @@
 namespace ds {
 
 // ds_kernels.cu's tags, repeated (the two files share this numbering).
-enum TileTag { tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp };
+enum TileTag { tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp, tProject, tMomentum };
+
+__host__ __device__ constexpr bool is_weight_tag(int T) { return T <= tRenorm || T >= tProject; }
 
 namespace {
 
@@ -343,7 +345,13 @@ __device__ __forceinline__ float4 gy_unit(const unsigned char *s1, int u)
     }
 }
 
-template <bool GY_BF16>
+// Epilogues of the two-reduction row (S = sum w^2, D = w . d; d staged as
+// array 1): MODE 0 = ds_wn_backward (grad_w, grad_g), 1 = ds_grad_project
+// (d <- d - w D/n^2 in place), 2 = ds_renorm_momentum (the same on the
+// momentum, and w <- rho w / n in place).  With the power-of-two rescale the
+// projection applies the scaled quotient to the scaled row, which stays
+// finite where D/n^2 alone would overflow.
+template <bool GY_BF16, int MODE>
 __device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, float g, const unsigned char *s0,
                                                   const unsigned char *s1, int lane, int nfull, int tail,
                                                   float eps, bool store)
@@ -403,6 +411,40 @@ __device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, 
         return;
     const float n2 = S + (m == 0 ? eps : scalbnf(eps, 2 * m));
     const float inv = 1.0f / sqrtf(n2);
+    if constexpr (MODE != 0) {
+        const float2 nqs = f2(-D / n2, -D / n2);      // -D/(S+eps) times 2^-m
+        const float sc = sg.radius * inv;             // rho / n times 2^-m
+        const float2 sc2 = f2(sc, sc);
+        float *dd = sg.grad_w + row * sg.ld;
+        float *wo = static_cast<float *>(sg.out) + row * sg.ld;
+        auto scaled = [&](float4 x) {
+            return m == 0 ? x : make_float4(scalbnf(x.x, m), scalbnf(x.y, m), scalbnf(x.z, m), scalbnf(x.w, m));
+        };
+#pragma unroll 4
+        for (int u = lane; u < nfull; u += 32) {
+            const float4 x = scaled(w[u]);
+            const float4 d = gy_unit<GY_BF16>(s1, u);
+            const float2 a = __ffma2_rn(f2(x.x, x.y), nqs, f2(d.x, d.y));
+            const float2 b = __ffma2_rn(f2(x.z, x.w), nqs, f2(d.z, d.w));
+            st16(dd + 4 * u, make_uint4(__float_as_uint(a.x), __float_as_uint(a.y), __float_as_uint(b.x),
+                                        __float_as_uint(b.y)));
+            if constexpr (MODE == 2) {
+                const float2 p = __fmul2_rn(f2(x.x, x.y), sc2), q = __fmul2_rn(f2(x.z, x.w), sc2);
+                st16(wo + 4 * u, make_uint4(__float_as_uint(p.x), __float_as_uint(p.y), __float_as_uint(q.x),
+                                            __float_as_uint(q.y)));
+            }
+        }
+        if (tl) {
+            const float4 x = scaled(xt);
+            const float e[3] = {x.x, x.y, x.z}, dv[3] = {dt.x, dt.y, dt.z};
+            for (int i = 0; i < tail; ++i) {
+                dd[4 * nfull + i] = fmaf(e[i], nqs.x, dv[i]);
+                if constexpr (MODE == 2)
+                    wo[4 * nfull + i] = e[i] * sc;
+            }
+        }
+        return;
+    }
     const float q = m == 0 ? D / n2 : scalbnf(D / n2, m);
     const float pre = (g * sg.radius) * (m == 0 ? inv : scalbnf(inv, m));
     if (lane == 0 && sg.gain)
@@ -690,7 +732,7 @@ __device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, in
 // =============================================================== kernel ==
 
 template <int T>
-using TParams = typename std::conditional<(T <= tRenorm), WParams, AParams>::type;
+using TParams = typename std::conditional<is_weight_tag(T), WParams, AParams>::type;
 
 // Ring shape per operation: 13 ring positions of 16 KB.  The weight calls
 // give each position one consumer warp.  The activation calls, one 16 KB
@@ -844,7 +886,7 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
             const int pitch0 = (sg.nu * u0 + 15) & ~15;
             const int pitch1 = (sg.nu * u1 + 15) & ~15;
             unsigned char *a1 = base + pitch0 * rps;
-            constexpr int E = (T <= tRenorm) ? 4 : 8;
+            constexpr int E = is_weight_tag(T) ? 4 : 8;
             const int nfull = sg.cols / E, tail = sg.cols % E;
             // hand the position back: the slot may hold this warp's
             // generic-proxy writes (s, t, masked tails), so order them
@@ -875,9 +917,13 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
                 else if constexpr (T == tRenorm)
                     tile_scale_row<false, true>(sg, row, 1.f, s0, lane, nfull, tail, p.eps, store);
                 else if constexpr (T == tBwdBf16)
-                    tile_backward_row<true>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, store);
+                    tile_backward_row<true, 0>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, store);
                 else if constexpr (T == tBwdF32)
-                    tile_backward_row<false>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, store);
+                    tile_backward_row<false, 0>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, store);
+                else if constexpr (T == tProject)
+                    tile_backward_row<false, 1>(sg, row, 1.f, s0, s1, lane, nfull, tail, p.eps, store);
+                else if constexpr (T == tMomentum)
+                    tile_backward_row<false, 2>(sg, row, 1.f, s0, s1, lane, nfull, tail, p.eps, store);
                 else if constexpr (T == tL2) {
                     if (has_r)
                         tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
@@ -924,6 +970,8 @@ int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *str
     case tRenorm: return launch_tile_t<tRenorm>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
     case tL2: return launch_tile_t<tL2>(*static_cast<const AParams *>(params), grid, slot_bytes, stream);
     case tSlerp: return launch_tile_t<tSlerp>(*static_cast<const AParams *>(params), grid, slot_bytes, stream);
+    case tProject: return launch_tile_t<tProject>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
+    case tMomentum: return launch_tile_t<tMomentum>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
     default: return cudaErrorInvalidValue;
     }
 }

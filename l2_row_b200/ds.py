@@ -9,6 +9,8 @@ The five calls keep their C names and take lists of segments:
     ds_wn_forward(segs, out_dtype, eps, stream=None)
     ds_wn_backward(segs, gy_dtype, eps, stream=None)
     ds_row_renorm(segs, eps, stream=None)
+    ds_grad_project(segs, eps, stream=None)       (grad_w = the gradient, in place)
+    ds_renorm_momentum(segs, eps, stream=None)    (grad_w = the momentum, in place)
     ds_l2_rows(segs, eps, stream=None)
     ds_slerp_rows(segs, eps, stream=None)
 
@@ -36,6 +38,7 @@ DS_OK, DS_ERR_INVALID_ARG, DS_ERR_ALIGNMENT, DS_ERR_UNSUPPORTED_DTYPE = 0, 1, 2,
 DS_ERR_TOO_MANY_SEGMENTS, DS_ERR_CUDA, DS_ERR_DEVICE_TIMEOUT, DS_ERR_OVERLAP = 4, 5, 6, 7
 DS_F32, DS_BF16 = 0, 1
 DS_OP_WN_FORWARD, DS_OP_WN_BACKWARD, DS_OP_ROW_RENORM, DS_OP_L2_ROWS, DS_OP_SLERP_ROWS = range(5)
+DS_OP_GRAD_PROJECT, DS_OP_RENORM_MOMENTUM = 5, 6
 DS_PATH_AUTO, DS_PATH_WARP, DS_PATH_CTA, DS_PATH_CLUSTER, DS_PATH_TWO_PASS = range(5)
 DS_MAX_SEGMENTS = 65536
 PATH_NAMES = {DS_PATH_WARP: "warp", DS_PATH_CTA: "cta", DS_PATH_CLUSTER: "cluster", DS_PATH_TWO_PASS: "two_pass"}
@@ -56,9 +59,12 @@ _st = ct.c_int
 _lib.ds_wn_forward.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_wn_backward.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_row_renorm.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_grad_project.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_renorm_momentum.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_l2_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_slerp_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_void_p]
-for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_l2_rows", "ds_slerp_rows",
+for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
+           "ds_l2_rows", "ds_slerp_rows",
            "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
            "ds_debug_wait_timeout_selftest"):
     getattr(_lib, _f).restype = _st
@@ -78,7 +84,8 @@ _lib.ds_debug_set_wait_limit_ns.argtypes = [ct.c_uint64]
 _lib.ds_debug_wait_timeout_selftest.argtypes = [ct.c_uint64, ct.c_void_p]
 
 #: every symbol include/ds.h declares
-EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_l2_rows", "ds_slerp_rows",
+EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
+           "ds_l2_rows", "ds_slerp_rows",
            "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
            "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest")
 
@@ -150,7 +157,9 @@ def _vec(t) -> int:
 @dataclass
 class WSeg:
     """One weight matrix.  w: fp32 [R, C]; gain: fp32 [R] or None; w_eff:
-    forward output [R, C]; gy, grad_w, grad_g: backward input/outputs."""
+    forward output [R, C]; gy, grad_w, grad_g: backward input/outputs.
+    For ds_grad_project grad_w is the gradient and for ds_renorm_momentum
+    the momentum buffer (fp32 [R, C], w's leading dimension, in place)."""
 
     w: Any
     gain: Any = None
@@ -213,6 +222,16 @@ def ds_wn_backward(segs: Sequence, gy_dtype="bf16", eps: float = 1e-6, stream=No
 def ds_row_renorm(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
     arr, n = _table(segs, ds_wseg)
     _check(_lib.ds_row_renorm(arr, n, eps, _stream_ptr(stream)), "ds_row_renorm")
+
+
+def ds_grad_project(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_wseg)
+    _check(_lib.ds_grad_project(arr, n, eps, _stream_ptr(stream)), "ds_grad_project")
+
+
+def ds_renorm_momentum(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_wseg)
+    _check(_lib.ds_renorm_momentum(arr, n, eps, _stream_ptr(stream)), "ds_renorm_momentum")
 
 
 def ds_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:

@@ -208,6 +208,15 @@ def long_rows(seed: int = 0, w_rows: int = 6, w_cols: int = 131072,
     return Workload("long_rows", 1e-6, [seg], [act])
 
 
+def with_fp32_state(weights: list[WeightSeg], seed: int, std: float = 1e-3) -> list[WeightSeg]:
+    """The same weight rows, each paired with an fp32 [rows, cols] N(0, std)
+    tensor in `gy`: the gradient G (before the optimizer step) or the
+    momentum m (after it) of method "rescale".  Drawn in segment order."""
+    rng = _rng(seed)
+    return [WeightSeg(s.name, s.w, s.g, (rng.standard_normal(s.w.shape, dtype=np.float32) * np.float32(std)),
+                      s.radius) for s in weights]
+
+
 def small_norm_rows(seed: int, rows: int, cols: int, sumsq: float = 1e-5) -> np.ndarray:
     """bf16 rows with sum of squares near `sumsq` (eps-sensitive control set)."""
     rng = _rng(seed)

@@ -105,6 +105,30 @@ def run_renorm(segs, eps: float):
     return ws
 
 
+def run_project(segs, eps: float):
+    """ds_grad_project with seg.gy (fp32) as the gradient; returns the updated G tensors."""
+    gs, cs = [], []
+    for s in segs:
+        G = dev_f32(s.gy)
+        cs.append(ds.WSeg(w=dev_f32(s.w), grad_w=G))
+        gs.append(G)
+    ds.ds_grad_project(cs, eps)
+    torch.cuda.synchronize()
+    return gs
+
+
+def run_momentum(segs, eps: float):
+    """ds_renorm_momentum with seg.gy (fp32) as the momentum; returns (w, m) tensors."""
+    res, cs = [], []
+    for s in segs:
+        w, m = dev_f32(s.w), dev_f32(s.gy)
+        cs.append(ds.WSeg(w=w, grad_w=m, radius=s.radius))
+        res.append((w, m))
+    ds.ds_renorm_momentum(cs, eps)
+    torch.cuda.synchronize()
+    return res
+
+
 def run_l2(acts, eps: float, residual: bool = True):
     ys, cs = [], []
     for a in acts:
@@ -190,6 +214,35 @@ def check_renorm(seg, got: torch.Tensor, eps: float, rows=None, what="row_renorm
     got_h = host_f32(got if rows is None else got[torch.as_tensor(rows, device=got.device)])
     bad = rel_violations(got_h, ref, 2e-6)
     assert not bad.any(), f"{what}: {int(bad.sum())} fp32 outputs beyond 2e-6 relative"
+
+
+def _proj_check(got, ref, d, what):
+    """The projection's tolerance: 1e-5 relative with a floor of the row's
+    RMS of the input (the subtraction d - w D/n^2 can cancel)."""
+    d64 = d.astype(np.float64)
+    floor = np.sqrt(np.mean(d64 ** 2, axis=1))[:, None]
+    bad = rel_violations(got, ref, 1e-5, floor)
+    assert not bad.any(), f"{what}: {int(bad.sum())} entries beyond tolerance (first at {np.argwhere(bad)[0].tolist()})"
+
+
+def check_project(seg, got: torch.Tensor, eps: float, rows=None, what="grad_project", flags=0):
+    sel = slice(None) if rows is None else rows
+    w, G = seg.w[sel], seg.gy[sel]
+    ref = oracle.grad_project(w, G, eps=eps, flags=flags, nthreads=oracle.default_threads())
+    got_h = host_f32(got if rows is None else got[torch.as_tensor(rows, device=got.device)])
+    _proj_check(got_h, ref, G, what)
+
+
+def check_momentum(seg, got_w: torch.Tensor, got_m: torch.Tensor, eps: float, rows=None, what="renorm_momentum"):
+    sel = slice(None) if rows is None else rows
+    w, m = seg.w[sel], seg.gy[sel]
+    ref_w, ref_m = oracle.renorm_momentum(w, m, rho=seg.radius, eps=eps, nthreads=oracle.default_threads())
+    idx = None if rows is None else torch.as_tensor(rows, device=got_w.device)
+    gw = host_f32(got_w if idx is None else got_w[idx])
+    gm = host_f32(got_m if idx is None else got_m[idx])
+    bad = rel_violations(gw, ref_w, 2e-6)
+    assert not bad.any(), f"{what}: {int(bad.sum())} renormed entries beyond 2e-6 relative"
+    _proj_check(gm, ref_m, m, what + " (momentum)")
 
 
 def check_l2(act, got: torch.Tensor, eps: float, residual=True, rows=None, what="l2_rows", flags=0):

@@ -36,7 +36,8 @@ def test_status_strings_and_version():
 
 # ------------------------------------------------------------- row classes --
 
-W_OPS = (ds.DS_OP_WN_FORWARD, ds.DS_OP_WN_BACKWARD, ds.DS_OP_ROW_RENORM)
+W_OPS = (ds.DS_OP_WN_FORWARD, ds.DS_OP_WN_BACKWARD, ds.DS_OP_ROW_RENORM, ds.DS_OP_GRAD_PROJECT,
+         ds.DS_OP_RENORM_MOMENTUM)
 A_OPS = (ds.DS_OP_L2_ROWS, ds.DS_OP_SLERP_ROWS)
 
 
@@ -53,6 +54,10 @@ A_OPS = (ds.DS_OP_L2_ROWS, ds.DS_OP_SLERP_ROWS)
     (ds.DS_OP_WN_FORWARD, 14336, (ds.DS_PATH_CLUSTER, 0, 2)),
     (ds.DS_OP_WN_BACKWARD, 14336, (ds.DS_PATH_CLUSTER, 0, 4)),
     (ds.DS_OP_WN_FORWARD, 131072, (ds.DS_PATH_TWO_PASS, 0, 8)),
+    (ds.DS_OP_GRAD_PROJECT, 2048, (ds.DS_PATH_WARP, 32, 1)),  # w + G fp32 = 16 KB
+    (ds.DS_OP_RENORM_MOMENTUM, 2049, (ds.DS_PATH_CTA, 256, 1)),
+    (ds.DS_OP_GRAD_PROJECT, 14336, (ds.DS_PATH_CLUSTER, 0, 4)),
+    (ds.DS_OP_RENORM_MOMENTUM, 65537, (ds.DS_PATH_TWO_PASS, 0, 8)),
     (ds.DS_OP_SLERP_ROWS, 262144, (ds.DS_PATH_TWO_PASS, 0, 8)),
 ])
 def test_row_class_for_workload_shapes(op, cols, want):
@@ -116,9 +121,12 @@ def aseg(**kw):
     return ds.ds_aseg(**d)
 
 
+NO_DTYPE = ("ds_row_renorm", "ds_grad_project", "ds_renorm_momentum")
+
+
 def call_w(fn, segs, dt=ds.DS_BF16, eps=1e-6):
     arr = (ds.ds_wseg * max(1, len(segs)))(*segs)
-    if fn == "ds_row_renorm":
+    if fn in NO_DTYPE:
         return getattr(ds.lib(), fn)(arr, len(segs), ct.c_float(eps), None)
     return getattr(ds.lib(), fn)(arr, len(segs), dt, ct.c_float(eps), None)
 
@@ -128,7 +136,8 @@ def call_a(fn, segs, eps=1e-6):
     return getattr(ds.lib(), fn)(arr, len(segs), ct.c_float(eps), None)
 
 
-@pytest.mark.parametrize("fn", ["ds_wn_forward", "ds_wn_backward", "ds_row_renorm"])
+@pytest.mark.parametrize("fn", ["ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project",
+                                "ds_renorm_momentum"])
 def test_weight_validation(fn):
     E = ds
     before = ds.ds_launch_count()
@@ -143,7 +152,7 @@ def test_weight_validation(fn):
     assert call_w(fn, [wseg()], eps=float("inf")) == E.DS_ERR_INVALID_ARG
     assert call_w(fn, [wseg(radius=float("nan"))]) == E.DS_ERR_INVALID_ARG
     arr = (ds.ds_wseg * 1)(wseg())
-    if fn == "ds_row_renorm":
+    if fn in NO_DTYPE:
         assert getattr(ds.lib(), fn)(None, 1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
         assert getattr(ds.lib(), fn)(arr, -1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
         assert getattr(ds.lib(), fn)(arr, E.DS_MAX_SEGMENTS + 1, ct.c_float(1e-6), None) == \
@@ -170,6 +179,23 @@ def test_weight_specific_validation():
     # bf16 W_eff rows need ld_out % 8 == 0; fp32 rows need ld_out % 4 == 0
     assert call_w("ds_wn_forward", [wseg(ld_out=12, ld=12)]) == E.DS_ERR_ALIGNMENT
     assert ds.ds_last_error().startswith("segment 0")
+
+
+def test_optimizer_call_validation():
+    E = ds
+    for fn in ("ds_grad_project", "ds_renorm_momentum"):
+        # grad_w holds the gradient / momentum: required, aligned, w's ld
+        assert call_w(fn, [wseg(grad_w=0)]) == E.DS_ERR_INVALID_ARG
+        assert call_w(fn, [wseg(grad_w=BASE + (3 << 30) + 4)]) == E.DS_ERR_ALIGNMENT
+        # gy, w_eff, gain, ld_out are not read: their values do not matter
+        before = ds.ds_launch_count()
+        assert call_w(fn, [wseg(gy=0, w_eff=0, ld_out=0, rows=0)]) == E.DS_OK
+        assert ds.ds_launch_count() == before
+        # the buffer must not overlap w (it is updated in place)
+        assert call_w(fn, [wseg(grad_w=BASE)]) == E.DS_ERR_OVERLAP
+        assert call_w(fn, [wseg(grad_w=BASE + 64)]) == E.DS_ERR_OVERLAP
+        # two segments updating the same gradient rows
+        assert call_w(fn, [wseg(), wseg(w=BASE + (8 << 30))]) == E.DS_ERR_OVERLAP
 
 
 def test_weight_overlap_rejected():
