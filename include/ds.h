@@ -186,17 +186,20 @@ typedef enum {
 
 typedef enum {
     DS_PATH_AUTO = 0,     /* chosen from the row length                       */
-    DS_PATH_WARP = 1,     /* staged: rows of <= 16 KB of input in shared-memory
-                             slots filled by bulk copies, one warp (weights)
-                             or a pair of warps (activations) per row         */
-    DS_PATH_CTA = 2,      /* 64..256 threads of a CTA per row, in registers   */
-    DS_PATH_CLUSTER = 3,  /* a cluster of 2..8 CTAs per row, DSMEM reduction  */
+    DS_PATH_WARP = 1,     /* staged: rows of <= 16 KB of input in a ring of
+                             shared-memory slots filled by bulk copies; one
+                             warp (weights) or two (activations) per row      */
+    DS_PATH_CTA = 2,      /* staged in 32 or 64 KB slots: a team of 2..8 warps
+                             per row (rows of <= 64 KB of input)              */
+    DS_PATH_CLUSTER = 3,  /* a cluster of 2..8 CTAs per row, row slices in
+                             registers, DSMEM reduction                       */
     DS_PATH_TWO_PASS = 4  /* a cluster streams the row twice through shared
                              memory with bulk (TMA) copies                    */
 } ds_path;
 
 /* The row class a call would use for rows of `cols` elements: path, threads
- * per row inside a CTA (warp/CTA paths) and CTAs per row (cluster/two-pass).
+ * per row (the staged paths' team; 0 on cluster paths) and CTAs per row
+ * (cluster/two-pass; 1 otherwise).
  * Depends on (op, cols) and the forced path only -- never on the row count. */
 ds_status ds_row_class(ds_op op, int64_t cols, int *path, int *group_threads,
                        int *cluster_ctas);

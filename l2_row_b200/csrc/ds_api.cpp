@@ -66,17 +66,24 @@ int64_t tile_row_bytes_worst(ds_op op, int64_t cols)
     }
 }
 
+// Warps of a staged team: one (weights) or two (activations) per 16 KB of slot.
+int team_warps(ds_op op, int slot)
+{
+    const int base = (op == DS_OP_L2_ROWS || op == DS_OP_SLERP_ROWS) ? 2 : 1;
+    return base * slot / ds::kTileSlotBytes;
+}
+
 RowClass classify(ds_op op, int64_t cols, int forced)
 {
     const int64_t E = ds::elems_per_unit(op);
     const int64_t nu = (cols + E - 1) / E;
     const int64_t kmax = ds::kmax_of(op);
-    const bool tile = tile_row_bytes_worst(op, cols) <= ds::kTileSlotBytes;
-    auto group_of = [&]() -> int {
-        for (int G = 64; G <= ds::kCta; G *= 2)
-            if ((nu + G - 1) / G <= kmax)
-                return G;
-        return 0;
+    const int64_t staged = tile_row_bytes_worst(op, cols);
+    auto staged_class = [&](int path, int min_slot) -> RowClass {
+        for (int slot = min_slot; slot <= ds::kTileSlotMaxBytes; slot *= 2)
+            if (staged <= slot)
+                return {path, 32 * team_warps(op, slot), 1, 0, slot};
+        return {0, 0, 0, 0, 0};
     };
     auto cluster_of = [&]() -> int {
         for (int CL = 2; CL <= ds::kMaxCluster; CL *= 2)
@@ -86,34 +93,34 @@ RowClass classify(ds_op op, int64_t cols, int forced)
     };
     switch (forced) {
     case DS_PATH_WARP:
-        if (tile)
-            return {DS_PATH_WARP, 32, 1, 0};
+        if (staged <= ds::kTileSlotBytes)
+            return staged_class(DS_PATH_WARP, ds::kTileSlotBytes);
         break;
     case DS_PATH_CTA:
-        if (const int G = group_of())
-            return {DS_PATH_CTA, G, 1, 0};
+        if (staged <= ds::kTileSlotMaxBytes)
+            return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
         break;
     case DS_PATH_CLUSTER:
         if (const int CL = cluster_of())
-            return {DS_PATH_CLUSTER, 0, CL, 0};
+            return {DS_PATH_CLUSTER, 0, CL, 0, 0};
         break;
     case DS_PATH_TWO_PASS:
-        return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0};
+        return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0, 0};
     default:
         break;
     }
-    if (tile)
-        return {DS_PATH_WARP, 32, 1, 0};
-    if (const int G = group_of())
-        return {DS_PATH_CTA, G, 1, 0};
+    if (staged <= ds::kTileSlotBytes)
+        return staged_class(DS_PATH_WARP, ds::kTileSlotBytes);
+    if (staged <= ds::kTileSlotMaxBytes)
+        return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
     if (const int CL = cluster_of())
-        return {DS_PATH_CLUSTER, 0, CL, 0};
-    return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0};
+        return {DS_PATH_CLUSTER, 0, CL, 0, 0};
+    return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0, 0};
 }
 
-// Rows per shared-memory slot on the warp-per-row path for the actual
-// layout (staged arrays of this segment), at most kTileMaxRowsPerSlot.
-int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r)
+// Rows per shared-memory slot of `slot` bytes on the staged paths for the
+// actual layout (staged arrays of this segment), at most kTileMaxRowsPerSlot.
+int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r, int slot)
 {
     const int64_t q = (cols + 3) / 4, o = (cols + 7) / 8;
     int64_t bytes = 0;
@@ -126,7 +133,7 @@ int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r)
     case DS_OP_L2_ROWS: bytes = o * 16 * (has_r ? 2 : 1); break;
     default: bytes = o * 32; break;
     }
-    return static_cast<int>(std::min<int64_t>(ds::kTileMaxRowsPerSlot, ds::kTileSlotBytes / bytes));
+    return static_cast<int>(std::min<int64_t>(ds::kTileMaxRowsPerSlot, slot / bytes));
 }
 
 int sm_count()
@@ -144,15 +151,11 @@ int sm_count()
     return cache[dev];
 }
 
-// Rows per work unit: a shared-memory slot (warp-per-row path), a CTA
-// (register group path), or one row (a cluster per row).
+// Rows per work unit: a shared-memory slot (staged paths) or one row (a
+// cluster per row).
 int64_t rows_per_unit(const RowClass &rc)
 {
-    if (rc.path == DS_PATH_WARP)
-        return rc.rps;
-    if (rc.path == DS_PATH_CTA)
-        return ds::kCta / rc.group;
-    return 1;
+    return ds::is_staged(rc) ? rc.rps : 1;
 }
 
 int64_t units_for(const RowClass &rc, int64_t rows)
@@ -239,13 +242,14 @@ ds_status check_matrix(const void *p, int64_t rows, int64_t ld, int esize, const
 // Splits, packs and launches.  `make(i, r0, nrows)` returns the device
 // segment for rows [r0, r0 + nrows) of segment i.
 // Slerp launches whose segments all use one alpha vector of at most
-// kTileAlphaCache columns let the staged kernel keep |alpha| in shared memory.
+// kTileAlphaCacheMax columns let the staged kernel keep |alpha| in shared
+// memory (the kernel checks the length against its own cache).
 inline void shared_alpha(WParams &p, int) { p.alpha_shared = nullptr; p.alpha_cols = 0; }
 inline void shared_alpha(AParams &p, int n)
 {
     p.alpha_shared = nullptr;
     p.alpha_cols = 0;
-    if (n == 0 || !p.seg[0].alpha || p.seg[0].cols > ds::kTileAlphaCache)
+    if (n == 0 || !p.seg[0].alpha || p.seg[0].cols > ds::kTileAlphaCacheMax)
         return;
     for (int i = 1; i < n; ++i)
         if (p.seg[i].alpha != p.seg[0].alpha || p.seg[i].cols != p.seg[0].cols)
@@ -303,7 +307,7 @@ ds_status launch_all(int nseg, const int64_t *rows, const std::vector<RowClass> 
                 }
                 const int64_t nr = std::min(rows[i] - r0, room * rpu);
                 params.seg[n] = make(i, r0, nr);
-                params.seg[n].group = ci.path == DS_PATH_WARP ? ci.rps : ci.group;
+                params.seg[n].group = ds::is_staged(ci) ? ci.rps : ci.group;
                 params.unit_start[n] = units;
                 units += units_for(ci, nr);
                 ++n;
@@ -423,8 +427,8 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
     std::vector<RowClass> cls(static_cast<size_t>(nseg));
     for (int i = 0; i < nseg; ++i) {
         cls[i] = classify(op, cols[i], forced);
-        if (cls[i].path == DS_PATH_WARP)
-            cls[i].rps = tile_rows_per_slot(op, cols[i], esize, true);
+        if (ds::is_staged(cls[i]))
+            cls[i].rps = tile_rows_per_slot(op, cols[i], esize, true, cls[i].slot);
     }
     auto make = [&](int i, int64_t r0, int64_t nr) {
         WSegK k = wseg_rows(segs[i], r0, nr, esize, esize);
@@ -444,13 +448,13 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
     };
     const bool bf16 = dt == DS_BF16;
     auto launch = [&](const RowClass &rc, const WParams &p, int64_t units, void *st) -> int {
-        if (rc.path == DS_PATH_WARP) {
+        if (ds::is_staged(rc)) {
             const int tag = wop == W_FWD ? (bf16 ? 0 : 1)
                           : wop == W_BWD ? (bf16 ? 2 : 3)
                           : wop == W_RENORM ? 4
                           : wop == W_PROJECT ? 7 : 8;
             const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
-            return ds::launch_tile(tag, &p, grid, ds::kTileSlotBytes, st);
+            return ds::launch_tile(tag, &p, grid, rc.slot, st);
         }
         switch (wop) {
         case W_FWD: return ds::launch_wn_forward(rc, p, units, bf16, st);
@@ -505,14 +509,14 @@ ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *st
     std::vector<RowClass> cls(static_cast<size_t>(nseg));
     for (int i = 0; i < nseg; ++i) {
         cls[i] = classify(op, cols[i], forced);
-        if (cls[i].path == DS_PATH_WARP)
-            cls[i].rps = tile_rows_per_slot(op, cols[i], 2, segs[i].r != nullptr);
+        if (ds::is_staged(cls[i]))
+            cls[i].rps = tile_rows_per_slot(op, cols[i], 2, segs[i].r != nullptr, cls[i].slot);
     }
     auto make = [&](int i, int64_t r0, int64_t nr) { return aseg_rows(segs[i], r0, nr); };
     auto launch = [&](const RowClass &rc, const AParams &p, int64_t units, void *st) -> int {
-        if (rc.path == DS_PATH_WARP) {
+        if (ds::is_staged(rc)) {
             const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
-            return ds::launch_tile(slerp ? 6 : 5, &p, grid, ds::kTileSlotBytes, st);
+            return ds::launch_tile(slerp ? 6 : 5, &p, grid, rc.slot, st);
         }
         return slerp ? ds::launch_slerp_rows(rc, p, units, st) : ds::launch_l2_rows(rc, p, units, st);
     };

@@ -143,63 +143,6 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
-// G threads of a 256-thread CTA per row, G in {32, 64, 128, 256}, the same
-// for every row of the CTA (it comes from the CTA's segment).
-struct GroupReducer {
-    float *sm; // [2][kWarps][4]
-    int G;
-    int slot = 0;
-
-    __device__ GroupReducer(float *scratch, int g) : sm(scratch), G(g) {}
-
-    template <int N, class Op>
-    __device__ __forceinline__ void across_warps(float (&v)[N], Op op)
-    {
-        if (G <= 32)
-            return;
-        const int warp = threadIdx.x >> 5;
-        float *s = sm + slot * (kWarps * 4);
-        if ((threadIdx.x & 31) == 0)
-#pragma unroll
-            for (int i = 0; i < N; ++i)
-                s[warp * 4 + i] = v[i];
-        __syncthreads();
-        const int nw = G >> 5;
-        const int w0 = (threadIdx.x / G) * nw;
-#pragma unroll
-        for (int i = 0; i < N; ++i) {
-            float t = s[w0 * 4 + i];
-            for (int w = 1; w < nw; ++w)
-                t = op(t, s[(w0 + w) * 4 + i]);
-            v[i] = t;
-        }
-        slot ^= 1;
-    }
-
-    template <int N>
-    __device__ __forceinline__ void sum(float (&v)[N])
-    {
-        static_assert(N <= 4, "at most 4 sums");
-        warp_sum(v);
-        across_warps(v, [](float a, float b) { return a + b; });
-    }
-
-    __device__ __forceinline__ float max(float v)
-    {
-        float a[1] = {warp_max(v)};
-        across_warps(a, [](float x, float y) { return fmaxf(x, y); });
-        return a[0];
-    }
-
-    // True if any row of the CTA needs it (keeps barriers CTA-uniform).
-    __device__ __forceinline__ bool any(bool b)
-    {
-        if (G > 32)
-            return __syncthreads_or(b) != 0;
-        return b;
-    }
-};
-
 __device__ __forceinline__ uint32_t cluster_ctarank()
 {
     uint32_t r;

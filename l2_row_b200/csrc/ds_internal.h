@@ -26,11 +26,13 @@ DS_HD constexpr int kmax_of(ds_op op) { return (op == DS_OP_WN_FORWARD || op == 
 constexpr int kMaxCluster = 8;
 // Segments per launch (kernel parameter block); larger tables are split.
 constexpr int kSegPerLaunch = 128;
-// Warp-per-row (tile) path: ring of shared-memory slots filled by bulk copies.
-constexpr int kTileSlotBytes = 16384;  // rows whose staged input fits a slot
-constexpr int kMaxTileSlots = 13;      // 13 x 16 KB = 208 KB of the 227 KB per CTA
+// Staged paths: a ring of shared-memory slots filled by bulk copies, 16 KB
+// (WARP path) or 32 / 64 KB (CTA path) per slot.
+constexpr int kTileSlotBytes = 16384;     // WARP path
+constexpr int kTileSlotMaxBytes = 65536;  // largest CTA-path slot
+constexpr int kMaxTileSlots = 13;         // 13 x 16 KB = 208 KB of the 227 KB per CTA
 constexpr int kTileMaxRowsPerSlot = 64;
-constexpr int kTileAlphaCache = 4096;  // slerp: |alpha| staged in shared memory up to this many columns
+constexpr int kTileAlphaCacheMax = 8192;  // slerp: |alpha| staged in shared memory up to this many columns
 // Two-pass path: units per thread per chunk, chunk size, pipeline stages.
 constexpr int kStreamK = 4;
 constexpr int kChunkUnits = kCta * kStreamK;
@@ -46,20 +48,22 @@ DS_HD constexpr int elems_per_unit(ds_op op) { return is_weight_op(op) ? 4 : 8; 
 
 struct RowClass {
     int path;    // ds_path (never DS_PATH_AUTO)
-    int group;   // threads per row: 32 on the WARP path, 64..256 on the CTA path
+    int group;   // threads per row (staged paths: the team), 0 on cluster paths
     int cluster; // CTAs per row for CLUSTER/TWO_PASS paths (1 otherwise)
-    int rps;     // WARP path: rows per shared-memory slot for this segment
+    int rps;     // staged paths: rows per shared-memory slot for this segment
+    int slot;    // staged paths: slot bytes (16, 32 or 64 KB); 0 otherwise
 };
 
-// Launch shape: all WARP-path segments of a call share one launch of the
-// warp-per-row kernel; all CTA-path segments one launch of the register
-// group kernel (each segment carries its own threads-per-row); CLUSTER and
-// TWO_PASS segments a launch per cluster size.
+inline bool is_staged(const RowClass &c) { return c.path == DS_PATH_WARP || c.path == DS_PATH_CTA; }
+
+// Launch shape: the staged segments of a call share one launch per slot
+// size (each segment carries its own rows per slot); CLUSTER and TWO_PASS
+// segments a launch per cluster size.
 inline bool same_launch(const RowClass &a, const RowClass &b)
 {
     if (a.path == DS_PATH_CLUSTER || a.path == DS_PATH_TWO_PASS)
         return a.path == b.path && a.cluster == b.cluster;
-    return a.path == b.path;
+    return a.path == b.path && a.slot == b.slot;
 }
 
 // Device copy of one weight segment.
@@ -76,7 +80,7 @@ struct WSegK {
     int32_t cols;
     int32_t nu;       // units per row
     float radius;
-    int32_t group;    // threads per row on the group path (32..256)
+    int32_t group;    // staged paths: rows per slot
 };
 
 // Device copy of one activation segment (bf16 carried as raw 16-bit words).
@@ -89,7 +93,7 @@ struct ASegK {
     int64_t ld;
     int32_t cols;
     int32_t nu;
-    int32_t group;    // threads per row on the group path (32..256)
+    int32_t group;    // staged paths: rows per slot
     int32_t pad_;
 };
 
@@ -116,8 +120,8 @@ enum DeviceErrorSite : uint32_t {
     kSiteTileWait = 4,
 };
 
-// Launchers (ds_kernels.cu).  `units` = grid size in rows-groups (WARP/CTA)
-// or rows (CLUSTER/TWO_PASS); return cudaError_t as int.
+// Launchers of the cluster paths (ds_kernels.cu).  `units` = rows
+// (CLUSTER/TWO_PASS); return cudaError_t as int.
 int launch_wn_forward(const RowClass &rc, const WParams &p, int64_t units, bool out_bf16, void *stream);
 int launch_wn_backward(const RowClass &rc, const WParams &p, int64_t units, bool gy_bf16, void *stream);
 int launch_row_renorm(const RowClass &rc, const WParams &p, int64_t units, void *stream);
@@ -126,10 +130,11 @@ int launch_renorm_momentum(const RowClass &rc, const WParams &p, int64_t units, 
 int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_wait_selftest(uint64_t limit_ns, void *stream);
-// Warp-per-row path (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,
-// 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp; params is a
-// WParams (tags 0-4) or AParams (5-6) whose segments carry rows per slot in
-// `group` and whose unit_start counts slots.
+// Staged paths (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,
+// 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp,
+// 7 gradient projection, 8 momentum projection + renorm; params is a WParams
+// (tags 0-4, 7, 8) or AParams (5-6) whose segments carry rows per slot in
+// `group` and whose unit_start counts slots; slot_bytes 16, 32 or 64 KB.
 int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream);
 int read_and_clear_device_error(uint32_t *code, uint32_t *site, void *stream);
 

@@ -1,11 +1,7 @@
-// ds_kernels.cu -- sm_100a kernels for per-row L2 normalisation.
+// ds_kernels.cu -- sm_100a kernels for rows too long for the staged path
+// (ds_tile.cu takes every row with at most 64 KB of input).
 //
-// Three shapes of kernel, chosen per row length (ds_api.cpp):
-//   * group   : G = 32..256 threads of a 256-thread CTA per row (G per
-//               segment, so one launch covers rows of every width that fits);
-//               the row sits in registers (<= 8 16-byte units per thread per
-//               input) between the reduction and the scaled store.  One HBM
-//               read.
+// Two shapes of kernel, chosen per row length (ds_api.cpp):
 //   * cluster : a cluster of 2..8 CTAs per row, each holding a contiguous
 //               slice in registers; partial sums meet through distributed
 //               shared memory.  One HBM read.
@@ -15,6 +11,7 @@
 //               length.
 // Operations (sources cited in include/ds.h):
 //   wn_forward, wn_backward, row_renorm : DragonScale unit rows with gains
+//   grad_project, renorm_momentum       : DragonScale "Optimizer" (rescale)
 //   l2_rows, slerp_rows                 : TensorFold tf_l2_rows, tf_slerp_rows
 #include <cuda_runtime.h>
 
@@ -538,22 +535,6 @@ struct MinBlocks {
     static constexpr int value = T == kSlerp ? 2 : 4;
 };
 
-// G threads per row, 256 / G rows per CTA; G comes from the CTA's segment,
-// so segments of different widths share one launch.
-template <int T>
-__global__ void __launch_bounds__(kCta, MinBlocks<T>::value) k_group(const __grid_constant__ ParamsOf<T> p)
-{
-    __shared__ float red_sm[2 * kWarps * 4];
-    const int64_t unit = blockIdx.x;
-    const int si = find_segment(p, unit);
-    const int G = p.seg[si].group;
-    const int64_t row = (unit - p.unit_start[si]) * (kCta / G) + threadIdx.x / G;
-    const bool active = row < p.seg[si].rows;
-    const int lane = threadIdx.x & (G - 1);
-    GroupReducer red(red_sm, G);
-    run_row<T>(p, si, row, active, lane == 0, lane, G, 0, p.seg[si].nu, red);
-}
-
 // A cluster of CTAs per row; each CTA holds a contiguous slice.
 template <int T>
 __global__ void __launch_bounds__(kCta, MinBlocks<T>::value) k_cluster(const __grid_constant__ ParamsOf<T> p)
@@ -1053,10 +1034,6 @@ cudaError_t launch_op(const RowClass &rc, const ParamsOf<T> &p, int64_t units, v
 {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (rc.path) {
-    case DS_PATH_WARP:
-    case DS_PATH_CTA:
-        k_group<T><<<static_cast<unsigned>(units), kCta, 0, s>>>(p);
-        return cudaGetLastError();
     case DS_PATH_CLUSTER:
         return launch_clustered(k_cluster<T>, p, units, rc.cluster, 0, stream);
     case DS_PATH_TWO_PASS: {

@@ -1,22 +1,23 @@
-// ds_tile.cu -- the warp-per-row path: a persistent, bulk-copy (TMA) fed
-// kernel for every row that fits a shared-memory slot (<= 16 KB of input).
+// ds_tile.cu -- the staged path: a persistent, bulk-copy (TMA) fed kernel
+// for every row whose input fits a shared-memory slot of 16, 32 or 64 KB.
 //
 // One CTA per SM.  The last warp is the producer: it walks the CTA's slots
-// (slot = a run of consecutive rows of one segment, at most kTileSlotBytes of
+// (slot = a run of consecutive rows of one segment, at most the slot size of
 // input) in order, waits until the slot's ring position is free, and fills
 // it with one cp.async.bulk per array (or per row when rows are padded)
 // completing on that position's "full" mbarrier.  The other warps own the
-// ring positions -- one warp each for the weight calls, a pair for the
-// activation calls: slot j of the CTA goes to position j % positions, whose
-// warp(s) wait on "full", normalise its rows out of shared memory, store the
-// results straight to global memory, and arrive on "empty".  Because a
-// position is consumed by its own warps, in order, no barrier is ever waited
+// ring positions, a team of warps each (one or two warps at 16 KB, more for
+// larger slots): slot j of the CTA goes to position j % positions, whose
+// team waits on "full", normalises its rows out of shared memory, stores the
+// results straight to global memory, and arrives on "empty".  Because a
+// position is consumed by its own team, in order, no barrier is ever waited
 // on more than one phase ahead of its current phase.  Every wait is bounded.
 //
-// Per row a warp sums in a fixed order -- each lane its units u = lane,
-// lane + 32, ... in order, two packed fp32 accumulators (even and odd
-// elements) added at the end, then an xor butterfly over the lanes -- so a
-// row's bits depend on its length and the operation only.
+// Per row a team sums in a fixed order -- each thread its units u = t,
+// t + G, ... in order (G threads in the team), two packed fp32 accumulators
+// (even and odd elements) added at the end, an xor butterfly over the lanes,
+// then the warps' partials as a balanced tree -- so a row's bits depend on
+// its length and the operation only.
 #include <cuda_runtime.h>
 
 #include "ds_device.cuh"
@@ -260,29 +261,30 @@ __device__ __forceinline__ int64_t tile_src_pitch(const ASegK &sg, int)
 // valid elements of unit nfull (0 if none), handled by lane nfull % 32 after
 // its full units, so every lane's units are summed in increasing order.
 
-template <bool OUT_BF16, bool RENORM>
-__device__ __forceinline__ void tile_scale_row(const WSegK &sg, int64_t row, float g, const unsigned char *s0,
-                                               int lane, int nfull, int tail, float eps, bool store)
+template <bool OUT_BF16, bool RENORM, int WP>
+__device__ __forceinline__ void tile_scale_row(Team<WP> &tm, const WSegK &sg, int64_t row, float g,
+                                               const unsigned char *s0, int nfull, int tail, float eps, bool store)
 {
+    constexpr int G = Team<WP>::G;
+    const int lane = tm.t;
     const float4 *w = reinterpret_cast<const float4 *>(s0);
     float2 acc = f2(0.f, 0.f);
 #pragma unroll 4
-    for (int u = lane; u < nfull; u += 32) {
+    for (int u = lane; u < nfull; u += G) {
         const float4 v = w[u];
         sq2(acc, f2(v.x, v.y));
         sq2(acc, f2(v.z, v.w));
     }
-    const bool tl = tail && lane == (nfull & 31);
+    const bool tl = tail && lane == nfull % G;
     float4 vt = make_float4(0.f, 0.f, 0.f, 0.f);
     if (tl) {
         vt = mask_quad(w[nfull], tail);
         sq2(acc, f2(vt.x, vt.y));
         sq2(acc, f2(vt.z, vt.w));
     }
-    Team<1> tm{lane, 0, nullptr};
-    const float S = warp_sum1(acc.x + acc.y);
+    const float S = tm.sum1(acc.x + acc.y);
     const RowScale rs = tile_scale(tm, S, eps, [&](auto f) {
-        for (int u = lane; u < nfull; u += 32) {
+        for (int u = lane; u < nfull; u += G) {
             const float4 v = w[u];
             f(f2(v.x, v.y));
             f(f2(v.z, v.w));
@@ -300,7 +302,7 @@ __device__ __forceinline__ void tile_scale_row(const WSegK &sg, int64_t row, flo
                        : static_cast<char *>(sg.out) + row * sg.ld_out * (OUT_BF16 ? 2 : 4);
     const bool plain = rs.pre == 1.f;
 #pragma unroll 4
-    for (int u = lane; u < nfull; u += 32) {
+    for (int u = lane; u < nfull; u += G) {
         const float4 v = w[u];
         float2 a = f2(v.x, v.y), b = f2(v.z, v.w);
         if (!plain) {
@@ -351,15 +353,17 @@ __device__ __forceinline__ float4 gy_unit(const unsigned char *s1, int u)
 // momentum, and w <- rho w / n in place).  With the power-of-two rescale the
 // projection applies the scaled quotient to the scaled row, which stays
 // finite where D/n^2 alone would overflow.
-template <bool GY_BF16, int MODE>
-__device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, float g, const unsigned char *s0,
-                                                  const unsigned char *s1, int lane, int nfull, int tail,
-                                                  float eps, bool store)
+template <bool GY_BF16, int MODE, int WP>
+__device__ __forceinline__ void tile_backward_row(Team<WP> &tm, const WSegK &sg, int64_t row, float g,
+                                                  const unsigned char *s0, const unsigned char *s1, int nfull,
+                                                  int tail, float eps, bool store)
 {
+    constexpr int G = Team<WP>::G;
+    const int lane = tm.t;
     const float4 *w = reinterpret_cast<const float4 *>(s0);
     float2 as = f2(0.f, 0.f), ad = f2(0.f, 0.f);
 #pragma unroll 4
-    for (int u = lane; u < nfull; u += 32) {
+    for (int u = lane; u < nfull; u += G) {
         const float4 x = w[u];
         const float4 d = gy_unit<GY_BF16>(s1, u);
         sq2(as, f2(x.x, x.y));
@@ -367,7 +371,7 @@ __device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, 
         ad = __ffma2_rn(f2(x.x, x.y), f2(d.x, d.y), ad);
         ad = __ffma2_rn(f2(x.z, x.w), f2(d.z, d.w), ad);
     }
-    const bool tl = tail && lane == (nfull & 31);
+    const bool tl = tail && lane == nfull % G;
     float4 xt = make_float4(0.f, 0.f, 0.f, 0.f), dt = xt;
     if (tl) {
         xt = mask_quad(w[nfull], tail);
@@ -377,18 +381,19 @@ __device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, 
         ad = __ffma2_rn(f2(xt.x, xt.y), f2(dt.x, dt.y), ad);
         ad = __ffma2_rn(f2(xt.z, xt.w), f2(dt.z, dt.w), ad);
     }
-    float S = warp_sum1(as.x + as.y);
-    float D = warp_sum1(ad.x + ad.y);
+    float sd[2] = {as.x + as.y, ad.x + ad.y};
+    tm.sum(sd);
+    float S = sd[0], D = sd[1];
     // Rows needing the rescale: w scaled by 2^m (exact), S and D re-summed,
     // 2^m carried into the row constants (as the register paths do).
     int m = 0;
     if (needs_rescale(S, eps)) {
         float M = 0.f;
-        for (int u = lane; u < nfull; u += 32)
+        for (int u = lane; u < nfull; u += G)
             each4_(w[u], [&](float v) { M = fmaxf(M, fabsf(v)); });
         if (tl)
             each4_(xt, [&](float v) { M = fmaxf(M, fabsf(v)); });
-        M = warp_max1(M);
+        M = tm.max(M);
         if (M > 0.f && M < __int_as_float(0x7f800000)) {
             m = 48 - ilogbf(M);
             float2 bs = f2(0.f, 0.f), bd = f2(0.f, 0.f);
@@ -399,12 +404,14 @@ __device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, 
                 bd = __ffma2_rn(p, f2(d.x, d.y), bd);
                 bd = __ffma2_rn(q, f2(d.z, d.w), bd);
             };
-            for (int u = lane; u < nfull; u += 32)
+            for (int u = lane; u < nfull; u += G)
                 add(w[u], gy_unit<GY_BF16>(s1, u));
             if (tl)
                 add(xt, dt);
-            S = warp_sum1(bs.x + bs.y);
-            D = warp_sum1(bd.x + bd.y);
+            float sd2[2] = {bs.x + bs.y, bd.x + bd.y};
+            tm.sum(sd2);
+            S = sd2[0];
+            D = sd2[1];
         }
     }
     if (!store)
@@ -421,7 +428,7 @@ __device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, 
             return m == 0 ? x : make_float4(scalbnf(x.x, m), scalbnf(x.y, m), scalbnf(x.z, m), scalbnf(x.w, m));
         };
 #pragma unroll 4
-        for (int u = lane; u < nfull; u += 32) {
+        for (int u = lane; u < nfull; u += G) {
             const float4 x = scaled(w[u]);
             const float4 d = gy_unit<GY_BF16>(s1, u);
             const float2 a = __ffma2_rn(f2(x.x, x.y), nqs, f2(d.x, d.y));
@@ -452,7 +459,7 @@ __device__ __forceinline__ void tile_backward_row(const WSegK &sg, int64_t row, 
     const float2 nq = f2(-q, -q), pre2 = f2(pre, pre);
     char *out = reinterpret_cast<char *>(sg.grad_w + row * sg.ld);
 #pragma unroll 4
-    for (int u = lane; u < nfull; u += 32) {
+    for (int u = lane; u < nfull; u += G) {
         const float4 x = w[u];
         const float4 d = gy_unit<GY_BF16>(s1, u);
         const float2 a = __fmul2_rn(__ffma2_rn(f2(x.x, x.y), nq, f2(d.x, d.y)), pre2);
@@ -603,12 +610,16 @@ __device__ __forceinline__ float2 lerp2(float2 a, float2 b, float2 m)
     return __ffma2_rn(m, __fadd2_rn(b, fneg2(a)), a);
 }
 
+// |alpha| of unit u: from the shared-memory cache (split layout: the first
+// four of each unit at abs_alpha[4u], the last four at abs_alpha[half + 4u])
+// or from global memory.
 template <bool CACHED>
-__device__ __forceinline__ void abs_alpha8(const float *abs_alpha, const float *alpha, int u, int cols, float2 (&m)[4])
+__device__ __forceinline__ void abs_alpha8(const float *abs_alpha, int half, const float *alpha, int u, int cols,
+                                           float2 (&m)[4])
 {
     if constexpr (CACHED) {
         const float4 m0 = *reinterpret_cast<const float4 *>(abs_alpha + 4 * u);
-        const float4 m1 = *reinterpret_cast<const float4 *>(abs_alpha + kTileAlphaCache / 2 + 4 * u);
+        const float4 m1 = *reinterpret_cast<const float4 *>(abs_alpha + half + 4 * u);
         m[0] = f2(m0.x, m0.y);
         m[1] = f2(m0.z, m0.w);
         m[2] = f2(m1.x, m1.y);
@@ -620,11 +631,12 @@ __device__ __forceinline__ void abs_alpha8(const float *abs_alpha, const float *
 
 template <bool CACHED>
 __device__ __forceinline__ void slerp_unit_t(uint4 p, uint4 q, RowScale ra, RowScale rb, const float *abs_alpha,
-                                             const float *alpha, int u, int cols, float2 &at, float4 &ta, float4 &tb)
+                                             int half, const float *alpha, int u, int cols, float2 &at, float4 &ta,
+                                             float4 &tb)
 {
     const uint4 a = scale8(p, ra), b = scale8(q, rb);
     float2 m[4];
-    abs_alpha8<CACHED>(abs_alpha, alpha, u, cols, m);
+    abs_alpha8<CACHED>(abs_alpha, half, alpha, u, cols, m);
     const float2 t0 = lerp2(lo2(a.x), lo2(b.x), m[0]), t1 = lerp2(lo2(a.y), lo2(b.y), m[1]);
     const float2 t2 = lerp2(lo2(a.z), lo2(b.z), m[2]), t3 = lerp2(lo2(a.w), lo2(b.w), m[3]);
     sq2(at, t0);
@@ -644,7 +656,7 @@ __device__ __forceinline__ uint4 slerp_unit_h(float4 p, float4 q, float2 s)
 template <int WP, bool CACHED>
 __device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
                                                unsigned char *s1, int nfull, int tail, float eps, bool store,
-                                               const float *abs_alpha)
+                                               const float *abs_alpha, int half)
 {
     constexpr int G = Team<WP>::G;
     const int t = tm.t;
@@ -683,13 +695,13 @@ __device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, in
 #pragma unroll 4
     for (int u = t; u < nfull; u += G) {
         float4 p, q;
-        slerp_unit_t<CACHED>(xa[u], xb[u], ra, rb, abs_alpha, sg.alpha, u, sg.cols, at, p, q);
+        slerp_unit_t<CACHED>(xa[u], xb[u], ra, rb, abs_alpha, half, sg.alpha, u, sg.cols, at, p, q);
         ta[u] = p;
         tb[u] = q;
     }
     if (tl) {
         float4 p, q;
-        slerp_unit_t<CACHED>(xa[nfull], xb[nfull], ra, rb, abs_alpha, sg.alpha, nfull, sg.cols, at, p, q);
+        slerp_unit_t<CACHED>(xa[nfull], xb[nfull], ra, rb, abs_alpha, half, sg.alpha, nfull, sg.cols, at, p, q);
         ta[nfull] = p;
         tb[nfull] = q;
     }
@@ -734,26 +746,33 @@ __device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, in
 template <int T>
 using TParams = typename std::conditional<is_weight_tag(T), WParams, AParams>::type;
 
-// Ring shape per operation: 13 ring positions of 16 KB.  The weight calls
-// give each position one consumer warp.  The activation calls, one 16 KB
-// row per position and more work per byte, give each position a pair of
-// warps that reduce every row together (27 warps; slerp's |alpha| cache
-// brings shared memory to ~225 KB of the 227 KB a CTA may hold).
-template <int T>
+// Ring shape per operation and slot size SB (16, 32 or 64 KB of staged
+// input per slot).  A position is owned by a team of warps that reduce each
+// row together: one warp (weight calls) or a pair (activation calls, more
+// work per byte) at 16 KB, and proportionally more warps for the larger
+// slots, so that every thread holds the same number of units per row.  The
+// ring keeps ~200 KB in flight: 13, 6 or 3 positions.  slerp caches |alpha|
+// in the shared memory left over (4,096 columns at 16 KB, 8,192 otherwise).
+template <int T, int SB>
 struct TileCfg {
-    static constexpr int kWP = (T == tL2 || T == tSlerp) ? 2 : 1;
-    static constexpr int kGroups = 13;
-    static constexpr int kSlots = kGroups; // one position per team
+    static_assert(SB == 16384 || SB == 32768 || SB == 65536, "slot size");
+    static constexpr int kSlotBytes = SB;
+    static constexpr int kScale = SB / 16384;                       // 1, 2, 4
+    static constexpr int kWP = ((T == tL2 || T == tSlerp) ? 2 : 1) * kScale;
+    static constexpr int kGroups = SB == 16384 ? 13 : SB == 32768 ? 6 : 3;
+    static constexpr int kSlots = kGroups;                          // one position per team
     static constexpr int kConsumers = kWP * kGroups;
     static constexpr int kThreads = (kConsumers + 1) * 32;
+    static constexpr int kAlphaCache = T == tSlerp ? (SB == 16384 ? 4096 : 8192) : 0;
     static_assert(kSlots <= kMaxTileSlots && kConsumers + 1 <= 32, "ring shape");
 };
 
-template <int T>
-__global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
-    k_tile(const __grid_constant__ TParams<T> p, int slot_bytes)
+template <int T, int SB>
+__global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
+    k_tile(const __grid_constant__ TParams<T> p)
 {
-    using Cfg = TileCfg<T>;
+    using Cfg = TileCfg<T, SB>;
+    constexpr int slot_bytes = SB;
     constexpr int WP = Cfg::kWP;
     constexpr int nslots = Cfg::kSlots;
     extern __shared__ __align__(128) unsigned char ring[];
@@ -764,7 +783,7 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
     __shared__ int vote[Cfg::kGroups * 2 * WP];           // team agreement on a wait: [team][2][warp]
     __shared__ volatile int abort_flag;                    // set by the first wait that runs out
     // slerp: |alpha| of the launch's (single) alpha vector
-    __shared__ __align__(16) float s_alpha[T == tSlerp ? kTileAlphaCache : 4];
+    __shared__ __align__(16) float s_alpha[T == tSlerp ? Cfg::kAlphaCache : 4];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t total = p.unit_start[p.nseg];
@@ -783,8 +802,8 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
         // |alpha| split by halves of each 8-element unit: unit u's first four
         // at [4u], its last four at [half + 4u], so that a warp reading one
         // float4 per lane touches consecutive 16-byte words (no bank conflict)
-        if (p.alpha_shared) {
-            const int nu = (p.alpha_cols + 7) / 8, half = kTileAlphaCache / 2;
+        if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache) {
+            const int nu = (p.alpha_cols + 7) / 8, half = Cfg::kAlphaCache / 2;
             for (int i = threadIdx.x; i < 8 * nu; i += blockDim.x) {
                 const int u = i >> 3, e = i & 7;
                 const float v = i < p.alpha_cols ? fabsf(__ldg(p.alpha_shared + i)) : 0.f;
@@ -911,28 +930,29 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
                 }
                 const float g = __shfl_sync(0xffffffffu, g_lane, r & 31);
                 if constexpr (T == tFwdBf16)
-                    tile_scale_row<true, false>(sg, row, g, s0, lane, nfull, tail, p.eps, store);
+                    tile_scale_row<true, false>(tm, sg, row, g, s0, nfull, tail, p.eps, store);
                 else if constexpr (T == tFwdF32)
-                    tile_scale_row<false, false>(sg, row, g, s0, lane, nfull, tail, p.eps, store);
+                    tile_scale_row<false, false>(tm, sg, row, g, s0, nfull, tail, p.eps, store);
                 else if constexpr (T == tRenorm)
-                    tile_scale_row<false, true>(sg, row, 1.f, s0, lane, nfull, tail, p.eps, store);
+                    tile_scale_row<false, true>(tm, sg, row, 1.f, s0, nfull, tail, p.eps, store);
                 else if constexpr (T == tBwdBf16)
-                    tile_backward_row<true, 0>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, store);
+                    tile_backward_row<true, 0>(tm, sg, row, g, s0, s1, nfull, tail, p.eps, store);
                 else if constexpr (T == tBwdF32)
-                    tile_backward_row<false, 0>(sg, row, g, s0, s1, lane, nfull, tail, p.eps, store);
+                    tile_backward_row<false, 0>(tm, sg, row, g, s0, s1, nfull, tail, p.eps, store);
                 else if constexpr (T == tProject)
-                    tile_backward_row<false, 1>(sg, row, 1.f, s0, s1, lane, nfull, tail, p.eps, store);
+                    tile_backward_row<false, 1>(tm, sg, row, 1.f, s0, s1, nfull, tail, p.eps, store);
                 else if constexpr (T == tMomentum)
-                    tile_backward_row<false, 2>(sg, row, 1.f, s0, s1, lane, nfull, tail, p.eps, store);
+                    tile_backward_row<false, 2>(tm, sg, row, 1.f, s0, s1, nfull, tail, p.eps, store);
                 else if constexpr (T == tL2) {
                     if (has_r)
                         tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
                     else
                         tile_l2_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
-                } else if (p.alpha_shared) {
-                    tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha);
+                } else if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache) {
+                    tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
+                                             Cfg::kAlphaCache / 2);
                 } else {
-                    tile_slerp_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr);
+                    tile_slerp_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr, 0);
                 }
             }
             if (!released)
@@ -945,33 +965,46 @@ __global__ void __launch_bounds__(TileCfg<T>::kThreads, 1)
 
 } // namespace
 
-template <int T>
-static cudaError_t launch_tile_t(const TParams<T> &p, int grid, int slot_bytes, void *stream)
+template <int T, int SB>
+static cudaError_t launch_tile_sb(const TParams<T> &p, int grid, void *stream)
 {
-    const int smem = slot_bytes * TileCfg<T>::kSlots;
-    static int attr_smem = 0; // benign race: idempotent
-    if (attr_smem < smem) {
-        cudaError_t e = cudaFuncSetAttribute(k_tile<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    using Cfg = TileCfg<T, SB>;
+    constexpr int smem = SB * Cfg::kSlots;
+    static bool attr_set = false; // benign race: idempotent
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_tile<T, SB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess)
             return e;
-        attr_smem = smem;
+        attr_set = true;
     }
-    k_tile<T><<<grid, TileCfg<T>::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(p, slot_bytes);
+    k_tile<T, SB><<<grid, Cfg::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError();
+}
+
+template <int T>
+static cudaError_t launch_tile_t(const void *params, int grid, int slot_bytes, void *stream)
+{
+    const TParams<T> &p = *static_cast<const TParams<T> *>(params);
+    switch (slot_bytes) {
+    case 16384: return launch_tile_sb<T, 16384>(p, grid, stream);
+    case 32768: return launch_tile_sb<T, 32768>(p, grid, stream);
+    case 65536: return launch_tile_sb<T, 65536>(p, grid, stream);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream)
 {
     switch (tag) {
-    case tFwdBf16: return launch_tile_t<tFwdBf16>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
-    case tFwdF32: return launch_tile_t<tFwdF32>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
-    case tBwdBf16: return launch_tile_t<tBwdBf16>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
-    case tBwdF32: return launch_tile_t<tBwdF32>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
-    case tRenorm: return launch_tile_t<tRenorm>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
-    case tL2: return launch_tile_t<tL2>(*static_cast<const AParams *>(params), grid, slot_bytes, stream);
-    case tSlerp: return launch_tile_t<tSlerp>(*static_cast<const AParams *>(params), grid, slot_bytes, stream);
-    case tProject: return launch_tile_t<tProject>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
-    case tMomentum: return launch_tile_t<tMomentum>(*static_cast<const WParams *>(params), grid, slot_bytes, stream);
+    case tFwdBf16: return launch_tile_t<tFwdBf16>(params, grid, slot_bytes, stream);
+    case tFwdF32: return launch_tile_t<tFwdF32>(params, grid, slot_bytes, stream);
+    case tBwdBf16: return launch_tile_t<tBwdBf16>(params, grid, slot_bytes, stream);
+    case tBwdF32: return launch_tile_t<tBwdF32>(params, grid, slot_bytes, stream);
+    case tRenorm: return launch_tile_t<tRenorm>(params, grid, slot_bytes, stream);
+    case tL2: return launch_tile_t<tL2>(params, grid, slot_bytes, stream);
+    case tSlerp: return launch_tile_t<tSlerp>(params, grid, slot_bytes, stream);
+    case tProject: return launch_tile_t<tProject>(params, grid, slot_bytes, stream);
+    case tMomentum: return launch_tile_t<tMomentum>(params, grid, slot_bytes, stream);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -46,16 +46,16 @@ A_OPS = (ds.DS_OP_L2_ROWS, ds.DS_OP_SLERP_ROWS)
     (ds.DS_OP_WN_FORWARD, 2048, (ds.DS_PATH_WARP, 32, 1)),
     (ds.DS_OP_WN_BACKWARD, 768, (ds.DS_PATH_WARP, 32, 1)),
     (ds.DS_OP_WN_BACKWARD, 2048, (ds.DS_PATH_WARP, 32, 1)),   # w + fp32 GY = 16 KB
-    (ds.DS_OP_WN_BACKWARD, 2049, (ds.DS_PATH_CTA, 256, 1)),  # 513 quads, 4 per thread at most
+    (ds.DS_OP_WN_BACKWARD, 2049, (ds.DS_PATH_CTA, 64, 1)),   # w + fp32 GY > 16 KB: 32 KB slots, 2 warps
     (ds.DS_OP_ROW_RENORM, 128, (ds.DS_PATH_WARP, 32, 1)),
-    (ds.DS_OP_L2_ROWS, 4096, (ds.DS_PATH_WARP, 32, 1)),       # x + r = 16 KB
-    (ds.DS_OP_SLERP_ROWS, 7168, (ds.DS_PATH_CTA, 256, 1)),
-    (ds.DS_OP_L2_ROWS, 16384, (ds.DS_PATH_CLUSTER, 0, 2)),
-    (ds.DS_OP_WN_FORWARD, 14336, (ds.DS_PATH_CLUSTER, 0, 2)),
+    (ds.DS_OP_L2_ROWS, 4096, (ds.DS_PATH_WARP, 64, 1)),       # x + r = 16 KB, a pair of warps
+    (ds.DS_OP_SLERP_ROWS, 7168, (ds.DS_PATH_CTA, 128, 1)),    # 28 KB: 32 KB slots, 4 warps
+    (ds.DS_OP_L2_ROWS, 16384, (ds.DS_PATH_CTA, 256, 1)),      # 64 KB slots, 8 warps
+    (ds.DS_OP_WN_FORWARD, 14336, (ds.DS_PATH_CTA, 128, 1)),   # 56 KB: 64 KB slots, 4 warps
     (ds.DS_OP_WN_BACKWARD, 14336, (ds.DS_PATH_CLUSTER, 0, 4)),
     (ds.DS_OP_WN_FORWARD, 131072, (ds.DS_PATH_TWO_PASS, 0, 8)),
     (ds.DS_OP_GRAD_PROJECT, 2048, (ds.DS_PATH_WARP, 32, 1)),  # w + G fp32 = 16 KB
-    (ds.DS_OP_RENORM_MOMENTUM, 2049, (ds.DS_PATH_CTA, 256, 1)),
+    (ds.DS_OP_RENORM_MOMENTUM, 2049, (ds.DS_PATH_CTA, 64, 1)),
     (ds.DS_OP_GRAD_PROJECT, 14336, (ds.DS_PATH_CLUSTER, 0, 4)),
     (ds.DS_OP_RENORM_MOMENTUM, 65537, (ds.DS_PATH_TWO_PASS, 0, 8)),
     (ds.DS_OP_SLERP_ROWS, 262144, (ds.DS_PATH_TWO_PASS, 0, 8)),
@@ -65,23 +65,29 @@ def test_row_class_for_workload_shapes(op, cols, want):
 
 
 def test_row_class_is_monotone_and_fits():
+    """Staged classes take rows by their staged bytes (the smallest slot of
+    16, 32 or 64 KB that holds one row, a team of warps per row); longer rows
+    go to clusters whose CTAs hold at most kmax units per thread, then to the
+    two-pass class.  The class never shrinks as rows grow."""
     order = {ds.DS_PATH_WARP: 0, ds.DS_PATH_CTA: 1, ds.DS_PATH_CLUSTER: 2, ds.DS_PATH_TWO_PASS: 3}
     for op in W_OPS + A_OPS:
         e = 4 if op in W_OPS else 8
+        base = 1 if op in W_OPS else 2
         kmax = 8 if op in (ds.DS_OP_WN_FORWARD, ds.DS_OP_ROW_RENORM) else 4
         prev = (0, 0, 0)
         for cols in sorted(set(list(range(1, 600, 7)) + [2 ** k + d for k in range(9, 19) for d in (-1, 0, 1)])):
             path, g, cl = ds.ds_row_class(op, cols)
             nu = -(-cols // e)
-            staged = {ds.DS_OP_WN_FORWARD: 16, ds.DS_OP_ROW_RENORM: 16, ds.DS_OP_WN_BACKWARD: 32}.get(op, 32) * nu
+            staged = (16 if op in (ds.DS_OP_WN_FORWARD, ds.DS_OP_ROW_RENORM) else 32) * nu
             if path == ds.DS_PATH_WARP:
-                assert staged <= 16384 and g == 32
-            else:
-                assert staged > 16384
-            if path == ds.DS_PATH_CTA:
-                assert -(-nu // g) <= kmax and g in (64, 128, 256)
+                assert staged <= 16384 and g == 32 * base and cl == 1
+            elif path == ds.DS_PATH_CTA:
+                slot = 32768 if staged <= 32768 else 65536
+                assert 16384 < staged <= 65536 and g == 32 * base * slot // 16384 and cl == 1
             elif path == ds.DS_PATH_CLUSTER:
-                assert -(-nu // cl) <= 256 * kmax and cl in (2, 4, 8)
+                assert staged > 65536 and -(-nu // cl) <= 256 * kmax and cl in (2, 4, 8)
+            else:
+                assert -(-nu // 8) > 256 * kmax
             key = (order[path], g, cl)
             assert key >= prev, (op, cols)
             prev = key

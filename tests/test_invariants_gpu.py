@@ -26,8 +26,8 @@ from tests.checks import SPREAD, bf16_interval_violations
 
 pytestmark = pytest.mark.gpu
 
-PATHS = [ds.DS_PATH_AUTO, ds.DS_PATH_CLUSTER, ds.DS_PATH_TWO_PASS]
-PATH_IDS = ["auto", "cluster", "two_pass"]
+PATHS = [ds.DS_PATH_AUTO, ds.DS_PATH_CTA, ds.DS_PATH_CLUSTER, ds.DS_PATH_TWO_PASS]
+PATH_IDS = ["auto", "cta", "cluster", "two_pass"]
 
 
 def bits(t):
@@ -235,4 +235,4 @@ def test_launch_counter_counts_kernels():
     wk = wl.whole_model(0, n_layer=1, vocab=512)
     before = ds.ds_launch_count()
     gu.run_forward(wk.weights, "bf16", wk.eps)
-    assert ds.ds_launch_count() - before == 1   # every register-resident row width in one launch
+    assert ds.ds_launch_count() - before == 1   # every staged row width in one launch

@@ -65,7 +65,7 @@ def test_whole_model_one_call(whole_model):
     before = ds.ds_launch_count()
     outs = gu.run_forward(wk.weights, "bf16", wk.eps)
     launches = ds.ds_launch_count() - before
-    assert launches == 1, launches            # 768- and 2048-wide rows share the group-kernel launch
+    assert launches == 1, launches            # 768- and 2048-wide rows share one staged launch
     grads = gu.run_backward(wk.weights, "bf16", wk.eps)
     ws = gu.run_renorm(wk.weights, wk.eps)
     for i, (s, o, (gw, gg), w) in enumerate(zip(wk.weights, outs, grads, ws)):
