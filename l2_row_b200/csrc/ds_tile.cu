@@ -764,6 +764,14 @@ struct TileCfg {
     static constexpr int kConsumers = kWP * kGroups;
     static constexpr int kThreads = (kConsumers + 1) * 32;
     static constexpr int kAlphaCache = T == tSlerp ? (SB == 16384 ? 4096 : 8192) : 0;
+    // Refill pacing: the producer sleeps this long after each refill.  For
+    // the operations below a paced read stream ran faster on B200 (l2 rows
+    // with a residual 74 -> 67 us, the momentum projection + renorm 274 ->
+    // 250 us, backward in 32 KB slots 97 -> 91 us on the benchmark shapes);
+    // for the others it only slowed them, so they refill at once.
+    static constexpr unsigned kPaceNs =
+        ((SB == 16384 && (T == tL2 || T == tMomentum)) || (SB == 32768 && (T == tBwdBf16 || T == tBwdF32))) ? 300
+                                                                                                           : 0;
     static_assert(kSlots <= kMaxTileSlots && kConsumers + 1 <= 32, "ring shape");
 };
 
@@ -818,48 +826,73 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
 
     if (warp == Cfg::kConsumers) {
         // ------------------------------------------------------ producer --
+        // One thread.  Its per-slot work sits between a consumer's release
+        // and the refill it waits for, so it is kept short: position,
+        // phase and slot advance incrementally, and the current segment's
+        // copy geometry is cached in registers until the walk leaves it.
+        // (The consumers fence their generic-proxy writes to a slot before
+        // releasing it, so the refill needs no fence here.)
         if (lane == 0) {
-            int si = 0;
-            for (int64_t j = 0; j < mine; ++j) {
-                const int s = static_cast<int>(j % nslots);
-                if (j >= nslots && (abort_flag ||
-                    !mbar_wait_bounded(&empty[s], static_cast<uint32_t>((j / nslots - 1) & 1), p.wait_limit_ns))) {
+            int si = -1;
+            int64_t seg_begin = 0, seg_end = 0, seg_rows = 0;
+            int rps = 1;
+            uint32_t pitch[2] = {0u, 0u}, off1 = 0u;
+            const char *src[2] = {nullptr, nullptr};
+            int64_t spitch[2] = {0, 0};
+            bool contig[2] = {false, false};
+            int s = 0;
+            uint32_t phase = 0;             // parity of the release a refill of position s waits for
+            int64_t slot = blockIdx.x;
+            for (int64_t j = 0; j < mine; ++j, slot += gridDim.x) {
+                if (j >= nslots && (abort_flag || !mbar_wait_bounded(&empty[s], phase, p.wait_limit_ns))) {
                     ok = false;
                     abort_flag = 1;
                     break;
                 }
-                const int64_t slot = blockIdx.x + j * gridDim.x;
-                while (si + 1 < p.nseg && p.unit_start[si + 1] <= slot) // slots increase: walk forward
-                    ++si;
-                const auto &sg = p.seg[si];
-                const int rps = sg.group; // rows per slot for this segment
-                const int64_t row0 = (slot - p.unit_start[si]) * rps;
-                const int nrows = static_cast<int>(sg.rows - row0 < rps ? sg.rows - row0 : rps);
-                hdr[s] = SlotHdr{si, nrows, row0};
-                const bool has_r = seg_has_r(sg);
-                unsigned char *dst = ring + static_cast<size_t>(s) * slot_bytes;
-                uint32_t bytes = 0, pitch[2], off[2];
+                if (slot >= seg_end) {      // slots increase: walk forward to the slot's segment
+                    do {
+                        ++si;
+                        seg_end = p.unit_start[si + 1];
+                    } while (seg_end <= slot);
+                    seg_begin = p.unit_start[si];
+                    const auto &sg = p.seg[si];
+                    seg_rows = sg.rows;
+                    rps = sg.group;         // rows per slot for this segment
+                    const bool has_r = seg_has_r(sg);
 #pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    const int u = a < Layout::kArrays ? Layout::ub(a, has_r) : 0;
-                    pitch[a] = (static_cast<uint32_t>(sg.nu) * u + 15u) & ~15u;
-                    off[a] = a == 0 ? 0u : pitch[0] * rps;
-                    bytes += pitch[a] * nrows;
+                    for (int a2 = 0; a2 < 2; ++a2) {
+                        const int u = a2 < Layout::kArrays ? Layout::ub(a2, has_r) : 0;
+                        pitch[a2] = (static_cast<uint32_t>(sg.nu) * u + 15u) & ~15u;
+                        src[a2] = pitch[a2] ? tile_src<T>(sg, a2, 0) : nullptr;
+                        spitch[a2] = tile_src_pitch<T>(sg, a2);
+                        contig[a2] = spitch[a2] == static_cast<int64_t>(pitch[a2]);
+                    }
+                    off1 = pitch[0] * rps;
                 }
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&full[s], bytes);
+                const int64_t row0 = (slot - seg_begin) * rps;
+                const int nrows = static_cast<int>(seg_rows - row0 < rps ? seg_rows - row0 : rps);
+                hdr[s] = SlotHdr{si, nrows, row0};
+                unsigned char *dst = ring + static_cast<size_t>(s) * slot_bytes;
+                mbar_arrive_expect_tx(&full[s], (pitch[0] + pitch[1]) * nrows);
 #pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    if (!pitch[a])
+                for (int a2 = 0; a2 < 2; ++a2) {
+                    if (!pitch[a2])
                         continue;
-                    const char *src = tile_src<T>(sg, a, row0);
-                    const int64_t src_pitch = tile_src_pitch<T>(sg, a);
-                    if (src_pitch == static_cast<int64_t>(pitch[a])) {
-                        bulk_g2s(dst + off[a], src, pitch[a] * nrows, &full[s]);
+                    unsigned char *d = dst + (a2 == 0 ? 0u : off1);
+                    const char *g = src[a2] + row0 * spitch[a2];
+                    if (contig[a2]) {
+                        bulk_g2s(d, g, pitch[a2] * nrows, &full[s]);
                     } else {
                         for (int r = 0; r < nrows; ++r)
-                            bulk_g2s(dst + off[a] + r * pitch[a], src + r * src_pitch, pitch[a], &full[s]);
+                            bulk_g2s(d + r * pitch[a2], g + r * spitch[a2], pitch[a2], &full[s]);
                     }
+                }
+                if constexpr (Cfg::kPaceNs != 0)
+                    __nanosleep(Cfg::kPaceNs);
+                if (++s == nslots) {        // a round of the ring ends; rounds 2, 3, ...
+                    s = 0;                  // wait for releases of parity 0, 1, 0, ...
+                    if (j >= 2 * nslots - 1)
+                        phase ^= 1u;
                 }
             }
         }
