@@ -66,11 +66,20 @@ int64_t tile_row_bytes_worst(ds_op op, int64_t cols)
     }
 }
 
-// Warps of a staged team: one (weights) or two (activations) per 16 KB of slot.
+// Warps of a staged team: one (weights) or two (activations) per 16 KB of
+// slot; eight for the 112 KB weight slots.
 int team_warps(ds_op op, int slot)
 {
+    if (slot == ds::kTileSlotMaxWeightBytes)
+        return 8;
     const int base = (op == DS_OP_L2_ROWS || op == DS_OP_SLERP_ROWS) ? 2 : 1;
     return base * slot / ds::kTileSlotBytes;
+}
+
+// Largest staged slot of an operation.
+int64_t max_slot(ds_op op)
+{
+    return ds::is_weight_op(op) ? ds::kTileSlotMaxWeightBytes : ds::kTileSlotMaxBytes;
 }
 
 RowClass classify(ds_op op, int64_t cols, int forced)
@@ -80,8 +89,8 @@ RowClass classify(ds_op op, int64_t cols, int forced)
     const int64_t kmax = ds::kmax_of(op);
     const int64_t staged = tile_row_bytes_worst(op, cols);
     auto staged_class = [&](int path, int min_slot) -> RowClass {
-        for (int slot = min_slot; slot <= ds::kTileSlotMaxBytes; slot *= 2)
-            if (staged <= slot)
+        for (const int slot : {16384, 32768, 65536, 114688})
+            if (slot >= min_slot && slot <= max_slot(op) && staged <= slot)
                 return {path, 32 * team_warps(op, slot), 1, 0, slot};
         return {0, 0, 0, 0, 0};
     };
@@ -97,7 +106,7 @@ RowClass classify(ds_op op, int64_t cols, int forced)
             return staged_class(DS_PATH_WARP, ds::kTileSlotBytes);
         break;
     case DS_PATH_CTA:
-        if (staged <= ds::kTileSlotMaxBytes)
+        if (staged <= max_slot(op))
             return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
         break;
     case DS_PATH_CLUSTER:
@@ -111,7 +120,7 @@ RowClass classify(ds_op op, int64_t cols, int forced)
     }
     if (staged <= ds::kTileSlotBytes)
         return staged_class(DS_PATH_WARP, ds::kTileSlotBytes);
-    if (staged <= ds::kTileSlotMaxBytes)
+    if (staged <= max_slot(op))
         return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
     if (const int CL = cluster_of())
         return {DS_PATH_CLUSTER, 0, CL, 0, 0};

@@ -27,9 +27,11 @@ constexpr int kMaxCluster = 8;
 // Segments per launch (kernel parameter block); larger tables are split.
 constexpr int kSegPerLaunch = 128;
 // Staged paths: a ring of shared-memory slots filled by bulk copies, 16 KB
-// (WARP path) or 32 / 64 KB (CTA path) per slot.
-constexpr int kTileSlotBytes = 16384;     // WARP path
-constexpr int kTileSlotMaxBytes = 65536;  // largest CTA-path slot
+// (WARP path) or 32 / 64 KB (CTA path) per slot, and 112 KB for weight rows
+// (two of them fill a CTA's shared memory).
+constexpr int kTileSlotBytes = 16384;          // WARP path
+constexpr int kTileSlotMaxBytes = 65536;       // largest CTA-path slot of the activation rows
+constexpr int kTileSlotMaxWeightBytes = 114688;
 constexpr int kMaxTileSlots = 13;         // 13 x 16 KB = 208 KB of the 227 KB per CTA
 constexpr int kTileMaxRowsPerSlot = 64;
 constexpr int kTileAlphaCacheMax = 8192;  // slerp: |alpha| staged in shared memory up to this many columns

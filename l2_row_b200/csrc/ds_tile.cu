@@ -747,19 +747,21 @@ template <int T>
 using TParams = typename std::conditional<is_weight_tag(T), WParams, AParams>::type;
 
 // Ring shape per operation and slot size SB (16, 32 or 64 KB of staged
-// input per slot).  A position is owned by a team of warps that reduce each
-// row together: one warp (weight calls) or a pair (activation calls, more
-// work per byte) at 16 KB, and proportionally more warps for the larger
-// slots, so that every thread holds the same number of units per row.  The
-// ring keeps ~200 KB in flight: 13, 6 or 3 positions.  slerp caches |alpha|
+// input per slot; 112 KB for weight rows).  A position is owned by a team
+// of warps that reduce each row together: one warp (weight calls) or a pair
+// (activation calls, more work per byte) at 16 KB, and proportionally more
+// warps for the larger slots, so that every thread holds about the same
+// number of units per row.  The ring keeps ~200 KB in flight: 13, 6, 3 or 2
+// positions.  slerp caches |alpha|
 // in the shared memory left over (4,096 columns at 16 KB, 8,192 otherwise).
 template <int T, int SB>
 struct TileCfg {
-    static_assert(SB == 16384 || SB == 32768 || SB == 65536, "slot size");
+    static_assert(SB == 16384 || SB == 32768 || SB == 65536 || SB == 114688, "slot size");
+    static_assert(SB != 114688 || is_weight_tag(T), "112 KB slots: weight rows only");
     static constexpr int kSlotBytes = SB;
-    static constexpr int kScale = SB / 16384;                       // 1, 2, 4
+    static constexpr int kScale = SB == 114688 ? 8 : SB / 16384;    // 1, 2, 4; 8 for 112 KB
     static constexpr int kWP = ((T == tL2 || T == tSlerp) ? 2 : 1) * kScale;
-    static constexpr int kGroups = SB == 16384 ? 13 : SB == 32768 ? 6 : 3;
+    static constexpr int kGroups = SB == 16384 ? 13 : SB == 32768 ? 6 : SB == 65536 ? 3 : 2;
     static constexpr int kSlots = kGroups;                          // one position per team
     static constexpr int kConsumers = kWP * kGroups;
     static constexpr int kThreads = (kConsumers + 1) * 32;
@@ -1022,6 +1024,11 @@ static cudaError_t launch_tile_t(const void *params, int grid, int slot_bytes, v
     case 16384: return launch_tile_sb<T, 16384>(p, grid, stream);
     case 32768: return launch_tile_sb<T, 32768>(p, grid, stream);
     case 65536: return launch_tile_sb<T, 65536>(p, grid, stream);
+    case 114688:
+        if constexpr (is_weight_tag(T))
+            return launch_tile_sb<T, 114688>(p, grid, stream);
+        else
+            return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
     }
 }

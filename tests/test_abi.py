@@ -52,11 +52,13 @@ A_OPS = (ds.DS_OP_L2_ROWS, ds.DS_OP_SLERP_ROWS)
     (ds.DS_OP_SLERP_ROWS, 7168, (ds.DS_PATH_CTA, 128, 1)),    # 28 KB: 32 KB slots, 4 warps
     (ds.DS_OP_L2_ROWS, 16384, (ds.DS_PATH_CTA, 256, 1)),      # 64 KB slots, 8 warps
     (ds.DS_OP_WN_FORWARD, 14336, (ds.DS_PATH_CTA, 128, 1)),   # 56 KB: 64 KB slots, 4 warps
-    (ds.DS_OP_WN_BACKWARD, 14336, (ds.DS_PATH_CLUSTER, 0, 4)),
+    (ds.DS_OP_WN_BACKWARD, 14336, (ds.DS_PATH_CTA, 256, 1)),  # 112 KB (fp32 GY layout): 112 KB slots, 8 warps
+    (ds.DS_OP_WN_BACKWARD, 14337, (ds.DS_PATH_CLUSTER, 0, 4)),
     (ds.DS_OP_WN_FORWARD, 131072, (ds.DS_PATH_TWO_PASS, 0, 8)),
     (ds.DS_OP_GRAD_PROJECT, 2048, (ds.DS_PATH_WARP, 32, 1)),  # w + G fp32 = 16 KB
     (ds.DS_OP_RENORM_MOMENTUM, 2049, (ds.DS_PATH_CTA, 64, 1)),
-    (ds.DS_OP_GRAD_PROJECT, 14336, (ds.DS_PATH_CLUSTER, 0, 4)),
+    (ds.DS_OP_GRAD_PROJECT, 14336, (ds.DS_PATH_CTA, 256, 1)),
+    (ds.DS_OP_GRAD_PROJECT, 16384, (ds.DS_PATH_CLUSTER, 0, 4)),
     (ds.DS_OP_RENORM_MOMENTUM, 65537, (ds.DS_PATH_TWO_PASS, 0, 8)),
     (ds.DS_OP_SLERP_ROWS, 262144, (ds.DS_PATH_TWO_PASS, 0, 8)),
 ])
@@ -82,10 +84,13 @@ def test_row_class_is_monotone_and_fits():
             if path == ds.DS_PATH_WARP:
                 assert staged <= 16384 and g == 32 * base and cl == 1
             elif path == ds.DS_PATH_CTA:
-                slot = 32768 if staged <= 32768 else 65536
-                assert 16384 < staged <= 65536 and g == 32 * base * slot // 16384 and cl == 1
+                top = 114688 if op in W_OPS else 65536
+                slot = next(x for x in (32768, 65536, 114688) if staged <= x)
+                warps = 8 if slot == 114688 else base * slot // 16384
+                assert 16384 < staged <= top and g == 32 * warps and cl == 1
             elif path == ds.DS_PATH_CLUSTER:
-                assert staged > 65536 and -(-nu // cl) <= 256 * kmax and cl in (2, 4, 8)
+                top = 114688 if op in W_OPS else 65536
+                assert staged > top and -(-nu // cl) <= 256 * kmax and cl in (2, 4, 8)
             else:
                 assert -(-nu // 8) > 256 * kmax
             key = (order[path], g, cl)

@@ -172,3 +172,39 @@ def test_eps_control_is_detected():
 
     with pytest.raises(AssertionError):
         gu.check_project(seg, Gp, 1e-6, flags=oracle.OR_EPS_ZERO)
+
+
+def test_largest_weight_slot_ragged_with_guards():
+    """Rows of 12,289 fp32 columns: 96 KB of staged input in the widest
+    layout, so the 112 KB-slot class (two positions, eight warps per row),
+    with a ragged last quad and padded rows."""
+    rng = np.random.default_rng(47)
+    rows, cols = 9, 12289
+    assert ds.ds_row_class(ds.DS_OP_WN_BACKWARD, cols)[:2] == (ds.DS_PATH_CTA, 256)
+    ld = ((cols + 3) // 4) * 4 + 4
+    seg = wl.WeightSeg("big", wl.drifted_rows(rng, rows, cols, 0.02), wl.gains(rng, rows),
+                       rng.standard_normal((rows, cols), dtype=np.float32))
+    w, wbuf = gu.padded(rows, cols, ld, torch.float32, gu.CANARY_F32)
+    w.copy_(gu.dev_f32(seg.w))
+    g = gu.dev_f32(seg.g)
+    gy, _ = gu.padded(rows, cols, ld, torch.float32, gu.CANARY_F32)
+    gy.copy_(gu.dev_f32(seg.gy))
+    gw, gwbuf = gu.padded(rows, cols, ld, torch.float32, gu.CANARY_F32)
+    gg = torch.empty(rows, device="cuda")
+    ds.ds_wn_backward([ds.WSeg(w=w, gain=g, gy=gy, grad_w=gw, grad_g=gg)], "f32", 1e-6)
+    torch.cuda.synchronize()
+    assert gu.guards_intact(gwbuf, rows, cols, ld, gu.CANARY_F32)
+    gu.check_backward(seg, gw, gg, 1e-6, what="backward 112 KB slots")
+    G, gbuf = gu.padded(rows, cols, ld, torch.float32, gu.CANARY_F32)
+    G.copy_(gu.dev_f32(seg.gy))
+    ds.ds_grad_project([ds.WSeg(w=w, grad_w=G)], 1e-6)
+    torch.cuda.synchronize()
+    assert gu.guards_intact(gbuf, rows, cols, ld, gu.CANARY_F32)
+    gu.check_project(seg, G, 1e-6, what="grad_project 112 KB slots")
+    m, mbuf = gu.padded(rows, cols, ld, torch.float32, gu.CANARY_F32)
+    m.copy_(gu.dev_f32(seg.gy))
+    ds.ds_renorm_momentum([ds.WSeg(w=w, grad_w=m)], 1e-6)
+    torch.cuda.synchronize()
+    assert gu.guards_intact(mbuf, rows, cols, ld, gu.CANARY_F32)
+    assert gu.guards_intact(wbuf, rows, cols, ld, gu.CANARY_F32)
+    gu.check_momentum(seg, w, m, 1e-6, what="renorm_momentum 112 KB slots")
