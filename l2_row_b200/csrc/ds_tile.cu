@@ -792,8 +792,8 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
     __shared__ float red[Cfg::kGroups * Team<WP>::kRed]; // team reductions
     __shared__ int vote[Cfg::kGroups * 2 * WP];           // team agreement on a wait: [team][2][warp]
     __shared__ volatile int abort_flag;                    // set by the first wait that runs out
-    // slerp: |alpha| of the launch's (single) alpha vector
-    __shared__ __align__(16) float s_alpha[T == tSlerp ? Cfg::kAlphaCache : 4];
+    // slerp: |alpha| of the launch's (single) alpha vector, after the ring
+    float *s_alpha = reinterpret_cast<float *>(ring + static_cast<size_t>(nslots) * slot_bytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t total = p.unit_start[p.nseg];
@@ -1004,7 +1004,7 @@ template <int T, int SB>
 static cudaError_t launch_tile_sb(const TParams<T> &p, int grid, void *stream)
 {
     using Cfg = TileCfg<T, SB>;
-    constexpr int smem = SB * Cfg::kSlots;
+    constexpr int smem = SB * Cfg::kSlots + 4 * Cfg::kAlphaCache;
     static bool attr_set = false; // benign race: idempotent
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_tile<T, SB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
