@@ -220,6 +220,83 @@ void or_slerp_row(const double *res, const double *out, const double *alpha,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Backward of the activation rows (derived: the pages give the forward
+ * only).  Gradients pass straight through the bf16 rounding points: the
+ * backward uses the rounded values wherever the forward does (s, a, b) and
+ * takes the rounding itself as the identity.                                */
+
+/* y = s / n, n = sqrt(S + eps), s = x or bf16(x + r):
+ *   dx_j = (dy_j - s_j D / (S + eps)) / n,  D = sum_k s_k dy_k
+ * (with a residual, dr = dx). */
+void or_l2_backward_row(const double *x, const double *r, const double *dy,
+                        int64_t C, double eps, unsigned flags, double *s,
+                        double *dx)
+{
+    for (int64_t j = 0; j < C; ++j) {
+        if (!r)
+            s[j] = x[j];
+        else if (flags & OR_DROP_SUM_ROUND)
+            s[j] = x[j] + r[j];
+        else
+            s[j] = round_bf16(x[j] + r[j]);
+    }
+    double S = sum_sq(s, C);
+    double D = 0.0;
+    for (int64_t j = 0; j < C; ++j)
+        D += s[j] * dy[j];
+    double e = (flags & OR_EPS_ZERO) ? 0.0 : eps;
+    double n = sqrt(S + e);
+    for (int64_t j = 0; j < C; ++j)
+        dx[j] = (dy[j] - s[j] * D / (S + e)) / n;
+}
+
+/* h = t / nt, t = a + |alpha| (b - a), a = bf16(res / na), b = bf16(out / nb):
+ *   dt = (dh - t (t . dh) / nt^2) / nt,
+ *   da = (1 - |alpha|) dt,  db = |alpha| dt,
+ *   dres = (da - res (res . da) / na^2) / na,  dout likewise with out, db, nb,
+ *   dalpha_j (this row's part) = sign(alpha_j) (b_j - a_j) dt_j  (sign(0) = 0).
+ * tmp holds 4*C doubles; dalpha_row may be NULL. */
+void or_slerp_backward_row(const double *res, const double *out,
+                           const double *alpha, const double *dh, int64_t C,
+                           double eps, unsigned flags, double *tmp,
+                           double *dres, double *dout, double *dalpha_row)
+{
+    double *a = tmp, *b = tmp + C, *t = tmp + 2 * C, *dt = tmp + 3 * C;
+    double e = (flags & OR_EPS_ZERO) ? 0.0 : eps;
+    double na2 = sum_sq(res, C) + e, nb2 = sum_sq(out, C) + e;
+    double na = sqrt(na2), nb = sqrt(nb2);
+    for (int64_t j = 0; j < C; ++j) {
+        a[j] = res[j] / na;
+        if (!(flags & OR_DROP_SLERP_A))
+            a[j] = round_bf16(a[j]);
+        b[j] = out[j] / nb;
+        if (!(flags & OR_DROP_SLERP_B))
+            b[j] = round_bf16(b[j]);
+        t[j] = a[j] + fabs(alpha[j]) * (b[j] - a[j]);
+    }
+    double nt2 = sum_sq(t, C) + e, Dt = 0.0;
+    for (int64_t j = 0; j < C; ++j)
+        Dt += t[j] * dh[j];
+    double nt = sqrt(nt2);
+    double Da = 0.0, Db = 0.0;
+    for (int64_t j = 0; j < C; ++j) {
+        double m = fabs(alpha[j]);
+        dt[j] = (dh[j] - t[j] * Dt / nt2) / nt;
+        Da += res[j] * ((1.0 - m) * dt[j]);
+        Db += out[j] * (m * dt[j]);
+    }
+    for (int64_t j = 0; j < C; ++j) {
+        double m = fabs(alpha[j]);
+        dres[j] = ((1.0 - m) * dt[j] - res[j] * Da / na2) / na;
+        dout[j] = (m * dt[j] - out[j] * Db / nb2) / nb;
+        if (dalpha_row) {
+            double sg = alpha[j] > 0.0 ? 1.0 : alpha[j] < 0.0 ? -1.0 : 0.0;
+            dalpha_row[j] = sg * (b[j] - a[j]) * dt[j];
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Interval forms.                                                           */
 
 static double dmin(double a, double b) { return a < b ? a : b; }
@@ -326,7 +403,8 @@ void or_slerp_row_interval(const double *res, const double *out,
 /* Matrix drivers.  Each worker owns a contiguous range of rows and its own
  * scratch rows; inputs are widened to double exactly before the row call.   */
 
-enum { OP_FWD, OP_BWD, OP_RENORM, OP_L2, OP_SLERP, OP_L2_IV, OP_SLERP_IV, OP_PROJECT, OP_MOMENTUM };
+enum { OP_FWD, OP_BWD, OP_RENORM, OP_L2, OP_SLERP, OP_L2_IV, OP_SLERP_IV, OP_PROJECT, OP_MOMENTUM,
+       OP_L2_BWD, OP_SLERP_BWD };
 
 typedef struct {
     int op;
@@ -342,6 +420,7 @@ typedef struct {
     double *out_d;   /* dense [R, C] doubles */
     double *out_g;   /* [R] */
     double *out_d2;  /* dense [R, C] doubles (second output) */
+    const uint16_t *dy; /* bf16 bits [R, ld] (activation backward) */
     uint16_t *out_h; /* dense [R, C] bf16 bits */
     uint16_t *out_h2; /* dense [R, C] bf16 bits (interval upper ends) */
     int status;
@@ -351,13 +430,13 @@ static void *run_job(void *arg)
 {
     job_t *jb = (job_t *)arg;
     int64_t C = jb->C;
-    double *buf = (double *)malloc(sizeof(double) * (size_t)(6 * C));
+    double *buf = (double *)malloc(sizeof(double) * (size_t)(9 * C));
     if (!buf) {
         jb->status = -1;
         return NULL;
     }
-    double *u = buf, *v = buf + C, *tmp = buf + 2 * C, *al = buf + 5 * C;
-    if (jb->op == OP_SLERP || jb->op == OP_SLERP_IV)
+    double *u = buf, *v = buf + C, *tmp = buf + 2 * C, *al = buf + 6 * C, *dv = buf + 7 * C;
+    if (jb->op == OP_SLERP || jb->op == OP_SLERP_IV || jb->op == OP_SLERP_BWD)
         for (int64_t j = 0; j < C; ++j)
             al[j] = (double)jb->alpha[j];
 
@@ -410,6 +489,26 @@ static void *run_job(void *arg)
             else
                 or_renorm_momentum_row(u, v, C, jb->rho, jb->eps, jb->flags,
                                        jb->out_d2 + o, jb->out_d + o);
+            break;
+        }
+        case OP_L2_BWD:
+        case OP_SLERP_BWD: {
+            const uint16_t *xr = jb->x + row * jb->ld;
+            const uint16_t *dr = jb->dy + row * jb->ld;
+            for (int64_t j = 0; j < C; ++j) {
+                u[j] = or_bf16_value(xr[j]);
+                dv[j] = or_bf16_value(dr[j]);
+            }
+            if (jb->r) {
+                const uint16_t *rr = jb->r + row * jb->ld;
+                for (int64_t j = 0; j < C; ++j)
+                    v[j] = or_bf16_value(rr[j]);
+            }
+            if (jb->op == OP_L2_BWD)
+                or_l2_backward_row(u, jb->r ? v : NULL, dv, C, jb->eps, jb->flags, tmp, jb->out_d + o);
+            else
+                or_slerp_backward_row(u, v, al, dv, C, jb->eps, jb->flags, tmp, jb->out_d + o,
+                                      jb->out_d2 + o, NULL);
             break;
         }
         case OP_L2:
@@ -591,6 +690,81 @@ int or_renorm_momentum(const float *w, int64_t R, int64_t C, int64_t ld,
     jb.out_d = m_out;
     jb.out_d2 = w_out;
     return run_rows(&jb, R, nthreads);
+}
+
+int or_l2_rows_backward(const uint16_t *x, const uint16_t *r,
+                        const uint16_t *dy, int64_t R, int64_t C, int64_t ld,
+                        double eps, unsigned flags, double *dx, int nthreads)
+{
+    if (bad_shape(R, C, ld) || (R > 0 && (!x || !dy || !dx)))
+        return -1;
+    if (flags & ~(OR_EPS_ZERO | OR_DROP_SUM_ROUND))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_L2_BWD;
+    jb.C = C;
+    jb.ld = ld;
+    jb.x = x;
+    jb.r = r;
+    jb.dy = dy;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_d = dx;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_slerp_rows_backward(const uint16_t *res, const uint16_t *out,
+                           const float *alpha, const uint16_t *dh, int64_t R,
+                           int64_t C, int64_t ld, double eps, unsigned flags,
+                           double *dres, double *dout, double *dalpha,
+                           int nthreads)
+{
+    if (bad_shape(R, C, ld) || !alpha || (R > 0 && (!res || !out || !dh || !dres || !dout)))
+        return -1;
+    if (flags & ~(OR_EPS_ZERO | OR_DROP_SLERP_A | OR_DROP_SLERP_B))
+        return -1;
+    job_t jb = {0};
+    jb.op = OP_SLERP_BWD;
+    jb.C = C;
+    jb.ld = ld;
+    jb.x = res;
+    jb.r = out;
+    jb.alpha = alpha;
+    jb.dy = dh;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.out_d = dres;
+    jb.out_d2 = dout;
+    int rc = run_rows(&jb, R, nthreads);
+    if (rc != 0 || !dalpha)
+        return rc;
+    /* dalpha: the rows' parts summed in row order (one thread) */
+    double *tmp = (double *)malloc(sizeof(double) * (size_t)(9 * C));
+    if (!tmp)
+        return -1;
+    double *u = tmp + 4 * C, *v = tmp + 5 * C, *al = tmp + 6 * C, *dv = tmp + 7 * C, *part = tmp + 8 * C;
+    double *scratch = (double *)malloc(sizeof(double) * (size_t)(2 * C));
+    if (!scratch) {
+        free(tmp);
+        return -1;
+    }
+    for (int64_t j = 0; j < C; ++j) {
+        al[j] = (double)alpha[j];
+        dalpha[j] = 0.0;
+    }
+    for (int64_t row = 0; row < R; ++row) {
+        for (int64_t j = 0; j < C; ++j) {
+            u[j] = or_bf16_value(res[row * ld + j]);
+            v[j] = or_bf16_value(out[row * ld + j]);
+            dv[j] = or_bf16_value(dh[row * ld + j]);
+        }
+        or_slerp_backward_row(u, v, al, dv, C, eps, flags, tmp, scratch, scratch + C, part);
+        for (int64_t j = 0; j < C; ++j)
+            dalpha[j] += part[j];
+    }
+    free(scratch);
+    free(tmp);
+    return 0;
 }
 
 int or_row_renorm(const float *w, int64_t R, int64_t C, int64_t ld, double rho,

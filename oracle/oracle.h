@@ -79,6 +79,22 @@ void or_renorm_momentum_row(const double *w, const double *m, int64_t C,
 void or_row_renorm_row(const double *w, int64_t C, double rho, double eps,
                        unsigned flags, double *out);
 
+/* Backward of the activation rows (derived; the pages give the forward
+ * only).  Gradients pass straight through the bf16 rounding points, which
+ * keep their rounded values (s, a, b) as in the forward.
+ *   l2:    dx_j = (dy_j - s_j (s . dy) / (S + eps)) / sqrt(S + eps);  s_tmp C doubles.
+ *   slerp: dt = (dh - t (t . dh)/nt^2)/nt, da = (1-|alpha|) dt, db = |alpha| dt,
+ *          dres = (da - res (res . da)/na^2)/na, dout likewise,
+ *          dalpha_row_j = sign(alpha_j) (b_j - a_j) dt_j (may be NULL);
+ *          tmp 4*C doubles. */
+void or_l2_backward_row(const double *x, const double *r, const double *dy,
+                        int64_t C, double eps, unsigned flags, double *s_tmp,
+                        double *dx);
+void or_slerp_backward_row(const double *res, const double *out,
+                           const double *alpha, const double *dh, int64_t C,
+                           double eps, unsigned flags, double *tmp,
+                           double *dres, double *dout, double *dalpha_row);
+
 /* [TF] tf_l2_rows: s = x or bf16(x + r); y = bf16(s / sqrt(sum s^2 + eps)).
  * r may be NULL.  s_tmp holds C doubles.  y_exact (may be NULL) receives the
  * value before the final rounding. */
@@ -149,6 +165,17 @@ int or_l2_rows(const uint16_t *x, const uint16_t *r, int64_t R, int64_t C,
 int or_slerp_rows(const uint16_t *res, const uint16_t *out, const float *alpha,
                   int64_t R, int64_t C, int64_t ld, double eps, unsigned flags,
                   uint16_t *h, double *h_exact, int nthreads);
+
+/* Backward of the activation rows over matrices (bf16 bits in, f64 out).
+ * dalpha (may be NULL) = the rows' parts summed in row order. */
+int or_l2_rows_backward(const uint16_t *x, const uint16_t *r,
+                        const uint16_t *dy, int64_t R, int64_t C, int64_t ld,
+                        double eps, unsigned flags, double *dx, int nthreads);
+int or_slerp_rows_backward(const uint16_t *res, const uint16_t *out,
+                           const float *alpha, const uint16_t *dh, int64_t R,
+                           int64_t C, int64_t ld, double eps, unsigned flags,
+                           double *dres, double *dout, double *dalpha,
+                           int nthreads);
 
 int or_l2_rows_interval(const uint16_t *x, const uint16_t *r, int64_t R,
                         int64_t C, int64_t ld, double eps, double delta,

@@ -41,6 +41,16 @@ def lib() -> ct.CDLL:
         _lib.or_grad_project_row.argtypes = [vp, vp, i64, dbl, uns, vp]
         _lib.or_grad_project_row.restype = None
         _lib.or_l2_rows.argtypes = [vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
+        _lib.or_l2_rows_backward.argtypes = [vp, vp, vp, i64, i64, i64, dbl, uns, vp, i32]
+        _lib.or_slerp_rows_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, vp, i32]
+        _lib.or_l2_row.argtypes = [vp, vp, i64, dbl, uns, vp, vp, vp]
+        _lib.or_l2_row.restype = None
+        _lib.or_slerp_row.argtypes = [vp, vp, vp, i64, dbl, uns, vp, vp, vp]
+        _lib.or_slerp_row.restype = None
+        _lib.or_l2_backward_row.argtypes = [vp, vp, vp, i64, dbl, uns, vp, vp]
+        _lib.or_l2_backward_row.restype = None
+        _lib.or_slerp_backward_row.argtypes = [vp, vp, vp, vp, i64, dbl, uns, vp, vp, vp, vp]
+        _lib.or_slerp_backward_row.restype = None
         _lib.or_slerp_rows.argtypes = [vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
         _lib.or_wn_backward_row.argtypes = [vp, vp, i64, dbl, dbl, dbl, uns, vp, vp]
         _lib.or_wn_forward_row.argtypes = [vp, i64, dbl, dbl, dbl, uns, vp]
@@ -163,6 +173,86 @@ def slerp_rows(res, out, alpha, *, eps=1e-6, flags=0, nthreads=1, exact=False):
     _check(lib().or_slerp_rows(_p(res), _p(out), _p(alpha), R, C, ld, eps, flags, _p(h), _p(he), nthreads),
            "slerp_rows")
     return (h, he) if exact else h
+
+
+def l2_rows_backward(x, r, dy, *, eps=1e-6, flags=0, nthreads=1):
+    """f64 dx [R, C] of l2_rows (x, r, dy: bf16 bits; r may be None).  With a
+    residual the same values are the gradient of r."""
+    x, ld = _rows(x, np.uint16)
+    R, C = x.shape
+    arrs = [x, np.ascontiguousarray(dy, np.uint16)] + ([] if r is None else [np.ascontiguousarray(r, np.uint16)])
+    if any(a.shape != (R, C) for a in arrs):
+        raise ValueError("shapes")
+    x = np.ascontiguousarray(x)
+    dy = arrs[1]
+    r = None if r is None else arrs[2]
+    dx = np.empty((R, C), np.float64)
+    _check(lib().or_l2_rows_backward(_p(x), _p(r), _p(dy), R, C, C, eps, flags, _p(dx), nthreads),
+           "l2_rows_backward")
+    return dx
+
+
+def slerp_rows_backward(res, out, alpha, dh, *, eps=1e-6, flags=0, nthreads=1, dalpha=True):
+    """f64 (dres, dout, dalpha | None) of slerp_rows (bf16 bits in)."""
+    res = np.ascontiguousarray(res, np.uint16)
+    out = np.ascontiguousarray(out, np.uint16)
+    dh = np.ascontiguousarray(dh, np.uint16)
+    R, C = res.shape
+    if out.shape != (R, C) or dh.shape != (R, C):
+        raise ValueError("shapes")
+    alpha = np.ascontiguousarray(alpha, np.float32)
+    if alpha.shape != (C,):
+        raise ValueError("alpha shape")
+    dres = np.empty((R, C), np.float64)
+    dout = np.empty((R, C), np.float64)
+    da = np.empty((C,), np.float64) if dalpha else None
+    _check(lib().or_slerp_rows_backward(_p(res), _p(out), _p(alpha), _p(dh), R, C, C, eps, flags, _p(dres),
+                                        _p(dout), _p(da), nthreads), "slerp_rows_backward")
+    return dres, dout, da
+
+
+def l2_row64(x, r=None, *, eps=1e-6, flags=0):
+    """One row with f64 inputs: the exact value before the output rounding."""
+    x = np.ascontiguousarray(x, np.float64)
+    r = None if r is None else np.ascontiguousarray(r, np.float64)
+    s = np.empty_like(x)
+    y = np.empty(x.shape, np.uint16)
+    ye = np.empty_like(x)
+    lib().or_l2_row(_p(x), _p(r), x.size, eps, flags, _p(s), _p(y), _p(ye))
+    return ye
+
+
+def slerp_row64(res, out, alpha, *, eps=1e-6, flags=0):
+    res = np.ascontiguousarray(res, np.float64)
+    out = np.ascontiguousarray(out, np.float64)
+    alpha = np.ascontiguousarray(alpha, np.float64)
+    tmp = np.empty(3 * res.size, np.float64)
+    h = np.empty(res.shape, np.uint16)
+    he = np.empty_like(res)
+    lib().or_slerp_row(_p(res), _p(out), _p(alpha), res.size, eps, flags, _p(tmp), _p(h), _p(he))
+    return he
+
+
+def l2_backward_row64(x, r, dy, *, eps=1e-6, flags=0):
+    x = np.ascontiguousarray(x, np.float64)
+    r = None if r is None else np.ascontiguousarray(r, np.float64)
+    dy = np.ascontiguousarray(dy, np.float64)
+    s = np.empty_like(x)
+    dx = np.empty_like(x)
+    lib().or_l2_backward_row(_p(x), _p(r), _p(dy), x.size, eps, flags, _p(s), _p(dx))
+    return dx
+
+
+def slerp_backward_row64(res, out, alpha, dh, *, eps=1e-6, flags=0):
+    res = np.ascontiguousarray(res, np.float64)
+    out = np.ascontiguousarray(out, np.float64)
+    alpha = np.ascontiguousarray(alpha, np.float64)
+    dh = np.ascontiguousarray(dh, np.float64)
+    tmp = np.empty(4 * res.size, np.float64)
+    dres, dout, da = np.empty_like(res), np.empty_like(res), np.empty_like(res)
+    lib().or_slerp_backward_row(_p(res), _p(out), _p(alpha), _p(dh), res.size, eps, flags, _p(tmp), _p(dres),
+                                _p(dout), _p(da))
+    return dres, dout, da
 
 
 def l2_rows_interval(x, r=None, *, eps=1e-6, delta=1e-5, flags=0, nthreads=1):
