@@ -2,7 +2,7 @@
  * ds.h -- C ABI of libds: per-row L2 normalisation of weight and activation
  * rows on NVIDIA B200 (sm_100a).
  *
- * Seven operations, each over a table of segments (matrices), so that every
+ * Nine operations, each over a table of segments (matrices), so that every
  * weight of a model is handled by one call:
  *
  *   ds_wn_forward   W_eff[r,:] = g_r * rho * w[r,:] / sqrt(sum_j w[r,j]^2 + eps)
@@ -34,6 +34,15 @@
  *                   t_j = a_j + |alpha_j| (b_j - a_j)  (fp32, one rounding),
  *                   y = bf16(t / sqrt(sum t^2 + eps)); same commit (tf_slerp_rows,
  *                   the normalised-lerp residual).
+ *   ds_l2_rows_backward, ds_slerp_rows_backward  the gradients of the two
+ *                   activation calls (derived: the pages give the forward only),
+ *                   straight through the bf16 rounding points, which keep the
+ *                   rounded values the forward uses:
+ *                   l2:    dx = (dy - s (s . dy) / n^2) / n   (= dr with a residual)
+ *                   slerp: dt = (dh - t (t . dh)/nt^2)/nt, da = (1-|alpha|) dt,
+ *                          db = |alpha| dt, dres = (da - res (res . da)/na^2)/na,
+ *                          dout likewise, dalpha_j = sum over rows of
+ *                          sign(alpha_j) (b_j - a_j) dt_j.
  *
  * Numerics: every row reduction accumulates in fp32 in an order fixed by the
  * row length and the operation alone, so a row's bits never depend on the
@@ -124,6 +133,26 @@ typedef struct {
     int64_t ld;   /* >= cols */
 } ds_aseg;
 
+/* One activation matrix for the backward calls.  x, r and dy share the
+ * leading dimension ld; dx and dr share ld_d.
+ *   l2_rows_backward:    x bf16, r bf16 residual or NULL, dy bf16 = dL/dy,
+ *                        dx fp32 = dL/dx (also dL/dr when r is set); dr ignored
+ *   slerp_rows_backward: x = res, r = out (both bf16, required), dy = dL/dh
+ *                        bf16, alpha fp32 [cols], dx = dL/dres and dr = dL/dout
+ *                        (fp32).  Outputs never overlap inputs. */
+typedef struct {
+    const void *x;
+    const void *r;
+    const void *dy;
+    float *dx;
+    float *dr;
+    const float *alpha;
+    int64_t rows; /* >= 0 */
+    int64_t cols; /* >= 1 */
+    int64_t ld;   /* >= cols, of x, r and dy */
+    int64_t ld_d; /* >= cols, of dx and dr  */
+} ds_agseg;
+
 /* out_dtype: DS_BF16 or DS_F32 for every segment's w_eff. */
 ds_status ds_wn_forward(const ds_wseg *segs, int nseg, ds_dtype out_dtype,
                         float eps, ds_stream stream);
@@ -155,6 +184,27 @@ ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps,
 ds_status ds_slerp_rows(const ds_aseg *segs, int nseg, float eps,
                         ds_stream stream);
 
+/* Rows must have at most 64 KB of staged input in the widest layout (x, r
+ * and dy, 48 bytes per 8 columns): at most 10,920 columns for either call;
+ * longer rows are refused with DS_ERR_INVALID_ARG. */
+ds_status ds_l2_rows_backward(const ds_agseg *segs, int nseg, float eps,
+                              ds_stream stream);
+
+/* dalpha: fp32 [cols] device output, or NULL to skip it.  With dalpha every
+ * segment must use the same alpha and cols, and `workspace` must be device
+ * memory of at least ds_slerp_rows_backward_workspace(cols) bytes, 256-byte
+ * aligned, owned by the caller and not touched by anything else until the
+ * call's work on `stream` ends (its contents on entry do not matter).  The
+ * column sums are deterministic: per-team partial sums in a fixed row order,
+ * then a second launch adds them in a fixed order. */
+ds_status ds_slerp_rows_backward(const ds_agseg *segs, int nseg, float eps,
+                                 float *dalpha, void *workspace,
+                                 uint64_t workspace_bytes, ds_stream stream);
+
+/* Workspace bytes ds_slerp_rows_backward needs for dalpha over rows of
+ * `cols` elements on the current device (0 if cols < 1). */
+uint64_t ds_slerp_rows_backward_workspace(int64_t cols);
+
 /* Static description of a status code. */
 const char *ds_status_string(ds_status status);
 
@@ -181,7 +231,9 @@ typedef enum {
     DS_OP_L2_ROWS = 3,
     DS_OP_SLERP_ROWS = 4,
     DS_OP_GRAD_PROJECT = 5,
-    DS_OP_RENORM_MOMENTUM = 6
+    DS_OP_RENORM_MOMENTUM = 6,
+    DS_OP_L2_ROWS_BACKWARD = 7,
+    DS_OP_SLERP_ROWS_BACKWARD = 8
 } ds_op;
 
 typedef enum {

@@ -21,8 +21,10 @@
 
 namespace {
 
+using ds::AGSegK;
 using ds::AParams;
 using ds::ASegK;
+using ds::GParams;
 using ds::RowClass;
 using ds::WParams;
 using ds::WSegK;
@@ -62,9 +64,13 @@ int64_t tile_row_bytes_worst(ds_op op, int64_t cols)
     case DS_OP_WN_BACKWARD:
     case DS_OP_GRAD_PROJECT:
     case DS_OP_RENORM_MOMENTUM: return 2 * q;
+    case DS_OP_L2_ROWS_BACKWARD:
+    case DS_OP_SLERP_ROWS_BACKWARD: return 3 * o;
     default: return 2 * o;
     }
 }
+
+bool is_act_bwd(ds_op op) { return op == DS_OP_L2_ROWS_BACKWARD || op == DS_OP_SLERP_ROWS_BACKWARD; }
 
 // Warps of a staged team: one (weights) or two (activations) per 16 KB of
 // slot; eight for the 112 KB weight slots.
@@ -72,7 +78,7 @@ int team_warps(ds_op op, int slot)
 {
     if (slot == ds::kTileSlotMaxWeightBytes)
         return 8;
-    const int base = (op == DS_OP_L2_ROWS || op == DS_OP_SLERP_ROWS) ? 2 : 1;
+    const int base = (op == DS_OP_L2_ROWS || op == DS_OP_SLERP_ROWS || is_act_bwd(op)) ? 2 : 1;
     return base * slot / ds::kTileSlotBytes;
 }
 
@@ -100,6 +106,16 @@ RowClass classify(ds_op op, int64_t cols, int forced)
                 return CL;
         return 0;
     };
+    if (is_act_bwd(op)) {
+        // staged classes only; longer rows are refused (path 0)
+        if (forced == DS_PATH_CTA && staged <= max_slot(op))
+            return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
+        if (staged <= ds::kTileSlotBytes)
+            return staged_class(DS_PATH_WARP, ds::kTileSlotBytes);
+        if (staged <= max_slot(op))
+            return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
+        return {0, 0, 0, 0, 0};
+    }
     switch (forced) {
     case DS_PATH_WARP:
         if (staged <= ds::kTileSlotBytes)
@@ -140,6 +156,8 @@ int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r, int slo
     case DS_OP_GRAD_PROJECT:
     case DS_OP_RENORM_MOMENTUM: bytes = 2 * q * 16; break;
     case DS_OP_L2_ROWS: bytes = o * 16 * (has_r ? 2 : 1); break;
+    case DS_OP_L2_ROWS_BACKWARD: bytes = o * 16 * (has_r ? 3 : 2); break;
+    case DS_OP_SLERP_ROWS_BACKWARD: bytes = o * 16 * 3; break;
     default: bytes = o * 32; break;
     }
     return static_cast<int>(std::min<int64_t>(ds::kTileMaxRowsPerSlot, slot / bytes));
@@ -254,7 +272,8 @@ ds_status check_matrix(const void *p, int64_t rows, int64_t ld, int esize, const
 // kTileAlphaCacheMax columns let the staged kernel keep |alpha| in shared
 // memory (the kernel checks the length against its own cache).
 inline void shared_alpha(WParams &p, int) { p.alpha_shared = nullptr; p.alpha_cols = 0; }
-inline void shared_alpha(AParams &p, int n)
+template <class P>
+inline void shared_alpha_act(P &p, int n)
 {
     p.alpha_shared = nullptr;
     p.alpha_cols = 0;
@@ -266,10 +285,18 @@ inline void shared_alpha(AParams &p, int n)
     p.alpha_shared = p.seg[0].alpha;
     p.alpha_cols = p.seg[0].cols;
 }
+inline void shared_alpha(AParams &p, int n) { shared_alpha_act(p, n); }
+inline void shared_alpha(GParams &p, int n) { shared_alpha_act(p, n); }
 
-template <class P, class SegK, class Make, class Launch>
+struct NoPrep {
+    template <class P>
+    void operator()(P &) const {}
+};
+
+// `prep(params)` runs on each packed parameter block just before its launch.
+template <class P, class SegK, class Make, class Launch, class Prep = NoPrep>
 ds_status launch_all(int nseg, const int64_t *rows, const std::vector<RowClass> &cls, float eps, Make make,
-                     Launch launch, void *stream)
+                     Launch launch, void *stream, Prep prep = Prep())
 {
     std::vector<char> done(static_cast<size_t>(nseg), 0);
 
@@ -289,6 +316,9 @@ ds_status launch_all(int nseg, const int64_t *rows, const std::vector<RowClass> 
             params.eps = eps;
             params.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
             shared_alpha(params, n);
+            params.ws = nullptr;
+            params.ws_ld = 0;
+            prep(params);
             const int e = launch(rc, params, units, stream);
             if (e != 0) {
                 char buf[160];
@@ -532,6 +562,148 @@ ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *st
     return launch_all<AParams, ASegK>(nseg, rows.data(), cls, eps, make, launch, stream);
 }
 
+AGSegK agseg_rows(const ds_agseg &s, int64_t r0, int64_t nr)
+{
+    AGSegK k{};
+    k.x = s.x ? static_cast<const uint16_t *>(s.x) + r0 * s.ld : nullptr;
+    k.r = s.r ? static_cast<const uint16_t *>(s.r) + r0 * s.ld : nullptr;
+    k.dy = s.dy ? static_cast<const uint16_t *>(s.dy) + r0 * s.ld : nullptr;
+    k.dx = s.dx ? s.dx + r0 * s.ld_d : nullptr;
+    k.dr = s.dr ? s.dr + r0 * s.ld_d : nullptr;
+    k.alpha = s.alpha;
+    k.rows = nr;
+    k.ld = s.ld;
+    k.ld_d = s.ld_d;
+    k.cols = static_cast<int32_t>(s.cols);
+    k.nu = static_cast<int32_t>((s.cols + 7) / 8);
+    return k;
+}
+
+// Floats per dalpha workspace line: the row's octets, 8 floats each.
+int64_t dalpha_ws_ld(int64_t cols) { return (cols + 7) / 8 * 8; }
+
+uint64_t dalpha_ws_bytes(int64_t cols)
+{
+    return static_cast<uint64_t>(sm_count()) * ds::kTileMaxGroups * static_cast<uint64_t>(dalpha_ws_ld(cols)) * 4u;
+}
+
+ds_status run_act_bwd(bool slerp, const ds_agseg *segs, int nseg, float eps, float *dalpha, void *ws,
+                      uint64_t ws_bytes, void *stream)
+{
+    g_last_error.clear();
+    if (ds_status s = check_common(nseg, segs, eps, stream))
+        return s;
+    const ds_op op = slerp ? DS_OP_SLERP_ROWS_BACKWARD : DS_OP_L2_ROWS_BACKWARD;
+    const int forced = g_force_path.load(std::memory_order_relaxed);
+    std::vector<Span> spans;
+    std::vector<int64_t> rows(static_cast<size_t>(nseg)), cols(static_cast<size_t>(nseg));
+    std::vector<RowClass> cls(static_cast<size_t>(nseg));
+    int64_t total_rows = 0;
+    for (int i = 0; i < nseg; ++i) {
+        const ds_agseg &s = segs[i];
+        if (ds_status st = check_shape(s.rows, s.cols, s.ld, i))
+            return st;
+        if (s.ld_d < s.cols)
+            return fail(DS_ERR_INVALID_ARG, where("ld_d < cols", i));
+        rows[i] = s.rows;
+        cols[i] = s.cols;
+        cls[i] = classify(op, s.cols, forced);
+        if (cls[i].path == 0)
+            return fail(DS_ERR_INVALID_ARG, where("row too long for the backward (more than 64 KB of staged input)", i));
+        if (s.rows == 0)
+            continue;
+        total_rows += s.rows;
+        if (ds_status st = check_matrix(s.x, s.rows, s.ld, 2, slerp ? "x (res)" : "x", i))
+            return st;
+        if (ds_status st = check_matrix(s.dy, s.rows, s.ld, 2, "dy", i))
+            return st;
+        if (ds_status st = check_matrix(s.dx, s.rows, s.ld_d, 4, "dx", i))
+            return st;
+        if (slerp || s.r)
+            if (ds_status st = check_matrix(s.r, s.rows, s.ld, 2, slerp ? "r (out)" : "r", i))
+                return st;
+        spans.push_back(span_of(s.x, s.rows, s.cols, s.ld, 2, i, 0, -1));
+        if (s.r)
+            spans.push_back(span_of(s.r, s.rows, s.cols, s.ld, 2, i, 0, -1));
+        spans.push_back(span_of(s.dy, s.rows, s.cols, s.ld, 2, i, 0, -1));
+        spans.push_back(span_of(s.dx, s.rows, s.cols, s.ld_d, 4, i, 1, -1));
+        if (slerp) {
+            if (ds_status st = check_matrix(s.dr, s.rows, s.ld_d, 4, "dr", i))
+                return st;
+            if (!s.alpha)
+                return fail(DS_ERR_INVALID_ARG, where("alpha is NULL", i));
+            if (!aligned(s.alpha, 16))
+                return fail(DS_ERR_ALIGNMENT, where("alpha is not 16-byte aligned", i));
+            spans.push_back(span_of(s.alpha, 1, s.cols, s.cols, 4, i, 0, -1));
+            spans.push_back(span_of(s.dr, s.rows, s.cols, s.ld_d, 4, i, 1, -1));
+        }
+    }
+    int64_t dcols = 0;
+    if (slerp && dalpha) {
+        // every segment shares alpha and cols, one launch covers them all
+        for (int i = 0; i < nseg; ++i)
+            if (segs[i].alpha != segs[0].alpha || segs[i].cols != segs[0].cols || !ds::same_launch(cls[i], cls[0]))
+                return fail(DS_ERR_INVALID_ARG, where("dalpha needs one alpha, one cols and one row class", i));
+        if (nseg > ds::kSegPerLaunch)
+            return fail(DS_ERR_INVALID_ARG, "dalpha: at most 128 segments");
+        dcols = nseg ? segs[0].cols : 0;
+        if (dcols > 0) {
+            if (!aligned(dalpha, 4))
+                return fail(DS_ERR_ALIGNMENT, "dalpha is not 4-byte aligned");
+            if (!ws || !aligned(ws, 256))
+                return fail(ws ? DS_ERR_ALIGNMENT : DS_ERR_INVALID_ARG, "workspace NULL or not 256-byte aligned");
+            if (ws_bytes < dalpha_ws_bytes(dcols))
+                return fail(DS_ERR_INVALID_ARG, "workspace smaller than ds_slerp_rows_backward_workspace(cols)");
+            spans.push_back(span_of(dalpha, 1, dcols, dcols, 4, -2, 1, -1));
+            spans.push_back({reinterpret_cast<uintptr_t>(ws), reinterpret_cast<uintptr_t>(ws) + ws_bytes, -3, 1, -1});
+        }
+    }
+    if (ds_status st = check_overlaps(spans))
+        return st;
+    for (int i = 0; i < nseg; ++i)
+        cls[i].rps = tile_rows_per_slot(op, cols[i], 2, segs[i].r != nullptr, cls[i].slot);
+    const int tag = slerp ? 10 : 9;
+    int grid_used = 0, groups_used = 0;
+    int64_t units_used = 0;
+    auto make = [&](int i, int64_t r0, int64_t nr) { return agseg_rows(segs[i], r0, nr); };
+    auto launch = [&](const RowClass &rc, const GParams &p, int64_t units, void *st) -> int {
+        const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
+        grid_used = grid;
+        groups_used = ds::tile_groups(tag, rc.slot);
+        units_used = units;
+        return ds::launch_tile(tag, &p, grid, rc.slot, st);
+    };
+    const bool want_dalpha = slerp && dalpha && dcols > 0;
+    auto prep = [&](GParams &p) {
+        if (want_dalpha) {
+            p.ws = static_cast<float *>(ws);
+            p.ws_ld = static_cast<int32_t>(dalpha_ws_ld(dcols));
+        }
+    };
+    const uint64_t before = g_launches.load(std::memory_order_relaxed);
+    if (ds_status st = launch_all<GParams, AGSegK>(nseg, rows.data(), cls, eps, make, launch, stream, prep))
+        return st;
+    if (want_dalpha) {
+        if (g_launches.load(std::memory_order_relaxed) - before > 1)
+            return fail(DS_ERR_INVALID_ARG, "dalpha: the rows need more than one launch");
+        if (total_rows == 0) {
+            // no rows: dalpha is zero
+            const cudaError_t e = cudaMemsetAsync(dalpha, 0, static_cast<size_t>(dcols) * 4,
+                                                  static_cast<cudaStream_t>(stream));
+            if (e != cudaSuccess)
+                return fail(DS_ERR_CUDA, "cudaMemsetAsync failed");
+            return DS_OK;
+        }
+        const int e = ds::launch_dalpha_reduce(static_cast<const float *>(ws), static_cast<int>(dalpha_ws_ld(dcols)),
+                                              grid_used, groups_used, units_used, static_cast<int>(dcols), dalpha,
+                                              stream);
+        if (e != 0)
+            return fail(DS_ERR_CUDA, "dalpha reduction launch failed");
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+    }
+    return DS_OK;
+}
+
 } // namespace
 
 extern "C" {
@@ -559,6 +731,24 @@ ds_status ds_grad_project(const ds_wseg *segs, int nseg, float eps, ds_stream st
 ds_status ds_renorm_momentum(const ds_wseg *segs, int nseg, float eps, ds_stream stream)
 {
     return run_weight(W_MOMENTUM, segs, nseg, DS_F32, eps, stream);
+}
+
+ds_status ds_l2_rows_backward(const ds_agseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_act_bwd(false, segs, nseg, eps, nullptr, nullptr, 0, stream);
+}
+
+ds_status ds_slerp_rows_backward(const ds_agseg *segs, int nseg, float eps, float *dalpha, void *workspace,
+                                 uint64_t workspace_bytes, ds_stream stream)
+{
+    return run_act_bwd(true, segs, nseg, eps, dalpha, workspace, workspace_bytes, stream);
+}
+
+uint64_t ds_slerp_rows_backward_workspace(int64_t cols)
+{
+    if (cols < 1 || cols > kMaxCols)
+        return 0;
+    return dalpha_ws_bytes(cols);
 }
 
 ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps, ds_stream stream)
@@ -610,11 +800,13 @@ int ds_version(void) { return 100; }
 
 ds_status ds_row_class(ds_op op, int64_t cols, int *path, int *group_threads, int *cluster_ctas)
 {
-    if (op < DS_OP_WN_FORWARD || op > DS_OP_RENORM_MOMENTUM)
+    if (op < DS_OP_WN_FORWARD || op > DS_OP_SLERP_ROWS_BACKWARD)
         return fail(DS_ERR_INVALID_ARG, "unknown op");
     if (cols < 1 || cols > kMaxCols)
         return fail(DS_ERR_INVALID_ARG, "cols outside [1, 2^31 - 1]");
     const RowClass rc = classify(op, cols, g_force_path.load(std::memory_order_relaxed));
+    if (rc.path == 0)
+        return fail(DS_ERR_INVALID_ARG, "row too long for the backward (more than 64 KB of staged input)");
     if (path)
         *path = rc.path;
     if (group_threads)

@@ -22,6 +22,8 @@ constexpr int kWarps = kCta / 32;
 // (backward: w and GY; l2 with residual; slerp: res and out).
 constexpr int kKmaxMax = 8;
 DS_HD constexpr int kmax_of(ds_op op) { return (op == DS_OP_WN_FORWARD || op == DS_OP_ROW_RENORM) ? 8 : 4; }
+// Largest number of ring positions of any staged launch (16 KB slots).
+constexpr int kTileMaxGroups = 13;
 // Largest cluster (portable limit).
 constexpr int kMaxCluster = 8;
 // Segments per launch (kernel parameter block); larger tables are split.
@@ -99,6 +101,23 @@ struct ASegK {
     int32_t pad_;
 };
 
+// Device copy of one activation segment of a backward call.
+struct AGSegK {
+    const uint16_t *x;
+    const uint16_t *r;
+    const uint16_t *dy;
+    float *dx;
+    float *dr;
+    const float *alpha;
+    int64_t rows;
+    int64_t ld;       // of x, r, dy (elements)
+    int64_t ld_d;     // of dx, dr (elements)
+    int32_t cols;
+    int32_t nu;
+    int32_t group;    // staged paths: rows per slot
+    int32_t pad_;
+};
+
 template <class Seg>
 struct LaunchParams {
     Seg seg[kSegPerLaunch];
@@ -108,11 +127,13 @@ struct LaunchParams {
     uint64_t wait_limit_ns;                // bound of every device-side wait
     const float *alpha_shared;             // slerp: alpha of every segment (or NULL if they differ)
     int32_t alpha_cols;                    //        its length
-    int32_t pad_;
+    int32_t ws_ld;                         // slerp backward: floats per workspace line
+    float *ws;                             //        per-team dalpha partial sums (NULL: no dalpha)
 };
 
 using WParams = LaunchParams<WSegK>;
 using AParams = LaunchParams<ASegK>;
+using GParams = LaunchParams<AGSegK>;
 
 // Error word written by kernels (see ds_get_device_status).
 enum DeviceErrorSite : uint32_t {
@@ -134,10 +155,17 @@ int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void 
 int launch_wait_selftest(uint64_t limit_ns, void *stream);
 // Staged paths (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,
 // 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp,
-// 7 gradient projection, 8 momentum projection + renorm; params is a WParams
-// (tags 0-4, 7, 8) or AParams (5-6) whose segments carry rows per slot in
-// `group` and whose unit_start counts slots; slot_bytes 16, 32 or 64 KB.
+// 7 gradient projection, 8 momentum projection + renorm, 9 l2 backward,
+// 10 slerp backward; params is a WParams (tags 0-4, 7, 8), AParams (5, 6) or
+// GParams (9, 10) whose segments carry rows per slot in `group` and whose
+// unit_start counts slots; slot_bytes 16, 32, 64 or (weights) 112 KB.
 int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream);
+// Ring positions (consumer teams) per CTA of a staged launch.
+int tile_groups(int tag, int slot_bytes);
+// dalpha[c] = sum over CTAs c0 < grid and their used teams q of
+// ws[(c0 * groups + q) * ws_ld + c], in that order (slerp backward).
+int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64_t total_units, int cols,
+                         float *dalpha, void *stream);
 int read_and_clear_device_error(uint32_t *code, uint32_t *site, void *stream);
 
 } // namespace ds

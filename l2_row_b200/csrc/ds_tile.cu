@@ -25,9 +25,11 @@
 namespace ds {
 
 // ds_kernels.cu's tags, repeated (the two files share this numbering).
-enum TileTag { tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp, tProject, tMomentum };
+enum TileTag { tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp, tProject, tMomentum, tL2Bwd, tSlerpBwd };
 
-__host__ __device__ constexpr bool is_weight_tag(int T) { return T <= tRenorm || T >= tProject; }
+__host__ __device__ constexpr bool is_weight_tag(int T) { return T <= tRenorm || T == tProject || T == tMomentum; }
+__host__ __device__ constexpr bool is_act_bwd_tag(int T) { return T == tL2Bwd || T == tSlerpBwd; }
+__host__ __device__ constexpr bool is_act_tag(int T) { return T == tL2 || T == tSlerp || is_act_bwd_tag(T); }
 
 namespace {
 
@@ -209,15 +211,15 @@ __device__ __forceinline__ void alpha_pairs(const float *alpha, int u, int cols,
 
 template <int T>
 struct TileLayout {
-    static constexpr int kArrays = (T == tFwdBf16 || T == tFwdF32 || T == tRenorm) ? 1 : 2;
-    // bytes per unit of array a
+    static constexpr int kArrays = (T == tFwdBf16 || T == tFwdF32 || T == tRenorm) ? 1 : is_act_bwd_tag(T) ? 3 : 2;
+    // bytes per unit of array a (the activation backward: x, r, dy)
     static __device__ __forceinline__ int ub(int a, bool has_r)
     {
         if (a == 0)
             return 16;
         if (T == tBwdBf16)
             return 8;
-        if (T == tL2)
+        if (T == tL2 || (T == tL2Bwd && a == 1))
             return has_r ? 16 : 0;
         return 16;
     }
@@ -238,8 +240,15 @@ __device__ __forceinline__ const char *tile_src(const ASegK &sg, int a, int64_t 
     return reinterpret_cast<const char *>((a == 0 ? sg.x : sg.r) + row * sg.ld);
 }
 
+template <int T>
+__device__ __forceinline__ const char *tile_src(const AGSegK &sg, int a, int64_t row)
+{
+    return reinterpret_cast<const char *>((a == 0 ? sg.x : a == 1 ? sg.r : sg.dy) + row * sg.ld);
+}
+
 __device__ __forceinline__ bool seg_has_r(const WSegK &) { return true; }
 __device__ __forceinline__ bool seg_has_r(const ASegK &s) { return s.r != nullptr; }
+__device__ __forceinline__ bool seg_has_r(const AGSegK &s) { return s.r != nullptr; }
 
 // Row pitch in global memory (bytes) of array a.
 template <int T>
@@ -250,6 +259,12 @@ __device__ __forceinline__ int64_t tile_src_pitch(const WSegK &sg, int a)
 
 template <int T>
 __device__ __forceinline__ int64_t tile_src_pitch(const ASegK &sg, int)
+{
+    return sg.ld * 2;
+}
+
+template <int T>
+__device__ __forceinline__ int64_t tile_src_pitch(const AGSegK &sg, int)
 {
     return sg.ld * 2;
 }
@@ -741,10 +756,308 @@ __device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, in
     }
 }
 
+// ===================================================== activation backward ==
+//
+// Derived gradients of the two activation calls, straight through their bf16
+// rounding points (which keep the rounded values the forward uses).  Inputs
+// come from the slot (x, r, dy bf16 as arrays 0, 1, 2); gradients go straight
+// to global memory in fp32.
+
+__device__ __forceinline__ void dot8(float2 &acc, uint4 a, uint4 b)
+{
+    acc = __ffma2_rn(lo2(a.x), lo2(b.x), acc);
+    acc = __ffma2_rn(lo2(a.y), lo2(b.y), acc);
+    acc = __ffma2_rn(lo2(a.z), lo2(b.z), acc);
+    acc = __ffma2_rn(lo2(a.w), lo2(b.w), acc);
+}
+
+__device__ __forceinline__ uint32_t word4(uint4 v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+// Eight fp32 values of one unit to row `o` at unit u (two 16-byte stores),
+// or only its first `valid` elements.
+__device__ __forceinline__ void store8f(float *o, int u, const float2 (&v)[4], int valid)
+{
+    if (valid >= 8) {
+        st16(o + 8 * u, make_uint4(__float_as_uint(v[0].x), __float_as_uint(v[0].y), __float_as_uint(v[1].x),
+                                   __float_as_uint(v[1].y)));
+        st16(o + 8 * u + 4, make_uint4(__float_as_uint(v[2].x), __float_as_uint(v[2].y), __float_as_uint(v[3].x),
+                                       __float_as_uint(v[3].y)));
+    } else {
+        for (int e = 0; e < valid; ++e)
+            o[8 * u + e] = (e & 1) ? v[e >> 1].y : v[e >> 1].x;
+    }
+}
+
+// l2 backward: s = x or bf16(x + r) (written back over x, as in the
+// forward), S = sum s^2 and D = sum s dy in one pass, then
+// dx = (dy - s D/(S+eps)) / sqrt(S+eps).  Rows needing the power-of-two
+// rescale re-sum with s scaled by 2^m and apply the scaled quotient to the
+// scaled row (exactly the unscaled product), with 2^m carried into 1/n.
+template <int WP, bool HAS_R>
+__device__ __forceinline__ void tile_l2_bwd_row(Team<WP> &tm, const AGSegK &sg, int64_t row, unsigned char *s0,
+                                                const unsigned char *s1, unsigned char *s2, int nfull, int tail,
+                                                float eps, bool store)
+{
+    constexpr int G = Team<WP>::G;
+    const int t = tm.t;
+    const bool tl = tail && t == nfull % G;
+    const int nunits = nfull + (tail ? 1 : 0);
+    uint4 *x = reinterpret_cast<uint4 *>(s0);
+    const uint4 *r = reinterpret_cast<const uint4 *>(s1);
+    uint4 *dy = reinterpret_cast<uint4 *>(s2);
+    float2 as = f2(0.f, 0.f), ad = f2(0.f, 0.f);
+#pragma unroll 4
+    for (int u = t; u < nfull; u += G) {
+        const uint4 sv = l2_unit_s<HAS_R>(x, r, u);
+        if constexpr (HAS_R)
+            x[u] = sv;
+        sq8w(as, sv);
+        dot8(ad, sv, dy[u]);
+    }
+    if (tl) {
+        const uint4 sv = mask_octet(l2_unit_s<HAS_R>(x, r, nfull), tail);
+        const uint4 d = mask_octet(dy[nfull], tail);
+        x[nfull] = sv;
+        dy[nfull] = d;
+        sq8w(as, sv);
+        dot8(ad, sv, d);
+    }
+    float sd[2] = {as.x + as.y, ad.x + ad.y};
+    tm.sum(sd);
+    float S = sd[0], D = sd[1];
+    int m = 0;
+    if (needs_rescale(S, eps)) {
+        float M = 0.f;
+        for (int u = t; u < nunits; u += G)
+            pairs8(x[u], [&](float2 v) { M = fmaxf(M, fmaxf(fabsf(v.x), fabsf(v.y))); });
+        M = tm.max(M);
+        if (M > 0.f && M < __int_as_float(0x7f800000)) {
+            m = 48 - ilogbf(M);
+            float2 bs = f2(0.f, 0.f), bd = f2(0.f, 0.f);
+            for (int u = t; u < nunits; u += G) {
+                const uint4 sv = x[u], d = dy[u];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 v = lo2(word4(sv, i));
+                    const float2 w2 = f2(scalbnf(v.x, m), scalbnf(v.y, m));
+                    sq2(bs, w2);
+                    bd = __ffma2_rn(w2, lo2(word4(d, i)), bd);
+                }
+            }
+            float sd2[2] = {bs.x + bs.y, bd.x + bd.y};
+            tm.sum(sd2);
+            S = sd2[0];
+            D = sd2[1];
+        }
+    }
+    if (!store)
+        return;
+    const float n2 = S + (m == 0 ? eps : scalbnf(eps, 2 * m));
+    const float inv = 1.0f / sqrtf(n2);
+    const float2 nq = f2(-D / n2, -D / n2);                      // -D/(S+eps) times 2^-m
+    const float os = m == 0 ? inv : scalbnf(inv, m);              // 1/n
+    const float2 os2 = f2(os, os);
+    float *o = sg.dx + row * sg.ld_d;
+#pragma unroll 2
+    for (int u = t; u < nunits; u += G) {
+        const uint4 sv = x[u], d = dy[u];
+        float2 v[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float2 sp = lo2(word4(sv, i));
+            if (m != 0)
+                sp = f2(scalbnf(sp.x, m), scalbnf(sp.y, m));
+            v[i] = __fmul2_rn(__ffma2_rn(sp, nq, lo2(word4(d, i))), os2);
+        }
+        store8f(o, u, v, u < nfull ? 8 : tail);
+    }
+}
+
+// alpha of unit u as four pairs, signed: from the cache (split layout) or
+// from global memory (0 past cols).
+template <bool CACHED>
+__device__ __forceinline__ void alpha8_signed(const float *cache, int half, const float *alpha, int u, int cols,
+                                              float2 (&m)[4])
+{
+    if constexpr (CACHED) {
+        const float4 m0 = *reinterpret_cast<const float4 *>(cache + 4 * u);
+        const float4 m1 = *reinterpret_cast<const float4 *>(cache + half + 4 * u);
+        m[0] = f2(m0.x, m0.y);
+        m[1] = f2(m0.z, m0.w);
+        m[2] = f2(m1.x, m1.y);
+        m[3] = f2(m1.z, m1.w);
+    } else {
+        const int e0 = 8 * u;
+        const float4 a = e0 < cols ? __ldg(reinterpret_cast<const float4 *>(alpha + e0)) : make_float4(0, 0, 0, 0);
+        const float4 b = e0 + 4 < cols ? __ldg(reinterpret_cast<const float4 *>(alpha + e0 + 4))
+                                       : make_float4(0, 0, 0, 0);
+        m[0] = f2(a.x, a.y);
+        m[1] = f2(a.z, a.w);
+        m[2] = f2(b.x, b.y);
+        m[3] = f2(b.z, b.w);
+        if (e0 + 8 > cols) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                m[i] = f2(e0 + 2 * i < cols ? m[i].x : 0.f, e0 + 2 * i + 1 < cols ? m[i].y : 0.f);
+        }
+    }
+}
+
+__device__ __forceinline__ float2 abs2(float2 v) { return f2(fabsf(v.x), fabsf(v.y)); }
+__device__ __forceinline__ float2 sgn2(float2 v)
+{
+    return f2(v.x > 0.f ? 1.f : v.x < 0.f ? -1.f : 0.f, v.y > 0.f ? 1.f : v.y < 0.f ? -1.f : 0.f);
+}
+
+// slerp backward.  Pass 1 sums res^2 and out^2; pass 2 forms a, b and t as
+// the forward does and sums t^2 and t . dh; pass 3 forms
+// dt = (dh - t (t . dh)/nt^2)/nt, da = (1 - |alpha|) dt, db = |alpha| dt and
+// sums ua . da, ub . db (ua = res/na, ub = out/nb before their rounding),
+// adding this row's sign(alpha) (b - a) dt to the team's dalpha line; pass 4
+// stores dres = (da - ua (ua . da)) / na and dout likewise.  t, dt and the
+// rest are recomputed from the slot in each pass.
+template <int WP, bool CACHED>
+__device__ __forceinline__ void tile_slerp_bwd_row(Team<WP> &tm, const AGSegK &sg, int64_t row, unsigned char *s0,
+                                                   unsigned char *s1, unsigned char *s2, int nfull, int tail, float eps,
+                                                   bool store, const float *acache, int half, float *wsl,
+                                                   bool ws_first)
+{
+    constexpr int G = Team<WP>::G;
+    const int t = tm.t;
+    const bool tl = tail && t == nfull % G;
+    const int nunits = nfull + (tail ? 1 : 0);
+    uint4 *xa = reinterpret_cast<uint4 *>(s0);
+    uint4 *xb = reinterpret_cast<uint4 *>(s1);
+    uint4 *xd = reinterpret_cast<uint4 *>(s2);
+    // pass 1
+    float2 aa = f2(0.f, 0.f), ab = f2(0.f, 0.f);
+#pragma unroll 2
+    for (int u = t; u < nfull; u += G) {
+        sq8(aa, xa[u]);
+        sq8(ab, xb[u]);
+    }
+    if (tl) {
+        const uint4 p = mask_octet(xa[nfull], tail), q = mask_octet(xb[nfull], tail);
+        xa[nfull] = p;
+        xb[nfull] = q;
+        xd[nfull] = mask_octet(xd[nfull], tail);
+        sq8(aa, p);
+        sq8(ab, q);
+    }
+    float sab[2] = {aa.x + aa.y, ab.x + ab.y};
+    tm.sum(sab);
+    const RowScale ra = tile_scale(tm, sab[0], eps, [&](auto f) {
+        for (int u = t; u < nunits; u += G)
+            pairs8(xa[u], f);
+    });
+    const RowScale rb = tile_scale(tm, sab[1], eps, [&](auto f) {
+        for (int u = t; u < nunits; u += G)
+            pairs8(xb[u], f);
+    });
+    // per unit: the forward's a, b (bf16), t (fp32), |alpha| pairs
+    auto unit_t = [&](int u, uint4 &a, uint4 &b, float2 (&al)[4], float2 (&tv)[4]) {
+        a = scale8(xa[u], ra);
+        b = scale8(xb[u], rb);
+        alpha8_signed<CACHED>(acache, half, sg.alpha, u, sg.cols, al);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            tv[i] = lerp2(lo2(word4(a, i)), lo2(word4(b, i)), abs2(al[i]));
+    };
+    // pass 2
+    float2 st = f2(0.f, 0.f), dt2 = f2(0.f, 0.f);
+#pragma unroll 2
+    for (int u = t; u < nunits; u += G) {
+        uint4 a, b;
+        float2 al[4], tv[4];
+        unit_t(u, a, b, al, tv);
+        const uint4 d = xd[u];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            sq2(st, tv[i]);
+            dt2 = __ffma2_rn(tv[i], lo2(word4(d, i)), dt2);
+        }
+    }
+    float sd[2] = {st.x + st.y, dt2.x + dt2.y};
+    tm.sum(sd);
+    const float nt2 = sd[0] + eps;
+    const float it = 1.0f / sqrtf(nt2);
+    const float2 nqt = f2(-sd[1] / nt2, -sd[1] / nt2), it2 = f2(it, it);
+    const float2 pa = f2(ra.pre, ra.pre), ia = f2(ra.inv, ra.inv);
+    const float2 pb = f2(rb.pre, rb.pre), ib = f2(rb.inv, rb.inv);
+    const float2 one = f2(1.f, 1.f);
+    // ua, ub: res/na and out/nb before the rounding, the forward's product
+    auto unit_u = [&](uint4 raw, float2 pp, float2 ii, int i) {
+        const float2 v = lo2(word4(raw, i));
+        return pp.x == 1.f ? __fmul2_rn(v, ii) : __fmul2_rn(__fmul2_rn(v, pp), ii);
+    };
+    // pass 3
+    float2 sa = f2(0.f, 0.f), sb = f2(0.f, 0.f);
+#pragma unroll 1
+    for (int u = t; u < nunits; u += G) {
+        uint4 a, b;
+        float2 al[4], tv[4];
+        unit_t(u, a, b, al, tv);
+        const uint4 d = xd[u], rr = xa[u], oo = xb[u];
+        float2 part[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 m = abs2(al[i]);
+            const float2 dt = __fmul2_rn(__ffma2_rn(tv[i], nqt, lo2(word4(d, i))), it2);
+            const float2 da = __fmul2_rn(__fadd2_rn(one, fneg2(m)), dt), db = __fmul2_rn(m, dt);
+            sa = __ffma2_rn(unit_u(rr, pa, ia, i), da, sa);
+            sb = __ffma2_rn(unit_u(oo, pb, ib, i), db, sb);
+            const float2 ba = __fadd2_rn(lo2(word4(b, i)), fneg2(lo2(word4(a, i))));
+            part[i] = __fmul2_rn(__fmul2_rn(sgn2(al[i]), ba), dt);
+        }
+        if (wsl != nullptr && store) {
+            float4 *l = reinterpret_cast<float4 *>(wsl + 8 * u);
+            float4 p0 = make_float4(part[0].x, part[0].y, part[1].x, part[1].y);
+            float4 p1 = make_float4(part[2].x, part[2].y, part[3].x, part[3].y);
+            if (!ws_first) {
+                const float4 o0 = l[0], o1 = l[1];
+                p0 = make_float4(o0.x + p0.x, o0.y + p0.y, o0.z + p0.z, o0.w + p0.w);
+                p1 = make_float4(o1.x + p1.x, o1.y + p1.y, o1.z + p1.z, o1.w + p1.w);
+            }
+            l[0] = p0;
+            l[1] = p1;
+        }
+    }
+    float sab2[2] = {sa.x + sa.y, sb.x + sb.y};
+    tm.sum(sab2);
+    if (!store)
+        return;
+    // pass 4
+    const float2 nDa = f2(-sab2[0], -sab2[0]), nDb = f2(-sab2[1], -sab2[1]);
+    const float ra_n = ra.inv * ra.pre, rb_n = rb.inv * rb.pre;      // 1/na, 1/nb
+    const float2 ra2 = f2(ra_n, ra_n), rb2 = f2(rb_n, rb_n);
+    float *odx = sg.dx + row * sg.ld_d;
+    float *odr = sg.dr + row * sg.ld_d;
+#pragma unroll 1
+    for (int u = t; u < nunits; u += G) {
+        uint4 a, b;
+        float2 al[4], tv[4];
+        unit_t(u, a, b, al, tv);
+        const uint4 d = xd[u], rr = xa[u], oo = xb[u];
+        float2 gx[4], gr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 m = abs2(al[i]);
+            const float2 dt = __fmul2_rn(__ffma2_rn(tv[i], nqt, lo2(word4(d, i))), it2);
+            const float2 da = __fmul2_rn(__fadd2_rn(one, fneg2(m)), dt), db = __fmul2_rn(m, dt);
+            gx[i] = __fmul2_rn(__ffma2_rn(unit_u(rr, pa, ia, i), nDa, da), ra2);
+            gr[i] = __fmul2_rn(__ffma2_rn(unit_u(oo, pb, ib, i), nDb, db), rb2);
+        }
+        const int valid = u < nfull ? 8 : tail;
+        store8f(odx, u, gx, valid);
+        store8f(odr, u, gr, valid);
+    }
+}
+
 // =============================================================== kernel ==
 
 template <int T>
-using TParams = typename std::conditional<is_weight_tag(T), WParams, AParams>::type;
+using TParams = typename std::conditional<is_weight_tag(T), WParams,
+                                          typename std::conditional<is_act_bwd_tag(T), GParams, AParams>::type>::type;
 
 // Ring shape per operation and slot size SB (16, 32 or 64 KB of staged
 // input per slot; 112 KB for weight rows).  A position is owned by a team
@@ -760,12 +1073,12 @@ struct TileCfg {
     static_assert(SB != 114688 || is_weight_tag(T), "112 KB slots: weight rows only");
     static constexpr int kSlotBytes = SB;
     static constexpr int kScale = SB == 114688 ? 8 : SB / 16384;    // 1, 2, 4; 8 for 112 KB
-    static constexpr int kWP = ((T == tL2 || T == tSlerp) ? 2 : 1) * kScale;
+    static constexpr int kWP = (is_act_tag(T) ? 2 : 1) * kScale;
     static constexpr int kGroups = SB == 16384 ? 13 : SB == 32768 ? 6 : SB == 65536 ? 3 : 2;
     static constexpr int kSlots = kGroups;                          // one position per team
     static constexpr int kConsumers = kWP * kGroups;
     static constexpr int kThreads = (kConsumers + 1) * 32;
-    static constexpr int kAlphaCache = T == tSlerp ? (SB == 16384 ? 4096 : 8192) : 0;
+    static constexpr int kAlphaCache = (T == tSlerp || T == tSlerpBwd) ? (SB == 16384 ? 4096 : 8192) : 0;
     // Refill pacing: the producer sleeps this long after each refill.  For
     // the operations below a paced read stream ran faster on B200 (l2 rows
     // with a residual 74 -> 67 us, the momentum projection + renorm 274 ->
@@ -808,7 +1121,7 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
         abort_flag = 0;
         mbar_init_fence();
     }
-    if constexpr (T == tSlerp) {
+    if constexpr (T == tSlerp || T == tSlerpBwd) {
         // |alpha| split by halves of each 8-element unit: unit u's first four
         // at [4u], its last four at [half + 4u], so that a warp reading one
         // float4 per lane touches consecutive 16-byte words (no bank conflict)
@@ -816,7 +1129,9 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
             const int nu = (p.alpha_cols + 7) / 8, half = Cfg::kAlphaCache / 2;
             for (int i = threadIdx.x; i < 8 * nu; i += blockDim.x) {
                 const int u = i >> 3, e = i & 7;
-                const float v = i < p.alpha_cols ? fabsf(__ldg(p.alpha_shared + i)) : 0.f;
+                // the backward keeps the sign (dalpha needs it); the forward |alpha|
+                const float a = i < p.alpha_cols ? __ldg(p.alpha_shared + i) : 0.f;
+                const float v = T == tSlerpBwd ? a : fabsf(a);
                 s_alpha[(e < 4 ? 0 : half) + 4 * u + (e & 3)] = v;
             }
         }
@@ -838,10 +1153,18 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
             int si = -1;
             int64_t seg_begin = 0, seg_end = 0, seg_rows = 0;
             int rps = 1;
-            uint32_t pitch[2] = {0u, 0u}, off1 = 0u;
-            const char *src[2] = {nullptr, nullptr};
-            int64_t spitch[2] = {0, 0};
-            bool contig[2] = {false, false};
+            constexpr int NA = Layout::kArrays;
+            uint32_t pitch[NA], off[NA];
+            const char *src[NA];
+            int64_t spitch[NA];
+            bool contig[NA];
+#pragma unroll
+            for (int a2 = 0; a2 < NA; ++a2) {
+                pitch[a2] = off[a2] = 0u;
+                src[a2] = nullptr;
+                spitch[a2] = 0;
+                contig[a2] = false;
+            }
             int s = 0;
             uint32_t phase = 0;             // parity of the release a refill of position s waits for
             int64_t slot = blockIdx.x;
@@ -861,26 +1184,32 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                     seg_rows = sg.rows;
                     rps = sg.group;         // rows per slot for this segment
                     const bool has_r = seg_has_r(sg);
+                    uint32_t o = 0u;
 #pragma unroll
-                    for (int a2 = 0; a2 < 2; ++a2) {
-                        const int u = a2 < Layout::kArrays ? Layout::ub(a2, has_r) : 0;
+                    for (int a2 = 0; a2 < NA; ++a2) {
+                        const int u = Layout::ub(a2, has_r);
                         pitch[a2] = (static_cast<uint32_t>(sg.nu) * u + 15u) & ~15u;
                         src[a2] = pitch[a2] ? tile_src<T>(sg, a2, 0) : nullptr;
                         spitch[a2] = tile_src_pitch<T>(sg, a2);
                         contig[a2] = spitch[a2] == static_cast<int64_t>(pitch[a2]);
+                        off[a2] = o;
+                        o += pitch[a2] * rps;
                     }
-                    off1 = pitch[0] * rps;
                 }
                 const int64_t row0 = (slot - seg_begin) * rps;
                 const int nrows = static_cast<int>(seg_rows - row0 < rps ? seg_rows - row0 : rps);
                 hdr[s] = SlotHdr{si, nrows, row0};
                 unsigned char *dst = ring + static_cast<size_t>(s) * slot_bytes;
-                mbar_arrive_expect_tx(&full[s], (pitch[0] + pitch[1]) * nrows);
+                uint32_t row_bytes = 0u;
 #pragma unroll
-                for (int a2 = 0; a2 < 2; ++a2) {
+                for (int a2 = 0; a2 < NA; ++a2)
+                    row_bytes += pitch[a2];
+                mbar_arrive_expect_tx(&full[s], row_bytes * nrows);
+#pragma unroll
+                for (int a2 = 0; a2 < NA; ++a2) {
                     if (!pitch[a2])
                         continue;
-                    unsigned char *d = dst + (a2 == 0 ? 0u : off1);
+                    unsigned char *d = dst + off[a2];
                     const char *g = src[a2] + row0 * spitch[a2];
                     if (contig[a2]) {
                         bulk_g2s(d, g, pitch[a2] * nrows, &full[s]);
@@ -907,6 +1236,7 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
         const int q = warp / WP, wi = warp % WP;
         Team<WP> tm{wi * 32 + lane, 1 + q, red + q * Team<WP>::kRed};
         bool store = true;
+        bool ws_first = true; // slerp backward: this team's dalpha line not yet written
         int vb = 0;
         for (int64_t j = q; j < mine; j += NG, vb ^= 1) {
             const int s = static_cast<int>(j % nslots);
@@ -937,9 +1267,12 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
             const int rps = sg.group;
             unsigned char *base = ring + static_cast<size_t>(s) * slot_bytes;
             const int u0 = Layout::ub(0, has_r), u1 = Layout::kArrays > 1 ? Layout::ub(1, has_r) : 0;
+            const int u2 = Layout::kArrays > 2 ? Layout::ub(2, has_r) : 0;
             const int pitch0 = (sg.nu * u0 + 15) & ~15;
             const int pitch1 = (sg.nu * u1 + 15) & ~15;
+            const int pitch2 = (sg.nu * u2 + 15) & ~15;
             unsigned char *a1 = base + pitch0 * rps;
+            unsigned char *a2p = a1 + pitch1 * rps;
             constexpr int E = is_weight_tag(T) ? 4 : 8;
             const int nfull = sg.cols / E, tail = sg.cols % E;
             // hand the position back: the slot may hold this warp's
@@ -958,6 +1291,7 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                 const int64_t row = h.row0 + r;
                 unsigned char *s0 = base + r * pitch0;
                 unsigned char *s1 = a1 + r * pitch1;
+                unsigned char *s2 = a2p + r * pitch2;
                 if constexpr (T == tFwdBf16 || T == tFwdF32 || T == tBwdBf16 || T == tBwdF32) {
                     // gains of the next 32 rows, one per lane
                     if ((r & 31) == 0)
@@ -983,6 +1317,20 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                         tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
                     else
                         tile_l2_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
+                } else if constexpr (T == tL2Bwd) {
+                    if (has_r)
+                        tile_l2_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
+                    else
+                        tile_l2_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
+                } else if constexpr (T == tSlerpBwd) {
+                    float *wsl = p.ws ? p.ws + (static_cast<int64_t>(blockIdx.x) * NG + q) * p.ws_ld : nullptr;
+                    if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache)
+                        tile_slerp_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, s_alpha,
+                                                     Cfg::kAlphaCache / 2, wsl, ws_first);
+                    else
+                        tile_slerp_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, nullptr, 0,
+                                                      wsl, ws_first);
+                    ws_first = false;
                 } else if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache) {
                     tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
                                              Cfg::kAlphaCache / 2);
@@ -1045,8 +1393,61 @@ int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *str
     case tSlerp: return launch_tile_t<tSlerp>(params, grid, slot_bytes, stream);
     case tProject: return launch_tile_t<tProject>(params, grid, slot_bytes, stream);
     case tMomentum: return launch_tile_t<tMomentum>(params, grid, slot_bytes, stream);
+    case tL2Bwd: return launch_tile_t<tL2Bwd>(params, grid, slot_bytes, stream);
+    case tSlerpBwd: return launch_tile_t<tSlerpBwd>(params, grid, slot_bytes, stream);
     default: return cudaErrorInvalidValue;
     }
+}
+
+template <int T>
+static int tile_groups_t(int slot_bytes)
+{
+    switch (slot_bytes) {
+    case 16384: return TileCfg<T, 16384>::kGroups;
+    case 32768: return TileCfg<T, 32768>::kGroups;
+    case 65536: return TileCfg<T, 65536>::kGroups;
+    default: return 0;
+    }
+}
+
+int tile_groups(int tag, int slot_bytes)
+{
+    switch (tag) {
+    case tL2Bwd: return tile_groups_t<tL2Bwd>(slot_bytes);
+    case tSlerpBwd: return tile_groups_t<tSlerpBwd>(slot_bytes);
+    default: return 0;
+    }
+}
+
+namespace {
+
+// dalpha of the slerp backward: column c sums the used teams' lines, CTA by
+// CTA and team by team (a fixed order, so the result is deterministic).  A
+// CTA's team q was used iff it took a slot: q < the CTA's slot count.
+__global__ void __launch_bounds__(256) k_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups,
+                                                       int64_t total_units, int cols, float *dalpha)
+{
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= cols)
+        return;
+    float acc = 0.f;
+    for (int cta = 0; cta < grid; ++cta) {
+        const int64_t mine = total_units > cta ? (total_units - 1 - cta) / grid + 1 : 0;
+        const int used = mine < groups ? static_cast<int>(mine) : groups;
+        for (int q = 0; q < used; ++q)
+            acc += ws[(static_cast<int64_t>(cta) * groups + q) * ws_ld + c];
+    }
+    dalpha[c] = acc;
+}
+
+} // namespace
+
+int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64_t total_units, int cols,
+                         float *dalpha, void *stream)
+{
+    k_dalpha_reduce<<<(cols + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(ws, ws_ld, grid, groups,
+                                                                                    total_units, cols, dalpha);
+    return cudaGetLastError();
 }
 
 } // namespace ds

@@ -13,6 +13,8 @@ The five calls keep their C names and take lists of segments:
     ds_renorm_momentum(segs, eps, stream=None)    (grad_w = the momentum, in place)
     ds_l2_rows(segs, eps, stream=None)
     ds_slerp_rows(segs, eps, stream=None)
+    ds_l2_rows_backward(segs, eps, stream=None)
+    ds_slerp_rows_backward(segs, eps, dalpha=None, workspace=None, stream=None)
 
 A segment is a ``WSeg`` / ``ASeg`` of CUDA tensors (2-D, unit column stride,
 row stride = leading dimension) or a raw ``ds_wseg`` / ``ds_aseg`` structure.
@@ -39,6 +41,7 @@ DS_ERR_TOO_MANY_SEGMENTS, DS_ERR_CUDA, DS_ERR_DEVICE_TIMEOUT, DS_ERR_OVERLAP = 4
 DS_F32, DS_BF16 = 0, 1
 DS_OP_WN_FORWARD, DS_OP_WN_BACKWARD, DS_OP_ROW_RENORM, DS_OP_L2_ROWS, DS_OP_SLERP_ROWS = range(5)
 DS_OP_GRAD_PROJECT, DS_OP_RENORM_MOMENTUM = 5, 6
+DS_OP_L2_ROWS_BACKWARD, DS_OP_SLERP_ROWS_BACKWARD = 7, 8
 DS_PATH_AUTO, DS_PATH_WARP, DS_PATH_CTA, DS_PATH_CLUSTER, DS_PATH_TWO_PASS = range(5)
 DS_MAX_SEGMENTS = 65536
 PATH_NAMES = {DS_PATH_WARP: "warp", DS_PATH_CTA: "cta", DS_PATH_CLUSTER: "cluster", DS_PATH_TWO_PASS: "two_pass"}
@@ -55,6 +58,12 @@ class ds_aseg(ct.Structure):
                 ("rows", ct.c_int64), ("cols", ct.c_int64), ("ld", ct.c_int64)]
 
 
+class ds_agseg(ct.Structure):
+    _fields_ = [("x", ct.c_void_p), ("r", ct.c_void_p), ("dy", ct.c_void_p), ("dx", ct.c_void_p),
+                ("dr", ct.c_void_p), ("alpha", ct.c_void_p), ("rows", ct.c_int64), ("cols", ct.c_int64),
+                ("ld", ct.c_int64), ("ld_d", ct.c_int64)]
+
+
 _st = ct.c_int
 _lib.ds_wn_forward.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_wn_backward.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_int, ct.c_float, ct.c_void_p]
@@ -63,8 +72,13 @@ _lib.ds_grad_project.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, ct.c
 _lib.ds_renorm_momentum.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_l2_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_slerp_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_l2_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_slerp_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p, ct.c_void_p,
+                                        ct.c_uint64, ct.c_void_p]
+_lib.ds_slerp_rows_backward_workspace.argtypes = [ct.c_int64]
+_lib.ds_slerp_rows_backward_workspace.restype = ct.c_uint64
 for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
-           "ds_l2_rows", "ds_slerp_rows",
+           "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
            "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
            "ds_debug_wait_timeout_selftest"):
     getattr(_lib, _f).restype = _st
@@ -85,8 +99,8 @@ _lib.ds_debug_wait_timeout_selftest.argtypes = [ct.c_uint64, ct.c_void_p]
 
 #: every symbol include/ds.h declares
 EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
-           "ds_l2_rows", "ds_slerp_rows",
-           "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
+           "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
+           "ds_slerp_rows_backward_workspace", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
            "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest")
 
 
@@ -203,6 +217,34 @@ class ASeg:
         return ds_aseg(x, r, y, _vec(self.alpha), R, C, ld)
 
 
+@dataclass
+class AGSeg:
+    """One activation matrix for the backward calls: x (slerp: res), r (l2:
+    residual or None; slerp: out), dy the upstream gradient (bf16 [R, C],
+    shared ld), dx (and for slerp dr) fp32 [R, C] outputs with a shared ld,
+    alpha fp32 [C] (slerp)."""
+
+    x: Any
+    dy: Any
+    dx: Any
+    r: Any = None
+    dr: Any = None
+    alpha: Any = None
+
+    def to_c(self) -> ds_agseg:
+        R, C = (int(self.x.shape[0]), int(self.x.shape[1]))
+        x, ld = _mat(self.x, "x", R, C)
+        dy, ldy = _mat(self.dy, "dy", R, C)
+        r, ldr = _mat(self.r, "r", R, C)
+        dx, ldd = _mat(self.dx, "dx", R, C)
+        dr, lddr = _mat(self.dr, "dr", R, C)
+        if ldy != ld or (self.r is not None and ldr != ld):
+            raise ValueError("x, r and dy must share a leading dimension")
+        if self.dr is not None and lddr != ldd:
+            raise ValueError("dx and dr must share a leading dimension")
+        return ds_agseg(x, r, dy, dx, dr, _vec(self.alpha), R, C, ld, ldd)
+
+
 def _table(segs, cls):
     items = [s if isinstance(s, cls) else s.to_c() for s in segs]
     arr = (cls * max(1, len(items)))(*items)
@@ -242,6 +284,35 @@ def ds_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
 def ds_slerp_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
     arr, n = _table(segs, ds_aseg)
     _check(_lib.ds_slerp_rows(arr, n, eps, _stream_ptr(stream)), "ds_slerp_rows")
+
+
+def ds_l2_rows_backward(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_agseg)
+    _check(_lib.ds_l2_rows_backward(arr, n, eps, _stream_ptr(stream)), "ds_l2_rows_backward")
+
+
+def ds_slerp_rows_backward_workspace(cols: int) -> int:
+    """Workspace bytes ds_slerp_rows_backward needs for dalpha over `cols` columns."""
+    return int(_lib.ds_slerp_rows_backward_workspace(cols))
+
+
+def ds_slerp_rows_backward(segs: Sequence, eps: float = 1e-6, dalpha=None, workspace=None, stream=None) -> None:
+    """dalpha: fp32 [cols] CUDA tensor or None.  workspace: a CUDA tensor of at
+    least ds_slerp_rows_backward_workspace(cols) bytes (256-byte aligned), or
+    None to have one allocated here for this call."""
+    arr, n = _table(segs, ds_agseg)
+    ws_ptr, ws_bytes = 0, 0
+    if dalpha is not None:
+        cols = int(arr[0].cols) if n else 0
+        need = ds_slerp_rows_backward_workspace(cols) if cols else 0
+        if workspace is None and need:
+            import torch
+
+            workspace = torch.empty(need, dtype=torch.uint8, device=dalpha.device)
+        if workspace is not None:
+            ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
+    _check(_lib.ds_slerp_rows_backward(arr, n, eps, _vec(dalpha), ws_ptr, ws_bytes, _stream_ptr(stream)),
+           "ds_slerp_rows_backward")
 
 
 def ds_get_device_status(stream=None) -> int:

@@ -278,3 +278,65 @@ def test_binding_accepts_empty_tensors_with_any_strides():
     w = torch.zeros(64, 0).t()          # shape (0, 64), stride (1, 0)
     c = ds.WSeg(w=w, w_eff=torch.zeros(0, 64)).to_c()
     assert (c.rows, c.cols) == (0, 64)
+
+
+# ------------------------------------------------- activation backward calls --
+
+def agseg(**kw):
+    d = dict(x=BASE, r=0, dy=BASE + (1 << 30), dx=BASE + (2 << 30), dr=BASE + (3 << 30),
+             alpha=BASE + (4 << 30), rows=4, cols=8, ld=8, ld_d=8)
+    d.update(kw)
+    return ds.ds_agseg(**d)
+
+
+def call_g(fn, segs, eps=1e-6, dalpha=0, ws=0, ws_bytes=0):
+    arr = (ds.ds_agseg * max(1, len(segs)))(*segs)
+    lib = ds.lib()
+    if fn == "ds_l2_rows_backward":
+        return lib.ds_l2_rows_backward(arr, len(segs), ct.c_float(eps), None)
+    return lib.ds_slerp_rows_backward(arr, len(segs), ct.c_float(eps), dalpha, ws, ws_bytes, None)
+
+
+def test_backward_row_classes():
+    # x, r, dy staged: 48 bytes per 8 columns, at most 64 KB
+    assert ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 2728) == (ds.DS_PATH_WARP, 64, 1)
+    assert ds.ds_row_class(ds.DS_OP_SLERP_ROWS_BACKWARD, 4096) == (ds.DS_PATH_CTA, 128, 1)
+    assert ds.ds_row_class(ds.DS_OP_SLERP_ROWS_BACKWARD, 7168) == (ds.DS_PATH_CTA, 256, 1)
+    assert ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 10920)[0] == ds.DS_PATH_CTA
+    with pytest.raises(ds.DSError):
+        ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 10921)
+    with ds.force_path(ds.DS_PATH_TWO_PASS):   # no cluster classes: the staged one is kept
+        assert ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 128)[0] == ds.DS_PATH_WARP
+
+
+@pytest.mark.parametrize("fn", ["ds_l2_rows_backward", "ds_slerp_rows_backward"])
+def test_backward_validation(fn):
+    E = ds
+    slerp = fn == "ds_slerp_rows_backward"
+    good = dict(r=BASE + (5 << 30)) if slerp else {}
+    before = ds.ds_launch_count()
+    assert call_g(fn, [agseg(rows=-1, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_g(fn, [agseg(ld_d=4, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_g(fn, [agseg(dx=0, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_g(fn, [agseg(dy=0, **good)]) == E.DS_ERR_INVALID_ARG
+    assert call_g(fn, [agseg(dx=BASE + (2 << 30) + 4, **good)]) == E.DS_ERR_ALIGNMENT
+    assert call_g(fn, [agseg(cols=10921, ld=10928, ld_d=10924, **good)]) == E.DS_ERR_INVALID_ARG
+    # dx over an input
+    assert call_g(fn, [agseg(dx=BASE + (1 << 30), **good)]) == E.DS_ERR_OVERLAP
+    assert call_g(fn, [agseg(rows=0, x=0, dy=0, dx=0, dr=0, **good)]) == E.DS_OK
+    if slerp:
+        assert call_g(fn, [agseg()]) == E.DS_ERR_INVALID_ARG                 # out (r) required
+        assert call_g(fn, [agseg(dr=0, **good)]) == E.DS_ERR_INVALID_ARG
+        assert call_g(fn, [agseg(alpha=0, **good)]) == E.DS_ERR_INVALID_ARG
+        assert call_g(fn, [agseg(dr=BASE + (2 << 30), **good)]) == E.DS_ERR_OVERLAP   # dr over dx
+        need = ds.ds_slerp_rows_backward_workspace(8)
+        assert need > 0 and ds.ds_slerp_rows_backward_workspace(0) == 0
+        da, ws = BASE + (6 << 30), BASE + (7 << 30)
+        assert call_g(fn, [agseg(**good)], dalpha=da) == E.DS_ERR_INVALID_ARG          # no workspace
+        assert call_g(fn, [agseg(**good)], dalpha=da, ws=ws + 16, ws_bytes=need) == E.DS_ERR_ALIGNMENT
+        assert call_g(fn, [agseg(**good)], dalpha=da, ws=ws, ws_bytes=need - 1) == E.DS_ERR_INVALID_ARG
+        other = agseg(x=BASE + (8 << 30), r=BASE + (9 << 30), dy=BASE + (10 << 30), dx=BASE + (11 << 30),
+                      dr=BASE + (12 << 30), alpha=BASE + (13 << 30))
+        assert call_g(fn, [agseg(**good), other], dalpha=da, ws=ws, ws_bytes=need) == E.DS_ERR_INVALID_ARG
+        assert call_g(fn, [agseg(**good)], dalpha=ws, ws=ws, ws_bytes=need) == E.DS_ERR_OVERLAP
+    assert ds.ds_launch_count() == before
