@@ -17,7 +17,7 @@ disjoint buffers (>= 268 MB of other traffic between two uses of one
 buffer), so inputs come from HBM without an explicit flush.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config step|mlp_pair|wide|optimizer]
+                    [--config step|mlp_pair|wide|optimizer|act_backward]
 
 `--config` selects another workload for a per-call report (default: the
 step above).  mlp_pair = up [2048,768] + down [768,2048] (fwd, bwd, renorm;
@@ -25,7 +25,8 @@ L2-resident, so each timed step uses the next of 16 buffer copies and a
 CUDA-graph replay of the calls is timed as well).  wide = weights
 [14336,4096], [4096,14336] (fwd, bwd) and activation rows [8192,7168],
 [4096,16384] (l2, l2 + residual, slerp).  optimizer = ds_grad_project and
-ds_renorm_momentum over the whole-model weights.
+ds_renorm_momentum over the whole-model weights.  act_backward = the
+backward of the activation calls on [16384,4096] (upstream gradient bf16).
 
 Prints one JSON line (rank 0).  `value` is algorithmic bytes moved by all
 ranks per second (GB/s); per-kernel GB/s and rows/s, the roofline of the
@@ -68,6 +69,8 @@ WORKLOADS = {
     "optimizer": "optimizer companions of method rescale on the whole-model weights (85 segments, 100,073,472 "
                  "fp32 elements): gradient projection before the step, momentum projection + renorm after it "
                  "(fp32 gradient and momentum, in place)",
+    "act_backward": "activation backward on rows [16384,4096] bf16: l2 (dx fp32), l2 with residual, slerp "
+                    "(dres, dout fp32 and dalpha [4096] through its workspace)",
 }
 
 
@@ -91,7 +94,9 @@ def call_bytes(kind: str, segs=None, act=None) -> int:
     written once (per-row gains and grad_g 4 B per row)."""
     if act is not None:
         A = act.rows * act.cols
-        return {"l2": A * (2 + 2), "l2res": A * (2 + 2 + 2), "slerp": A * (2 + 2 + 2) + act.cols * 4}[kind]
+        return {"l2": A * (2 + 2), "l2res": A * (2 + 2 + 2), "slerp": A * (2 + 2 + 2) + act.cols * 4,
+                "l2bwd": A * (2 + 2 + 4), "l2resbwd": A * (2 + 2 + 2 + 4),
+                "slerpbwd": A * (2 + 2 + 2 + 4 + 4) + act.cols * (4 + 4)}[kind]
     E = sum(s.w.size for s in segs)
     R = sum(s.rows for s in segs)
     return {"fwd": E * (4 + 2) + R * 4, "bwd": E * (4 + 2 + 4) + R * (4 + 4), "renorm": E * (4 + 4),
@@ -137,6 +142,11 @@ def plan(config: str, seed: int):
         for g in ag:
             calls += [(f"l2_rows_{g}", "l2", g), (f"l2_rows_residual_{g}", "l2res", g), (f"slerp_rows_{g}", "slerp", g)]
         return wg, ag, calls, 1
+    if config == "act_backward":
+        ag = {"x": wl.activations(seed, ACT_ROWS, ACT_COLS).acts[0]}
+        calls = [("l2_rows_backward", "l2bwd", "x"), ("l2_rows_residual_backward", "l2resbwd", "x"),
+                 ("slerp_rows_backward", "slerpbwd", "x")]
+        return {}, ag, calls, 1
     if config == "optimizer":
         wg = {"model": wl.with_fp32_state(wl.whole_model(seed).weights, seed + 1)}
         calls = [("grad_project", "project", "model"), ("renorm_momentum", "momentum", "model")]
@@ -264,6 +274,7 @@ class Step:
         import torch
 
         from l2_row_b200 import ds
+        from l2_row_b200 import workloads as wl
 
         self.torch, self.ds = torch, ds
         self.wg, self.ag, self.plan, self.copies = plan(config, seed)
@@ -313,15 +324,34 @@ class Step:
             if kinds & {"renorm", "momentum"}:
                 self.outputs.append(b0["w"])
         for name, a in self.ag.items():
+            kinds = {k for _, k, g in self.plan if g == name}
+            bwd = any(k.endswith("bwd") for k in kinds)
+            dy_host = None
+            if bwd:   # the upstream gradient: bf16 N(0,1), seeded after the rows
+                dy_host = wl.normal_bf16(np.random.default_rng(seed + 7), a.x.shape)
             copies = []
             for c in range(self.copies):
                 x = bf16(a.x)
-                copies.append({"x": x, "r": bf16(a.r), "alpha": f32(a.alpha), "y": torch.empty_like(x),
-                               "y2": torch.empty_like(x), "h": torch.empty_like(x)})
+                b = {"x": x, "r": bf16(a.r), "alpha": f32(a.alpha)}
+                if bwd:
+                    b["dy"] = bf16(dy_host)
+                    b["dx"] = torch.empty(a.x.shape, dtype=torch.float32, device=dev)
+                    b["dx2"] = torch.empty_like(b["dx"])
+                    b["dres"] = torch.empty_like(b["dx"])
+                    b["dout"] = torch.empty_like(b["dx"])
+                    b["dalpha"] = torch.empty(a.cols, dtype=torch.float32, device=dev)
+                    b["ws"] = torch.empty(ds.ds_slerp_rows_backward_workspace(a.cols), dtype=torch.uint8, device=dev)
+                else:
+                    b.update({"y": torch.empty_like(x), "y2": torch.empty_like(x), "h": torch.empty_like(x)})
+                copies.append(b)
             self.abuf[name] = copies
             b0 = copies[0]
             self.inputs += [(b0["x"], a.x.view(np.int16)), (b0["r"], a.r.view(np.int16)), (b0["alpha"], a.alpha)]
-            self.outputs += [b0["y"], b0["y2"], b0["h"]]
+            if bwd:
+                self.inputs.append((b0["dy"], dy_host.view(np.int16)))
+                self.outputs += [b0["dx"], b0["dx2"], b0["dres"], b0["dout"], b0["dalpha"]]
+            else:
+                self.outputs += [b0["y"], b0["y2"], b0["h"]]
 
         self.names = [c[0] for c in self.plan]
         self.bytes = {}
@@ -366,6 +396,21 @@ class Step:
                           "renorm": lambda s, t=tab, n=n: lib.ds_row_renorm(t, n, eps, s),
                           "project": lambda s, t=tab, n=n: lib.ds_grad_project(t, n, eps, s),
                           "momentum": lambda s, t=tab, n=n: lib.ds_renorm_momentum(t, n, eps, s)}[kind]
+                elif kind.endswith("bwd"):
+                    b = self.abuf[g][c]
+                    if kind == "l2bwd":
+                        seg = ds.AGSeg(x=b["x"], dy=b["dy"], dx=b["dx"])
+                    elif kind == "l2resbwd":
+                        seg = ds.AGSeg(x=b["x"], r=b["r"], dy=b["dy"], dx=b["dx2"])
+                    else:
+                        seg = ds.AGSeg(x=b["x"], r=b["r"], dy=b["dy"], dx=b["dres"], dr=b["dout"], alpha=b["alpha"])
+                    tab = (ds.ds_agseg * 1)(seg.to_c())
+                    if kind == "slerpbwd":
+                        da, ws = b["dalpha"], b["ws"]
+                        fn = (lambda s, t=tab, da=da, ws=ws: lib.ds_slerp_rows_backward(
+                            t, 1, eps, da.data_ptr(), ws.data_ptr(), ws.numel(), s))
+                    else:
+                        fn = lambda s, t=tab: lib.ds_l2_rows_backward(t, 1, eps, s)
                 else:
                     b = self.abuf[g][c]
                     if kind == "l2":
