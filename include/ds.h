@@ -205,6 +205,16 @@ ds_status ds_slerp_rows_backward(const ds_agseg *segs, int nseg, float eps,
  * `cols` elements on the current device (0 if cols < 1). */
 uint64_t ds_slerp_rows_backward_workspace(int64_t cols);
 
+/* ds_slerp_rows_backward without a caller workspace: dalpha's partial sums go
+ * to a scratch array built into the library (one static device array per
+ * device, 64 MB: rows up to 8,712 columns on a 148-SM B200; wider rows are
+ * refused with DS_ERR_INVALID_ARG).  The scratch is shared, so calls of this
+ * entry point must not overlap in time (use one stream, or synchronise).
+ * Results are bitwise those of ds_slerp_rows_backward.  The pages have no
+ * counterpart: this is a convenience entry point of this library. */
+ds_status ds_slerp_rows_backward_noalloc(const ds_agseg *segs, int nseg, float eps,
+                                         float *dalpha, ds_stream stream);
+
 /* Static description of a status code. */
 const char *ds_status_string(ds_status status);
 

@@ -744,6 +744,17 @@ ds_status ds_slerp_rows_backward(const ds_agseg *segs, int nseg, float eps, floa
     return run_act_bwd(true, segs, nseg, eps, dalpha, workspace, workspace_bytes, stream);
 }
 
+ds_status ds_slerp_rows_backward_noalloc(const ds_agseg *segs, int nseg, float eps, float *dalpha, ds_stream stream)
+{
+    void *ws = nullptr;
+    uint64_t bytes = 0;
+    if (dalpha) {
+        if (ds::builtin_scratch(&ws, &bytes) != 0)
+            return fail(DS_ERR_CUDA, "built-in scratch not available");
+    }
+    return run_act_bwd(true, segs, nseg, eps, dalpha, ws, bytes, stream);
+}
+
 uint64_t ds_slerp_rows_backward_workspace(int64_t cols)
 {
     if (cols < 1 || cols > kMaxCols)

@@ -162,6 +162,9 @@ int launch_wait_selftest(uint64_t limit_ns, void *stream);
 int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream);
 // Ring positions (consumer teams) per CTA of a staged launch.
 int tile_groups(int tag, int slot_bytes);
+// The built-in device scratch of the no-alloc slerp backward (ds_tile.cu).
+constexpr int64_t kBuiltinScratchFloats = int64_t(16) << 20; // 64 MB
+int builtin_scratch(void **ptr, uint64_t *bytes);
 // dalpha[c] = sum over CTAs c0 < grid and their used teams q of
 // ws[(c0 * groups + q) * ws_ld + c], in that order (slerp backward).
 int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64_t total_units, int cols,

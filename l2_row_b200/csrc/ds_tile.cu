@@ -1442,6 +1442,18 @@ __global__ void __launch_bounds__(256) k_dalpha_reduce(const float *ws, int ws_l
 
 } // namespace
 
+// Built-in scratch for the no-alloc slerp backward entry point: one
+// module-level device array (64 MB, enough for the dalpha lines of rows up to
+// 8,712 columns on 148 SMs).  Calls that use it must not overlap in time.
+static __device__ __align__(256) float g_builtin_scratch[kBuiltinScratchFloats];
+
+int builtin_scratch(void **ptr, uint64_t *bytes)
+{
+    const cudaError_t e = cudaGetSymbolAddress(ptr, g_builtin_scratch);
+    *bytes = static_cast<uint64_t>(kBuiltinScratchFloats) * sizeof(float);
+    return e;
+}
+
 int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64_t total_units, int cols,
                          float *dalpha, void *stream)
 {

@@ -75,6 +75,9 @@ _lib.ds_slerp_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_v
 _lib.ds_l2_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_slerp_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p, ct.c_void_p,
                                         ct.c_uint64, ct.c_void_p]
+_lib.ds_slerp_rows_backward_noalloc.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p,
+                                                ct.c_void_p]
+_lib.ds_slerp_rows_backward_noalloc.restype = ct.c_int
 _lib.ds_slerp_rows_backward_workspace.argtypes = [ct.c_int64]
 _lib.ds_slerp_rows_backward_workspace.restype = ct.c_uint64
 for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
@@ -100,7 +103,7 @@ _lib.ds_debug_wait_timeout_selftest.argtypes = [ct.c_uint64, ct.c_void_p]
 #: every symbol include/ds.h declares
 EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
-           "ds_slerp_rows_backward_workspace", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
+           "ds_slerp_rows_backward_workspace", "ds_slerp_rows_backward_noalloc", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
            "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest")
 
 
@@ -313,6 +316,13 @@ def ds_slerp_rows_backward(segs: Sequence, eps: float = 1e-6, dalpha=None, works
             ws_ptr, ws_bytes = workspace.data_ptr(), workspace.numel() * workspace.element_size()
     _check(_lib.ds_slerp_rows_backward(arr, n, eps, _vec(dalpha), ws_ptr, ws_bytes, _stream_ptr(stream)),
            "ds_slerp_rows_backward")
+
+
+def ds_slerp_rows_backward_noalloc(segs: Sequence, eps: float = 1e-6, dalpha=None, stream=None) -> None:
+    """ds_slerp_rows_backward with the library's built-in scratch (no workspace)."""
+    arr, n = _table(segs, ds_agseg)
+    _check(_lib.ds_slerp_rows_backward_noalloc(arr, n, eps, _vec(dalpha), _stream_ptr(stream)),
+           "ds_slerp_rows_backward_noalloc")
 
 
 def ds_get_device_status(stream=None) -> int:
