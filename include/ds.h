@@ -184,9 +184,11 @@ ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps,
 ds_status ds_slerp_rows(const ds_aseg *segs, int nseg, float eps,
                         ds_stream stream);
 
-/* Rows must have at most 64 KB of staged input in the widest layout (x, r
- * and dy, 48 bytes per 8 columns): at most 10,920 columns for either call;
- * longer rows are refused with DS_ERR_INVALID_ARG. */
+/* Rows must have at most 64 KB of staged input (x, r and dy: 48 bytes per 8
+ * columns; l2 rows without a residual 32): at most 10,920 columns for slerp
+ * and for l2 with a residual, 16,384 for l2 without one; longer rows are
+ * refused with DS_ERR_INVALID_ARG.  ds_row_class reports the l2 backward's
+ * class for rows with a residual. */
 ds_status ds_l2_rows_backward(const ds_agseg *segs, int nseg, float eps,
                               ds_stream stream);
 

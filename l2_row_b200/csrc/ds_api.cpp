@@ -52,10 +52,11 @@ std::string where(const char *what, int seg)
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// Bytes a row stages in shared memory on the warp-per-row path, for the
-// widest layout of the operation (fp32 GY; a residual present), so that the
-// path -- and with it the row's arithmetic -- depends on (op, cols) only.
-int64_t tile_row_bytes_worst(ds_op op, int64_t cols)
+// Bytes a row stages in shared memory on the staged paths, for the widest
+// layout of the operation (fp32 GY; a residual present), so that the path --
+// and with it the row's arithmetic -- depends on (op, cols) only.  The l2
+// backward without a residual (has_r false) is its own layout: two arrays.
+int64_t tile_row_bytes_worst(ds_op op, int64_t cols, bool has_r = true)
 {
     const int64_t q = (cols + 3) / 4 * 16, o = (cols + 7) / 8 * 16;
     switch (op) {
@@ -64,7 +65,7 @@ int64_t tile_row_bytes_worst(ds_op op, int64_t cols)
     case DS_OP_WN_BACKWARD:
     case DS_OP_GRAD_PROJECT:
     case DS_OP_RENORM_MOMENTUM: return 2 * q;
-    case DS_OP_L2_ROWS_BACKWARD:
+    case DS_OP_L2_ROWS_BACKWARD: return (has_r ? 3 : 2) * o;
     case DS_OP_SLERP_ROWS_BACKWARD: return 3 * o;
     default: return 2 * o;
     }
@@ -88,12 +89,12 @@ int64_t max_slot(ds_op op)
     return ds::is_weight_op(op) ? ds::kTileSlotMaxWeightBytes : ds::kTileSlotMaxBytes;
 }
 
-RowClass classify(ds_op op, int64_t cols, int forced)
+RowClass classify(ds_op op, int64_t cols, int forced, bool has_r = true)
 {
     const int64_t E = ds::elems_per_unit(op);
     const int64_t nu = (cols + E - 1) / E;
     const int64_t kmax = ds::kmax_of(op);
-    const int64_t staged = tile_row_bytes_worst(op, cols);
+    const int64_t staged = tile_row_bytes_worst(op, cols, has_r);
     auto staged_class = [&](int path, int min_slot) -> RowClass {
         for (const int slot : {16384, 32768, 65536, 114688})
             if (slot >= min_slot && slot <= max_slot(op) && staged <= slot)
@@ -607,7 +608,7 @@ ds_status run_act_bwd(bool slerp, const ds_agseg *segs, int nseg, float eps, flo
             return fail(DS_ERR_INVALID_ARG, where("ld_d < cols", i));
         rows[i] = s.rows;
         cols[i] = s.cols;
-        cls[i] = classify(op, s.cols, forced);
+        cls[i] = classify(op, s.cols, forced, slerp || s.r != nullptr);
         if (cls[i].path == 0)
             return fail(DS_ERR_INVALID_ARG, where("row too long for the backward (more than 64 KB of staged input)", i));
         if (s.rows == 0)

@@ -320,7 +320,11 @@ def test_backward_validation(fn):
     assert call_g(fn, [agseg(dx=0, **good)]) == E.DS_ERR_INVALID_ARG
     assert call_g(fn, [agseg(dy=0, **good)]) == E.DS_ERR_INVALID_ARG
     assert call_g(fn, [agseg(dx=BASE + (2 << 30) + 4, **good)]) == E.DS_ERR_ALIGNMENT
-    assert call_g(fn, [agseg(cols=10921, ld=10928, ld_d=10924, **good)]) == E.DS_ERR_INVALID_ARG
+    if slerp:   # x, r, dy staged: 10,920 columns at most
+        assert call_g(fn, [agseg(cols=10921, ld=10928, ld_d=10924, **good)]) == E.DS_ERR_INVALID_ARG
+    else:       # without a residual x and dy: 16,384 columns; with one 10,920
+        assert call_g(fn, [agseg(cols=16385, ld=16392, ld_d=16388)]) == E.DS_ERR_INVALID_ARG
+        assert call_g(fn, [agseg(cols=10921, ld=10928, ld_d=10924, r=BASE + (5 << 30))]) == E.DS_ERR_INVALID_ARG
     # dx over an input
     assert call_g(fn, [agseg(dx=BASE + (1 << 30), **good)]) == E.DS_ERR_OVERLAP
     assert call_g(fn, [agseg(rows=0, x=0, dy=0, dx=0, dr=0, **good)]) == E.DS_OK
