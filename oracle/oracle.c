@@ -400,11 +400,208 @@ void or_slerp_row_interval(const double *res, const double *out,
 }
 
 /* ------------------------------------------------------------------------ */
+/* [TF] Dory's gated and SwiGLU rows and their L2 norm: the rounding points
+ * are the ones the pages list (the gated row; the scaled gate, the scaled up
+ * and the product), then the output.  sigmoid and silu are the plain
+ * definitions 1/(1+exp(-x)) and x/(1+exp(-x)) in double.                    */
+
+static double sigmoid64(double z) { return 1.0 / (1.0 + exp(-z)); }
+static double silu64(double x) { return x / (1.0 + exp(-x)); }
+
+static double gate_value(double o, double g, double sg, unsigned flags)
+{
+    double v = o * sigmoid64(g * sg);
+    return (flags & OR_DROP_GATED) ? v : round_bf16(v);
+}
+
+static double swiglu_value(double g, double u, double sug, double suu,
+                           unsigned flags)
+{
+    double gs = g * sug, us = u * suu;
+    if (!(flags & OR_DROP_SGATE))
+        gs = round_bf16(gs);
+    if (!(flags & OR_DROP_SUP))
+        us = round_bf16(us);
+    double v = silu64(gs) * us;
+    return (flags & OR_DROP_PRODUCT) ? v : round_bf16(v);
+}
+
+/* y = bf16(s / sqrt(sum s^2 + eps)) for a row whose s is already formed. */
+static void l2_of(const double *s, int64_t C, double eps, unsigned flags,
+                  uint16_t *y, double *y_exact)
+{
+    double n = row_norm(sum_sq(s, C), eps, flags);
+    for (int64_t j = 0; j < C; ++j) {
+        double v = s[j] / n;
+        y[j] = or_bf16_rne(v);
+        if (y_exact)
+            y_exact[j] = v;
+    }
+}
+
+/* The range an fp32 evaluation of sigmoid(z) can reach: the argument's own
+ * rounding (2^-24 relative, through exp a relative |z| 2^-24), exp's 2 ulps,
+ * 1 + e and the division move it by about (1 - s)(|z| 2^-23 + 2^-21) + 2^-22
+ * (never less than delta); where -z > 87, exp(-z) is at or past fp32's
+ * largest value and 1/(1+e) is subnormal or 0, so 0 is reachable. */
+static void sigmoid_range(double z, double delta, double *lo, double *hi)
+{
+    double s = sigmoid64(z);
+    double rel = (1.0 - s) * (fabs(z) * 0x1p-23 + 0x1p-21) + 0x1p-22;
+    if (rel < delta)
+        rel = delta;
+    *lo = s * (1.0 - rel);
+    *hi = s * (1.0 + rel);
+    if (-z > 87.0) {
+        *lo = 0.0;
+        *hi = s * (1.0 + rel) + 0x1p-149;
+    }
+}
+
+/* silu over [xl, xh] (xl <= xh), with the fp32 spread of each evaluation;
+ * silu falls to its minimum at x0 = -1.2784645... and rises on both sides. */
+static void silu_range(double xl, double xh, double delta, double *lo,
+                       double *hi)
+{
+    double l = 1e300, h = -1e300;
+    const double xs[2] = {xl, xh};
+    for (int k = 0; k < 2; ++k) {
+        double x = xs[k];
+        double sl, sh;
+        sigmoid_range(x, delta, &sl, &sh);
+        double a = x * sl, b = x * sh; /* silu = x sigmoid(x) */
+        double vl = dmin(a, b), vh = dmax(a, b);
+        vl -= fabs(vl) * delta;
+        vh += fabs(vh) * delta;
+        if (-x > 87.0) { /* x / (1 + exp(-x)) is -0 once exp overflows */
+            vh = dmax(vh, 0.0);
+        }
+        l = dmin(l, vl);
+        h = dmax(h, vh);
+    }
+    const double x0 = -1.2784645427610738;
+    if (xl <= x0 && x0 <= xh) {
+        double m = silu64(x0);
+        l = dmin(l, m - fabs(m) * delta);
+    }
+    *lo = l;
+    *hi = h;
+}
+
+/* bf16 ends of [vl, vh] (or the ends themselves when the point is dropped). */
+static void bf16_ends(double vl, double vh, int drop, double *l, double *h)
+{
+    if (drop) {
+        *l = vl;
+        *h = vh;
+    } else {
+        *l = round_bf16(vl);
+        *h = round_bf16(vh);
+    }
+}
+
+/* The product of two ranges. */
+static void mul_range(double al, double ah, double bl, double bh, double *l,
+                      double *h)
+{
+    double c0 = al * bl, c1 = al * bh, c2 = ah * bl, c3 = ah * bh;
+    *l = dmin(dmin(c0, c1), dmin(c2, c3));
+    *h = dmax(dmax(c0, c1), dmax(c2, c3));
+}
+
+/* l2 of a row whose elements lie in [sl_j, sh_j]: bf16 ends of each output. */
+static void l2_interval_of(const double *sl, const double *sh, int64_t C,
+                           double eps, double delta, unsigned flags,
+                           uint16_t *lo, uint16_t *hi)
+{
+    double Sl = 0.0, Sh = 0.0;
+    for (int64_t j = 0; j < C; ++j) {
+        double ql = sl[j] * sl[j], qh = sh[j] * sh[j];
+        Sl += (sl[j] > 0.0 || sh[j] < 0.0) ? dmin(ql, qh) : 0.0;
+        Sh += dmax(ql, qh);
+    }
+    double nl = row_norm(Sl * (1.0 - delta), eps, flags);
+    double nh = row_norm(Sh * (1.0 + delta), eps, flags);
+    for (int64_t j = 0; j < C; ++j) {
+        double ql, qh;
+        if (!(nl > 0.0) || !isfinite(nh)) {
+            ql = -INFINITY;
+            qh = INFINITY;
+        } else {
+            quotient_ends(sl[j], sh[j], nl, nh, delta, &ql, &qh);
+        }
+        lo[j] = or_bf16_rne(ql);
+        hi[j] = or_bf16_rne(qh);
+    }
+}
+
+static void gate_row(const double *o, const double *g, const double *sg,
+                     int64_t C, double eps, unsigned flags, double *s,
+                     uint16_t *y, double *y_exact)
+{
+    for (int64_t j = 0; j < C; ++j)
+        s[j] = gate_value(o[j], g[j], sg[j], flags);
+    l2_of(s, C, eps, flags, y, y_exact);
+}
+
+static void swiglu_row(const double *g, const double *u, const double *sug,
+                       const double *suu, int64_t C, double eps,
+                       unsigned flags, double *s, uint16_t *y, double *y_exact)
+{
+    for (int64_t j = 0; j < C; ++j)
+        s[j] = swiglu_value(g[j], u[j], sug[j], suu[j], flags);
+    l2_of(s, C, eps, flags, y, y_exact);
+}
+
+static void gate_row_interval(const double *o, const double *g,
+                              const double *sg, int64_t C, double eps,
+                              double delta, unsigned flags, double *tmp,
+                              uint16_t *lo, uint16_t *hi)
+{
+    double *sl = tmp, *sh = tmp + C;
+    for (int64_t j = 0; j < C; ++j) {
+        /* z = g sg is one fp32 product */
+        double z = g[j] * sg[j], zl = z - fabs(z) * 0x1p-24, zh = z + fabs(z) * 0x1p-24;
+        double a0, a1, b0, b1;
+        sigmoid_range(zl, delta, &a0, &a1);
+        sigmoid_range(zh, delta, &b0, &b1);
+        double gl = dmin(a0, b0), gh = dmax(a1, b1), vl, vh;
+        mul_range(o[j], o[j], gl, gh, &vl, &vh);
+        vl -= fabs(vl) * delta;
+        vh += fabs(vh) * delta;
+        bf16_ends(vl, vh, flags & OR_DROP_GATED, &sl[j], &sh[j]);
+    }
+    l2_interval_of(sl, sh, C, eps, delta, flags, lo, hi);
+}
+
+static void swiglu_row_interval(const double *g, const double *u,
+                                const double *sug, const double *suu,
+                                int64_t C, double eps, double delta,
+                                unsigned flags, double *tmp, uint16_t *lo,
+                                uint16_t *hi)
+{
+    double *sl = tmp, *sh = tmp + C;
+    for (int64_t j = 0; j < C; ++j) {
+        double p = g[j] * sug[j], q = u[j] * suu[j];
+        double gl, gh, ul, uh;
+        bf16_ends(p - fabs(p) * 0x1p-24, p + fabs(p) * 0x1p-24, flags & OR_DROP_SGATE, &gl, &gh);
+        bf16_ends(q - fabs(q) * 0x1p-24, q + fabs(q) * 0x1p-24, flags & OR_DROP_SUP, &ul, &uh);
+        double fl, fh, vl, vh;
+        silu_range(gl, gh, delta, &fl, &fh);
+        mul_range(fl, fh, ul, uh, &vl, &vh);
+        vl -= fabs(vl) * delta;
+        vh += fabs(vh) * delta;
+        bf16_ends(vl, vh, flags & OR_DROP_PRODUCT, &sl[j], &sh[j]);
+    }
+    l2_interval_of(sl, sh, C, eps, delta, flags, lo, hi);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Matrix drivers.  Each worker owns a contiguous range of rows and its own
  * scratch rows; inputs are widened to double exactly before the row call.   */
 
 enum { OP_FWD, OP_BWD, OP_RENORM, OP_L2, OP_SLERP, OP_L2_IV, OP_SLERP_IV, OP_PROJECT, OP_MOMENTUM,
-       OP_L2_BWD, OP_SLERP_BWD };
+       OP_L2_BWD, OP_SLERP_BWD, OP_GATE, OP_SWIGLU, OP_GATE_IV, OP_SWIGLU_IV };
 
 typedef struct {
     int op;
@@ -415,6 +612,7 @@ typedef struct {
     int gy_bf16;
     const uint16_t *x, *r;
     const float *alpha;
+    const float *alpha2; /* swiglu: suu (alpha holds sg / sug) */
     double rho, eps, delta;
     unsigned flags;
     double *out_d;   /* dense [R, C] doubles */
@@ -435,10 +633,13 @@ static void *run_job(void *arg)
         jb->status = -1;
         return NULL;
     }
-    double *u = buf, *v = buf + C, *tmp = buf + 2 * C, *al = buf + 6 * C, *dv = buf + 7 * C;
-    if (jb->op == OP_SLERP || jb->op == OP_SLERP_IV || jb->op == OP_SLERP_BWD)
+    double *u = buf, *v = buf + C, *tmp = buf + 2 * C, *al = buf + 6 * C, *dv = buf + 7 * C, *al2 = buf + 8 * C;
+    if (jb->op == OP_SLERP || jb->op == OP_SLERP_IV || jb->op == OP_SLERP_BWD || jb->op >= OP_GATE)
         for (int64_t j = 0; j < C; ++j)
             al[j] = (double)jb->alpha[j];
+    if (jb->op == OP_SWIGLU || jb->op == OP_SWIGLU_IV)
+        for (int64_t j = 0; j < C; ++j)
+            al2[j] = (double)jb->alpha2[j];
 
     for (int64_t row = jb->r0; row < jb->r1; ++row) {
         size_t o = (size_t)row * (size_t)C;
@@ -489,6 +690,29 @@ static void *run_job(void *arg)
             else
                 or_renorm_momentum_row(u, v, C, jb->rho, jb->eps, jb->flags,
                                        jb->out_d2 + o, jb->out_d + o);
+            break;
+        }
+        case OP_GATE:
+        case OP_SWIGLU:
+        case OP_GATE_IV:
+        case OP_SWIGLU_IV: {
+            const uint16_t *xr = jb->x + row * jb->ld;
+            const uint16_t *rr = jb->r + row * jb->ld;
+            for (int64_t j = 0; j < C; ++j) {
+                u[j] = or_bf16_value(xr[j]);
+                v[j] = or_bf16_value(rr[j]);
+            }
+            double *ye = jb->out_d ? jb->out_d + o : NULL;
+            if (jb->op == OP_GATE)
+                gate_row(u, v, al, C, jb->eps, jb->flags, tmp, jb->out_h + o, ye);
+            else if (jb->op == OP_SWIGLU)
+                swiglu_row(u, v, al, al2, C, jb->eps, jb->flags, tmp, jb->out_h + o, ye);
+            else if (jb->op == OP_GATE_IV)
+                gate_row_interval(u, v, al, C, jb->eps, jb->delta, jb->flags, tmp, jb->out_h + o,
+                                  jb->out_h2 + o);
+            else
+                swiglu_row_interval(u, v, al, al2, C, jb->eps, jb->delta, jb->flags, tmp, jb->out_h + o,
+                                    jb->out_h2 + o);
             break;
         }
         case OP_L2_BWD:
@@ -690,6 +914,66 @@ int or_renorm_momentum(const float *w, int64_t R, int64_t C, int64_t ld,
     jb.out_d = m_out;
     jb.out_d2 = w_out;
     return run_rows(&jb, R, nthreads);
+}
+
+static int fused_rows(int op, const uint16_t *a, const uint16_t *b,
+                      const float *sa, const float *sb, int64_t R, int64_t C,
+                      int64_t ld, double eps, double delta, unsigned flags,
+                      uint16_t *y, uint16_t *y2, double *y_exact, int nthreads)
+{
+    const unsigned allowed = (op == OP_GATE || op == OP_GATE_IV)
+                                 ? (OR_DROP_GATED | OR_EPS_ZERO | OR_EPS_OUTSIDE)
+                                 : (OR_DROP_SGATE | OR_DROP_SUP | OR_DROP_PRODUCT | OR_EPS_ZERO | OR_EPS_OUTSIDE);
+    if (bad_shape(R, C, ld) || !sa || ((op == OP_SWIGLU || op == OP_SWIGLU_IV) && !sb) ||
+        (R > 0 && (!a || !b || !y || ((op == OP_GATE_IV || op == OP_SWIGLU_IV) && !y2))) || (flags & ~allowed))
+        return -1;
+    job_t jb = {0};
+    jb.op = op;
+    jb.C = C;
+    jb.ld = ld;
+    jb.x = a;
+    jb.r = b;
+    jb.alpha = sa;
+    jb.alpha2 = sb;
+    jb.eps = eps;
+    jb.delta = delta;
+    jb.flags = flags;
+    jb.out_h = y;
+    jb.out_h2 = y2;
+    jb.out_d = y_exact;
+    return run_rows(&jb, R, nthreads);
+}
+
+int or_gate_l2_rows(const uint16_t *o, const uint16_t *g, const float *sg,
+                    int64_t R, int64_t C, int64_t ld, double eps,
+                    unsigned flags, uint16_t *y, double *y_exact, int nthreads)
+{
+    return fused_rows(OP_GATE, o, g, sg, NULL, R, C, ld, eps, 0.0, flags, y, NULL, y_exact, nthreads);
+}
+
+int or_swiglu_l2_rows(const uint16_t *g, const uint16_t *u, const float *sug,
+                      const float *suu, int64_t R, int64_t C, int64_t ld,
+                      double eps, unsigned flags, uint16_t *y, double *y_exact,
+                      int nthreads)
+{
+    return fused_rows(OP_SWIGLU, g, u, sug, suu, R, C, ld, eps, 0.0, flags, y, NULL, y_exact, nthreads);
+}
+
+int or_gate_l2_rows_interval(const uint16_t *o, const uint16_t *g,
+                             const float *sg, int64_t R, int64_t C, int64_t ld,
+                             double eps, double delta, unsigned flags,
+                             uint16_t *lo, uint16_t *hi, int nthreads)
+{
+    return fused_rows(OP_GATE_IV, o, g, sg, NULL, R, C, ld, eps, delta, flags, lo, hi, NULL, nthreads);
+}
+
+int or_swiglu_l2_rows_interval(const uint16_t *g, const uint16_t *u,
+                               const float *sug, const float *suu, int64_t R,
+                               int64_t C, int64_t ld, double eps, double delta,
+                               unsigned flags, uint16_t *lo, uint16_t *hi,
+                               int nthreads)
+{
+    return fused_rows(OP_SWIGLU_IV, g, u, sug, suu, R, C, ld, eps, delta, flags, lo, hi, NULL, nthreads);
 }
 
 int or_l2_rows_backward(const uint16_t *x, const uint16_t *r,

@@ -41,6 +41,10 @@ extern "C" {
 #define OR_EPS_ZERO       0x10u /* norm = sqrt(S), eps ignored                           */
 #define OR_BWD_PRINTED    0x20u /* backward: project with S instead of S + eps (the
                                    eps-free form of the printed dL/dW)                   */
+#define OR_DROP_GATED     0x40u /* gate_l2: use o * sigmoid(g sg) unrounded (the gated row) */
+#define OR_DROP_SGATE     0x80u /* swiglu_l2: use g * sug unrounded (the scaled gate)       */
+#define OR_DROP_SUP       0x100u /* swiglu_l2: use u * suu unrounded (the scaled up)        */
+#define OR_DROP_PRODUCT   0x200u /* swiglu_l2: use silu(.) * (.) unrounded (the product)    */
 
 /* bf16 helpers.  or_bf16_rne rounds a double straight to bf16 bits. */
 uint16_t or_bf16_rne(double v);
@@ -165,6 +169,31 @@ int or_l2_rows(const uint16_t *x, const uint16_t *r, int64_t R, int64_t C,
 int or_slerp_rows(const uint16_t *res, const uint16_t *out, const float *alpha,
                   int64_t R, int64_t C, int64_t ld, double eps, unsigned flags,
                   uint16_t *h, double *h_exact, int nthreads);
+
+/* [TF] Dory's gated and SwiGLU rows, then their L2 norm (the norms.cu
+ * family; sigmoid and silu in torch's fp32 forms 1/(1+exp(-x)), x/(1+exp(-x))):
+ *   gate_l2:   y = bf16(l2(bf16(o * sigmoid(g * sg))))
+ *   swiglu_l2: y = bf16(l2(bf16(silu(bf16(g * sug)) * bf16(u * suu))))
+ * o, g, u bf16 bits [R, ld]; sg, sug, suu fp32 [C].  The interval forms give,
+ * per output, the bf16 ends any fp32 evaluation within relative `delta` per
+ * step (and 2 ulps in exp) can reach, with fp32's exp range (exp(-x)
+ * overflows for -x > 88.72: the gate or silu is 0) and subnormal steps. */
+int or_gate_l2_rows(const uint16_t *o, const uint16_t *g, const float *sg,
+                    int64_t R, int64_t C, int64_t ld, double eps,
+                    unsigned flags, uint16_t *y, double *y_exact, int nthreads);
+int or_swiglu_l2_rows(const uint16_t *g, const uint16_t *u, const float *sug,
+                      const float *suu, int64_t R, int64_t C, int64_t ld,
+                      double eps, unsigned flags, uint16_t *y, double *y_exact,
+                      int nthreads);
+int or_gate_l2_rows_interval(const uint16_t *o, const uint16_t *g,
+                             const float *sg, int64_t R, int64_t C, int64_t ld,
+                             double eps, double delta, unsigned flags,
+                             uint16_t *lo, uint16_t *hi, int nthreads);
+int or_swiglu_l2_rows_interval(const uint16_t *g, const uint16_t *u,
+                               const float *sug, const float *suu, int64_t R,
+                               int64_t C, int64_t ld, double eps, double delta,
+                               unsigned flags, uint16_t *lo, uint16_t *hi,
+                               int nthreads);
 
 /* Backward of the activation rows over matrices (bf16 bits in, f64 out).
  * dalpha (may be NULL) = the rows' parts summed in row order. */

@@ -18,6 +18,10 @@ OR_DROP_SLERP_B = 0x04
 OR_EPS_OUTSIDE = 0x08
 OR_EPS_ZERO = 0x10
 OR_BWD_PRINTED = 0x20
+OR_DROP_GATED = 0x40
+OR_DROP_SGATE = 0x80
+OR_DROP_SUP = 0x100
+OR_DROP_PRODUCT = 0x200
 
 _lib = None
 
@@ -42,6 +46,10 @@ def lib() -> ct.CDLL:
         _lib.or_grad_project_row.restype = None
         _lib.or_l2_rows.argtypes = [vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
         _lib.or_l2_rows_backward.argtypes = [vp, vp, vp, i64, i64, i64, dbl, uns, vp, i32]
+        _lib.or_gate_l2_rows.argtypes = [vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
+        _lib.or_swiglu_l2_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
+        _lib.or_gate_l2_rows_interval.argtypes = [vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
+        _lib.or_swiglu_l2_rows_interval.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
         _lib.or_slerp_rows_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, vp, i32]
         _lib.or_l2_row.argtypes = [vp, vp, i64, dbl, uns, vp, vp, vp]
         _lib.or_l2_row.restype = None
@@ -173,6 +181,55 @@ def slerp_rows(res, out, alpha, *, eps=1e-6, flags=0, nthreads=1, exact=False):
     _check(lib().or_slerp_rows(_p(res), _p(out), _p(alpha), R, C, ld, eps, flags, _p(h), _p(he), nthreads),
            "slerp_rows")
     return (h, he) if exact else h
+
+
+def _fused_args(a, b, *vecs):
+    a = np.ascontiguousarray(a, np.uint16)
+    b = np.ascontiguousarray(b, np.uint16)
+    R, C = a.shape
+    if b.shape != (R, C):
+        raise ValueError("shapes")
+    vs = [np.ascontiguousarray(v, np.float32) for v in vecs]
+    if any(v.shape != (C,) for v in vs):
+        raise ValueError("scale vector shape")
+    return a, b, vs, R, C
+
+
+def gate_l2_rows(o, g, sg, *, eps=1e-6, flags=0, nthreads=1, exact=False):
+    """bf16 bits y of bf16(l2(bf16(o * sigmoid(g * sg)))) (o, g bf16 bits, sg fp32 [C])."""
+    o, g, (sg,), R, C = _fused_args(o, g, sg)
+    y = np.empty((R, C), np.uint16)
+    ye = np.empty((R, C), np.float64) if exact else None
+    _check(lib().or_gate_l2_rows(_p(o), _p(g), _p(sg), R, C, C, eps, flags, _p(y), _p(ye), nthreads), "gate_l2")
+    return (y, ye) if exact else y
+
+
+def swiglu_l2_rows(g, u, sug, suu, *, eps=1e-6, flags=0, nthreads=1, exact=False):
+    """bf16 bits y of bf16(l2(bf16(silu(bf16(g * sug)) * bf16(u * suu))))."""
+    g, u, (sug, suu), R, C = _fused_args(g, u, sug, suu)
+    y = np.empty((R, C), np.uint16)
+    ye = np.empty((R, C), np.float64) if exact else None
+    _check(lib().or_swiglu_l2_rows(_p(g), _p(u), _p(sug), _p(suu), R, C, C, eps, flags, _p(y), _p(ye), nthreads),
+           "swiglu_l2")
+    return (y, ye) if exact else y
+
+
+def gate_l2_rows_interval(o, g, sg, *, eps=1e-6, delta=1e-5, flags=0, nthreads=1):
+    o, g, (sg,), R, C = _fused_args(o, g, sg)
+    lo = np.empty((R, C), np.uint16)
+    hi = np.empty((R, C), np.uint16)
+    _check(lib().or_gate_l2_rows_interval(_p(o), _p(g), _p(sg), R, C, C, eps, delta, flags, _p(lo), _p(hi),
+                                          nthreads), "gate_l2_interval")
+    return lo, hi
+
+
+def swiglu_l2_rows_interval(g, u, sug, suu, *, eps=1e-6, delta=1e-5, flags=0, nthreads=1):
+    g, u, (sug, suu), R, C = _fused_args(g, u, sug, suu)
+    lo = np.empty((R, C), np.uint16)
+    hi = np.empty((R, C), np.uint16)
+    _check(lib().or_swiglu_l2_rows_interval(_p(g), _p(u), _p(sug), _p(suu), R, C, C, eps, delta, flags, _p(lo),
+                                            _p(hi), nthreads), "swiglu_l2_interval")
+    return lo, hi
 
 
 def l2_rows_backward(x, r, dy, *, eps=1e-6, flags=0, nthreads=1):
