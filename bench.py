@@ -17,7 +17,7 @@ disjoint buffers (>= 268 MB of other traffic between two uses of one
 buffer), so inputs come from HBM without an explicit flush.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config step|mlp_pair|wide|optimizer|act_backward]
+                    [--config step|mlp_pair|wide|optimizer|act_backward|dory]
 
 `--config` selects another workload for a per-call report (default: the
 step above).  mlp_pair = up [2048,768] + down [768,2048] (fwd, bwd, renorm;
@@ -27,6 +27,8 @@ CUDA-graph replay of the calls is timed as well).  wide = weights
 [4096,16384] (l2, l2 + residual, slerp).  optimizer = ds_grad_project and
 ds_renorm_momentum over the whole-model weights.  act_backward = the
 backward of the activation calls on [16384,4096] (upstream gradient bf16).
+dory = Dory's gated and SwiGLU l2 rows on [16384,4096] and [8192,7168]
+(scale vectors fp32 U(0.5, 2)).
 
 Prints one JSON line (rank 0).  `value` is algorithmic bytes moved by all
 ranks per second (GB/s); per-kernel GB/s and rows/s, the roofline of the
@@ -71,6 +73,8 @@ WORKLOADS = {
                  "(fp32 gradient and momentum, in place)",
     "act_backward": "activation backward on rows [16384,4096] bf16: l2 (dx fp32), l2 with residual, slerp "
                     "(dres, dout fp32 and dalpha [4096] through its workspace)",
+    "dory": "Dory's fused activation rows: gated l2 rows (o, g bf16, sg fp32) and SwiGLU l2 rows (g, u bf16, "
+            "sug, suu fp32) on [16384,4096] and [8192,7168]",
 }
 
 
@@ -96,7 +100,8 @@ def call_bytes(kind: str, segs=None, act=None) -> int:
         A = act.rows * act.cols
         return {"l2": A * (2 + 2), "l2res": A * (2 + 2 + 2), "slerp": A * (2 + 2 + 2) + act.cols * 4,
                 "l2bwd": A * (2 + 2 + 4), "l2resbwd": A * (2 + 2 + 2 + 4),
-                "slerpbwd": A * (2 + 2 + 2 + 4 + 4) + act.cols * (4 + 4)}[kind]
+                "slerpbwd": A * (2 + 2 + 2 + 4 + 4) + act.cols * (4 + 4),
+                "gate": A * (2 + 2 + 2) + act.cols * 4, "swiglu": A * (2 + 2 + 2) + act.cols * (4 + 4)}[kind]
     E = sum(s.w.size for s in segs)
     R = sum(s.rows for s in segs)
     return {"fwd": E * (4 + 2) + R * 4, "bwd": E * (4 + 2 + 4) + R * (4 + 4), "renorm": E * (4 + 4),
@@ -146,6 +151,14 @@ def plan(config: str, seed: int):
         ag = {"x": wl.activations(seed, ACT_ROWS, ACT_COLS).acts[0]}
         calls = [("l2_rows_backward", "l2bwd", "x"), ("l2_rows_residual_backward", "l2resbwd", "x"),
                  ("slerp_rows_backward", "slerpbwd", "x")]
+        return {}, ag, calls, 1
+    if config == "dory":
+        ag = {"x": wl.activations(seed, ACT_ROWS, ACT_COLS).acts[0],
+              "7168": wl.activations(seed + 1, 8192, 7168).acts[0]}
+        calls = []
+        for g in ag:
+            sfx = "" if g == "x" else f"_{g}"
+            calls += [(f"gate_l2_rows{sfx}", "gate", g), (f"swiglu_l2_rows{sfx}", "swiglu", g)]
         return {}, ag, calls, 1
     if config == "optimizer":
         wg = {"model": wl.with_fp32_state(wl.whole_model(seed).weights, seed + 1)}
@@ -326,13 +339,18 @@ class Step:
         for name, a in self.ag.items():
             kinds = {k for _, k, g in self.plan if g == name}
             bwd = any(k.endswith("bwd") for k in kinds)
-            dy_host = None
+            dy_host = scales = None
+            if kinds & {"gate", "swiglu"}:   # per-column scales U(0.5, 2), seeded after the rows
+                srng = np.random.default_rng(seed + 11)
+                scales = [srng.uniform(0.5, 2.0, a.cols).astype(np.float32) for _ in range(2)]
             if bwd:   # the upstream gradient: bf16 N(0,1), seeded after the rows
                 dy_host = wl.normal_bf16(np.random.default_rng(seed + 7), a.x.shape)
             copies = []
             for c in range(self.copies):
                 x = bf16(a.x)
                 b = {"x": x, "r": bf16(a.r), "alpha": f32(a.alpha)}
+                if scales is not None:
+                    b["sa"], b["sb"] = f32(scales[0]), f32(scales[1])
                 if bwd:
                     b["dy"] = bf16(dy_host)
                     b["dx"] = torch.empty(a.x.shape, dtype=torch.float32, device=dev)
@@ -347,6 +365,8 @@ class Step:
             self.abuf[name] = copies
             b0 = copies[0]
             self.inputs += [(b0["x"], a.x.view(np.int16)), (b0["r"], a.r.view(np.int16)), (b0["alpha"], a.alpha)]
+            if scales is not None:
+                self.inputs += [(b0["sa"], scales[0]), (b0["sb"], scales[1])]
             if bwd:
                 self.inputs.append((b0["dy"], dy_host.view(np.int16)))
                 self.outputs += [b0["dx"], b0["dx2"], b0["dres"], b0["dout"], b0["dalpha"]]
@@ -411,6 +431,12 @@ class Step:
                             t, 1, eps, da.data_ptr(), ws.data_ptr(), ws.numel(), s))
                     else:
                         fn = lambda s, t=tab: lib.ds_l2_rows_backward(t, 1, eps, s)
+                elif kind in ("gate", "swiglu"):
+                    b = self.abuf[g][c]
+                    fseg = ds.FSeg(a=b["x"], b=b["r"], y=b["y"], sa=b["sa"], sb=b["sb"] if kind == "swiglu" else None)
+                    tab = (ds.ds_fseg * 1)(fseg.to_c())
+                    fn = (lambda s, t=tab: lib.ds_gate_l2_rows(t, 1, eps, s)) if kind == "gate" else \
+                         (lambda s, t=tab: lib.ds_swiglu_l2_rows(t, 1, eps, s))
                 else:
                     b = self.abuf[g][c]
                     if kind == "l2":

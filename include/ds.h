@@ -2,7 +2,7 @@
  * ds.h -- C ABI of libds: per-row L2 normalisation of weight and activation
  * rows on NVIDIA B200 (sm_100a).
  *
- * Nine operations, each over a table of segments (matrices), so that every
+ * Eleven operations, each over a table of segments (matrices), so that every
  * weight of a model is handled by one call:
  *
  *   ds_wn_forward   W_eff[r,:] = g_r * rho * w[r,:] / sqrt(sum_j w[r,j]^2 + eps)
@@ -34,6 +34,12 @@
  *                   t_j = a_j + |alpha_j| (b_j - a_j)  (fp32, one rounding),
  *                   y = bf16(t / sqrt(sum t^2 + eps)); same commit (tf_slerp_rows,
  *                   the normalised-lerp residual).
+ *   ds_gate_l2_rows  y = bf16(l2(bf16(o * sigmoid(g * sg))))  and
+ *   ds_swiglu_l2_rows  y = bf16(l2(bf16(silu(bf16(g * sug)) * bf16(u * suu)))):
+ *                   Dory's output gate and SwiGLU MLP rows, then the norm over
+ *                   the whole row; same PR (tf_gate_l2_rows, tf_swiglu_l2_rows),
+ *                   sigmoid and silu in fp32 as 1/(1+expf(-x)) and
+ *                   x/(1+expf(-x)) with IEEE division.
  *   ds_l2_rows_backward, ds_slerp_rows_backward  the gradients of the two
  *                   activation calls (derived: the pages give the forward only),
  *                   straight through the bf16 rounding points, which keep the
@@ -133,6 +139,21 @@ typedef struct {
     int64_t ld;   /* >= cols */
 } ds_aseg;
 
+/* One activation matrix for the Dory rows: a, b and y bf16 [rows, ld]
+ * (y may be exactly a or b), scale vectors fp32 [cols].
+ *   gate_l2_rows:   a = o, b = g, sa = sg (sb ignored)
+ *   swiglu_l2_rows: a = g (gate), b = u (up), sa = sug, sb = suu */
+typedef struct {
+    const void *a;
+    const void *b;
+    void *y;
+    const float *sa;
+    const float *sb;
+    int64_t rows; /* >= 0 */
+    int64_t cols; /* >= 1 */
+    int64_t ld;   /* >= cols */
+} ds_fseg;
+
 /* One activation matrix for the backward calls.  x, r and dy share the
  * leading dimension ld; dx and dr share ld_d.
  *   l2_rows_backward:    x bf16, r bf16 residual or NULL, dy bf16 = dL/dy,
@@ -183,6 +204,14 @@ ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps,
 
 ds_status ds_slerp_rows(const ds_aseg *segs, int nseg, float eps,
                         ds_stream stream);
+
+/* Rows must have at most 64 KB of staged input (a and b: 32 bytes per 8
+ * columns, so at most 16,384 columns); longer rows are refused with
+ * DS_ERR_INVALID_ARG.  Dory's widths are 4,096 and 7,168. */
+ds_status ds_gate_l2_rows(const ds_fseg *segs, int nseg, float eps,
+                          ds_stream stream);
+ds_status ds_swiglu_l2_rows(const ds_fseg *segs, int nseg, float eps,
+                            ds_stream stream);
 
 /* Rows must have at most 64 KB of staged input (x, r and dy: 48 bytes per 8
  * columns; l2 rows without a residual 32): at most 10,920 columns for slerp
@@ -245,7 +274,9 @@ typedef enum {
     DS_OP_GRAD_PROJECT = 5,
     DS_OP_RENORM_MOMENTUM = 6,
     DS_OP_L2_ROWS_BACKWARD = 7,
-    DS_OP_SLERP_ROWS_BACKWARD = 8
+    DS_OP_SLERP_ROWS_BACKWARD = 8,
+    DS_OP_GATE_L2_ROWS = 9,
+    DS_OP_SWIGLU_L2_ROWS = 10
 } ds_op;
 
 typedef enum {

@@ -72,6 +72,9 @@ int64_t tile_row_bytes_worst(ds_op op, int64_t cols, bool has_r = true)
 }
 
 bool is_act_bwd(ds_op op) { return op == DS_OP_L2_ROWS_BACKWARD || op == DS_OP_SLERP_ROWS_BACKWARD; }
+bool is_fused(ds_op op) { return op == DS_OP_GATE_L2_ROWS || op == DS_OP_SWIGLU_L2_ROWS; }
+// Operations with staged classes only (rows above the largest slot are refused).
+bool staged_only(ds_op op) { return is_act_bwd(op) || is_fused(op); }
 
 // Warps of a staged team: one (weights) or two (activations) per 16 KB of
 // slot; eight for the 112 KB weight slots.
@@ -79,7 +82,7 @@ int team_warps(ds_op op, int slot)
 {
     if (slot == ds::kTileSlotMaxWeightBytes)
         return 8;
-    const int base = (op == DS_OP_L2_ROWS || op == DS_OP_SLERP_ROWS || is_act_bwd(op)) ? 2 : 1;
+    const int base = (op == DS_OP_L2_ROWS || op == DS_OP_SLERP_ROWS || staged_only(op)) ? 2 : 1;
     return base * slot / ds::kTileSlotBytes;
 }
 
@@ -107,7 +110,7 @@ RowClass classify(ds_op op, int64_t cols, int forced, bool has_r = true)
                 return CL;
         return 0;
     };
-    if (is_act_bwd(op)) {
+    if (staged_only(op)) {
         // staged classes only; longer rows are refused (path 0)
         if (forced == DS_PATH_CTA && staged <= max_slot(op))
             return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
@@ -158,6 +161,8 @@ int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r, int slo
     case DS_OP_RENORM_MOMENTUM: bytes = 2 * q * 16; break;
     case DS_OP_L2_ROWS: bytes = o * 16 * (has_r ? 2 : 1); break;
     case DS_OP_L2_ROWS_BACKWARD: bytes = o * 16 * (has_r ? 3 : 2); break;
+    case DS_OP_GATE_L2_ROWS:
+    case DS_OP_SWIGLU_L2_ROWS: bytes = o * 16 * 2; break;
     case DS_OP_SLERP_ROWS_BACKWARD: bytes = o * 16 * 3; break;
     default: bytes = o * 32; break;
     }
@@ -563,6 +568,70 @@ ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *st
     return launch_all<AParams, ASegK>(nseg, rows.data(), cls, eps, make, launch, stream);
 }
 
+ds_status run_fused(bool swiglu, const ds_fseg *segs, int nseg, float eps, void *stream)
+{
+    g_last_error.clear();
+    if (ds_status s = check_common(nseg, segs, eps, stream))
+        return s;
+    const ds_op op = swiglu ? DS_OP_SWIGLU_L2_ROWS : DS_OP_GATE_L2_ROWS;
+    const int forced = g_force_path.load(std::memory_order_relaxed);
+    std::vector<Span> spans;
+    std::vector<int64_t> rows(static_cast<size_t>(nseg)), cols(static_cast<size_t>(nseg));
+    std::vector<RowClass> cls(static_cast<size_t>(nseg));
+    for (int i = 0; i < nseg; ++i) {
+        const ds_fseg &s = segs[i];
+        if (ds_status st = check_shape(s.rows, s.cols, s.ld, i))
+            return st;
+        rows[i] = s.rows;
+        cols[i] = s.cols;
+        cls[i] = classify(op, s.cols, forced);
+        if (cls[i].path == 0)
+            return fail(DS_ERR_INVALID_ARG, where("row too long (more than 64 KB of staged input)", i));
+        cls[i].rps = tile_rows_per_slot(op, s.cols, 2, true, cls[i].slot);
+        if (s.rows == 0)
+            continue;
+        if (ds_status st = check_matrix(s.a, s.rows, s.ld, 2, "a", i))
+            return st;
+        if (ds_status st = check_matrix(s.b, s.rows, s.ld, 2, "b", i))
+            return st;
+        if (ds_status st = check_matrix(s.y, s.rows, s.ld, 2, "y", i))
+            return st;
+        for (int k = 0; k < (swiglu ? 2 : 1); ++k) {
+            const float *v = k == 0 ? s.sa : s.sb;
+            if (!v)
+                return fail(DS_ERR_INVALID_ARG, where(k == 0 ? "sa is NULL" : "sb is NULL", i));
+            if (!aligned(v, 16))
+                return fail(DS_ERR_ALIGNMENT, where(k == 0 ? "sa is not 16-byte aligned" : "sb is not 16-byte aligned", i));
+            spans.push_back(span_of(v, 1, s.cols, s.cols, 4, i, 0, -1));
+        }
+        // y may be exactly a or exactly b (alias key = the segment)
+        spans.push_back(span_of(s.a, s.rows, s.cols, s.ld, 2, i, 0, i));
+        spans.push_back(span_of(s.b, s.rows, s.cols, s.ld, 2, i, 0, i));
+        spans.push_back(span_of(s.y, s.rows, s.cols, s.ld, 2, i, 1, i));
+    }
+    if (ds_status st = check_overlaps(spans))
+        return st;
+    auto make = [&](int i, int64_t r0, int64_t nr) {
+        const ds_fseg &s = segs[i];
+        ASegK k{};
+        k.x = s.a ? static_cast<const uint16_t *>(s.a) + r0 * s.ld : nullptr;
+        k.r = s.b ? static_cast<const uint16_t *>(s.b) + r0 * s.ld : nullptr;
+        k.y = s.y ? static_cast<uint16_t *>(s.y) + r0 * s.ld : nullptr;
+        k.alpha = s.sa;
+        k.s2 = swiglu ? s.sb : nullptr;
+        k.rows = nr;
+        k.ld = s.ld;
+        k.cols = static_cast<int32_t>(s.cols);
+        k.nu = static_cast<int32_t>((s.cols + 7) / 8);
+        return k;
+    };
+    auto launch = [&](const RowClass &rc, const AParams &p, int64_t units, void *st) -> int {
+        const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
+        return ds::launch_tile(swiglu ? 12 : 11, &p, grid, rc.slot, st);
+    };
+    return launch_all<AParams, ASegK>(nseg, rows.data(), cls, eps, make, launch, stream);
+}
+
 AGSegK agseg_rows(const ds_agseg &s, int64_t r0, int64_t nr)
 {
     AGSegK k{};
@@ -734,6 +803,16 @@ ds_status ds_renorm_momentum(const ds_wseg *segs, int nseg, float eps, ds_stream
     return run_weight(W_MOMENTUM, segs, nseg, DS_F32, eps, stream);
 }
 
+ds_status ds_gate_l2_rows(const ds_fseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_fused(false, segs, nseg, eps, stream);
+}
+
+ds_status ds_swiglu_l2_rows(const ds_fseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_fused(true, segs, nseg, eps, stream);
+}
+
 ds_status ds_l2_rows_backward(const ds_agseg *segs, int nseg, float eps, ds_stream stream)
 {
     return run_act_bwd(false, segs, nseg, eps, nullptr, nullptr, 0, stream);
@@ -812,7 +891,7 @@ int ds_version(void) { return 100; }
 
 ds_status ds_row_class(ds_op op, int64_t cols, int *path, int *group_threads, int *cluster_ctas)
 {
-    if (op < DS_OP_WN_FORWARD || op > DS_OP_SLERP_ROWS_BACKWARD)
+    if (op < DS_OP_WN_FORWARD || op > DS_OP_SWIGLU_L2_ROWS)
         return fail(DS_ERR_INVALID_ARG, "unknown op");
     if (cols < 1 || cols > kMaxCols)
         return fail(DS_ERR_INVALID_ARG, "cols outside [1, 2^31 - 1]");

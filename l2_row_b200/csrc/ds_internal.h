@@ -92,7 +92,8 @@ struct ASegK {
     const uint16_t *x;
     const uint16_t *r;
     uint16_t *y;
-    const float *alpha;
+    const float *alpha;  // slerp: alpha; Dory rows: the first scale vector
+    const float *s2;     // SwiGLU rows: the second scale vector
     int64_t rows;
     int64_t ld;
     int32_t cols;
@@ -156,8 +157,9 @@ int launch_wait_selftest(uint64_t limit_ns, void *stream);
 // Staged paths (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,
 // 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp,
 // 7 gradient projection, 8 momentum projection + renorm, 9 l2 backward,
-// 10 slerp backward; params is a WParams (tags 0-4, 7, 8), AParams (5, 6) or
-// GParams (9, 10) whose segments carry rows per slot in `group` and whose
+// 10 slerp backward, 11 gated l2 rows, 12 SwiGLU l2 rows; params is a WParams
+// (tags 0-4, 7, 8), AParams (5, 6, 11, 12) or GParams (9, 10) whose segments
+// carry rows per slot in `group` and whose
 // unit_start counts slots; slot_bytes 16, 32, 64 or (weights) 112 KB.
 int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream);
 // Ring positions (consumer teams) per CTA of a staged launch.

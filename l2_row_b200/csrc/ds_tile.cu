@@ -25,11 +25,18 @@
 namespace ds {
 
 // ds_kernels.cu's tags, repeated (the two files share this numbering).
-enum TileTag { tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp, tProject, tMomentum, tL2Bwd, tSlerpBwd };
+enum TileTag {
+    tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp, tProject, tMomentum, tL2Bwd, tSlerpBwd, tGateL2,
+    tSwigluL2
+};
 
 __host__ __device__ constexpr bool is_weight_tag(int T) { return T <= tRenorm || T == tProject || T == tMomentum; }
 __host__ __device__ constexpr bool is_act_bwd_tag(int T) { return T == tL2Bwd || T == tSlerpBwd; }
-__host__ __device__ constexpr bool is_act_tag(int T) { return T == tL2 || T == tSlerp || is_act_bwd_tag(T); }
+__host__ __device__ constexpr bool is_fused_tag(int T) { return T == tGateL2 || T == tSwigluL2; }
+__host__ __device__ constexpr bool is_act_tag(int T)
+{
+    return T == tL2 || T == tSlerp || is_act_bwd_tag(T) || is_fused_tag(T);
+}
 
 namespace {
 
@@ -1053,6 +1060,85 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP> &tm, const AGSegK &s
     }
 }
 
+// ============================================================ Dory rows ==
+//
+// Gated and SwiGLU rows, then their l2 over the whole row (a pair of warps
+// per row, as tile_l2_row).  Pass 1 forms the row's bf16 value s from the
+// two staged inputs (a, b) and the scale vectors, writes it back over a in
+// the slot and sums s^2; pass 2 is l2's.  Every fp32 step is the one the
+// definition names, in its order, with no contraction:
+//   gate:   z = b sa, e = expf(-z), sig = 1 / (1 + e), s = bf16(a sig)
+//   swiglu: gs = bf16(a sa), us = bf16(b sb), sl = gs / (1 + expf(-gs)),
+//           s = bf16(sl us)
+template <int PRO>
+__device__ __forceinline__ uint4 fused_unit(uint4 a, uint4 b, const float2 (&sa)[4], const float2 (&sb)[4])
+{
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 av = lo2(word4(a, i)), bv = lo2(word4(b, i));
+        float v0, v1;
+        if constexpr (PRO == 0) {
+            const float z0 = __fmul_rn(bv.x, sa[i].x), z1 = __fmul_rn(bv.y, sa[i].y);
+            const float g0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z0)));
+            const float g1 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z1)));
+            v0 = __fmul_rn(av.x, g0);
+            v1 = __fmul_rn(av.y, g1);
+        } else {
+            const float2 gs = lo2(pack_bf2(__fmul_rn(av.x, sa[i].x), __fmul_rn(av.y, sa[i].y)));
+            const float2 us = lo2(pack_bf2(__fmul_rn(bv.x, sb[i].x), __fmul_rn(bv.y, sb[i].y)));
+            const float s0 = __fdiv_rn(gs.x, __fadd_rn(1.0f, expf(-gs.x)));
+            const float s1 = __fdiv_rn(gs.y, __fadd_rn(1.0f, expf(-gs.y)));
+            v0 = __fmul_rn(s0, us.x);
+            v1 = __fmul_rn(s1, us.y);
+        }
+        w[i] = pack_bf2(v0, v1);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <int WP, int PRO>
+__device__ __forceinline__ void tile_fused_row(Team<WP> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
+                                               const unsigned char *s1, int nfull, int tail, float eps, bool store)
+{
+    constexpr int G = Team<WP>::G;
+    const int t = tm.t;
+    const bool tl = tail && t == nfull % G;
+    const int nunits = nfull + (tail ? 1 : 0);
+    uint4 *x = reinterpret_cast<uint4 *>(s0);
+    const uint4 *r = reinterpret_cast<const uint4 *>(s1);
+    float2 acc = f2(0.f, 0.f);
+#pragma unroll 2
+    for (int u = t; u < nunits; u += G) {
+        float2 va[4], vb[4];
+        alpha8_signed<false>(nullptr, 0, sg.alpha, u, sg.cols, va);
+        if constexpr (PRO == 1)
+            alpha8_signed<false>(nullptr, 0, sg.s2, u, sg.cols, vb);
+        else
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                vb[i] = f2(0.f, 0.f);
+        uint4 sv = fused_unit<PRO>(x[u], r[u], va, vb);
+        if (u == nfull && tl)
+            sv = mask_octet(sv, tail);
+        x[u] = sv;
+        sq8w(acc, sv);
+    }
+    const float S = tm.sum1(acc.x + acc.y);
+    const RowScale rs = tile_scale(tm, S, eps, [&](auto f) {
+        for (int u = t; u < nunits; u += G)
+            pairs8(x[u], f);
+    });
+    if (!store)
+        return;
+    uint16_t *y = sg.y + row * sg.ld;
+#pragma unroll 4
+    for (int u = t; u < nfull; u += G)
+        st16(y + 8 * u, scale8(x[u], rs));
+    if (tl)
+        store_tail8(y + 8 * nfull, scale8(x[nfull], rs), tail);
+}
+
 // =============================================================== kernel ==
 
 template <int T>
@@ -1317,6 +1403,10 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                         tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
                     else
                         tile_l2_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
+                } else if constexpr (T == tGateL2) {
+                    tile_fused_row<WP, 0>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
+                } else if constexpr (T == tSwigluL2) {
+                    tile_fused_row<WP, 1>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
                 } else if constexpr (T == tL2Bwd) {
                     if (has_r)
                         tile_l2_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
@@ -1395,6 +1485,8 @@ int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *str
     case tMomentum: return launch_tile_t<tMomentum>(params, grid, slot_bytes, stream);
     case tL2Bwd: return launch_tile_t<tL2Bwd>(params, grid, slot_bytes, stream);
     case tSlerpBwd: return launch_tile_t<tSlerpBwd>(params, grid, slot_bytes, stream);
+    case tGateL2: return launch_tile_t<tGateL2>(params, grid, slot_bytes, stream);
+    case tSwigluL2: return launch_tile_t<tSwigluL2>(params, grid, slot_bytes, stream);
     default: return cudaErrorInvalidValue;
     }
 }

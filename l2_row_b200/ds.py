@@ -13,6 +13,8 @@ The five calls keep their C names and take lists of segments:
     ds_renorm_momentum(segs, eps, stream=None)    (grad_w = the momentum, in place)
     ds_l2_rows(segs, eps, stream=None)
     ds_slerp_rows(segs, eps, stream=None)
+    ds_gate_l2_rows(segs, eps, stream=None)       (Dory's gated rows)
+    ds_swiglu_l2_rows(segs, eps, stream=None)     (Dory's SwiGLU rows)
     ds_l2_rows_backward(segs, eps, stream=None)
     ds_slerp_rows_backward(segs, eps, dalpha=None, workspace=None, stream=None)
 
@@ -42,6 +44,7 @@ DS_F32, DS_BF16 = 0, 1
 DS_OP_WN_FORWARD, DS_OP_WN_BACKWARD, DS_OP_ROW_RENORM, DS_OP_L2_ROWS, DS_OP_SLERP_ROWS = range(5)
 DS_OP_GRAD_PROJECT, DS_OP_RENORM_MOMENTUM = 5, 6
 DS_OP_L2_ROWS_BACKWARD, DS_OP_SLERP_ROWS_BACKWARD = 7, 8
+DS_OP_GATE_L2_ROWS, DS_OP_SWIGLU_L2_ROWS = 9, 10
 DS_PATH_AUTO, DS_PATH_WARP, DS_PATH_CTA, DS_PATH_CLUSTER, DS_PATH_TWO_PASS = range(5)
 DS_MAX_SEGMENTS = 65536
 PATH_NAMES = {DS_PATH_WARP: "warp", DS_PATH_CTA: "cta", DS_PATH_CLUSTER: "cluster", DS_PATH_TWO_PASS: "two_pass"}
@@ -56,6 +59,11 @@ class ds_wseg(ct.Structure):
 class ds_aseg(ct.Structure):
     _fields_ = [("x", ct.c_void_p), ("r", ct.c_void_p), ("y", ct.c_void_p), ("alpha", ct.c_void_p),
                 ("rows", ct.c_int64), ("cols", ct.c_int64), ("ld", ct.c_int64)]
+
+
+class ds_fseg(ct.Structure):
+    _fields_ = [("a", ct.c_void_p), ("b", ct.c_void_p), ("y", ct.c_void_p), ("sa", ct.c_void_p),
+                ("sb", ct.c_void_p), ("rows", ct.c_int64), ("cols", ct.c_int64), ("ld", ct.c_int64)]
 
 
 class ds_agseg(ct.Structure):
@@ -73,6 +81,8 @@ _lib.ds_renorm_momentum.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, c
 _lib.ds_l2_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_slerp_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_l2_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_gate_l2_rows.argtypes = [ct.POINTER(ds_fseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_swiglu_l2_rows.argtypes = [ct.POINTER(ds_fseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_slerp_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p, ct.c_void_p,
                                         ct.c_uint64, ct.c_void_p]
 _lib.ds_slerp_rows_backward_noalloc.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p,
@@ -82,7 +92,7 @@ _lib.ds_slerp_rows_backward_workspace.argtypes = [ct.c_int64]
 _lib.ds_slerp_rows_backward_workspace.restype = ct.c_uint64
 for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
-           "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
+           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
            "ds_debug_wait_timeout_selftest"):
     getattr(_lib, _f).restype = _st
 _lib.ds_status_string.argtypes = [ct.c_int]
@@ -103,7 +113,7 @@ _lib.ds_debug_wait_timeout_selftest.argtypes = [ct.c_uint64, ct.c_void_p]
 #: every symbol include/ds.h declares
 EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
-           "ds_slerp_rows_backward_workspace", "ds_slerp_rows_backward_noalloc", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
+           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_slerp_rows_backward_workspace", "ds_slerp_rows_backward_noalloc", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
            "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest")
 
 
@@ -221,6 +231,28 @@ class ASeg:
 
 
 @dataclass
+class FSeg:
+    """One activation matrix for Dory's rows: a, b, y bf16 [R, C] with a
+    shared ld; sa (and for SwiGLU sb) fp32 [C].  Gate: a = o, b = g, sa = sg;
+    SwiGLU: a = g, b = u, sa = sug, sb = suu."""
+
+    a: Any
+    b: Any
+    y: Any
+    sa: Any
+    sb: Any = None
+
+    def to_c(self) -> ds_fseg:
+        R, C = (int(self.a.shape[0]), int(self.a.shape[1]))
+        a, ld = _mat(self.a, "a", R, C)
+        b, ldb = _mat(self.b, "b", R, C)
+        y, ldy = _mat(self.y, "y", R, C)
+        if ldb != ld or ldy != ld:
+            raise ValueError("a, b and y must share a leading dimension")
+        return ds_fseg(a, b, y, _vec(self.sa), _vec(self.sb), R, C, ld)
+
+
+@dataclass
 class AGSeg:
     """One activation matrix for the backward calls: x (slerp: res), r (l2:
     residual or None; slerp: out), dy the upstream gradient (bf16 [R, C],
@@ -287,6 +319,16 @@ def ds_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
 def ds_slerp_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
     arr, n = _table(segs, ds_aseg)
     _check(_lib.ds_slerp_rows(arr, n, eps, _stream_ptr(stream)), "ds_slerp_rows")
+
+
+def ds_gate_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_fseg)
+    _check(_lib.ds_gate_l2_rows(arr, n, eps, _stream_ptr(stream)), "ds_gate_l2_rows")
+
+
+def ds_swiglu_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_fseg)
+    _check(_lib.ds_swiglu_l2_rows(arr, n, eps, _stream_ptr(stream)), "ds_swiglu_l2_rows")
 
 
 def ds_l2_rows_backward(segs: Sequence, eps: float = 1e-6, stream=None) -> None:

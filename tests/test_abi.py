@@ -344,3 +344,46 @@ def test_backward_validation(fn):
         assert call_g(fn, [agseg(**good), other], dalpha=da, ws=ws, ws_bytes=need) == E.DS_ERR_INVALID_ARG
         assert call_g(fn, [agseg(**good)], dalpha=ws, ws=ws, ws_bytes=need) == E.DS_ERR_OVERLAP
     assert ds.ds_launch_count() == before
+
+
+# ----------------------------------------------------------- Dory's rows --
+
+def fseg(**kw):
+    d = dict(a=BASE, b=BASE + (1 << 30), y=BASE + (2 << 30), sa=BASE + (3 << 30), sb=BASE + (4 << 30),
+             rows=4, cols=8, ld=8)
+    d.update(kw)
+    return ds.ds_fseg(**d)
+
+
+def call_f(fn, segs, eps=1e-6):
+    arr = (ds.ds_fseg * max(1, len(segs)))(*segs)
+    return getattr(ds.lib(), fn)(arr, len(segs), ct.c_float(eps), None)
+
+
+def test_fused_row_classes():
+    # a and b staged: 32 bytes per 8 columns; a pair of warps per 16 KB of slot
+    assert ds.ds_row_class(ds.DS_OP_GATE_L2_ROWS, 4096) == (ds.DS_PATH_WARP, 64, 1)
+    assert ds.ds_row_class(ds.DS_OP_SWIGLU_L2_ROWS, 7168) == (ds.DS_PATH_CTA, 128, 1)
+    assert ds.ds_row_class(ds.DS_OP_SWIGLU_L2_ROWS, 16384) == (ds.DS_PATH_CTA, 256, 1)
+    with pytest.raises(ds.DSError):
+        ds.ds_row_class(ds.DS_OP_GATE_L2_ROWS, 16385)
+
+
+@pytest.mark.parametrize("fn", ["ds_gate_l2_rows", "ds_swiglu_l2_rows"])
+def test_fused_validation(fn):
+    E = ds
+    before = ds.ds_launch_count()
+    assert call_f(fn, [fseg(rows=-1)]) == E.DS_ERR_INVALID_ARG
+    assert call_f(fn, [fseg(a=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_f(fn, [fseg(b=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_f(fn, [fseg(y=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_f(fn, [fseg(sa=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_f(fn, [fseg(sa=BASE + (3 << 30) + 4)]) == E.DS_ERR_ALIGNMENT
+    assert call_f(fn, [fseg(a=BASE + 2)]) == E.DS_ERR_ALIGNMENT
+    assert call_f(fn, [fseg(cols=16385, ld=16392)]) == E.DS_ERR_INVALID_ARG
+    assert call_f(fn, [fseg(y=BASE + 16)]) == E.DS_ERR_OVERLAP            # partial overlap with a
+    assert call_f(fn, [fseg()], eps=-1.0) == E.DS_ERR_INVALID_ARG
+    if fn == "ds_swiglu_l2_rows":
+        assert call_f(fn, [fseg(sb=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_f(fn, [fseg(rows=0, a=0, b=0, y=0)]) == E.DS_OK
+    assert ds.ds_launch_count() == before
