@@ -277,11 +277,17 @@ ds_status check_matrix(const void *p, int64_t rows, int64_t ld, int esize, const
 // Slerp launches whose segments all use one alpha vector of at most
 // kTileAlphaCacheMax columns let the staged kernel keep |alpha| in shared
 // memory (the kernel checks the length against its own cache).
-inline void shared_alpha(WParams &p, int) { p.alpha_shared = nullptr; p.alpha_cols = 0; }
+// The Dory rows do the same with their scale vectors (sa, and sb when every
+// segment shares one).
+inline void shared_alpha(WParams &p, int)
+{
+    p.alpha_shared = p.alpha2_shared = nullptr;
+    p.alpha_cols = 0;
+}
 template <class P>
 inline void shared_alpha_act(P &p, int n)
 {
-    p.alpha_shared = nullptr;
+    p.alpha_shared = p.alpha2_shared = nullptr;
     p.alpha_cols = 0;
     if (n == 0 || !p.seg[0].alpha || p.seg[0].cols > ds::kTileAlphaCacheMax)
         return;
@@ -291,7 +297,16 @@ inline void shared_alpha_act(P &p, int n)
     p.alpha_shared = p.seg[0].alpha;
     p.alpha_cols = p.seg[0].cols;
 }
-inline void shared_alpha(AParams &p, int n) { shared_alpha_act(p, n); }
+inline void shared_alpha(AParams &p, int n)
+{
+    shared_alpha_act(p, n);
+    if (!p.alpha_shared || n == 0 || !p.seg[0].s2)
+        return;
+    for (int i = 1; i < n; ++i)
+        if (p.seg[i].s2 != p.seg[0].s2)
+            return;
+    p.alpha2_shared = p.seg[0].s2;
+}
 inline void shared_alpha(GParams &p, int n) { shared_alpha_act(p, n); }
 
 struct NoPrep {

@@ -126,8 +126,10 @@ struct LaunchParams {
     int32_t nseg;
     float eps;
     uint64_t wait_limit_ns;                // bound of every device-side wait
-    const float *alpha_shared;             // slerp: alpha of every segment (or NULL if they differ)
-    int32_t alpha_cols;                    //        its length
+    const float *alpha_shared;             // slerp: alpha of every segment (or NULL if they differ);
+                                           // Dory rows: the first scale vector
+    const float *alpha2_shared;            // SwiGLU rows: the second scale vector (or NULL)
+    int32_t alpha_cols;                    //        their length
     int32_t ws_ld;                         // slerp backward: floats per workspace line
     float *ws;                             //        per-team dalpha partial sums (NULL: no dalpha)
 };

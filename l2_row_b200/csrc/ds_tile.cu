@@ -1080,8 +1080,9 @@ __device__ __forceinline__ uint4 fused_unit(uint4 a, uint4 b, const float2 (&sa)
         float v0, v1;
         if constexpr (PRO == 0) {
             const float z0 = __fmul_rn(bv.x, sa[i].x), z1 = __fmul_rn(bv.y, sa[i].y);
-            const float g0 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z0)));
-            const float g1 = __fdiv_rn(1.0f, __fadd_rn(1.0f, expf(-z1)));
+            // 1 / d with IEEE division is d's correctly rounded reciprocal
+            const float g0 = __frcp_rn(__fadd_rn(1.0f, expf(-z0)));
+            const float g1 = __frcp_rn(__fadd_rn(1.0f, expf(-z1)));
             v0 = __fmul_rn(av.x, g0);
             v1 = __fmul_rn(av.y, g1);
         } else {
@@ -1097,9 +1098,10 @@ __device__ __forceinline__ uint4 fused_unit(uint4 a, uint4 b, const float2 (&sa)
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-template <int WP, int PRO>
+template <int WP, int PRO, bool CACHED>
 __device__ __forceinline__ void tile_fused_row(Team<WP> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
-                                               const unsigned char *s1, int nfull, int tail, float eps, bool store)
+                                               const unsigned char *s1, int nfull, int tail, float eps, bool store,
+                                               const float *ca, const float *cb, int half)
 {
     constexpr int G = Team<WP>::G;
     const int t = tm.t;
@@ -1111,9 +1113,9 @@ __device__ __forceinline__ void tile_fused_row(Team<WP> &tm, const ASegK &sg, in
 #pragma unroll 2
     for (int u = t; u < nunits; u += G) {
         float2 va[4], vb[4];
-        alpha8_signed<false>(nullptr, 0, sg.alpha, u, sg.cols, va);
+        alpha8_signed<CACHED>(ca, half, sg.alpha, u, sg.cols, va);
         if constexpr (PRO == 1)
-            alpha8_signed<false>(nullptr, 0, sg.s2, u, sg.cols, vb);
+            alpha8_signed<CACHED>(cb, half, sg.s2, u, sg.cols, vb);
         else
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -1160,11 +1162,19 @@ struct TileCfg {
     static constexpr int kSlotBytes = SB;
     static constexpr int kScale = SB == 114688 ? 8 : SB / 16384;    // 1, 2, 4; 8 for 112 KB
     static constexpr int kWP = (is_act_tag(T) ? 2 : 1) * kScale;
-    static constexpr int kGroups = SB == 16384 ? 13 : SB == 32768 ? 6 : SB == 65536 ? 3 : 2;
+    // SwiGLU rows keep two scale vectors in shared memory: one position fewer
+    static constexpr int kGroups = SB == 16384 ? (T == tSwigluL2 ? 12 : 13)
+                                   : SB == 32768 ? (T == tSwigluL2 ? 5 : 6)
+                                   : SB == 65536 ? 3 : 2;
     static constexpr int kSlots = kGroups;                          // one position per team
     static constexpr int kConsumers = kWP * kGroups;
     static constexpr int kThreads = (kConsumers + 1) * 32;
-    static constexpr int kAlphaCache = (T == tSlerp || T == tSlerpBwd) ? (SB == 16384 ? 4096 : 8192) : 0;
+    // Columns of each per-column vector held in shared memory after the ring
+    // (slerp: alpha; Dory rows: the scale vectors, none in 64 KB slots)
+    static constexpr int kAlphaCache = (T == tSlerp || T == tSlerpBwd) ? (SB == 16384 ? 4096 : 8192)
+                                       : (T == tGateL2 || T == tSwigluL2) ? (SB == 16384 ? 4096 : SB == 32768 ? 8192 : 0)
+                                                                         : 0;
+    static constexpr int kVecs = T == tSwigluL2 ? 2 : 1;
     // Refill pacing: the producer sleeps this long after each refill.  For
     // the operations below a paced read stream ran faster on B200 (l2 rows
     // with a residual 74 -> 67 us, the momentum projection + renorm 274 ->
@@ -1174,6 +1184,8 @@ struct TileCfg {
         ((SB == 16384 && (T == tL2 || T == tMomentum)) || (SB == 32768 && (T == tBwdBf16 || T == tBwdF32))) ? 300
                                                                                                            : 0;
     static_assert(kSlots <= kMaxTileSlots && kConsumers + 1 <= 32, "ring shape");
+    static constexpr int kSmem = SB * kSlots + 4 * kAlphaCache * kVecs;
+    static_assert(kSmem <= 229376, "ring and vector caches fit 224 KB");
 };
 
 template <int T, int SB>
@@ -1219,6 +1231,18 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                 const float a = i < p.alpha_cols ? __ldg(p.alpha_shared + i) : 0.f;
                 const float v = T == tSlerpBwd ? a : fabsf(a);
                 s_alpha[(e < 4 ? 0 : half) + 4 * u + (e & 3)] = v;
+            }
+        }
+    }
+    if constexpr (T == tGateL2 || T == tSwigluL2) {
+        // the scale vectors in the same split layout, sb after sa
+        if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache && (T == tGateL2 || p.alpha2_shared)) {
+            const int nu = (p.alpha_cols + 7) / 8, half = Cfg::kAlphaCache / 2;
+            for (int i = threadIdx.x; i < 8 * nu; i += blockDim.x) {
+                const int u = i >> 3, e = i & 7, at = (e < 4 ? 0 : half) + 4 * u + (e & 3);
+                s_alpha[at] = i < p.alpha_cols ? __ldg(p.alpha_shared + i) : 0.f;
+                if constexpr (T == tSwigluL2)
+                    s_alpha[Cfg::kAlphaCache + at] = i < p.alpha_cols ? __ldg(p.alpha2_shared + i) : 0.f;
             }
         }
     }
@@ -1403,10 +1427,15 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                         tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
                     else
                         tile_l2_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
-                } else if constexpr (T == tGateL2) {
-                    tile_fused_row<WP, 0>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
-                } else if constexpr (T == tSwigluL2) {
-                    tile_fused_row<WP, 1>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
+                } else if constexpr (T == tGateL2 || T == tSwigluL2) {
+                    constexpr int PRO = T == tGateL2 ? 0 : 1;
+                    constexpr int H = Cfg::kAlphaCache / 2;
+                    if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache && (PRO == 0 || p.alpha2_shared))
+                        tile_fused_row<WP, PRO, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
+                                                      s_alpha + Cfg::kAlphaCache, H);
+                    else
+                        tile_fused_row<WP, PRO, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr,
+                                                       nullptr, 0);
                 } else if constexpr (T == tL2Bwd) {
                     if (has_r)
                         tile_l2_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
@@ -1442,7 +1471,7 @@ template <int T, int SB>
 static cudaError_t launch_tile_sb(const TParams<T> &p, int grid, void *stream)
 {
     using Cfg = TileCfg<T, SB>;
-    constexpr int smem = SB * Cfg::kSlots + 4 * Cfg::kAlphaCache;
+    constexpr int smem = Cfg::kSmem;
     static bool attr_set = false; // benign race: idempotent
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_tile<T, SB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1507,6 +1536,8 @@ int tile_groups(int tag, int slot_bytes)
     switch (tag) {
     case tL2Bwd: return tile_groups_t<tL2Bwd>(slot_bytes);
     case tSlerpBwd: return tile_groups_t<tSlerpBwd>(slot_bytes);
+    case tGateL2: return tile_groups_t<tGateL2>(slot_bytes);
+    case tSwigluL2: return tile_groups_t<tSwigluL2>(slot_bytes);
     default: return 0;
     }
 }
