@@ -313,6 +313,15 @@ ds_status ds_debug_set_wait_limit_ns(uint64_t limit_ns);
  * ds_get_device_status returns DS_ERR_DEVICE_TIMEOUT.  No copy is in flight. */
 ds_status ds_debug_wait_timeout_selftest(uint64_t limit_ns, ds_stream stream);
 
+/* Checks, over every fp32 bit pattern v, the reciprocal and quotient the Dory
+ * rows compute where their fast range applies (gate: 1/(1 + expf(-v));
+ * silu: v/(1 + expf(-v))) against IEEE division (__frcp_rn, __fdiv_rn),
+ * bit for bit.  counts: DEVICE array of 4 uint64, overwritten with
+ * {reciprocal mismatches, quotient mismatches, inputs checked for the
+ * reciprocal, inputs checked for the quotient}.  Asynchronous on `stream`.
+ * The pages have no counterpart: it tests this library's arithmetic. */
+ds_status ds_debug_division_check(uint64_t *counts, ds_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -947,4 +947,17 @@ ds_status ds_debug_wait_timeout_selftest(uint64_t limit_ns, ds_stream stream)
     return DS_OK;
 }
 
+ds_status ds_debug_division_check(uint64_t *counts, ds_stream stream)
+{
+    if (!counts)
+        return fail(DS_ERR_INVALID_ARG, "counts is NULL");
+    if (reinterpret_cast<uintptr_t>(counts) % 8)
+        return fail(DS_ERR_ALIGNMENT, "counts must be 8-byte aligned");
+    const int e = ds::launch_division_check(reinterpret_cast<unsigned long long *>(counts), stream);
+    if (e != 0)
+        return fail(DS_ERR_CUDA, "division check launch failed");
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return DS_OK;
+}
+
 } // extern "C"

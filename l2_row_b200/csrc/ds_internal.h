@@ -173,6 +173,8 @@ int builtin_scratch(void **ptr, uint64_t *bytes);
 // ws[(c0 * groups + q) * ws_ld + c], in that order (slerp backward).
 int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64_t total_units, int cols,
                          float *dalpha, void *stream);
+// Exhaustive check of the Dory rows' fast reciprocal and quotient (ds_tile.cu).
+int launch_division_check(unsigned long long *counts, void *stream);
 int read_and_clear_device_error(uint32_t *code, uint32_t *site, void *stream);
 
 } // namespace ds

@@ -1070,32 +1070,129 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP> &tm, const AGSegK &s
 //   gate:   z = b sa, e = expf(-z), sig = 1 / (1 + e), s = bf16(a sig)
 //   swiglu: gs = bf16(a sa), us = bf16(b sb), sl = gs / (1 + expf(-gs)),
 //           s = bf16(sl us)
+//
+// The IEEE reciprocal and quotient come from Markstein's fused multiply-add
+// iteration (P. Markstein, "Computation of elementary functions on the IBM
+// RISC System/6000 processor", IBM J. Res. Develop. 34(1), 1990): from y0,
+// the hardware's approximate reciprocal of d, y = y0 + y0 (1 - d y0) is 1/d
+// rounded to nearest, and with q = RN(x y), q + y (x - d q) is x/d rounded to
+// nearest; the quotient takes x's sign, so that -0 stays -0.  This runs where
+// every d of the unit lies in [1, 2^126) (no subnormal reciprocal) and, for
+// silu, no x is +inf; any other unit takes __frcp_rn / __fdiv_rn.  On that
+// range both agree with IEEE division for every fp32 input, which
+// ds_debug_division_check counts on the device.
+__device__ __forceinline__ float2 rcp_approx2(float2 d)
+{
+    float2 y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y.x) : "f"(d.x));
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y.y) : "f"(d.y));
+    return y;
+}
+
+__device__ __forceinline__ float2 neg2(float2 v) { return f2(-v.x, -v.y); }
+
+// 1/d, d in [1, 2^126)
+__device__ __forceinline__ float2 rcp_fast2(float2 d)
+{
+    const float2 y0 = rcp_approx2(d);
+    const float2 e = __ffma2_rn(neg2(d), y0, f2(1.f, 1.f));
+    return __ffma2_rn(e, y0, y0);
+}
+
+__device__ __forceinline__ float copy_sign_bit(float q, float x)
+{
+    return __int_as_float((__float_as_int(q) & 0x7fffffff) | (__float_as_int(x) & int(0x80000000u)));
+}
+
+// x/d from y = RN(1/d), d in [1, 2^126), x finite
+__device__ __forceinline__ float2 div_fast2(float2 x, float2 d, float2 y)
+{
+    const float2 q = __fmul2_rn(x, y);
+    const float2 r = __ffma2_rn(neg2(d), q, x);
+    const float2 v = __ffma2_rn(r, y, q);
+    return f2(copy_sign_bit(v.x, x.x), copy_sign_bit(v.y, x.y));
+}
+
+constexpr uint32_t kFastDLimit = 0x7E800000u; // bits of 2^126
+
 template <int PRO>
 __device__ __forceinline__ uint4 fused_unit(uint4 a, uint4 b, const float2 (&sa)[4], const float2 (&sb)[4])
 {
-    uint32_t w[4];
+    float2 x[4], d[4], m[4]; // gate: m = a; swiglu: x = gs, m = us
+    uint32_t dmax = 0;
+    int xmax = int(0x80000000u);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const float2 av = lo2(word4(a, i)), bv = lo2(word4(b, i));
-        float v0, v1;
         if constexpr (PRO == 0) {
-            const float z0 = __fmul_rn(bv.x, sa[i].x), z1 = __fmul_rn(bv.y, sa[i].y);
-            // 1 / d with IEEE division is d's correctly rounded reciprocal
-            const float g0 = __frcp_rn(__fadd_rn(1.0f, expf(-z0)));
-            const float g1 = __frcp_rn(__fadd_rn(1.0f, expf(-z1)));
-            v0 = __fmul_rn(av.x, g0);
-            v1 = __fmul_rn(av.y, g1);
+            const float2 z = __fmul2_rn(lo2(word4(b, i)), sa[i]);
+            d[i] = __fadd2_rn(f2(1.f, 1.f), f2(expf(-z.x), expf(-z.y)));
+            m[i] = lo2(word4(a, i));
         } else {
-            const float2 gs = lo2(pack_bf2(__fmul_rn(av.x, sa[i].x), __fmul_rn(av.y, sa[i].y)));
-            const float2 us = lo2(pack_bf2(__fmul_rn(bv.x, sb[i].x), __fmul_rn(bv.y, sb[i].y)));
-            const float s0 = __fdiv_rn(gs.x, __fadd_rn(1.0f, expf(-gs.x)));
-            const float s1 = __fdiv_rn(gs.y, __fadd_rn(1.0f, expf(-gs.y)));
-            v0 = __fmul_rn(s0, us.x);
-            v1 = __fmul_rn(s1, us.y);
+            x[i] = lo2(pk(__fmul2_rn(lo2(word4(a, i)), sa[i])));
+            m[i] = lo2(pk(__fmul2_rn(lo2(word4(b, i)), sb[i])));
+            d[i] = __fadd2_rn(f2(1.f, 1.f), f2(expf(-x[i].x), expf(-x[i].y)));
+            xmax = max(xmax, max(__float_as_int(x[i].x), __float_as_int(x[i].y)));
         }
-        w[i] = pack_bf2(v0, v1);
+        dmax = max(dmax, max(__float_as_uint(d[i].x), __float_as_uint(d[i].y)));
+    }
+    // unsigned bits order d >= 1 and put NaN past every finite d; signed
+    // bits put +inf past every other x
+    const bool fast = dmax < kFastDLimit && (PRO == 0 || xmax < 0x7F800000);
+    uint32_t w[4];
+    if (fast) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 y = rcp_fast2(d[i]);
+            if constexpr (PRO == 0)
+                w[i] = pk(__fmul2_rn(m[i], y));
+            else
+                w[i] = pk(__fmul2_rn(div_fast2(x[i], d[i], y), m[i]));
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if constexpr (PRO == 0)
+                w[i] = pack_bf2(__fmul_rn(m[i].x, __frcp_rn(d[i].x)), __fmul_rn(m[i].y, __frcp_rn(d[i].y)));
+            else
+                w[i] = pack_bf2(__fmul_rn(__fdiv_rn(x[i].x, d[i].x), m[i].x),
+                                __fmul_rn(__fdiv_rn(x[i].y, d[i].y), m[i].y));
+        }
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Every fp32 bit pattern v as the gate argument z = v and as silu's x = v:
+// counts[0] / counts[1] = inputs where the fast reciprocal / quotient runs
+// and its bits differ from __frcp_rn / __fdiv_rn; counts[2] / counts[3] =
+// inputs where it runs.
+__global__ void __launch_bounds__(256) k_division_check(unsigned long long *counts)
+{
+    unsigned long long bad_r = 0, bad_q = 0, n_r = 0, n_q = 0;
+    const uint64_t step = uint64_t(gridDim.x) * blockDim.x;
+    for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < (uint64_t(1) << 32); i += 2 * step) {
+        // two inputs per iteration through the packed forms
+        const uint64_t j = i + step < (uint64_t(1) << 32) ? i + step : i;
+        const float2 v = f2(__uint_as_float(uint32_t(i)), __uint_as_float(uint32_t(j)));
+        const float2 d = __fadd2_rn(f2(1.f, 1.f), f2(expf(-v.x), expf(-v.y)));
+        const float2 y = rcp_fast2(d);
+        const float2 q = div_fast2(v, d, y);
+        const float dd[2] = {d.x, d.y}, yy[2] = {y.x, y.y}, qq[2] = {q.x, q.y}, vv[2] = {v.x, v.y};
+        const int nk = j == i ? 1 : 2;
+        for (int k = 0; k < nk; ++k) {
+            if (__float_as_uint(dd[k]) >= kFastDLimit)
+                continue;
+            ++n_r;
+            bad_r += __float_as_uint(yy[k]) != __float_as_uint(__frcp_rn(dd[k]));
+            if (__float_as_int(vv[k]) >= 0x7F800000)
+                continue;
+            ++n_q;
+            bad_q += __float_as_uint(qq[k]) != __float_as_uint(__fdiv_rn(vv[k], dd[k]));
+        }
+    }
+    atomicAdd(&counts[0], bad_r);
+    atomicAdd(&counts[1], bad_q);
+    atomicAdd(&counts[2], n_r);
+    atomicAdd(&counts[3], n_q);
 }
 
 template <int WP, int PRO, bool CACHED>
@@ -1529,6 +1626,16 @@ static int tile_groups_t(int slot_bytes)
     case 65536: return TileCfg<T, 65536>::kGroups;
     default: return 0;
     }
+}
+
+int launch_division_check(unsigned long long *counts, void *stream)
+{
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(counts, 0, 4 * sizeof(unsigned long long), st);
+    if (e != cudaSuccess)
+        return e;
+    k_division_check<<<148 * 8, 256, 0, st>>>(counts);
+    return cudaGetLastError();
 }
 
 int tile_groups(int tag, int slot_bytes)

@@ -93,7 +93,7 @@ _lib.ds_slerp_rows_backward_workspace.restype = ct.c_uint64
 for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
            "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
-           "ds_debug_wait_timeout_selftest"):
+           "ds_debug_wait_timeout_selftest", "ds_debug_division_check"):
     getattr(_lib, _f).restype = _st
 _lib.ds_status_string.argtypes = [ct.c_int]
 _lib.ds_status_string.restype = ct.c_char_p
@@ -109,12 +109,14 @@ _lib.ds_row_class.argtypes = [ct.c_int, ct.c_int64, ct.POINTER(ct.c_int), ct.POI
 _lib.ds_debug_force_path.argtypes = [ct.c_int]
 _lib.ds_debug_set_wait_limit_ns.argtypes = [ct.c_uint64]
 _lib.ds_debug_wait_timeout_selftest.argtypes = [ct.c_uint64, ct.c_void_p]
+_lib.ds_debug_division_check.argtypes = [ct.c_void_p, ct.c_void_p]
 
 #: every symbol include/ds.h declares
 EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
            "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_slerp_rows_backward_workspace", "ds_slerp_rows_backward_noalloc", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
-           "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest")
+           "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest",
+           "ds_debug_division_check")
 
 
 def lib() -> ct.CDLL:
@@ -405,6 +407,18 @@ def ds_debug_set_wait_limit_ns(limit_ns: int) -> None:
 
 def ds_debug_wait_timeout_selftest(limit_ns: int, stream=None) -> None:
     _check(_lib.ds_debug_wait_timeout_selftest(limit_ns, _stream_ptr(stream)), "ds_debug_wait_timeout_selftest")
+
+
+def ds_debug_division_check(stream=None) -> tuple[int, int, int, int]:
+    """(reciprocal mismatches, quotient mismatches, reciprocal inputs checked,
+    quotient inputs checked) of the Dory rows' fast division over every fp32
+    input; synchronises the stream."""
+    import torch
+
+    counts = torch.zeros(4, dtype=torch.int64, device="cuda")
+    _check(_lib.ds_debug_division_check(counts.data_ptr(), _stream_ptr(stream)), "ds_debug_division_check")
+    torch.cuda.synchronize()
+    return tuple(int(v) for v in counts.tolist())
 
 
 class force_path:

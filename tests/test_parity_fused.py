@@ -155,3 +155,34 @@ def test_in_place(swiglu):
         (ds.ds_swiglu_l2_rows if swiglu else ds.ds_gate_l2_rows)([seg], 1e-6)
         torch.cuda.synchronize()
         assert np.array_equal(gu.host_bits(y), ref)
+
+
+def test_fast_division_matches_ieee_on_every_fp32_input():
+    """Markstein's reciprocal and quotient, where the rows use them, give
+    the bits of IEEE division for every fp32 argument (2^32 of each)."""
+    bad_r, bad_q, n_r, n_q = ds.ds_debug_division_check()
+    assert bad_r == 0 and bad_q == 0, (bad_r, bad_q)
+    # the fast range covers every argument above -87.3 (about 3.2e9 patterns
+    # once the NaNs and those below are left out)
+    assert n_r > 3_000_000_000 and n_q > 3_000_000_000, (n_r, n_q)
+
+
+def test_negative_zero_and_tiny_gates():
+    """-0, subnormal and +-inf entries in the scaled gate take the
+    definition's value (silu(-0) = -0 and so on) with the rest of the unit."""
+    C = 64
+    g = np.zeros((4, C), np.uint16)
+    g[0, ::2] = 0x8000                      # -0
+    g[1, :] = 0x0001                        # smallest bf16 subnormal
+    g[1, 1::2] = 0x8003
+    g[2, :8] = 0x7F80                       # +inf: the unit takes IEEE division
+    g[2, 8:] = wl.to_bf16_bits(np.linspace(-3, 3, C - 8).astype(np.float32))
+    g[3, :] = wl.to_bf16_bits(np.linspace(-100, 100, C).astype(np.float32))
+    u = wl.to_bf16_bits(np.ones((4, C), np.float32))
+    one = np.ones(C, np.float32)
+    for swiglu in (False, True):
+        got = run(swiglu, u if not swiglu else g, g if not swiglu else u, one, one, 1e-6)
+        a, b = (u, g) if not swiglu else (g, u)
+        check(swiglu, a[[0, 1, 3]], b[[0, 1, 3]], one, one, got[[0, 1, 3]], 1e-6, what="special gates")
+        if swiglu:   # silu(-0) = -0/2 = -0, kept through the product and the scaling
+            assert np.all(got[0, ::2] == 0x8000) and np.all(got[0, 1::2] == 0)
