@@ -1115,47 +1115,56 @@ __device__ __forceinline__ float2 div_fast2(float2 x, float2 d, float2 y)
 
 constexpr uint32_t kFastDLimit = 0x7E800000u; // bits of 2^126
 
+// Words (pairs of columns) that share one range check: fewer keep fewer
+// values live across the check.
+constexpr int kFusedCheckWords = 4;
+
 template <int PRO>
 __device__ __forceinline__ uint4 fused_unit(uint4 a, uint4 b, const float2 (&sa)[4], const float2 (&sb)[4])
 {
-    float2 x[4], d[4], m[4]; // gate: m = a; swiglu: x = gs, m = us
-    uint32_t dmax = 0;
-    int xmax = int(0x80000000u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if constexpr (PRO == 0) {
-            const float2 z = __fmul2_rn(lo2(word4(b, i)), sa[i]);
-            d[i] = __fadd2_rn(f2(1.f, 1.f), f2(expf(-z.x), expf(-z.y)));
-            m[i] = lo2(word4(a, i));
-        } else {
-            x[i] = lo2(pk(__fmul2_rn(lo2(word4(a, i)), sa[i])));
-            m[i] = lo2(pk(__fmul2_rn(lo2(word4(b, i)), sb[i])));
-            d[i] = __fadd2_rn(f2(1.f, 1.f), f2(expf(-x[i].x), expf(-x[i].y)));
-            xmax = max(xmax, max(__float_as_int(x[i].x), __float_as_int(x[i].y)));
-        }
-        dmax = max(dmax, max(__float_as_uint(d[i].x), __float_as_uint(d[i].y)));
-    }
-    // unsigned bits order d >= 1 and put NaN past every finite d; signed
-    // bits put +inf past every other x
-    const bool fast = dmax < kFastDLimit && (PRO == 0 || xmax < 0x7F800000);
+    constexpr int H = kFusedCheckWords;
     uint32_t w[4];
-    if (fast) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 y = rcp_fast2(d[i]);
-            if constexpr (PRO == 0)
-                w[i] = pk(__fmul2_rn(m[i], y));
-            else
-                w[i] = pk(__fmul2_rn(div_fast2(x[i], d[i], y), m[i]));
+    for (int h = 0; h < 4; h += H) {
+        float2 x[H], d[H], m[H]; // gate: m = a; swiglu: x = gs, m = us
+        uint32_t dmax = 0;
+        int xmax = int(0x80000000u);
+#pragma unroll
+        for (int k = 0; k < H; ++k) {
+            const int i = h + k;
+            if constexpr (PRO == 0) {
+                const float2 z = __fmul2_rn(lo2(word4(b, i)), sa[i]);
+                d[k] = __fadd2_rn(f2(1.f, 1.f), f2(expf(-z.x), expf(-z.y)));
+                m[k] = lo2(word4(a, i));
+            } else {
+                x[k] = lo2(pk(__fmul2_rn(lo2(word4(a, i)), sa[i])));
+                m[k] = lo2(pk(__fmul2_rn(lo2(word4(b, i)), sb[i])));
+                d[k] = __fadd2_rn(f2(1.f, 1.f), f2(expf(-x[k].x), expf(-x[k].y)));
+                xmax = max(xmax, max(__float_as_int(x[k].x), __float_as_int(x[k].y)));
+            }
+            dmax = max(dmax, max(__float_as_uint(d[k].x), __float_as_uint(d[k].y)));
         }
-    } else {
+        // unsigned bits order d >= 1 and put NaN past every finite d; signed
+        // bits put +inf past every other x
+        const bool fast = dmax < kFastDLimit && (PRO == 0 || xmax < 0x7F800000);
+        if (fast) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if constexpr (PRO == 0)
-                w[i] = pack_bf2(__fmul_rn(m[i].x, __frcp_rn(d[i].x)), __fmul_rn(m[i].y, __frcp_rn(d[i].y)));
-            else
-                w[i] = pack_bf2(__fmul_rn(__fdiv_rn(x[i].x, d[i].x), m[i].x),
-                                __fmul_rn(__fdiv_rn(x[i].y, d[i].y), m[i].y));
+            for (int k = 0; k < H; ++k) {
+                const float2 y = rcp_fast2(d[k]);
+                if constexpr (PRO == 0)
+                    w[h + k] = pk(__fmul2_rn(m[k], y));
+                else
+                    w[h + k] = pk(__fmul2_rn(div_fast2(x[k], d[k], y), m[k]));
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < H; ++k) {
+                if constexpr (PRO == 0)
+                    w[h + k] = pack_bf2(__fmul_rn(m[k].x, __frcp_rn(d[k].x)), __fmul_rn(m[k].y, __frcp_rn(d[k].y)));
+                else
+                    w[h + k] = pack_bf2(__fmul_rn(__fdiv_rn(x[k].x, d[k].x), m[k].x),
+                                        __fmul_rn(__fdiv_rn(x[k].y, d[k].y), m[k].y));
+            }
         }
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
@@ -1207,7 +1216,7 @@ __device__ __forceinline__ void tile_fused_row(Team<WP> &tm, const ASegK &sg, in
     uint4 *x = reinterpret_cast<uint4 *>(s0);
     const uint4 *r = reinterpret_cast<const uint4 *>(s1);
     float2 acc = f2(0.f, 0.f);
-#pragma unroll 2
+#pragma unroll 1
     for (int u = t; u < nunits; u += G) {
         float2 va[4], vb[4];
         alpha8_signed<CACHED>(ca, half, sg.alpha, u, sg.cols, va);
