@@ -233,3 +233,47 @@ def integer_rows(seed: int, rows: int, cols: int, max_sumsq: int = (1 << 24) - 1
     lim = max(1, min(lim, 256))           # |v| <= 256 is exact in bf16
     a = rng.integers(-lim, lim + 1, size=(rows, cols)).astype(np.float32)
     return to_bf16_bits(a)
+
+
+@dataclass
+class QKRows:
+    """Dory's attention rows for tf_qk_rows_l2: q [R, hq*D], k and v [R, hk*D]
+    bf16 bits, positions [R] int32, inverse frequencies fp32 [D/2], q's scale
+    vector fp32 [hq*D]."""
+
+    q: np.ndarray
+    k: np.ndarray
+    v: np.ndarray
+    pos: np.ndarray
+    inv: np.ndarray
+    q_scale: np.ndarray
+    head_dim: int
+    hq: int
+    hk: int
+
+    @property
+    def rows(self) -> int:
+        return self.q.shape[0]
+
+
+def rope_inv(head_dim: int, theta: float = 10000.0) -> np.ndarray:
+    """1 / theta^(2i/D) in fp32 steps, the way the tern-tc listing forms its
+    RoPE cache (rope_cache): the exponent, the power and the reciprocal each
+    rounded to fp32."""
+    e = np.arange(0, head_dim, 2, dtype=np.float32) / np.float32(head_dim)
+    return (np.float32(1.0) / np.power(np.float32(theta), e, dtype=np.float32)).astype(np.float32)
+
+
+def qk_rows(seed: int = 0, rows: int = 2048, head_dim: int = 256, hq: int = 16, hk: int = 4,
+            theta: float = 10000.0, far_pos: int = 199_800) -> QKRows:
+    """q, k, v ~ N(0,1) bf16; the first two thirds of the rows at positions
+    0, 1, ... and the last third at far_pos, far_pos + 1, ...; q_scale ~
+    U(0.5, 2) fp32 (the pages form it on the host and give no values)."""
+    rng = _rng(seed)
+    q = normal_bf16(rng, (rows, hq * head_dim))
+    k = normal_bf16(rng, (rows, hk * head_dim))
+    v = normal_bf16(rng, (rows, hk * head_dim))
+    near = rows - rows // 3
+    pos = np.concatenate([np.arange(near), far_pos + np.arange(rows - near)]).astype(np.int32)
+    q_scale = rng.uniform(0.5, 2.0, hq * head_dim).astype(np.float32)
+    return QKRows(q, k, v, pos, rope_inv(head_dim, theta), q_scale, head_dim, hq, hk)

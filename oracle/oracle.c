@@ -1151,3 +1151,287 @@ int or_slerp_rows_interval(const uint16_t *res, const uint16_t *out,
     jb.out_h2 = hi;
     return run_rows(&jb, R, nthreads);
 }
+
+/* ------------------------------------------------------------------------ */
+/* [TF] tf_qk_rows_l2: rotate-half RoPE on a head's bf16 values (the halves
+ * x_i, x_{i+h} turned by the fp32 angle p inv_i, as the tern-tc listing's
+ * apply_rope computes in fp32 and casts back), the head's L2 norm with eps on
+ * the sum, and q's fp32 scale after the normalized head's rounding.         */
+
+/* The angle torch forms: fp32(p) * inv_i, one fp32 product.  A 24-bit by
+ * 24-bit product is exact in double; the cast rounds it to fp32. */
+static double rope_angle(int32_t p, float inv)
+{
+    return (double)(float)((double)(float)p * (double)inv);
+}
+
+static void rope_head(const double *x, int32_t D, int32_t p, const float *inv,
+                      unsigned flags, double *rot)
+{
+    const int32_t h = D / 2;
+    for (int32_t i = 0; i < h; ++i) {
+        double th = rope_angle(p, inv[i]);
+        double c = cos(th), s = sin(th);
+        double a = x[i] * c - x[i + h] * s;
+        double b = x[i] * s + x[i + h] * c;
+        rot[i] = (flags & OR_DROP_ROT) ? a : round_bf16(a);
+        rot[i + h] = (flags & OR_DROP_ROT) ? b : round_bf16(b);
+    }
+}
+
+/* One head: rot, then y = rot / n; q scales y (rounded unless dropped). */
+static void qk_head(const double *x, int32_t D, int32_t p, const float *inv,
+                    const float *scale, int is_q, double eps, unsigned flags,
+                    double *rot, uint16_t *out, double *out_exact)
+{
+    rope_head(x, D, p, inv, flags, rot);
+    double n = row_norm(sum_sq(rot, D), eps, flags);
+    for (int32_t j = 0; j < D; ++j) {
+        double y = rot[j] / n, v;
+        if (is_q) {
+            double yr = (flags & OR_DROP_QNORM) ? y : round_bf16(y);
+            v = scale ? yr * (double)scale[j] : yr;
+        } else {
+            v = y;
+        }
+        out[j] = or_bf16_rne(v);
+        if (out_exact)
+            out_exact[j] = v;
+    }
+}
+
+/* fp32's unit in the last place of v (subnormal spacing below 2^-126). */
+static double ulp32(double v)
+{
+    double a = fabs(v);
+    if (!(a >= 0x1p-126))
+        return 0x1p-149;
+    int e;
+    (void)frexp(a, &e); /* a in [2^(e-1), 2^e) */
+    return ldexp(1.0, e - 1 - 23);
+}
+
+static void qk_head_interval(const double *x, int32_t D, int32_t p,
+                             const float *inv, const float *scale, int is_q,
+                             double eps, double delta, unsigned flags,
+                             double *tmp, uint16_t *lo, uint16_t *hi)
+{
+    const int32_t h = D / 2;
+    double *sl = tmp, *sh = tmp + D, *yl = tmp + 2 * D, *yh = tmp + 3 * D;
+    const double w32 = delta > 0x1p-23 ? delta : 0x1p-23;
+    for (int32_t i = 0; i < h; ++i) {
+        double th = rope_angle(p, inv[i]);
+        double c = cos(th), s = sin(th);
+        /* cosf / sinf: 2 ulps of the result, never less than delta */
+        double ec = 2.0 * ulp32(c) + fabs(c) * delta, es = 2.0 * ulp32(s) + fabs(s) * delta;
+        double cl = c - ec, ch = c + ec, s_l = s - es, s_h = s + es;
+        double cm = dmax(fabs(cl), fabs(ch)), smx = dmax(fabs(s_l), fabs(s_h));
+        const double x1 = x[i], x2 = x[i + h];
+        double p0, p1, q0, q1, r0, r1, t0, t1;
+        mul_range(x1, x1, cl, ch, &p0, &p1);  /* x1 cos */
+        mul_range(x2, x2, s_l, s_h, &q0, &q1); /* x2 sin */
+        mul_range(x1, x1, s_l, s_h, &r0, &r1); /* x1 sin */
+        mul_range(x2, x2, cl, ch, &t0, &t1);  /* x2 cos */
+        /* two fp32 products and their sum: each rounding within w32 of
+         * the magnitudes it touches */
+        double wa = w32 * (fabs(x1) * cm + fabs(x2) * smx) * 2.0;
+        double wb = w32 * (fabs(x1) * smx + fabs(x2) * cm) * 2.0;
+        bf16_ends(p0 - q1 - wa, p1 - q0 + wa, flags & OR_DROP_ROT, &sl[i], &sh[i]);
+        bf16_ends(r0 + t0 - wb, r1 + t1 + wb, flags & OR_DROP_ROT, &sl[i + h], &sh[i + h]);
+    }
+    double Sl = 0.0, Sh = 0.0;
+    for (int32_t j = 0; j < D; ++j) {
+        double ql = sl[j] * sl[j], qh = sh[j] * sh[j];
+        Sl += (sl[j] > 0.0 || sh[j] < 0.0) ? dmin(ql, qh) : 0.0;
+        Sh += dmax(ql, qh);
+    }
+    double nl = row_norm(Sl * (1.0 - delta), eps, flags);
+    double nh = row_norm(Sh * (1.0 + delta), eps, flags);
+    for (int32_t j = 0; j < D; ++j) {
+        if (!(nl > 0.0) || !isfinite(nh)) {
+            yl[j] = -INFINITY;
+            yh[j] = INFINITY;
+        } else {
+            quotient_ends(sl[j], sh[j], nl, nh, delta, &yl[j], &yh[j]);
+        }
+        double vl = yl[j], vh = yh[j];
+        if (is_q) {
+            bf16_ends(vl, vh, flags & OR_DROP_QNORM, &vl, &vh);
+            if (scale) {
+                double a = vl * (double)scale[j], b = vh * (double)scale[j];
+                vl = dmin(a, b);
+                vh = dmax(a, b);
+                vl -= fabs(vl) * delta;
+                vh += fabs(vh) * delta;
+            }
+        }
+        lo[j] = or_bf16_rne(vl);
+        hi[j] = or_bf16_rne(vh);
+    }
+}
+
+typedef struct {
+    int iv;
+    int64_t r0, r1, ld_q, ld_k;
+    int32_t D, hq, hk;
+    const uint16_t *q, *k;
+    const int32_t *pos;
+    const float *inv, *scale;
+    double eps, delta;
+    unsigned flags;
+    uint16_t *qa, *qb, *ka, *kb; /* point: q_out, -, k_out, -; interval: lo, hi */
+    double *qe, *ke;
+    int status;
+} qk_job_t;
+
+static void *run_qk_job(void *arg)
+{
+    qk_job_t *jb = (qk_job_t *)arg;
+    const int32_t D = jb->D;
+    double *buf = (double *)malloc(sizeof(double) * (size_t)(5 * D));
+    if (!buf) {
+        jb->status = -1;
+        return NULL;
+    }
+    double *x = buf, *tmp = buf + D;
+    for (int64_t row = jb->r0; row < jb->r1; ++row) {
+        const int32_t p = jb->pos[row];
+        for (int part = 0; part < 2; ++part) {
+            const int is_q = part == 0;
+            const int32_t H = is_q ? jb->hq : jb->hk;
+            const uint16_t *src = is_q ? jb->q + row * jb->ld_q : jb->k + row * jb->ld_k;
+            const int64_t o = row * (int64_t)H * D;
+            for (int32_t hd = 0; hd < H; ++hd) {
+                for (int32_t j = 0; j < D; ++j)
+                    x[j] = or_bf16_value(src[(int64_t)hd * D + j]);
+                const float *sc = (is_q && jb->scale) ? jb->scale + (int64_t)hd * D : NULL;
+                const int64_t oo = o + (int64_t)hd * D;
+                if (jb->iv) {
+                    qk_head_interval(x, D, p, jb->inv, sc, is_q, jb->eps, jb->delta, jb->flags, tmp,
+                                     (is_q ? jb->qa : jb->ka) + oo, (is_q ? jb->qb : jb->kb) + oo);
+                } else {
+                    double *ex = is_q ? jb->qe : jb->ke;
+                    qk_head(x, D, p, jb->inv, sc, is_q, jb->eps, jb->flags, tmp,
+                            (is_q ? jb->qa : jb->ka) + oo, ex ? ex + oo : NULL);
+                }
+            }
+        }
+    }
+    free(buf);
+    jb->status = 0;
+    return NULL;
+}
+
+static int run_qk(const qk_job_t *proto, int64_t R, int nthreads)
+{
+    if (R <= 0)
+        return 0;
+    if (nthreads < 1)
+        nthreads = 1;
+    if ((int64_t)nthreads > R)
+        nthreads = (int)R;
+    qk_job_t *jobs = (qk_job_t *)calloc((size_t)nthreads, sizeof(qk_job_t));
+    pthread_t *tid = (pthread_t *)calloc((size_t)nthreads, sizeof(pthread_t));
+    int *started = (int *)calloc((size_t)nthreads, sizeof(int));
+    if (!jobs || !tid || !started) {
+        free(jobs);
+        free(tid);
+        free(started);
+        return -1;
+    }
+    for (int t = 0; t < nthreads; ++t) {
+        jobs[t] = *proto;
+        jobs[t].r0 = R * t / nthreads;
+        jobs[t].r1 = R * (t + 1) / nthreads;
+        jobs[t].status = -1;
+    }
+    for (int t = 1; t < nthreads; ++t)
+        started[t] = pthread_create(&tid[t], NULL, run_qk_job, &jobs[t]) == 0;
+    run_qk_job(&jobs[0]);
+    int rc = jobs[0].status;
+    for (int t = 1; t < nthreads; ++t) {
+        if (started[t])
+            pthread_join(tid[t], NULL);
+        else
+            run_qk_job(&jobs[t]);
+        if (jobs[t].status != 0)
+            rc = -1;
+    }
+    free(jobs);
+    free(tid);
+    free(started);
+    return rc;
+}
+
+static int qk_bad(int64_t R, int32_t D, int32_t hq, int32_t hk, int64_t ld_q,
+                  int64_t ld_k, const uint16_t *q, const uint16_t *k,
+                  const int32_t *pos, const float *inv, unsigned flags)
+{
+    const unsigned allowed = OR_DROP_ROT | OR_DROP_QNORM | OR_EPS_ZERO | OR_EPS_OUTSIDE;
+    if (R < 0 || D < 2 || D % 2 || hq < 0 || hk < 0 || (flags & ~allowed))
+        return 1;
+    if (ld_q < (int64_t)hq * D || ld_k < (int64_t)hk * D)
+        return 1;
+    return R > 0 && (!pos || !inv || (hq && !q) || (hk && !k));
+}
+
+int or_qk_rows_l2(const uint16_t *q, int64_t ld_q, const uint16_t *k,
+                  int64_t ld_k, int64_t R, int32_t D, int32_t hq, int32_t hk,
+                  const int32_t *pos, const float *inv, const float *q_scale,
+                  double eps, unsigned flags, uint16_t *q_out, uint16_t *k_out,
+                  double *q_exact, double *k_exact, int nthreads)
+{
+    if (qk_bad(R, D, hq, hk, ld_q, ld_k, q, k, pos, inv, flags) ||
+        (R > 0 && ((hq && !q_out) || (hk && !k_out))))
+        return -1;
+    qk_job_t jb = {0};
+    jb.ld_q = ld_q;
+    jb.ld_k = ld_k;
+    jb.D = D;
+    jb.hq = hq;
+    jb.hk = hk;
+    jb.q = q;
+    jb.k = k;
+    jb.pos = pos;
+    jb.inv = inv;
+    jb.scale = q_scale;
+    jb.eps = eps;
+    jb.flags = flags;
+    jb.qa = q_out;
+    jb.ka = k_out;
+    jb.qe = q_exact;
+    jb.ke = k_exact;
+    return run_qk(&jb, R, nthreads);
+}
+
+int or_qk_rows_l2_interval(const uint16_t *q, int64_t ld_q, const uint16_t *k,
+                           int64_t ld_k, int64_t R, int32_t D, int32_t hq,
+                           int32_t hk, const int32_t *pos, const float *inv,
+                           const float *q_scale, double eps, double delta,
+                           unsigned flags, uint16_t *q_lo, uint16_t *q_hi,
+                           uint16_t *k_lo, uint16_t *k_hi, int nthreads)
+{
+    if (qk_bad(R, D, hq, hk, ld_q, ld_k, q, k, pos, inv, flags) ||
+        (R > 0 && ((hq && (!q_lo || !q_hi)) || (hk && (!k_lo || !k_hi)))))
+        return -1;
+    qk_job_t jb = {0};
+    jb.iv = 1;
+    jb.ld_q = ld_q;
+    jb.ld_k = ld_k;
+    jb.D = D;
+    jb.hq = hq;
+    jb.hk = hk;
+    jb.q = q;
+    jb.k = k;
+    jb.pos = pos;
+    jb.inv = inv;
+    jb.scale = q_scale;
+    jb.eps = eps;
+    jb.delta = delta;
+    jb.flags = flags;
+    jb.qa = q_lo;
+    jb.qb = q_hi;
+    jb.ka = k_lo;
+    jb.kb = k_hi;
+    return run_qk(&jb, R, nthreads);
+}

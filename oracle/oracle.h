@@ -45,6 +45,8 @@ extern "C" {
 #define OR_DROP_SGATE     0x80u /* swiglu_l2: use g * sug unrounded (the scaled gate)       */
 #define OR_DROP_SUP       0x100u /* swiglu_l2: use u * suu unrounded (the scaled up)        */
 #define OR_DROP_PRODUCT   0x200u /* swiglu_l2: use silu(.) * (.) unrounded (the product)    */
+#define OR_DROP_ROT       0x400u /* qk_rows_l2: use the rotated head unrounded              */
+#define OR_DROP_QNORM     0x800u /* qk_rows_l2: use q's normalized head unrounded           */
 
 /* bf16 helpers.  or_bf16_rne rounds a double straight to bf16 bits. */
 uint16_t or_bf16_rne(double v);
@@ -194,6 +196,31 @@ int or_swiglu_l2_rows_interval(const uint16_t *g, const uint16_t *u,
                                int64_t C, int64_t ld, double eps, double delta,
                                unsigned flags, uint16_t *lo, uint16_t *hi,
                                int nthreads);
+
+/* [TF] tf_qk_rows_l2 (Dory's q and k rows, in dory.py's order): per row t and
+ * head, with D = head_dim, h = D/2 and the fp32 angle th_i = fp32(p_t * inv_i),
+ *   rot_i   = bf16(x_i cos th_i - x_{i+h} sin th_i)        (rotate-half RoPE,
+ *   rot_i+h = bf16(x_i sin th_i + x_{i+h} cos th_i)         the rotated head)
+ *   y = bf16(rot / sqrt(sum rot^2 + eps))                   (the normalized head)
+ *   q: out = bf16(y * q_scale_j) (q_scale fp32 [hq*D], or NULL: out = y);
+ *   k: out = y.
+ * q bf16 bits [R, ld_q] (hq heads), k [R, ld_k] (hk heads), pos [R], inv fp32
+ * [h].  Outputs dense: q_out [R, hq*D], k_out [R, hk*D]; the *_exact outputs
+ * (may be NULL) hold each output before its last rounding.  The interval form
+ * gives the bf16 ends reachable with cosf/sinf within 2 ulps of the fp32
+ * angle's cosine and sine, the rotation's fp32 products and sum, and each
+ * later fp32 step within relative `delta`. */
+int or_qk_rows_l2(const uint16_t *q, int64_t ld_q, const uint16_t *k,
+                  int64_t ld_k, int64_t R, int32_t D, int32_t hq, int32_t hk,
+                  const int32_t *pos, const float *inv, const float *q_scale,
+                  double eps, unsigned flags, uint16_t *q_out, uint16_t *k_out,
+                  double *q_exact, double *k_exact, int nthreads);
+int or_qk_rows_l2_interval(const uint16_t *q, int64_t ld_q, const uint16_t *k,
+                           int64_t ld_k, int64_t R, int32_t D, int32_t hq,
+                           int32_t hk, const int32_t *pos, const float *inv,
+                           const float *q_scale, double eps, double delta,
+                           unsigned flags, uint16_t *q_lo, uint16_t *q_hi,
+                           uint16_t *k_lo, uint16_t *k_hi, int nthreads);
 
 /* Backward of the activation rows over matrices (bf16 bits in, f64 out).
  * dalpha (may be NULL) = the rows' parts summed in row order. */

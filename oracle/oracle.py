@@ -22,6 +22,8 @@ OR_DROP_GATED = 0x40
 OR_DROP_SGATE = 0x80
 OR_DROP_SUP = 0x100
 OR_DROP_PRODUCT = 0x200
+OR_DROP_ROT = 0x400
+OR_DROP_QNORM = 0x800
 
 _lib = None
 
@@ -50,6 +52,10 @@ def lib() -> ct.CDLL:
         _lib.or_swiglu_l2_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
         _lib.or_gate_l2_rows_interval.argtypes = [vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
         _lib.or_swiglu_l2_rows_interval.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
+        _lib.or_qk_rows_l2.argtypes = [vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, vp, dbl, uns, vp, vp, vp, vp,
+                                       i32]
+        _lib.or_qk_rows_l2_interval.argtypes = [vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, vp, dbl, dbl, uns, vp,
+                                                vp, vp, vp, i32]
         _lib.or_slerp_rows_backward.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, vp, i32]
         _lib.or_l2_row.argtypes = [vp, vp, i64, dbl, uns, vp, vp, vp]
         _lib.or_l2_row.restype = None
@@ -65,7 +71,7 @@ def lib() -> ct.CDLL:
         _lib.or_l2_rows_interval.argtypes = [vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
         _lib.or_slerp_rows_interval.argtypes = [vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
         for f in ("or_wn_forward", "or_wn_backward", "or_row_renorm", "or_l2_rows", "or_slerp_rows",
-                  "or_l2_rows_interval", "or_slerp_rows_interval"):
+                  "or_l2_rows_interval", "or_slerp_rows_interval", "or_qk_rows_l2", "or_qk_rows_l2_interval"):
             getattr(_lib, f).restype = i32
     return _lib
 
@@ -230,6 +236,49 @@ def swiglu_l2_rows_interval(g, u, sug, suu, *, eps=1e-6, delta=1e-5, flags=0, nt
     _check(lib().or_swiglu_l2_rows_interval(_p(g), _p(u), _p(sug), _p(suu), R, C, C, eps, delta, flags, _p(lo),
                                             _p(hi), nthreads), "swiglu_l2_interval")
     return lo, hi
+
+
+def _qk_args(q, k, pos, inv, q_scale, head_dim):
+    q = np.ascontiguousarray(q, np.uint16)
+    k = np.ascontiguousarray(k, np.uint16)
+    if q.ndim != 2 or k.ndim != 2 or q.shape[0] != k.shape[0]:
+        raise ValueError("q and k must be [R, heads * head_dim] with the same R")
+    R = q.shape[0]
+    if q.shape[1] % head_dim or k.shape[1] % head_dim:
+        raise ValueError("widths must be whole heads")
+    pos = np.ascontiguousarray(pos, np.int32)
+    inv = np.ascontiguousarray(inv, np.float32)
+    if pos.shape != (R,) or inv.shape != (head_dim // 2,):
+        raise ValueError("pos [R], inv [head_dim / 2]")
+    if q_scale is not None:
+        q_scale = np.ascontiguousarray(q_scale, np.float32)
+        if q_scale.shape != (q.shape[1],):
+            raise ValueError("q_scale [hq * head_dim]")
+    return q, k, pos, inv, q_scale, R, q.shape[1] // head_dim, k.shape[1] // head_dim
+
+
+def qk_rows_l2(q, k, pos, inv, q_scale=None, *, head_dim, eps=1e-6, flags=0, nthreads=1, exact=False):
+    """(q_out, k_out) bf16 bits of Dory's q and k rows: rotate-half RoPE at the
+    fp32 angles fp32(pos * inv), per-head l2 with eps, q times q_scale
+    (fp32 [hq * head_dim] or None).  q [R, hq*D], k [R, hk*D] bf16 bits."""
+    q, k, pos, inv, sc, R, hq, hk = _qk_args(q, k, pos, inv, q_scale, head_dim)
+    qo = np.empty((R, hq * head_dim), np.uint16)
+    ko = np.empty((R, hk * head_dim), np.uint16)
+    qe = np.empty(qo.shape, np.float64) if exact else None
+    ke = np.empty(ko.shape, np.float64) if exact else None
+    _check(lib().or_qk_rows_l2(_p(q), q.shape[1], _p(k), k.shape[1], R, head_dim, hq, hk, _p(pos), _p(inv), _p(sc),
+                               eps, flags, _p(qo), _p(ko), _p(qe), _p(ke), nthreads), "qk_rows_l2")
+    return (qo, ko, qe, ke) if exact else (qo, ko)
+
+
+def qk_rows_l2_interval(q, k, pos, inv, q_scale=None, *, head_dim, eps=1e-6, delta=1e-5, flags=0, nthreads=1):
+    """(q_lo, q_hi, k_lo, k_hi): the bf16 ends each output can reach."""
+    q, k, pos, inv, sc, R, hq, hk = _qk_args(q, k, pos, inv, q_scale, head_dim)
+    out = [np.empty((R, h * head_dim), np.uint16) for h in (hq, hq, hk, hk)]
+    _check(lib().or_qk_rows_l2_interval(_p(q), q.shape[1], _p(k), k.shape[1], R, head_dim, hq, hk, _p(pos), _p(inv),
+                                        _p(sc), eps, delta, flags, *[_p(o) for o in out], nthreads),
+           "qk_rows_l2_interval")
+    return tuple(out)
 
 
 def l2_rows_backward(x, r, dy, *, eps=1e-6, flags=0, nthreads=1):
