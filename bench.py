@@ -28,7 +28,8 @@ CUDA-graph replay of the calls is timed as well).  wide = weights
 ds_renorm_momentum over the whole-model weights.  act_backward = the
 backward of the activation calls on [16384,4096] (upstream gradient bf16).
 dory = Dory's gated and SwiGLU l2 rows on [16384,4096] and [8192,7168]
-(scale vectors fp32 U(0.5, 2)).
+(scale vectors fp32 U(0.5, 2)) and its q/k rows on 16384 rows of 16 + 4 + 4
+heads of 256.
 
 Prints one JSON line (rank 0).  `value` is algorithmic bytes moved by all
 ranks per second (GB/s); per-kernel GB/s and rows/s, the roofline of the
@@ -59,6 +60,7 @@ if ROOT not in sys.path:
 METRIC = "achieved HBM GB/s (fraction of B200 peak) and rows/s per kernel, fwd+bwd"
 EPS = 1e-6
 ACT_ROWS, ACT_COLS = 16384, 4096
+QK_ROWS = 16384
 WORKLOAD = ("whole-model weights: 85 segments (12 layers x {q,k,v,o,gate,up,down} + tied embedding "
             "[32000,768]), 100,073,472 fp32 elements, fwd (bf16 W_eff) + bwd (bf16 GY) + renorm; "
             "activation rows [16384,4096] bf16: l2, l2 + residual, slerp")
@@ -74,7 +76,8 @@ WORKLOADS = {
     "act_backward": "activation backward on rows [16384,4096] bf16: l2 (dx fp32), l2 with residual, slerp "
                     "(dres, dout fp32 and dalpha [4096] through its workspace)",
     "dory": "Dory's fused activation rows: gated l2 rows (o, g bf16, sg fp32) and SwiGLU l2 rows (g, u bf16, "
-            "sug, suu fp32) on [16384,4096] and [8192,7168]",
+            "sug, suu fp32) on [16384,4096] and [8192,7168]; q/k rows (rotate-half RoPE, per-head l2, q scale; "
+            "16 q heads over 4 kv heads of 256, v copied to the cache) on 16384 rows, a third past position 199,800",
 }
 
 
@@ -96,6 +99,9 @@ def parse_args():
 def call_bytes(kind: str, segs=None, act=None) -> int:
     """Algorithmic bytes of one call: every input read once, every output
     written once (per-row gains and grad_g 4 B per row)."""
+    if kind == "qk":   # q read + written, k and v read + written to the cache, pos; inv and q_scale per call
+        wq, wk = act.hq * act.head_dim * 2, act.hk * act.head_dim * 2
+        return act.rows * (2 * wq + 4 * wk + 4) + act.head_dim // 2 * 4 + act.hq * act.head_dim * 4
     if act is not None:
         A = act.rows * act.cols
         return {"l2": A * (2 + 2), "l2res": A * (2 + 2 + 2), "slerp": A * (2 + 2 + 2) + act.cols * 4,
@@ -159,6 +165,8 @@ def plan(config: str, seed: int):
         for g in ag:
             sfx = "" if g == "x" else f"_{g}"
             calls += [(f"gate_l2_rows{sfx}", "gate", g), (f"swiglu_l2_rows{sfx}", "swiglu", g)]
+        ag["qk"] = wl.qk_rows(seed, rows=QK_ROWS)
+        calls.append(("qk_rows_l2", "qk", "qk"))
         return {}, ag, calls, 1
     if config == "optimizer":
         wg = {"model": wl.with_fp32_state(wl.whole_model(seed).weights, seed + 1)}
@@ -197,7 +205,8 @@ def measured_peaks() -> tuple[float, str]:
 
 def kernel_source_digest() -> str:
     h = hashlib.sha256()
-    for rel in ("l2_row_b200/csrc/ds_kernels.cu", "l2_row_b200/csrc/ds_tile.cu", "l2_row_b200/csrc/ds_api.cpp",
+    for rel in ("l2_row_b200/csrc/ds_kernels.cu", "l2_row_b200/csrc/ds_tile.cu", "l2_row_b200/csrc/ds_qk.cu",
+                "l2_row_b200/csrc/ds_api.cpp",
                 "l2_row_b200/csrc/ds_device.cuh", "l2_row_b200/csrc/ds_internal.h"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
@@ -338,6 +347,24 @@ class Step:
                 self.outputs.append(b0["w"])
         for name, a in self.ag.items():
             kinds = {k for _, k, g in self.plan if g == name}
+            if kinds == {"qk"}:
+                def i32(x):
+                    return torch.from_numpy(np.ascontiguousarray(x, np.int32)).to(dev)
+
+                copies = []
+                for c in range(self.copies):
+                    b = {"q": bf16(a.q), "k": bf16(a.k), "v": bf16(a.v), "pos": i32(a.pos), "inv": f32(a.inv),
+                         "q_scale": f32(a.q_scale)}
+                    b.update({"q_out": torch.empty_like(b["q"]), "k_cache": torch.empty_like(b["k"]),
+                              "v_cache": torch.empty_like(b["v"])})
+                    copies.append(b)
+                self.abuf[name] = copies
+                b0 = copies[0]
+                self.inputs += [(b0["q"], a.q.view(np.int16)), (b0["k"], a.k.view(np.int16)),
+                                (b0["v"], a.v.view(np.int16)), (b0["pos"], a.pos), (b0["inv"], a.inv),
+                                (b0["q_scale"], a.q_scale)]
+                self.outputs += [b0["q_out"], b0["k_cache"], b0["v_cache"]]
+                continue
             bwd = any(k.endswith("bwd") for k in kinds)
             dy_host = scales = None
             if kinds & {"gate", "swiglu"}:   # per-column scales U(0.5, 2), seeded after the rows
@@ -431,6 +458,13 @@ class Step:
                             t, 1, eps, da.data_ptr(), ws.data_ptr(), ws.numel(), s))
                     else:
                         fn = lambda s, t=tab: lib.ds_l2_rows_backward(t, 1, eps, s)
+                elif kind == "qk":
+                    b, a = self.abuf[g][c], self.ag[g]
+                    seg = ds.QKSeg(head_dim=a.head_dim, pos=b["pos"], inv_freq=b["inv"], q=b["q"], q_out=b["q_out"],
+                                   k=b["k"], k_cache=b["k_cache"], v=b["v"], v_cache=b["v_cache"],
+                                   q_scale=b["q_scale"])
+                    tab = (ds.ds_qkseg * 1)(seg.to_c())
+                    fn = lambda s, t=tab: lib.ds_qk_rows_l2(t, 1, eps, s)
                 elif kind in ("gate", "swiglu"):
                     b = self.abuf[g][c]
                     fseg = ds.FSeg(a=b["x"], b=b["r"], y=b["y"], sa=b["sa"], sb=b["sb"] if kind == "swiglu" else None)

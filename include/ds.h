@@ -2,7 +2,7 @@
  * ds.h -- C ABI of libds: per-row L2 normalisation of weight and activation
  * rows on NVIDIA B200 (sm_100a).
  *
- * Eleven operations, each over a table of segments (matrices), so that every
+ * Twelve operations, each over a table of segments (matrices), so that every
  * weight of a model is handled by one call:
  *
  *   ds_wn_forward   W_eff[r,:] = g_r * rho * w[r,:] / sqrt(sum_j w[r,j]^2 + eps)
@@ -40,6 +40,17 @@
  *                   the whole row; same PR (tf_gate_l2_rows, tf_swiglu_l2_rows),
  *                   sigmoid and silu in fp32 as 1/(1+expf(-x)) and
  *                   x/(1+expf(-x)) with IEEE division.
+ *   ds_qk_rows_l2   Dory's attention rows, in dory.py's order: rotate-half
+ *                   RoPE on each bf16 head of q and k at the fp32 angle
+ *                   th_i = fp32(pos) * inv_i,
+ *                     r_i   = bf16(x_i cos th_i - x_{i+D/2} sin th_i),
+ *                     r_i+D/2 = bf16(x_i sin th_i + x_{i+D/2} cos th_i),
+ *                   then y = bf16(r / sqrt(sum r^2 + eps)) per head; q out =
+ *                   bf16(y * q_scale) (q_scale fp32, (sqk f)^2 as torch forms
+ *                   it), k out = y into its cache row, v copied as is into its
+ *                   cache row; same PR (tf_qk_rows_l2).  cos and sin are
+ *                   CUDA's cosf / sinf of the fp32 angle, the products and sums
+ *                   fp32 as the tern-tc listing's apply_rope computes them.
  *   ds_l2_rows_backward, ds_slerp_rows_backward  the gradients of the two
  *                   activation calls (derived: the pages give the forward only),
  *                   straight through the bf16 rounding points, which keep the
@@ -70,7 +81,9 @@
  * default stream) and never synchronise, except ds_get_device_status.
  * Arguments are validated on the host before anything is launched; a failed
  * call launches nothing.  Kernels never trap: a bounded device-side wait that
- * runs out records DS_ERR_DEVICE_TIMEOUT, read by ds_get_device_status.
+ * runs out records DS_ERR_DEVICE_TIMEOUT, and ds_qk_rows_l2 records
+ * DS_ERR_INVALID_ARG for a cache slot out of range (device data the host does
+ * not read); ds_get_device_status returns and clears the first such record.
  */
 #ifndef DS_H
 #define DS_H
@@ -212,6 +225,50 @@ ds_status ds_gate_l2_rows(const ds_fseg *segs, int nseg, float eps,
                           ds_stream stream);
 ds_status ds_swiglu_l2_rows(const ds_fseg *segs, int nseg, float eps,
                             ds_stream stream);
+
+/* One set of attention rows for ds_qk_rows_l2 (bf16 unless noted; every
+ * matrix row-major, rows 16-byte aligned).
+ *   q        [rows, hq*head_dim], leading dimension ld_q (hq may be 0)
+ *   k        [rows, hk*head_dim], ld_kv (hk may be 0; hq + hk >= 1)
+ *   v        [rows, hk*head_dim], ld_kv, or NULL (nothing copied)
+ *   q_out    [rows, hq*head_dim], ld_q; may be exactly q
+ *   k_cache  [cache_rows, hk*head_dim], ld_cache: row slot[t] (or t when slot
+ *            is NULL) receives row t's normalized k heads; may be exactly k
+ *            when slot is NULL and ld_cache == ld_kv
+ *   v_cache  like k_cache for v (required iff v is set; may be exactly v on
+ *            the same terms)
+ *   pos      int32 [rows] device positions (any int32; the angle uses
+ *            fp32(pos))
+ *   slot     int32 [rows] device cache rows, or NULL.  Slots must be distinct;
+ *            a slot outside [0, cache_rows) skips that row's k and v stores
+ *            and records DS_ERR_INVALID_ARG for ds_get_device_status.
+ *   inv_freq fp32 [head_dim/2] device (1/theta^(2i/D) as the caller forms it)
+ *   q_scale  fp32 [hq*head_dim] device, 16-byte aligned, or NULL (scale 1)
+ * head_dim is 16, 32, 64, 128, 256 or 512.  Buffers written by the call must
+ * not overlap anything else it touches, except the exact aliases above. */
+typedef struct {
+    const void *q;
+    const void *k;
+    const void *v;
+    void *q_out;
+    void *k_cache;
+    void *v_cache;
+    const int32_t *pos;
+    const int32_t *slot;
+    const float *inv_freq;
+    const float *q_scale;
+    int64_t rows;       /* >= 0 */
+    int64_t cache_rows; /* rows of k_cache / v_cache (>= rows when slot is NULL) */
+    int64_t ld_q;
+    int64_t ld_kv;
+    int64_t ld_cache;
+    int32_t head_dim;
+    int32_t hq;
+    int32_t hk;
+} ds_qkseg;
+
+ds_status ds_qk_rows_l2(const ds_qkseg *segs, int nseg, float eps,
+                        ds_stream stream);
 
 /* Rows must have at most 64 KB of staged input (x, r and dy: 48 bytes per 8
  * columns; l2 rows without a residual 32): at most 10,920 columns for slerp

@@ -647,6 +647,151 @@ ds_status run_fused(bool swiglu, const ds_fseg *segs, int nseg, float eps, void 
     return launch_all<AParams, ASegK>(nseg, rows.data(), cls, eps, make, launch, stream);
 }
 
+// ------------------------------------------------------- Dory's q/k rows --
+
+bool qk_head_dim_ok(int32_t d)
+{
+    return d == 16 || d == 32 || d == 64 || d == 128 || d == 256 || d == 512;
+}
+
+ds_status run_qk(const ds_qkseg *segs, int nseg, float eps, void *stream)
+{
+    g_last_error.clear();
+    if (ds_status s = check_common(nseg, segs, eps, stream))
+        return s;
+    std::vector<Span> spans;
+    std::vector<int32_t> rb(static_cast<size_t>(nseg), 1);
+    for (int i = 0; i < nseg; ++i) {
+        const ds_qkseg &s = segs[i];
+        const int32_t D = s.head_dim;
+        if (s.rows < 0 || s.rows > (int64_t(1) << 40))
+            return fail(DS_ERR_INVALID_ARG, where("rows outside [0, 2^40]", i));
+        if (!qk_head_dim_ok(D))
+            return fail(DS_ERR_INVALID_ARG, where("head_dim must be 16, 32, 64, 128, 256 or 512", i));
+        if (s.hq < 0 || s.hk < 0 || s.hq + s.hk < 1 || s.hq > 4096 || s.hk > 4096)
+            return fail(DS_ERR_INVALID_ARG, where("hq, hk must be in [0, 4096] with hq + hk >= 1", i));
+        if (s.v && s.hk == 0)
+            return fail(DS_ERR_INVALID_ARG, where("v needs hk >= 1", i));
+        const int hw = 32 / (D / 16);
+        const int tpr = (s.hq + hw - 1) / hw + (s.hk + hw - 1) / hw * (s.v ? 2 : 1);
+        // rows per block iteration: as many as give each warp kQkTasks tasks
+        rb[i] = std::max(1, std::min(ds::kQkWarps * ds::kQkTasks / tpr, ds::kQkTable / (D / 2)));
+        if (s.rows == 0)
+            continue;
+        const int64_t wq = int64_t(s.hq) * D, wk = int64_t(s.hk) * D;
+        if (!s.pos)
+            return fail(DS_ERR_INVALID_ARG, where("pos is NULL", i));
+        if (!s.inv_freq)
+            return fail(DS_ERR_INVALID_ARG, where("inv_freq is NULL", i));
+        if (!aligned(s.pos, 4) || !aligned(s.inv_freq, 4) || (s.slot && !aligned(s.slot, 4)))
+            return fail(DS_ERR_ALIGNMENT, where("pos, slot and inv_freq must be 4-byte aligned", i));
+        spans.push_back(span_of(s.pos, 1, s.rows, s.rows, 4, i, 0, -1));
+        spans.push_back(span_of(s.inv_freq, 1, D / 2, D / 2, 4, i, 0, -1));
+        if (s.slot)
+            spans.push_back(span_of(s.slot, 1, s.rows, s.rows, 4, i, 0, -1));
+        if (s.hq > 0) {
+            if (s.ld_q < wq || s.ld_q > (int64_t(1) << 40))
+                return fail(DS_ERR_INVALID_ARG, where("ld_q below hq * head_dim (or too large)", i));
+            if (ds_status st = check_matrix(s.q, s.rows, s.ld_q, 2, "q", i))
+                return st;
+            if (ds_status st = check_matrix(s.q_out, s.rows, s.ld_q, 2, "q_out", i))
+                return st;
+            if (s.q_scale) {
+                if (!aligned(s.q_scale, 16))
+                    return fail(DS_ERR_ALIGNMENT, where("q_scale is not 16-byte aligned", i));
+                spans.push_back(span_of(s.q_scale, 1, wq, wq, 4, i, 0, -1));
+            }
+            spans.push_back(span_of(s.q, s.rows, wq, s.ld_q, 2, i, 0, 3 * i));
+            spans.push_back(span_of(s.q_out, s.rows, wq, s.ld_q, 2, i, 1, 3 * i));
+        }
+        if (s.hk > 0) {
+            if (s.ld_kv < wk || s.ld_kv > (int64_t(1) << 40) || s.ld_cache < wk || s.ld_cache > (int64_t(1) << 40))
+                return fail(DS_ERR_INVALID_ARG, where("ld_kv or ld_cache below hk * head_dim (or too large)", i));
+            if (s.cache_rows < 1 || s.cache_rows > (int64_t(1) << 40) || (!s.slot && s.cache_rows < s.rows))
+                return fail(DS_ERR_INVALID_ARG, where("cache_rows below rows (no slot) or outside [1, 2^40]", i));
+            if (ds_status st = check_matrix(s.k, s.rows, s.ld_kv, 2, "k", i))
+                return st;
+            if (ds_status st = check_matrix(s.k_cache, s.cache_rows, s.ld_cache, 2, "k_cache", i))
+                return st;
+            // in place only row for row (no slots) over the same matrix
+            const int key_k = s.slot ? -1 : 3 * i + 1, key_v = s.slot ? -1 : 3 * i + 2;
+            spans.push_back(span_of(s.k, s.rows, wk, s.ld_kv, 2, i, 0, key_k));
+            spans.push_back(span_of(s.k_cache, s.cache_rows, wk, s.ld_cache, 2, i, 1, key_k));
+            if (s.v) {
+                if (ds_status st = check_matrix(s.v, s.rows, s.ld_kv, 2, "v", i))
+                    return st;
+                if (ds_status st = check_matrix(s.v_cache, s.cache_rows, s.ld_cache, 2, "v_cache", i))
+                    return st;
+                spans.push_back(span_of(s.v, s.rows, wk, s.ld_kv, 2, i, 0, key_v));
+                spans.push_back(span_of(s.v_cache, s.cache_rows, wk, s.ld_cache, 2, i, 1, key_v));
+            }
+        }
+    }
+    if (ds_status st = check_overlaps(spans))
+        return st;
+
+    static thread_local ds::QKParams params; // ~20 KB: kept off the stack
+    // one launch per head size present
+    for (int pass = 0; pass < 6; ++pass) {
+        const int32_t head_dim = 16 << pass;
+        int n = 0;
+        int64_t units = 0;
+        auto flush = [&]() -> ds_status {
+            if (n == 0)
+                return DS_OK;
+            params.nseg = n;
+            params.unit_start[n] = units;
+            params.eps = eps;
+            const int grid = static_cast<int>(std::min<int64_t>(int64_t(sm_count()) * 3, units));
+            const int e = ds::launch_qk(params, grid, stream);
+            if (e != 0) {
+                char buf[160];
+                std::snprintf(buf, sizeof(buf), "kernel launch failed (cudaError %d)", e);
+                return fail(DS_ERR_CUDA, buf);
+            }
+            g_launches.fetch_add(1, std::memory_order_relaxed);
+            n = 0;
+            units = 0;
+            return DS_OK;
+        };
+        for (int i = 0; i < nseg; ++i) {
+            const ds_qkseg &s = segs[i];
+            if (s.rows == 0 || s.head_dim != head_dim)
+                continue;
+            if (n == ds::kSegPerLaunch)
+                if (ds_status st = flush())
+                    return st;
+            ds::QKSegK &k = params.seg[n];
+            k = ds::QKSegK{};
+            k.q = static_cast<const uint16_t *>(s.q);
+            k.k = static_cast<const uint16_t *>(s.k);
+            k.v = static_cast<const uint16_t *>(s.v);
+            k.q_out = static_cast<uint16_t *>(s.q_out);
+            k.k_cache = static_cast<uint16_t *>(s.k_cache);
+            k.v_cache = s.v ? static_cast<uint16_t *>(s.v_cache) : nullptr;
+            k.pos = s.pos;
+            k.slot = s.slot;
+            k.inv = s.inv_freq;
+            k.q_scale = s.hq > 0 ? s.q_scale : nullptr;
+            k.rows = s.rows;
+            k.cache_rows = s.cache_rows;
+            k.ld_q = s.ld_q;
+            k.ld_kv = s.ld_kv;
+            k.ld_cache = s.ld_cache;
+            k.D = s.head_dim;
+            k.hq = s.hq;
+            k.hk = s.hk;
+            k.rb = rb[i];
+            params.unit_start[n] = units;
+            units += (s.rows + rb[i] - 1) / rb[i];
+            ++n;
+        }
+        if (ds_status st = flush())
+            return st;
+    }
+    return DS_OK;
+}
+
 AGSegK agseg_rows(const ds_agseg &s, int64_t r0, int64_t nr)
 {
     AGSegK k{};
@@ -828,6 +973,11 @@ ds_status ds_swiglu_l2_rows(const ds_fseg *segs, int nseg, float eps, ds_stream 
     return run_fused(true, segs, nseg, eps, stream);
 }
 
+ds_status ds_qk_rows_l2(const ds_qkseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_qk(segs, nseg, eps, stream);
+}
+
 ds_status ds_l2_rows_backward(const ds_agseg *segs, int nseg, float eps, ds_stream stream)
 {
     return run_act_bwd(false, segs, nseg, eps, nullptr, nullptr, 0, stream);
@@ -897,7 +1047,10 @@ ds_status ds_get_device_status(ds_stream stream)
         return DS_OK;
     char buf[96];
     std::snprintf(buf, sizeof(buf), "device error %u at site %u", code, site);
-    return fail(code == DS_ERR_DEVICE_TIMEOUT ? DS_ERR_DEVICE_TIMEOUT : DS_ERR_CUDA, buf);
+    // codes the kernels record: a wait that ran out, an argument only the
+    // device could check (a cache slot out of range)
+    const bool known = code == DS_ERR_DEVICE_TIMEOUT || code == DS_ERR_INVALID_ARG;
+    return fail(known ? static_cast<ds_status>(code) : DS_ERR_CUDA, buf);
 }
 
 uint64_t ds_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

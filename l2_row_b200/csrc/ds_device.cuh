@@ -12,6 +12,10 @@
 
 namespace ds {
 
+// The device error word.  Without relocatable device code every .cu file
+// that includes this header is a module of its own with its own copy, so
+// each module exports a reader (module_read_and_clear_error) and the host
+// reads them all.
 __device__ uint32_t g_device_error[4]; // [0] status code, [1] site, [2] block
 
 __device__ __forceinline__ void raise_device_error(uint32_t code, uint32_t site)
@@ -20,6 +24,22 @@ __device__ __forceinline__ void raise_device_error(uint32_t code, uint32_t site)
         g_device_error[1] = site;
         g_device_error[2] = blockIdx.x;
     }
+}
+
+// This module's word, read and cleared (the caller has synchronised).
+static inline int module_read_and_clear_error(uint32_t *code, uint32_t *site)
+{
+    uint32_t h[4] = {0, 0, 0, 0};
+    cudaError_t e = cudaMemcpyFromSymbol(h, g_device_error, sizeof(h));
+    if (e != cudaSuccess)
+        return e;
+    const uint32_t zero[4] = {0, 0, 0, 0};
+    e = cudaMemcpyToSymbol(g_device_error, zero, sizeof(zero));
+    if (e != cudaSuccess)
+        return e;
+    *code = h[0];
+    *site = h[1];
+    return cudaSuccess;
 }
 
 // ---------------------------------------------------------------- memory --

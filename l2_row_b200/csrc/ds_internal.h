@@ -138,12 +138,34 @@ using WParams = LaunchParams<WSegK>;
 using AParams = LaunchParams<ASegK>;
 using GParams = LaunchParams<AGSegK>;
 
+// Dory's q and k rows (ds_qk.cu): one segment after host validation.
+constexpr int kQkThreads = 256;
+constexpr int kQkWarps = kQkThreads / 32;
+constexpr int kQkTasks = 3;     // warp tasks held in registers at once
+constexpr int kQkTable = 1024;  // cos (and sin) entries per block iteration: rb * head_dim / 2
+struct QKSegK {
+    const uint16_t *q, *k, *v;
+    uint16_t *q_out, *k_cache, *v_cache;
+    const int32_t *pos, *slot;
+    const float *inv, *q_scale;
+    int64_t rows, cache_rows;
+    int64_t ld_q, ld_kv, ld_cache;
+    int32_t D, hq, hk, rb; // rb: rows per block iteration
+};
+struct QKParams {
+    QKSegK seg[kSegPerLaunch];
+    int64_t unit_start[kSegPerLaunch + 1]; // prefix sums of block iterations
+    int32_t nseg;
+    float eps;
+};
+
 // Error word written by kernels (see ds_get_device_status).
 enum DeviceErrorSite : uint32_t {
     kSiteStreamWait = 1,
     kSiteStreamDrain = 2,
     kSiteSelftest = 3,
     kSiteTileWait = 4,
+    kSiteQkSlot = 5,
 };
 
 // Launchers of the cluster paths (ds_kernels.cu).  `units` = rows
@@ -175,6 +197,13 @@ int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64
                          float *dalpha, void *stream);
 // Exhaustive check of the Dory rows' fast reciprocal and quotient (ds_tile.cu).
 int launch_division_check(unsigned long long *counts, void *stream);
+// Every .cu file is its own device module with its own error word: the
+// reader syncs the stream, then reads and clears each module's word.
 int read_and_clear_device_error(uint32_t *code, uint32_t *site, void *stream);
+int tile_read_and_clear_error(uint32_t *code, uint32_t *site);
+int qk_read_and_clear_error(uint32_t *code, uint32_t *site);
+// Dory's q and k rows (ds_qk.cu): `grid` blocks of kQkThreads; every
+// segment of `p` has the same head size.
+int launch_qk(const QKParams &p, int grid, void *stream);
 
 } // namespace ds

@@ -1101,16 +1101,21 @@ int read_and_clear_device_error(uint32_t *code, uint32_t *site, void *stream)
     cudaError_t e = cudaStreamSynchronize(s);
     if (e != cudaSuccess)
         return e;
-    uint32_t h[4] = {0, 0, 0, 0};
-    e = cudaMemcpyFromSymbol(h, g_device_error, sizeof(h));
-    if (e != cudaSuccess)
-        return e;
-    const uint32_t zero[4] = {0, 0, 0, 0};
-    e = cudaMemcpyToSymbol(g_device_error, zero, sizeof(zero));
-    if (e != cudaSuccess)
-        return e;
-    *code = h[0];
-    *site = h[1];
+    *code = 0;
+    *site = 0;
+    // every module's word is cleared; the first error found is reported
+    int (*const readers[3])(uint32_t *, uint32_t *) = {module_read_and_clear_error, tile_read_and_clear_error,
+                                                       qk_read_and_clear_error};
+    for (auto rd : readers) {
+        uint32_t c = 0, st = 0;
+        const int r = rd(&c, &st);
+        if (r != cudaSuccess)
+            return r;
+        if (c != 0 && *code == 0) {
+            *code = c;
+            *site = st;
+        }
+    }
     return cudaSuccess;
 }
 

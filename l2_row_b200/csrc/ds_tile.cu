@@ -1637,6 +1637,8 @@ static int tile_groups_t(int slot_bytes)
     }
 }
 
+int tile_read_and_clear_error(uint32_t *code, uint32_t *site) { return module_read_and_clear_error(code, site); }
+
 int launch_division_check(unsigned long long *counts, void *stream)
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -72,6 +72,14 @@ class ds_agseg(ct.Structure):
                 ("ld", ct.c_int64), ("ld_d", ct.c_int64)]
 
 
+class ds_qkseg(ct.Structure):
+    _fields_ = [("q", ct.c_void_p), ("k", ct.c_void_p), ("v", ct.c_void_p), ("q_out", ct.c_void_p),
+                ("k_cache", ct.c_void_p), ("v_cache", ct.c_void_p), ("pos", ct.c_void_p), ("slot", ct.c_void_p),
+                ("inv_freq", ct.c_void_p), ("q_scale", ct.c_void_p), ("rows", ct.c_int64),
+                ("cache_rows", ct.c_int64), ("ld_q", ct.c_int64), ("ld_kv", ct.c_int64), ("ld_cache", ct.c_int64),
+                ("head_dim", ct.c_int32), ("hq", ct.c_int32), ("hk", ct.c_int32)]
+
+
 _st = ct.c_int
 _lib.ds_wn_forward.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_wn_backward.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_int, ct.c_float, ct.c_void_p]
@@ -83,6 +91,7 @@ _lib.ds_slerp_rows.argtypes = [ct.POINTER(ds_aseg), ct.c_int, ct.c_float, ct.c_v
 _lib.ds_l2_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_gate_l2_rows.argtypes = [ct.POINTER(ds_fseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_swiglu_l2_rows.argtypes = [ct.POINTER(ds_fseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_qk_rows_l2.argtypes = [ct.POINTER(ds_qkseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_slerp_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p, ct.c_void_p,
                                         ct.c_uint64, ct.c_void_p]
 _lib.ds_slerp_rows_backward_noalloc.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p,
@@ -92,7 +101,7 @@ _lib.ds_slerp_rows_backward_workspace.argtypes = [ct.c_int64]
 _lib.ds_slerp_rows_backward_workspace.restype = ct.c_uint64
 for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
-           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
+           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_qk_rows_l2", "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
            "ds_debug_wait_timeout_selftest", "ds_debug_division_check"):
     getattr(_lib, _f).restype = _st
 _lib.ds_status_string.argtypes = [ct.c_int]
@@ -114,7 +123,7 @@ _lib.ds_debug_division_check.argtypes = [ct.c_void_p, ct.c_void_p]
 #: every symbol include/ds.h declares
 EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
-           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_slerp_rows_backward_workspace", "ds_slerp_rows_backward_noalloc", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
+           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_qk_rows_l2", "ds_slerp_rows_backward_workspace", "ds_slerp_rows_backward_noalloc", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
            "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest",
            "ds_debug_division_check")
 
@@ -255,6 +264,58 @@ class FSeg:
 
 
 @dataclass
+class QKSeg:
+    """Dory's attention rows for ds_qk_rows_l2.  q [R, hq*D], k and v
+    [R, hk*D] bf16; q_out [R, hq*D]; k_cache, v_cache [cache_rows, hk*D]
+    (row slot[t], or t without slot, receives row t); pos, slot int32 [R];
+    inv_freq fp32 [D/2]; q_scale fp32 [hq*D] or None.  Any of q/q_out or
+    k/k_cache (v/v_cache) may be None when hq (hk) is 0."""
+
+    head_dim: int
+    pos: Any
+    inv_freq: Any
+    q: Any = None
+    q_out: Any = None
+    k: Any = None
+    k_cache: Any = None
+    v: Any = None
+    v_cache: Any = None
+    slot: Any = None
+    q_scale: Any = None
+
+    def to_c(self) -> ds_qkseg:
+        D = int(self.head_dim)
+        R = int(self.pos.shape[0])
+        if self.q is not None:
+            if self.q.shape[1] % D:
+                raise ValueError("q: width is not a whole number of heads")
+            hq = int(self.q.shape[1]) // D
+        else:
+            hq = 0
+        if self.k is not None:
+            if self.k.shape[1] % D:
+                raise ValueError("k: width is not a whole number of heads")
+            hk = int(self.k.shape[1]) // D
+        else:
+            hk = 0
+        q, ld_q = _mat(self.q, "q", R, hq * D)
+        qo, ld_qo = _mat(self.q_out, "q_out", R, hq * D)
+        k, ld_kv = _mat(self.k, "k", R, hk * D)
+        v, ld_v = _mat(self.v, "v", R, hk * D)
+        C = 0 if self.k_cache is None else int(self.k_cache.shape[0])
+        kc, ld_c = _mat(self.k_cache, "k_cache", C, hk * D)
+        vc, ld_vc = _mat(self.v_cache, "v_cache", C, hk * D)
+        if hq and ld_qo != ld_q:
+            raise ValueError("q and q_out must share a leading dimension")
+        if self.v is not None and ld_v != ld_kv:
+            raise ValueError("k and v must share a leading dimension")
+        if self.v_cache is not None and ld_vc != ld_c:
+            raise ValueError("k_cache and v_cache must share a leading dimension")
+        return ds_qkseg(q, k, v, qo, kc, vc, _vec(self.pos), _vec(self.slot), _vec(self.inv_freq),
+                        _vec(self.q_scale), R, C, ld_q, ld_kv, ld_c, D, hq, hk)
+
+
+@dataclass
 class AGSeg:
     """One activation matrix for the backward calls: x (slerp: res), r (l2:
     residual or None; slerp: out), dy the upstream gradient (bf16 [R, C],
@@ -331,6 +392,11 @@ def ds_gate_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
 def ds_swiglu_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
     arr, n = _table(segs, ds_fseg)
     _check(_lib.ds_swiglu_l2_rows(arr, n, eps, _stream_ptr(stream)), "ds_swiglu_l2_rows")
+
+
+def ds_qk_rows_l2(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_qkseg)
+    _check(_lib.ds_qk_rows_l2(arr, n, eps, _stream_ptr(stream)), "ds_qk_rows_l2")
 
 
 def ds_l2_rows_backward(segs: Sequence, eps: float = 1e-6, stream=None) -> None:

@@ -387,3 +387,52 @@ def test_fused_validation(fn):
         assert call_f(fn, [fseg(sb=0)]) == E.DS_ERR_INVALID_ARG
     assert call_f(fn, [fseg(rows=0, a=0, b=0, y=0)]) == E.DS_OK
     assert ds.ds_launch_count() == before
+
+
+# ------------------------------------------------------- Dory's q/k rows --
+
+def qkseg(**kw):
+    d = dict(q=BASE, k=BASE + (1 << 30), v=BASE + (2 << 30), q_out=BASE + (3 << 30), k_cache=BASE + (4 << 30),
+             v_cache=BASE + (5 << 30), pos=BASE + (6 << 30), slot=None, inv_freq=BASE + (6 << 30) + 4096,
+             q_scale=BASE + (6 << 30) + 8192, rows=4, cache_rows=4, ld_q=4 * 64, ld_kv=2 * 64, ld_cache=2 * 64,
+             head_dim=64, hq=4, hk=2)
+    d.update(kw)
+    return ds.ds_qkseg(**d)
+
+
+def call_qk(segs, eps=1e-6):
+    arr = (ds.ds_qkseg * max(1, len(segs)))(*segs)
+    return ds.lib().ds_qk_rows_l2(arr, len(segs), ct.c_float(eps), None)
+
+
+def test_qk_validation():
+    E = ds
+    before = ds.ds_launch_count()
+    assert call_qk([qkseg(head_dim=48, ld_q=4 * 48, ld_kv=96, ld_cache=96)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(head_dim=1024, ld_q=4096, ld_kv=2048, ld_cache=2048)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(hq=0, hk=0)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(hk=0, v=BASE + (2 << 30))]) == E.DS_ERR_INVALID_ARG   # v without k heads
+    assert call_qk([qkseg(rows=-1)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(pos=None)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(inv_freq=None)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(q=None)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(k_cache=None)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(v_cache=None)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(ld_q=4 * 64 - 8)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(ld_cache=64)]) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(cache_rows=3)]) == E.DS_ERR_INVALID_ARG                # rows above cache rows, no slot
+    assert call_qk([qkseg(q=BASE + 2)]) == E.DS_ERR_ALIGNMENT
+    assert call_qk([qkseg(q_scale=BASE + (6 << 30) + 8192 + 4)]) == E.DS_ERR_ALIGNMENT
+    assert call_qk([qkseg(pos=BASE + (6 << 30) + 2)]) == E.DS_ERR_ALIGNMENT
+    assert call_qk([qkseg(q_out=BASE + 16)]) == E.DS_ERR_OVERLAP                 # partial overlap with q
+    assert call_qk([qkseg(k_cache=BASE + (1 << 30), slot=BASE + (7 << 30))]) == E.DS_ERR_OVERLAP  # k in place with slots
+    assert call_qk([qkseg(v_cache=BASE + (4 << 30))]) == E.DS_ERR_OVERLAP        # the two caches
+    assert call_qk([qkseg()], eps=float("nan")) == E.DS_ERR_INVALID_ARG
+    assert call_qk([qkseg(rows=0, q=None, k=None, pos=None)]) == E.DS_OK
+    assert ds.ds_launch_count() == before
+
+
+def test_qk_shifted_cache_alias_refused():
+    """k_cache may be exactly k (row for row); a cache that starts one row
+    into k overlaps it and is refused before anything runs."""
+    assert call_qk([qkseg(k_cache=BASE + (1 << 30) + 128)]) == ds.DS_ERR_OVERLAP
