@@ -1435,3 +1435,50 @@ int or_qk_rows_l2_interval(const uint16_t *q, int64_t ld_q, const uint16_t *k,
     jb.kb = k_hi;
     return run_qk(&jb, R, nthreads);
 }
+
+/* ------------------------------------------------------------------------ */
+/* [DS] "Monitor" and `init` "preserve": the row length sqrt(sum w^2 + eps),
+ * divided by `div` (1, or rho for the gain that keeps W_eff = w).           */
+
+int or_row_norms(const float *w, int64_t R, int64_t C, int64_t ld, double eps,
+                 double div, double *out, int nthreads)
+{
+    (void)nthreads; /* one pass of R sums: no threads needed */
+    if (bad_shape(R, C, ld) || (R > 0 && (!w || !out)) || !(div > 0.0))
+        return -1;
+    for (int64_t r = 0; r < R; ++r) {
+        const float *wr = w + r * ld;
+        double S = 0.0;
+        for (int64_t j = 0; j < C; ++j)
+            S += (double)wr[j] * (double)wr[j];
+        out[r] = sqrt(S + eps) / div;
+    }
+    return 0;
+}
+
+/* [DS] `gain` "scalar": the channel backward with every g_r = g, and the
+ * per-row gain gradients summed in row order. */
+int or_wn_backward_scalar_gain(const float *w, int64_t R, int64_t C,
+                               int64_t ld, const void *gy, int gy_is_bf16,
+                               int64_t ld_gy, float g, double rho, double eps,
+                               unsigned flags, double *grad_w, double *gg_rows,
+                               double *gg_sum, int nthreads)
+{
+    if (bad_shape(R, C, ld) || !gg_sum || (R > 0 && !gg_rows))
+        return -1;
+    float *gv = (float *)calloc((size_t)(R > 0 ? R : 1), sizeof(float));
+    if (!gv)
+        return -1;
+    for (int64_t r = 0; r < R; ++r)
+        gv[r] = g;
+    int rc = or_wn_backward(w, R, C, ld, gy, gy_is_bf16, ld_gy, gv, rho, eps,
+                            flags, grad_w, gg_rows, nthreads);
+    free(gv);
+    if (rc != 0)
+        return rc;
+    double acc = 0.0;
+    for (int64_t r = 0; r < R; ++r)
+        acc += gg_rows[r];
+    *gg_sum = acc;
+    return 0;
+}

@@ -197,6 +197,24 @@ int or_swiglu_l2_rows_interval(const uint16_t *g, const uint16_t *u,
                                unsigned flags, uint16_t *lo, uint16_t *hi,
                                int nthreads);
 
+/* [DS] "Monitor" (each layer's raw row lengths) and options table, `init`
+ * "preserve" (gain = row length, same output): len[r] = sqrt(sum_j w^2 + eps)
+ * / div for fp32 rows w [R, ld]; div = 1 for the lengths, div = rho for the
+ * preserving gain (W_eff = g rho w / len = w).  f64 out [R]. */
+int or_row_norms(const float *w, int64_t R, int64_t C, int64_t ld, double eps,
+                 double div, double *out, int nthreads);
+
+/* [DS] options table, `gain` "scalar" (one gain for the layer): W_eff =
+ * g rho w_r / n_r for every row, so dL/dg = sum_r rho (w_r . GY_r) / n_r, the
+ * per-row grad_g of the channel form summed over the rows in row order.
+ * gg_rows [R] (those parts) and *gg_sum.  grad_w as or_wn_backward with
+ * every g_r = g. */
+int or_wn_backward_scalar_gain(const float *w, int64_t R, int64_t C,
+                               int64_t ld, const void *gy, int gy_is_bf16,
+                               int64_t ld_gy, float g, double rho, double eps,
+                               unsigned flags, double *grad_w, double *gg_rows,
+                               double *gg_sum, int nthreads);
+
 /* [TF] tf_qk_rows_l2 (Dory's q and k rows, in dory.py's order): per row t and
  * head, with D = head_dim, h = D/2 and the fp32 angle th_i = fp32(p_t * inv_i),
  *   rot_i   = bf16(x_i cos th_i - x_{i+h} sin th_i)        (rotate-half RoPE,

@@ -52,6 +52,9 @@ def lib() -> ct.CDLL:
         _lib.or_swiglu_l2_rows.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, uns, vp, vp, i32]
         _lib.or_gate_l2_rows_interval.argtypes = [vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
         _lib.or_swiglu_l2_rows_interval.argtypes = [vp, vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
+        _lib.or_row_norms.argtypes = [vp, i64, i64, i64, dbl, dbl, vp, i32]
+        _lib.or_wn_backward_scalar_gain.argtypes = [vp, i64, i64, i64, vp, i32, i64, ct.c_float, dbl, dbl, uns, vp,
+                                                    vp, vp, i32]
         _lib.or_qk_rows_l2.argtypes = [vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, vp, dbl, uns, vp, vp, vp, vp,
                                        i32]
         _lib.or_qk_rows_l2_interval.argtypes = [vp, i64, vp, i64, i64, i32, i32, i32, vp, vp, vp, dbl, dbl, uns, vp,
@@ -71,7 +74,8 @@ def lib() -> ct.CDLL:
         _lib.or_l2_rows_interval.argtypes = [vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
         _lib.or_slerp_rows_interval.argtypes = [vp, vp, vp, i64, i64, i64, dbl, dbl, uns, vp, vp, i32]
         for f in ("or_wn_forward", "or_wn_backward", "or_row_renorm", "or_l2_rows", "or_slerp_rows",
-                  "or_l2_rows_interval", "or_slerp_rows_interval", "or_qk_rows_l2", "or_qk_rows_l2_interval"):
+                  "or_l2_rows_interval", "or_slerp_rows_interval", "or_qk_rows_l2", "or_qk_rows_l2_interval",
+                  "or_row_norms", "or_wn_backward_scalar_gain"):
             getattr(_lib, f).restype = i32
     return _lib
 
@@ -143,6 +147,30 @@ def wn_backward(w, gy, g=None, *, rho=1.0, eps=1e-6, flags=0, nthreads=1):
     _check(lib().or_wn_backward(_p(w), R, C, ld, _p(gy), int(is_bf16), ldg, _p(g), rho, eps, flags,
                                 _p(gw), _p(gg), nthreads), "wn_backward")
     return gw, gg
+
+
+def row_norms(w, *, eps=1e-6, div=1.0):
+    """f64 [R]: sqrt(sum_j w[r,j]^2 + eps) / div (div = rho: the preserving gain)."""
+    w, ld = _rows(w, np.float32)
+    R, C = w.shape
+    out = np.empty((R,), np.float64)
+    _check(lib().or_row_norms(_p(w), R, C, ld, eps, div, _p(out), 1), "row_norms")
+    return out
+
+
+def wn_backward_scalar_gain(w, gy, g, *, rho=1.0, eps=1e-6, flags=0, nthreads=1):
+    """f64 (grad_w [R, C], per-row gain gradients [R], their sum) for one
+    scalar gain g shared by every row."""
+    w, ld = _rows(w, np.float32)
+    is_bf16 = gy.dtype == np.uint16
+    gy, ldg = _rows(gy, np.uint16 if is_bf16 else np.float32)
+    R, C = w.shape
+    gw = np.empty((R, C), np.float64)
+    gg = np.empty((R,), np.float64)
+    tot = ct.c_double()
+    _check(lib().or_wn_backward_scalar_gain(_p(w), R, C, ld, _p(gy), int(is_bf16), ldg, float(g), rho, eps, flags,
+                                            _p(gw), _p(gg), ct.byref(tot), nthreads), "wn_backward_scalar_gain")
+    return gw, gg, tot.value
 
 
 def row_renorm(w, *, rho=1.0, eps=1e-6, flags=0, nthreads=1):
