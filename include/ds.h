@@ -2,8 +2,8 @@
  * ds.h -- C ABI of libds: per-row L2 normalisation of weight and activation
  * rows on NVIDIA B200 (sm_100a).
  *
- * Twelve operations, each over a table of segments (matrices), so that every
- * weight of a model is handled by one call:
+ * Fourteen operations, each over a table of segments (matrices), so that
+ * every weight of a model is handled by one call:
  *
  *   ds_wn_forward   W_eff[r,:] = g_r * rho * w[r,:] / sqrt(sum_j w[r,j]^2 + eps)
  *                   DragonScale package description, "What DragonScale
@@ -27,6 +27,9 @@
  *                   the same part is removed from the momentum -- Adam's
  *                   exp_avg, SGD's or Muon's momentum_buffer -- and each row
  *                   is rescaled back to its radius).
+ *   ds_row_norms, ds_gain_preserve  the row lengths sqrt(sum w^2 + eps) (over
+ *                   rho for the preserving gain); DragonScale, "Monitor" and
+ *                   the options table (`init` "preserve").
  *   ds_l2_rows      y = bf16(s / sqrt(sum s^2 + eps)), s = x or s = bf16(x + r);
  *                   TensorFold PR #1260, Conversation, the norms.cu commit
  *                   (tf_l2_rows: a loop's entry l2(state + input), or its exit).
@@ -122,19 +125,30 @@ typedef void *ds_stream; /* cudaStream_t */
  *   renorm_momentum: w (read and written in place), grad_w = the momentum
  *                    buffer m (read and written in place), rows, cols, ld,
  *                    radius
- * (gain, w_eff, gy, grad_g and ld_out are ignored by the last three.)       */
+ *   row_norms, gain_preserve: w (read), rnorm (written), rows, cols, ld,
+ *                    radius (gain_preserve)
+ * (gain, w_eff, gy, grad_g and ld_out are ignored by the projections and
+ * renorm; rnorm by every call but the last two.)
+ *
+ * gain_scalar (DragonScale options table, `gain` "scalar": one gain for the
+ * layer): gain points to ONE float used by every row, and the backward's
+ * grad_g holds rows + 1 floats: grad_g[r] = rho (w_r . GY_r) / n_r for each
+ * row, then grad_g[rows] = their sum (dL/dg), summed in a fixed order so
+ * that it is the same on every run. */
 typedef struct {
     float *w;          /* fp32 [rows, ld] master rows                                */
-    const float *gain; /* fp32 [rows], or NULL: mode "unit" (g = 1, no grad_g)       */
+    const float *gain; /* fp32 [rows] ([1] with gain_scalar), or NULL: mode "unit"   */
     void *w_eff;       /* forward output [rows, ld_out], dtype per call               */
     const void *gy;    /* backward input dL/dW_eff [rows, ld_out], dtype per call     */
     float *grad_w;     /* backward output fp32 [rows, ld], overwritten                */
-    float *grad_g;     /* backward output fp32 [rows], overwritten (gain != NULL)     */
+    float *grad_g;     /* backward output fp32 [rows] ([rows + 1] with gain_scalar)   */
     int64_t rows;      /* >= 0                                                        */
     int64_t cols;      /* >= 1, <= 2^31 - 1                                           */
     int64_t ld;        /* leading dimension of w and grad_w, >= cols                  */
     int64_t ld_out;    /* leading dimension of w_eff and gy, >= cols                  */
     float radius;      /* rho: 1 for linears and convs, sqrt(cols) for embeddings     */
+    int32_t gain_scalar; /* 0: one gain per row; 1: one gain for the matrix          */
+    float *rnorm;      /* row_norms / gain_preserve output fp32 [rows]                */
 } ds_wseg;
 
 /* One activation matrix; x, r and y share the leading dimension ld.
@@ -211,6 +225,18 @@ ds_status ds_grad_project(const ds_wseg *segs, int nseg, float eps,
  * m <- m - w D/(S+eps) and w <- rho w/sqrt(S+eps).  w and m must not overlap. */
 ds_status ds_renorm_momentum(const ds_wseg *segs, int nseg, float eps,
                              ds_stream stream);
+
+/* rnorm[r] = sqrt(sum_j w[r,j]^2 + eps): DragonScale, "Monitor" (each
+ * layer's raw row lengths; eps = 0 gives the plain length).  w is read
+ * only; rnorm must not overlap it. */
+ds_status ds_row_norms(const ds_wseg *segs, int nseg, float eps,
+                       ds_stream stream);
+
+/* rnorm[r] = sqrt(sum_j w[r,j]^2 + eps) / radius: the gain of DragonScale's
+ * `init` "preserve" (options table: gain = row length, same output), so that
+ * ds_wn_forward with gain = rnorm returns w.  Point rnorm at the gain. */
+ds_status ds_gain_preserve(const ds_wseg *segs, int nseg, float eps,
+                           ds_stream stream);
 
 ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps,
                      ds_stream stream);

@@ -384,7 +384,8 @@ WSegK wseg_rows(const ds_wseg &s, int64_t r0, int64_t nr, int out_esize, int gy_
 {
     WSegK k{};
     k.w = s.w ? s.w + r0 * s.ld : nullptr;
-    k.gain = s.gain ? s.gain + r0 : nullptr;
+    k.gain = s.gain ? (s.gain_scalar ? s.gain : s.gain + r0) : nullptr;
+    k.gain_stride = s.gain_scalar ? 0 : 1;
     k.out = s.w_eff ? static_cast<char *>(s.w_eff) + r0 * s.ld_out * out_esize : nullptr;
     k.gy = s.gy ? static_cast<const char *>(s.gy) + r0 * s.ld_out * gy_esize : nullptr;
     k.grad_w = s.grad_w ? s.grad_w + r0 * s.ld : nullptr;
@@ -441,12 +442,18 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
             return st;
         if (fwd_bwd && s.gain && !aligned(s.gain, 4))
             return fail(DS_ERR_ALIGNMENT, where("gain is not 4-byte aligned", i));
+        if (fwd_bwd && s.gain_scalar != 0 && s.gain_scalar != 1)
+            return fail(DS_ERR_INVALID_ARG, where("gain_scalar must be 0 or 1", i));
+        if (fwd_bwd && s.gain_scalar && !s.gain)
+            return fail(DS_ERR_INVALID_ARG, where("gain_scalar needs a gain", i));
+        // gain: [rows], or [1] for a scalar gain; grad_g: [rows] or [rows + 1]
+        const int64_t ng = s.gain_scalar ? 1 : s.rows, ngg = s.gain_scalar ? s.rows + 1 : s.rows;
         if (wop == W_FWD) {
             if (ds_status st = check_matrix(s.w_eff, s.rows, s.ld_out, esize, "w_eff", i))
                 return st;
             spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 0, -1));
             if (s.gain)
-                spans.push_back(span_of(s.gain, 1, s.rows, s.rows, 4, i, 0, -1));
+                spans.push_back(span_of(s.gain, 1, ng, ng, 4, i, 0, -1));
             spans.push_back(span_of(s.w_eff, s.rows, s.cols, s.ld_out, esize, i, 1, -1));
         } else if (wop == W_BWD) {
             if (ds_status st = check_matrix(s.gy, s.rows, s.ld_out, esize, "gy", i))
@@ -461,8 +468,8 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
             spans.push_back(span_of(s.gy, s.rows, s.cols, s.ld_out, esize, i, 0, -1));
             spans.push_back(span_of(s.grad_w, s.rows, s.cols, s.ld, 4, i, 1, -1));
             if (s.gain) {
-                spans.push_back(span_of(s.gain, 1, s.rows, s.rows, 4, i, 0, -1));
-                spans.push_back(span_of(s.grad_g, 1, s.rows, s.rows, 4, i, 1, -1));
+                spans.push_back(span_of(s.gain, 1, ng, ng, 4, i, 0, -1));
+                spans.push_back(span_of(s.grad_g, 1, ngg, ngg, 4, i, 1, -1));
             }
         } else if (wop == W_PROJECT || wop == W_MOMENTUM) {
             if (ds_status st = check_matrix(s.grad_w, s.rows, s.ld, 4,
@@ -524,7 +531,91 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         default: return ds::launch_row_renorm(rc, p, units, st);
         }
     };
-    return launch_all<WParams, WSegK>(nseg, rows.data(), cls, eps, make, launch, stream);
+    if (ds_status st = launch_all<WParams, WSegK>(nseg, rows.data(), cls, eps, make, launch, stream))
+        return st;
+    if (wop != W_BWD)
+        return DS_OK;
+    // scalar gains: dL/dg = the per-row parts summed (fixed order), after them
+    static thread_local ds::GainSumParams sums;
+    sums.nseg = 0;
+    auto flush_sums = [&]() -> ds_status {
+        if (sums.nseg == 0)
+            return DS_OK;
+        if (ds::launch_gain_sums(sums, stream) != 0)
+            return fail(DS_ERR_CUDA, "gain-sum launch failed");
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        sums.nseg = 0;
+        return DS_OK;
+    };
+    for (int i = 0; i < nseg; ++i) {
+        const ds_wseg &s = segs[i];
+        if (!s.gain || !s.gain_scalar)
+            continue;
+        if (sums.nseg == ds::kSegPerLaunch)
+            if (ds_status st = flush_sums())
+                return st;
+        sums.seg[sums.nseg++] = ds::GainSumK{s.grad_g, s.rows};
+    }
+    return flush_sums();
+}
+
+// ------------------------------------------------------------ row lengths --
+
+ds_status run_norms(bool preserve, const ds_wseg *segs, int nseg, float eps, void *stream)
+{
+    g_last_error.clear();
+    if (ds_status s = check_common(nseg, segs, eps, stream))
+        return s;
+    std::vector<Span> spans;
+    for (int i = 0; i < nseg; ++i) {
+        const ds_wseg &s = segs[i];
+        if (ds_status st = check_shape(s.rows, s.cols, s.ld, i))
+            return st;
+        if (preserve && !(std::isfinite(s.radius) && s.radius > 0.f))
+            return fail(DS_ERR_INVALID_ARG, where("radius must be finite and > 0", i));
+        if (s.rows == 0)
+            continue;
+        if (ds_status st = check_matrix(s.w, s.rows, s.ld, 4, "w", i))
+            return st;
+        if (!s.rnorm)
+            return fail(DS_ERR_INVALID_ARG, where("rnorm is NULL", i));
+        if (!aligned(s.rnorm, 4))
+            return fail(DS_ERR_ALIGNMENT, where("rnorm is not 4-byte aligned", i));
+        spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 0, -1));
+        spans.push_back(span_of(s.rnorm, 1, s.rows, s.rows, 4, i, 1, -1));
+    }
+    if (ds_status st = check_overlaps(spans))
+        return st;
+    static thread_local ds::RNParams params;
+    int n = 0;
+    int64_t units = 0;
+    auto flush = [&]() -> ds_status {
+        if (n == 0)
+            return DS_OK;
+        params.nseg = n;
+        params.unit_start[n] = units;
+        params.eps = eps;
+        if (ds::launch_row_norms(params, stream) != 0)
+            return fail(DS_ERR_CUDA, "kernel launch failed");
+        g_launches.fetch_add(1, std::memory_order_relaxed);
+        n = 0;
+        units = 0;
+        return DS_OK;
+    };
+    for (int i = 0; i < nseg; ++i) {
+        const ds_wseg &s = segs[i];
+        if (s.rows == 0)
+            continue;
+        if (n == ds::kSegPerLaunch)
+            if (ds_status st = flush())
+                return st;
+        params.seg[n] = ds::RNSegK{s.w, s.rnorm, s.rows, s.ld, static_cast<int32_t>(s.cols),
+                                   preserve ? s.radius : 1.f};
+        params.unit_start[n] = units;
+        units += s.rows;
+        ++n;
+    }
+    return flush();
 }
 
 ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *stream)
@@ -971,6 +1062,16 @@ ds_status ds_gate_l2_rows(const ds_fseg *segs, int nseg, float eps, ds_stream st
 ds_status ds_swiglu_l2_rows(const ds_fseg *segs, int nseg, float eps, ds_stream stream)
 {
     return run_fused(true, segs, nseg, eps, stream);
+}
+
+ds_status ds_row_norms(const ds_wseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_norms(false, segs, nseg, eps, stream);
+}
+
+ds_status ds_gain_preserve(const ds_wseg *segs, int nseg, float eps, ds_stream stream)
+{
+    return run_norms(true, segs, nseg, eps, stream);
 }
 
 ds_status ds_qk_rows_l2(const ds_qkseg *segs, int nseg, float eps, ds_stream stream)

@@ -85,6 +85,8 @@ struct WSegK {
     int32_t nu;       // units per row
     float radius;
     int32_t group;    // staged paths: rows per slot
+    int32_t gain_stride; // 1: gain[row]; 0: one gain for every row
+    int32_t pad_;
 };
 
 // Device copy of one activation segment (bf16 carried as raw 16-bit words).
@@ -159,6 +161,31 @@ struct QKParams {
     float eps;
 };
 
+// Row lengths (ds_kernels.cu): out[r] = sqrt(sum w[r,:]^2 + eps) / div.
+struct RNSegK {
+    const float *w;
+    float *out;
+    int64_t rows, ld;
+    int32_t cols;
+    float div;
+};
+struct RNParams {
+    RNSegK seg[kSegPerLaunch];
+    int64_t unit_start[kSegPerLaunch + 1]; // prefix sums of rows
+    int32_t nseg;
+    float eps;
+};
+// Scalar gains (ds_kernels.cu): parts[rows] = sum of parts[0..rows) in a
+// fixed order, for each listed buffer.
+struct GainSumK {
+    float *parts;
+    int64_t rows;
+};
+struct GainSumParams {
+    GainSumK seg[kSegPerLaunch];
+    int32_t nseg;
+};
+
 // Error word written by kernels (see ds_get_device_status).
 enum DeviceErrorSite : uint32_t {
     kSiteStreamWait = 1,
@@ -178,6 +205,8 @@ int launch_renorm_momentum(const RowClass &rc, const WParams &p, int64_t units, 
 int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_wait_selftest(uint64_t limit_ns, void *stream);
+int launch_row_norms(const RNParams &p, void *stream);
+int launch_gain_sums(const GainSumParams &p, void *stream);
 // Staged paths (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,
 // 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp,
 // 7 gradient projection, 8 momentum projection + renorm, 9 l2 backward,

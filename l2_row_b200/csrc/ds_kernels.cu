@@ -13,6 +13,7 @@
 //   wn_forward, wn_backward, row_renorm : DragonScale unit rows with gains
 //   grad_project, renorm_momentum       : DragonScale "Optimizer" (rescale)
 //   l2_rows, slerp_rows                 : TensorFold tf_l2_rows, tf_slerp_rows
+#include <algorithm>
 #include <cuda_runtime.h>
 
 #include "ds_device.cuh"
@@ -223,7 +224,7 @@ __device__ __forceinline__ void wn_scale_row(const WSegK &sg, int64_t row, bool 
         const int u = ubeg + lane + k * stride;
         x[k] = (active && u < uend) ? quad_f32(w, u, sg.cols) : make_float4(kZero, kZero, kZero, kZero);
     }
-    const float g = (!RENORM && active && sg.gain) ? __ldg(sg.gain + row) : 1.f;
+    const float g = (!RENORM && active && sg.gain) ? __ldg(sg.gain + row * sg.gain_stride) : 1.f;
     float acc[1] = {0.f};
 #pragma unroll
     for (int k = 0; k < KMAX; ++k)
@@ -272,7 +273,7 @@ __device__ __forceinline__ void wn_backward_row(const WSegK &sg, int64_t row, bo
         x[k] = ok ? quad_f32(w, u, sg.cols) : make_float4(kZero, kZero, kZero, kZero);
         d[k] = ok ? quad_gy<GY_BF16>(gy, u, sg.cols) : make_float4(kZero, kZero, kZero, kZero);
     }
-    const float g = (active && sg.gain) ? __ldg(sg.gain + row) : 1.f;
+    const float g = (active && sg.gain) ? __ldg(sg.gain + row * sg.gain_stride) : 1.f;
     float acc[2] = {0.f, 0.f};
 #pragma unroll
     for (int k = 0; k < KMAX; ++k) {
@@ -605,7 +606,7 @@ struct SScale {
             for (int ul = threadIdx.x; ul < c.len; ul += kCta)
                 each4(quad_f32(w, c.ubeg + ul, c.cols), f);
         });
-        const float g = (!RENORM && sg.gain) ? __ldg(sg.gain + row) : 1.f;
+        const float g = (!RENORM && sg.gain) ? __ldg(sg.gain + row * sg.gain_stride) : 1.f;
         sc = (g * sg.radius) * rs.inv;
         pre = rs.pre;
     }
@@ -711,7 +712,7 @@ struct SBackward {
             sc = sg.radius * inv;   // rho / n times 2^-m
             return;
         }
-        const float g = sg.gain ? __ldg(sg.gain + row) : 1.f;
+        const float g = sg.gain ? __ldg(sg.gain + row * sg.gain_stride) : 1.f;
         q = m == 0 ? acc[1] / n2 : scalbnf(acc[1] / n2, m);
         pre = (g * sg.radius) * (m == 0 ? inv : scalbnf(inv, m));
         gg = sg.radius * acc[1] * inv;
@@ -1052,6 +1053,92 @@ cudaError_t launch_op(const RowClass &rc, const ParamsOf<T> &p, int64_t units, v
     }
 }
 
+// ============================================================ row lengths ==
+//
+// One warp per row (the rows of every segment in one grid-stride walk): the
+// lanes sum quads lane, lane + 32, ... in order into two accumulators, then
+// the butterfly; rows whose fp32 sum overflows (or, at eps = 0, underflows)
+// are summed again after an exact power-of-two scaling, as every row op
+// here does.  Lane 0 writes sqrt(S + eps) / div.
+
+struct WarpRowRed {
+    __device__ __forceinline__ bool any(bool b) const { return __any_sync(0xffffffffu, b); }
+    __device__ __forceinline__ float max(float v) const
+    {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        return v;
+    }
+    template <int N>
+    __device__ __forceinline__ void sum(float (&v)[N]) const
+    {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int i = 0; i < N; ++i)
+                v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+    }
+};
+
+__global__ void __launch_bounds__(kCta) k_row_norms(const __grid_constant__ RNParams p)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = (static_cast<int64_t>(blockIdx.x) * kCta + threadIdx.x) >> 5;
+    const int64_t nw = (static_cast<int64_t>(gridDim.x) * kCta) >> 5;
+    const int64_t total = p.unit_start[p.nseg];
+    const WarpRowRed red;
+    for (int64_t u = gw; u < total; u += nw) {
+        const int si = find_segment(p, u);
+        const RNSegK &sg = p.seg[si];
+        const int64_t row = u - p.unit_start[si];
+        const float *w = sg.w + row * sg.ld;
+        const int nq = (sg.cols + 3) / 4;
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+        for (int q = lane; q < nq; q += 32) {
+            const float4 v = quad_f32(w, q, sg.cols);
+            a0 = fmaf(v.x, v.x, a0);
+            a1 = fmaf(v.y, v.y, a1);
+            a0 = fmaf(v.z, v.z, a0);
+            a1 = fmaf(v.w, v.w, a1);
+        }
+        float S[1] = {a0 + a1};
+        red.sum(S);
+        float Ss = S[0];
+        const int m = rescale_exponent(S[0], p.eps, red, [&](auto f) {
+            for (int q = lane; q < nq; q += 32)
+                each4(quad_f32(w, q, sg.cols), f);
+        }, Ss);
+        const float len = m == 0 ? sqrtf(S[0] + p.eps) : scalbnf(sqrtf(Ss + scalbnf(p.eps, 2 * m)), -m);
+        if (lane == 0)
+            sg.out[row] = __fdiv_rn(len, sg.div);
+    }
+}
+
+// ===================================================== scalar gain sums ==
+//
+// One block per buffer: thread t adds parts t, t + 1024, ... in order in
+// double, then a fixed tree over the block; the sum is rounded once to fp32.
+
+__global__ void __launch_bounds__(1024) k_gain_sums(const __grid_constant__ GainSumParams p)
+{
+    __shared__ double part[1024];
+    const GainSumK &sg = p.seg[blockIdx.x];
+    double acc = 0.0;
+    for (int64_t i = threadIdx.x; i < sg.rows; i += 1024)
+        acc += static_cast<double>(sg.parts[i]);
+    part[threadIdx.x] = acc;
+    __syncthreads();
+    for (int o = 512; o > 0; o >>= 1) {
+        if (threadIdx.x < o)
+            part[threadIdx.x] += part[threadIdx.x + o];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0)
+        sg.parts[sg.rows] = static_cast<float>(part[0]);
+}
+
 } // namespace
 
 int launch_wn_forward(const RowClass &rc, const WParams &p, int64_t units, bool out_bf16, void *stream)
@@ -1087,6 +1174,20 @@ int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *st
 int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream)
 {
     return launch_op<kSlerp>(rc, p, units, stream);
+}
+
+int launch_row_norms(const RNParams &p, void *stream)
+{
+    const int64_t warps = p.unit_start[p.nseg];
+    const int64_t blocks = std::min<int64_t>((warps + kWarps - 1) / kWarps, 148 * 8);
+    k_row_norms<<<static_cast<int>(blocks), kCta, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError();
+}
+
+int launch_gain_sums(const GainSumParams &p, void *stream)
+{
+    k_gain_sums<<<p.nseg, 1024, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError();
 }
 
 int launch_wait_selftest(uint64_t limit_ns, void *stream)

@@ -1511,7 +1511,7 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                 if constexpr (T == tFwdBf16 || T == tFwdF32 || T == tBwdBf16 || T == tBwdF32) {
                     // gains of the next 32 rows, one per lane
                     if ((r & 31) == 0)
-                        g_lane = (sg.gain && r + lane < h.nrows) ? __ldg(sg.gain + row + lane) : 1.f;
+                        g_lane = (sg.gain && r + lane < h.nrows) ? __ldg(sg.gain + (row + lane) * sg.gain_stride) : 1.f;
                 }
                 const float g = __shfl_sync(0xffffffffu, g_lane, r & 31);
                 if constexpr (T == tFwdBf16)

@@ -53,7 +53,8 @@ PATH_NAMES = {DS_PATH_WARP: "warp", DS_PATH_CTA: "cta", DS_PATH_CLUSTER: "cluste
 class ds_wseg(ct.Structure):
     _fields_ = [("w", ct.c_void_p), ("gain", ct.c_void_p), ("w_eff", ct.c_void_p), ("gy", ct.c_void_p),
                 ("grad_w", ct.c_void_p), ("grad_g", ct.c_void_p), ("rows", ct.c_int64), ("cols", ct.c_int64),
-                ("ld", ct.c_int64), ("ld_out", ct.c_int64), ("radius", ct.c_float)]
+                ("ld", ct.c_int64), ("ld_out", ct.c_int64), ("radius", ct.c_float), ("gain_scalar", ct.c_int32),
+                ("rnorm", ct.c_void_p)]
 
 
 class ds_aseg(ct.Structure):
@@ -92,6 +93,8 @@ _lib.ds_l2_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float,
 _lib.ds_gate_l2_rows.argtypes = [ct.POINTER(ds_fseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_swiglu_l2_rows.argtypes = [ct.POINTER(ds_fseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_qk_rows_l2.argtypes = [ct.POINTER(ds_qkseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_row_norms.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, ct.c_void_p]
+_lib.ds_gain_preserve.argtypes = [ct.POINTER(ds_wseg), ct.c_int, ct.c_float, ct.c_void_p]
 _lib.ds_slerp_rows_backward.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p, ct.c_void_p,
                                         ct.c_uint64, ct.c_void_p]
 _lib.ds_slerp_rows_backward_noalloc.argtypes = [ct.POINTER(ds_agseg), ct.c_int, ct.c_float, ct.c_void_p,
@@ -101,7 +104,8 @@ _lib.ds_slerp_rows_backward_workspace.argtypes = [ct.c_int64]
 _lib.ds_slerp_rows_backward_workspace.restype = ct.c_uint64
 for _f in ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
-           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_qk_rows_l2", "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
+           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_qk_rows_l2", "ds_row_norms", "ds_gain_preserve",
+           "ds_get_device_status", "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns",
            "ds_debug_wait_timeout_selftest", "ds_debug_division_check"):
     getattr(_lib, _f).restype = _st
 _lib.ds_status_string.argtypes = [ct.c_int]
@@ -123,7 +127,8 @@ _lib.ds_debug_division_check.argtypes = [ct.c_void_p, ct.c_void_p]
 #: every symbol include/ds.h declares
 EXPORTS = ("ds_wn_forward", "ds_wn_backward", "ds_row_renorm", "ds_grad_project", "ds_renorm_momentum",
            "ds_l2_rows", "ds_slerp_rows", "ds_l2_rows_backward", "ds_slerp_rows_backward",
-           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_qk_rows_l2", "ds_slerp_rows_backward_workspace", "ds_slerp_rows_backward_noalloc", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
+           "ds_gate_l2_rows", "ds_swiglu_l2_rows", "ds_qk_rows_l2", "ds_row_norms", "ds_gain_preserve",
+           "ds_slerp_rows_backward_workspace", "ds_slerp_rows_backward_noalloc", "ds_status_string", "ds_last_error", "ds_get_device_status", "ds_launch_count", "ds_version",
            "ds_row_class", "ds_debug_force_path", "ds_debug_set_wait_limit_ns", "ds_debug_wait_timeout_selftest",
            "ds_debug_division_check")
 
@@ -197,7 +202,10 @@ class WSeg:
     """One weight matrix.  w: fp32 [R, C]; gain: fp32 [R] or None; w_eff:
     forward output [R, C]; gy, grad_w, grad_g: backward input/outputs.
     For ds_grad_project grad_w is the gradient and for ds_renorm_momentum
-    the momentum buffer (fp32 [R, C], w's leading dimension, in place)."""
+    the momentum buffer (fp32 [R, C], w's leading dimension, in place).
+    gain_scalar: gain is fp32 [1] shared by every row and grad_g fp32 [R + 1]
+    (per-row parts, then their sum).  rnorm: fp32 [R] output of
+    ds_row_norms / ds_gain_preserve."""
 
     w: Any
     gain: Any = None
@@ -206,6 +214,8 @@ class WSeg:
     grad_w: Any = None
     grad_g: Any = None
     radius: float = 1.0
+    gain_scalar: bool = False
+    rnorm: Any = None
 
     def to_c(self) -> ds_wseg:
         R, C = (int(self.w.shape[0]), int(self.w.shape[1]))
@@ -218,7 +228,8 @@ class WSeg:
         if self.grad_w is not None and ld_gw != ld:
             raise ValueError("grad_w must share w's leading dimension")
         return ds_wseg(w, _vec(self.gain), weff, gy, gw, _vec(self.grad_g), R, C, ld,
-                       ld_out if self.w_eff is not None else ld_gy, float(self.radius))
+                       ld_out if self.w_eff is not None else ld_gy, float(self.radius), int(bool(self.gain_scalar)),
+                       _vec(self.rnorm))
 
 
 @dataclass
@@ -392,6 +403,16 @@ def ds_gate_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
 def ds_swiglu_l2_rows(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
     arr, n = _table(segs, ds_fseg)
     _check(_lib.ds_swiglu_l2_rows(arr, n, eps, _stream_ptr(stream)), "ds_swiglu_l2_rows")
+
+
+def ds_row_norms(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_wseg)
+    _check(_lib.ds_row_norms(arr, n, eps, _stream_ptr(stream)), "ds_row_norms")
+
+
+def ds_gain_preserve(segs: Sequence, eps: float = 1e-6, stream=None) -> None:
+    arr, n = _table(segs, ds_wseg)
+    _check(_lib.ds_gain_preserve(arr, n, eps, _stream_ptr(stream)), "ds_gain_preserve")
 
 
 def ds_qk_rows_l2(segs: Sequence, eps: float = 1e-6, stream=None) -> None:

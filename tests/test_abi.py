@@ -436,3 +436,21 @@ def test_qk_shifted_cache_alias_refused():
     """k_cache may be exactly k (row for row); a cache that starts one row
     into k overlaps it and is refused before anything runs."""
     assert call_qk([qkseg(k_cache=BASE + (1 << 30) + 128)]) == ds.DS_ERR_OVERLAP
+
+
+# ------------------------------------------- scalar gain and row lengths --
+
+def test_scalar_gain_and_row_norm_validation():
+    E = ds
+    before = ds.ds_launch_count()
+    assert call_w("ds_wn_forward", [wseg(gain=None, gain_scalar=1)]) == E.DS_ERR_INVALID_ARG
+    assert call_w("ds_wn_forward", [wseg(gain_scalar=2)]) == E.DS_ERR_INVALID_ARG
+    arr = (ds.ds_wseg * 1)(wseg(rnorm=None))
+    assert ds.lib().ds_row_norms(arr, 1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
+    arr = (ds.ds_wseg * 1)(wseg(rnorm=BASE + (5 << 30) + 2))
+    assert ds.lib().ds_row_norms(arr, 1, ct.c_float(1e-6), None) == E.DS_ERR_ALIGNMENT
+    arr = (ds.ds_wseg * 1)(wseg(rnorm=BASE + 64))                  # inside w
+    assert ds.lib().ds_row_norms(arr, 1, ct.c_float(1e-6), None) == E.DS_ERR_OVERLAP
+    arr = (ds.ds_wseg * 1)(wseg(rnorm=BASE + (5 << 30), radius=0.0))
+    assert ds.lib().ds_gain_preserve(arr, 1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
+    assert ds.ds_launch_count() == before
