@@ -206,7 +206,7 @@ def measured_peaks() -> tuple[float, str]:
 def kernel_source_digest() -> str:
     h = hashlib.sha256()
     for rel in ("l2_row_b200/csrc/ds_kernels.cu", "l2_row_b200/csrc/ds_tile.cu", "l2_row_b200/csrc/ds_qk.cu",
-                "l2_row_b200/csrc/ds_api.cpp",
+                "l2_row_b200/csrc/ds_col.cu", "l2_row_b200/csrc/ds_api.cpp",
                 "l2_row_b200/csrc/ds_device.cuh", "l2_row_b200/csrc/ds_internal.h"):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())

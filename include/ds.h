@@ -149,6 +149,10 @@ typedef struct {
     float radius;      /* rho: 1 for linears and convs, sqrt(cols) for embeddings     */
     int32_t gain_scalar; /* 0: one gain per row; 1: one gain for the matrix          */
     float *rnorm;      /* row_norms / gain_preserve output fp32 [rows]                */
+    int32_t transposed; /* 1: the rows are the COLUMNS of w, w_eff, gy and grad_w,
+                          stored [cols, ld] (element j of row r at [j * ld + r],
+                          ld >= rows): GPT-2's Conv1D [in, out] weights.  Forward,
+                          backward, renorm and the projections; not row_norms. */
 } ds_wseg;
 
 /* One activation matrix; x, r and y share the leading dimension ld.

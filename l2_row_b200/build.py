@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libds.so")
-SOURCES = ["ds_kernels.cu", "ds_tile.cu", "ds_qk.cu", "ds_api.cpp"]
+SOURCES = ["ds_kernels.cu", "ds_tile.cu", "ds_qk.cu", "ds_col.cu", "ds_api.cpp"]
 HEADERS = ["ds_internal.h", "ds_device.cuh"]
 
 NVCC_FLAGS = [

@@ -428,17 +428,27 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
     std::vector<int64_t> rows(static_cast<size_t>(nseg)), cols(static_cast<size_t>(nseg));
     for (int i = 0; i < nseg; ++i) {
         const ds_wseg &s = segs[i];
-        if (ds_status st = check_shape(s.rows, s.cols, s.ld, i))
+        if (s.transposed != 0 && s.transposed != 1)
+            return fail(DS_ERR_INVALID_ARG, where("transposed must be 0 or 1", i));
+        const bool tr = s.transposed != 0;
+        // the stored matrix: [rows, ld] with cols used per row, or
+        // (transposed) [cols, ld] with rows used per stored row
+        const int64_t sr = tr ? s.cols : s.rows, sc = tr ? s.rows : s.cols;
+        if (ds_status st = check_shape(s.rows, s.cols, tr ? std::max<int64_t>(s.ld, s.cols) : s.ld, i))
             return st;
-        if (fwd_bwd && s.ld_out < s.cols)
-            return fail(DS_ERR_INVALID_ARG, where("ld_out < cols", i));
+        if (tr && s.ld < s.rows)
+            return fail(DS_ERR_INVALID_ARG, where("transposed: leading dimension < rows", i));
+        if (tr && s.rows > (int64_t(1) << 31) - 1)
+            return fail(DS_ERR_INVALID_ARG, where("transposed: rows above 2^31 - 1", i));
+        if (fwd_bwd && s.ld_out < sc)
+            return fail(DS_ERR_INVALID_ARG, where(tr ? "transposed: ld_out < rows" : "ld_out < cols", i));
         if (!std::isfinite(s.radius))
             return fail(DS_ERR_INVALID_ARG, where("radius is not finite", i));
-        rows[i] = s.rows;
+        rows[i] = tr ? 0 : s.rows; // transposed segments launch on their own
         cols[i] = s.cols;
         if (s.rows == 0)
             continue;
-        if (ds_status st = check_matrix(s.w, s.rows, s.ld, 4, "w", i))
+        if (ds_status st = check_matrix(s.w, sr, s.ld, 4, "w", i))
             return st;
         if (fwd_bwd && s.gain && !aligned(s.gain, 4))
             return fail(DS_ERR_ALIGNMENT, where("gain is not 4-byte aligned", i));
@@ -449,38 +459,38 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         // gain: [rows], or [1] for a scalar gain; grad_g: [rows] or [rows + 1]
         const int64_t ng = s.gain_scalar ? 1 : s.rows, ngg = s.gain_scalar ? s.rows + 1 : s.rows;
         if (wop == W_FWD) {
-            if (ds_status st = check_matrix(s.w_eff, s.rows, s.ld_out, esize, "w_eff", i))
+            if (ds_status st = check_matrix(s.w_eff, sr, s.ld_out, esize, "w_eff", i))
                 return st;
-            spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 0, -1));
+            spans.push_back(span_of(s.w, sr, sc, s.ld, 4, i, 0, -1));
             if (s.gain)
                 spans.push_back(span_of(s.gain, 1, ng, ng, 4, i, 0, -1));
-            spans.push_back(span_of(s.w_eff, s.rows, s.cols, s.ld_out, esize, i, 1, -1));
+            spans.push_back(span_of(s.w_eff, sr, sc, s.ld_out, esize, i, 1, -1));
         } else if (wop == W_BWD) {
-            if (ds_status st = check_matrix(s.gy, s.rows, s.ld_out, esize, "gy", i))
+            if (ds_status st = check_matrix(s.gy, sr, s.ld_out, esize, "gy", i))
                 return st;
-            if (ds_status st = check_matrix(s.grad_w, s.rows, s.ld, 4, "grad_w", i))
+            if (ds_status st = check_matrix(s.grad_w, sr, s.ld, 4, "grad_w", i))
                 return st;
             if (s.gain && !s.grad_g)
                 return fail(DS_ERR_INVALID_ARG, where("grad_g is NULL while gain is set", i));
             if (s.gain && !aligned(s.grad_g, 4))
                 return fail(DS_ERR_ALIGNMENT, where("grad_g is not 4-byte aligned", i));
-            spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 0, -1));
-            spans.push_back(span_of(s.gy, s.rows, s.cols, s.ld_out, esize, i, 0, -1));
-            spans.push_back(span_of(s.grad_w, s.rows, s.cols, s.ld, 4, i, 1, -1));
+            spans.push_back(span_of(s.w, sr, sc, s.ld, 4, i, 0, -1));
+            spans.push_back(span_of(s.gy, sr, sc, s.ld_out, esize, i, 0, -1));
+            spans.push_back(span_of(s.grad_w, sr, sc, s.ld, 4, i, 1, -1));
             if (s.gain) {
                 spans.push_back(span_of(s.gain, 1, ng, ng, 4, i, 0, -1));
                 spans.push_back(span_of(s.grad_g, 1, ngg, ngg, 4, i, 1, -1));
             }
         } else if (wop == W_PROJECT || wop == W_MOMENTUM) {
-            if (ds_status st = check_matrix(s.grad_w, s.rows, s.ld, 4,
+            if (ds_status st = check_matrix(s.grad_w, sr, s.ld, 4,
                                             wop == W_PROJECT ? "grad_w (the gradient)" : "grad_w (the momentum)", i))
                 return st;
             // the gradient / momentum is updated in place; w is read (project)
             // or updated in place (momentum); the two must not overlap
-            spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, wop == W_MOMENTUM ? 1 : 0, -1));
-            spans.push_back(span_of(s.grad_w, s.rows, s.cols, s.ld, 4, i, 1, -1));
+            spans.push_back(span_of(s.w, sr, sc, s.ld, 4, i, wop == W_MOMENTUM ? 1 : 0, -1));
+            spans.push_back(span_of(s.grad_w, sr, sc, s.ld, 4, i, 1, -1));
         } else {
-            spans.push_back(span_of(s.w, s.rows, s.cols, s.ld, 4, i, 1, -1));
+            spans.push_back(span_of(s.w, sr, sc, s.ld, 4, i, 1, -1));
         }
     }
     if (ds_status st = check_overlaps(spans))
@@ -533,6 +543,40 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
     };
     if (ds_status st = launch_all<WParams, WSegK>(nseg, rows.data(), cls, eps, make, launch, stream))
         return st;
+    // transposed rows: one launch over all of them (tiles of col_tile_rows())
+    {
+        static thread_local WParams tp;
+        const int tile = ds::col_tile_rows();
+        const int cop = wop == W_FWD ? 0 : wop == W_BWD ? 1 : wop == W_RENORM ? 2 : wop == W_PROJECT ? 3 : 4;
+        int n = 0;
+        int64_t units = 0;
+        auto flush = [&]() -> ds_status {
+            if (n == 0)
+                return DS_OK;
+            tp.nseg = n;
+            tp.unit_start[n] = units;
+            tp.eps = eps;
+            if (ds::launch_col(cop, bf16, tp, units, stream) != 0)
+                return fail(DS_ERR_CUDA, "kernel launch failed (transposed rows)");
+            g_launches.fetch_add(1, std::memory_order_relaxed);
+            n = 0;
+            units = 0;
+            return DS_OK;
+        };
+        for (int i = 0; i < nseg; ++i) {
+            if (!segs[i].transposed || segs[i].rows == 0)
+                continue;
+            if (n == ds::kSegPerLaunch)
+                if (ds_status st = flush())
+                    return st;
+            tp.seg[n] = make(i, 0, segs[i].rows);
+            tp.unit_start[n] = units;
+            units += (segs[i].rows + tile - 1) / tile;
+            ++n;
+        }
+        if (ds_status st = flush())
+            return st;
+    }
     if (wop != W_BWD)
         return DS_OK;
     // scalar gains: dL/dg = the per-row parts summed (fixed order), after them
@@ -573,6 +617,8 @@ ds_status run_norms(bool preserve, const ds_wseg *segs, int nseg, float eps, voi
             return st;
         if (preserve && !(std::isfinite(s.radius) && s.radius > 0.f))
             return fail(DS_ERR_INVALID_ARG, where("radius must be finite and > 0", i));
+        if (s.transposed)
+            return fail(DS_ERR_INVALID_ARG, where("transposed rows are not supported here", i));
         if (s.rows == 0)
             continue;
         if (ds_status st = check_matrix(s.w, s.rows, s.ld, 4, "w", i))

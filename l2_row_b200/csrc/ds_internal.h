@@ -206,6 +206,11 @@ int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *st
 int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_wait_selftest(uint64_t limit_ns, void *stream);
 int launch_row_norms(const RNParams &p, void *stream);
+// Transposed rows (ds_col.cu): op 0 forward, 1 backward, 2 renorm,
+// 3 gradient projection, 4 momentum projection; b16: bf16 W_eff / GY.
+// p's unit_start counts tiles of col_tile_rows() rows.
+int launch_col(int op, bool b16, const WParams &p, int64_t units, void *stream);
+int col_tile_rows();
 int launch_gain_sums(const GainSumParams &p, void *stream);
 // Staged paths (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,
 // 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp,

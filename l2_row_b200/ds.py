@@ -54,7 +54,7 @@ class ds_wseg(ct.Structure):
     _fields_ = [("w", ct.c_void_p), ("gain", ct.c_void_p), ("w_eff", ct.c_void_p), ("gy", ct.c_void_p),
                 ("grad_w", ct.c_void_p), ("grad_g", ct.c_void_p), ("rows", ct.c_int64), ("cols", ct.c_int64),
                 ("ld", ct.c_int64), ("ld_out", ct.c_int64), ("radius", ct.c_float), ("gain_scalar", ct.c_int32),
-                ("rnorm", ct.c_void_p)]
+                ("rnorm", ct.c_void_p), ("transposed", ct.c_int32)]
 
 
 class ds_aseg(ct.Structure):
@@ -205,7 +205,9 @@ class WSeg:
     the momentum buffer (fp32 [R, C], w's leading dimension, in place).
     gain_scalar: gain is fp32 [1] shared by every row and grad_g fp32 [R + 1]
     (per-row parts, then their sum).  rnorm: fp32 [R] output of
-    ds_row_norms / ds_gain_preserve."""
+    ds_row_norms / ds_gain_preserve.  transposed: the unit rows are the
+    columns of w (GPT-2 Conv1D, stored [in, out] = [C, R]); w, w_eff, gy and
+    grad_w are then given in that stored layout."""
 
     w: Any
     gain: Any = None
@@ -216,20 +218,22 @@ class WSeg:
     radius: float = 1.0
     gain_scalar: bool = False
     rnorm: Any = None
+    transposed: bool = False
 
     def to_c(self) -> ds_wseg:
-        R, C = (int(self.w.shape[0]), int(self.w.shape[1]))
-        w, ld = _mat(self.w, "w", R, C)
-        weff, ld_out = _mat(self.w_eff, "w_eff", R, C)
-        gy, ld_gy = _mat(self.gy, "gy", R, C)
-        gw, ld_gw = _mat(self.grad_w, "grad_w", R, C)
+        SR, SC = (int(self.w.shape[0]), int(self.w.shape[1]))   # the stored shape
+        R, C = (SC, SR) if self.transposed else (SR, SC)
+        w, ld = _mat(self.w, "w", SR, SC)
+        weff, ld_out = _mat(self.w_eff, "w_eff", SR, SC)
+        gy, ld_gy = _mat(self.gy, "gy", SR, SC)
+        gw, ld_gw = _mat(self.grad_w, "grad_w", SR, SC)
         if self.w_eff is not None and self.gy is not None and ld_out != ld_gy:
             raise ValueError("w_eff and gy must share a leading dimension")
         if self.grad_w is not None and ld_gw != ld:
             raise ValueError("grad_w must share w's leading dimension")
         return ds_wseg(w, _vec(self.gain), weff, gy, gw, _vec(self.grad_g), R, C, ld,
                        ld_out if self.w_eff is not None else ld_gy, float(self.radius), int(bool(self.gain_scalar)),
-                       _vec(self.rnorm))
+                       _vec(self.rnorm), int(bool(self.transposed)))
 
 
 @dataclass

@@ -454,3 +454,15 @@ def test_scalar_gain_and_row_norm_validation():
     arr = (ds.ds_wseg * 1)(wseg(rnorm=BASE + (5 << 30), radius=0.0))
     assert ds.lib().ds_gain_preserve(arr, 1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
     assert ds.ds_launch_count() == before
+
+
+def test_transposed_validation():
+    E = ds
+    before = ds.ds_launch_count()
+    # stored [cols, ld] with ld >= rows: rows 8, cols 4 -> ld 8 is fine, ld 4 is not
+    assert call_w("ds_wn_forward", [wseg(transposed=1, rows=8, cols=4, ld=4, ld_out=8)]) == E.DS_ERR_INVALID_ARG
+    assert call_w("ds_wn_forward", [wseg(transposed=1, rows=8, cols=4, ld=8, ld_out=4)]) == E.DS_ERR_INVALID_ARG
+    assert call_w("ds_wn_forward", [wseg(transposed=2)]) == E.DS_ERR_INVALID_ARG
+    arr = (ds.ds_wseg * 1)(wseg(transposed=1, rnorm=BASE + (5 << 30)))
+    assert ds.lib().ds_row_norms(arr, 1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
+    assert ds.ds_launch_count() == before

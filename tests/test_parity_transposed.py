@@ -1,0 +1,128 @@
+"""GPU parity of the weight calls on transposed rows (GPT-2's Conv1D keeps
+its weight as [in, out], so each unit row -- one output channel -- is a
+column of the stored matrix; DragonScale package description, "Supported
+layers").  Every result is compared, transposed back, with the float64
+oracle applied to the transposed matrix: the same definitions, row by row."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from l2_row_b200 import ds
+from l2_row_b200 import workloads as wl
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+# (stored rows = in, stored cols = out): GPT-2 small's Conv1D shapes, and
+# ragged ones (out not a multiple of 4; one output channel)
+SHAPES = [(768, 2304), (768, 768), (768, 3072), (3072, 768), (100, 13), (7, 1), (5, 6)]
+
+
+def _stored(rng, K, N, ld_pad=0):
+    """fp32 [K, N] rows drifted per output channel (column), in a padded
+    [K, N + pad] buffer; returns (host [K, N], device view)."""
+    w_t = wl.drifted_rows(rng, N, K, 0.02)            # [N, K]: one row per channel
+    host = np.ascontiguousarray(w_t.T)                 # stored [K, N]
+    ld = (N + 3) // 4 * 4 + ld_pad
+    dev, buf = gu.padded(K, N, ld, torch.float32, gu.CANARY_F32)
+    dev.copy_(gu.dev_f32(host))
+    return host, dev, buf, ld
+
+
+def _seg_t(w_host, g, gy_host, radius=1.0):
+    """The row-major (unit rows = output channels) view the oracle takes."""
+    return wl.WeightSeg("t", np.ascontiguousarray(w_host.T), g,
+                        None if gy_host is None else np.ascontiguousarray(gy_host.T), radius=radius)
+
+
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
+def test_forward(out_dtype):
+    rng = np.random.default_rng(91)
+    for K, N in SHAPES:
+        w, wd, _, ld = _stored(rng, K, N, ld_pad=4)
+        g = wl.gains(rng, N)
+        dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+        canary = gu.CANARY_BF16 if out_dtype == "bf16" else gu.CANARY_F32
+        ld_o = (N + 7) // 8 * 8 + 8          # rows of W_eff start on 16 bytes in either dtype
+        o, obuf = gu.padded(K, N, ld_o, dt, canary)
+        ds.ds_wn_forward([ds.WSeg(w=wd, gain=gu.dev_f32(g), w_eff=o, transposed=True)], out_dtype, 1e-6)
+        torch.cuda.synchronize()
+        assert gu.guards_intact(obuf, K, N, ld_o, canary), (K, N)
+        gu.check_forward(_seg_t(w, g, None), o.t().contiguous(), 1e-6, out_dtype, what=f"fwd [{K},{N}]")
+
+
+@pytest.mark.parametrize("gy_dtype", ["bf16", "f32"])
+def test_backward(gy_dtype):
+    rng = np.random.default_rng(92)
+    for K, N in SHAPES:
+        w, wd, _, ld = _stored(rng, K, N)
+        g = wl.gains(rng, N)
+        gy = rng.standard_normal((K, N)).astype(np.float32) * np.float32(1e-3)
+        if gy_dtype == "bf16":
+            gy = wl.to_bf16_bits(gy)
+        ld_g = (N + 7) // 8 * 8                # rows of GY start on 16 bytes
+        gyd, _ = gu.padded(K, N, ld_g, torch.bfloat16 if gy_dtype == "bf16" else torch.float32,
+                           gu.CANARY_BF16 if gy_dtype == "bf16" else gu.CANARY_F32)
+        gyd.copy_(gu.dev_bf16(gy) if gy_dtype == "bf16" else gu.dev_f32(gy))
+        gw, gwbuf = gu.padded(K, N, ld, torch.float32, gu.CANARY_F32)
+        gg = torch.empty(N, dtype=torch.float32, device="cuda")
+        ds.ds_wn_backward([ds.WSeg(w=wd, gain=gu.dev_f32(g), gy=gyd, grad_w=gw, grad_g=gg, transposed=True)],
+                          gy_dtype, 1e-6)
+        torch.cuda.synchronize()
+        assert gu.guards_intact(gwbuf, K, N, ld, gu.CANARY_F32), (K, N)
+        gu.check_backward(_seg_t(w, g, gy), gw.t().contiguous(), gg, 1e-6, what=f"bwd [{K},{N}]")
+
+
+def test_renorm_and_projections():
+    rng = np.random.default_rng(93)
+    for K, N in SHAPES:
+        w, wd, _, ld = _stored(rng, K, N)
+        G = rng.standard_normal((K, N)).astype(np.float32)
+        # renorm in place
+        ds.ds_row_renorm([ds.WSeg(w=wd, transposed=True)], 1e-6)
+        torch.cuda.synchronize()
+        gu.check_renorm(_seg_t(w, None, None), wd.t().contiguous(), 1e-6, what=f"renorm [{K},{N}]")
+        # gradient projection
+        w2, wd2, _, _ = _stored(rng, K, N)
+        Gd, _ = gu.padded(K, N, ld, torch.float32, gu.CANARY_F32)
+        Gd.copy_(gu.dev_f32(G))
+        ds.ds_grad_project([ds.WSeg(w=wd2, grad_w=Gd, transposed=True)], 1e-6)
+        torch.cuda.synchronize()
+        gu.check_project(_seg_t(w2, None, G), Gd.t().contiguous(), 1e-6, what=f"project [{K},{N}]")
+        # momentum projection + renorm
+        md, _ = gu.padded(K, N, ld, torch.float32, gu.CANARY_F32)
+        md.copy_(gu.dev_f32(G))
+        ds.ds_renorm_momentum([ds.WSeg(w=wd2, grad_w=md, transposed=True)], 1e-6)
+        torch.cuda.synchronize()
+        gu.check_momentum(_seg_t(w2, None, G), wd2.t().contiguous(), md.t().contiguous(), 1e-6,
+                          what=f"momentum [{K},{N}]")
+
+
+def test_mixed_table_and_scalar_gain():
+    """A table mixing normal and transposed segments in one call; a scalar
+    gain on a transposed segment."""
+    rng = np.random.default_rng(94)
+    K, N = 768, 2304
+    w, wd, _, _ = _stored(rng, K, N)
+    gy = wl.to_bf16_bits(rng.standard_normal((K, N)).astype(np.float32) * np.float32(1e-3))
+    row = wl.WeightSeg("r", wl.drifted_rows(rng, 64, 768, 0.02), wl.gains(rng, 64),
+                       wl.to_bf16_bits(rng.standard_normal((64, 768)).astype(np.float32)))
+    gs = torch.full((1,), 0.75, dtype=torch.float32, device="cuda")
+    gw_t = torch.empty(K, N, dtype=torch.float32, device="cuda")
+    gg_t = torch.empty(N + 1, dtype=torch.float32, device="cuda")
+    gw_r = torch.empty(64, 768, dtype=torch.float32, device="cuda")
+    gg_r = torch.empty(64, dtype=torch.float32, device="cuda")
+    before = ds.ds_launch_count()
+    ds.ds_wn_backward([ds.WSeg(w=gu.dev_f32(row.w), gain=gu.dev_f32(row.g), gy=gu.dev_bf16(row.gy), grad_w=gw_r,
+                               grad_g=gg_r),
+                       ds.WSeg(w=wd, gain=gs, gy=gu.dev_bf16(gy), grad_w=gw_t, grad_g=gg_t, transposed=True,
+                               gain_scalar=True)], "bf16", 1e-6)
+    torch.cuda.synchronize()
+    assert ds.ds_launch_count() - before == 3          # rows, transposed rows, the gain sum
+    gu.check_backward(row, gw_r, gg_r, 1e-6, what="row segment")
+    seg = _seg_t(w, np.full(N, 0.75, np.float32), gy)
+    gu.check_backward(seg, gw_t.t().contiguous(), gg_t[:N], 1e-6, what="transposed, scalar gain")
+    h = gu.host_f32(gg_t)
+    assert abs(float(h[N]) - float(np.sum(h[:N], dtype=np.float64))) <= np.spacing(np.float32(abs(h[N])))
