@@ -17,7 +17,7 @@ disjoint buffers (>= 268 MB of other traffic between two uses of one
 buffer), so inputs come from HBM without an explicit flush.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config step|mlp_pair|wide|optimizer|act_backward|dory]
+                    [--config step|mlp_pair|wide|optimizer|act_backward|dory|gain]
 
 `--config` selects another workload for a per-call report (default: the
 step above).  mlp_pair = up [2048,768] + down [768,2048] (fwd, bwd, renorm;
@@ -29,7 +29,9 @@ ds_renorm_momentum over the whole-model weights.  act_backward = the
 backward of the activation calls on [16384,4096] (upstream gradient bf16).
 dory = Dory's gated and SwiGLU l2 rows on [16384,4096] and [8192,7168]
 (scale vectors fp32 U(0.5, 2)) and its q/k rows on 16384 rows of 16 + 4 + 4
-heads of 256.
+heads of 256.  gain = the row lengths and the scalar-gain backward of the
+whole model, and forward + backward of 12 GPT-2 XL Conv1D weights
+[1600, 6400] stored [in, out] (transposed rows).
 
 Prints one JSON line (rank 0).  `value` is algorithmic bytes moved by all
 ranks per second (GB/s); per-kernel GB/s and rows/s, the roofline of the
@@ -75,6 +77,9 @@ WORKLOADS = {
                  "(fp32 gradient and momentum, in place)",
     "act_backward": "activation backward on rows [16384,4096] bf16: l2 (dx fp32), l2 with residual, slerp "
                     "(dres, dout fp32 and dalpha [4096] through its workspace)",
+    "gain": "row lengths (Monitor) and the scalar-gain backward (bf16 GY) of the whole-model weights (85 "
+            "segments, 100,073,472 fp32 elements); forward (bf16 W_eff) and backward (bf16 GY) of 12 GPT-2 XL "
+            "Conv1D weights [1600, 6400] stored [in, out] (transposed rows, 122,880,000 elements)",
     "dory": "Dory's fused activation rows: gated l2 rows (o, g bf16, sg fp32) and SwiGLU l2 rows (g, u bf16, "
             "sug, suu fp32) on [16384,4096] and [8192,7168]; q/k rows (rotate-half RoPE, per-head l2, q scale; "
             "16 q heads over 4 kv heads of 256, v copied to the cache) on 16384 rows, a third past position 199,800",
@@ -109,13 +114,21 @@ def call_bytes(kind: str, segs=None, act=None) -> int:
                 "slerpbwd": A * (2 + 2 + 2 + 4 + 4) + act.cols * (4 + 4),
                 "gate": A * (2 + 2 + 2) + act.cols * 4, "swiglu": A * (2 + 2 + 2) + act.cols * (4 + 4)}[kind]
     E = sum(s.w.size for s in segs)
-    R = sum(s.rows for s in segs)
+    R = sum(unit_rows(s) for s in segs)
     return {"fwd": E * (4 + 2) + R * 4, "bwd": E * (4 + 2 + 4) + R * (4 + 4), "renorm": E * (4 + 4),
-            "project": E * (4 + 4 + 4), "momentum": E * (4 + 4 + 4 + 4)}[kind]
+            "project": E * (4 + 4 + 4), "momentum": E * (4 + 4 + 4 + 4), "norms": E * 4 + R * 4,
+            # scalar gain: grad_w, the per-row parts, then their sum re-reads the parts
+            "bwd_scalar": E * (4 + 2 + 4) + R * (4 + 4) + len(segs) * 8}[kind]
+
+
+def unit_rows(s) -> int:
+    """Unit rows of a weight segment: its rows, or for a transposed
+    (Conv1D, stored [in, out]) segment its stored columns."""
+    return s.w.shape[1] if getattr(s, "transposed", False) else s.w.shape[0]
 
 
 def call_rows(kind: str, segs=None, act=None) -> int:
-    return act.rows if act is not None else sum(s.rows for s in segs)
+    return act.rows if act is not None else sum(unit_rows(s) for s in segs)
 
 
 def step_bytes(weights, act_rows=ACT_ROWS, act_cols=ACT_COLS) -> dict[str, int]:
@@ -168,6 +181,20 @@ def plan(config: str, seed: int):
         ag["qk"] = wl.qk_rows(seed, rows=QK_ROWS)
         calls.append(("qk_rows_l2", "qk", "qk"))
         return {}, ag, calls, 1
+    if config == "gain":
+        import types as _types
+
+        rng = np.random.default_rng(seed + 21)
+        conv = []
+        for layer in range(12):   # GPT-2 XL mlp c_fc: Conv1D(nf=6400, nx=1600) keeps weight [1600, 6400]
+            w = np.ascontiguousarray(wl.drifted_rows(rng, 6400, 1600, 0.02).T)
+            conv.append(_types.SimpleNamespace(name=f"c_fc{layer}", w=w, g=wl.gains(rng, 6400),
+                                               gy=wl.normal_bf16(rng, (1600, 6400), 1e-3), radius=1.0,
+                                               transposed=True, rows=1600, cols=6400))
+        wg = {"model": wl.whole_model(seed).weights, "conv1d": conv}
+        calls = [("row_norms", "norms", "model"), ("wn_backward_scalar_gain", "bwd_scalar", "model"),
+                 ("wn_forward_conv1d", "fwd", "conv1d"), ("wn_backward_conv1d", "bwd", "conv1d")]
+        return wg, {}, calls, 1
     if config == "optimizer":
         wg = {"model": wl.with_fp32_state(wl.whole_model(seed).weights, seed + 1)}
         calls = [("grad_project", "project", "model"), ("renorm_momentum", "momentum", "model")]
@@ -326,10 +353,14 @@ class Step:
                     b["gain"] = f32(host["gain"])
                 if "fwd" in kinds:
                     b["weff"] = torch.empty(n_el, dtype=torch.bfloat16, device=dev)
-                if "bwd" in kinds:
+                if kinds & {"bwd", "bwd_scalar"}:
                     b["gy"] = bf16(host["gy"])
                     b["grad_w"] = torch.empty(n_el, dtype=torch.float32, device=dev)
-                    b["grad_g"] = torch.empty(n_rows, dtype=torch.float32, device=dev)
+                    b["grad_g"] = torch.empty(n_rows + len(segs), dtype=torch.float32, device=dev)
+                if "bwd_scalar" in kinds:   # one gain per segment
+                    b["gscalar"] = torch.full((len(segs),), 0.5, dtype=torch.float32, device=dev)
+                if "norms" in kinds:
+                    b["rnorm"] = torch.empty(n_rows, dtype=torch.float32, device=dev)
                 if state:
                     b["state"] = f32(host["gy"])
                 copies.append(b)
@@ -342,7 +373,9 @@ class Step:
                 self.inputs.append((b0["gy"], host["gy"].view(np.int16)))
             if "state" in b0:
                 self.inputs.append((b0["state"], host["gy"]))
-            self.outputs += [b0[k] for k in ("weff", "grad_w", "grad_g", "state") if k in b0]
+            if "gscalar" in b0:
+                self.inputs.append((b0["gscalar"], np.full(len(segs), 0.5, np.float32)))
+            self.outputs += [b0[k] for k in ("weff", "grad_w", "grad_g", "state", "rnorm") if k in b0]
             if kinds & {"renorm", "momentum"}:
                 self.outputs.append(b0["w"])
         for name, a in self.ag.items():
@@ -419,27 +452,38 @@ class Step:
                     b, segs = self.wbuf[g][c], self.wg[g]
                     rows = []
                     eo = ro = 0
-                    for sgm in segs:
-                        R, C = sgm.rows, sgm.cols
+                    for si, sgm in enumerate(segs):
+                        R, C = sgm.w.shape          # as stored
+                        tr = bool(getattr(sgm, "transposed", False))
+                        U = unit_rows(sgm)
                         sl = slice(eo, eo + R * C)
                         w = b["w"][sl].view(R, C)
-                        gain = b["gain"][ro:ro + R] if "gain" in b else None
+                        gain = b["gain"][ro:ro + U] if "gain" in b else None
                         if kind == "fwd":
-                            rows.append(ds.WSeg(w=w, gain=gain, w_eff=b["weff"][sl].view(R, C)).to_c())
+                            rows.append(ds.WSeg(w=w, gain=gain, w_eff=b["weff"][sl].view(R, C), transposed=tr).to_c())
                         elif kind == "bwd":
                             rows.append(ds.WSeg(w=w, gain=gain, gy=b["gy"][sl].view(R, C),
                                                 grad_w=b["grad_w"][sl].view(R, C),
-                                                grad_g=b["grad_g"][ro:ro + R]).to_c())
+                                                grad_g=b["grad_g"][ro:ro + U], transposed=tr).to_c())
+                        elif kind == "bwd_scalar":   # grad_g: the parts then their sum, U + 1 per segment
+                            rows.append(ds.WSeg(w=w, gain=b["gscalar"][si:si + 1], gy=b["gy"][sl].view(R, C),
+                                                grad_w=b["grad_w"][sl].view(R, C),
+                                                grad_g=b["grad_g"][ro + si:ro + si + U + 1], radius=sgm.radius,
+                                                gain_scalar=True).to_c())
+                        elif kind == "norms":
+                            rows.append(ds.WSeg(w=w, rnorm=b["rnorm"][ro:ro + U]).to_c())
                         elif kind in ("project", "momentum"):
                             rows.append(ds.WSeg(w=w, grad_w=b["state"][sl].view(R, C), radius=sgm.radius).to_c())
                         else:
                             rows.append(ds.WSeg(w=w).to_c())
                         eo += R * C
-                        ro += R
+                        ro += U
                     tab = (ds.ds_wseg * len(rows))(*rows)
                     n = len(rows)
                     fn = {"fwd": lambda s, t=tab, n=n: lib.ds_wn_forward(t, n, ds.DS_BF16, eps, s),
                           "bwd": lambda s, t=tab, n=n: lib.ds_wn_backward(t, n, ds.DS_BF16, eps, s),
+                          "bwd_scalar": lambda s, t=tab, n=n: lib.ds_wn_backward(t, n, ds.DS_BF16, eps, s),
+                          "norms": lambda s, t=tab, n=n: lib.ds_row_norms(t, n, eps, s),
                           "renorm": lambda s, t=tab, n=n: lib.ds_row_renorm(t, n, eps, s),
                           "project": lambda s, t=tab, n=n: lib.ds_grad_project(t, n, eps, s),
                           "momentum": lambda s, t=tab, n=n: lib.ds_renorm_momentum(t, n, eps, s)}[kind]

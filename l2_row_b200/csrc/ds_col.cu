@@ -6,9 +6,11 @@
 // "Optimizer"), applied to those columns.
 //
 // One block owns a tile of kColTile consecutive unit rows (the stored
-// matrix's columns) over the whole row length.  Its 256 threads are 4 quads
-// (16 rows, 64 contiguous bytes of a stored row) by 64 lanes along the row;
-// a warp reads 8 stored rows x 64 bytes per step.  Pass 1 sums w^2 (and
+// matrix's columns) over the whole row length.  Its 256 threads are 8 quads
+// (32 rows, 128 contiguous bytes of a stored row) by 32 lanes along the row;
+// a warp reads 4 stored rows x 128 bytes per step, four steps in flight.
+// (Capping the grid at four blocks per SM, so that the tiles in flight fit
+// L2 for pass 2's re-read, measured slower: fewer bytes in flight.)  Pass 1 sums w^2 (and
 // w . d) per unit row in double -- no fp32 overflow or underflow is
 // possible, so no rescale path is needed -- and reduces the 64 lanes in a
 // fixed tree; pass 2 re-reads the tile (from L2) and writes each result as
@@ -22,7 +24,7 @@ namespace ds {
 
 namespace {
 
-constexpr int kColQuads = 4;                    // quads of unit rows per block
+constexpr int kColQuads = 8;                    // quads of unit rows per block
 constexpr int kColTile = 4 * kColQuads;         // unit rows per block
 constexpr int kColLanes = kCta / kColQuads;     // lanes along the row
 
@@ -87,6 +89,7 @@ __global__ void __launch_bounds__(kCta) k_col(const __grid_constant__ WParams p)
 
         double s[4] = {0, 0, 0, 0}, dd[4] = {0, 0, 0, 0};
         if (valid > 0) {
+#pragma unroll 4
             for (int j = ks; j < K; j += kColLanes) {
                 const float4 w = col_quad_f32(sg.w + j * sg.ld + r0);
                 float4 d = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -146,6 +149,7 @@ __global__ void __launch_bounds__(kCta) k_col(const __grid_constant__ WParams p)
                 if constexpr (TWO)
                     qt[i] = fac[1][4 * q + i];
             }
+#pragma unroll 4
             for (int j = ks; j < K; j += kColLanes) {
                 const float4 w = col_quad_f32(sg.w + j * sg.ld + r0);
                 float4 d = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -226,7 +226,8 @@ int tile_groups(int tag, int slot_bytes);
 constexpr int64_t kBuiltinScratchFloats = int64_t(16) << 20; // 64 MB
 int builtin_scratch(void **ptr, uint64_t *bytes);
 // dalpha[c] = sum over CTAs c0 < grid and their used teams q of
-// ws[(c0 * groups + q) * ws_ld + c], in that order (slerp backward).
+// ws[(c0 * groups + q) * ws_ld + c] (slerp backward), in a fixed order:
+// 32 interleaved partial sums over the lines, then a fixed tree.
 int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64_t total_units, int cols,
                          float *dalpha, void *stream);
 // Exhaustive check of the Dory rows' fast reciprocal and quotient (ds_tile.cu).

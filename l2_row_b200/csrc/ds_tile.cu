@@ -1662,23 +1662,37 @@ int tile_groups(int tag, int slot_bytes)
 
 namespace {
 
-// dalpha of the slerp backward: column c sums the used teams' lines, CTA by
-// CTA and team by team (a fixed order, so the result is deterministic).  A
-// CTA's team q was used iff it took a slot: q < the CTA's slot count.
-__global__ void __launch_bounds__(256) k_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups,
-                                                       int64_t total_units, int cols, float *dalpha)
+// dalpha of the slerp backward: the used teams' lines (line L = CTA *
+// groups + team; a CTA's team q was used iff q < the CTA's slot count) are
+// summed per column in a fixed order: thread row lg of a block adds lines
+// lg, lg + 32, ... in increasing order, then the 32 partial sums meet in a
+// fixed tree.  32 columns per block (one 128-byte segment of a line per
+// warp), so a 4,096-column alpha spreads over 128 blocks of 1,024 threads.
+__global__ void __launch_bounds__(1024) k_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups,
+                                                        int64_t total_units, int cols, float *dalpha)
 {
-    const int c = blockIdx.x * blockDim.x + threadIdx.x;
-    if (c >= cols)
-        return;
+    __shared__ float part[32][33];
+    const int cg = threadIdx.x & 31, lg = threadIdx.x >> 5;
+    const int c = blockIdx.x * 32 + cg;
     float acc = 0.f;
-    for (int cta = 0; cta < grid; ++cta) {
-        const int64_t mine = total_units > cta ? (total_units - 1 - cta) / grid + 1 : 0;
-        const int used = mine < groups ? static_cast<int>(mine) : groups;
-        for (int q = 0; q < used; ++q)
-            acc += ws[(static_cast<int64_t>(cta) * groups + q) * ws_ld + c];
+    if (c < cols) {
+        const int nlines = grid * groups;
+        for (int L = lg; L < nlines; L += 32) {
+            const int cta = L / groups, q = L - cta * groups;
+            const int64_t mine = total_units > cta ? (total_units - 1 - cta) / grid + 1 : 0;
+            if (q < mine)
+                acc += ws[static_cast<int64_t>(L) * ws_ld + c];
+        }
     }
-    dalpha[c] = acc;
+    part[lg][cg] = acc;
+    __syncthreads();
+    for (int o = 16; o > 0; o >>= 1) {
+        if (lg < o)
+            part[lg][cg] += part[lg + o][cg];
+        __syncthreads();
+    }
+    if (lg == 0 && c < cols)
+        dalpha[c] = part[0][cg];
 }
 
 } // namespace
@@ -1698,8 +1712,8 @@ int builtin_scratch(void **ptr, uint64_t *bytes)
 int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64_t total_units, int cols,
                          float *dalpha, void *stream)
 {
-    k_dalpha_reduce<<<(cols + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(ws, ws_ld, grid, groups,
-                                                                                    total_units, cols, dalpha);
+    k_dalpha_reduce<<<(cols + 31) / 32, 1024, 0, static_cast<cudaStream_t>(stream)>>>(ws, ws_ld, grid, groups,
+                                                                                   total_units, cols, dalpha);
     return cudaGetLastError();
 }
 
