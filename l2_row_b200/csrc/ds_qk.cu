@@ -262,19 +262,24 @@ __device__ __forceinline__ IterGeom iter_geom(const QKParams &p, int64_t u)
 
 // A block iteration's warps load their tasks' octets straight from global
 // memory (up to kQkTasks per warp at once) while the table is computed.
+// The table is double-buffered: iteration k writes buffer k % 2, whose last
+// readers (iteration k - 2) all passed iteration k - 1's barrier, so one
+// barrier per iteration (table written) is enough.
 template <int D>
 __global__ void __launch_bounds__(kQkThreads, 3) k_qk(const __grid_constant__ QKParams p)
 {
     constexpr int H2 = D / 2, L = D / 16;
-    __shared__ __align__(16) float s_cos[kQkTable];
-    __shared__ __align__(16) float s_sin[kQkTable];
+    __shared__ __align__(16) float s_cos2[2][kQkTable];
+    __shared__ __align__(16) float s_sin2[2][kQkTable];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int j = lane & (L - 1), lane_head = lane / L;
     const int64_t total = p.unit_start[p.nseg];
 
-    for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
+    int parity = 0;
+    for (int64_t u = blockIdx.x; u < total; u += gridDim.x, parity ^= 1) {
         const IterGeom g = iter_geom<D>(p, u);
         const QKSegK &sg = p.seg[g.seg];
+        float *s_cos = s_cos2[parity], *s_sin = s_sin2[parity];
         for (int base = 0; base < g.ntask; base += kQkWarps * kQkTasks) {
             uint4 xa[kQkTasks], xb[kQkTasks];
             TaskWalk wk;
@@ -310,7 +315,6 @@ __global__ void __launch_bounds__(kQkThreads, 3) k_qk(const __grid_constant__ QK
                 w0.step(g.tpr);
             }
         }
-        __syncthreads(); // the next iteration rewrites the table
     }
 }
 
