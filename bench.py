@@ -638,7 +638,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                    "frac_of_peak": round(fb_b / fb_t / 1e9 / peak, 4)}
     dom = max(names, key=lambda n: call_ms[n])
     ach = bytes_per[dom] / (call_ms[dom] * 1e-3) / 1e9
-    traffic = recorded_traffic(dom) if args.config == "step" else None
+    traffic = recorded_traffic(f"ds_{dom}") if args.config == "step" else None
     roofline = {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(ach / peak, 4), "traffic": traffic, "kernel": f"ds_{dom}",
                 "algorithmic_bytes": bytes_per[dom], "peak_source": peak_src}
