@@ -1,0 +1,49 @@
+"""Host-side checks of the benchmark's workload plans (no GPU): every
+configuration names known call kinds, its algorithmic bytes follow the
+per-element figures of the design table, and the step's bytes are the
+documented 3,476,900,864."""
+from __future__ import annotations
+
+import pytest
+
+import bench
+
+KINDS = {"fwd", "bwd", "renorm", "project", "momentum", "norms", "bwd_scalar", "l2", "l2res", "slerp", "l2bwd",
+         "l2resbwd", "slerpbwd", "gate", "swiglu", "qk"}
+
+
+@pytest.mark.parametrize("config", sorted(bench.WORKLOADS))
+def test_plans_are_well_formed(config):
+    wg, ag, calls, copies = bench.plan(config, 0)
+    assert copies >= 1 and calls
+    names = [c[0] for c in calls]
+    assert len(set(names)) == len(names)
+    for name, kind, group in calls:
+        assert kind in KINDS, kind
+        assert (group in wg) != (group in ag), group
+        segs, act = (wg[group], None) if group in wg else (None, ag[group])
+        b = bench.call_bytes(kind, segs, act)
+        r = bench.call_rows(kind, segs, act)
+        assert b > 0 and r > 0
+
+
+def test_step_bytes_and_per_element_figures():
+    wg, ag, calls, _ = bench.plan("step", 0)
+    segs, act = wg["model"], ag["x"]
+    E = sum(s.w.size for s in segs)
+    R = sum(s.rows for s in segs)
+    assert (E, R) == (100_073_472, 114_944)
+    got = {name: bench.call_bytes(kind, segs if group in wg else None, None if group in wg else act)
+           for name, kind, group in calls}
+    A = 16384 * 4096
+    assert got == {"wn_forward": E * 6 + R * 4, "l2_rows": A * 4, "wn_backward": E * 10 + R * 8,
+                   "l2_rows_residual": A * 6, "row_renorm": E * 8, "slerp_rows": A * 6 + 4096 * 4}
+    assert sum(got.values()) == 3_476_900_864
+
+
+def test_transposed_rows_count_output_channels():
+    wg, _, calls, _ = bench.plan("gain", 0)
+    conv = wg["conv1d"]
+    assert all(s.w.shape == (1600, 6400) and s.transposed for s in conv)
+    assert bench.call_rows("fwd", conv) == 12 * 6400          # unit rows = the stored columns
+    assert bench.call_bytes("fwd", conv) == 12 * 1600 * 6400 * 6 + 12 * 6400 * 4
