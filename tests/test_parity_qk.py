@@ -183,3 +183,24 @@ def test_sampled_rows_at_bench_size():
     rows = gu.sample_rows(16384, 48, 47, must=(0, 16383, 10922, 10923))
     check(w, qo, kc, rows=rows, what="bench size")
     assert np.array_equal(vc, w.v)
+
+
+def test_segments_of_several_head_sizes_in_one_call():
+    """A table mixing head sizes runs one launch per head size; every
+    segment matches the oracle."""
+    ws = [wl.qk_rows(50 + i, rows=r, head_dim=D, hq=hq, hk=hk)
+          for i, (r, D, hq, hk) in enumerate([(9, 64, 4, 2), (5, 256, 2, 1), (7, 64, 2, 2), (3, 128, 1, 1)])]
+    segs, outs = [], []
+    for w in ws:
+        q, k, v = gu.dev_bf16(w.q), gu.dev_bf16(w.k), gu.dev_bf16(w.v)
+        qo, kc, vc = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        segs.append(ds.QKSeg(head_dim=w.head_dim, pos=_dev_i32(w.pos), inv_freq=gu.dev_f32(w.inv), q=q, q_out=qo,
+                             k=k, k_cache=kc, v=v, v_cache=vc, q_scale=gu.dev_f32(w.q_scale)))
+        outs.append((qo, kc, vc))
+    before = ds.ds_launch_count()
+    ds.ds_qk_rows_l2(segs)
+    torch.cuda.synchronize()
+    assert ds.ds_launch_count() - before == 3          # head sizes 64, 128, 256
+    for w, (qo, kc, vc) in zip(ws, outs):
+        check(w, gu.host_bits(qo), gu.host_bits(kc), what=f"D={w.head_dim}")
+        assert np.array_equal(gu.host_bits(vc), w.v)
