@@ -466,3 +466,24 @@ def test_transposed_validation():
     arr = (ds.ds_wseg * 1)(wseg(transposed=1, rnorm=BASE + (5 << 30)))
     assert ds.lib().ds_row_norms(arr, 1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
     assert ds.ds_launch_count() == before
+
+
+def test_python_segments_map_shapes():
+    """The binding's segment builders: a transposed weight gives rows = its
+    stored columns; q/k segments count heads from the widths and refuse a
+    width that is not whole heads.  (Host memory only: nothing is launched.)"""
+    import torch
+
+    w = torch.zeros(6, 10)                       # stored [in = 6, out = 10]
+    c = ds.WSeg(w=w, transposed=True).to_c()
+    assert (c.rows, c.cols, c.ld, c.transposed) == (10, 6, 10, 1)
+    c = ds.WSeg(w=w).to_c()
+    assert (c.rows, c.cols, c.transposed) == (6, 10, 0)
+    q = torch.zeros(3, 4 * 64, dtype=torch.bfloat16)
+    k = torch.zeros(3, 2 * 64, dtype=torch.bfloat16)
+    pos = torch.zeros(3, dtype=torch.int32)
+    inv = torch.zeros(32)
+    c = ds.QKSeg(head_dim=64, pos=pos, inv_freq=inv, q=q, q_out=q, k=k, k_cache=k).to_c()
+    assert (c.rows, c.hq, c.hk, c.head_dim, c.ld_q, c.ld_kv, c.cache_rows) == (3, 4, 2, 64, 256, 128, 3)
+    with pytest.raises(ValueError):
+        ds.QKSeg(head_dim=64, pos=pos, inv_freq=inv, q=torch.zeros(3, 100, dtype=torch.bfloat16)).to_c()
