@@ -323,7 +323,7 @@ def test_interval_forms_bracket_point_forms():
 def test_controls_escape_the_sharp_interval():
     """Each control drops one rounding point or moves eps.  Within 1 ulp it can
     hide (dropping a rounding point moves a result by at most ~half an ulp), so
-    the controls are judged by the interval check: on the control inputs each
+    the controls are decided by the interval check: on the control inputs each
     must put at least one row outside the definition's interval."""
     act = wl.activations(0, rows=256, cols=4096).acts[0]
     lo, hi = oracle.l2_rows_interval(act.x, act.r, delta=SPREAD)
