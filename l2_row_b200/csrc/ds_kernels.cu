@@ -1033,7 +1033,6 @@ cudaError_t launch_clustered(K kernel, const P &p, int64_t rows, int cluster, si
 template <int T>
 cudaError_t launch_op(const RowClass &rc, const ParamsOf<T> &p, int64_t units, void *stream)
 {
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     switch (rc.path) {
     case DS_PATH_CLUSTER:
         return launch_clustered(k_cluster<T>, p, units, rc.cluster, 0, stream);
