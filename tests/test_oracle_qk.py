@@ -146,3 +146,24 @@ def test_threads_do_not_change_results():
     a = oracle.qk_rows_l2(w.q, w.k, w.pos, w.inv, w.q_scale, head_dim=D, nthreads=1)
     b = oracle.qk_rows_l2(w.q, w.k, w.pos, w.inv, w.q_scale, head_dim=D, nthreads=7)
     assert all(np.array_equal(x, y) for x, y in zip(a, b))
+
+
+def test_intervals_contain_points_at_extremes():
+    """Heads of huge, tiny and mixed magnitudes, zero heads, and positions
+    up to 2^24 (angles far past 2 pi): the interval still holds the point."""
+    rng = np.random.default_rng(12)
+    D, R = 64, 6
+    inv = wl.rope_inv(D)
+    pos = np.array([0, 1, 199_800, 1 << 20, (1 << 24) - 1, 12345], np.int32)
+    for scale in (1e30, 1e-30, 1.0):
+        x = (rng.standard_normal((R, 2 * D)) * scale).astype(np.float32)
+        x[1, :D] = 0.0                                   # one zero head
+        q = wl.to_bf16_bits(x)
+        k = wl.to_bf16_bits((rng.standard_normal((R, D)) * scale).astype(np.float32))
+        for eps in (1e-6, 0.0):
+            qo, ko = oracle.qk_rows_l2(q, k, pos, inv, head_dim=D, eps=eps)
+            ql, qh, kl, kh = oracle.qk_rows_l2_interval(q, k, pos, inv, head_dim=D, eps=eps)
+            fin = ~np.isnan(wl.bf16_bits_to_f32(qo))
+            assert not bf16_interval_violations(qo[fin], ql[fin], qh[fin]).any(), (scale, eps)
+            fin = ~np.isnan(wl.bf16_bits_to_f32(ko))
+            assert not bf16_interval_violations(ko[fin], kl[fin], kh[fin]).any(), (scale, eps)
