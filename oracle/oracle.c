@@ -426,6 +426,17 @@ static double swiglu_value(double g, double u, double sug, double suu,
     return (flags & OR_DROP_PRODUCT) ? v : round_bf16(v);
 }
 
+/* The sigmoid, silu and per-element values above, exported so that the
+ * tests can pin them at interior points against independent identities
+ * (they are otherwise reachable only through a row's norm). */
+double or_sigmoid(double z) { return sigmoid64(z); }
+double or_silu(double x) { return silu64(x); }
+double or_gate_value(double o, double g, double sg, unsigned flags) { return gate_value(o, g, sg, flags); }
+double or_swiglu_value(double g, double u, double sug, double suu, unsigned flags)
+{
+    return swiglu_value(g, u, sug, suu, flags);
+}
+
 /* y = bf16(s / sqrt(sum s^2 + eps)) for a row whose s is already formed. */
 static void l2_of(const double *s, int64_t C, double eps, unsigned flags,
                   uint16_t *y, double *y_exact)

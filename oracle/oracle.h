@@ -51,6 +51,14 @@ extern "C" {
 /* bf16 helpers.  or_bf16_rne rounds a double straight to bf16 bits. */
 uint16_t or_bf16_rne(double v);
 double   or_bf16_value(uint16_t bits);
+
+/* [TF] Dory rows, one element: sigmoid(z) = 1/(1+exp(-z)), silu(x) =
+ * x/(1+exp(-x)), the gated value bf16(o sigmoid(g sg)) and the SwiGLU value
+ * bf16(silu(bf16(g sug)) bf16(u suu)) (flags drop their rounding points). */
+double or_sigmoid(double z);
+double or_silu(double x);
+double or_gate_value(double o, double g, double sg, unsigned flags);
+double or_swiglu_value(double g, double u, double sug, double suu, unsigned flags);
 /* or_bf16_rne over an array (dst[i] = or_bf16_rne(src[i])). */
 void     or_bf16_rne_array(const double *src, int64_t n, uint16_t *dst);
 

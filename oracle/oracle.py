@@ -38,6 +38,13 @@ def lib() -> ct.CDLL:
         _lib.or_bf16_value.argtypes = [ct.c_uint16]
         _lib.or_bf16_value.restype = dbl
         _lib.or_bf16_rne_array.argtypes = [vp, i64, vp]
+        for name, n in (("or_sigmoid", 1), ("or_silu", 1)):
+            getattr(_lib, name).argtypes = [dbl] * n
+            getattr(_lib, name).restype = dbl
+        _lib.or_gate_value.argtypes = [dbl, dbl, dbl, uns]
+        _lib.or_gate_value.restype = dbl
+        _lib.or_swiglu_value.argtypes = [dbl, dbl, dbl, dbl, uns]
+        _lib.or_swiglu_value.restype = dbl
         _lib.or_bf16_rne_array.restype = None
         _lib.or_wn_forward.argtypes = [vp, i64, i64, i64, vp, dbl, dbl, uns, vp, i32]
         _lib.or_wn_backward.argtypes = [vp, i64, i64, i64, vp, i32, i64, vp, dbl, dbl, uns, vp, vp, i32]
@@ -121,6 +128,26 @@ def bf16_rne_array(a) -> np.ndarray:
 
 def bf16_value(bits: int) -> float:
     return float(lib().or_bf16_value(int(bits) & 0xFFFF))
+
+
+def sigmoid(z: float) -> float:
+    """The oracle's sigmoid, 1/(1+exp(-z)) in double."""
+    return lib().or_sigmoid(float(z))
+
+
+def silu(x: float) -> float:
+    """The oracle's silu, x/(1+exp(-x)) in double."""
+    return lib().or_silu(float(x))
+
+
+def gate_value(o: float, g: float, sg: float, flags: int = 0) -> float:
+    """One element of the gated row: bf16(o sigmoid(g sg)) (OR_DROP_GATED: unrounded)."""
+    return lib().or_gate_value(float(o), float(g), float(sg), flags)
+
+
+def swiglu_value(g: float, u: float, sug: float, suu: float, flags: int = 0) -> float:
+    """One element of the SwiGLU row: bf16(silu(bf16(g sug)) bf16(u suu))."""
+    return lib().or_swiglu_value(float(g), float(u), float(sug), float(suu), flags)
 
 
 def wn_forward(w, g=None, *, rho=1.0, eps=1e-6, flags=0, nthreads=1):

@@ -119,3 +119,68 @@ def test_threads_do_not_change_results():
     assert np.array_equal(oracle.gate_l2_rows(a, b, s, nthreads=1), oracle.gate_l2_rows(a, b, s, nthreads=6))
     assert np.array_equal(oracle.swiglu_l2_rows(a, b, s, s, nthreads=1),
                           oracle.swiglu_l2_rows(a, b, s, s, nthreads=5))
+
+
+# ---------------------------------------------------- interior pins -----
+#
+# sigmoid and silu across the range the Dory rows use, against identities
+# evaluated independently with Python's math module: sigmoid(z) =
+# (1 + tanh(z/2)) / 2, sigmoid(z) + sigmoid(-z) = 1, silu(x) = x sigmoid(x).
+# A wrong sign in exp, a dropped 1 or a swapped numerator fails them.
+
+import math  # noqa: E402
+
+Z = np.concatenate([np.linspace(-20.0, 20.0, 4001), np.random.default_rng(131).uniform(-20, 20, 2000),
+                    [-1.2784645427610738, -1e-300, 0.0, 1e-300]])
+
+
+def _sig_ref(z: float) -> float:
+    """sigmoid by Python's math: (1 + tanh(z/2)) / 2 where it does not cancel
+    (z >= 0), else e^z / (1 + e^z)."""
+    if z >= 0:
+        return 0.5 * (1.0 + math.tanh(0.5 * z))
+    return math.exp(z) / (1.0 + math.exp(z))
+
+
+def test_sigmoid_interior_matches_tanh_identity():
+    for z in Z:
+        s, ref = oracle.sigmoid(z), _sig_ref(z)
+        assert abs(s - ref) <= 4.5e-16 * ref, (z, s, ref)
+        assert abs(s + oracle.sigmoid(-z) - 1.0) <= 2.3e-16, z
+    assert oracle.sigmoid(0.0) == 0.5
+
+
+def test_silu_interior_is_x_times_sigmoid():
+    for x in Z:
+        ref = x * _sig_ref(x)
+        assert abs(oracle.silu(x) - ref) <= 6e-16 * abs(ref) + 1e-300, (x, oracle.silu(x), ref)
+    # silu's minimum near x0 = -1.27846...: silu'(x0) = 0, value -0.27846...
+    x0 = -1.2784645427610738
+    assert abs(oracle.silu(x0) - (-0.2784645427610738)) < 1e-15
+    assert oracle.silu(x0 - 1e-4) > oracle.silu(x0) < oracle.silu(x0 + 1e-4)
+
+
+def test_gate_and_swiglu_values_at_interior_points():
+    """One element of each row: the unrounded values are o sigmoid(g sg) and
+    silu(g sug) u suu, and the rounded ones their nearest bf16 (every
+    rounding point applied)."""
+    rng = np.random.default_rng(132)
+    o = wl.bf16_bits_to_f32(wl.normal_bf16(rng, (500,))).astype(np.float64)
+    g = wl.bf16_bits_to_f32(wl.normal_bf16(rng, (500,), 4.0)).astype(np.float64)
+    s = rng.uniform(0.5, 2.0, 500).astype(np.float32).astype(np.float64)
+    u = wl.bf16_bits_to_f32(wl.normal_bf16(rng, (500,))).astype(np.float64)
+    s2 = rng.uniform(0.5, 2.0, 500).astype(np.float32).astype(np.float64)
+    for i in range(500):
+        v = o[i] * _sig_ref(g[i] * s[i])
+        assert abs(oracle.gate_value(o[i], g[i], s[i], oracle.OR_DROP_GATED) - v) <= 1e-15 * abs(v) + 1e-300
+        assert oracle.gate_value(o[i], g[i], s[i]) == oracle.bf16_value(oracle.bf16_rne(v)) or \
+            abs(v * 256 / 2 ** math.floor(math.log2(abs(v))) % 1 - 0.5) < 1e-9
+        flags = oracle.OR_DROP_SGATE | oracle.OR_DROP_SUP | oracle.OR_DROP_PRODUCT
+        gs, us = g[i] * s[i], u[i] * s2[i]
+        w = gs * _sig_ref(gs) * us
+        assert abs(oracle.swiglu_value(g[i], u[i], s[i], s2[i], flags) - w) <= 2e-15 * abs(w) + 1e-300
+        gs_b = oracle.bf16_value(oracle.bf16_rne(gs))
+        us_b = oracle.bf16_value(oracle.bf16_rne(us))
+        wr = gs_b * _sig_ref(gs_b) * us_b
+        assert oracle.swiglu_value(g[i], u[i], s[i], s2[i]) == oracle.bf16_value(oracle.bf16_rne(wr)) or \
+            abs(wr * 256 / 2 ** math.floor(math.log2(abs(wr))) % 1 - 0.5) < 1e-9
