@@ -323,13 +323,30 @@ ds_status ds_slerp_rows_backward(const ds_agseg *segs, int nseg, float eps,
  * `cols` elements on the current device (0 if cols < 1). */
 uint64_t ds_slerp_rows_backward_workspace(int64_t cols);
 
-/* ds_slerp_rows_backward without a caller workspace: dalpha's partial sums go
- * to a scratch array built into the library (one static device array per
- * device, 64 MB: rows up to 8,712 columns on a 148-SM B200; wider rows are
- * refused with DS_ERR_INVALID_ARG).  The scratch is shared, so calls of this
- * entry point must not overlap in time (use one stream, or synchronise).
+/* ds_slerp_rows_backward for callers that cannot allocate device memory
+ * where they run the backward: a runtime that hands all device memory to its
+ * own pool at start-up and forbids later cudaMalloc calls, or code that must
+ * not risk the implicit device-wide synchronisation cudaMalloc and cudaFree
+ * may cause.  Such a caller cannot provide the workspace of
+ * ds_slerp_rows_backward, so this entry point allocates nothing: dalpha's
+ * per-team partial sums go to a static device array built into the library
+ * (64 MB, held on every device that loads the library until the process
+ * exits).  Inputs and outputs are still the caller's, as for
+ * ds_slerp_rows_backward.
+ *   - Limit: the partial sums of rows of cols columns take
+ *     ds_slerp_rows_backward_workspace(cols) bytes; rows that need more than
+ *     64 MB (more than 8,712 columns on a 148-SM B200) are refused with
+ *     DS_ERR_INVALID_ARG and a message in ds_last_error.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (a host-side runtime query, with that device current) and
+ *     caches it; make that first call before any stream capture.
+ *   - Sharing: every call of this entry point, on any stream, uses the same
+ *     array, so calls that overlap on the GPU race and give wrong dalpha; use
+ *     one stream or synchronise between calls.  Nothing in the array needs to
+ *     start at zero (each call overwrites every partial sum it reads), so a
+ *     previous call's leftover contents do no harm.
  * Results are bitwise those of ds_slerp_rows_backward.  The pages have no
- * counterpart: this is a convenience entry point of this library. */
+ * counterpart: this entry point is this library's own. */
 ds_status ds_slerp_rows_backward_noalloc(const ds_agseg *segs, int nseg, float eps,
                                          float *dalpha, ds_stream stream);
 

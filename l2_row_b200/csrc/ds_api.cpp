@@ -1141,8 +1141,23 @@ ds_status ds_slerp_rows_backward_noalloc(const ds_agseg *segs, int nseg, float e
     void *ws = nullptr;
     uint64_t bytes = 0;
     if (dalpha) {
-        if (ds::builtin_scratch(&ws, &bytes) != 0)
-            return fail(DS_ERR_CUDA, "built-in scratch not available");
+        g_last_error.clear();
+        if (nseg > 0 && segs && segs[0].cols >= 1 && segs[0].cols <= kMaxCols &&
+            dalpha_ws_bytes(segs[0].cols) > static_cast<uint64_t>(ds::kBuiltinScratchFloats) * 4u) {
+            char buf[200];
+            std::snprintf(buf, sizeof(buf),
+                          "rows of %lld columns need %llu bytes of dalpha scratch; the built-in scratch holds %llu "
+                          "(use ds_slerp_rows_backward with a workspace)",
+                          static_cast<long long>(segs[0].cols),
+                          static_cast<unsigned long long>(dalpha_ws_bytes(segs[0].cols)),
+                          static_cast<unsigned long long>(ds::kBuiltinScratchFloats) * 4u);
+            return fail(DS_ERR_INVALID_ARG, buf);
+        }
+        if (const int e = ds::builtin_scratch(&ws, &bytes)) {
+            char buf[96];
+            std::snprintf(buf, sizeof(buf), "built-in scratch address lookup failed (cudaError %d)", e);
+            return fail(DS_ERR_CUDA, buf);
+        }
     }
     return run_act_bwd(true, segs, nseg, eps, dalpha, ws, bytes, stream);
 }

@@ -42,6 +42,24 @@ static inline int module_read_and_clear_error(uint32_t *code, uint32_t *site)
     return cudaSuccess;
 }
 
+// Kernels with more than 48 KB of dynamic shared memory must opt in, per
+// device: the attribute is set the first time the kernel launches with each
+// device current (a process may drive several GPUs).
+template <class K>
+inline cudaError_t enable_dynamic_smem(K kernel, int bytes, DeviceFlags &done)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (done.has(dev))
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        done.set(dev);
+    return e;
+}
+
 // ---------------------------------------------------------------- memory --
 
 // Streaming 16-byte load through the read-only path.  Safe with the exact

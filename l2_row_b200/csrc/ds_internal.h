@@ -2,6 +2,7 @@
 // sm_100a kernels (ds_kernels.cu).  Not part of the public ABI.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 
 #include "ds.h"
@@ -13,6 +14,23 @@
 #endif
 
 namespace ds {
+
+// A one-time host step per device (a kernel attribute, a symbol address):
+// one bit per device id 0..63, set once the step succeeded with that device
+// current.  Devices past 63 are never marked, so their callers redo the step
+// on every call, which is correct, only slower.
+struct DeviceFlags {
+    std::atomic<uint64_t> bits{0};
+    bool has(int dev) const
+    {
+        return dev >= 0 && dev < 64 && ((bits.load(std::memory_order_acquire) >> dev) & 1u) != 0;
+    }
+    void set(int dev)
+    {
+        if (dev >= 0 && dev < 64)
+            bits.fetch_or(uint64_t(1) << dev, std::memory_order_release);
+    }
+};
 
 // Every kernel runs 256-thread CTAs.
 constexpr int kCta = 256;

@@ -1038,13 +1038,9 @@ cudaError_t launch_op(const RowClass &rc, const ParamsOf<T> &p, int64_t units, v
         return launch_clustered(k_cluster<T>, p, units, rc.cluster, 0, stream);
     case DS_PATH_TWO_PASS: {
         constexpr int smem = kStages * stream_stage_bytes<T>();
-        static bool attr_set = false; // benign race: idempotent
-        if (!attr_set) {
-            cudaError_t e = cudaFuncSetAttribute(k_stream<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-            if (e != cudaSuccess)
-                return e;
-            attr_set = true;
-        }
+        static DeviceFlags attr_set;
+        if (const cudaError_t e = enable_dynamic_smem(k_stream<T>, smem, attr_set))
+            return e;
         return launch_clustered(k_stream<T>, p, units, rc.cluster, smem, stream);
     }
     default:

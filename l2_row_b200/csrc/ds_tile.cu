@@ -1578,13 +1578,9 @@ static cudaError_t launch_tile_sb(const TParams<T> &p, int grid, void *stream)
 {
     using Cfg = TileCfg<T, SB>;
     constexpr int smem = Cfg::kSmem;
-    static bool attr_set = false; // benign race: idempotent
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_tile<T, SB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    static DeviceFlags attr_set;
+    if (const cudaError_t e = enable_dynamic_smem(k_tile<T, SB>, smem, attr_set))
+        return e;
     k_tile<T, SB><<<grid, Cfg::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError();
 }
@@ -1699,14 +1695,36 @@ __global__ void __launch_bounds__(1024) k_dalpha_reduce(const float *ws, int ws_
 
 // Built-in scratch for the no-alloc slerp backward entry point: one
 // module-level device array (64 MB, enough for the dalpha lines of rows up to
-// 8,712 columns on 148 SMs).  Calls that use it must not overlap in time.
+// 8,712 columns on 148 SMs), present on every device that loads the library
+// until the process exits.  Host code cannot use the array's name as a
+// device address, so its address is looked up once per device, with that
+// device current, and cached.  Calls that use it must not overlap in time.
 static __device__ __align__(256) float g_builtin_scratch[kBuiltinScratchFloats];
 
 int builtin_scratch(void **ptr, uint64_t *bytes)
 {
-    const cudaError_t e = cudaGetSymbolAddress(ptr, g_builtin_scratch);
+    static DeviceFlags looked_up;
+    static void *addr[64] = {};
+    *ptr = nullptr;
     *bytes = static_cast<uint64_t>(kBuiltinScratchFloats) * sizeof(float);
-    return e;
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (looked_up.has(dev)) {
+        *ptr = addr[dev];
+        return cudaSuccess;
+    }
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_builtin_scratch);
+    if (e != cudaSuccess)
+        return e;
+    if (dev >= 0 && dev < 64) {
+        addr[dev] = p;     // written before the flag is published
+        looked_up.set(dev);
+    }
+    *ptr = p;
+    return cudaSuccess;
 }
 
 int launch_dalpha_reduce(const float *ws, int ws_ld, int grid, int groups, int64_t total_units, int cols,

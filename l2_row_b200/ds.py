@@ -454,7 +454,12 @@ def ds_slerp_rows_backward(segs: Sequence, eps: float = 1e-6, dalpha=None, works
 
 
 def ds_slerp_rows_backward_noalloc(segs: Sequence, eps: float = 1e-6, dalpha=None, stream=None) -> None:
-    """ds_slerp_rows_backward with the library's built-in scratch (no workspace)."""
+    """ds_slerp_rows_backward for callers that cannot allocate device memory
+    where they run the backward (their device memory all belongs to a pool
+    of their own, or they must avoid the implicit synchronisation of
+    cudaMalloc / cudaFree): dalpha's partial sums go to the library's
+    built-in 64 MB scratch instead of a workspace.  Rows needing more than
+    that are refused; calls must not overlap on the GPU."""
     arr, n = _table(segs, ds_agseg)
     _check(_lib.ds_slerp_rows_backward_noalloc(arr, n, eps, _vec(dalpha), _stream_ptr(stream)),
            "ds_slerp_rows_backward_noalloc")

@@ -11,9 +11,9 @@ forward's value, and one bf16 step of a_j or b_j moves t_j, dt_j and the row's
 dalpha part at that column by about 2^-8 of their size.  So: exactly
 representable rows (+-1 entries, 4^k columns, eps = 0, where a and b are
 exact) are checked at 1e-5 everywhere, dalpha included.  Random rows are
-checked at 1e-5 plus the bounded effect of each flagged rounding: locally (the
-flagged element itself within 2e-2) and on its row, through the row's sum of
-squares (a common factor 1/nt) and t . dh; dalpha per column likewise.
+checked at 1e-5 plus the bounded effect of each flagged rounding: on its row
+through the row's sum of squares (a common factor 1/nt) and t . dh, and at
+the flagged column through its own dt_j; dalpha per column likewise.
 """
 from __future__ import annotations
 
@@ -101,14 +101,19 @@ def check_slerp_bwd(res, out, alpha, dh, got, eps, strict, what=""):
     dDt = (dtj * np.abs(d64)).sum(1)
     rowrel = 2 * dSt / (2 * St)
     rowabs = 2 * np.abs(t) * ((dDt + np.abs(Dt) * dSt / St) / St * it)[:, None]
+    # At the flagged column itself the flip also moves dt_j = (dh_j - t_j Dt/nt^2)/nt
+    # by dt_j's share of it, |delta t_j| |Dt| / nt^3, and with it da_j, db_j and
+    # dres_j, dout_j (divided by na, nb; the factors (1 - |alpha|), |alpha| are
+    # at most 1); margin 2 on top of dtj, itself an upper bound of the step.
+    local = 2 * dtj * (np.abs(Dt) * it ** 3)[:, None]
     for got_x, ref_x, nrm, name in ((dres, rr, na, "dres"), (dout, ro, nb, "dout")):
         floor = (g / nrm)[:, None]
-        allowed = 1e-5 * np.maximum(np.abs(ref_x), floor) + rowrel[:, None] * np.abs(ref_x) + rowabs / nrm[:, None]
+        allowed = 1e-5 * np.maximum(np.abs(ref_x), floor) + rowrel[:, None] * np.abs(ref_x) + rowabs / nrm[:, None] \
+            + local / nrm[:, None]
         diff = np.abs(got_x - ref_x)
-        bad = (diff > allowed) & ~flag
-        assert not bad.any(), f"{what}: {int(bad.sum())} {name} entries beyond tolerance (first {np.argwhere(bad)[0]})"
-        loose = rel_violations(got_x, ref_x, 2e-2, floor)
-        assert not loose.any(), f"{what}: {int(loose.sum())} {name} entries beyond 2e-2"
+        bad = ~(diff <= allowed) & ~(np.isnan(got_x) & np.isnan(ref_x))
+        assert not bad.any(), f"{what}: {int(bad.sum())} {name} entries beyond tolerance (first {np.argwhere(bad)[0]}, " \
+                              f"flagged {int(flag.sum())})"
     if da is not None:
         # dalpha_j sums the rows' sign(alpha_j) (b_j - a_j) dt_j.  Each part
         # carries fp32 error of order 1e-5 |b_j - a_j| |dh|/nt (dt is a

@@ -1,12 +1,16 @@
 """GPU parity at the workloads' full sizes, in the launch configuration the
-benchmark times (one call per operation over the whole segment table), on
-sampled rows the oracle computes one by one:
+benchmark times (one call per operation over the whole segment table), every
+output element compared with the oracle (the oracle runs threaded over rows,
+in blocks of rows to bound host memory):
 
-* MLP pair: up [2048,768] + down [768,2048] (compared in full);
+* MLP pair: up [2048,768] + down [768,2048];
 * activation rows [16384,4096] with 1% of rows scaled by 1e3;
 * the whole 12-layer d_model-768 decoder: 85 weight segments in one call;
 * wide rows: weights [14336,4096], [4096,14336]; activations [8192,7168], [4096,16384];
 * rows past the single-pass limit: [6,131072] fp32 weights, [4,262144] bf16 activations.
+
+The forced two-pass runs on the wide shapes repeat a path the long rows
+already cover in full, and stay sampled.
 """
 from __future__ import annotations
 
@@ -37,19 +41,29 @@ def activations():
     return wl.activations(0)
 
 
-def test_activation_rows_sampled(activations):
+def blocks(n: int, size: int = 2048):
+    """Row indices 0..n-1 in consecutive blocks."""
+    for r0 in range(0, n, size):
+        yield np.arange(r0, min(n, r0 + size))
+
+
+def test_activation_rows_full(activations):
     a = activations.acts[0]
-    # every spiked row (x or r scaled by 1e3) plus a random sample
     scale = np.abs(wl.bf16_bits_to_f32(a.x)).max(axis=1) + np.abs(wl.bf16_bits_to_f32(a.r)).max(axis=1)
-    spiked = np.nonzero(scale > 100)[0]
-    assert len(spiked) >= 300
-    rows = gu.sample_rows(a.rows, 512, 1, must=spiked)
+    assert (scale > 100).sum() >= 300          # the spiked rows (x or r scaled by 1e3) are in
     (y0,) = gu.run_l2([a], activations.eps, residual=False)
-    gu.check_l2(a, y0, activations.eps, residual=False, rows=rows, what="l2 without residual")
     (y1,) = gu.run_l2([a], activations.eps, residual=True)
-    gu.check_l2(a, y1, activations.eps, residual=True, rows=rows, what="l2 with residual")
     (h,) = gu.run_slerp([a], activations.eps)
-    gu.check_slerp(a, h, activations.eps, rows=rows, what="slerp")
+    far = {"l2": 0, "l2 + residual": 0, "slerp": 0}
+    for rows in blocks(a.rows):
+        far["l2"] += gu.check_l2(a, y0, activations.eps, residual=False, rows=rows, what="l2 without residual")
+        far["l2 + residual"] += gu.check_l2(a, y1, activations.eps, residual=True, rows=rows,
+                                            what="l2 with residual")
+        far["slerp"] += gu.check_slerp(a, h, activations.eps, rows=rows, what="slerp")
+    print(f"\n[16384, 4096] outputs more than 1 bf16 ulp from the oracle's point value, of "
+          f"{a.rows * a.cols:,} each: {far} (slerp's all at a column whose a_j or b_j rounding is "
+          f"halfway-ambiguous)")
+    assert far["l2"] == 0 and far["l2 + residual"] == 0
 
 
 @pytest.fixture(scope="module")
@@ -68,11 +82,10 @@ def test_whole_model_one_call(whole_model):
     assert launches == 1, launches            # 768- and 2048-wide rows share one staged launch
     grads = gu.run_backward(wk.weights, "bf16", wk.eps)
     ws = gu.run_renorm(wk.weights, wk.eps)
-    for i, (s, o, (gw, gg), w) in enumerate(zip(wk.weights, outs, grads, ws)):
-        rows = gu.sample_rows(s.rows, 6 if s.rows < 30000 else 64, 100 + i)
-        gu.check_forward(s, o, wk.eps, "bf16", rows=rows, what=f"{s.name} forward")
-        gu.check_backward(s, gw, gg, wk.eps, rows=rows, what=f"{s.name} backward")
-        gu.check_renorm(s, w, wk.eps, rows=rows, what=f"{s.name} renorm")
+    for s, o, (gw, gg), w in zip(wk.weights, outs, grads, ws):
+        gu.check_forward(s, o, wk.eps, "bf16", what=f"{s.name} forward")
+        gu.check_backward(s, gw, gg, wk.eps, what=f"{s.name} backward")
+        gu.check_renorm(s, w, wk.eps, what=f"{s.name} renorm")
 
 
 @pytest.fixture(scope="module")
@@ -82,28 +95,31 @@ def wide():
 
 @pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
 def test_wide_weights(wide, out_dtype):
-    for i, s in enumerate(wide.weights):
-        rows = gu.sample_rows(s.rows, 48, 200 + i)
+    for s in wide.weights:
         (o,) = gu.run_forward([s], out_dtype, wide.eps)
-        gu.check_forward(s, o, wide.eps, out_dtype, rows=rows, what=f"{s.name} forward {out_dtype}")
+        for rows in blocks(s.rows):
+            gu.check_forward(s, o, wide.eps, out_dtype, rows=rows, what=f"{s.name} forward {out_dtype}")
         del o
         if out_dtype == "bf16":
             (gw, gg), = gu.run_backward([s], "bf16", wide.eps)
-            gu.check_backward(s, gw, gg, wide.eps, rows=rows, what=f"{s.name} backward")
+            for rows in blocks(s.rows):
+                gu.check_backward(s, gw, gg, wide.eps, rows=rows, what=f"{s.name} backward")
             del gw, gg
             (w,) = gu.run_renorm([s], wide.eps)
-            gu.check_renorm(s, w, wide.eps, rows=rows, what=f"{s.name} renorm")
+            for rows in blocks(s.rows):
+                gu.check_renorm(s, w, wide.eps, rows=rows, what=f"{s.name} renorm")
         torch.cuda.empty_cache()
 
 
 def test_wide_activations(wide):
-    for i, a in enumerate(wide.acts):
-        rows = gu.sample_rows(a.rows, 48, 300 + i)
+    for a in wide.acts:
         for res in (False, True):
             (y,) = gu.run_l2([a], wide.eps, residual=res)
-            gu.check_l2(a, y, wide.eps, residual=res, rows=rows, what=f"{a.name} l2 residual={res}")
+            for rows in blocks(a.rows):
+                gu.check_l2(a, y, wide.eps, residual=res, rows=rows, what=f"{a.name} l2 residual={res}")
         (h,) = gu.run_slerp([a], wide.eps)
-        gu.check_slerp(a, h, wide.eps, rows=rows, what=f"{a.name} slerp")
+        for rows in blocks(a.rows):
+            gu.check_slerp(a, h, wide.eps, rows=rows, what=f"{a.name} slerp")
 
 
 def test_wide_forced_two_pass(wide):

@@ -68,9 +68,9 @@ def check(w: wl.QKRows, qo, ko, eps=1e-6, scale=True, flags=0, rows=None, what="
     ql, qh, kl, kh = oracle.qk_rows_l2_interval(w.q[sel], w.k[sel], w.pos[sel], w.inv, sc, head_dim=w.head_dim,
                                                 eps=eps, flags=flags, nthreads=nt)
     if w.hq:
-        gu.assert_bf16_rows(qo[sel], qr, ql, qh, what + " q")
+        gu.assert_bf16_rows(qo[sel], qr, ql, qh, what + " q", ambiguous=gu.interval_admits_beyond_ulp(qr, ql, qh))
     if w.hk:
-        gu.assert_bf16_rows(ko[sel], kr, kl, kh, what + " k")
+        gu.assert_bf16_rows(ko[sel], kr, kl, kh, what + " k", ambiguous=gu.interval_admits_beyond_ulp(kr, kl, kh))
 
 
 def test_dory_heads_all_rows():
@@ -126,8 +126,9 @@ def test_bad_slot_is_reported_and_skipped():
     ok = slot != 99
     qr, kr = oracle.qk_rows_l2(w.q, w.k, w.pos, w.inv, w.q_scale, head_dim=64)
     ql, qh, kl, kh = oracle.qk_rows_l2_interval(w.q, w.k, w.pos, w.inv, w.q_scale, head_dim=64)
-    gu.assert_bf16_rows(qo, qr, ql, qh, "q rows are all written")
-    gu.assert_bf16_rows(kc[slot[ok]], kr[ok], kl[ok], kh[ok], "k rows with good slots")
+    gu.assert_bf16_rows(qo, qr, ql, qh, "q rows are all written", ambiguous=gu.interval_admits_beyond_ulp(qr, ql, qh))
+    gu.assert_bf16_rows(kc[slot[ok]], kr[ok], kl[ok], kh[ok], "k rows with good slots",
+                        ambiguous=gu.interval_admits_beyond_ulp(kr[ok], kl[ok], kh[ok]))
     assert np.all(kc[3] == gu.CANARY_BF16)     # row 3's slot 99 wrote nothing; cache row 3 is nobody's
 
 

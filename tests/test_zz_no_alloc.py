@@ -1,7 +1,18 @@
-"""The no-alloc slerp backward entry point (a convenience of this library;
-the pages have no counterpart): dalpha's partial sums go to a scratch array
-built into the library instead of a caller workspace.  Its results must be
-bitwise those of ds_slerp_rows_backward with a workspace."""
+"""The no-alloc slerp backward entry point, ds_slerp_rows_backward_noalloc.
+
+It serves callers that cannot allocate device memory where they run the
+backward (a runtime whose device memory all belongs to its own pool, or code
+that must not risk the device-wide synchronisation of cudaMalloc / cudaFree)
+and so cannot hand ds_slerp_rows_backward a workspace: dalpha's partial sums
+go to a 64 MB static device array built into the library instead.  The pages
+have no counterpart.  Its results must be bitwise those of
+ds_slerp_rows_backward with a caller workspace, call after call (the array is
+shared and keeps the previous call's contents), and rows whose partial sums
+need more than the array holds must be refused.
+
+This file is collected last (test_zz_...), so a run that stops at the first
+failure has run every other test before it.
+"""
 from __future__ import annotations
 
 import ctypes as ct
@@ -68,10 +79,38 @@ def test_noalloc_matches_workspace_bitwise(shape):
     assert torch.equal(b[2], c[2])
 
 
+SCRATCH_BYTES = 64 << 20   # the built-in array
+
+
+def widest_accepted_cols() -> int:
+    """The widest row (a multiple of 8) whose dalpha partial sums fit the
+    built-in array on this device (8,712 on a 148-SM B200)."""
+    c = 8
+    while ds.ds_slerp_rows_backward_workspace(c + 8) <= SCRATCH_BYTES:
+        c += 8
+    return c
+
+
+@pytest.mark.gpu
+def test_noalloc_widest_accepted_rows_match_workspace_bitwise():
+    C = widest_accepted_cols()
+    assert ds.ds_slerp_rows_backward_workspace(C) <= SCRATCH_BYTES < ds.ds_slerp_rows_backward_workspace(C + 8)
+    rng = np.random.default_rng(93)
+    res, out, dh = (wl.normal_bf16(rng, (600, C)) for _ in range(3))
+    alpha = wl.alpha_vec(rng, C)
+    a = _run(res, out, alpha, dh, noalloc=False)
+    for _ in range(2):
+        b = _run(res, out, alpha, dh, noalloc=True)
+        for x, y in zip(a, b):
+            assert torch.equal(x, y)
+
+
 @pytest.mark.gpu
 def test_noalloc_refuses_rows_wider_than_its_scratch():
     rng = np.random.default_rng(92)
-    C = 8720  # dalpha lines of 8,720 columns on 148 SMs need more than the 64 MB scratch
+    C = widest_accepted_cols() + 8
     res, out, dh = (wl.normal_bf16(rng, (4, C)) for _ in range(3))
-    with pytest.raises(ds.DSError):
+    with pytest.raises(ds.DSError) as e:
         _run(res, out, wl.alpha_vec(rng, C), dh, noalloc=True)
+    assert e.value.status == ds.DS_ERR_INVALID_ARG
+    assert "built-in scratch" in ds.ds_last_error()
