@@ -80,6 +80,10 @@ WORKLOADS = {
     "gain": "row lengths (Monitor) and the scalar-gain backward (bf16 GY) of the whole-model weights (85 "
             "segments, 100,073,472 fp32 elements); forward (bf16 W_eff) and backward (bf16 GY) of 12 GPT-2 XL "
             "Conv1D weights [1600, 6400] stored [in, out] (transposed rows, 122,880,000 elements)",
+    "long_rows": "rows longer than one CTA's shared memory: wn_forward [2048,40000] and slerp_rows [4096,24576] "
+                 "(clusters of 4 and 2 CTAs, each staging a slice of the row; partial sums through distributed "
+                 "shared memory), wn_forward [256,262144] and slerp_rows [512,262144] (the two-pass stream); inputs "
+                 "drawn on the device",
     "dory": "Dory's fused activation rows: gated l2 rows (o, g bf16, sg fp32) and SwiGLU l2 rows (g, u bf16, "
             "sug, suu fp32) on [16384,4096] and [8192,7168]; q/k rows (rotate-half RoPE, per-head l2, q scale; "
             "16 q heads over 4 kv heads of 256, v copied to the cache) on 16384 rows, a third past position 199,800",
@@ -95,6 +99,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=6)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the per-call report of the config-5 wide calls and the long-row classes")
     p.add_argument("--config", choices=tuple(WORKLOADS), default="step")
     return p.parse_args()
 
@@ -543,6 +549,116 @@ class Step:
             events[len(self.names)].record()
 
 
+# (name, kind, rows, cols): long rows of one length per call, each call's
+# inputs larger than L2; drawn on the device from a seeded generator.
+LONG_CALLS = [("wn_forward_40000", "fwd", 2048, 40000), ("slerp_rows_24576", "slerp", 4096, 24576),
+              ("wn_forward_262144", "fwd", 256, 262144), ("slerp_rows_262144", "slerp", 512, 262144)]
+
+
+class LongRows:
+    """The long-row calls of LONG_CALLS, with the interface of Step that the
+    timing loop uses (names, bytes, rows, plan, copies, run).  Weight rows
+    are N(0, 0.02) times a per-row lognormal factor with gains U(0.5, 2);
+    activation rows bf16 N(0, 1), alpha N(0, 0.05): the recipes of the wide
+    workload, drawn on the device (seeded) to keep set-up short."""
+
+    def __init__(self, seed: int):
+        import torch
+
+        from l2_row_b200 import ds
+
+        self.torch, self.ds = torch, ds
+        gen = torch.Generator(device="cuda")
+        gen.manual_seed(1000 + seed)
+        lib = ds.lib()
+        eps = ct.c_float(EPS)
+        self.plan = [(name, kind, None) for name, kind, _, _ in LONG_CALLS]
+        self.names = [c[0] for c in self.plan]
+        self.copies = 1
+        self.bytes, self.rows, self.tables, self.keep, fns = {}, {}, [], [], []
+        self.classes = {}
+        for name, kind, R, C in LONG_CALLS:
+            act = types.SimpleNamespace(rows=R, cols=C)
+            if kind == "fwd":
+                w = torch.randn(R, C, generator=gen, device="cuda") * 0.02
+                w *= torch.exp(torch.randn(R, 1, generator=gen, device="cuda"))
+                g = torch.rand(R, generator=gen, device="cuda") * 1.5 + 0.5
+                out = torch.empty(R, C, dtype=torch.bfloat16, device="cuda")
+                tab = (ds.ds_wseg * 1)(ds.WSeg(w=w, gain=g, w_eff=out).to_c())
+                fns.append(lambda st, t=tab: lib.ds_wn_forward(t, 1, ds.DS_BF16, eps, st))
+                self.keep += [w, g, out]
+                self.bytes[name] = R * C * (4 + 2) + R * 4
+                op = ds.DS_OP_WN_FORWARD
+            else:
+                x = torch.randn(R, C, generator=gen, device="cuda").to(torch.bfloat16)
+                r = torch.randn(R, C, generator=gen, device="cuda").to(torch.bfloat16)
+                al = torch.randn(C, generator=gen, device="cuda") * 0.05
+                h = torch.empty_like(x)
+                tab = (ds.ds_aseg * 1)(ds.ASeg(x=x, r=r, y=h, alpha=al).to_c())
+                fns.append(lambda st, t=tab: lib.ds_slerp_rows(t, 1, eps, st))
+                self.keep += [x, r, al, h]
+                self.bytes[name] = call_bytes("slerp", act=act)
+                op = ds.DS_OP_SLERP_ROWS
+            self.rows[name] = R
+            self.tables.append(tab)
+            p, grp, cl = ds.ds_row_class(op, C)
+            self.classes[name] = {ds.DS_PATH_CLUSTER: f"cluster of {cl} CTAs", ds.DS_PATH_TWO_PASS:
+                                  f"two-pass stream, {cl} CTAs per row"}.get(p, f"staged ({grp} threads per row)")
+        self.calls = [fns]
+        self.inputs, self.outputs = [], []
+
+    def run(self, stream_ptr: int, events=None, k: int = 0) -> None:
+        Step.run(self, stream_ptr, events, k)
+
+
+def time_calls(step, K: int, W: int, sp: int) -> dict[str, float]:
+    """Mean CUDA-event time (ms) of each call of `step` over K timed steps
+    after W warm-up steps (calls run in the step's order, so each call's
+    inputs were pushed out of L2 by the calls between two uses)."""
+    import torch
+
+    for k in range(W):
+        step.run(sp, None, k)
+    torch.cuda.synchronize()
+    n = len(step.names)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(K)]
+    for k in range(K):
+        step.run(sp, evs[k], k)
+    torch.cuda.synchronize()
+    return {name: statistics.fmean(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K))
+            for i, name in enumerate(step.names)}
+
+
+def extra_calls(seed: int, K: int, sp: int, peak: float) -> dict:
+    """The config-5 wide calls and the long-row classes, each call timed on
+    its own (CUDA events) and reported against the HBM peak; not part of the
+    step's `value`."""
+    import torch
+
+    from l2_row_b200 import ds
+
+    out = {}
+    for label, make in (("config5_wide", lambda: Step(seed=seed, config="wide")),
+                        ("long_rows", lambda: LongRows(seed))):
+        st = make()
+        ms = time_calls(st, K, 3, sp)
+        if ds.ds_get_device_status(sp) != ds.DS_OK:
+            raise RuntimeError(f"device error in the {label} calls")
+        calls = {}
+        for name in st.names:
+            t_s = ms[name] * 1e-3
+            gbs = st.bytes[name] / t_s / 1e9
+            calls[name] = {"us": round(ms[name] * 1e3, 2), "bytes": st.bytes[name], "gb_s": round(gbs, 1),
+                           "frac_of_peak": round(gbs / peak, 4), "rows_s": round(st.rows[name] / t_s, 1)}
+            if isinstance(st, LongRows):
+                calls[name]["class"] = st.classes[name]
+        out[label] = {"workload": WORKLOADS["wide" if label == "config5_wide" else "long_rows"], "steps": K,
+                      "calls": calls}
+        del st
+        torch.cuda.empty_cache()
+    return out
+
+
 def graph_replay_ms(step: Step, reps: int = 20) -> float:
     """Per-step time of the calls replayed from one CUDA graph that holds one
     step on each buffer copy (launch-bound workloads)."""
@@ -583,7 +699,7 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
 
     from l2_row_b200 import ds
 
-    step = Step(seed=rank, config=args.config)
+    step = LongRows(rank) if args.config == "long_rows" else Step(seed=rank, config=args.config)
     names = step.names
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
@@ -650,8 +766,12 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
                  "calls_per_replay": step.copies * len(names)}
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and step.inputs:
         e2e = measure_e2e(step, args.e2e_steps, step_total, sp, world, dist)
+
+    extras = None
+    if args.config == "step" and world == 1 and not args.no_extras:
+        extras = extra_calls(rank, max(5, min(args.steps, 20)), sp, peak)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == "step":
@@ -677,6 +797,8 @@ def run_ours(args, rank: int, world: int, local_rank: int) -> None:
     }
     if graph:
         line["graph"] = graph
+    if extras:
+        line["extras"] = extras
     print(json.dumps(line), flush=True)
 
 

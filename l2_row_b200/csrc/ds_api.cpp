@@ -52,28 +52,29 @@ std::string where(const char *what, int seg)
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-// Bytes a row stages in shared memory on the staged paths, for the widest
-// layout of the operation (fp32 GY; a residual present), so that the path --
-// and with it the row's arithmetic -- depends on (op, cols) only.  The l2
-// backward without a residual (has_r false) is its own layout: two arrays.
-int64_t tile_row_bytes_worst(ds_op op, int64_t cols, bool has_r = true)
+// Bytes per unit (quad of a weight row, octet of an activation row) that a
+// row stages in shared memory on the staged paths, for the widest layout of
+// the operation (fp32 GY; a residual present), so that the class -- and with
+// it the row's arithmetic -- depends on (op, cols) only.  The l2 backward
+// without a residual (has_r false) is its own layout: two arrays.
+int64_t unit_bytes_worst(ds_op op, bool has_r = true)
 {
-    const int64_t q = (cols + 3) / 4 * 16, o = (cols + 7) / 8 * 16;
     switch (op) {
     case DS_OP_WN_FORWARD:
-    case DS_OP_ROW_RENORM: return q;
+    case DS_OP_ROW_RENORM: return 16;
     case DS_OP_WN_BACKWARD:
     case DS_OP_GRAD_PROJECT:
-    case DS_OP_RENORM_MOMENTUM: return 2 * q;
-    case DS_OP_L2_ROWS_BACKWARD: return (has_r ? 3 : 2) * o;
-    case DS_OP_SLERP_ROWS_BACKWARD: return 3 * o;
-    default: return 2 * o;
+    case DS_OP_RENORM_MOMENTUM: return 32;
+    case DS_OP_L2_ROWS_BACKWARD: return has_r ? 48 : 32;
+    case DS_OP_SLERP_ROWS_BACKWARD: return 48;
+    default: return 32;
     }
 }
 
 bool is_act_bwd(ds_op op) { return op == DS_OP_L2_ROWS_BACKWARD || op == DS_OP_SLERP_ROWS_BACKWARD; }
 bool is_fused(ds_op op) { return op == DS_OP_GATE_L2_ROWS || op == DS_OP_SWIGLU_L2_ROWS; }
-// Operations with staged classes only (rows above the largest slot are refused).
+// Operations with staged classes only (no two-pass stream): rows longer
+// than a cluster of 8 staged slices are refused.
 bool staged_only(ds_op op) { return is_act_bwd(op) || is_fused(op); }
 
 // Warps of a staged team: one (weights) or two (activations) per 16 KB of
@@ -86,72 +87,77 @@ int team_warps(ds_op op, int slot)
     return base * slot / ds::kTileSlotBytes;
 }
 
-// Largest staged slot of an operation.
+// Largest staged slot of an operation for one CTA per row; a slice of a row
+// split over a cluster takes at most 64 KB (three ring positions or more).
 int64_t max_slot(ds_op op)
 {
     return ds::is_weight_op(op) ? ds::kTileSlotMaxWeightBytes : ds::kTileSlotMaxBytes;
 }
+constexpr int64_t kClusterSliceMax = 65536;
 
+// Row classes, from (op, cols) alone:
+//   WARP     one CTA per row, the row's staged input <= 16 KB (16 KB slots)
+//   CTA      one CTA per row, <= 64 KB (activations) or 112 KB (weights)
+//   CLUSTER  2, 4 or 8 CTAs per row, each staging a slice of <= 64 KB: the
+//            smallest cluster whose slices fit, in the smallest slot that
+//            holds a slice
+//   TWO_PASS anything longer (operations with a streaming kernel)
+// `forced` (a test knob) picks a class where the row allows it.
 RowClass classify(ds_op op, int64_t cols, int forced, bool has_r = true)
 {
     const int64_t E = ds::elems_per_unit(op);
-    const int64_t nu = (cols + E - 1) / E;
-    const int64_t kmax = ds::kmax_of(op);
-    const int64_t staged = tile_row_bytes_worst(op, cols, has_r);
-    auto staged_class = [&](int path, int min_slot) -> RowClass {
+    const int nu = static_cast<int>((cols + E - 1) / E);
+    const int64_t ubw = unit_bytes_worst(op, has_r);
+    auto staged = [&](int path, int cl, int min_slot, int64_t top) -> RowClass {
+        const int64_t bytes = ds::slice_per(nu, cl) * ubw;
         for (const int slot : {16384, 32768, 65536, 114688})
-            if (slot >= min_slot && slot <= max_slot(op) && staged <= slot)
-                return {path, 32 * team_warps(op, slot), 1, 0, slot};
+            if (slot >= min_slot && slot <= top && bytes <= slot)
+                return {path, 32 * team_warps(op, slot), cl, 0, slot};
         return {0, 0, 0, 0, 0};
     };
-    auto cluster_of = [&]() -> int {
-        for (int CL = 2; CL <= ds::kMaxCluster; CL *= 2)
-            if ((nu + CL - 1) / CL <= ds::kCta * kmax)
-                return CL;
-        return 0;
-    };
-    if (staged_only(op)) {
-        // staged classes only; longer rows are refused (path 0)
-        if (forced == DS_PATH_CTA && staged <= max_slot(op))
-            return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
-        if (staged <= ds::kTileSlotBytes)
-            return staged_class(DS_PATH_WARP, ds::kTileSlotBytes);
-        if (staged <= max_slot(op))
-            return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
+    auto cluster = [&]() -> RowClass {
+        for (int cl = 2; cl <= ds::kMaxCluster; cl *= 2)
+            if (const RowClass c = staged(DS_PATH_CLUSTER, cl, 16384, kClusterSliceMax); c.path)
+                return c;
         return {0, 0, 0, 0, 0};
-    }
+    };
+    const RowClass two_pass = staged_only(op) ? RowClass{0, 0, 0, 0, 0}
+                                              : RowClass{DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0, 0};
     switch (forced) {
     case DS_PATH_WARP:
-        if (staged <= ds::kTileSlotBytes)
-            return staged_class(DS_PATH_WARP, ds::kTileSlotBytes);
+        if (const RowClass c = staged(DS_PATH_WARP, 1, 16384, 16384); c.path)
+            return c;
         break;
     case DS_PATH_CTA:
-        if (staged <= max_slot(op))
-            return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
+        if (const RowClass c = staged(DS_PATH_CTA, 1, 32768, max_slot(op)); c.path)
+            return c;
         break;
     case DS_PATH_CLUSTER:
-        if (const int CL = cluster_of())
-            return {DS_PATH_CLUSTER, 0, CL, 0, 0};
+        if (const RowClass c = cluster(); c.path)
+            return c;
         break;
     case DS_PATH_TWO_PASS:
-        return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0, 0};
+        if (two_pass.path)
+            return two_pass;
+        break;
     default:
         break;
     }
-    if (staged <= ds::kTileSlotBytes)
-        return staged_class(DS_PATH_WARP, ds::kTileSlotBytes);
-    if (staged <= max_slot(op))
-        return staged_class(DS_PATH_CTA, 2 * ds::kTileSlotBytes);
-    if (const int CL = cluster_of())
-        return {DS_PATH_CLUSTER, 0, CL, 0, 0};
-    return {DS_PATH_TWO_PASS, 0, ds::kMaxCluster, 0, 0};
+    if (const RowClass c = staged(DS_PATH_WARP, 1, 16384, 16384); c.path)
+        return c;
+    if (const RowClass c = staged(DS_PATH_CTA, 1, 32768, max_slot(op)); c.path)
+        return c;
+    if (const RowClass c = cluster(); c.path)
+        return c;
+    return two_pass;
 }
 
 // Rows per shared-memory slot of `slot` bytes on the staged paths for the
-// actual layout (staged arrays of this segment), at most kTileMaxRowsPerSlot.
-int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r, int slot)
+// actual layout (staged arrays of this segment) of a row slice of `units`
+// units (the whole row with one CTA per row), at most kTileMaxRowsPerSlot.
+int tile_rows_per_slot(ds_op op, int units, int gy_esize, bool has_r, int slot)
 {
-    const int64_t q = (cols + 3) / 4, o = (cols + 7) / 8;
+    const int64_t q = units, o = units;
     int64_t bytes = 0;
     switch (op) {
     case DS_OP_WN_FORWARD:
@@ -166,7 +172,16 @@ int tile_rows_per_slot(ds_op op, int64_t cols, int gy_esize, bool has_r, int slo
     case DS_OP_SLERP_ROWS_BACKWARD: bytes = o * 16 * 3; break;
     default: bytes = o * 32; break;
     }
+    if (bytes == 0)
+        return ds::kTileMaxRowsPerSlot;
     return static_cast<int>(std::min<int64_t>(ds::kTileMaxRowsPerSlot, slot / bytes));
+}
+
+// Units of the largest slice of a row of `cols` columns in class rc.
+int slice_units(ds_op op, int64_t cols, const RowClass &rc)
+{
+    const int64_t E = ds::elems_per_unit(op);
+    return ds::slice_per(static_cast<int>((cols + E - 1) / E), rc.cluster);
 }
 
 int sm_count()
@@ -505,7 +520,7 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
     for (int i = 0; i < nseg; ++i) {
         cls[i] = classify(op, cols[i], forced);
         if (ds::is_staged(cls[i]))
-            cls[i].rps = tile_rows_per_slot(op, cols[i], esize, true, cls[i].slot);
+            cls[i].rps = tile_rows_per_slot(op, slice_units(op, cols[i], cls[i]), esize, true, cls[i].slot);
     }
     auto make = [&](int i, int64_t r0, int64_t nr) {
         WSegK k = wseg_rows(segs[i], r0, nr, esize, esize);
@@ -530,8 +545,8 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
                           : wop == W_BWD ? (bf16 ? 2 : 3)
                           : wop == W_RENORM ? 4
                           : wop == W_PROJECT ? 7 : 8;
-            const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
-            return ds::launch_tile(tag, &p, grid, rc.slot, st);
+            int used = 0;
+            return ds::launch_tile(tag, &p, units, rc.slot, rc.cluster, &used, st);
         }
         switch (wop) {
         case W_FWD: return ds::launch_wn_forward(rc, p, units, bf16, st);
@@ -707,13 +722,14 @@ ds_status run_act(bool slerp, const ds_aseg *segs, int nseg, float eps, void *st
     for (int i = 0; i < nseg; ++i) {
         cls[i] = classify(op, cols[i], forced);
         if (ds::is_staged(cls[i]))
-            cls[i].rps = tile_rows_per_slot(op, cols[i], 2, segs[i].r != nullptr, cls[i].slot);
+            cls[i].rps = tile_rows_per_slot(op, slice_units(op, cols[i], cls[i]), 2, segs[i].r != nullptr,
+                                            cls[i].slot);
     }
     auto make = [&](int i, int64_t r0, int64_t nr) { return aseg_rows(segs[i], r0, nr); };
     auto launch = [&](const RowClass &rc, const AParams &p, int64_t units, void *st) -> int {
         if (ds::is_staged(rc)) {
-            const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
-            return ds::launch_tile(slerp ? 6 : 5, &p, grid, rc.slot, st);
+            int used = 0;
+            return ds::launch_tile(slerp ? 6 : 5, &p, units, rc.slot, rc.cluster, &used, st);
         }
         return slerp ? ds::launch_slerp_rows(rc, p, units, st) : ds::launch_l2_rows(rc, p, units, st);
     };
@@ -738,8 +754,8 @@ ds_status run_fused(bool swiglu, const ds_fseg *segs, int nseg, float eps, void 
         cols[i] = s.cols;
         cls[i] = classify(op, s.cols, forced);
         if (cls[i].path == 0)
-            return fail(DS_ERR_INVALID_ARG, where("row too long (more than 64 KB of staged input)", i));
-        cls[i].rps = tile_rows_per_slot(op, s.cols, 2, true, cls[i].slot);
+            return fail(DS_ERR_INVALID_ARG, where("row too long (more than 8 staged slices of 64 KB)", i));
+        cls[i].rps = tile_rows_per_slot(op, slice_units(op, s.cols, cls[i]), 2, true, cls[i].slot);
         if (s.rows == 0)
             continue;
         if (ds_status st = check_matrix(s.a, s.rows, s.ld, 2, "a", i))
@@ -778,8 +794,8 @@ ds_status run_fused(bool swiglu, const ds_fseg *segs, int nseg, float eps, void 
         return k;
     };
     auto launch = [&](const RowClass &rc, const AParams &p, int64_t units, void *st) -> int {
-        const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
-        return ds::launch_tile(swiglu ? 12 : 11, &p, grid, rc.slot, st);
+        int used = 0;
+        return ds::launch_tile(swiglu ? 12 : 11, &p, units, rc.slot, rc.cluster, &used, st);
     };
     return launch_all<AParams, ASegK>(nseg, rows.data(), cls, eps, make, launch, stream);
 }
@@ -976,7 +992,7 @@ ds_status run_act_bwd(bool slerp, const ds_agseg *segs, int nseg, float eps, flo
         cols[i] = s.cols;
         cls[i] = classify(op, s.cols, forced, slerp || s.r != nullptr);
         if (cls[i].path == 0)
-            return fail(DS_ERR_INVALID_ARG, where("row too long for the backward (more than 64 KB of staged input)", i));
+            return fail(DS_ERR_INVALID_ARG, where("row too long for the backward (more than 8 staged slices of 64 KB)", i));
         if (s.rows == 0)
             continue;
         total_rows += s.rows;
@@ -1028,17 +1044,16 @@ ds_status run_act_bwd(bool slerp, const ds_agseg *segs, int nseg, float eps, flo
     if (ds_status st = check_overlaps(spans))
         return st;
     for (int i = 0; i < nseg; ++i)
-        cls[i].rps = tile_rows_per_slot(op, cols[i], 2, segs[i].r != nullptr, cls[i].slot);
+        cls[i].rps = tile_rows_per_slot(op, slice_units(op, cols[i], cls[i]), 2, segs[i].r != nullptr,
+                                        cls[i].slot);
     const int tag = slerp ? 10 : 9;
     int grid_used = 0, groups_used = 0;
     int64_t units_used = 0;
     auto make = [&](int i, int64_t r0, int64_t nr) { return agseg_rows(segs[i], r0, nr); };
     auto launch = [&](const RowClass &rc, const GParams &p, int64_t units, void *st) -> int {
-        const int grid = static_cast<int>(std::min<int64_t>(sm_count(), units));
-        grid_used = grid;
         groups_used = ds::tile_groups(tag, rc.slot);
         units_used = units;
-        return ds::launch_tile(tag, &p, grid, rc.slot, st);
+        return ds::launch_tile(tag, &p, units, rc.slot, rc.cluster, &grid_used, st);
     };
     const bool want_dalpha = slerp && dalpha && dcols > 0;
     auto prep = [&](GParams &p) {
@@ -1227,7 +1242,7 @@ ds_status ds_row_class(ds_op op, int64_t cols, int *path, int *group_threads, in
         return fail(DS_ERR_INVALID_ARG, "cols outside [1, 2^31 - 1]");
     const RowClass rc = classify(op, cols, g_force_path.load(std::memory_order_relaxed));
     if (rc.path == 0)
-        return fail(DS_ERR_INVALID_ARG, "row too long for the backward (more than 64 KB of staged input)");
+        return fail(DS_ERR_INVALID_ARG, "row too long for this operation (more than 8 staged slices of 64 KB)");
     if (path)
         *path = rc.path;
     if (group_threads)

@@ -60,6 +60,15 @@ constexpr int kStreamK = 4;
 constexpr int kChunkUnits = kCta * kStreamK;
 constexpr int kStages = 4;
 
+// Rows split over a cluster of `ncta` CTAs (staged cluster classes): CTA k
+// stages units [k * per, min(nu, (k + 1) * per)) of every row, per =
+// ceil(nu / ncta) rounded up to even, so that every slice of an array with
+// 8-byte units (bf16 GY quads) still starts on 16 bytes.  One CTA: the row.
+DS_HD constexpr int slice_per(int nu, int ncta)
+{
+    return ncta <= 1 ? nu : (((nu + ncta - 1) / ncta) + 1) & ~1;
+}
+
 // Row length in 16-byte units: weight ops work on quads of fp32 (w is fp32),
 // activation ops on octets of bf16.
 DS_HD constexpr bool is_weight_op(ds_op op)
@@ -70,22 +79,27 @@ DS_HD constexpr int elems_per_unit(ds_op op) { return is_weight_op(op) ? 4 : 8; 
 
 struct RowClass {
     int path;    // ds_path (never DS_PATH_AUTO)
-    int group;   // threads per row (staged paths: the team), 0 on cluster paths
-    int cluster; // CTAs per row for CLUSTER/TWO_PASS paths (1 otherwise)
+    int group;   // threads per row in each CTA (staged paths: the team), 0 on the two-pass path
+    int cluster; // CTAs per row: 1 on WARP/CTA, 2..8 on CLUSTER (a staged slice each) and TWO_PASS
     int rps;     // staged paths: rows per shared-memory slot for this segment
-    int slot;    // staged paths: slot bytes (16, 32 or 64 KB); 0 otherwise
+    int slot;    // staged paths: slot bytes (16, 32, 64 or 112 KB); 0 on the two-pass path
 };
 
-inline bool is_staged(const RowClass &c) { return c.path == DS_PATH_WARP || c.path == DS_PATH_CTA; }
+// WARP, CTA and CLUSTER rows all run on the staged kernel (a cluster stages
+// one slice of each row per CTA); TWO_PASS rows on the streaming kernel.
+inline bool is_staged(const RowClass &c)
+{
+    return c.path == DS_PATH_WARP || c.path == DS_PATH_CTA || c.path == DS_PATH_CLUSTER;
+}
 
-// Launch shape: the staged segments of a call share one launch per slot
-// size (each segment carries its own rows per slot); CLUSTER and TWO_PASS
-// segments a launch per cluster size.
+// Launch shape: the staged segments of a call share one launch per (slot
+// size, cluster size) (each segment carries its own rows per slot); TWO_PASS
+// segments one launch per cluster size.
 inline bool same_launch(const RowClass &a, const RowClass &b)
 {
-    if (a.path == DS_PATH_CLUSTER || a.path == DS_PATH_TWO_PASS)
+    if (a.path == DS_PATH_TWO_PASS || b.path == DS_PATH_TWO_PASS)
         return a.path == b.path && a.cluster == b.cluster;
-    return a.path == b.path && a.slot == b.slot;
+    return is_staged(b) && a.slot == b.slot && a.cluster == b.cluster && a.path == b.path;
 }
 
 // Device copy of one weight segment.
@@ -237,7 +251,11 @@ int launch_gain_sums(const GainSumParams &p, void *stream);
 // (tags 0-4, 7, 8), AParams (5, 6, 11, 12) or GParams (9, 10) whose segments
 // carry rows per slot in `group` and whose
 // unit_start counts slots; slot_bytes 16, 32, 64 or (weights) 112 KB.
-int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream);
+// cluster: CTAs per row (1, 2, 4 or 8); units: the launch's slots; the
+// kernel gets min(units, resident clusters) clusters, returned in
+// *clusters_used (lines of the slerp backward's dalpha workspace).
+int launch_tile(int tag, const void *params, int64_t units, int slot_bytes, int cluster, int *clusters_used,
+                void *stream);
 // Ring positions (consumer teams) per CTA of a staged launch.
 int tile_groups(int tag, int slot_bytes);
 // The built-in device scratch of the no-alloc slerp backward (ds_tile.cu).

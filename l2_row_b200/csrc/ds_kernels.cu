@@ -1,14 +1,12 @@
 // ds_kernels.cu -- sm_100a kernels for rows too long for the staged path
-// (ds_tile.cu takes every row with at most 64 KB of input).
+// (ds_tile.cu takes every row whose slices fit 8 CTAs' shared memory), and
+// the small kernels around the row calls (row lengths, scalar-gain sums, the
+// bounded-wait self-test).
 //
-// Two shapes of kernel, chosen per row length (ds_api.cpp):
-//   * cluster : a cluster of 2..8 CTAs per row, each holding a contiguous
-//               slice in registers; partial sums meet through distributed
-//               shared memory.  One HBM read.
 //   * stream  : a cluster of 8 CTAs per row, each streaming its slice
 //               through a 4-stage shared-memory ring filled by bulk (TMA)
 //               copies, once per pass (the re-reads hit L2).  Rows of any
-//               length.
+//               length; partial sums meet through distributed shared memory.
 // Operations (sources cited in include/ds.h):
 //   wn_forward, wn_backward, row_renorm : DragonScale unit rows with gains
 //   grad_project, renorm_momentum       : DragonScale "Optimizer" (rescale)
@@ -206,50 +204,7 @@ __device__ __forceinline__ void alpha8(const float *alpha, int u, int cols, floa
 // since b - a itself may round when a and b are far apart in magnitude).
 __device__ __forceinline__ float lerp_t(float a, float b, float m) { return m == 1.f ? b : fmaf(m, b - a, a); }
 
-// ===================================================== register-row bodies ==
-//
-// A row (or a cluster CTA's slice of it) is processed by `stride` threads;
-// thread `lane` holds units ubeg + lane + k*stride, k < KMAX, below uend.
-// `active` is false for padding rows of the last CTA (they still take part
-// in barriers).  `leader` marks the one thread that writes per-row scalars.
-
-template <int KMAX, bool OUT_BF16, bool RENORM, class Red>
-__device__ __forceinline__ void wn_scale_row(const WSegK &sg, int64_t row, bool active, int lane, int stride,
-                                             int ubeg, int uend, float eps, Red &red)
-{
-    const float *w = sg.w + row * sg.ld;
-    float4 x[KMAX];
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        x[k] = (active && u < uend) ? quad_f32(w, u, sg.cols) : make_float4(kZero, kZero, kZero, kZero);
-    }
-    const float g = (!RENORM && active && sg.gain) ? __ldg(sg.gain + row * sg.gain_stride) : 1.f;
-    float acc[1] = {0.f};
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k)
-        acc_sq4(acc[0], x[k]);
-    red.sum(acc);
-    const RowScale rs = row_scale(acc[0], eps, red, [&](auto f) {
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k)
-            each4(x[k], f);
-    });
-    const float sc = (g * sg.radius) * rs.inv;
-    if (!active)
-        return;
-    void *out = RENORM ? static_cast<void *>(const_cast<float *>(sg.w) + row * sg.ld)
-                       : static_cast<void *>(static_cast<char *>(sg.out) +
-                                             row * sg.ld_out * (OUT_BF16 ? 2 : 4));
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        if (u < uend)
-            store_quad<OUT_BF16>(out, u, sg.cols, scale4(x[k], rs.pre, sc));
-    }
-}
-
-// Epilogues of the two-reduction row body (S = sum w^2, D = w . d):
+// Epilogues of the two-reduction row (S = sum w^2, D = w . d):
 //   kModeGrad      ds_wn_backward: grad_w = (g rho / n)(d - w D/n^2), grad_g = rho D / n
 //   kModeProject   ds_grad_project: d <- d - w D/n^2 (d = the gradient, in place)
 //   kModeMomentum  ds_renorm_momentum: d <- d - w D/n^2 (d = the momentum) and
@@ -258,226 +213,6 @@ __device__ __forceinline__ void wn_scale_row(const WSegK &sg, int64_t row, bool 
 // scaled row and the scaled quotient, xs * (Ds / n2s) = w * D / n^2, which
 // stays finite where the unscaled quotient D / n^2 would overflow.
 enum BwdMode { kModeGrad = 0, kModeProject = 1, kModeMomentum = 2 };
-
-template <int KMAX, bool GY_BF16, int MODE, class Red>
-__device__ __forceinline__ void wn_backward_row(const WSegK &sg, int64_t row, bool active, bool leader, int lane,
-                                                int stride, int ubeg, int uend, float eps, Red &red)
-{
-    const float *w = sg.w + row * sg.ld;
-    const void *gy = static_cast<const char *>(sg.gy) + row * sg.ld_out * (GY_BF16 ? 2 : 4);
-    float4 x[KMAX], d[KMAX];
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        const bool ok = active && u < uend;
-        x[k] = ok ? quad_f32(w, u, sg.cols) : make_float4(kZero, kZero, kZero, kZero);
-        d[k] = ok ? quad_gy<GY_BF16>(gy, u, sg.cols) : make_float4(kZero, kZero, kZero, kZero);
-    }
-    const float g = (active && sg.gain) ? __ldg(sg.gain + row * sg.gain_stride) : 1.f;
-    float acc[2] = {0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        acc_sq4(acc[0], x[k]);
-        acc_dot4(acc[1], x[k], d[k]);
-    }
-    red.sum(acc);
-    // Rows whose sum of squares needs rescaling: scale w by 2^m (exact),
-    // re-sum S and D, and carry 2^m into the row constants.
-    int m = 0;
-    const bool need = needs_rescale(acc[0], eps);
-    if (red.any(need)) {
-        float M = 0.f;
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k)
-            each4(x[k], [&](float v) { M = fmaxf(M, fabsf(v)); });
-        M = red.max(M);
-        if (need && M > 0.f && M < __int_as_float(0x7f800000))
-            m = 48 - ilogbf(M);
-        float a2[2] = {0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            const float4 xs = make_float4(scalbnf(x[k].x, m), scalbnf(x[k].y, m), scalbnf(x[k].z, m),
-                                          scalbnf(x[k].w, m));
-            acc_sq4(a2[0], xs);
-            acc_dot4(a2[1], xs, d[k]);
-        }
-        red.sum(a2);
-        if (m != 0) {
-            acc[0] = a2[0];
-            acc[1] = a2[1];
-        }
-    }
-    const float n2 = acc[0] + (m == 0 ? eps : scalbnf(eps, 2 * m));
-    const float inv = 1.0f / sqrtf(n2);
-    if constexpr (MODE != kModeGrad) {
-        const float qs = acc[1] / n2;          // D / (S + eps) times 2^-m
-        const float sc = sg.radius * inv;      // rho / n times 2^-m
-        if (!active)
-            return;
-        float *dd = sg.grad_w + row * sg.ld;
-        float *wo = static_cast<float *>(sg.out) + row * sg.ld;
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            const int u = ubeg + lane + k * stride;
-            if (u < uend) {
-                const float4 xs = m == 0 ? x[k]
-                                         : make_float4(scalbnf(x[k].x, m), scalbnf(x[k].y, m), scalbnf(x[k].z, m),
-                                                       scalbnf(x[k].w, m));
-                float4 y;
-                y.x = fmaf(-xs.x, qs, d[k].x);
-                y.y = fmaf(-xs.y, qs, d[k].y);
-                y.z = fmaf(-xs.z, qs, d[k].z);
-                y.w = fmaf(-xs.w, qs, d[k].w);
-                store_quad<false>(dd, u, sg.cols, y);
-                if constexpr (MODE == kModeMomentum)
-                    store_quad<false>(wo, u, sg.cols, make_float4(xs.x * sc, xs.y * sc, xs.z * sc, xs.w * sc));
-            }
-        }
-        return;
-    }
-    const float q = m == 0 ? acc[1] / n2 : scalbnf(acc[1] / n2, m);  // D / (S + eps)
-    const float pre = (g * sg.radius) * (m == 0 ? inv : scalbnf(inv, m));
-    if (!active)
-        return;
-    if (leader && sg.gain)
-        sg.grad_g[row] = sg.radius * acc[1] * inv;                     // rho D / n
-    float *gw = sg.grad_w + row * sg.ld;
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        if (u < uend) {
-            float4 y;
-            y.x = pre * fmaf(-x[k].x, q, d[k].x);
-            y.y = pre * fmaf(-x[k].y, q, d[k].y);
-            y.z = pre * fmaf(-x[k].z, q, d[k].z);
-            y.w = pre * fmaf(-x[k].w, q, d[k].w);
-            store_quad<false>(gw, u, sg.cols, y);
-        }
-    }
-}
-
-template <int KMAX, class Red>
-__device__ __forceinline__ void l2_row(const ASegK &sg, int64_t row, bool active, int lane, int stride, int ubeg,
-                                       int uend, float eps, Red &red)
-{
-    const uint16_t *x = sg.x + row * sg.ld;
-    const uint16_t *r = sg.r ? sg.r + row * sg.ld : nullptr;
-    uint4 s[KMAX];
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        s[k] = (active && u < uend) ? ld16(x + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    if (r) {
-        uint4 b[KMAX];
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            const int u = ubeg + lane + k * stride;
-            b[k] = (active && u < uend) ? ld16(r + 8 * u) : make_uint4(0u, 0u, 0u, 0u);
-        }
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k)
-            s[k] = add_bf16x8(s[k], b[k]);
-    }
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        const int valid = sg.cols - 8 * u;
-        if (valid < 8)
-            s[k] = mask_octet(s[k], valid > 0 ? valid : 0);
-    }
-    float acc[1] = {0.f};
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k)
-        acc_sq8(acc[0], s[k]);
-    red.sum(acc);
-    const RowScale rs = row_scale(acc[0], eps, red, [&](auto f) {
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k)
-            each8(s[k], f);
-    });
-    if (!active)
-        return;
-    uint16_t *y = sg.y + row * sg.ld;
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        if (u < uend)
-            store_octet(y, u, sg.cols, scale_bf16x8(s[k], rs));
-    }
-}
-
-template <int KMAX, class Red>
-__device__ __forceinline__ void slerp_row(const ASegK &sg, int64_t row, bool active, int lane, int stride,
-                                          int ubeg, int uend, float eps, Red &red)
-{
-    const uint16_t *xr = sg.x + row * sg.ld;
-    const uint16_t *orow = sg.r + row * sg.ld;
-    uint4 a[KMAX], b[KMAX];
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        const bool ok = active && u < uend;
-        a[k] = ok ? octet(xr, u, sg.cols) : make_uint4(0u, 0u, 0u, 0u);
-        b[k] = ok ? octet(orow, u, sg.cols) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    float acc[2] = {0.f, 0.f};
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        acc_sq8(acc[0], a[k]);
-        acc_sq8(acc[1], b[k]);
-    }
-    red.sum(acc);
-    const RowScale ra = row_scale(acc[0], eps, red, [&](auto f) {
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k)
-            each8(a[k], f);
-    });
-    const RowScale rb = row_scale(acc[1], eps, red, [&](auto f) {
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k)
-            each8(b[k], f);
-    });
-    // the rounding points a = bf16(l2(res)), b = bf16(l2(out))
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        a[k] = scale_bf16x8(a[k], ra);
-        b[k] = scale_bf16x8(b[k], rb);
-    }
-    auto each_t = [&](auto f) {
-#pragma unroll
-        for (int k = 0; k < KMAX; ++k) {
-            const int u = ubeg + lane + k * stride;
-            float m[8];
-            alpha8(sg.alpha, u, sg.cols, m); // zero past cols; a = b = 0 there anyway
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                f(lerp_t(bf_get(a[k], e), bf_get(b[k], e), m[e]));
-        }
-    };
-    float at[1] = {0.f};
-    each_t([&](float t) { at[0] = fmaf(t, t, at[0]); });
-    red.sum(at);
-    const RowScale rt = row_scale(at[0], eps, red, each_t);
-    if (!active)
-        return;
-    uint16_t *y = sg.y + row * sg.ld;
-#pragma unroll
-    for (int k = 0; k < KMAX; ++k) {
-        const int u = ubeg + lane + k * stride;
-        if (u < uend) {
-            float m[8];
-            alpha8(sg.alpha, u, sg.cols, m);
-            float h[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                h[e] = (lerp_t(bf_get(a[k], e), bf_get(b[k], e), m[e]) * rt.pre) * rt.inv;
-            store_octet(y, u, sg.cols,
-                        make_uint4(pack_bf2(h[0], h[1]), pack_bf2(h[2], h[3]), pack_bf2(h[4], h[5]),
-                                   pack_bf2(h[6], h[7])));
-        }
-    }
-}
 
 // ================================================================ kernels ==
 
@@ -499,61 +234,8 @@ struct OpOf {
                                  : T == kL2 ? DS_OP_L2_ROWS : DS_OP_SLERP_ROWS;
 };
 
-template <int T, class P, class Red>
-__device__ __forceinline__ void run_row(const P &p, int si, int64_t row, bool active, bool leader, int lane,
-                                        int stride, int ubeg, int uend, Red &red)
-{
-    const auto &sg = p.seg[si];
-    constexpr int K = kmax_of(OpOf<T>::value);
-    if constexpr (T == kFwdBf16)
-        wn_scale_row<K, true, false>(sg, row, active, lane, stride, ubeg, uend, p.eps, red);
-    else if constexpr (T == kFwdF32)
-        wn_scale_row<K, false, false>(sg, row, active, lane, stride, ubeg, uend, p.eps, red);
-    else if constexpr (T == kRenorm)
-        wn_scale_row<K, false, true>(sg, row, active, lane, stride, ubeg, uend, p.eps, red);
-    else if constexpr (T == kBwdBf16)
-        wn_backward_row<K, true, kModeGrad>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
-    else if constexpr (T == kBwdF32)
-        wn_backward_row<K, false, kModeGrad>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
-    else if constexpr (T == kProject)
-        wn_backward_row<K, false, kModeProject>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
-    else if constexpr (T == kMomentum)
-        wn_backward_row<K, false, kModeMomentum>(sg, row, active, leader, lane, stride, ubeg, uend, p.eps, red);
-    else if constexpr (T == kL2)
-        l2_row<K>(sg, row, active, lane, stride, ubeg, uend, p.eps, red);
-    else
-        slerp_row<K>(sg, row, active, lane, stride, ubeg, uend, p.eps, red);
-}
-
 template <int T>
 using ParamsOf = typename std::conditional<IsWeight<T>::value, WParams, AParams>::type;
-
-// Resident CTAs per SM the register paths are compiled for (register cap
-// 65536 / (256 * blocks)): 4 where a thread holds one or two inputs of up to
-// 32 registers each, 2 for slerp (two rows of inputs plus its lerp).
-template <int T>
-struct MinBlocks {
-    static constexpr int value = T == kSlerp ? 2 : 4;
-};
-
-// A cluster of CTAs per row; each CTA holds a contiguous slice.
-template <int T>
-__global__ void __launch_bounds__(kCta, MinBlocks<T>::value) k_cluster(const __grid_constant__ ParamsOf<T> p)
-{
-    __shared__ float red_sm[2 * kWarps * 4];
-    __shared__ float red_dsm[2 * kMaxCluster * 4];
-    cluster_arrive_relaxed();
-    ClusterReducer red(red_sm, red_dsm);
-    const int64_t unit = blockIdx.x / red.ncta;
-    const int si = find_segment(p, unit);
-    const int64_t row = unit - p.unit_start[si];
-    const int nu = p.seg[si].nu;
-    const int per = (nu + red.ncta - 1) / red.ncta;
-    const int ubeg = min(nu, static_cast<int>(red.rank) * per);
-    const int uend = min(nu, ubeg + per);
-    run_row<T>(p, si, row, true, threadIdx.x == 0 && red.rank == 0, threadIdx.x, kCta, ubeg, uend, red);
-    red.finish();
-}
 
 // ======================================================= streaming rows ====
 //
@@ -1034,8 +716,6 @@ template <int T>
 cudaError_t launch_op(const RowClass &rc, const ParamsOf<T> &p, int64_t units, void *stream)
 {
     switch (rc.path) {
-    case DS_PATH_CLUSTER:
-        return launch_clustered(k_cluster<T>, p, units, rc.cluster, 0, stream);
     case DS_PATH_TWO_PASS: {
         constexpr int smem = kStages * stream_stage_bytes<T>();
         static DeviceFlags attr_set;

@@ -18,6 +18,9 @@
 // (even and odd elements) added at the end, an xor butterfly over the lanes,
 // then the warps' partials as a balanced tree -- so a row's bits depend on
 // its length and the operation only.
+#include <algorithm>
+#include <atomic>
+
 #include <cuda_runtime.h>
 
 #include "ds_device.cuh"
@@ -88,13 +91,79 @@ __device__ __forceinline__ void named_sync(int id, int nthreads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Distributed shared memory helpers for rows split over a cluster: the
+// address of a variable of this CTA as seen in peer `rank`'s shared memory,
+// a store and an mbarrier arrival there (release at cluster scope: the
+// values written before it are visible to whoever acquires the phase).
+__device__ __forceinline__ uint32_t peer_addr(const void *local, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void peer_store_f32(uint32_t addr, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void peer_store_u32(uint32_t addr, uint32_t v)
+{
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void peer_arrive(uint32_t bar_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(smem_u32(bar)), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Exchange area of one team when its rows are split over a cluster: two
+// alternating buffers of [kMaxCluster CTAs][2 values] and their mbarriers
+// (each CTA of the cluster arrives once per exchange).
+constexpr int kXchgFloats = 2 * kMaxCluster * 2;
+constexpr int kXchgBytesPerTeam = kXchgFloats * 4 + 2 * 8;
+
+// The cluster context of a CTA: its rank, the cluster's size, the CTA-wide
+// abort flag (set here, and in every peer, by the first wait that gives up)
+// and the bound of every wait.
+struct ClusterCtx {
+    uint32_t rank, ncta;
+    volatile int *abort_flag;
+    uint64_t limit_ns;
+
+    __device__ void abort_all() const
+    {
+        *abort_flag = 1;
+        for (uint32_t k = 0; k < ncta; ++k)
+            if (k != rank)
+                peer_store_u32(peer_addr(const_cast<int *>(abort_flag), k), 1u);
+    }
+};
+
 // The threads that normalise one row: one warp (weight calls) or the team
-// of WP warps that share a group of ring positions (activation calls).  A
-// sum comes back to every thread with the same bits: the xor butterfly in
-// each warp, then the warps' partials through shared memory and the group's
-// named barrier, added as a balanced tree in warp order ((w0 + w1) + (w2 +
-// w3) ...).  Two alternating slots make back-to-back reductions safe with one
-// barrier each (all warps of a team run the same sequence of reductions).
+// of WP warps that share a group of ring positions (activation calls), in
+// each CTA of the row's cluster.  A sum comes back to every thread of every
+// CTA with the same bits: the xor butterfly in each warp, then the warps'
+// partials through shared memory and the group's named barrier, added as a
+// balanced tree in warp order ((w0 + w1) + (w2 + w3) ...), then -- rows split
+// over a cluster -- the CTAs' totals through distributed shared memory,
+// added in rank order.  Two alternating slots make back-to-back reductions
+// safe with one barrier each (all warps of a team run the same sequence of
+// reductions; all CTAs of a cluster the same sequence of exchanges, and a
+// CTA writes exchange k + 2 only after every peer's part of exchange k + 1
+// arrived, which each peer sends after reading exchange k).
 template <int N>
 __device__ __forceinline__ float tree_sum(const float *r, int i)
 {
@@ -113,14 +182,80 @@ __device__ __forceinline__ float tree_max(const float *r)
         return fmaxf(tree_max<N / 2>(r), tree_max<N / 2>(r + N));
 }
 
-template <int WP>
+template <int WP, bool SPLIT = false>
 struct Team {
-    static constexpr int G = 32 * WP; // threads per row
+    static constexpr int G = 32 * WP; // threads per row in this CTA
     static constexpr int kRed = 4 * WP; // floats of `red`: [2 slots][WP warps][2 values]
     int t;                            // this thread's index in the team
     int bar;                          // named barrier (teams of several warps)
     float *red;
     int slot = 0;
+    // rows split over a cluster (SPLIT): this team's exchange area (unused,
+    // and dropped by the compiler, with one CTA per row)
+    const ClusterCtx *ctx = nullptr;
+    float *xbuf = nullptr;            // [2][kMaxCluster][2]
+    uint64_t *xbar = nullptr;         // [2]
+    uint32_t xuse = 0;                // exchanges so far
+    bool failed = false;              // an exchange gave up: store nothing more
+
+    __device__ __forceinline__ uint32_t rank() const
+    {
+        if constexpr (SPLIT)
+            return ctx->rank;
+        else
+            return 0u;
+    }
+    __device__ __forceinline__ bool good() const
+    {
+        if constexpr (SPLIT)
+            return !failed;
+        else
+            return true;
+    }
+
+    // The CTAs' totals v[0..N) through the cluster, combined in rank order.
+    template <int N, class Op>
+    __device__ __noinline__ void exchange(float (&v)[N], Op op)
+    {
+        const int b = static_cast<int>(xuse & 1u);
+        const uint32_t parity = (xuse >> 1) & 1u;
+        ++xuse;
+        float *buf = xbuf + b * (kMaxCluster * 2);
+        uint64_t *bb = xbar + b;
+        const uint32_t n = ctx->ncta, me = ctx->rank;
+        __syncwarp();
+        if (t == 0 && !failed) {
+            for (uint32_t k = 0; k < n; ++k) {
+#pragma unroll
+                for (int i = 0; i < N; ++i)
+                    peer_store_f32(peer_addr(buf + me * 2 + i, k), v[i]);
+                peer_arrive(peer_addr(bb, k));
+            }
+        }
+        bool ok = !failed;
+        if (ok && !mbar_try_wait_cluster(bb, parity)) {
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait_cluster(bb, parity)) {
+                if (*ctx->abort_flag || global_timer_ns() - t0 > ctx->limit_ns) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        if (!ok) {
+            if (!failed)
+                ctx->abort_all();
+            failed = true;
+            return;
+        }
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            float a = buf[i];
+            for (uint32_t k = 1; k < n; ++k)
+                a = op(a, buf[k * 2 + i]);
+            v[i] = a;
+        }
+    }
 
     template <int N>
     __device__ __forceinline__ void sum(float (&v)[N])
@@ -141,6 +276,8 @@ struct Team {
                 v[i] = tree_sum<WP>(r, i);
             slot ^= 1;
         }
+        if constexpr (SPLIT)
+            exchange(v, [](float a, float b) { return a + b; });
     }
 
     __device__ __forceinline__ float sum1(float v)
@@ -160,6 +297,11 @@ struct Team {
             named_sync(bar, G);
             v = tree_max<WP>(r);
             slot ^= 1;
+        }
+        if constexpr (SPLIT) {
+            float a[1] = {v};
+            exchange(a, [](float x, float y) { return fmaxf(x, y); });
+            v = a[0];
         }
         return v;
     }
@@ -283,8 +425,8 @@ __device__ __forceinline__ int64_t tile_src_pitch(const AGSegK &sg, int)
 // valid elements of unit nfull (0 if none), handled by lane nfull % 32 after
 // its full units, so every lane's units are summed in increasing order.
 
-template <bool OUT_BF16, bool RENORM, int WP>
-__device__ __forceinline__ void tile_scale_row(Team<WP> &tm, const WSegK &sg, int64_t row, float g,
+template <bool OUT_BF16, bool RENORM, int WP, bool SPLIT>
+__device__ __forceinline__ void tile_scale_row(Team<WP, SPLIT> &tm, const WSegK &sg, int64_t row, float g,
                                                const unsigned char *s0, int nfull, int tail, float eps, bool store)
 {
     constexpr int G = Team<WP>::G;
@@ -316,7 +458,7 @@ __device__ __forceinline__ void tile_scale_row(Team<WP> &tm, const WSegK &sg, in
             f(f2(vt.z, vt.w));
         }
     });
-    if (!store)
+    if (!store || !tm.good())
         return;
     const float sc = (g * sg.radius) * rs.inv;
     const float2 sc2 = f2(sc, sc), pre2 = f2(rs.pre, rs.pre);
@@ -375,8 +517,8 @@ __device__ __forceinline__ float4 gy_unit(const unsigned char *s1, int u)
 // momentum, and w <- rho w / n in place).  With the power-of-two rescale the
 // projection applies the scaled quotient to the scaled row, which stays
 // finite where D/n^2 alone would overflow.
-template <bool GY_BF16, int MODE, int WP>
-__device__ __forceinline__ void tile_backward_row(Team<WP> &tm, const WSegK &sg, int64_t row, float g,
+template <bool GY_BF16, int MODE, int WP, bool SPLIT>
+__device__ __forceinline__ void tile_backward_row(Team<WP, SPLIT> &tm, const WSegK &sg, int64_t row, float g,
                                                   const unsigned char *s0, const unsigned char *s1, int nfull,
                                                   int tail, float eps, bool store)
 {
@@ -436,7 +578,7 @@ __device__ __forceinline__ void tile_backward_row(Team<WP> &tm, const WSegK &sg,
             D = sd2[1];
         }
     }
-    if (!store)
+    if (!store || !tm.good())
         return;
     const float n2 = S + (m == 0 ? eps : scalbnf(eps, 2 * m));
     const float inv = 1.0f / sqrtf(n2);
@@ -476,7 +618,7 @@ __device__ __forceinline__ void tile_backward_row(Team<WP> &tm, const WSegK &sg,
     }
     const float q = m == 0 ? D / n2 : scalbnf(D / n2, m);
     const float pre = (g * sg.radius) * (m == 0 ? inv : scalbnf(inv, m));
-    if (lane == 0 && sg.gain)
+    if (lane == 0 && sg.gain && tm.rank() == 0)
         sg.grad_g[row] = sg.radius * D * inv;
     const float2 nq = f2(-q, -q), pre2 = f2(pre, pre);
     char *out = reinterpret_cast<char *>(sg.grad_w + row * sg.ld);
@@ -582,8 +724,8 @@ __device__ __forceinline__ uint4 l2_unit_s(const uint4 *x, const uint4 *r, int u
     return s;
 }
 
-template <int WP, bool HAS_R>
-__device__ __forceinline__ void tile_l2_row(Team<WP> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
+template <int WP, bool HAS_R, bool SPLIT>
+__device__ __forceinline__ void tile_l2_row(Team<WP, SPLIT> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
                                             const unsigned char *s1, int nfull, int tail, float eps, bool store)
 {
     constexpr int G = Team<WP>::G;
@@ -610,7 +752,7 @@ __device__ __forceinline__ void tile_l2_row(Team<WP> &tm, const ASegK &sg, int64
         for (int u = t; u < nunits; u += G)
             pairs8(x[u], f);
     });
-    if (!store)
+    if (!store || !tm.good())
         return;
     uint16_t *y = sg.y + row * sg.ld;
 #pragma unroll 4
@@ -675,8 +817,8 @@ __device__ __forceinline__ uint4 slerp_unit_h(float4 p, float4 q, float2 s)
                       pk(__fmul2_rn(f2(q.x, q.y), s)), pk(__fmul2_rn(f2(q.z, q.w), s)));
 }
 
-template <int WP, bool CACHED>
-__device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
+template <int WP, bool CACHED, bool SPLIT>
+__device__ __forceinline__ void tile_slerp_row(Team<WP, SPLIT> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
                                                unsigned char *s1, int nfull, int tail, float eps, bool store,
                                                const float *abs_alpha, int half)
 {
@@ -737,7 +879,7 @@ __device__ __forceinline__ void tile_slerp_row(Team<WP> &tm, const ASegK &sg, in
             f(f2(q.z, q.w));
         }
     });
-    if (!store)
+    if (!store || !tm.good())
         return;
     // pass 3
     uint16_t *y = sg.y + row * sg.ld;
@@ -800,8 +942,8 @@ __device__ __forceinline__ void store8f(float *o, int u, const float2 (&v)[4], i
 // dx = (dy - s D/(S+eps)) / sqrt(S+eps).  Rows needing the power-of-two
 // rescale re-sum with s scaled by 2^m and apply the scaled quotient to the
 // scaled row (exactly the unscaled product), with 2^m carried into 1/n.
-template <int WP, bool HAS_R>
-__device__ __forceinline__ void tile_l2_bwd_row(Team<WP> &tm, const AGSegK &sg, int64_t row, unsigned char *s0,
+template <int WP, bool HAS_R, bool SPLIT>
+__device__ __forceinline__ void tile_l2_bwd_row(Team<WP, SPLIT> &tm, const AGSegK &sg, int64_t row, unsigned char *s0,
                                                 const unsigned char *s1, unsigned char *s2, int nfull, int tail,
                                                 float eps, bool store)
 {
@@ -857,7 +999,7 @@ __device__ __forceinline__ void tile_l2_bwd_row(Team<WP> &tm, const AGSegK &sg, 
             D = sd2[1];
         }
     }
-    if (!store)
+    if (!store || !tm.good())
         return;
     const float n2 = S + (m == 0 ? eps : scalbnf(eps, 2 * m));
     const float inv = 1.0f / sqrtf(n2);
@@ -923,8 +1065,8 @@ __device__ __forceinline__ float2 sgn2(float2 v)
 // adding this row's sign(alpha) (b - a) dt to the team's dalpha line; pass 4
 // stores dres = (da - ua (ua . da)) / na and dout likewise.  t, dt and the
 // rest are recomputed from the slot in each pass.
-template <int WP, bool CACHED>
-__device__ __forceinline__ void tile_slerp_bwd_row(Team<WP> &tm, const AGSegK &sg, int64_t row, unsigned char *s0,
+template <int WP, bool CACHED, bool SPLIT>
+__device__ __forceinline__ void tile_slerp_bwd_row(Team<WP, SPLIT> &tm, const AGSegK &sg, int64_t row, unsigned char *s0,
                                                    unsigned char *s1, unsigned char *s2, int nfull, int tail, float eps,
                                                    bool store, const float *acache, int half, float *wsl,
                                                    bool ws_first)
@@ -1016,7 +1158,7 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP> &tm, const AGSegK &s
             const float2 ba = __fadd2_rn(lo2(word4(b, i)), fneg2(lo2(word4(a, i))));
             part[i] = __fmul2_rn(__fmul2_rn(sgn2(al[i]), ba), dt);
         }
-        if (wsl != nullptr && store) {
+        if (wsl != nullptr && store && tm.good()) {
             float4 *l = reinterpret_cast<float4 *>(wsl + 8 * u);
             float4 p0 = make_float4(part[0].x, part[0].y, part[1].x, part[1].y);
             float4 p1 = make_float4(part[2].x, part[2].y, part[3].x, part[3].y);
@@ -1031,7 +1173,7 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP> &tm, const AGSegK &s
     }
     float sab2[2] = {sa.x + sa.y, sb.x + sb.y};
     tm.sum(sab2);
-    if (!store)
+    if (!store || !tm.good())
         return;
     // pass 4
     const float2 nDa = f2(-sab2[0], -sab2[0]), nDb = f2(-sab2[1], -sab2[1]);
@@ -1204,8 +1346,8 @@ __global__ void __launch_bounds__(256) k_division_check(unsigned long long *coun
     atomicAdd(&counts[3], n_q);
 }
 
-template <int WP, int PRO, bool CACHED>
-__device__ __forceinline__ void tile_fused_row(Team<WP> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
+template <int WP, int PRO, bool CACHED, bool SPLIT>
+__device__ __forceinline__ void tile_fused_row(Team<WP, SPLIT> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
                                                const unsigned char *s1, int nfull, int tail, float eps, bool store,
                                                const float *ca, const float *cb, int half)
 {
@@ -1237,7 +1379,7 @@ __device__ __forceinline__ void tile_fused_row(Team<WP> &tm, const ASegK &sg, in
         for (int u = t; u < nunits; u += G)
             pairs8(x[u], f);
     });
-    if (!store)
+    if (!store || !tm.good())
         return;
     uint16_t *y = sg.y + row * sg.ld;
 #pragma unroll 4
@@ -1294,7 +1436,77 @@ struct TileCfg {
     static_assert(kSmem <= 229376, "ring and vector caches fit 224 KB");
 };
 
+// Segment view of CTA `rank`'s slice of every row: the row pointers (and
+// the per-column vectors) moved to column c0 and the row length cut to the
+// slice's `cols` columns in `nu` units (per-row vectors -- gains, grad_g --
+// stay), so that a row body sees the slice as a row of its own; the
+// per-column vectors are then read only up to the slice's end.
+template <int T>
+__device__ __forceinline__ WSegK shifted(const WSegK &s, int c0, int cols, int nu)
+{
+    WSegK k = s;
+    k.cols = cols;
+    k.nu = nu;
+    constexpr int oe = (T == tFwdBf16 || T == tBwdBf16) ? 2 : 4; // bytes of an element of out / gy
+    k.w = s.w + c0;
+    if (s.out)
+        k.out = static_cast<char *>(s.out) + static_cast<int64_t>(c0) * (T == tRenorm || T == tProject ||
+                                                                        T == tMomentum ? 4 : oe);
+    if (s.gy)
+        k.gy = static_cast<const char *>(s.gy) + static_cast<int64_t>(c0) * (T == tBwdBf16 ? 2 : 4);
+    if (s.grad_w)
+        k.grad_w = s.grad_w + c0;
+    return k;
+}
+
+template <int T>
+__device__ __forceinline__ ASegK shifted(const ASegK &s, int c0, int cols, int nu)
+{
+    ASegK k = s;
+    k.cols = cols;
+    k.nu = nu;
+    k.x = s.x + c0;
+    if (s.r)
+        k.r = s.r + c0;
+    k.y = s.y + c0;
+    if (s.alpha)
+        k.alpha = s.alpha + c0;
+    if (s.s2)
+        k.s2 = s.s2 + c0;
+    return k;
+}
+
+template <int T>
+__device__ __forceinline__ AGSegK shifted(const AGSegK &s, int c0, int cols, int nu)
+{
+    AGSegK k = s;
+    k.cols = cols;
+    k.nu = nu;
+    k.x = s.x + c0;
+    if (s.r)
+        k.r = s.r + c0;
+    k.dy = s.dy + c0;
+    k.dx = s.dx + c0;
+    if (s.dr)
+        k.dr = s.dr + c0;
+    if (s.alpha)
+        k.alpha = s.alpha + c0;
+    return k;
+}
+
+// Exchange area bytes of a staged launch whose rows are split over a
+// cluster (after the ring and the vector caches); none for one CTA per row.
 template <int T, int SB>
+constexpr int tile_xchg_bytes()
+{
+    return TileCfg<T, SB>::kGroups * kXchgBytesPerTeam;
+}
+
+// The staged kernel.  One CTA per SM; with a cluster launch (2, 4 or 8 CTAs
+// per cluster) the cluster's CTAs walk the same slots, each staging and
+// normalising its slice of the rows (slice_per), and the teams' reductions
+// meet through distributed shared memory.
+template <int T, int SB, bool SPLIT>
 __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
     k_tile(const __grid_constant__ TParams<T> p)
 {
@@ -1302,39 +1514,67 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
     constexpr int slot_bytes = SB;
     constexpr int WP = Cfg::kWP;
     constexpr int nslots = Cfg::kSlots;
+    constexpr int E = is_weight_tag(T) ? 4 : 8;   // elements per 16-byte unit of array 0
     extern __shared__ __align__(128) unsigned char ring[];
     __shared__ __align__(8) uint64_t full[nslots];
     __shared__ __align__(8) uint64_t empty[nslots];
     __shared__ SlotHdr hdr[nslots];
     __shared__ float red[Cfg::kGroups * Team<WP>::kRed]; // team reductions
     __shared__ int vote[Cfg::kGroups * 2 * WP];           // team agreement on a wait: [team][2][warp]
-    __shared__ volatile int abort_flag;                    // set by the first wait that runs out
+    __shared__ volatile int abort_flag;                    // set by the first wait that runs out (or by a peer)
     // slerp: |alpha| of the launch's (single) alpha vector, after the ring
     float *s_alpha = reinterpret_cast<float *>(ring + static_cast<size_t>(nslots) * slot_bytes);
+    // rows split over a cluster: the teams' exchange areas after the caches
+    unsigned char *xarea = ring + Cfg::kSmem;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ncta = SPLIT ? cluster_nctarank() : 1u, rank = SPLIT ? cluster_ctarank() : 0u;
+    constexpr bool split = SPLIT;
+    const int64_t cid = blockIdx.x / ncta, ncl = gridDim.x / ncta;   // this cluster, the clusters
     const int64_t total = p.unit_start[p.nseg];
-    // this CTA's slots: blockIdx.x, blockIdx.x + gridDim.x, ...
-    const int64_t mine = total > blockIdx.x ? (total - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    // this cluster's slots: cid, cid + ncl, ...
+    const int64_t mine = total > cid ? (total - 1 - cid) / ncl + 1 : 0;
+    const ClusterCtx ctx{rank, ncta, &abort_flag, p.wait_limit_ns};
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < nslots; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], WP); // every warp of the owning team arrives
         }
+        if (split)
+            for (int q = 0; q < Cfg::kGroups; ++q) {
+                uint64_t *xb = reinterpret_cast<uint64_t *>(xarea + q * kXchgBytesPerTeam + kXchgFloats * 4);
+                mbar_init(&xb[0], ncta); // every CTA of the cluster arrives once per exchange
+                mbar_init(&xb[1], ncta);
+            }
         abort_flag = 0;
         mbar_init_fence();
     }
+    // |alpha| (slerp), alpha (slerp backward) or the scale vectors (Dory
+    // rows) of this CTA's slice of the columns, when every segment of the
+    // launch shares them and the slice fits the cache
+    int acols = p.alpha_cols, ac0 = 0;
+    if (SPLIT && p.alpha_shared) {
+        const int anu = (p.alpha_cols + 7) / 8, aper = slice_per(anu, static_cast<int>(ncta));
+        const int au0 = min(anu, static_cast<int>(rank) * aper), au1 = min(anu, au0 + aper);
+        ac0 = 8 * au0;
+        acols = max(0, min(p.alpha_cols - ac0, 8 * (au1 - au0)));
+    }
+    // (one CTA per row: read from the parameters where it is used)
+    auto cached = [&]() {
+        return p.alpha_shared != nullptr && (SPLIT ? acols : p.alpha_cols) <= Cfg::kAlphaCache;
+    };
+    const bool acached = cached();
     if constexpr (T == tSlerp || T == tSlerpBwd) {
         // |alpha| split by halves of each 8-element unit: unit u's first four
         // at [4u], its last four at [half + 4u], so that a warp reading one
         // float4 per lane touches consecutive 16-byte words (no bank conflict)
-        if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache) {
-            const int nu = (p.alpha_cols + 7) / 8, half = Cfg::kAlphaCache / 2;
+        if (acached) {
+            const int nu = (acols + 7) / 8, half = Cfg::kAlphaCache / 2;
             for (int i = threadIdx.x; i < 8 * nu; i += blockDim.x) {
                 const int u = i >> 3, e = i & 7;
                 // the backward keeps the sign (dalpha needs it); the forward |alpha|
-                const float a = i < p.alpha_cols ? __ldg(p.alpha_shared + i) : 0.f;
+                const float a = i < acols ? __ldg(p.alpha_shared + ac0 + i) : 0.f;
                 const float v = T == tSlerpBwd ? a : fabsf(a);
                 s_alpha[(e < 4 ? 0 : half) + 4 * u + (e & 3)] = v;
             }
@@ -1342,17 +1582,23 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
     }
     if constexpr (T == tGateL2 || T == tSwigluL2) {
         // the scale vectors in the same split layout, sb after sa
-        if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache && (T == tGateL2 || p.alpha2_shared)) {
-            const int nu = (p.alpha_cols + 7) / 8, half = Cfg::kAlphaCache / 2;
+        if (acached && (T == tGateL2 || p.alpha2_shared)) {
+            const int nu = (acols + 7) / 8, half = Cfg::kAlphaCache / 2;
             for (int i = threadIdx.x; i < 8 * nu; i += blockDim.x) {
                 const int u = i >> 3, e = i & 7, at = (e < 4 ? 0 : half) + 4 * u + (e & 3);
-                s_alpha[at] = i < p.alpha_cols ? __ldg(p.alpha_shared + i) : 0.f;
+                s_alpha[at] = i < acols ? __ldg(p.alpha_shared + ac0 + i) : 0.f;
                 if constexpr (T == tSwigluL2)
-                    s_alpha[Cfg::kAlphaCache + at] = i < p.alpha_cols ? __ldg(p.alpha2_shared + i) : 0.f;
+                    s_alpha[Cfg::kAlphaCache + at] = i < acols ? __ldg(p.alpha2_shared + ac0 + i) : 0.f;
             }
         }
     }
     __syncthreads();
+    if (split) {
+        // every CTA of the cluster has initialised its barriers before any
+        // peer arrives on them
+        cluster_arrive();
+        cluster_wait();
+    }
 
     using Layout = TileLayout<T>;
     bool ok = true;
@@ -1383,10 +1629,12 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
             }
             int s = 0;
             uint32_t phase = 0;             // parity of the release a refill of position s waits for
-            int64_t slot = blockIdx.x;
-            for (int64_t j = 0; j < mine; ++j, slot += gridDim.x) {
+            int64_t slot = cid;
+            for (int64_t j = 0; j < mine; ++j, slot += ncl) {
                 if (j >= nslots && (abort_flag || !mbar_wait_bounded(&empty[s], phase, p.wait_limit_ns))) {
                     ok = false;
+                    if (split && !abort_flag)
+                        ctx.abort_all();
                     abort_flag = 1;
                     break;
                 }
@@ -1400,14 +1648,18 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                     seg_rows = sg.rows;
                     rps = sg.group;         // rows per slot for this segment
                     const bool has_r = seg_has_r(sg);
+                    // this CTA's slice of the row: units [u0, u0 + nuk)
+                    const int per = slice_per(sg.nu, static_cast<int>(ncta));
+                    const int u0 = min(sg.nu, static_cast<int>(rank) * per);
+                    const int nuk = min(sg.nu, u0 + per) - u0;
                     uint32_t o = 0u;
 #pragma unroll
                     for (int a2 = 0; a2 < NA; ++a2) {
                         const int u = Layout::ub(a2, has_r);
-                        pitch[a2] = (static_cast<uint32_t>(sg.nu) * u + 15u) & ~15u;
-                        src[a2] = pitch[a2] ? tile_src<T>(sg, a2, 0) : nullptr;
+                        pitch[a2] = (static_cast<uint32_t>(nuk) * u + 15u) & ~15u;
+                        src[a2] = pitch[a2] ? tile_src<T>(sg, a2, 0) + static_cast<int64_t>(u0) * u : nullptr;
                         spitch[a2] = tile_src_pitch<T>(sg, a2);
-                        contig[a2] = spitch[a2] == static_cast<int64_t>(pitch[a2]);
+                        contig[a2] = !split && spitch[a2] == static_cast<int64_t>(pitch[a2]);
                         off[a2] = o;
                         o += pitch[a2] * rps;
                     }
@@ -1450,14 +1702,19 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
         // takes slots j = q, q + kGroups, ... in order
         constexpr int NG = Cfg::kGroups;
         const int q = warp / WP, wi = warp % WP;
-        Team<WP> tm{wi * 32 + lane, 1 + q, red + q * Team<WP>::kRed};
+        Team<WP, SPLIT> tm{wi * 32 + lane, 1 + q, red + q * Team<WP>::kRed};
+        if constexpr (SPLIT) {
+            tm.ctx = &ctx;
+            tm.xbuf = reinterpret_cast<float *>(xarea + q * kXchgBytesPerTeam);
+            tm.xbar = reinterpret_cast<uint64_t *>(xarea + q * kXchgBytesPerTeam + kXchgFloats * 4);
+        }
         bool store = true;
         bool ws_first = true; // slerp backward: this team's dalpha line not yet written
         int vb = 0;
         for (int64_t j = q; j < mine; j += NG, vb ^= 1) {
             const int s = static_cast<int>(j % nslots);
             const uint32_t phase = static_cast<uint32_t>((j / nslots) & 1);
-            bool got = !abort_flag && mbar_wait_bounded(&full[s], phase, p.wait_limit_ns);
+            bool got = !abort_flag && !tm.failed && mbar_wait_bounded(&full[s], phase, p.wait_limit_ns);
             got = __all_sync(0xffffffffu, got);
             if constexpr (WP > 1) {
                 // all warps of the team take the same decision (their row
@@ -1472,25 +1729,37 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
             }
             if (!got) {
                 // nothing more will arrive: store nothing from here on, but
-                // keep releasing positions so that every wait ends
+                // keep releasing positions so that every wait ends; the
+                // peers of a cluster are told, so that none waits for this
+                // CTA's part of an exchange
                 ok = false;
+                if (split && !abort_flag && tm.t == 0)
+                    ctx.abort_all();
                 abort_flag = 1;
                 store = false;
             }
             const SlotHdr h = got ? hdr[s] : SlotHdr{0, 0, 0};
-            const auto &sg = p.seg[h.seg];
-            const bool has_r = seg_has_r(sg);
-            const int rps = sg.group;
+            const auto &sg0 = p.seg[h.seg];
+            const bool has_r = seg_has_r(sg0);
+            const int rps = sg0.group;
+            // this CTA's slice of the rows
+            int nuk = sg0.nu, c0 = 0, colsk = sg0.cols;
+            if constexpr (SPLIT) {
+                const int per = slice_per(sg0.nu, static_cast<int>(ncta));
+                const int ub0 = min(sg0.nu, static_cast<int>(rank) * per);
+                nuk = min(sg0.nu, ub0 + per) - ub0;
+                c0 = E * ub0;
+                colsk = max(0, min(sg0.cols - c0, E * nuk));
+            }
             unsigned char *base = ring + static_cast<size_t>(s) * slot_bytes;
             const int u0 = Layout::ub(0, has_r), u1 = Layout::kArrays > 1 ? Layout::ub(1, has_r) : 0;
             const int u2 = Layout::kArrays > 2 ? Layout::ub(2, has_r) : 0;
-            const int pitch0 = (sg.nu * u0 + 15) & ~15;
-            const int pitch1 = (sg.nu * u1 + 15) & ~15;
-            const int pitch2 = (sg.nu * u2 + 15) & ~15;
+            const int pitch0 = (nuk * u0 + 15) & ~15;
+            const int pitch1 = (nuk * u1 + 15) & ~15;
+            const int pitch2 = (nuk * u2 + 15) & ~15;
             unsigned char *a1 = base + pitch0 * rps;
             unsigned char *a2p = a1 + pitch1 * rps;
-            constexpr int E = is_weight_tag(T) ? 4 : 8;
-            const int nfull = sg.cols / E, tail = sg.cols % E;
+            const int nfull = colsk / E, tail = colsk % E;
             // hand the position back: the slot may hold this warp's
             // generic-proxy writes (s, t, masked tails), so order them
             // before the next bulk copy into it
@@ -1503,6 +1772,9 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                 released = true;
             };
             float g_lane = 1.f;
+            // the rows, through the segment itself or (a slice per CTA) a
+            // view of it moved to the slice's first column
+            auto rows = [&](const auto &sg) {
             for (int r = 0; r < h.nrows; ++r) {
                 const int64_t row = h.row0 + r;
                 unsigned char *s0 = base + r * pitch0;
@@ -1536,7 +1808,7 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                 } else if constexpr (T == tGateL2 || T == tSwigluL2) {
                     constexpr int PRO = T == tGateL2 ? 0 : 1;
                     constexpr int H = Cfg::kAlphaCache / 2;
-                    if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache && (PRO == 0 || p.alpha2_shared))
+                    if (cached() && (PRO == 0 || p.alpha2_shared))
                         tile_fused_row<WP, PRO, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
                                                       s_alpha + Cfg::kAlphaCache, H);
                     else
@@ -1548,76 +1820,180 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                     else
                         tile_l2_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
                 } else if constexpr (T == tSlerpBwd) {
-                    float *wsl = p.ws ? p.ws + (static_cast<int64_t>(blockIdx.x) * NG + q) * p.ws_ld : nullptr;
-                    if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache)
+                    // this team's dalpha line (one per cluster and team; each
+                    // CTA of the cluster writes its slice of the columns)
+                    float *wsl = p.ws ? p.ws + (cid * NG + q) * p.ws_ld + c0 : nullptr;
+                    if (cached())
                         tile_slerp_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, s_alpha,
                                                      Cfg::kAlphaCache / 2, wsl, ws_first);
                     else
                         tile_slerp_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, nullptr, 0,
                                                       wsl, ws_first);
                     ws_first = false;
-                } else if (p.alpha_shared && p.alpha_cols <= Cfg::kAlphaCache) {
+                } else if (cached()) {
                     tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
                                              Cfg::kAlphaCache / 2);
                 } else {
                     tile_slerp_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr, 0);
                 }
             }
+            };
+            if constexpr (SPLIT)
+                rows(shifted<T>(sg0, c0, colsk, nuk));
+            else
+                rows(sg0);
             if (!released)
                 release();
         }
+        if (tm.failed)
+            ok = false;
     }
     if (!ok)
         raise_device_error(DS_ERR_DEVICE_TIMEOUT, kSiteTileWait);
+    if (split) {
+        // no CTA leaves while a peer may still write into its shared memory
+        __syncwarp();
+        cluster_arrive();
+        cluster_wait();
+    }
 }
 
 } // namespace
 
+// Clusters of `cluster` CTAs of k_tile<T, SB> that fit the device at once,
+// looked up once per device and cluster size.
 template <int T, int SB>
-static cudaError_t launch_tile_sb(const TParams<T> &p, int grid, void *stream)
+static cudaError_t resident_clusters(int cluster, int smem, int *n)
+{
+    static std::atomic<int> cache[64][4];
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    const int ci = cluster == 2 ? 0 : cluster == 4 ? 1 : cluster == 8 ? 2 : 3;
+    if (dev >= 0 && dev < 64 && ci < 3) {
+        const int c = cache[dev][ci].load(std::memory_order_relaxed);
+        if (c > 0) {
+            *n = c;
+            return cudaSuccess;
+        }
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cluster), 1, 1);
+    cfg.blockDim = dim3(TileCfg<T, SB>::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    e = cudaOccupancyMaxActiveClusters(&c, k_tile<T, SB, true>, &cfg);
+    if (e != cudaSuccess)
+        return e;
+    if (c <= 0)
+        return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < 64 && ci < 3)
+        cache[dev][ci].store(c, std::memory_order_relaxed);
+    *n = c;
+    return cudaSuccess;
+}
+
+static int device_sms()
+{
+    static std::atomic<int> cache[64];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return 148;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+template <int T, int SB>
+static cudaError_t launch_tile_sb(const TParams<T> &p, int64_t units, int cluster, int *used, void *stream)
 {
     using Cfg = TileCfg<T, SB>;
-    constexpr int smem = Cfg::kSmem;
-    static DeviceFlags attr_set;
-    if (const cudaError_t e = enable_dynamic_smem(k_tile<T, SB>, smem, attr_set))
-        return e;
-    k_tile<T, SB><<<grid, Cfg::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
-    return cudaGetLastError();
+    if (cluster == 1) {
+        constexpr int smem = Cfg::kSmem;
+        static DeviceFlags attr_set;
+        if (const cudaError_t e = enable_dynamic_smem(k_tile<T, SB, false>, smem, attr_set))
+            return e;
+        const int grid = static_cast<int>(std::min<int64_t>(device_sms(), units));
+        *used = grid;
+        k_tile<T, SB, false><<<grid, Cfg::kThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
+        return cudaGetLastError();
+    }
+    if constexpr (SB > kTileSlotMaxBytes) {
+        return cudaErrorInvalidValue;   // slices of a row split over a cluster take at most 64 KB
+    } else {
+        constexpr int smem = Cfg::kSmem + tile_xchg_bytes<T, SB>();
+        static DeviceFlags attr_set;
+        if (const cudaError_t e = enable_dynamic_smem(k_tile<T, SB, true>, smem, attr_set))
+            return e;
+        int resident = 0;
+        if (const cudaError_t e = resident_clusters<T, SB>(cluster, smem, &resident))
+            return e;
+        const int64_t ncl = std::min<int64_t>(resident, units);
+        *used = static_cast<int>(ncl);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(ncl * cluster), 1, 1);
+        cfg.blockDim = dim3(Cfg::kThreads, 1, 1);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+        cfg.stream = static_cast<cudaStream_t>(stream);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, k_tile<T, SB, true>, p);
+    }
 }
 
 template <int T>
-static cudaError_t launch_tile_t(const void *params, int grid, int slot_bytes, void *stream)
+static cudaError_t launch_tile_t(const void *params, int64_t units, int slot_bytes, int cluster, int *used,
+                                 void *stream)
 {
     const TParams<T> &p = *static_cast<const TParams<T> *>(params);
+    if (cluster != 1 && cluster != 2 && cluster != 4 && cluster != 8)
+        return cudaErrorInvalidValue;
     switch (slot_bytes) {
-    case 16384: return launch_tile_sb<T, 16384>(p, grid, stream);
-    case 32768: return launch_tile_sb<T, 32768>(p, grid, stream);
-    case 65536: return launch_tile_sb<T, 65536>(p, grid, stream);
+    case 16384: return launch_tile_sb<T, 16384>(p, units, cluster, used, stream);
+    case 32768: return launch_tile_sb<T, 32768>(p, units, cluster, used, stream);
+    case 65536: return launch_tile_sb<T, 65536>(p, units, cluster, used, stream);
     case 114688:
         if constexpr (is_weight_tag(T))
-            return launch_tile_sb<T, 114688>(p, grid, stream);
+            return launch_tile_sb<T, 114688>(p, units, cluster, used, stream);
         else
             return cudaErrorInvalidValue;
     default: return cudaErrorInvalidValue;
     }
 }
 
-int launch_tile(int tag, const void *params, int grid, int slot_bytes, void *stream)
+int launch_tile(int tag, const void *params, int64_t units, int slot_bytes, int cluster, int *used, void *stream)
 {
     switch (tag) {
-    case tFwdBf16: return launch_tile_t<tFwdBf16>(params, grid, slot_bytes, stream);
-    case tFwdF32: return launch_tile_t<tFwdF32>(params, grid, slot_bytes, stream);
-    case tBwdBf16: return launch_tile_t<tBwdBf16>(params, grid, slot_bytes, stream);
-    case tBwdF32: return launch_tile_t<tBwdF32>(params, grid, slot_bytes, stream);
-    case tRenorm: return launch_tile_t<tRenorm>(params, grid, slot_bytes, stream);
-    case tL2: return launch_tile_t<tL2>(params, grid, slot_bytes, stream);
-    case tSlerp: return launch_tile_t<tSlerp>(params, grid, slot_bytes, stream);
-    case tProject: return launch_tile_t<tProject>(params, grid, slot_bytes, stream);
-    case tMomentum: return launch_tile_t<tMomentum>(params, grid, slot_bytes, stream);
-    case tL2Bwd: return launch_tile_t<tL2Bwd>(params, grid, slot_bytes, stream);
-    case tSlerpBwd: return launch_tile_t<tSlerpBwd>(params, grid, slot_bytes, stream);
-    case tGateL2: return launch_tile_t<tGateL2>(params, grid, slot_bytes, stream);
-    case tSwigluL2: return launch_tile_t<tSwigluL2>(params, grid, slot_bytes, stream);
+    case tFwdBf16: return launch_tile_t<tFwdBf16>(params, units, slot_bytes, cluster, used, stream);
+    case tFwdF32: return launch_tile_t<tFwdF32>(params, units, slot_bytes, cluster, used, stream);
+    case tBwdBf16: return launch_tile_t<tBwdBf16>(params, units, slot_bytes, cluster, used, stream);
+    case tBwdF32: return launch_tile_t<tBwdF32>(params, units, slot_bytes, cluster, used, stream);
+    case tRenorm: return launch_tile_t<tRenorm>(params, units, slot_bytes, cluster, used, stream);
+    case tL2: return launch_tile_t<tL2>(params, units, slot_bytes, cluster, used, stream);
+    case tSlerp: return launch_tile_t<tSlerp>(params, units, slot_bytes, cluster, used, stream);
+    case tProject: return launch_tile_t<tProject>(params, units, slot_bytes, cluster, used, stream);
+    case tMomentum: return launch_tile_t<tMomentum>(params, units, slot_bytes, cluster, used, stream);
+    case tL2Bwd: return launch_tile_t<tL2Bwd>(params, units, slot_bytes, cluster, used, stream);
+    case tSlerpBwd: return launch_tile_t<tSlerpBwd>(params, units, slot_bytes, cluster, used, stream);
+    case tGateL2: return launch_tile_t<tGateL2>(params, units, slot_bytes, cluster, used, stream);
+    case tSwigluL2: return launch_tile_t<tSwigluL2>(params, units, slot_bytes, cluster, used, stream);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -196,10 +196,11 @@ def wide(seed: int = 0) -> Workload:
     return Workload("wide", 1e-6, segs, acts)
 
 
-def long_rows(seed: int = 0, w_rows: int = 6, w_cols: int = 131072,
+def long_rows(seed: int = 0, w_rows: int = 6, w_cols: int = 262144,
               a_rows: int = 4, a_cols: int = 262144) -> Workload:
-    """Rows past the single-pass limit: fp32 weights [6, 131072] with gains and
-    bf16 GY, bf16 activations [4, 262144] with alpha."""
+    """Rows past the single-pass limit (more than 8 CTAs' staged slices):
+    fp32 weights [6, 262144] with gains and bf16 GY, bf16 activations
+    [4, 262144] with alpha."""
     rng = _rng(seed)
     w = drifted_rows(rng, w_rows, w_cols, 0.02)
     seg = WeightSeg("w_long", w, gains(rng, w_rows), normal_bf16(rng, (w_rows, w_cols), 1e-3))

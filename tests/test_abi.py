@@ -53,13 +53,17 @@ A_OPS = (ds.DS_OP_L2_ROWS, ds.DS_OP_SLERP_ROWS)
     (ds.DS_OP_L2_ROWS, 16384, (ds.DS_PATH_CTA, 256, 1)),      # 64 KB slots, 8 warps
     (ds.DS_OP_WN_FORWARD, 14336, (ds.DS_PATH_CTA, 128, 1)),   # 56 KB: 64 KB slots, 4 warps
     (ds.DS_OP_WN_BACKWARD, 14336, (ds.DS_PATH_CTA, 256, 1)),  # 112 KB (fp32 GY layout): 112 KB slots, 8 warps
-    (ds.DS_OP_WN_BACKWARD, 14337, (ds.DS_PATH_CLUSTER, 0, 4)),
-    (ds.DS_OP_WN_FORWARD, 131072, (ds.DS_PATH_TWO_PASS, 0, 8)),
+    (ds.DS_OP_WN_BACKWARD, 14337, (ds.DS_PATH_CLUSTER, 128, 2)),   # two 56 KB slices: 64 KB slots
+    (ds.DS_OP_WN_FORWARD, 131072, (ds.DS_PATH_CLUSTER, 128, 8)),   # eight 64 KB slices
+    (ds.DS_OP_WN_FORWARD, 131073, (ds.DS_PATH_TWO_PASS, 0, 8)),
     (ds.DS_OP_GRAD_PROJECT, 2048, (ds.DS_PATH_WARP, 32, 1)),  # w + G fp32 = 16 KB
     (ds.DS_OP_RENORM_MOMENTUM, 2049, (ds.DS_PATH_CTA, 64, 1)),
     (ds.DS_OP_GRAD_PROJECT, 14336, (ds.DS_PATH_CTA, 256, 1)),
-    (ds.DS_OP_GRAD_PROJECT, 16384, (ds.DS_PATH_CLUSTER, 0, 4)),
+    (ds.DS_OP_GRAD_PROJECT, 16384, (ds.DS_PATH_CLUSTER, 128, 2)),
     (ds.DS_OP_RENORM_MOMENTUM, 65537, (ds.DS_PATH_TWO_PASS, 0, 8)),
+    (ds.DS_OP_SLERP_ROWS, 16385, (ds.DS_PATH_CLUSTER, 256, 2)),
+    (ds.DS_OP_L2_ROWS_BACKWARD, 16384, (ds.DS_PATH_CLUSTER, 256, 2)),  # x, r, dy: 96 KB in two slices
+    (ds.DS_OP_SWIGLU_L2_ROWS, 131072, (ds.DS_PATH_CLUSTER, 256, 8)),
     (ds.DS_OP_SLERP_ROWS, 262144, (ds.DS_PATH_TWO_PASS, 0, 8)),
 ])
 def test_row_class_for_workload_shapes(op, cols, want):
@@ -67,20 +71,26 @@ def test_row_class_for_workload_shapes(op, cols, want):
 
 
 def test_row_class_is_monotone_and_fits():
-    """Staged classes take rows by their staged bytes (the smallest slot of
-    16, 32 or 64 KB that holds one row, a team of warps per row); longer rows
-    go to clusters whose CTAs hold at most kmax units per thread, then to the
-    two-pass class.  The class never shrinks as rows grow."""
+    """Staged classes take rows by their staged bytes: one CTA per row in the
+    smallest slot of 16, 32 or 64 KB (112 KB for weights) that holds the row;
+    longer rows are split over the smallest cluster of 2, 4 or 8 CTAs whose
+    slices (units rounded up to an even count) fit 64 KB, in the smallest
+    slot that holds a slice; then the two-pass class.  The class never
+    shrinks as rows grow."""
     order = {ds.DS_PATH_WARP: 0, ds.DS_PATH_CTA: 1, ds.DS_PATH_CLUSTER: 2, ds.DS_PATH_TWO_PASS: 3}
     for op in W_OPS + A_OPS:
         e = 4 if op in W_OPS else 8
         base = 1 if op in W_OPS else 2
-        kmax = 8 if op in (ds.DS_OP_WN_FORWARD, ds.DS_OP_ROW_RENORM) else 4
+        ub = 16 if op in (ds.DS_OP_WN_FORWARD, ds.DS_OP_ROW_RENORM) else 32
         prev = (0, 0, 0)
         for cols in sorted(set(list(range(1, 600, 7)) + [2 ** k + d for k in range(9, 19) for d in (-1, 0, 1)])):
             path, g, cl = ds.ds_row_class(op, cols)
             nu = -(-cols // e)
-            staged = (16 if op in (ds.DS_OP_WN_FORWARD, ds.DS_OP_ROW_RENORM) else 32) * nu
+            staged = ub * nu
+
+            def slice_bytes(n):
+                return ub * ((-(-nu // n) + 1) // 2 * 2)
+
             if path == ds.DS_PATH_WARP:
                 assert staged <= 16384 and g == 32 * base and cl == 1
             elif path == ds.DS_PATH_CTA:
@@ -90,10 +100,13 @@ def test_row_class_is_monotone_and_fits():
                 assert 16384 < staged <= top and g == 32 * warps and cl == 1
             elif path == ds.DS_PATH_CLUSTER:
                 top = 114688 if op in W_OPS else 65536
-                assert staged > top and -(-nu // cl) <= 256 * kmax and cl in (2, 4, 8)
+                assert staged > top and cl in (2, 4, 8)
+                assert slice_bytes(cl) <= 65536 and (cl == 2 or slice_bytes(cl // 2) > 65536)
+                slot = next(x for x in (16384, 32768, 65536) if slice_bytes(cl) <= x)
+                assert g == 32 * base * slot // 16384
             else:
-                assert -(-nu // 8) > 256 * kmax
-            key = (order[path], g, cl)
+                assert slice_bytes(8) > 65536
+            key = (order[path], cl)
             assert key >= prev, (op, cols)
             prev = key
 
@@ -101,8 +114,8 @@ def test_row_class_is_monotone_and_fits():
 def test_forced_paths():
     with ds.force_path(ds.DS_PATH_TWO_PASS):
         assert ds.ds_row_class(ds.DS_OP_L2_ROWS, 128)[0] == ds.DS_PATH_TWO_PASS
-    with ds.force_path(ds.DS_PATH_CLUSTER):
-        assert ds.ds_row_class(ds.DS_OP_WN_FORWARD, 768) == (ds.DS_PATH_CLUSTER, 0, 2)
+    with ds.force_path(ds.DS_PATH_CLUSTER):       # two 1.5 KB slices in 16 KB slots
+        assert ds.ds_row_class(ds.DS_OP_WN_FORWARD, 768) == (ds.DS_PATH_CLUSTER, 32, 2)
     with ds.force_path(ds.DS_PATH_WARP):  # does not fit: automatic choice
         assert ds.ds_row_class(ds.DS_OP_L2_ROWS, 8192)[0] == ds.DS_PATH_CTA
     with ds.force_path(ds.DS_PATH_CTA):
@@ -303,9 +316,13 @@ def test_backward_row_classes():
     assert ds.ds_row_class(ds.DS_OP_SLERP_ROWS_BACKWARD, 4096) == (ds.DS_PATH_CTA, 128, 1)
     assert ds.ds_row_class(ds.DS_OP_SLERP_ROWS_BACKWARD, 7168) == (ds.DS_PATH_CTA, 256, 1)
     assert ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 10920)[0] == ds.DS_PATH_CTA
+    # longer rows: 2, 4 or 8 CTAs, each staging a slice of at most 64 KB
+    assert ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 10921) == (ds.DS_PATH_CLUSTER, 256, 2)
+    assert ds.ds_row_class(ds.DS_OP_SLERP_ROWS_BACKWARD, 16384) == (ds.DS_PATH_CLUSTER, 256, 2)
+    assert ds.ds_row_class(ds.DS_OP_SLERP_ROWS_BACKWARD, 87296) == (ds.DS_PATH_CLUSTER, 256, 8)
     with pytest.raises(ds.DSError):
-        ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 10921)
-    with ds.force_path(ds.DS_PATH_TWO_PASS):   # no cluster classes: the staged one is kept
+        ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 87297)
+    with ds.force_path(ds.DS_PATH_TWO_PASS):   # no two-pass class: the staged one is kept
         assert ds.ds_row_class(ds.DS_OP_L2_ROWS_BACKWARD, 128)[0] == ds.DS_PATH_WARP
 
 
@@ -320,11 +337,11 @@ def test_backward_validation(fn):
     assert call_g(fn, [agseg(dx=0, **good)]) == E.DS_ERR_INVALID_ARG
     assert call_g(fn, [agseg(dy=0, **good)]) == E.DS_ERR_INVALID_ARG
     assert call_g(fn, [agseg(dx=BASE + (2 << 30) + 4, **good)]) == E.DS_ERR_ALIGNMENT
-    if slerp:   # x, r, dy staged: 10,920 columns at most
-        assert call_g(fn, [agseg(cols=10921, ld=10928, ld_d=10924, **good)]) == E.DS_ERR_INVALID_ARG
-    else:       # without a residual x and dy: 16,384 columns; with one 10,920
-        assert call_g(fn, [agseg(cols=16385, ld=16392, ld_d=16388)]) == E.DS_ERR_INVALID_ARG
-        assert call_g(fn, [agseg(cols=10921, ld=10928, ld_d=10924, r=BASE + (5 << 30))]) == E.DS_ERR_INVALID_ARG
+    if slerp:   # x, r, dy staged in 8 slices of 64 KB: 87,296 columns at most
+        assert call_g(fn, [agseg(cols=87297, ld=87304, ld_d=87300, **good)]) == E.DS_ERR_INVALID_ARG
+    else:       # without a residual x and dy: 131,072 columns; with one 87,296
+        assert call_g(fn, [agseg(cols=131073, ld=131080, ld_d=131076)]) == E.DS_ERR_INVALID_ARG
+        assert call_g(fn, [agseg(cols=87297, ld=87304, ld_d=87300, r=BASE + (5 << 30))]) == E.DS_ERR_INVALID_ARG
     # dx over an input
     assert call_g(fn, [agseg(dx=BASE + (1 << 30), **good)]) == E.DS_ERR_OVERLAP
     assert call_g(fn, [agseg(rows=0, x=0, dy=0, dx=0, dr=0, **good)]) == E.DS_OK
@@ -365,8 +382,10 @@ def test_fused_row_classes():
     assert ds.ds_row_class(ds.DS_OP_GATE_L2_ROWS, 4096) == (ds.DS_PATH_WARP, 64, 1)
     assert ds.ds_row_class(ds.DS_OP_SWIGLU_L2_ROWS, 7168) == (ds.DS_PATH_CTA, 128, 1)
     assert ds.ds_row_class(ds.DS_OP_SWIGLU_L2_ROWS, 16384) == (ds.DS_PATH_CTA, 256, 1)
+    assert ds.ds_row_class(ds.DS_OP_GATE_L2_ROWS, 16385) == (ds.DS_PATH_CLUSTER, 256, 2)
+    assert ds.ds_row_class(ds.DS_OP_GATE_L2_ROWS, 131072) == (ds.DS_PATH_CLUSTER, 256, 8)
     with pytest.raises(ds.DSError):
-        ds.ds_row_class(ds.DS_OP_GATE_L2_ROWS, 16385)
+        ds.ds_row_class(ds.DS_OP_GATE_L2_ROWS, 131073)
 
 
 @pytest.mark.parametrize("fn", ["ds_gate_l2_rows", "ds_swiglu_l2_rows"])
@@ -380,7 +399,7 @@ def test_fused_validation(fn):
     assert call_f(fn, [fseg(sa=0)]) == E.DS_ERR_INVALID_ARG
     assert call_f(fn, [fseg(sa=BASE + (3 << 30) + 4)]) == E.DS_ERR_ALIGNMENT
     assert call_f(fn, [fseg(a=BASE + 2)]) == E.DS_ERR_ALIGNMENT
-    assert call_f(fn, [fseg(cols=16385, ld=16392)]) == E.DS_ERR_INVALID_ARG
+    assert call_f(fn, [fseg(cols=131073, ld=131080)]) == E.DS_ERR_INVALID_ARG   # past 8 slices of 64 KB
     assert call_f(fn, [fseg(y=BASE + 16)]) == E.DS_ERR_OVERLAP            # partial overlap with a
     assert call_f(fn, [fseg()], eps=-1.0) == E.DS_ERR_INVALID_ARG
     if fn == "ds_swiglu_l2_rows":

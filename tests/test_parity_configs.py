@@ -7,7 +7,8 @@ in blocks of rows to bound host memory):
 * activation rows [16384,4096] with 1% of rows scaled by 1e3;
 * the whole 12-layer d_model-768 decoder: 85 weight segments in one call;
 * wide rows: weights [14336,4096], [4096,14336]; activations [8192,7168], [4096,16384];
-* rows past the single-pass limit: [6,131072] fp32 weights, [4,262144] bf16 activations.
+* rows past the staged classes (more than 8 slices of 64 KB): [6,262144] fp32 weights, [4,262144] bf16
+  activations (the two-pass stream).
 
 The forced two-pass runs on the wide shapes repeat a path the long rows
 already cover in full, and stay sampled.

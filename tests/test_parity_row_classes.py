@@ -3,9 +3,10 @@ the float64 oracle element by element.
 
 The class of a row depends on (operation, cols) alone.  `AUTO_CASES` lists,
 per operation, widths that land in each class the planner can pick (staged
-slots of 16 to 112 KB, register clusters of 4 and 8 CTAs with their
-partial sums meeting in distributed shared memory, the two-pass stream); a
-CPU test walks every width up to 70,000 columns and fails if a class has no
+slots of 16 to 112 KB, clusters of 2, 4 and 8 CTAs that each stage a slice
+of the row, their partial sums meeting in distributed shared memory, the
+two-pass stream); a
+CPU test walks every width up to 140,000 columns and fails if a class has no
 case here.  The GPU tests run each case with ragged column counts, padded
 leading dimensions and canary guard rows, then check the cluster widths
 for the two bit-exact invariants (TensorFold PR #1260: "a row's bits never
@@ -24,27 +25,36 @@ from l2_row_b200 import workloads as wl
 W, C, T = ds.DS_PATH_WARP, ds.DS_PATH_CTA, ds.DS_PATH_CLUSTER
 P2 = ds.DS_PATH_TWO_PASS
 
-# (operation, cols, expected (path, threads per row, CTAs per row))
+# (operation, cols, expected (path, threads per row, CTAs per row)); the
+# activation backward and Dory cases run on dense matrices, so their widths
+# keep rows 16-byte aligned (multiples of 8)
 AUTO_CASES = {
     "fwd": [(768, (W, 32, 1)), (4100, (C, 64, 1)), (8200, (C, 128, 1)), (16390, (C, 256, 1)),
-            (28680, (T, 0, 4)), (32768, (T, 0, 4)), (40001, (T, 0, 8)), (65536, (T, 0, 8)),
-            (65541, (P2, 0, 8))],
+            (28680, (T, 128, 2)), (32768, (T, 128, 2)), (40001, (T, 128, 4)), (65536, (T, 128, 4)),
+            (65541, (T, 128, 8)), (131072, (T, 128, 8)), (131077, (P2, 0, 8))],
     "bwd": [(1000, (W, 32, 1)), (3001, (C, 64, 1)), (6001, (C, 128, 1)), (12289, (C, 256, 1)),
-            (16384, (T, 0, 4)), (20003, (T, 0, 8)), (32768, (T, 0, 8)), (50000, (P2, 0, 8))],
+            (16384, (T, 128, 2)), (20003, (T, 128, 4)), (32768, (T, 128, 4)), (50000, (T, 128, 8)),
+            (65536, (T, 128, 8)), (65541, (P2, 0, 8))],
     "renorm": [(768, (W, 32, 1)), (4100, (C, 64, 1)), (8200, (C, 128, 1)), (16390, (C, 256, 1)),
-               (30001, (T, 0, 4)), (50003, (T, 0, 8)), (65537, (P2, 0, 8))],
-    "l2": [(1000, (W, 64, 1)), (6001, (C, 128, 1)), (12289, (C, 256, 1)), (16392, (T, 0, 4)),
-           (24579, (T, 0, 4)), (40000, (T, 0, 8)), (65536, (T, 0, 8)), (65543, (P2, 0, 8))],
-    "slerp": [(1000, (W, 64, 1)), (6001, (C, 128, 1)), (12289, (C, 256, 1)), (16392, (T, 0, 4)),
-              (24579, (T, 0, 4)), (40000, (T, 0, 8)), (65536, (T, 0, 8)), (65543, (P2, 0, 8))],
+               (30001, (T, 128, 2)), (50003, (T, 128, 4)), (100001, (T, 128, 8)), (131077, (P2, 0, 8))],
+    "l2": [(1000, (W, 64, 1)), (6001, (C, 128, 1)), (12289, (C, 256, 1)), (16392, (T, 256, 2)),
+           (24579, (T, 256, 2)), (40000, (T, 256, 4)), (65536, (T, 256, 4)), (65543, (T, 256, 8)),
+           (131072, (T, 256, 8)), (131079, (P2, 0, 8))],
+    "slerp": [(1000, (W, 64, 1)), (6001, (C, 128, 1)), (12289, (C, 256, 1)), (16392, (T, 256, 2)),
+              (24579, (T, 256, 2)), (40000, (T, 256, 4)), (65536, (T, 256, 4)), (65543, (T, 256, 8)),
+              (131072, (T, 256, 8)), (131079, (P2, 0, 8))],
     "project": [(1000, (W, 32, 1)), (3001, (C, 64, 1)), (6001, (C, 128, 1)), (12289, (C, 256, 1)),
-                (16384, (T, 0, 4)), (20003, (T, 0, 8)), (50000, (P2, 0, 8))],
+                (16384, (T, 128, 2)), (20003, (T, 128, 4)), (50000, (T, 128, 8)), (65541, (P2, 0, 8))],
     "momentum": [(1000, (W, 32, 1)), (3001, (C, 64, 1)), (6001, (C, 128, 1)), (12289, (C, 256, 1)),
-                 (16384, (T, 0, 4)), (20003, (T, 0, 8)), (50000, (P2, 0, 8))],
-    "l2_bwd": [(1000, (W, 64, 1)), (4001, (C, 128, 1)), (10920, (C, 256, 1))],
-    "slerp_bwd": [(1000, (W, 64, 1)), (4001, (C, 128, 1)), (10920, (C, 256, 1))],
-    "gate": [(1000, (W, 64, 1)), (7168, (C, 128, 1)), (16384, (C, 256, 1))],
-    "swiglu": [(1000, (W, 64, 1)), (7168, (C, 128, 1)), (16384, (C, 256, 1))],
+                 (16384, (T, 128, 2)), (20003, (T, 128, 4)), (50000, (T, 128, 8)), (65541, (P2, 0, 8))],
+    "l2_bwd": [(1000, (W, 64, 1)), (4008, (C, 128, 1)), (10920, (C, 256, 1)), (10928, (T, 256, 2)),
+               (16384, (T, 256, 2)), (30000, (T, 256, 4)), (50000, (T, 256, 8)), (87296, (T, 256, 8))],
+    "slerp_bwd": [(1000, (W, 64, 1)), (4008, (C, 128, 1)), (10920, (C, 256, 1)), (10928, (T, 256, 2)),
+                  (16384, (T, 256, 2)), (30000, (T, 256, 4)), (50000, (T, 256, 8)), (87296, (T, 256, 8))],
+    "gate": [(1000, (W, 64, 1)), (7168, (C, 128, 1)), (16384, (C, 256, 1)), (16392, (T, 256, 2)),
+             (40000, (T, 256, 4)), (100000, (T, 256, 8))],
+    "swiglu": [(1000, (W, 64, 1)), (7168, (C, 128, 1)), (16384, (C, 256, 1)), (16392, (T, 256, 2)),
+               (40000, (T, 256, 4)), (100000, (T, 256, 8))],
 }
 OPS = {"fwd": ds.DS_OP_WN_FORWARD, "bwd": ds.DS_OP_WN_BACKWARD, "renorm": ds.DS_OP_ROW_RENORM,
        "l2": ds.DS_OP_L2_ROWS, "slerp": ds.DS_OP_SLERP_ROWS, "project": ds.DS_OP_GRAD_PROJECT,
@@ -62,11 +72,11 @@ def row_class(op: str, cols: int):
 
 
 def test_every_auto_class_has_a_case():
-    """Walk every width up to 70,000 columns (and a few beyond): each class
+    """Walk every width up to 140,000 columns (and a few beyond): each class
     the planner picks has a case above, and each case is in its class."""
     assert set(AUTO_CASES) == set(OPS)
     for op, cases in AUTO_CASES.items():
-        picked = {row_class(op, c) for c in list(range(1, 70001)) + [131072, 262144, 1 << 20]}
+        picked = {row_class(op, c) for c in list(range(1, 140001)) + [262144, 1 << 20]}
         picked.discard(None)
         covered = {cls for _, cls in cases}
         assert picked == covered, (op, sorted(picked - covered), sorted(covered - picked))
@@ -199,8 +209,8 @@ def test_auto_class_matches_oracle(op, cols):
     assert ds.ds_get_device_status() == ds.DS_OK
 
 
-CLUSTER_WIDTHS = {"fwd": [30001, 40001, 65536], "bwd": [16384, 20003], "l2": [24579, 40000, 65536],
-                  "slerp": [24579, 40000, 65536]}
+CLUSTER_WIDTHS = {"fwd": [30001, 40001, 100001], "bwd": [16384, 20003, 50000], "l2": [24579, 40000, 100000],
+                  "slerp": [24579, 40000, 100000]}
 
 
 def _bits(t):
@@ -218,10 +228,18 @@ def test_cluster_rows_count_invariance(op):
     eps = 1e-6
     for cols in CLUSTER_WIDTHS[op]:
         R = 7
+        ld = _ld(cols)
+
+        def pad(t, canary):
+            return _padded_copy(t, ld, canary)[0]
+
+        def empty(dt):
+            return gu.padded(R, cols, ld, dt, gu.CANARY_BF16 if dt == torch.bfloat16 else gu.CANARY_F32)[0]
+
         if op in ("fwd", "bwd"):
-            w = gu.dev_f32(wl.drifted_rows(rng, R, cols, 0.02))
+            w = pad(gu.dev_f32(wl.drifted_rows(rng, R, cols, 0.02)), gu.CANARY_F32)
             g = gu.dev_f32(wl.gains(rng, R))
-            gy = gu.dev_bf16(wl.normal_bf16(rng, (R, cols), 1e-3))
+            gy = pad(gu.dev_bf16(wl.normal_bf16(rng, (R, cols), 1e-3)), gu.CANARY_BF16)
 
             def call(lo, hi, out, gout=None):
                 if op == "fwd":
@@ -232,8 +250,8 @@ def test_cluster_rows_count_invariance(op):
             fn = (lambda segs: ds.ds_wn_forward(segs, "bf16", eps)) if op == "fwd" else \
                  (lambda segs: ds.ds_wn_backward(segs, "bf16", eps))
         else:
-            x = gu.dev_bf16(wl.normal_bf16(rng, (R, cols)))
-            r = gu.dev_bf16(wl.normal_bf16(rng, (R, cols)))
+            x = pad(gu.dev_bf16(wl.normal_bf16(rng, (R, cols))), gu.CANARY_BF16)
+            r = pad(gu.dev_bf16(wl.normal_bf16(rng, (R, cols))), gu.CANARY_BF16)
             al = gu.dev_f32(wl.alpha_vec(rng, cols))
 
             def call(lo, hi, out, gout=None):
@@ -242,15 +260,15 @@ def test_cluster_rows_count_invariance(op):
             dt = torch.bfloat16
             fn = (lambda segs: ds.ds_slerp_rows(segs, eps)) if op == "slerp" else \
                  (lambda segs: ds.ds_l2_rows(segs, eps))
-        full = torch.empty(R, cols, dtype=dt, device="cuda")
+        full = empty(dt)
         gfull = torch.empty(R, device="cuda")
         fn([call(0, R, full, gfull)])
-        parts = torch.empty_like(full)
+        parts = empty(dt)
         gparts = torch.empty_like(gfull)
         cuts = [0, 1, 3, 4, 7]
         fn([call(a, b, parts, gparts) for a, b in zip(cuts, cuts[1:])])
         for k in (0, 4, 6):
-            one = torch.empty_like(full)
+            one = empty(dt)
             gone = torch.empty_like(gfull)
             fn([call(k, k + 1, one, gone)])
             torch.cuda.synchronize()
@@ -271,7 +289,7 @@ def test_cluster_rows_power_of_two_scale_invariance():
     from tests import gpu_util as gu
 
     rng = np.random.default_rng(72)
-    for cols in (30001, 40001, 65536):
+    for cols in (30004, 40004, 100004):       # dense fp32 rows: multiples of 4
         w = wl.drifted_rows(rng, 3, cols, 1.0)
         base = gu.run_forward([wl.WeightSeg("w", w, None, None)], "f32", 0.0)[0]
         for k in (-70, -20, 20, 70):
@@ -279,7 +297,7 @@ def test_cluster_rows_power_of_two_scale_invariance():
             assert np.array_equal(np.ldexp(ws, -k), w)
             got = gu.run_forward([wl.WeightSeg("w", ws, None, None)], "f32", 0.0)[0]
             assert torch.equal(got, base), (cols, k)
-    for cols in (24579, 40000, 65536):
+    for cols in (24584, 40000, 100000):       # dense bf16 rows: multiples of 8
         xf = wl.bf16_bits_to_f32(wl.normal_bf16(rng, (3, cols)))
         ybase = gu.run_l2([wl.ActRows("x", wl.to_bf16_bits(xf), None)], 0.0, residual=False)[0]
         for k in (-60, -20, 20, 60):
