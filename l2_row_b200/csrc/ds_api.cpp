@@ -558,39 +558,74 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
     };
     if (ds_status st = launch_all<WParams, WSegK>(nseg, rows.data(), cls, eps, make, launch, stream))
         return st;
-    // transposed rows: one launch over all of them (tiles of col_tile_rows())
+    // transposed rows: whole column tiles staged over a cluster where they
+    // fit shared memory (one launch per tile shape), else the column kernel
+    // (one launch over the rest, tiles of col_tile_rows())
     {
         static thread_local WParams tp;
-        const int tile = ds::col_tile_rows();
         const int cop = wop == W_FWD ? 0 : wop == W_BWD ? 1 : wop == W_RENORM ? 2 : wop == W_PROJECT ? 3 : 4;
-        int n = 0;
-        int64_t units = 0;
-        auto flush = [&]() -> ds_status {
-            if (n == 0)
-                return DS_OK;
-            tp.nseg = n;
-            tp.unit_start[n] = units;
-            tp.eps = eps;
-            if (ds::launch_col(cop, bf16, tp, units, stream) != 0)
-                return fail(DS_ERR_CUDA, "kernel launch failed (transposed rows)");
-            g_launches.fetch_add(1, std::memory_order_relaxed);
-            n = 0;
-            units = 0;
-            return DS_OK;
-        };
+        // bytes per element staged: w, and the second input (GY or the
+        // gradient / momentum) where the operation reads one
+        const int eb = 4 + (cop == 1 ? esize : (cop == 3 || cop == 4) ? 4 : 0);
+        std::vector<int> ct_of(static_cast<size_t>(nseg), 0), cl_of(static_cast<size_t>(nseg), 0);
         for (int i = 0; i < nseg; ++i) {
             if (!segs[i].transposed || segs[i].rows == 0)
                 continue;
-            if (n == ds::kSegPerLaunch)
+            const int64_t K = segs[i].cols;
+            for (const int ct : {128, 64, 32}) {
+                for (const int cl : {1, 2, 4, 8})
+                    if (ds::col_tile_smem(ct, cl, (K + cl - 1) / cl, eb) <= ds::kColTileSmemMax) {
+                        ct_of[i] = ct;
+                        cl_of[i] = cl;
+                        break;
+                    }
+                if (ct_of[i])
+                    break;
+            }
+        }
+        for (const int ct : {128, 64, 32, 0})
+            for (const int cl : {1, 2, 4, 8}) {
+                if (ct == 0 && cl != 1)
+                    continue;
+                int n = 0, smem = 0;
+                int64_t units = 0;
+                auto flush = [&]() -> ds_status {
+                    if (n == 0)
+                        return DS_OK;
+                    tp.nseg = n;
+                    tp.unit_start[n] = units;
+                    tp.eps = eps;
+                    tp.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+                    const int e = ct ? ds::launch_colt(cop, bf16, ct, cl, smem, tp, units, stream)
+                                     : ds::launch_col(cop, bf16, tp, units, stream);
+                    if (e != 0) {
+                        char buf[160];
+                        std::snprintf(buf, sizeof(buf), "kernel launch failed (transposed rows, cudaError %d)", e);
+                        return fail(DS_ERR_CUDA, buf);
+                    }
+                    g_launches.fetch_add(1, std::memory_order_relaxed);
+                    n = 0;
+                    units = 0;
+                    smem = 0;
+                    return DS_OK;
+                };
+                for (int i = 0; i < nseg; ++i) {
+                    if (!segs[i].transposed || segs[i].rows == 0 || ct_of[i] != ct || (ct && cl_of[i] != cl))
+                        continue;
+                    if (n == ds::kSegPerLaunch)
+                        if (ds_status st = flush())
+                            return st;
+                    const int tile = ct ? ct : ds::col_tile_rows();
+                    tp.seg[n] = make(i, 0, segs[i].rows);
+                    tp.unit_start[n] = units;
+                    units += (segs[i].rows + tile - 1) / tile;
+                    if (ct)
+                        smem = std::max(smem, ds::col_tile_smem(ct, cl, (segs[i].cols + cl - 1) / cl, eb));
+                    ++n;
+                }
                 if (ds_status st = flush())
                     return st;
-            tp.seg[n] = make(i, 0, segs[i].rows);
-            tp.unit_start[n] = units;
-            units += (segs[i].rows + tile - 1) / tile;
-            ++n;
-        }
-        if (ds_status st = flush())
-            return st;
+            }
     }
     if (wop != W_BWD)
         return DS_OK;

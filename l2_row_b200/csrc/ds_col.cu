@@ -183,6 +183,202 @@ __global__ void __launch_bounds__(kCta) k_col(const __grid_constant__ WParams p)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Transposed rows in column tiles staged whole.  A tile is CT consecutive
+// unit rows (stored columns c0 .. c0 + CT) over the whole unit-row length K
+// (every stored row); a cluster of CL CTAs owns one tile, CTA k staging the
+// band of stored rows [k * band, (k + 1) * band) of it in shared memory with
+// one bulk copy per stored row (CT * 4 contiguous bytes, and CT * 2 or 4 of
+// the second input), so HBM sees whole row pieces, each read once.  Each
+// CTA sums w^2 (and w . d) per column over its band in double (8 lanes down
+// the band, then a fixed tree), the CTAs' partials meet through distributed
+// shared memory and are added in rank order, and every CTA then scales its
+// staged band straight to global memory.  The results are those of the
+// column kernel above (double sums, each output its double value rounded
+// once), with the band and tree orders of this tiling.
+template <int OP>
+__host__ __device__ constexpr bool col_two() { return OP == 1 || OP == 3 || OP == 4; }
+
+template <int OP, bool B16, int CT>
+__global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ WParams p)
+{
+    constexpr bool TWO = col_two<OP>();
+    constexpr int Q = CT / 4;                      // column quads of a tile
+    constexpr int L = kCta / Q;                    // lanes down the band
+    static_assert(Q * L == kCta && Q <= 32, "tile shape");
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) uint64_t full;
+    __shared__ double red[2][L][CT];
+    __shared__ double fac[2][CT];
+    cluster_arrive_relaxed();
+    const uint32_t rank = cluster_ctarank(), ncta = cluster_nctarank();
+    const int64_t unit = blockIdx.x / ncta;
+    const int si = find_segment(p, unit);
+    const WSegK &sg = p.seg[si];
+    const int64_t c0 = (unit - p.unit_start[si]) * CT;          // first unit row of the tile
+    const int ncols = static_cast<int>(sg.rows - c0 < CT ? sg.rows - c0 : CT);
+    const int K = sg.cols;
+    const int band = (K + static_cast<int>(ncta) - 1) / static_cast<int>(ncta);
+    const int k0 = min(K, static_cast<int>(rank) * band), nk = min(K, k0 + band) - k0;
+    const bool d_bf16 = OP == 1 && B16;
+    const int64_t ld_d = OP == 1 ? sg.ld_out : sg.ld;
+    const int de = d_bf16 ? 2 : 4;
+    float *tw = reinterpret_cast<float *>(smem);                          // [band][CT]
+    unsigned char *td = smem + static_cast<size_t>(band) * CT * 4;        // [band][CT] d
+    double *xch = reinterpret_cast<double *>(td + (TWO ? static_cast<size_t>(band) * CT * de : 0));
+    // xch: [2][kMaxCluster][CT] the CTAs' partial sums, written by every peer
+
+    if (threadIdx.x == 0) {
+        mbar_init(&full, 1);
+        mbar_init_fence();
+    }
+    __syncthreads();
+    bool ok = true;
+    if (threadIdx.x == 0) {
+        const uint32_t wbytes = (static_cast<uint32_t>(ncols) * 4u + 15u) & ~15u;
+        const uint32_t dbytes = TWO ? (static_cast<uint32_t>(ncols) * de + 15u) & ~15u : 0u;
+        mbar_arrive_expect_tx(&full, (wbytes + dbytes) * static_cast<uint32_t>(nk));
+        for (int i = 0; i < nk; ++i) {
+            const int64_t j = k0 + i;
+            bulk_g2s(tw + static_cast<size_t>(i) * CT, sg.w + j * sg.ld + c0, wbytes, &full);
+            if constexpr (TWO)
+                bulk_g2s(td + static_cast<size_t>(i) * CT * de,
+                         static_cast<const char *>(sg.gy) + (j * ld_d + c0) * de, dbytes, &full);
+        }
+    }
+    if (!mbar_wait_bounded(&full, 0, p.wait_limit_ns)) {
+        ok = false;
+        // no copy may still be writing this CTA's shared memory when it
+        // leaves: wait (bounded) once more before going on without data
+        if (threadIdx.x == 0 && !mbar_wait_bounded(&full, 0, p.wait_limit_ns))
+            raise_device_error(DS_ERR_DEVICE_TIMEOUT, kSiteTileWait);
+    }
+    const int q = threadIdx.x % Q, ln = threadIdx.x / Q;
+    auto dval = [&](int i, int e) -> double {
+        if constexpr (TWO) {
+            if (d_bf16)
+                return static_cast<double>(bf_lo(reinterpret_cast<const uint16_t *>(td)[static_cast<size_t>(i) * CT + 4 * q + e]));
+            return static_cast<double>(reinterpret_cast<const float *>(td)[static_cast<size_t>(i) * CT + 4 * q + e]);
+        } else {
+            return 0.0;
+        }
+    };
+    // pass 1: this CTA's band, per column, in double
+    double s[4] = {0, 0, 0, 0}, dd[4] = {0, 0, 0, 0};
+    for (int i = ln; i < nk; i += L) {
+        const float4 w = *reinterpret_cast<const float4 *>(tw + static_cast<size_t>(i) * CT + 4 * q);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const double wi = comp(w, e);
+            s[e] = fma(wi, wi, s[e]);
+            if constexpr (TWO)
+                dd[e] = fma(wi, dval(i, e), dd[e]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        red[0][ln][4 * q + e] = s[e];
+        if constexpr (TWO)
+            red[1][ln][4 * q + e] = dd[e];
+    }
+    __syncthreads();
+    for (int o = L / 2; o > 0; o >>= 1) {
+        if (ln < o) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                red[0][ln][4 * q + e] += red[0][ln + o][4 * q + e];
+                if constexpr (TWO)
+                    red[1][ln][4 * q + e] += red[1][ln + o][4 * q + e];
+            }
+        }
+        __syncthreads();
+    }
+    // the band's partials to every CTA of the cluster (slot [rank])
+    cluster_wait();   // every peer has started (arrival at kernel start)
+    if (threadIdx.x < CT) {
+        const int c = threadIdx.x;
+        for (uint32_t k = 0; k < ncta; ++k) {
+            namespace cg = cooperative_groups;
+            double *x0 = cg::this_cluster().map_shared_rank(xch + rank * CT + c, static_cast<int>(k));
+            *x0 = red[0][0][c];
+            if constexpr (TWO) {
+                double *x1 = cg::this_cluster().map_shared_rank(xch + (kMaxCluster + rank) * CT + c, static_cast<int>(k));
+                *x1 = red[1][0][c];
+            }
+        }
+    }
+    cluster_arrive();
+    cluster_wait();
+    if (threadIdx.x < CT) {
+        const int c = threadIdx.x;
+        const int64_t r = c0 + c;
+        double S = xch[c], D = 0.0;
+        for (uint32_t k = 1; k < ncta; ++k)
+            S += xch[k * CT + c];
+        if constexpr (TWO) {
+            D = xch[kMaxCluster * CT + c];
+            for (uint32_t k = 1; k < ncta; ++k)
+                D += xch[(kMaxCluster + k) * CT + c];
+        }
+        if (r < sg.rows) {
+            S += static_cast<double>(p.eps);
+            const double n = sqrt(S);
+            const double g = (OP <= 1 && sg.gain) ? static_cast<double>(__ldg(sg.gain + r * sg.gain_stride)) : 1.0;
+            fac[0][c] = g * static_cast<double>(sg.radius) / n;
+            if constexpr (TWO)
+                fac[1][c] = D / S;
+            if constexpr (OP == 1) {
+                if (sg.gain && rank == 0 && ok)
+                    sg.grad_g[r] = static_cast<float>(static_cast<double>(sg.radius) * D / n);
+            }
+        } else {
+            fac[0][c] = 0.0;
+            fac[1][c] = 0.0;
+        }
+    }
+    __syncthreads();
+    ok = __syncthreads_and(ok) != 0;
+    if (ok) {
+        double sc[4], qt[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sc[e] = fac[0][4 * q + e];
+            if constexpr (TWO)
+                qt[e] = fac[1][4 * q + e];
+        }
+        const int valid = ncols - 4 * q >= 4 ? 4 : (ncols - 4 * q > 0 ? ncols - 4 * q : 0);
+        if (valid > 0) {
+            for (int i = ln; i < nk; i += L) {
+                const int64_t j = k0 + i;
+                const float4 w = *reinterpret_cast<const float4 *>(tw + static_cast<size_t>(i) * CT + 4 * q);
+                float y[4], ev[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const double wi = comp(w, e);
+                    y[e] = static_cast<float>(wi * sc[e]);
+                    if constexpr (TWO) {
+                        const double ei = dval(i, e) - wi * qt[e];
+                        ev[e] = static_cast<float>(OP == 1 ? sc[e] * ei : ei);
+                    }
+                }
+                const float4 yv = make_float4(y[0], y[1], y[2], y[3]);
+                const int64_t col = c0 + 4 * q;
+                if constexpr (OP == 0) {
+                    col_store<B16>(static_cast<char *>(sg.out) + (j * sg.ld_out + col) * (B16 ? 2 : 4), yv, valid);
+                } else if constexpr (OP == 2) {
+                    col_store<false>(const_cast<float *>(sg.w) + j * sg.ld + col, yv, valid);
+                } else {
+                    col_store<false>(sg.grad_w + j * sg.ld + col, make_float4(ev[0], ev[1], ev[2], ev[3]), valid);
+                    if constexpr (OP == 4)
+                        col_store<false>(const_cast<float *>(sg.w) + j * sg.ld + col, yv, valid);
+                }
+            }
+        }
+    } else if (threadIdx.x == 0) {
+        raise_device_error(DS_ERR_DEVICE_TIMEOUT, kSiteTileWait);
+    }
+}
+
 template <int OP, bool B16>
 cudaError_t launch_col_t(const WParams &p, int64_t units, cudaStream_t st)
 {
@@ -191,9 +387,64 @@ cudaError_t launch_col_t(const WParams &p, int64_t units, cudaStream_t st)
     return cudaGetLastError();
 }
 
+template <int OP, bool B16, int CT>
+cudaError_t launch_colt_t(const WParams &p, int64_t units, int cl, int smem, cudaStream_t st)
+{
+    static DeviceFlags attr_set;
+    if (const cudaError_t e = enable_dynamic_smem(k_colt<OP, B16, CT>, kColTileSmemMax, attr_set))
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(units * cl), 1, 1);
+    cfg.blockDim = dim3(kCta, 1, 1);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cl);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_colt<OP, B16, CT>, p);
+}
+
+template <int OP, bool B16>
+cudaError_t launch_colt_ct(const WParams &p, int64_t units, int ct, int cl, int smem, cudaStream_t st)
+{
+    switch (ct) {
+    case 32: return launch_colt_t<OP, B16, 32>(p, units, cl, smem, st);
+    case 64: return launch_colt_t<OP, B16, 64>(p, units, cl, smem, st);
+    case 128: return launch_colt_t<OP, B16, 128>(p, units, cl, smem, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 } // namespace
 
 int col_tile_rows() { return kColTile; }
+
+int col_tile_smem(int ct, int cl, int64_t band, int elem_bytes)
+{
+    const int64_t tile = band * ct * elem_bytes;
+    const int64_t xch = int64_t(2) * kMaxCluster * ct * 8;
+    (void)cl;
+    return static_cast<int>(tile + xch);
+}
+
+int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &p, int64_t units, void *stream)
+{
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (smem > kColTileSmemMax)
+        return cudaErrorInvalidValue;
+    switch (op) {
+    case 0: return b16 ? launch_colt_ct<0, true>(p, units, ct, cl, smem, st) : launch_colt_ct<0, false>(p, units, ct, cl, smem, st);
+    case 1: return b16 ? launch_colt_ct<1, true>(p, units, ct, cl, smem, st) : launch_colt_ct<1, false>(p, units, ct, cl, smem, st);
+    case 2: return launch_colt_ct<2, false>(p, units, ct, cl, smem, st);
+    case 3: return launch_colt_ct<3, false>(p, units, ct, cl, smem, st);
+    case 4: return launch_colt_ct<4, false>(p, units, ct, cl, smem, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 int launch_col(int op, bool b16, const WParams &p, int64_t units, void *stream)
 {

@@ -1058,13 +1058,18 @@ __device__ __forceinline__ float2 sgn2(float2 v)
     return f2(v.x > 0.f ? 1.f : v.x < 0.f ? -1.f : 0.f, v.y > 0.f ? 1.f : v.y < 0.f ? -1.f : 0.f);
 }
 
-// slerp backward.  Pass 1 sums res^2 and out^2; pass 2 forms a, b and t as
-// the forward does and sums t^2 and t . dh; pass 3 forms
-// dt = (dh - t (t . dh)/nt^2)/nt, da = (1 - |alpha|) dt, db = |alpha| dt and
-// sums ua . da, ub . db (ua = res/na, ub = out/nb before their rounding),
-// adding this row's sign(alpha) (b - a) dt to the team's dalpha line; pass 4
-// stores dres = (da - ua (ua . da)) / na and dout likewise.  t, dt and the
-// rest are recomputed from the slot in each pass.
+// slerp backward, three passes over the slot.  Pass 1 sums res^2 and
+// out^2.  Pass 2 forms a, b and t as the forward does and sums, besides
+// St = t . t and Dt = t . dh, the four sums that fold the projections of
+// da = (1 - |alpha|) dt and db = |alpha| dt onto ua = res/na and ub = out/nb
+// (before their rounding) into the same pass: with q = Dt/(St + eps) and
+// it = 1/sqrt(St + eps), dt = (dh - t q) it, so
+//   ua . da = it (ua (1-|alpha|) . dh - q  ua (1-|alpha|) . t),
+//   ub . db = it (ub |alpha| . dh    - q  ub |alpha| . t).
+// Pass 3 forms dt, da, db, stores dres = (da - ua (ua . da))/na and dout
+// likewise, and adds this row's sign(alpha) (b - a) dt to the team's dalpha
+// line.  The terms of each sum are exact rearrangements of the definition;
+// only the fp32 rounding order differs.
 template <int WP, bool CACHED, bool SPLIT>
 __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP, SPLIT> &tm, const AGSegK &sg, int64_t row, unsigned char *s0,
                                                    unsigned char *s1, unsigned char *s2, int nfull, int tail, float eps,
@@ -1103,62 +1108,85 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP, SPLIT> &tm, const AG
         for (int u = t; u < nunits; u += G)
             pairs8(xb[u], f);
     });
-    // per unit: the forward's a, b (bf16), t (fp32), |alpha| pairs
-    auto unit_t = [&](int u, uint4 &a, uint4 &b, float2 (&al)[4], float2 (&tv)[4]) {
-        a = scale8(xa[u], ra);
-        b = scale8(xb[u], rb);
+    const float2 pa = f2(ra.pre, ra.pre), ia = f2(ra.inv, ra.inv);
+    const float2 pb = f2(rb.pre, rb.pre), ib = f2(rb.inv, rb.inv);
+    const bool plain = ra.pre == 1.f && rb.pre == 1.f;
+    // per unit: ua, ub (the forward's products before rounding), a, b
+    // (bf16), t (fp32) and alpha (signed) as pairs
+    auto unit = [&](int u, float2 (&ua)[4], float2 (&ub)[4], float2 (&a)[4], float2 (&b)[4], float2 (&al)[4],
+                    float2 (&tv)[4]) {
+        const uint4 r = xa[u], o = xb[u];
         alpha8_signed<CACHED>(acache, half, sg.alpha, u, sg.cols, al);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            tv[i] = lerp2(lo2(word4(a, i)), lo2(word4(b, i)), abs2(al[i]));
+        for (int i = 0; i < 4; ++i) {
+            const float2 vr = lo2(word4(r, i)), vo = lo2(word4(o, i));
+            ua[i] = plain ? __fmul2_rn(vr, ia) : __fmul2_rn(__fmul2_rn(vr, pa), ia);
+            ub[i] = plain ? __fmul2_rn(vo, ib) : __fmul2_rn(__fmul2_rn(vo, pb), ib);
+            a[i] = lo2(pk(ua[i]));
+            b[i] = lo2(pk(ub[i]));
+            tv[i] = lerp2(a[i], b[i], abs2(al[i]));
+        }
     };
+    const float2 one = f2(1.f, 1.f);
     // pass 2
-    float2 st = f2(0.f, 0.f), dt2 = f2(0.f, 0.f);
-#pragma unroll 2
+    float2 st = f2(0.f, 0.f), sd = f2(0.f, 0.f), a_d = f2(0.f, 0.f), a_t = f2(0.f, 0.f), b_d = f2(0.f, 0.f),
+           b_t = f2(0.f, 0.f);
+#pragma unroll 1
     for (int u = t; u < nunits; u += G) {
-        uint4 a, b;
-        float2 al[4], tv[4];
-        unit_t(u, a, b, al, tv);
+        float2 ua[4], ub[4], a[4], b[4], al[4], tv[4];
+        unit(u, ua, ub, a, b, al, tv);
         const uint4 d = xd[u];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
+            const float2 dh = lo2(word4(d, i)), m = abs2(al[i]);
+            const float2 wa = __fmul2_rn(ua[i], __fadd2_rn(one, fneg2(m))), wb = __fmul2_rn(ub[i], m);
             sq2(st, tv[i]);
-            dt2 = __ffma2_rn(tv[i], lo2(word4(d, i)), dt2);
+            sd = __ffma2_rn(tv[i], dh, sd);
+            a_d = __ffma2_rn(wa, dh, a_d);
+            a_t = __ffma2_rn(wa, tv[i], a_t);
+            b_d = __ffma2_rn(wb, dh, b_d);
+            b_t = __ffma2_rn(wb, tv[i], b_t);
         }
     }
-    float sd[2] = {st.x + st.y, dt2.x + dt2.y};
-    tm.sum(sd);
-    const float nt2 = sd[0] + eps;
+    float s1v[2] = {st.x + st.y, sd.x + sd.y};
+    tm.sum(s1v);
+    float s2v[2] = {a_d.x + a_d.y, a_t.x + a_t.y};
+    tm.sum(s2v);
+    float s3v[2] = {b_d.x + b_d.y, b_t.x + b_t.y};
+    tm.sum(s3v);
+    if (!store || !tm.good())
+        return;
+    const float nt2 = s1v[0] + eps;
     const float it = 1.0f / sqrtf(nt2);
-    const float2 nqt = f2(-sd[1] / nt2, -sd[1] / nt2), it2 = f2(it, it);
-    const float2 pa = f2(ra.pre, ra.pre), ia = f2(ra.inv, ra.inv);
-    const float2 pb = f2(rb.pre, rb.pre), ib = f2(rb.inv, rb.inv);
-    const float2 one = f2(1.f, 1.f);
-    // ua, ub: res/na and out/nb before the rounding, the forward's product
-    auto unit_u = [&](uint4 raw, float2 pp, float2 ii, int i) {
-        const float2 v = lo2(word4(raw, i));
-        return pp.x == 1.f ? __fmul2_rn(v, ii) : __fmul2_rn(__fmul2_rn(v, pp), ii);
-    };
+    const float q = s1v[1] / nt2;
+    const float Sa = it * (s2v[0] - q * s2v[1]);   // ua . da
+    const float Sb = it * (s3v[0] - q * s3v[1]);   // ub . db
+    const float2 nq = f2(-q, -q), it2 = f2(it, it);
+    const float2 nDa = f2(-Sa, -Sa), nDb = f2(-Sb, -Sb);
+    const float ra_n = ra.inv * ra.pre, rb_n = rb.inv * rb.pre;      // 1/na, 1/nb
+    const float2 ra2 = f2(ra_n, ra_n), rb2 = f2(rb_n, rb_n);
+    float *odx = sg.dx + row * sg.ld_d;
+    float *odr = sg.dr + row * sg.ld_d;
     // pass 3
-    float2 sa = f2(0.f, 0.f), sb = f2(0.f, 0.f);
 #pragma unroll 1
     for (int u = t; u < nunits; u += G) {
-        uint4 a, b;
-        float2 al[4], tv[4];
-        unit_t(u, a, b, al, tv);
-        const uint4 d = xd[u], rr = xa[u], oo = xb[u];
-        float2 part[4];
+        float2 ua[4], ub[4], a[4], b[4], al[4], tv[4];
+        unit(u, ua, ub, a, b, al, tv);
+        const uint4 d = xd[u];
+        float2 gx[4], gr[4], part[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const float2 m = abs2(al[i]);
-            const float2 dt = __fmul2_rn(__ffma2_rn(tv[i], nqt, lo2(word4(d, i))), it2);
+            const float2 dt = __fmul2_rn(__ffma2_rn(tv[i], nq, lo2(word4(d, i))), it2);
             const float2 da = __fmul2_rn(__fadd2_rn(one, fneg2(m)), dt), db = __fmul2_rn(m, dt);
-            sa = __ffma2_rn(unit_u(rr, pa, ia, i), da, sa);
-            sb = __ffma2_rn(unit_u(oo, pb, ib, i), db, sb);
-            const float2 ba = __fadd2_rn(lo2(word4(b, i)), fneg2(lo2(word4(a, i))));
-            part[i] = __fmul2_rn(__fmul2_rn(sgn2(al[i]), ba), dt);
+            gx[i] = __fmul2_rn(__ffma2_rn(ua[i], nDa, da), ra2);
+            gr[i] = __fmul2_rn(__ffma2_rn(ub[i], nDb, db), rb2);
+            part[i] = __fmul2_rn(__fmul2_rn(sgn2(al[i]), __fadd2_rn(b[i], fneg2(a[i]))), dt);
         }
-        if (wsl != nullptr && store && tm.good()) {
+        const int valid = u < nfull ? 8 : tail;
+        store8f(odx, u, gx, valid);
+        store8f(odr, u, gr, valid);
+        if (wsl != nullptr) {
             float4 *l = reinterpret_cast<float4 *>(wsl + 8 * u);
             float4 p0 = make_float4(part[0].x, part[0].y, part[1].x, part[1].y);
             float4 p1 = make_float4(part[2].x, part[2].y, part[3].x, part[3].y);
@@ -1170,35 +1198,6 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP, SPLIT> &tm, const AG
             l[0] = p0;
             l[1] = p1;
         }
-    }
-    float sab2[2] = {sa.x + sa.y, sb.x + sb.y};
-    tm.sum(sab2);
-    if (!store || !tm.good())
-        return;
-    // pass 4
-    const float2 nDa = f2(-sab2[0], -sab2[0]), nDb = f2(-sab2[1], -sab2[1]);
-    const float ra_n = ra.inv * ra.pre, rb_n = rb.inv * rb.pre;      // 1/na, 1/nb
-    const float2 ra2 = f2(ra_n, ra_n), rb2 = f2(rb_n, rb_n);
-    float *odx = sg.dx + row * sg.ld_d;
-    float *odr = sg.dr + row * sg.ld_d;
-#pragma unroll 1
-    for (int u = t; u < nunits; u += G) {
-        uint4 a, b;
-        float2 al[4], tv[4];
-        unit_t(u, a, b, al, tv);
-        const uint4 d = xd[u], rr = xa[u], oo = xb[u];
-        float2 gx[4], gr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 m = abs2(al[i]);
-            const float2 dt = __fmul2_rn(__ffma2_rn(tv[i], nqt, lo2(word4(d, i))), it2);
-            const float2 da = __fmul2_rn(__fadd2_rn(one, fneg2(m)), dt), db = __fmul2_rn(m, dt);
-            gx[i] = __fmul2_rn(__ffma2_rn(unit_u(rr, pa, ia, i), nDa, da), ra2);
-            gr[i] = __fmul2_rn(__ffma2_rn(unit_u(oo, pb, ib, i), nDb, db), rb2);
-        }
-        const int valid = u < nfull ? 8 : tail;
-        store8f(odx, u, gx, valid);
-        store8f(odr, u, gr, valid);
     }
 }
 
