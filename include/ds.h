@@ -248,9 +248,11 @@ ds_status ds_l2_rows(const ds_aseg *segs, int nseg, float eps,
 ds_status ds_slerp_rows(const ds_aseg *segs, int nseg, float eps,
                         ds_stream stream);
 
-/* Rows must have at most 64 KB of staged input (a and b: 32 bytes per 8
- * columns, so at most 16,384 columns); longer rows are refused with
- * DS_ERR_INVALID_ARG.  Dory's widths are 4,096 and 7,168. */
+/* a and b are staged in shared memory (32 bytes per 8 columns): rows up to
+ * 16,384 columns on one CTA, longer ones split over a cluster of 2, 4 or 8
+ * CTAs (a slice of at most 64 KB each), so at most 131,072 columns; longer
+ * rows are refused with DS_ERR_INVALID_ARG.  Dory's widths are 4,096 and
+ * 7,168. */
 ds_status ds_gate_l2_rows(const ds_fseg *segs, int nseg, float eps,
                           ds_stream stream);
 ds_status ds_swiglu_l2_rows(const ds_fseg *segs, int nseg, float eps,
@@ -300,11 +302,13 @@ typedef struct {
 ds_status ds_qk_rows_l2(const ds_qkseg *segs, int nseg, float eps,
                         ds_stream stream);
 
-/* Rows must have at most 64 KB of staged input (x, r and dy: 48 bytes per 8
- * columns; l2 rows without a residual 32): at most 10,920 columns for slerp
- * and for l2 with a residual, 16,384 for l2 without one; longer rows are
- * refused with DS_ERR_INVALID_ARG.  ds_row_class reports the l2 backward's
- * class for rows with a residual. */
+/* x, r and dy are staged in shared memory (48 bytes per 8 columns; l2 rows
+ * without a residual 32): rows up to 10,920 columns (16,384 without a
+ * residual) on one CTA, longer ones split over a cluster of 2, 4 or 8 CTAs (a
+ * slice of at most 64 KB each), so at most 87,296 columns for slerp and for
+ * l2 with a residual, 131,072 for l2 without one; longer rows are refused
+ * with DS_ERR_INVALID_ARG.  ds_row_class reports the l2 backward's class for
+ * rows with a residual. */
 ds_status ds_l2_rows_backward(const ds_agseg *segs, int nseg, float eps,
                               ds_stream stream);
 
@@ -388,17 +392,22 @@ typedef enum {
     DS_PATH_WARP = 1,     /* staged: rows of <= 16 KB of input in a ring of
                              shared-memory slots filled by bulk copies; one
                              warp (weights) or two (activations) per row      */
-    DS_PATH_CTA = 2,      /* staged in 32 or 64 KB slots: a team of 2..8 warps
-                             per row (rows of <= 64 KB of input)              */
-    DS_PATH_CLUSTER = 3,  /* a cluster of 2..8 CTAs per row, row slices in
-                             registers, DSMEM reduction                       */
+    DS_PATH_CTA = 2,      /* staged in 32, 64 or (weights) 112 KB slots: a
+                             team of 2..8 warps per row (rows of <= 64 KB of
+                             input; weights 112 KB)                           */
+    DS_PATH_CLUSTER = 3,  /* staged, a cluster of 2, 4 or 8 CTAs per row:
+                             each CTA stages a slice of <= 64 KB of every row
+                             of its slots, partial sums meet through
+                             distributed shared memory                        */
     DS_PATH_TWO_PASS = 4  /* a cluster streams the row twice through shared
-                             memory with bulk (TMA) copies                    */
+                             memory with bulk (TMA) copies (rows longer than
+                             eight slices; not the activation backward or the
+                             Dory rows)                                       */
 } ds_path;
 
 /* The row class a call would use for rows of `cols` elements: path, threads
- * per row (the staged paths' team; 0 on cluster paths) and CTAs per row
- * (cluster/two-pass; 1 otherwise).
+ * per row in each CTA (the staged paths' team; 0 on the two-pass path) and
+ * CTAs per row (cluster / two-pass; 1 otherwise).
  * Depends on (op, cols) and the forced path only -- never on the row count. */
 ds_status ds_row_class(ds_op op, int64_t cols, int *path, int *group_threads,
                        int *cluster_ctas);

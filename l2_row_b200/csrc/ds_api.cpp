@@ -289,9 +289,9 @@ ds_status check_matrix(const void *p, int64_t rows, int64_t ld, int esize, const
 
 // Splits, packs and launches.  `make(i, r0, nrows)` returns the device
 // segment for rows [r0, r0 + nrows) of segment i.
-// Slerp launches whose segments all use one alpha vector of at most
-// kTileAlphaCacheMax columns let the staged kernel keep |alpha| in shared
-// memory (the kernel checks the length against its own cache).
+// Slerp launches whose segments all use one alpha vector let the staged
+// kernel keep |alpha| in shared memory (the kernel checks the length of its
+// slice of the columns against its own cache).
 // The Dory rows do the same with their scale vectors (sa, and sb when every
 // segment shares one).
 inline void shared_alpha(WParams &p, int)
@@ -304,7 +304,7 @@ inline void shared_alpha_act(P &p, int n)
 {
     p.alpha_shared = p.alpha2_shared = nullptr;
     p.alpha_cols = 0;
-    if (n == 0 || !p.seg[0].alpha || p.seg[0].cols > ds::kTileAlphaCacheMax)
+    if (n == 0 || !p.seg[0].alpha)
         return;
     for (int i = 1; i < n; ++i)
         if (p.seg[i].alpha != p.seg[0].alpha || p.seg[i].cols != p.seg[0].cols)
@@ -574,7 +574,7 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
             const int64_t K = segs[i].cols;
             for (const int ct : {128, 64, 32}) {
                 for (const int cl : {1, 2, 4, 8})
-                    if (ds::col_tile_smem(ct, cl, (K + cl - 1) / cl, eb) <= ds::kColTileSmemMax) {
+                    if (ds::col_tile_smem(ct, cl, (K + cl - 1) / cl, eb) <= ds::kColTileBudget) {
                         ct_of[i] = ct;
                         cl_of[i] = cl;
                         break;

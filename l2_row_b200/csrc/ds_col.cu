@@ -189,7 +189,9 @@ __global__ void __launch_bounds__(kCta) k_col(const __grid_constant__ WParams p)
 // (every stored row); a cluster of CL CTAs owns one tile, CTA k staging the
 // band of stored rows [k * band, (k + 1) * band) of it in shared memory with
 // one bulk copy per stored row (CT * 4 contiguous bytes, and CT * 2 or 4 of
-// the second input), so HBM sees whole row pieces, each read once.  Each
+// the second input; warp 0's lanes issue them), so HBM sees whole row
+// pieces, each read once.  Tiles are sized so that two or three CTAs share
+// an SM: one's loads overlap another's stores.  Each
 // CTA sums w^2 (and w . d) per column over its band in double (8 lanes down
 // the band, then a fixed tree), the CTAs' partials meet through distributed
 // shared memory and are added in rank order, and every CTA then scales its
@@ -234,11 +236,15 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ WParams p
     }
     __syncthreads();
     bool ok = true;
-    if (threadIdx.x == 0) {
+    if (threadIdx.x < 32) {
+        // warp 0 issues the band's row pieces, a lane every 32nd row (lane
+        // 0 arms the barrier; copies completing before that only run the
+        // transaction count ahead, the phase still needs lane 0's arrival)
         const uint32_t wbytes = (static_cast<uint32_t>(ncols) * 4u + 15u) & ~15u;
         const uint32_t dbytes = TWO ? (static_cast<uint32_t>(ncols) * de + 15u) & ~15u : 0u;
-        mbar_arrive_expect_tx(&full, (wbytes + dbytes) * static_cast<uint32_t>(nk));
-        for (int i = 0; i < nk; ++i) {
+        if (threadIdx.x == 0)
+            mbar_arrive_expect_tx(&full, (wbytes + dbytes) * static_cast<uint32_t>(nk));
+        for (int i = threadIdx.x; i < nk; i += 32) {
             const int64_t j = k0 + i;
             bulk_g2s(tw + static_cast<size_t>(i) * CT, sg.w + j * sg.ld + c0, wbytes, &full);
             if constexpr (TWO)

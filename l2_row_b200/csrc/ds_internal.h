@@ -54,7 +54,6 @@ constexpr int kTileSlotMaxBytes = 65536;       // largest CTA-path slot of the a
 constexpr int kTileSlotMaxWeightBytes = 114688;
 constexpr int kMaxTileSlots = 13;         // 13 x 16 KB = 208 KB of the 227 KB per CTA
 constexpr int kTileMaxRowsPerSlot = 64;
-constexpr int kTileAlphaCacheMax = 8192;  // slerp: |alpha| staged in shared memory up to this many columns
 // Two-pass path: units per thread per chunk, chunk size, pipeline stages.
 constexpr int kStreamK = 4;
 constexpr int kChunkUnits = kCta * kStreamK;
@@ -249,6 +248,7 @@ int col_tile_rows();
 // Dynamic shared memory of a launch: col_tile_smem(ct, cl, largest band,
 // bytes of w plus d per element), at most kColTileSmemMax.
 constexpr int kColTileSmemMax = 200 * 1024;
+constexpr int kColTileBudget = 96 * 1024;   // the planner's target: two or more CTAs per SM
 int col_tile_smem(int ct, int cl, int64_t band, int elem_bytes);
 int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &p, int64_t units, void *stream);
 int launch_gain_sums(const GainSumParams &p, void *stream);

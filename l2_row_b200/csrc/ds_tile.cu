@@ -112,26 +112,21 @@ __device__ __forceinline__ void peer_store_u32(uint32_t addr, uint32_t v)
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void peer_arrive(uint32_t bar_addr)
+// Two floats to peer `rank`'s shared memory at `addr`, completing 8 bytes of
+// the transaction count of its mbarrier at `bar` (an asynchronous store: no
+// fence on this thread's earlier global stores is needed, and the peer sees
+// the values once it observes the barrier's phase complete).
+__device__ __forceinline__ void peer_store2_tx(uint32_t addr, float a, float b, uint32_t bar)
 {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_addr) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t *bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok)
-                 : "r"(smem_u32(bar)), "r"(parity)
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(addr),
+                 "f"(a), "f"(b), "r"(bar)
                  : "memory");
-    return ok != 0;
 }
 
 // Exchange area of one team when its rows are split over a cluster: two
 // alternating buffers of [kMaxCluster CTAs][2 values] and their mbarriers
-// (each CTA of the cluster arrives once per exchange).
+// (one arrival per exchange, the team's own, with the transaction bytes of
+// the cluster's ncta asynchronous stores).
 constexpr int kXchgFloats = 2 * kMaxCluster * 2;
 constexpr int kXchgBytesPerTeam = kXchgFloats * 4 + 2 * 8;
 
@@ -214,9 +209,15 @@ struct Team {
     }
 
     // The CTAs' totals v[0..N) through the cluster, combined in rank order.
+    // Thread 0 sends this CTA's totals to slot [rank] of every CTA's buffer
+    // (its own included) with asynchronous stores that complete bytes on
+    // that CTA's barrier, and arms its own barrier for the ncta stores it
+    // will receive (the transaction count may run ahead of the arming);
+    // every thread waits for the phase and adds the slots in rank order.
     template <int N, class Op>
     __device__ __noinline__ void exchange(float (&v)[N], Op op)
     {
+        static_assert(N <= 2, "two values at most");
         const int b = static_cast<int>(xuse & 1u);
         const uint32_t parity = (xuse >> 1) & 1u;
         ++xuse;
@@ -225,17 +226,15 @@ struct Team {
         const uint32_t n = ctx->ncta, me = ctx->rank;
         __syncwarp();
         if (t == 0 && !failed) {
-            for (uint32_t k = 0; k < n; ++k) {
-#pragma unroll
-                for (int i = 0; i < N; ++i)
-                    peer_store_f32(peer_addr(buf + me * 2 + i, k), v[i]);
-                peer_arrive(peer_addr(bb, k));
-            }
+            const float v1 = N > 1 ? v[N > 1 ? 1 : 0] : 0.f;
+            for (uint32_t k = 0; k < n; ++k)
+                peer_store2_tx(peer_addr(buf + me * 2, k), v[0], v1, peer_addr(bb, k));
+            mbar_arrive_expect_tx(bb, 8u * n);
         }
         bool ok = !failed;
-        if (ok && !mbar_try_wait_cluster(bb, parity)) {
+        if (ok && !mbar_try_wait(bb, parity)) {
             const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait_cluster(bb, parity)) {
+            while (!mbar_try_wait(bb, parity)) {
                 if (*ctx->abort_flag || global_timer_ns() - t0 > ctx->limit_ns) {
                     ok = false;
                     break;
@@ -1543,8 +1542,8 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
         if (split)
             for (int q = 0; q < Cfg::kGroups; ++q) {
                 uint64_t *xb = reinterpret_cast<uint64_t *>(xarea + q * kXchgBytesPerTeam + kXchgFloats * 4);
-                mbar_init(&xb[0], ncta); // every CTA of the cluster arrives once per exchange
-                mbar_init(&xb[1], ncta);
+                mbar_init(&xb[0], 1); // the team's own arrival, with the peers' store bytes
+                mbar_init(&xb[1], 1);
             }
         abort_flag = 0;
         mbar_init_fence();

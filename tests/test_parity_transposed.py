@@ -2,7 +2,9 @@
 its weight as [in, out], so each unit row -- one output channel -- is a
 column of the stored matrix; DragonScale package description, "Supported
 layers").  Every result is compared, transposed back, with the float64
-oracle applied to the transposed matrix: the same definitions, row by row."""
+oracle applied to the transposed matrix: the same definitions, row by row.
+Both kernels are covered: whole column tiles staged over a cluster, and the
+column kernel for stored matrices too tall for that."""
 from __future__ import annotations
 
 import numpy as np
@@ -15,9 +17,12 @@ from tests import gpu_util as gu
 
 pytestmark = pytest.mark.gpu
 
-# (stored rows = in, stored cols = out): GPT-2 small's Conv1D shapes, and
-# ragged ones (out not a multiple of 4; one output channel)
-SHAPES = [(768, 2304), (768, 768), (768, 3072), (3072, 768), (100, 13), (7, 1), (5, 6)]
+# (stored rows = in, stored cols = out): GPT-2 small's Conv1D shapes,
+# GPT-2 XL's MLP pair (c_fc [1600, 6400], c_proj [6400, 1600]), ragged ones
+# (out not a multiple of 4; one output channel), and one too tall for eight
+# CTAs' shared memory, which takes the column kernel
+SHAPES = [(768, 2304), (768, 768), (768, 3072), (3072, 768), (1600, 6400), (6400, 1600), (100, 13), (7, 1),
+          (5, 6), (13000, 24)]
 
 
 def _stored(rng, K, N, ld_pad=0):
