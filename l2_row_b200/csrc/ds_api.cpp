@@ -612,7 +612,7 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
                 for (int i = 0; i < nseg; ++i) {
                     if (!segs[i].transposed || segs[i].rows == 0 || ct_of[i] != ct || (ct && cl_of[i] != cl))
                         continue;
-                    if (n == ds::kSegPerLaunch)
+                    if (n == (ct ? ds::col_tile_segments() : ds::kSegPerLaunch))
                         if (ds_status st = flush())
                             return st;
                     const int tile = ct ? ct : ds::col_tile_rows();

@@ -16,6 +16,11 @@
 // fixed tree; pass 2 re-reads the tile (from L2) and writes each result as
 // its double value rounded once.  Every access is a 16-byte (fp32 quad) or
 // 8-byte (bf16 quad) vector; the unit rows past `rows` are masked.
+#include <algorithm>
+#include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include "ds_device.cuh"
@@ -201,8 +206,33 @@ __global__ void __launch_bounds__(kCta) k_col(const __grid_constant__ WParams p)
 template <int OP>
 __host__ __device__ constexpr bool col_two() { return OP == 1 || OP == 3 || OP == 4; }
 
+// Segments of one tile launch, each with the tensor maps (TMA descriptors)
+// of its stored matrix w and of its second input d: 2-D row-major
+// [K stored rows][N stored columns], boxes of CT columns by `box_h` rows.
+constexpr int kColtSeg = 16;
+struct ColtParams {
+    CUtensorMap tmw[kColtSeg];
+    CUtensorMap tmd[kColtSeg];
+    WSegK seg[kColtSeg];
+    int64_t unit_start[kColtSeg + 1];   // prefix sums of tiles
+    int32_t box_h[kColtSeg];            // rows per box (<= 256)
+    int32_t nseg;
+    float eps;
+    uint64_t wait_limit_ns;
+};
+
+// One 2-D tile of a tensor map into this CTA's shared memory (no
+// multicast), completing its bytes on `bar`: columns x.., rows y...
+// x * element size is a multiple of 16 bytes (x is a multiple of CT).
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+                 ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 template <int OP, bool B16, int CT>
-__global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ WParams p)
+__global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParams p)
 {
     constexpr bool TWO = col_two<OP>();
     constexpr int Q = CT / 4;                      // column quads of a tile
@@ -217,7 +247,7 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ WParams p
     const int64_t unit = blockIdx.x / ncta;
     const int si = find_segment(p, unit);
     const WSegK &sg = p.seg[si];
-    const int64_t c0 = (unit - p.unit_start[si]) * CT;          // first unit row of the tile
+    const int64_t c0 = (unit - p.unit_start[si]) * CT;          // first unit row of the tile (a stored column)
     const int ncols = static_cast<int>(sg.rows - c0 < CT ? sg.rows - c0 : CT);
     const int K = sg.cols;
     const int band = (K + static_cast<int>(ncta) - 1) / static_cast<int>(ncta);
@@ -225,9 +255,10 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ WParams p
     const bool d_bf16 = OP == 1 && B16;
     const int64_t ld_d = OP == 1 ? sg.ld_out : sg.ld;
     const int de = d_bf16 ? 2 : 4;
-    float *tw = reinterpret_cast<float *>(smem);                          // [band][CT]
-    unsigned char *td = smem + static_cast<size_t>(band) * CT * 4;        // [band][CT] d
-    double *xch = reinterpret_cast<double *>(td + (TWO ? static_cast<size_t>(band) * CT * de : 0));
+    const int brows = (band + p.box_h[si] - 1) / p.box_h[si] * p.box_h[si];   // band rows rounded to boxes
+    float *tw = reinterpret_cast<float *>(smem);                          // [brows][CT]
+    unsigned char *td = smem + static_cast<size_t>(brows) * CT * 4;       // [brows][CT] d
+    double *xch = reinterpret_cast<double *>(td + (TWO ? static_cast<size_t>(brows) * CT * de : 0));
     // xch: [2][kMaxCluster][CT] the CTAs' partial sums, written by every peer
 
     if (threadIdx.x == 0) {
@@ -236,20 +267,19 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ WParams p
     }
     __syncthreads();
     bool ok = true;
-    if (threadIdx.x < 32) {
-        // warp 0 issues the band's row pieces, a lane every 32nd row (lane
-        // 0 arms the barrier; copies completing before that only run the
-        // transaction count ahead, the phase still needs lane 0's arrival)
-        const uint32_t wbytes = (static_cast<uint32_t>(ncols) * 4u + 15u) & ~15u;
-        const uint32_t dbytes = TWO ? (static_cast<uint32_t>(ncols) * de + 15u) & ~15u : 0u;
-        if (threadIdx.x == 0)
-            mbar_arrive_expect_tx(&full, (wbytes + dbytes) * static_cast<uint32_t>(nk));
-        for (int i = threadIdx.x; i < nk; i += 32) {
-            const int64_t j = k0 + i;
-            bulk_g2s(tw + static_cast<size_t>(i) * CT, sg.w + j * sg.ld + c0, wbytes, &full);
+    if (threadIdx.x == 0) {
+        // the band as boxes of box_h stored rows by CT columns (a box
+        // reaching past the matrix is filled with zeros and still counts
+        // its full bytes)
+        const int bh = p.box_h[si];
+        const int nbox = (nk + bh - 1) / bh;
+        const uint32_t box_bytes = static_cast<uint32_t>(bh) * CT * (4u + (TWO ? de : 0));
+        mbar_arrive_expect_tx(&full, box_bytes * static_cast<uint32_t>(nbox));
+        for (int b = 0; b < nbox; ++b) {
+            tma_load_2d(tw + static_cast<size_t>(b) * bh * CT, &p.tmw[si], static_cast<int>(c0), k0 + b * bh, &full);
             if constexpr (TWO)
-                bulk_g2s(td + static_cast<size_t>(i) * CT * de,
-                         static_cast<const char *>(sg.gy) + (j * ld_d + c0) * de, dbytes, &full);
+                tma_load_2d(td + static_cast<size_t>(b) * bh * CT * de, &p.tmd[si], static_cast<int>(c0), k0 + b * bh,
+                            &full);
         }
     }
     if (!mbar_wait_bounded(&full, 0, p.wait_limit_ns)) {
@@ -394,7 +424,7 @@ cudaError_t launch_col_t(const WParams &p, int64_t units, cudaStream_t st)
 }
 
 template <int OP, bool B16, int CT>
-cudaError_t launch_colt_t(const WParams &p, int64_t units, int cl, int smem, cudaStream_t st)
+cudaError_t launch_colt_t(const ColtParams &p, int64_t units, int cl, int smem, cudaStream_t st)
 {
     static DeviceFlags attr_set;
     if (const cudaError_t e = enable_dynamic_smem(k_colt<OP, B16, CT>, kColTileSmemMax, attr_set))
@@ -415,7 +445,7 @@ cudaError_t launch_colt_t(const WParams &p, int64_t units, int cl, int smem, cud
 }
 
 template <int OP, bool B16>
-cudaError_t launch_colt_ct(const WParams &p, int64_t units, int ct, int cl, int smem, cudaStream_t st)
+cudaError_t launch_colt_ct(const ColtParams &p, int64_t units, int ct, int cl, int smem, cudaStream_t st)
 {
     switch (ct) {
     case 32: return launch_colt_t<OP, B16, 32>(p, units, cl, smem, st);
@@ -425,42 +455,99 @@ cudaError_t launch_colt_ct(const WParams &p, int64_t units, int ct, int cl, int 
     }
 }
 
+// cuTensorMapEncodeTiled, from the driver through the runtime (the library
+// links the runtime only).
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled()
+{
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// The map of a row-major [K][N] matrix with row pitch `ld` elements,
+// boxes of ct columns by bh rows.
+bool encode_map(CUtensorMap *m, const void *base, bool bf16, int64_t K, int64_t N, int64_t ld, int ct, int bh)
+{
+    const auto fn = encode_tiled();
+    if (!fn)
+        return false;
+    const int es = bf16 ? 2 : 4;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(K)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * es};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(ct), static_cast<cuuint32_t>(bh)};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base),
+              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 } // namespace
 
 int col_tile_rows() { return kColTile; }
 
+// Rows per box: the band in as few boxes of at most 256 rows (the TMA box
+// limit) as possible, all of one height, so that no box reaches far into
+// the next band.
+int col_tile_box_rows(int64_t band)
+{
+    if (band <= 0)
+        return 1;
+    const int64_t nbox = (band + 255) / 256;
+    return static_cast<int>((band + nbox - 1) / nbox);
+}
+
 int col_tile_smem(int ct, int cl, int64_t band, int elem_bytes)
 {
-    const int64_t tile = band * ct * elem_bytes;
-    const int64_t xch = int64_t(2) * kMaxCluster * ct * 8;
     (void)cl;
+    const int64_t bh = col_tile_box_rows(band);
+    const int64_t rows = band > 0 ? (band + bh - 1) / bh * bh : 0;
+    const int64_t tile = rows * ct * elem_bytes;
+    const int64_t xch = int64_t(2) * kMaxCluster * ct * 8;
     return static_cast<int>(tile + xch);
 }
 
-int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &p, int64_t units, void *stream)
+int col_tile_segments() { return kColtSeg; }
+
+int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &w, int64_t units, void *stream)
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (smem > kColTileSmemMax)
+    if (smem > kColTileSmemMax || w.nseg > kColtSeg)
         return cudaErrorInvalidValue;
+    static thread_local ColtParams p;
+    const bool two = op == 1 || op == 3 || op == 4;
+    for (int i = 0; i < w.nseg; ++i) {
+        const WSegK &sg = w.seg[i];
+        const int64_t K = sg.cols, band = (K + cl - 1) / cl;
+        const int bh = col_tile_box_rows(band);
+        p.seg[i] = sg;
+        p.unit_start[i] = w.unit_start[i];
+        p.box_h[i] = bh;
+        if (!encode_map(&p.tmw[i], sg.w, false, K, sg.rows, sg.ld, ct, bh))
+            return cudaErrorInvalidValue;
+        if (two) {
+            const bool d16 = op == 1 && b16;
+            const int64_t ld_d = op == 1 ? sg.ld_out : sg.ld;
+            if (!encode_map(&p.tmd[i], sg.gy, d16, K, sg.rows, ld_d, ct, bh))
+                return cudaErrorInvalidValue;
+        }
+    }
+    p.unit_start[w.nseg] = w.unit_start[w.nseg];
+    p.nseg = w.nseg;
+    p.eps = w.eps;
+    p.wait_limit_ns = w.wait_limit_ns;
     switch (op) {
     case 0: return b16 ? launch_colt_ct<0, true>(p, units, ct, cl, smem, st) : launch_colt_ct<0, false>(p, units, ct, cl, smem, st);
     case 1: return b16 ? launch_colt_ct<1, true>(p, units, ct, cl, smem, st) : launch_colt_ct<1, false>(p, units, ct, cl, smem, st);
     case 2: return launch_colt_ct<2, false>(p, units, ct, cl, smem, st);
     case 3: return launch_colt_ct<3, false>(p, units, ct, cl, smem, st);
     case 4: return launch_colt_ct<4, false>(p, units, ct, cl, smem, st);
-    default: return cudaErrorInvalidValue;
-    }
-}
-
-int launch_col(int op, bool b16, const WParams &p, int64_t units, void *stream)
-{
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    switch (op) {
-    case 0: return b16 ? launch_col_t<0, true>(p, units, st) : launch_col_t<0, false>(p, units, st);
-    case 1: return b16 ? launch_col_t<1, true>(p, units, st) : launch_col_t<1, false>(p, units, st);
-    case 2: return launch_col_t<2, false>(p, units, st);
-    case 3: return launch_col_t<3, false>(p, units, st);
-    case 4: return launch_col_t<4, false>(p, units, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -244,12 +244,14 @@ int launch_col(int op, bool b16, const WParams &p, int64_t units, void *stream);
 int col_tile_rows();
 // Transposed rows in whole column tiles (ds_col.cu): tiles of ct unit rows
 // (32, 64 or 128) over every stored row, a cluster of cl CTAs per tile
-// (bands of ceil(K / cl) stored rows each); p's unit_start counts tiles.
+// (bands of ceil(K / cl) stored rows each, loaded as 2-D TMA boxes); p's
+// unit_start counts tiles; at most col_tile_segments() segments.
 // Dynamic shared memory of a launch: col_tile_smem(ct, cl, largest band,
 // bytes of w plus d per element), at most kColTileSmemMax.
 constexpr int kColTileSmemMax = 200 * 1024;
 constexpr int kColTileBudget = 96 * 1024;   // the planner's target: two or more CTAs per SM
 int col_tile_smem(int ct, int cl, int64_t band, int elem_bytes);
+int col_tile_segments();   // segments per tile launch (each carries two TMA descriptors)
 int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &p, int64_t units, void *stream);
 int launch_gain_sums(const GainSumParams &p, void *stream);
 // Staged paths (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,

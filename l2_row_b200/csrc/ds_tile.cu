@@ -638,6 +638,17 @@ __device__ __forceinline__ void tile_backward_row(Team<WP, SPLIT> &tm, const WSe
     }
 }
 
+// p[0..4) += v at the memory (fp32 adds rounded to nearest), without the
+// round trip of reading the line back: the slerp backward's dalpha lines.
+// Only the calling thread ever updates these floats, so the additions take
+// place in its program order, row after row -- the same sums, in the same
+// order, as a read-modify-write.
+__device__ __forceinline__ void red_add4(float *p, float4 v)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
 // Octet helpers: 8 bf16 as four packed pairs.
 //
 // Squares of a bf16 pair into the (even, odd) accumulators with one fused
@@ -1186,16 +1197,16 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP, SPLIT> &tm, const AG
         store8f(odx, u, gx, valid);
         store8f(odr, u, gr, valid);
         if (wsl != nullptr) {
-            float4 *l = reinterpret_cast<float4 *>(wsl + 8 * u);
-            float4 p0 = make_float4(part[0].x, part[0].y, part[1].x, part[1].y);
-            float4 p1 = make_float4(part[2].x, part[2].y, part[3].x, part[3].y);
-            if (!ws_first) {
-                const float4 o0 = l[0], o1 = l[1];
-                p0 = make_float4(o0.x + p0.x, o0.y + p0.y, o0.z + p0.z, o0.w + p0.w);
-                p1 = make_float4(o1.x + p1.x, o1.y + p1.y, o1.z + p1.z, o1.w + p1.w);
+            float *l = wsl + 8 * u;
+            const float4 p0 = make_float4(part[0].x, part[0].y, part[1].x, part[1].y);
+            const float4 p1 = make_float4(part[2].x, part[2].y, part[3].x, part[3].y);
+            if (ws_first) {
+                st16(l, as_u4(p0));
+                st16(l + 4, as_u4(p1));
+            } else {
+                red_add4(l, p0);
+                red_add4(l + 4, p1);
             }
-            l[0] = p0;
-            l[1] = p1;
         }
     }
 }
