@@ -515,6 +515,19 @@ int col_tile_smem(int ct, int cl, int64_t band, int elem_bytes)
 
 int col_tile_segments() { return kColtSeg; }
 
+int launch_col(int op, bool b16, const WParams &p, int64_t units, void *stream)
+{
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (op) {
+    case 0: return b16 ? launch_col_t<0, true>(p, units, st) : launch_col_t<0, false>(p, units, st);
+    case 1: return b16 ? launch_col_t<1, true>(p, units, st) : launch_col_t<1, false>(p, units, st);
+    case 2: return launch_col_t<2, false>(p, units, st);
+    case 3: return launch_col_t<3, false>(p, units, st);
+    case 4: return launch_col_t<4, false>(p, units, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &w, int64_t units, void *stream)
 {
     cudaStream_t st = static_cast<cudaStream_t>(stream);
