@@ -1445,6 +1445,81 @@ struct TileCfg {
     static_assert(kSmem <= 229376, "ring and vector caches fit 224 KB");
 };
 
+// The rows of one slot, each through its operation's row body.  `sg` is
+// the segment, or with a row split over a cluster the view of this CTA's
+// slice; `wsl` the team's dalpha line (slerp backward) at the slice's
+// first column.
+template <int T, int SB, bool SPLIT, int WP, class Seg>
+__device__ __forceinline__ void tile_rows(Team<WP, SPLIT> &tm, const Seg &sg, const TParams<T> &p, const SlotHdr &h,
+                                          unsigned char *base, unsigned char *a1, unsigned char *a2p, int pitch0,
+                                          int pitch1, int pitch2, int nfull, int tail, bool store, bool &ws_first,
+                                          float *s_alpha, bool acached, float *wsl)
+{
+    using Cfg = TileCfg<T, SB>;
+    const int lane = threadIdx.x & 31;
+    const bool has_r = seg_has_r(sg);
+    float g_lane = 1.f;
+            for (int r = 0; r < h.nrows; ++r) {
+                const int64_t row = h.row0 + r;
+                unsigned char *s0 = base + r * pitch0;
+                unsigned char *s1 = a1 + r * pitch1;
+                unsigned char *s2 = a2p + r * pitch2;
+                if constexpr (T == tFwdBf16 || T == tFwdF32 || T == tBwdBf16 || T == tBwdF32) {
+                    // gains of the next 32 rows, one per lane
+                    if ((r & 31) == 0)
+                        g_lane = (sg.gain && r + lane < h.nrows) ? __ldg(sg.gain + (row + lane) * sg.gain_stride) : 1.f;
+                }
+                const float g = __shfl_sync(0xffffffffu, g_lane, r & 31);
+                if constexpr (T == tFwdBf16)
+                    tile_scale_row<true, false>(tm, sg, row, g, s0, nfull, tail, p.eps, store);
+                else if constexpr (T == tFwdF32)
+                    tile_scale_row<false, false>(tm, sg, row, g, s0, nfull, tail, p.eps, store);
+                else if constexpr (T == tRenorm)
+                    tile_scale_row<false, true>(tm, sg, row, 1.f, s0, nfull, tail, p.eps, store);
+                else if constexpr (T == tBwdBf16)
+                    tile_backward_row<true, 0>(tm, sg, row, g, s0, s1, nfull, tail, p.eps, store);
+                else if constexpr (T == tBwdF32)
+                    tile_backward_row<false, 0>(tm, sg, row, g, s0, s1, nfull, tail, p.eps, store);
+                else if constexpr (T == tProject)
+                    tile_backward_row<false, 1>(tm, sg, row, 1.f, s0, s1, nfull, tail, p.eps, store);
+                else if constexpr (T == tMomentum)
+                    tile_backward_row<false, 2>(tm, sg, row, 1.f, s0, s1, nfull, tail, p.eps, store);
+                else if constexpr (T == tL2) {
+                    if (has_r)
+                        tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
+                    else
+                        tile_l2_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
+                } else if constexpr (T == tGateL2 || T == tSwigluL2) {
+                    constexpr int PRO = T == tGateL2 ? 0 : 1;
+                    constexpr int H = Cfg::kAlphaCache / 2;
+                    if (acached && (PRO == 0 || p.alpha2_shared))
+                        tile_fused_row<WP, PRO, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
+                                                      s_alpha + Cfg::kAlphaCache, H);
+                    else
+                        tile_fused_row<WP, PRO, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr,
+                                                       nullptr, 0);
+                } else if constexpr (T == tL2Bwd) {
+                    if (has_r)
+                        tile_l2_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
+                    else
+                        tile_l2_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
+                } else if constexpr (T == tSlerpBwd) {
+                    if (acached)
+                        tile_slerp_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, s_alpha,
+                                                     Cfg::kAlphaCache / 2, wsl, ws_first);
+                    else
+                        tile_slerp_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, nullptr, 0,
+                                                      wsl, ws_first);
+                    ws_first = false;
+                } else if (acached) {
+                    tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
+                                             Cfg::kAlphaCache / 2);
+                } else {
+                    tile_slerp_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr, 0);
+                }
+            }
+}
+
 // Segment view of CTA `rank`'s slice of every row: the row pointers (and
 // the per-column vectors) moved to column c0 and the row length cut to the
 // slice's `cols` columns in `nu` units (per-row vectors -- gains, grad_g --
@@ -1780,77 +1855,16 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
                     mbar_arrive(&empty[s]);
                 released = true;
             };
-            float g_lane = 1.f;
             // the rows, through the segment itself or (a slice per CTA) a
             // view of it moved to the slice's first column
-            auto rows = [&](const auto &sg) {
-            for (int r = 0; r < h.nrows; ++r) {
-                const int64_t row = h.row0 + r;
-                unsigned char *s0 = base + r * pitch0;
-                unsigned char *s1 = a1 + r * pitch1;
-                unsigned char *s2 = a2p + r * pitch2;
-                if constexpr (T == tFwdBf16 || T == tFwdF32 || T == tBwdBf16 || T == tBwdF32) {
-                    // gains of the next 32 rows, one per lane
-                    if ((r & 31) == 0)
-                        g_lane = (sg.gain && r + lane < h.nrows) ? __ldg(sg.gain + (row + lane) * sg.gain_stride) : 1.f;
-                }
-                const float g = __shfl_sync(0xffffffffu, g_lane, r & 31);
-                if constexpr (T == tFwdBf16)
-                    tile_scale_row<true, false>(tm, sg, row, g, s0, nfull, tail, p.eps, store);
-                else if constexpr (T == tFwdF32)
-                    tile_scale_row<false, false>(tm, sg, row, g, s0, nfull, tail, p.eps, store);
-                else if constexpr (T == tRenorm)
-                    tile_scale_row<false, true>(tm, sg, row, 1.f, s0, nfull, tail, p.eps, store);
-                else if constexpr (T == tBwdBf16)
-                    tile_backward_row<true, 0>(tm, sg, row, g, s0, s1, nfull, tail, p.eps, store);
-                else if constexpr (T == tBwdF32)
-                    tile_backward_row<false, 0>(tm, sg, row, g, s0, s1, nfull, tail, p.eps, store);
-                else if constexpr (T == tProject)
-                    tile_backward_row<false, 1>(tm, sg, row, 1.f, s0, s1, nfull, tail, p.eps, store);
-                else if constexpr (T == tMomentum)
-                    tile_backward_row<false, 2>(tm, sg, row, 1.f, s0, s1, nfull, tail, p.eps, store);
-                else if constexpr (T == tL2) {
-                    if (has_r)
-                        tile_l2_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
-                    else
-                        tile_l2_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store);
-                } else if constexpr (T == tGateL2 || T == tSwigluL2) {
-                    constexpr int PRO = T == tGateL2 ? 0 : 1;
-                    constexpr int H = Cfg::kAlphaCache / 2;
-                    if (cached() && (PRO == 0 || p.alpha2_shared))
-                        tile_fused_row<WP, PRO, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
-                                                      s_alpha + Cfg::kAlphaCache, H);
-                    else
-                        tile_fused_row<WP, PRO, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr,
-                                                       nullptr, 0);
-                } else if constexpr (T == tL2Bwd) {
-                    if (has_r)
-                        tile_l2_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
-                    else
-                        tile_l2_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
-                } else if constexpr (T == tSlerpBwd) {
-                    // this team's dalpha line (one per cluster and team; each
-                    // CTA of the cluster writes its slice of the columns)
-                    float *wsl = p.ws ? p.ws + (cid * NG + q) * p.ws_ld + c0 : nullptr;
-                    if (cached())
-                        tile_slerp_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, s_alpha,
-                                                     Cfg::kAlphaCache / 2, wsl, ws_first);
-                    else
-                        tile_slerp_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, nullptr, 0,
-                                                      wsl, ws_first);
-                    ws_first = false;
-                } else if (cached()) {
-                    tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
-                                             Cfg::kAlphaCache / 2);
-                } else {
-                    tile_slerp_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr, 0);
-                }
-            }
-            };
             if constexpr (SPLIT)
-                rows(shifted<T>(sg0, c0, colsk, nuk));
+                tile_rows<T, SB, SPLIT>(tm, shifted<T>(sg0, c0, colsk, nuk), p, h, base, a1, a2p, pitch0, pitch1,
+                                        pitch2, nfull, tail, store, ws_first, s_alpha, acached,
+                                        p.ws ? p.ws + (cid * NG + q) * p.ws_ld + c0 : nullptr);
             else
-                rows(sg0);
+                tile_rows<T, SB, SPLIT>(tm, sg0, p, h, base, a1, a2p, pitch0, pitch1, pitch2, nfull, tail, store,
+                                        ws_first, s_alpha, acached,
+                                        p.ws ? p.ws + (static_cast<int64_t>(blockIdx.x) * NG + q) * p.ws_ld : nullptr);
             if (!released)
                 release();
         }
