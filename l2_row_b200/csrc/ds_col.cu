@@ -197,8 +197,9 @@ __global__ void __launch_bounds__(kCta) k_col(const __grid_constant__ WParams p)
 // the second input; warp 0's lanes issue them), so HBM sees whole row
 // pieces, each read once.  Tiles are sized so that two or three CTAs share
 // an SM: one's loads overlap another's stores.  Each
-// CTA sums w^2 (and w . d) per column over its band in double (8 lanes down
-// the band, then a fixed tree), the CTAs' partials meet through distributed
+// CTA sums w^2 (and w . d) per column over its band in double (lanes down
+// the band in row order, an xor butterfly over a warp's lanes, the warps in
+// order), the CTAs' partials meet through distributed
 // shared memory and are added in rank order, and every CTA then scales its
 // staged band straight to global memory.  The results are those of the
 // column kernel above (double sums, each output its double value rounded
@@ -240,7 +241,8 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
     static_assert(Q * L == kCta && Q <= 32, "tile shape");
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) uint64_t full;
-    __shared__ double red[2][L][CT];
+    constexpr int NW = kCta / 32;                  // warps
+    __shared__ double red[2][NW][CT];              // the warps' partials per column
     __shared__ double fac[2][CT];
     cluster_arrive_relaxed();
     const uint32_t rank = cluster_ctarank(), ncta = cluster_nctarank();
@@ -311,25 +313,41 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
                 dd[e] = fma(wi, dval(i, e), dd[e]);
         }
     }
+    // the lanes of a warp that hold the same columns (32 / Q of them, Q
+    // apart) by an xor butterfly, then the warps in order: one barrier
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        red[0][ln][4 * q + e] = s[e];
-        if constexpr (TWO)
-            red[1][ln][4 * q + e] = dd[e];
+    for (int o = Q; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            s[e] += __shfl_xor_sync(0xffffffffu, s[e], o);
+            if constexpr (TWO)
+                dd[e] += __shfl_xor_sync(0xffffffffu, dd[e], o);
+        }
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) < Q) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            red[0][warp][4 * q + e] = s[e];
+            if constexpr (TWO)
+                red[1][warp][4 * q + e] = dd[e];
+        }
     }
     __syncthreads();
-    for (int o = L / 2; o > 0; o >>= 1) {
-        if (ln < o) {
+    if (threadIdx.x < CT) {
+        const int c = threadIdx.x;
+        double a0 = red[0][0][c], a1 = TWO ? red[1][0][c] : 0.0;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                red[0][ln][4 * q + e] += red[0][ln + o][4 * q + e];
-                if constexpr (TWO)
-                    red[1][ln][4 * q + e] += red[1][ln + o][4 * q + e];
-            }
+        for (int w = 1; w < NW; ++w) {
+            a0 += red[0][w][c];
+            if constexpr (TWO)
+                a1 += red[1][w][c];
         }
-        __syncthreads();
+        red[0][0][c] = a0;
+        if constexpr (TWO)
+            red[1][0][c] = a1;
     }
-    // the band's partials to every CTA of the cluster (slot [rank])
+    // the band's partials (each written by the thread that sends it) to
+    // every CTA of the cluster (slot [rank])
     cluster_wait();   // every peer has started (arrival at kernel start)
     if (threadIdx.x < CT) {
         const int c = threadIdx.x;

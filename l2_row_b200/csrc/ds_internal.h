@@ -55,7 +55,7 @@ constexpr int kTileSlotMaxWeightBytes = 114688;
 constexpr int kMaxTileSlots = 13;         // 13 x 16 KB = 208 KB of the 227 KB per CTA
 constexpr int kTileMaxRowsPerSlot = 64;
 // Two-pass path: units per thread per chunk, chunk size, pipeline stages.
-constexpr int kStreamK = 4;
+constexpr int kStreamK = 2;
 constexpr int kChunkUnits = kCta * kStreamK;
 constexpr int kStages = 4;
 

@@ -188,6 +188,7 @@ struct Team {
     // rows split over a cluster (SPLIT): this team's exchange area (unused,
     // and dropped by the compiler, with one CTA per row)
     const ClusterCtx *ctx = nullptr;
+    uint32_t xrank = 0, xn = 1;       // this CTA's rank, the cluster's CTAs (ctx's, in registers)
     float *xbuf = nullptr;            // [2][kMaxCluster][2]
     uint64_t *xbar = nullptr;         // [2]
     uint32_t xuse = 0;                // exchanges so far
@@ -196,7 +197,7 @@ struct Team {
     __device__ __forceinline__ uint32_t rank() const
     {
         if constexpr (SPLIT)
-            return ctx->rank;
+            return xrank;
         else
             return 0u;
     }
@@ -208,6 +209,18 @@ struct Team {
             return true;
     }
 
+    // The bounded wait for an exchange's phase, out of line (rarely taken
+    // long); gives up at the limit or when this CTA or a peer aborted.
+    __device__ __noinline__ bool wait_slow(uint64_t *bb, uint32_t parity) const
+    {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bb, parity)) {
+            if (*ctx->abort_flag || global_timer_ns() - t0 > ctx->limit_ns)
+                return false;
+        }
+        return true;
+    }
+
     // The CTAs' totals v[0..N) through the cluster, combined in rank order.
     // Thread 0 sends this CTA's totals to slot [rank] of every CTA's buffer
     // (its own included) with asynchronous stores that complete bytes on
@@ -215,7 +228,7 @@ struct Team {
     // will receive (the transaction count may run ahead of the arming);
     // every thread waits for the phase and adds the slots in rank order.
     template <int N, class Op>
-    __device__ __noinline__ void exchange(float (&v)[N], Op op)
+    __device__ __forceinline__ void exchange(float (&v)[N], Op op)
     {
         static_assert(N <= 2, "two values at most");
         const int b = static_cast<int>(xuse & 1u);
@@ -223,7 +236,7 @@ struct Team {
         ++xuse;
         float *buf = xbuf + b * (kMaxCluster * 2);
         uint64_t *bb = xbar + b;
-        const uint32_t n = ctx->ncta, me = ctx->rank;
+        const uint32_t n = xn, me = xrank;
         __syncwarp();
         if (t == 0 && !failed) {
             const float v1 = N > 1 ? v[N > 1 ? 1 : 0] : 0.f;
@@ -232,15 +245,8 @@ struct Team {
             mbar_arrive_expect_tx(bb, 8u * n);
         }
         bool ok = !failed;
-        if (ok && !mbar_try_wait(bb, parity)) {
-            const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(bb, parity)) {
-                if (*ctx->abort_flag || global_timer_ns() - t0 > ctx->limit_ns) {
-                    ok = false;
-                    break;
-                }
-            }
-        }
+        if (ok && !mbar_try_wait(bb, parity))
+            ok = wait_slow(bb, parity);
         if (!ok) {
             if (!failed)
                 ctx->abort_all();
@@ -942,8 +948,12 @@ __device__ __forceinline__ void store8f(float *o, int u, const float2 (&v)[4], i
         st16(o + 8 * u + 4, make_uint4(__float_as_uint(v[2].x), __float_as_uint(v[2].y), __float_as_uint(v[3].x),
                                        __float_as_uint(v[3].y)));
     } else {
-        for (int e = 0; e < valid; ++e)
-            o[8 * u + e] = (e & 1) ? v[e >> 1].y : v[e >> 1].x;
+        // fully unrolled: v stays in registers (a runtime index would put it
+        // in local memory)
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (e < valid)
+                o[8 * u + e] = (e & 1) ? v[e >> 1].y : v[e >> 1].x;
     }
 }
 
@@ -1789,6 +1799,8 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
         Team<WP, SPLIT> tm{wi * 32 + lane, 1 + q, red + q * Team<WP>::kRed};
         if constexpr (SPLIT) {
             tm.ctx = &ctx;
+            tm.xrank = rank;
+            tm.xn = ncta;
             tm.xbuf = reinterpret_cast<float *>(xarea + q * kXchgBytesPerTeam);
             tm.xbar = reinterpret_cast<uint64_t *>(xarea + q * kXchgBytesPerTeam + kXchgFloats * 4);
         }
