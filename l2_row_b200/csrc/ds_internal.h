@@ -54,9 +54,7 @@ constexpr int kTileSlotMaxBytes = 65536;       // largest CTA-path slot of the a
 constexpr int kTileSlotMaxWeightBytes = 114688;
 constexpr int kMaxTileSlots = 13;         // 13 x 16 KB = 208 KB of the 227 KB per CTA
 constexpr int kTileMaxRowsPerSlot = 64;
-// Two-pass path: units per thread per chunk, chunk size, pipeline stages.
-constexpr int kStreamK = 2;
-constexpr int kChunkUnits = kCta * kStreamK;
+// Two-pass path: pipeline stages (the chunk size is per operation).
 constexpr int kStages = 4;
 
 // Rows split over a cluster of `ncta` CTAs (staged cluster classes): CTA k

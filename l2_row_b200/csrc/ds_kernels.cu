@@ -558,20 +558,37 @@ template <> struct StreamOp<kMomentum> { using type = SBackward<false, kModeMome
 template <> struct StreamOp<kL2> { using type = SL2; };
 template <> struct StreamOp<kSlerp> { using type = SSlerp; };
 
+// Units per thread per chunk: 4 where one array streams (16 KB stages), 2
+// where two do (16 KB stages for two 16-byte arrays), so that several CTAs
+// share an SM (each streams one row slice and leaves).
 template <int T>
-constexpr int stream_stage_bytes()
+__host__ __device__ constexpr int stream_k()
+{
+    return (T == kFwdBf16 || T == kFwdF32 || T == kRenorm) ? 4 : 2;
+}
+
+template <int T>
+__host__ __device__ constexpr int stream_chunk_units()
+{
+    return kCta * stream_k<T>();
+}
+
+template <int T>
+__host__ __device__ constexpr int stream_stage_bytes()
 {
     // widest layout of the operation's arrays per stage
-    return (T == kBwdF32 || T == kProject || T == kMomentum) ? 2 * 16 * kChunkUnits
-         : T == kBwdBf16 ? (16 + 8) * kChunkUnits
-         : (T == kL2 || T == kSlerp) ? 2 * 16 * kChunkUnits
-         : 16 * kChunkUnits;
+    constexpr int cu = stream_chunk_units<T>();
+    return (T == kBwdF32 || T == kProject || T == kMomentum) ? 2 * 16 * cu
+         : T == kBwdBf16 ? (16 + 8) * cu
+         : (T == kL2 || T == kSlerp) ? 2 * 16 * cu
+         : 16 * cu;
 }
 
 template <int T>
 __global__ void __launch_bounds__(kCta, 1) k_stream(const __grid_constant__ ParamsOf<T> p)
 {
     using Op = typename StreamOp<T>::type;
+    constexpr int CU = stream_chunk_units<T>();
     extern __shared__ __align__(128) unsigned char ring[];
     __shared__ __align__(8) uint64_t full[kStages];
     __shared__ float red_sm[2 * kWarps * 4];
@@ -593,7 +610,7 @@ __global__ void __launch_bounds__(kCta, 1) k_stream(const __grid_constant__ Para
     per = (per + 1) & ~1;
     c.ubeg = min(c.nu, static_cast<int>(red.rank) * per);
     c.len = min(c.nu, c.ubeg + per) - c.ubeg;
-    const int nch = (c.len + kChunkUnits - 1) / kChunkUnits;
+    const int nch = (c.len + CU - 1) / CU;
     const int total = Op::kPasses * nch;
 
     int ub[2], off[2];
@@ -604,7 +621,7 @@ __global__ void __launch_bounds__(kCta, 1) k_stream(const __grid_constant__ Para
         ub[a] = a < Op::kArrays ? op.unit_bytes(a) : 0;
         src[a] = ub[a] ? op.src(a) + static_cast<int64_t>(c.ubeg) * ub[a] : nullptr;
         off[a] = stage_bytes;
-        stage_bytes += ub[a] * kChunkUnits;
+        stage_bytes += ub[a] * CU;
     }
 
     if (threadIdx.x == 0) {
@@ -618,8 +635,8 @@ __global__ void __launch_bounds__(kCta, 1) k_stream(const __grid_constant__ Para
     auto issue = [&](int i) {
         const int ch = i % nch;
         const int s = i % kStages;
-        const int u0 = ch * kChunkUnits;
-        const int n = min(kChunkUnits, c.len - u0);
+        const int u0 = ch * CU;
+        const int n = min(CU, c.len - u0);
         uint32_t bytes[2], tot = 0;
 #pragma unroll
         for (int a = 0; a < 2; ++a) {
@@ -649,9 +666,9 @@ __global__ void __launch_bounds__(kCta, 1) k_stream(const __grid_constant__ Para
                 ok = false;
             const unsigned char *st[2] = {ring + s * stage_bytes + off[0], ring + s * stage_bytes + off[1]};
 #pragma unroll
-            for (int k = 0; k < kStreamK; ++k) {
+            for (int k = 0; k < stream_k<T>(); ++k) {
                 const int j = threadIdx.x + k * kCta;
-                const int ul = ch * kChunkUnits + j;
+                const int ul = ch * CU + j;
                 if (ul < c.len)
                     op.consume(pass, st, j, c.ubeg + ul, c, ok);
             }

@@ -1429,9 +1429,11 @@ struct TileCfg {
     static constexpr int kSlotBytes = SB;
     static constexpr int kScale = SB == 114688 ? 8 : SB / 16384;    // 1, 2, 4; 8 for 112 KB
     static constexpr int kWP = (is_act_tag(T) ? 2 : 1) * kScale;
-    // SwiGLU rows keep two scale vectors in shared memory: one position fewer
+    // SwiGLU rows keep two scale vectors in shared memory: one position fewer;
+    // the slerp backward in 32 KB slots takes one fewer too, so that its
+    // 672 threads get 80 registers each (800 threads get 72 and spill)
     static constexpr int kGroups = SB == 16384 ? (T == tSwigluL2 ? 12 : 13)
-                                   : SB == 32768 ? (T == tSwigluL2 ? 5 : 6)
+                                   : SB == 32768 ? ((T == tSwigluL2 || T == tSlerpBwd) ? 5 : 6)
                                    : SB == 65536 ? 3 : 2;
     static constexpr int kSlots = kGroups;                          // one position per team
     static constexpr int kConsumers = kWP * kGroups;
