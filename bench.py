@@ -17,10 +17,12 @@ disjoint buffers (>= 268 MB of other traffic between two uses of one
 buffer), so inputs come from HBM without an explicit flush.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--config step|mlp_pair|wide|optimizer|act_backward|dory|gain]
+                    [--config step|mlp_pair|wide|optimizer|act_backward|dory|gain|long_rows]
+                    [--no-extras]
 
 `--config` selects another workload for a per-call report (default: the
-step above).  mlp_pair = up [2048,768] + down [768,2048] (fwd, bwd, renorm;
+step above); after the default step, every other workload's calls are
+timed and reported under "extras" (skip with --no-extras).  mlp_pair = up [2048,768] + down [768,2048] (fwd, bwd, renorm;
 L2-resident, so each timed step uses the next of 16 buffer copies and a
 CUDA-graph replay of the calls is timed as well).  wide = weights
 [14336,4096], [4096,14336] (fwd, bwd) and activation rows [8192,7168],
@@ -31,7 +33,9 @@ dory = Dory's gated and SwiGLU l2 rows on [16384,4096] and [8192,7168]
 (scale vectors fp32 U(0.5, 2)) and its q/k rows on 16384 rows of 16 + 4 + 4
 heads of 256.  gain = the row lengths and the scalar-gain backward of the
 whole model, and forward + backward of 12 GPT-2 XL Conv1D weights
-[1600, 6400] stored [in, out] (transposed rows).
+[1600, 6400] stored [in, out] (transposed rows).  long_rows = rows split
+over a cluster ([2048,40000] forward, [4096,24576] slerp) and rows on the
+two-pass stream ([256,262144] forward, [512,262144] slerp).
 
 Prints one JSON line (rank 0).  `value` is algorithmic bytes moved by all
 ranks per second (GB/s); per-kernel GB/s and rows/s, the roofline of the
@@ -100,7 +104,7 @@ def parse_args():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
-                   help="skip the per-call report of the config-5 wide calls and the long-row classes")
+                   help="skip the per-call report of the other workloads after the default step")
     p.add_argument("--config", choices=tuple(WORKLOADS), default="step")
     return p.parse_args()
 
@@ -629,18 +633,21 @@ def time_calls(step, K: int, W: int, sp: int) -> dict[str, float]:
             for i, name in enumerate(step.names)}
 
 
+EXTRA_CONFIGS = ("wide", "long_rows", "optimizer", "act_backward", "dory", "gain", "mlp_pair")
+
+
 def extra_calls(seed: int, K: int, sp: int, peak: float) -> dict:
-    """The config-5 wide calls and the long-row classes, each call timed on
-    its own (CUDA events) and reported against the HBM peak; not part of the
-    step's `value`."""
+    """Every other workload's calls, each call timed on its own (CUDA events,
+    mean over K steps after 3 warm-up steps) and reported against the HBM
+    peak; not part of the step's `value`.  The L2-resident MLP pair also
+    reports its calls replayed from one CUDA graph."""
     import torch
 
     from l2_row_b200 import ds
 
     out = {}
-    for label, make in (("config5_wide", lambda: Step(seed=seed, config="wide")),
-                        ("long_rows", lambda: LongRows(seed))):
-        st = make()
+    for label in EXTRA_CONFIGS:
+        st = LongRows(seed) if label == "long_rows" else Step(seed=seed, config=label)
         ms = time_calls(st, K, 3, sp)
         if ds.ds_get_device_status(sp) != ds.DS_OK:
             raise RuntimeError(f"device error in the {label} calls")
@@ -652,8 +659,12 @@ def extra_calls(seed: int, K: int, sp: int, peak: float) -> dict:
                            "frac_of_peak": round(gbs / peak, 4), "rows_s": round(st.rows[name] / t_s, 1)}
             if isinstance(st, LongRows):
                 calls[name]["class"] = st.classes[name]
-        out[label] = {"workload": WORKLOADS["wide" if label == "config5_wide" else "long_rows"], "steps": K,
-                      "calls": calls}
+        out[label] = {"workload": WORKLOADS[label], "steps": K, "calls": calls}
+        if st.copies > 1:
+            gms = graph_replay_ms(st)
+            total = sum(st.bytes.values())
+            out[label]["graph"] = {"ms_per_step": round(gms, 5), "gb_s": round(total / (gms * 1e-3) / 1e9, 1),
+                                   "calls_per_replay": st.copies * len(st.names)}
         del st
         torch.cuda.empty_cache()
     return out

@@ -790,14 +790,19 @@ __device__ __forceinline__ float2 lerp2(float2 a, float2 b, float2 m)
     return __ffma2_rn(m, __fadd2_rn(b, fneg2(a)), a);
 }
 
+// How much of a launch's per-column vector a CTA holds in shared memory:
+// none, all of its columns, or (slerp rows longer than the cache) the first
+// columns, with the rest read from global memory.
+enum AlphaCache { kAlphaNone = 0, kAlphaAll = 1, kAlphaHead = 2 };
+
 // |alpha| of unit u: from the shared-memory cache (split layout: the first
-// four of each unit at abs_alpha[4u], the last four at abs_alpha[half + 4u])
-// or from global memory.
-template <bool CACHED>
+// four of each unit at abs_alpha[4u], the last four at abs_alpha[half + 4u];
+// units below half / 4) or from global memory.
+template <int AC>
 __device__ __forceinline__ void abs_alpha8(const float *abs_alpha, int half, const float *alpha, int u, int cols,
                                            float2 (&m)[4])
 {
-    if constexpr (CACHED) {
+    if (AC == kAlphaAll || (AC == kAlphaHead && 4 * u < half)) {
         const float4 m0 = *reinterpret_cast<const float4 *>(abs_alpha + 4 * u);
         const float4 m1 = *reinterpret_cast<const float4 *>(abs_alpha + half + 4 * u);
         m[0] = f2(m0.x, m0.y);
@@ -809,14 +814,14 @@ __device__ __forceinline__ void abs_alpha8(const float *abs_alpha, int half, con
     }
 }
 
-template <bool CACHED>
+template <int AC>
 __device__ __forceinline__ void slerp_unit_t(uint4 p, uint4 q, RowScale ra, RowScale rb, const float *abs_alpha,
                                              int half, const float *alpha, int u, int cols, float2 &at, float4 &ta,
                                              float4 &tb)
 {
     const uint4 a = scale8(p, ra), b = scale8(q, rb);
     float2 m[4];
-    abs_alpha8<CACHED>(abs_alpha, half, alpha, u, cols, m);
+    abs_alpha8<AC>(abs_alpha, half, alpha, u, cols, m);
     const float2 t0 = lerp2(lo2(a.x), lo2(b.x), m[0]), t1 = lerp2(lo2(a.y), lo2(b.y), m[1]);
     const float2 t2 = lerp2(lo2(a.z), lo2(b.z), m[2]), t3 = lerp2(lo2(a.w), lo2(b.w), m[3]);
     sq2(at, t0);
@@ -833,7 +838,7 @@ __device__ __forceinline__ uint4 slerp_unit_h(float4 p, float4 q, float2 s)
                       pk(__fmul2_rn(f2(q.x, q.y), s)), pk(__fmul2_rn(f2(q.z, q.w), s)));
 }
 
-template <int WP, bool CACHED, bool SPLIT>
+template <int WP, int AC, bool SPLIT>
 __device__ __forceinline__ void tile_slerp_row(Team<WP, SPLIT> &tm, const ASegK &sg, int64_t row, unsigned char *s0,
                                                unsigned char *s1, int nfull, int tail, float eps, bool store,
                                                const float *abs_alpha, int half)
@@ -875,13 +880,13 @@ __device__ __forceinline__ void tile_slerp_row(Team<WP, SPLIT> &tm, const ASegK 
 #pragma unroll 4
     for (int u = t; u < nfull; u += G) {
         float4 p, q;
-        slerp_unit_t<CACHED>(xa[u], xb[u], ra, rb, abs_alpha, half, sg.alpha, u, sg.cols, at, p, q);
+        slerp_unit_t<AC>(xa[u], xb[u], ra, rb, abs_alpha, half, sg.alpha, u, sg.cols, at, p, q);
         ta[u] = p;
         tb[u] = q;
     }
     if (tl) {
         float4 p, q;
-        slerp_unit_t<CACHED>(xa[nfull], xb[nfull], ra, rb, abs_alpha, half, sg.alpha, nfull, sg.cols, at, p, q);
+        slerp_unit_t<AC>(xa[nfull], xb[nfull], ra, rb, abs_alpha, half, sg.alpha, nfull, sg.cols, at, p, q);
         ta[nfull] = p;
         tb[nfull] = q;
     }
@@ -1465,7 +1470,7 @@ template <int T, int SB, bool SPLIT, int WP, class Seg>
 __device__ __forceinline__ void tile_rows(Team<WP, SPLIT> &tm, const Seg &sg, const TParams<T> &p, const SlotHdr &h,
                                           unsigned char *base, unsigned char *a1, unsigned char *a2p, int pitch0,
                                           int pitch1, int pitch2, int nfull, int tail, bool store, bool &ws_first,
-                                          float *s_alpha, bool acached, float *wsl)
+                                          float *s_alpha, int acache, float *wsl)
 {
     using Cfg = TileCfg<T, SB>;
     const int lane = threadIdx.x & 31;
@@ -1504,7 +1509,7 @@ __device__ __forceinline__ void tile_rows(Team<WP, SPLIT> &tm, const Seg &sg, co
                 } else if constexpr (T == tGateL2 || T == tSwigluL2) {
                     constexpr int PRO = T == tGateL2 ? 0 : 1;
                     constexpr int H = Cfg::kAlphaCache / 2;
-                    if (acached && (PRO == 0 || p.alpha2_shared))
+                    if (acache == kAlphaAll && (PRO == 0 || p.alpha2_shared))
                         tile_fused_row<WP, PRO, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
                                                       s_alpha + Cfg::kAlphaCache, H);
                     else
@@ -1516,18 +1521,21 @@ __device__ __forceinline__ void tile_rows(Team<WP, SPLIT> &tm, const Seg &sg, co
                     else
                         tile_l2_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store);
                 } else if constexpr (T == tSlerpBwd) {
-                    if (acached)
+                    if (acache == kAlphaAll)
                         tile_slerp_bwd_row<WP, true>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, s_alpha,
                                                      Cfg::kAlphaCache / 2, wsl, ws_first);
                     else
                         tile_slerp_bwd_row<WP, false>(tm, sg, row, s0, s1, s2, nfull, tail, p.eps, store, nullptr, 0,
                                                       wsl, ws_first);
                     ws_first = false;
-                } else if (acached) {
-                    tile_slerp_row<WP, true>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
-                                             Cfg::kAlphaCache / 2);
+                } else if (acache == kAlphaAll) {
+                    tile_slerp_row<WP, kAlphaAll>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
+                                                  Cfg::kAlphaCache / 2);
+                } else if (acache == kAlphaHead) {
+                    tile_slerp_row<WP, kAlphaHead>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, s_alpha,
+                                                   Cfg::kAlphaCache / 2);
                 } else {
-                    tile_slerp_row<WP, false>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr, 0);
+                    tile_slerp_row<WP, kAlphaNone>(tm, sg, row, s0, s1, nfull, tail, p.eps, store, nullptr, 0);
                 }
             }
 }
@@ -1656,17 +1664,22 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
         ac0 = 8 * au0;
         acols = max(0, min(p.alpha_cols - ac0, 8 * (au1 - au0)));
     }
-    // (one CTA per row: read from the parameters where it is used)
+    // (one CTA per row: read from the parameters where it is used).  The
+    // slerp forward caches the head of a longer |alpha| and reads the rest.
     auto cached = [&]() {
-        return p.alpha_shared != nullptr && (SPLIT ? acols : p.alpha_cols) <= Cfg::kAlphaCache;
+        if (p.alpha_shared == nullptr || Cfg::kAlphaCache == 0)
+            return static_cast<int>(kAlphaNone);
+        if ((SPLIT ? acols : p.alpha_cols) <= Cfg::kAlphaCache)
+            return static_cast<int>(kAlphaAll);
+        return static_cast<int>(T == tSlerp ? kAlphaHead : kAlphaNone);
     };
-    const bool acached = cached();
+    const int acache = cached();
     if constexpr (T == tSlerp || T == tSlerpBwd) {
         // |alpha| split by halves of each 8-element unit: unit u's first four
         // at [4u], its last four at [half + 4u], so that a warp reading one
         // float4 per lane touches consecutive 16-byte words (no bank conflict)
-        if (acached) {
-            const int nu = (acols + 7) / 8, half = Cfg::kAlphaCache / 2;
+        if (acache != kAlphaNone) {
+            const int nu = min((acols + 7) / 8, Cfg::kAlphaCache / 8), half = Cfg::kAlphaCache / 2;
             for (int i = threadIdx.x; i < 8 * nu; i += blockDim.x) {
                 const int u = i >> 3, e = i & 7;
                 // the backward keeps the sign (dalpha needs it); the forward |alpha|
@@ -1678,7 +1691,7 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
     }
     if constexpr (T == tGateL2 || T == tSwigluL2) {
         // the scale vectors in the same split layout, sb after sa
-        if (acached && (T == tGateL2 || p.alpha2_shared)) {
+        if (acache == kAlphaAll && (T == tGateL2 || p.alpha2_shared)) {
             const int nu = (acols + 7) / 8, half = Cfg::kAlphaCache / 2;
             for (int i = threadIdx.x; i < 8 * nu; i += blockDim.x) {
                 const int u = i >> 3, e = i & 7, at = (e < 4 ? 0 : half) + 4 * u + (e & 3);
@@ -1873,11 +1886,11 @@ __global__ void __launch_bounds__(TileCfg<T, SB>::kThreads, 1)
             // view of it moved to the slice's first column
             if constexpr (SPLIT)
                 tile_rows<T, SB, SPLIT>(tm, shifted<T>(sg0, c0, colsk, nuk), p, h, base, a1, a2p, pitch0, pitch1,
-                                        pitch2, nfull, tail, store, ws_first, s_alpha, acached,
+                                        pitch2, nfull, tail, store, ws_first, s_alpha, acache,
                                         p.ws ? p.ws + (cid * NG + q) * p.ws_ld + c0 : nullptr);
             else
                 tile_rows<T, SB, SPLIT>(tm, sg0, p, h, base, a1, a2p, pitch0, pitch1, pitch2, nfull, tail, store,
-                                        ws_first, s_alpha, acached,
+                                        ws_first, s_alpha, acache,
                                         p.ws ? p.ws + (static_cast<int64_t>(blockIdx.x) * NG + q) * p.ws_ld : nullptr);
             if (!released)
                 release();

@@ -63,3 +63,9 @@ def test_long_rows_cover_both_long_classes():
         act = types.SimpleNamespace(rows=rows, cols=cols)
         b = rows * cols * 6 + rows * 4 if kind == "fwd" else bench.call_bytes("slerp", act=act)
         assert b > 126 * 2 ** 20
+
+
+def test_extras_cover_every_other_workload():
+    """After the default step the bench reports every other workload."""
+    assert set(bench.EXTRA_CONFIGS) == set(bench.WORKLOADS) - {"step"}
+    assert len(bench.EXTRA_CONFIGS) == len(set(bench.EXTRA_CONFIGS))
