@@ -682,6 +682,36 @@ ds_status run_norms(bool preserve, const ds_wseg *segs, int nseg, float eps, voi
     }
     if (ds_status st = check_overlaps(spans))
         return st;
+    // rows that a CTA (or a cluster's slices) can stage take the staged
+    // kernel, with the forward's row classes (it stages the same rows);
+    // longer rows take the warp-per-row kernel
+    const int forced = g_force_path.load(std::memory_order_relaxed);
+    std::vector<RowClass> cls(static_cast<size_t>(nseg));
+    std::vector<int64_t> staged_rows(static_cast<size_t>(nseg), 0);
+    for (int i = 0; i < nseg; ++i) {
+        cls[i] = classify(DS_OP_WN_FORWARD, segs[i].cols, forced);
+        if (ds::is_staged(cls[i])) {
+            cls[i].rps = tile_rows_per_slot(DS_OP_WN_FORWARD, slice_units(DS_OP_WN_FORWARD, segs[i].cols, cls[i]), 4,
+                                            true, cls[i].slot);
+            staged_rows[i] = segs[i].rows;
+        }
+    }
+    auto make = [&](int i, int64_t r0, int64_t nr) {
+        WSegK k = wseg_rows(segs[i], r0, nr, 4, 4);
+        k.gain = nullptr;
+        k.gy = nullptr;
+        k.grad_w = nullptr;
+        k.grad_g = nullptr;
+        k.out = segs[i].rnorm + r0;
+        k.radius = preserve ? segs[i].radius : 1.f;
+        return k;
+    };
+    auto launch = [&](const RowClass &rc, const WParams &p, int64_t units, void *st) -> int {
+        int used = 0;
+        return ds::launch_tile(13, &p, units, rc.slot, rc.cluster, &used, st);
+    };
+    if (ds_status st = launch_all<WParams, WSegK>(nseg, staged_rows.data(), cls, eps, make, launch, stream))
+        return st;
     static thread_local ds::RNParams params;
     int n = 0;
     int64_t units = 0;
@@ -691,7 +721,7 @@ ds_status run_norms(bool preserve, const ds_wseg *segs, int nseg, float eps, voi
         params.nseg = n;
         params.unit_start[n] = units;
         params.eps = eps;
-        if (ds::launch_row_norms(params, stream) != 0)
+        if (ds::launch_row_norms(params, sm_count(), stream) != 0)
             return fail(DS_ERR_CUDA, "kernel launch failed");
         g_launches.fetch_add(1, std::memory_order_relaxed);
         n = 0;
@@ -700,7 +730,7 @@ ds_status run_norms(bool preserve, const ds_wseg *segs, int nseg, float eps, voi
     };
     for (int i = 0; i < nseg; ++i) {
         const ds_wseg &s = segs[i];
-        if (s.rows == 0)
+        if (s.rows == 0 || staged_rows[i] != 0)
             continue;
         if (n == ds::kSegPerLaunch)
             if (ds_status st = flush())

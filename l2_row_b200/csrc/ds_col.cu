@@ -17,6 +17,7 @@
 // its double value rounded once.  Every access is a 16-byte (fp32 quad) or
 // 8-byte (bf16 quad) vector; the unit rows past `rows` are masked.
 #include <algorithm>
+#include <cfloat>
 #include <mutex>
 
 #include <cuda.h>
@@ -255,7 +256,6 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
     const int band = (K + static_cast<int>(ncta) - 1) / static_cast<int>(ncta);
     const int k0 = min(K, static_cast<int>(rank) * band), nk = min(K, k0 + band) - k0;
     const bool d_bf16 = OP == 1 && B16;
-    const int64_t ld_d = OP == 1 ? sg.ld_out : sg.ld;
     const int de = d_bf16 ? 2 : 4;
     const int brows = (band + p.box_h[si] - 1) / p.box_h[si] * p.box_h[si];   // band rows rounded to boxes
     float *tw = reinterpret_cast<float *>(smem);                          // [brows][CT]
@@ -292,88 +292,136 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
             raise_device_error(DS_ERR_DEVICE_TIMEOUT, kSiteTileWait);
     }
     const int q = threadIdx.x % Q, ln = threadIdx.x / Q;
-    auto dval = [&](int i, int e) -> double {
+    const int warp = threadIdx.x >> 5;
+    auto dvalf = [&](int i, int e) -> float {
         if constexpr (TWO) {
             if (d_bf16)
-                return static_cast<double>(bf_lo(reinterpret_cast<const uint16_t *>(td)[static_cast<size_t>(i) * CT + 4 * q + e]));
-            return static_cast<double>(reinterpret_cast<const float *>(td)[static_cast<size_t>(i) * CT + 4 * q + e]);
+                return bf_lo(reinterpret_cast<const uint16_t *>(td)[static_cast<size_t>(i) * CT + 4 * q + e]);
+            return reinterpret_cast<const float *>(td)[static_cast<size_t>(i) * CT + 4 * q + e];
         } else {
-            return 0.0;
+            return 0.f;
         }
     };
-    // pass 1: this CTA's band, per column, in double
-    double s[4] = {0, 0, 0, 0}, dd[4] = {0, 0, 0, 0};
-    for (int i = ln; i < nk; i += L) {
-        const float4 w = *reinterpret_cast<const float4 *>(tw + static_cast<size_t>(i) * CT + 4 * q);
+    // The warps' per-column partials (red[.][warp]) summed in warp order,
+    // sent to slot [rank] of every CTA of the cluster, and added there in
+    // rank order after the cluster barrier: S (and D) per column in fac's
+    // place, identical in every CTA.
+    auto cluster_sums = [&](double &S, double &D) {
+        __syncthreads();
+        if (threadIdx.x < CT) {
+            const int c = threadIdx.x;
+            double a0 = red[0][0][c], a1 = TWO ? red[1][0][c] : 0.0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const double wi = comp(w, e);
-            s[e] = fma(wi, wi, s[e]);
-            if constexpr (TWO)
-                dd[e] = fma(wi, dval(i, e), dd[e]);
+            for (int w = 1; w < NW; ++w) {
+                a0 += red[0][w][c];
+                if constexpr (TWO)
+                    a1 += red[1][w][c];
+            }
+            for (uint32_t k = 0; k < ncta; ++k) {
+                namespace cg = cooperative_groups;
+                double *x0 = cg::this_cluster().map_shared_rank(xch + rank * CT + c, static_cast<int>(k));
+                *x0 = a0;
+                if constexpr (TWO) {
+                    double *x1 = cg::this_cluster().map_shared_rank(xch + (kMaxCluster + rank) * CT + c,
+                                                                    static_cast<int>(k));
+                    *x1 = a1;
+                }
+            }
         }
-    }
-    // the lanes of a warp that hold the same columns (32 / Q of them, Q
-    // apart) by an xor butterfly, then the warps in order: one barrier
-#pragma unroll
-    for (int o = Q; o < 32; o <<= 1)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            s[e] += __shfl_xor_sync(0xffffffffu, s[e], o);
-            if constexpr (TWO)
-                dd[e] += __shfl_xor_sync(0xffffffffu, dd[e], o);
-        }
-    const int warp = threadIdx.x >> 5;
-    if ((threadIdx.x & 31) < Q) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            red[0][warp][4 * q + e] = s[e];
-            if constexpr (TWO)
-                red[1][warp][4 * q + e] = dd[e];
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < CT) {
-        const int c = threadIdx.x;
-        double a0 = red[0][0][c], a1 = TWO ? red[1][0][c] : 0.0;
-#pragma unroll
-        for (int w = 1; w < NW; ++w) {
-            a0 += red[0][w][c];
-            if constexpr (TWO)
-                a1 += red[1][w][c];
-        }
-        red[0][0][c] = a0;
-        if constexpr (TWO)
-            red[1][0][c] = a1;
-    }
-    // the band's partials (each written by the thread that sends it) to
-    // every CTA of the cluster (slot [rank])
-    cluster_wait();   // every peer has started (arrival at kernel start)
-    if (threadIdx.x < CT) {
-        const int c = threadIdx.x;
-        for (uint32_t k = 0; k < ncta; ++k) {
-            namespace cg = cooperative_groups;
-            double *x0 = cg::this_cluster().map_shared_rank(xch + rank * CT + c, static_cast<int>(k));
-            *x0 = red[0][0][c];
+        cluster_arrive();
+        cluster_wait();
+        S = 0.0;
+        D = 0.0;
+        if (threadIdx.x < CT) {
+            const int c = threadIdx.x;
+            S = xch[c];
+            for (uint32_t k = 1; k < ncta; ++k)
+                S += xch[k * CT + c];
             if constexpr (TWO) {
-                double *x1 = cg::this_cluster().map_shared_rank(xch + (kMaxCluster + rank) * CT + c, static_cast<int>(k));
-                *x1 = red[1][0][c];
+                D = xch[kMaxCluster * CT + c];
+                for (uint32_t k = 1; k < ncta; ++k)
+                    D += xch[(kMaxCluster + k) * CT + c];
+            }
+        }
+    };
+    // pass 1: this CTA's band, per column, in fp32 (lanes down the band in
+    // row order); the lanes of a warp that hold the same columns (32 / Q of
+    // them, Q apart) by an xor butterfly
+    {
+        float s[4] = {0.f, 0.f, 0.f, 0.f}, dd[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int i = ln; i < nk; i += L) {
+            const float4 w = *reinterpret_cast<const float4 *>(tw + static_cast<size_t>(i) * CT + 4 * q);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float wi = comp(w, e);
+                s[e] = fmaf(wi, wi, s[e]);
+                if constexpr (TWO)
+                    dd[e] = fmaf(wi, dvalf(i, e), dd[e]);
+            }
+        }
+#pragma unroll
+        for (int o = Q; o < 32; o <<= 1)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                s[e] += __shfl_xor_sync(0xffffffffu, s[e], o);
+                if constexpr (TWO)
+                    dd[e] += __shfl_xor_sync(0xffffffffu, dd[e], o);
+            }
+        if ((threadIdx.x & 31) < Q) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                red[0][warp][4 * q + e] = s[e];
+                if constexpr (TWO)
+                    red[1][warp][4 * q + e] = dd[e];
             }
         }
     }
-    cluster_arrive();
-    cluster_wait();
+    cluster_wait();   // every peer has started (arrival at kernel start)
+    double S, D;
+    cluster_sums(S, D);
+    // A column whose fp32 sum overflowed (or, at eps = 0, fell below
+    // 2^-100) takes the tile through an exact pass: the band summed again
+    // in double and a second exchange, then double arithmetic in pass 2.
+    // S is the same in every CTA, so every CTA takes the same branch.
+    const bool need = threadIdx.x < CT && c0 + threadIdx.x < sg.rows &&
+                      (!(S <= static_cast<double>(FLT_MAX)) || (p.eps == 0.f && S < 0x1p-100));
+    const bool exact = __syncthreads_or(need) != 0;
+    if (exact) {
+        double s[4] = {0, 0, 0, 0}, dd[4] = {0, 0, 0, 0};
+        for (int i = ln; i < nk; i += L) {
+            const float4 w = *reinterpret_cast<const float4 *>(tw + static_cast<size_t>(i) * CT + 4 * q);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const double wi = comp(w, e);
+                s[e] = fma(wi, wi, s[e]);
+                if constexpr (TWO)
+                    dd[e] = fma(wi, static_cast<double>(dvalf(i, e)), dd[e]);
+            }
+        }
+#pragma unroll
+        for (int o = Q; o < 32; o <<= 1)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                s[e] += __shfl_xor_sync(0xffffffffu, s[e], o);
+                if constexpr (TWO)
+                    dd[e] += __shfl_xor_sync(0xffffffffu, dd[e], o);
+            }
+        // every CTA has read the first exchange before any is overwritten
+        cluster_arrive();
+        cluster_wait();
+        if ((threadIdx.x & 31) < Q) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                red[0][warp][4 * q + e] = s[e];
+                if constexpr (TWO)
+                    red[1][warp][4 * q + e] = dd[e];
+            }
+        }
+        cluster_sums(S, D);
+    }
     if (threadIdx.x < CT) {
         const int c = threadIdx.x;
         const int64_t r = c0 + c;
-        double S = xch[c], D = 0.0;
-        for (uint32_t k = 1; k < ncta; ++k)
-            S += xch[k * CT + c];
-        if constexpr (TWO) {
-            D = xch[kMaxCluster * CT + c];
-            for (uint32_t k = 1; k < ncta; ++k)
-                D += xch[(kMaxCluster + k) * CT + c];
-        }
         if (r < sg.rows) {
             S += static_cast<double>(p.eps);
             const double n = sqrt(S);
@@ -392,7 +440,52 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
     }
     __syncthreads();
     ok = __syncthreads_and(ok) != 0;
-    if (ok) {
+    if (!ok) {
+        if (threadIdx.x == 0)
+            raise_device_error(DS_ERR_DEVICE_TIMEOUT, kSiteTileWait);
+        return;
+    }
+    const int valid = ncols - 4 * q >= 4 ? 4 : (ncols - 4 * q > 0 ? ncols - 4 * q : 0);
+    if (valid == 0)
+        return;
+    const int64_t col = c0 + 4 * q;
+    auto store = [&](int64_t j, const float (&y)[4], const float (&ev)[4]) {
+        const float4 yv = make_float4(y[0], y[1], y[2], y[3]);
+        if constexpr (OP == 0) {
+            col_store<B16>(static_cast<char *>(sg.out) + (j * sg.ld_out + col) * (B16 ? 2 : 4), yv, valid);
+        } else if constexpr (OP == 2) {
+            col_store<false>(const_cast<float *>(sg.w) + j * sg.ld + col, yv, valid);
+        } else {
+            col_store<false>(sg.grad_w + j * sg.ld + col, make_float4(ev[0], ev[1], ev[2], ev[3]), valid);
+            if constexpr (OP == 4)
+                col_store<false>(const_cast<float *>(sg.w) + j * sg.ld + col, yv, valid);
+        }
+    };
+    // pass 2: the scale (and D / n^2) rounded once to fp32, fp32 products;
+    // the exact pass keeps them in double, each output rounded once
+    if (!exact) {
+        float sc[4], qt[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            sc[e] = static_cast<float>(fac[0][4 * q + e]);
+            if constexpr (TWO)
+                qt[e] = static_cast<float>(fac[1][4 * q + e]);
+        }
+        for (int i = ln; i < nk; i += L) {
+            const float4 w = *reinterpret_cast<const float4 *>(tw + static_cast<size_t>(i) * CT + 4 * q);
+            float y[4], ev[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float wi = comp(w, e);
+                y[e] = wi * sc[e];
+                if constexpr (TWO) {
+                    const float ei = fmaf(-wi, qt[e], dvalf(i, e));
+                    ev[e] = OP == 1 ? sc[e] * ei : ei;
+                }
+            }
+            store(k0 + i, y, ev);
+        }
+    } else {
         double sc[4], qt[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -400,36 +493,20 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
             if constexpr (TWO)
                 qt[e] = fac[1][4 * q + e];
         }
-        const int valid = ncols - 4 * q >= 4 ? 4 : (ncols - 4 * q > 0 ? ncols - 4 * q : 0);
-        if (valid > 0) {
-            for (int i = ln; i < nk; i += L) {
-                const int64_t j = k0 + i;
-                const float4 w = *reinterpret_cast<const float4 *>(tw + static_cast<size_t>(i) * CT + 4 * q);
-                float y[4], ev[4];
+        for (int i = ln; i < nk; i += L) {
+            const float4 w = *reinterpret_cast<const float4 *>(tw + static_cast<size_t>(i) * CT + 4 * q);
+            float y[4], ev[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const double wi = comp(w, e);
-                    y[e] = static_cast<float>(wi * sc[e]);
-                    if constexpr (TWO) {
-                        const double ei = dval(i, e) - wi * qt[e];
-                        ev[e] = static_cast<float>(OP == 1 ? sc[e] * ei : ei);
-                    }
-                }
-                const float4 yv = make_float4(y[0], y[1], y[2], y[3]);
-                const int64_t col = c0 + 4 * q;
-                if constexpr (OP == 0) {
-                    col_store<B16>(static_cast<char *>(sg.out) + (j * sg.ld_out + col) * (B16 ? 2 : 4), yv, valid);
-                } else if constexpr (OP == 2) {
-                    col_store<false>(const_cast<float *>(sg.w) + j * sg.ld + col, yv, valid);
-                } else {
-                    col_store<false>(sg.grad_w + j * sg.ld + col, make_float4(ev[0], ev[1], ev[2], ev[3]), valid);
-                    if constexpr (OP == 4)
-                        col_store<false>(const_cast<float *>(sg.w) + j * sg.ld + col, yv, valid);
+            for (int e = 0; e < 4; ++e) {
+                const double wi = comp(w, e);
+                y[e] = static_cast<float>(wi * sc[e]);
+                if constexpr (TWO) {
+                    const double ei = static_cast<double>(dvalf(i, e)) - wi * qt[e];
+                    ev[e] = static_cast<float>(OP == 1 ? sc[e] * ei : ei);
                 }
             }
+            store(k0 + i, y, ev);
         }
-    } else if (threadIdx.x == 0) {
-        raise_device_error(DS_ERR_DEVICE_TIMEOUT, kSiteTileWait);
     }
 }
 

@@ -234,7 +234,8 @@ int launch_renorm_momentum(const RowClass &rc, const WParams &p, int64_t units, 
 int launch_l2_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void *stream);
 int launch_wait_selftest(uint64_t limit_ns, void *stream);
-int launch_row_norms(const RNParams &p, void *stream);
+// `sms`: the device's SM count (the grid holds every CTA at once).
+int launch_row_norms(const RNParams &p, int sms, void *stream);
 // Transposed rows (ds_col.cu): op 0 forward, 1 backward, 2 renorm,
 // 3 gradient projection, 4 momentum projection; b16: bf16 W_eff / GY.
 // p's unit_start counts tiles of col_tile_rows() rows.
@@ -255,8 +256,9 @@ int launch_gain_sums(const GainSumParams &p, void *stream);
 // Staged paths (ds_tile.cu).  tag: 0 forward bf16, 1 forward f32,
 // 2 backward bf16 GY, 3 backward f32 GY, 4 renorm, 5 l2, 6 slerp,
 // 7 gradient projection, 8 momentum projection + renorm, 9 l2 backward,
-// 10 slerp backward, 11 gated l2 rows, 12 SwiGLU l2 rows; params is a WParams
-// (tags 0-4, 7, 8), AParams (5, 6, 11, 12) or GParams (9, 10) whose segments
+// 10 slerp backward, 11 gated l2 rows, 12 SwiGLU l2 rows, 13 row lengths
+// (out: rnorm, radius: the divisor); params is a WParams
+// (tags 0-4, 7, 8, 13), AParams (5, 6, 11, 12) or GParams (9, 10) whose segments
 // carry rows per slot in `group` and whose
 // unit_start counts slots; slot_bytes 16, 32, 64 or (weights) 112 KB.
 // cluster: CTAs per row (1, 2, 4 or 8); units: the launch's slots; the

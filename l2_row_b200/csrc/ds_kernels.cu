@@ -868,10 +868,10 @@ int launch_slerp_rows(const RowClass &rc, const AParams &p, int64_t units, void 
     return launch_op<kSlerp>(rc, p, units, stream);
 }
 
-int launch_row_norms(const RNParams &p, void *stream)
+int launch_row_norms(const RNParams &p, int sms, void *stream)
 {
     const int64_t warps = p.unit_start[p.nseg];
-    const int64_t blocks = std::min<int64_t>((warps + kWarps - 1) / kWarps, 148 * 8);
+    const int64_t blocks = std::min<int64_t>((warps + kWarps - 1) / kWarps, int64_t(sms) * 8);
     k_row_norms<<<static_cast<int>(blocks), kCta, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError();
 }

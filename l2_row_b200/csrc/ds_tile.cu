@@ -30,10 +30,13 @@ namespace ds {
 // ds_kernels.cu's tags, repeated (the two files share this numbering).
 enum TileTag {
     tFwdBf16, tFwdF32, tBwdBf16, tBwdF32, tRenorm, tL2, tSlerp, tProject, tMomentum, tL2Bwd, tSlerpBwd, tGateL2,
-    tSwigluL2
+    tSwigluL2, tNorms
 };
 
-__host__ __device__ constexpr bool is_weight_tag(int T) { return T <= tRenorm || T == tProject || T == tMomentum; }
+__host__ __device__ constexpr bool is_weight_tag(int T)
+{
+    return T <= tRenorm || T == tProject || T == tMomentum || T == tNorms;
+}
 __host__ __device__ constexpr bool is_act_bwd_tag(int T) { return T == tL2Bwd || T == tSlerpBwd; }
 __host__ __device__ constexpr bool is_fused_tag(int T) { return T == tGateL2 || T == tSwigluL2; }
 __host__ __device__ constexpr bool is_act_tag(int T)
@@ -365,7 +368,9 @@ __device__ __forceinline__ void alpha_pairs(const float *alpha, int u, int cols,
 
 template <int T>
 struct TileLayout {
-    static constexpr int kArrays = (T == tFwdBf16 || T == tFwdF32 || T == tRenorm) ? 1 : is_act_bwd_tag(T) ? 3 : 2;
+    static constexpr int kArrays = (T == tFwdBf16 || T == tFwdF32 || T == tRenorm || T == tNorms) ? 1
+                                   : is_act_bwd_tag(T)                                          ? 3
+                                                                                                : 2;
     // bytes per unit of array a (the activation backward: x, r, dy)
     static __device__ __forceinline__ int ub(int a, bool has_r)
     {
@@ -503,6 +508,63 @@ __device__ __forceinline__ void tile_scale_row(Team<WP, SPLIT> &tm, const WSegK 
             if (tail > 2) o[2] = y.z;
         }
     }
+}
+
+// Row lengths (ds_row_norms; ds_gain_preserve with the radius as divisor):
+// S summed as the forward sums it, then out[row] = sqrt(S + eps) / radius.
+// A row whose fp32 sum overflows (or, at eps = 0, underflows) is summed
+// again scaled by 2^m (exact) and its length scaled back.
+template <int WP, bool SPLIT>
+__device__ __forceinline__ void tile_norm_row(Team<WP, SPLIT> &tm, const WSegK &sg, int64_t row,
+                                              const unsigned char *s0, int nfull, int tail, float eps, bool store)
+{
+    constexpr int G = Team<WP>::G;
+    const int lane = tm.t;
+    const float4 *w = reinterpret_cast<const float4 *>(s0);
+    float2 acc = f2(0.f, 0.f);
+#pragma unroll 4
+    for (int u = lane; u < nfull; u += G) {
+        const float4 v = w[u];
+        sq2(acc, f2(v.x, v.y));
+        sq2(acc, f2(v.z, v.w));
+    }
+    const bool tl = tail && lane == nfull % G;
+    float4 vt = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tl) {
+        vt = mask_quad(w[nfull], tail);
+        sq2(acc, f2(vt.x, vt.y));
+        sq2(acc, f2(vt.z, vt.w));
+    }
+    const float S = tm.sum1(acc.x + acc.y);
+    float len = sqrtf(S + eps);
+    if (needs_rescale(S, eps)) {
+        float M = 0.f;
+        for (int u = lane; u < nfull; u += G) {
+            const float4 v = w[u];
+            M = fmaxf(M, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+        M = fmaxf(M, fmaxf(fmaxf(fabsf(vt.x), fabsf(vt.y)), fmaxf(fabsf(vt.z), fabsf(vt.w))));
+        M = tm.max(M);
+        if (M > 0.f && M < __int_as_float(0x7f800000)) {
+            const int m = 48 - ilogbf(M);
+            float2 as = f2(0.f, 0.f);
+            auto add = [&](float4 v) {
+                const float2 a = f2(scalbnf(v.x, m), scalbnf(v.y, m)), b = f2(scalbnf(v.z, m), scalbnf(v.w, m));
+                as = __ffma2_rn(a, a, as);
+                as = __ffma2_rn(b, b, as);
+            };
+            for (int u = lane; u < nfull; u += G)
+                add(w[u]);
+            if (tl)
+                add(vt);
+            const float Ss = tm.sum1(as.x + as.y);
+            len = scalbnf(sqrtf(Ss + scalbnf(eps, 2 * m)), -m);
+        }
+    }
+    if (!store || !tm.good())
+        return;
+    if (lane == 0 && tm.rank() == 0)
+        static_cast<float *>(sg.out)[row] = __fdiv_rn(len, sg.radius);
 }
 
 template <bool GY_BF16>
@@ -1493,6 +1555,8 @@ __device__ __forceinline__ void tile_rows(Team<WP, SPLIT> &tm, const Seg &sg, co
                     tile_scale_row<false, false>(tm, sg, row, g, s0, nfull, tail, p.eps, store);
                 else if constexpr (T == tRenorm)
                     tile_scale_row<false, true>(tm, sg, row, 1.f, s0, nfull, tail, p.eps, store);
+                else if constexpr (T == tNorms)
+                    tile_norm_row(tm, sg, row, s0, nfull, tail, p.eps, store);
                 else if constexpr (T == tBwdBf16)
                     tile_backward_row<true, 0>(tm, sg, row, g, s0, s1, nfull, tail, p.eps, store);
                 else if constexpr (T == tBwdF32)
@@ -2044,6 +2108,7 @@ int launch_tile(int tag, const void *params, int64_t units, int slot_bytes, int 
     case tSlerpBwd: return launch_tile_t<tSlerpBwd>(params, units, slot_bytes, cluster, used, stream);
     case tGateL2: return launch_tile_t<tGateL2>(params, units, slot_bytes, cluster, used, stream);
     case tSwigluL2: return launch_tile_t<tSwigluL2>(params, units, slot_bytes, cluster, used, stream);
+    case tNorms: return launch_tile_t<tNorms>(params, units, slot_bytes, cluster, used, stream);
     default: return cudaErrorInvalidValue;
     }
 }

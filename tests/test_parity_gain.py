@@ -35,14 +35,43 @@ def run_norms(w: np.ndarray, eps: float, preserve=False, radius=1.0, ld_pad=0):
 
 
 @pytest.mark.parametrize("eps", [1e-6, 0.0])
-def test_row_norms_shapes(eps):
+@pytest.mark.parametrize("path", PATHS, ids=PATH_IDS)
+def test_row_norms_shapes(eps, path):
+    """Every row class: the staged kernel (a row per warp, per CTA or split
+    over a cluster) and the warp-per-row kernel for rows past the staged
+    classes (forced here with the two-pass path)."""
     rng = np.random.default_rng(81)
-    for R, C in ((1, 1), (7, 3), (33, 129), (64, 768), (5, 4097), (3, 131072), (300, 2048)):
-        w = wl.drifted_rows(rng, R, C, 0.02)
-        got = run_norms(w, eps, ld_pad=4)
-        ref = oracle.row_norms(w, eps=eps)
-        bad = rel_violations(got, ref, 2e-6)
-        assert not bad.any(), (R, C, got[bad][:3], ref[bad][:3])
+    with ds.force_path(path):
+        for R, C in ((1, 1), (7, 3), (33, 129), (64, 768), (5, 4097), (3, 131072), (300, 2048), (9, 40000)):
+            w = wl.drifted_rows(rng, R, C, 0.02)
+            got = run_norms(w, eps, ld_pad=4)
+            ref = oracle.row_norms(w, eps=eps)
+            bad = rel_violations(got, ref, 2e-6)
+            assert not bad.any(), (R, C, got[bad][:3], ref[bad][:3])
+
+
+@pytest.mark.parametrize("path", [ds.DS_PATH_AUTO, ds.DS_PATH_TWO_PASS], ids=["staged", "warp_per_row"])
+def test_row_norms_whole_model(path):
+    """The whole-model table (85 segments) in one call, every row against
+    the oracle; the staged kernel takes it in one launch."""
+    wk = wl.whole_model(0)
+    outs, segs = [], []
+    for s in wk.weights:
+        wd = gu.dev_f32(s.w)
+        out = torch.full((s.rows,), -1.0, dtype=torch.float32, device="cuda")
+        outs.append((s, out, wd))
+        segs.append(ds.WSeg(w=wd, rnorm=out))
+    with ds.force_path(path):
+        before = ds.ds_launch_count()
+        ds.ds_row_norms(segs, 1e-6)
+        torch.cuda.synchronize()
+        launches = ds.ds_launch_count() - before
+    if path == ds.DS_PATH_AUTO:
+        assert launches == 1, launches
+    for s, out, _ in outs:
+        ref = oracle.row_norms(s.w, eps=1e-6)
+        bad = rel_violations(gu.host_f32(out), ref, 2e-6)
+        assert not bad.any(), (s.name, int(bad.sum()))
 
 
 def test_row_norms_extreme_and_zero_rows():

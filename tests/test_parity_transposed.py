@@ -131,3 +131,35 @@ def test_mixed_table_and_scalar_gain():
     gu.check_backward(seg, gw_t.t().contiguous(), gg_t[:N], 1e-6, what="transposed, scalar gain")
     h = gu.host_f32(gg_t)
     assert abs(float(h[N]) - float(np.sum(h[:N], dtype=np.float64))) <= np.spacing(np.float32(abs(h[N])))
+
+
+@pytest.mark.parametrize("eps", [1e-6, 0.0])
+def test_extreme_columns(eps):
+    """Column tiles whose fp32 sums overflow (|w| ~ 1e25), or at eps = 0 fall
+    below 2^-100 (|w| ~ 1e-30), take the exact pass; a tile of ordinary
+    columns beside them keeps the fp32 pass.  Both against the oracle."""
+    rng = np.random.default_rng(95)
+    K, N = 768, 384
+    w, wd, _, ld = _stored(rng, K, N)
+    w[:, 5] *= np.float32(1e27)          # tile 0: one overflowing column
+    w[:, 200] *= np.float32(1e-28)       # a later tile: one tiny column
+    wd.copy_(gu.dev_f32(w))
+    g = wl.gains(rng, N)
+    for out_dtype in ("f32", "bf16"):
+        dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+        o = torch.empty(K, N, dtype=dt, device="cuda")
+        ds.ds_wn_forward([ds.WSeg(w=wd, gain=gu.dev_f32(g), w_eff=o, transposed=True)], out_dtype, eps)
+        torch.cuda.synchronize()
+        gu.check_forward(_seg_t(w, g, None), o.t().contiguous(), eps, out_dtype, what=f"extreme fwd {out_dtype}")
+    gy = wl.to_bf16_bits(rng.standard_normal((K, N)).astype(np.float32) * np.float32(1e-3))
+    gw = torch.empty(K, N, dtype=torch.float32, device="cuda")
+    gg = torch.empty(N, dtype=torch.float32, device="cuda")
+    gyd = torch.empty(K, N, dtype=torch.bfloat16, device="cuda")
+    gyd.copy_(gu.dev_bf16(gy))
+    ds.ds_wn_backward([ds.WSeg(w=wd, gain=gu.dev_f32(g), gy=gyd, grad_w=gw, grad_g=gg, transposed=True)],
+                      "bf16", eps)
+    torch.cuda.synchronize()
+    gu.check_backward(_seg_t(w, g, gy), gw.t().contiguous(), gg, eps, what="extreme bwd")
+    ds.ds_row_renorm([ds.WSeg(w=wd, transposed=True)], eps)
+    torch.cuda.synchronize()
+    gu.check_renorm(_seg_t(w, None, None), wd.t().contiguous(), eps, what="extreme renorm")
