@@ -572,13 +572,17 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
             if (!segs[i].transposed || segs[i].rows == 0)
                 continue;
             const int64_t K = segs[i].cols;
-            for (const int ct : {128, 64, 32}) {
-                for (const int cl : {1, 2, 4, 8})
-                    if (ds::col_tile_smem(ct, cl, (K + cl - 1) / cl, eb) <= ds::kColTileBudget) {
-                        ct_of[i] = ct;
-                        cl_of[i] = cl;
+            for (const int budget : ds::kColTileBudgets) {
+                for (const int ct : {128, 64, 32}) {
+                    for (const int cl : {1, 2, 4, 8})
+                        if (ds::col_tile_smem(ct, cl, (K + cl - 1) / cl, eb) <= budget) {
+                            ct_of[i] = ct;
+                            cl_of[i] = cl;
+                            break;
+                        }
+                    if (ct_of[i])
                         break;
-                    }
+                }
                 if (ct_of[i])
                     break;
             }

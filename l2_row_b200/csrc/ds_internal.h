@@ -248,7 +248,9 @@ int col_tile_rows();
 // Dynamic shared memory of a launch: col_tile_smem(ct, cl, largest band,
 // bytes of w plus d per element), at most kColTileSmemMax.
 constexpr int kColTileSmemMax = 200 * 1024;
-constexpr int kColTileBudget = 96 * 1024;   // the planner's target: two or more CTAs per SM
+// The planner's budgets, tried in order: the first that holds some tile
+// shape of a segment decides it (two or more CTAs per SM, else one).
+constexpr int kColTileBudgets[2] = {96 * 1024, kColTileSmemMax};
 int col_tile_smem(int ct, int cl, int64_t band, int elem_bytes);
 int col_tile_segments();   // segments per tile launch (each carries two TMA descriptors)
 int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &p, int64_t units, void *stream);

@@ -18,9 +18,10 @@ from tests import gpu_util as gu
 pytestmark = pytest.mark.gpu
 
 # (stored rows = in, stored cols = out): GPT-2 small's Conv1D shapes,
-# GPT-2 XL's MLP pair (c_fc [1600, 6400], c_proj [6400, 1600]), ragged ones
-# (out not a multiple of 4; one output channel), and one too tall for eight
-# CTAs' shared memory, which takes the column kernel
+# GPT-2 XL's MLP pair (c_fc [1600, 6400]: tiles over clusters of 8 with two
+# or three CTAs per SM; c_proj [6400, 1600]: 32-column tiles, one CTA per
+# SM), ragged ones (out not a multiple of 4; one output channel), and one too
+# tall for eight CTAs' shared memory, which takes the column kernel
 SHAPES = [(768, 2304), (768, 768), (768, 3072), (3072, 768), (1600, 6400), (6400, 1600), (100, 13), (7, 1),
           (5, 6), (13000, 24)]
 
