@@ -96,6 +96,14 @@ __device__ __forceinline__ void st16(void *p, uint4 v)
                  : "memory");
 }
 
+// One 32-byte store (sm_100's 256-bit vector store); p 32-byte aligned.
+__device__ __forceinline__ void st32(void *p, uint4 a, uint4 b)
+{
+    asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+                 "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+}
+
 __device__ __forceinline__ void st8(void *p, uint2 v)
 {
     asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");

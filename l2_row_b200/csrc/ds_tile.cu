@@ -1005,15 +1005,23 @@ __device__ __forceinline__ void dot8(float2 &acc, uint4 a, uint4 b)
 
 __device__ __forceinline__ uint32_t word4(uint4 v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
 
-// Eight fp32 values of one unit to row `o` at unit u (two 16-byte stores),
-// or only its first `valid` elements.
-__device__ __forceinline__ void store8f(float *o, int u, const float2 (&v)[4], int valid)
+// Eight fp32 values of one unit to row `o` at unit u: one 32-byte store
+// where the row starts on 32 bytes (a32), so that a warp's store covers its
+// 1 KB of the row whole; else two 16-byte stores; or only the first `valid`
+// elements.
+__device__ __forceinline__ void store8f(float *o, int u, const float2 (&v)[4], int valid, bool a32)
 {
     if (valid >= 8) {
-        st16(o + 8 * u, make_uint4(__float_as_uint(v[0].x), __float_as_uint(v[0].y), __float_as_uint(v[1].x),
-                                   __float_as_uint(v[1].y)));
-        st16(o + 8 * u + 4, make_uint4(__float_as_uint(v[2].x), __float_as_uint(v[2].y), __float_as_uint(v[3].x),
-                                       __float_as_uint(v[3].y)));
+        const uint4 lo = make_uint4(__float_as_uint(v[0].x), __float_as_uint(v[0].y), __float_as_uint(v[1].x),
+                                    __float_as_uint(v[1].y));
+        const uint4 hi = make_uint4(__float_as_uint(v[2].x), __float_as_uint(v[2].y), __float_as_uint(v[3].x),
+                                    __float_as_uint(v[3].y));
+        if (a32) {
+            st32(o + 8 * u, lo, hi);
+        } else {
+            st16(o + 8 * u, lo);
+            st16(o + 8 * u + 4, hi);
+        }
     } else {
         // fully unrolled: v stays in registers (a runtime index would put it
         // in local memory)
@@ -1094,6 +1102,7 @@ __device__ __forceinline__ void tile_l2_bwd_row(Team<WP, SPLIT> &tm, const AGSeg
     const float os = m == 0 ? inv : scalbnf(inv, m);              // 1/n
     const float2 os2 = f2(os, os);
     float *o = sg.dx + row * sg.ld_d;
+    const bool a32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
 #pragma unroll 2
     for (int u = t; u < nunits; u += G) {
         const uint4 sv = x[u], d = dy[u];
@@ -1105,7 +1114,7 @@ __device__ __forceinline__ void tile_l2_bwd_row(Team<WP, SPLIT> &tm, const AGSeg
                 sp = f2(scalbnf(sp.x, m), scalbnf(sp.y, m));
             v[i] = __fmul2_rn(__ffma2_rn(sp, nq, lo2(word4(d, i))), os2);
         }
-        store8f(o, u, v, u < nfull ? 8 : tail);
+        store8f(o, u, v, u < nfull ? 8 : tail, a32);
     }
 }
 
@@ -1254,6 +1263,7 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP, SPLIT> &tm, const AG
     const float2 ra2 = f2(ra_n, ra_n), rb2 = f2(rb_n, rb_n);
     float *odx = sg.dx + row * sg.ld_d;
     float *odr = sg.dr + row * sg.ld_d;
+    const bool a32 = ((reinterpret_cast<uintptr_t>(odx) | reinterpret_cast<uintptr_t>(odr)) & 31u) == 0;
     // pass 3
 #pragma unroll 1
     for (int u = t; u < nunits; u += G) {
@@ -1271,8 +1281,8 @@ __device__ __forceinline__ void tile_slerp_bwd_row(Team<WP, SPLIT> &tm, const AG
             part[i] = __fmul2_rn(__fmul2_rn(sgn2(al[i]), __fadd2_rn(b[i], fneg2(a[i]))), dt);
         }
         const int valid = u < nfull ? 8 : tail;
-        store8f(odx, u, gx, valid);
-        store8f(odr, u, gr, valid);
+        store8f(odx, u, gx, valid, a32);
+        store8f(odr, u, gr, valid, a32);
         if (wsl != nullptr) {
             float *l = wsl + 8 * u;
             const float4 p0 = make_float4(part[0].x, part[0].y, part[1].x, part[1].y);
