@@ -153,6 +153,16 @@ typedef struct {
                           stored [cols, ld] (element j of row r at [j * ld + r],
                           ld >= rows): GPT-2's Conv1D [in, out] weights.  Forward,
                           backward, renorm and the projections; not row_norms. */
+    int32_t tgroup;     /* with transposed = 1: G >= 1 consecutive stored columns
+                          per row (0 reads as 1), for ConvTranspose weights
+                          [in, out, k...] stored [in, out * G] with G the kernel's
+                          volume: row r holds the stored columns [r G, r G + G) of
+                          every stored row, element (j, m) at [j * ld + r G + m],
+                          so cols = in * G (a multiple of G), ld and ld_out >=
+                          rows * G.  1 <= G <= 256.  Must be 0 or 1 when
+                          transposed = 0.  (Grouped ConvTranspose: one segment per
+                          group.)  DragonScale package description, "Supported
+                          layers": ConvTranspose1d/2d/3d. */
 } ds_wseg;
 
 /* One activation matrix; x, r and y share the leading dimension ld.

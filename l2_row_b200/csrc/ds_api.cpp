@@ -446,17 +446,24 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         if (s.transposed != 0 && s.transposed != 1)
             return fail(DS_ERR_INVALID_ARG, where("transposed must be 0 or 1", i));
         const bool tr = s.transposed != 0;
+        if (s.tgroup < 0 || s.tgroup > 256 || (!tr && s.tgroup > 1))
+            return fail(DS_ERR_INVALID_ARG, where("tgroup must be 0 or 1, or 1..256 with transposed", i));
+        // G stored columns per unit row (ConvTranspose weights; 1 for Conv1D)
+        const int64_t G = tr ? std::max<int32_t>(1, s.tgroup) : 1;
+        if (tr && s.cols % G != 0)
+            return fail(DS_ERR_INVALID_ARG, where("transposed: cols is not a multiple of tgroup", i));
         // the stored matrix: [rows, ld] with cols used per row, or
-        // (transposed) [cols, ld] with rows used per stored row
-        const int64_t sr = tr ? s.cols : s.rows, sc = tr ? s.rows : s.cols;
+        // (transposed) [cols / G, ld] with rows * G used per stored row
+        const int64_t sr = tr ? s.cols / G : s.rows, sc = tr ? s.rows * G : s.cols;
         if (ds_status st = check_shape(s.rows, s.cols, tr ? std::max<int64_t>(s.ld, s.cols) : s.ld, i))
             return st;
-        if (tr && s.ld < s.rows)
-            return fail(DS_ERR_INVALID_ARG, where("transposed: leading dimension < rows", i));
-        if (tr && s.rows > (int64_t(1) << 31) - 1)
-            return fail(DS_ERR_INVALID_ARG, where("transposed: rows above 2^31 - 1", i));
+        if (tr && s.ld < sc)
+            return fail(DS_ERR_INVALID_ARG, where("transposed: leading dimension < rows * tgroup", i));
+        if (tr && sc > (int64_t(1) << 31) - 1)
+            return fail(DS_ERR_INVALID_ARG, where("transposed: rows * tgroup above 2^31 - 1", i));
         if (fwd_bwd && s.ld_out < sc)
-            return fail(DS_ERR_INVALID_ARG, where(tr ? "transposed: ld_out < rows" : "ld_out < cols", i));
+            return fail(DS_ERR_INVALID_ARG,
+                        where(tr ? "transposed: ld_out < rows * tgroup" : "ld_out < cols", i));
         if (!std::isfinite(s.radius))
             return fail(DS_ERR_INVALID_ARG, where("radius is not finite", i));
         rows[i] = tr ? 0 : s.rows; // transposed segments launch on their own
@@ -568,8 +575,9 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         // gradient / momentum) where the operation reads one
         const int eb = 4 + (cop == 1 ? esize : (cop == 3 || cop == 4) ? 4 : 0);
         std::vector<int> ct_of(static_cast<size_t>(nseg), 0), cl_of(static_cast<size_t>(nseg), 0);
+        auto grouped = [&](int i) { return segs[i].transposed && segs[i].tgroup > 1; };
         for (int i = 0; i < nseg; ++i) {
-            if (!segs[i].transposed || segs[i].rows == 0)
+            if (!segs[i].transposed || segs[i].rows == 0 || grouped(i))
                 continue;
             const int64_t K = segs[i].cols;
             for (const int budget : ds::kColTileBudgets) {
@@ -614,7 +622,8 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
                     return DS_OK;
                 };
                 for (int i = 0; i < nseg; ++i) {
-                    if (!segs[i].transposed || segs[i].rows == 0 || ct_of[i] != ct || (ct && cl_of[i] != cl))
+                    if (!segs[i].transposed || segs[i].rows == 0 || grouped(i) || ct_of[i] != ct ||
+                        (ct && cl_of[i] != cl))
                         continue;
                     if (n == (ct ? ds::col_tile_segments() : ds::kSegPerLaunch))
                         if (ds_status st = flush())
@@ -630,6 +639,43 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
                 if (ds_status st = flush())
                     return st;
             }
+        // grouped transposed rows (ConvTranspose): blocks of col_group_units(G)
+        // unit rows, one launch per table of segments
+        int n = 0;
+        int64_t units = 0;
+        auto flush_g = [&]() -> ds_status {
+            if (n == 0)
+                return DS_OK;
+            tp.nseg = n;
+            tp.unit_start[n] = units;
+            tp.eps = eps;
+            tp.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
+            if (const int e = ds::launch_colg(cop, bf16, tp, units, stream)) {
+                char buf[160];
+                std::snprintf(buf, sizeof(buf), "kernel launch failed (grouped transposed rows, cudaError %d)", e);
+                return fail(DS_ERR_CUDA, buf);
+            }
+            g_launches.fetch_add(1, std::memory_order_relaxed);
+            n = 0;
+            units = 0;
+            return DS_OK;
+        };
+        for (int i = 0; i < nseg; ++i) {
+            if (!grouped(i) || segs[i].rows == 0)
+                continue;
+            if (n == ds::kSegPerLaunch)
+                if (ds_status st = flush_g())
+                    return st;
+            const int G = segs[i].tgroup, U = ds::col_group_units(G);
+            tp.seg[n] = make(i, 0, segs[i].rows);
+            tp.seg[n].group = G;
+            tp.seg[n].nu = U;
+            tp.unit_start[n] = units;
+            units += (segs[i].rows + U - 1) / U;
+            ++n;
+        }
+        if (ds_status st = flush_g())
+            return st;
     }
     if (wop != W_BWD)
         return DS_OK;
@@ -671,8 +717,10 @@ ds_status run_norms(bool preserve, const ds_wseg *segs, int nseg, float eps, voi
             return st;
         if (preserve && !(std::isfinite(s.radius) && s.radius > 0.f))
             return fail(DS_ERR_INVALID_ARG, where("radius must be finite and > 0", i));
-        if (s.transposed)
+        if (s.transposed || s.tgroup > 1)
             return fail(DS_ERR_INVALID_ARG, where("transposed rows are not supported here", i));
+        if (s.tgroup < 0)
+            return fail(DS_ERR_INVALID_ARG, where("tgroup must be 0 or 1 here", i));
         if (s.rows == 0)
             continue;
         if (ds_status st = check_matrix(s.w, s.rows, s.ld, 4, "w", i))

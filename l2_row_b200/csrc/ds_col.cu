@@ -190,6 +190,158 @@ __global__ void __launch_bounds__(kCta) k_col(const __grid_constant__ WParams p)
 }
 
 // ---------------------------------------------------------------------------
+// Grouped transposed rows (ConvTranspose weights [in, out, k...] stored as
+// [in, out * G], G = the kernel's volume): unit row r is the G consecutive
+// stored columns [r G, r G + G) of every stored row, element (j, m) at
+// w[j * ld + r G + m].  A block owns U consecutive unit rows (the host
+// passes U in nu and G in group), i.e. the W = U G contiguous stored
+// columns of every stored row: thread t takes column t % W and the stored
+// rows t / W, t / W + S, ... (S = 256 / W lanes down the rows; threads past
+// S W idle).  Pass 1 sums w^2 (and w . d) per column in fp32, lane by lane
+// in row order, eight rows' loads in flight; each unit row then adds its
+// columns' sums in double, lane by lane and column by column.  A block
+// holding a unit row whose fp32 sum overflowed (or, at eps = 0, fell below
+// 2^-100) sums again in double.  Pass 2 re-reads the block's columns (from
+// L2) and writes the fp32 products with the scale rounded once (in double
+// for the blocks summed in double, each result rounded once).  Loads are
+// scalar: a unit row's G columns need not start on 16 bytes.
+template <int OP, bool B16>
+__global__ void __launch_bounds__(kCta) k_colg(const __grid_constant__ WParams p)
+{
+    constexpr bool TWO = OP == 1 || OP == 3 || OP == 4;
+    __shared__ double red[2][kCta]; // [lane ks][column c] at ks * W + c
+    __shared__ double fac[2][kCta]; // per unit row of the block (U <= 256)
+    const int64_t total = p.unit_start[p.nseg];
+    for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
+        const int si = find_segment(p, u);
+        const WSegK &sg = p.seg[si];
+        const int G = sg.group, U = sg.nu;
+        const int W = U * G, S = kCta / W;
+        const int64_t r0 = (u - p.unit_start[si]) * U;
+        const int nur = sg.rows - r0 < U ? static_cast<int>(sg.rows - r0) : U;
+        const int c = threadIdx.x % W, ks = threadIdx.x / W;
+        const bool act = ks < S && c < nur * G;
+        const int K = sg.cols / G;              // stored rows
+        const int64_t col = r0 * G + c;         // this thread's stored column
+        const bool d_bf16 = OP == 1 && B16;
+        const int64_t ld_d = OP == 1 ? sg.ld_out : sg.ld;
+        auto dval = [&](int j) -> float {
+            if constexpr (TWO) {
+                if (d_bf16)
+                    return bf_lo(static_cast<const uint16_t *>(sg.gy)[j * ld_d + col]);
+                return static_cast<const float *>(sg.gy)[j * ld_d + col];
+            } else {
+                return 0.f;
+            }
+        };
+        float s = 0.f, dd = 0.f;
+        if (act) {
+#pragma unroll 8
+            for (int j = ks; j < K; j += S) {
+                const float w = sg.w[j * sg.ld + col];
+                s = fmaf(w, w, s);
+                if constexpr (TWO)
+                    dd = fmaf(w, dval(j), dd);
+            }
+        }
+        if (threadIdx.x < S * W) {
+            red[0][threadIdx.x] = s;
+            red[1][threadIdx.x] = dd;
+        }
+        __syncthreads();
+        // each unit row's sums: lane by lane, column by column
+        auto unit_sums = [&](int rr, double &Sr, double &Dr) {
+            Sr = 0.0;
+            Dr = 0.0;
+            for (int k = 0; k < S; ++k)
+                for (int m = 0; m < G; ++m) {
+                    Sr += red[0][k * W + rr * G + m];
+                    if constexpr (TWO)
+                        Dr += red[1][k * W + rr * G + m];
+                }
+        };
+        bool need = false;
+        if (threadIdx.x < nur) {
+            double Sr, Dr;
+            unit_sums(threadIdx.x, Sr, Dr);
+            need = !(Sr <= static_cast<double>(FLT_MAX)) || (p.eps == 0.f && Sr < 0x1p-100);
+        }
+        const bool exact = __syncthreads_or(need) != 0;
+        if (exact) {
+            double se = 0.0, de = 0.0;
+            if (act) {
+                for (int j = ks; j < K; j += S) {
+                    const double w = sg.w[j * sg.ld + col];
+                    se = fma(w, w, se);
+                    if constexpr (TWO)
+                        de = fma(w, static_cast<double>(dval(j)), de);
+                }
+            }
+            if (threadIdx.x < S * W) {
+                red[0][threadIdx.x] = se;
+                red[1][threadIdx.x] = de;
+            }
+            __syncthreads();
+        }
+        if (threadIdx.x < nur) {
+            const int rr = threadIdx.x;
+            const int64_t r = r0 + rr;
+            double Sr, Dr;
+            unit_sums(rr, Sr, Dr);
+            Sr += static_cast<double>(p.eps);
+            const double n = sqrt(Sr);
+            const double g = (OP <= 1 && sg.gain) ? static_cast<double>(__ldg(sg.gain + r * sg.gain_stride)) : 1.0;
+            fac[0][rr] = g * static_cast<double>(sg.radius) / n;
+            fac[1][rr] = TWO ? Dr / Sr : 0.0;
+            if constexpr (OP == 1) {
+                if (sg.gain)
+                    sg.grad_g[r] = static_cast<float>(static_cast<double>(sg.radius) * Dr / n);
+            }
+        }
+        __syncthreads();
+        auto put = [&](int j, float w, float y, float e) {
+            if constexpr (OP == 0) {
+                if constexpr (B16)
+                    static_cast<uint16_t *>(sg.out)[j * sg.ld_out + col] = static_cast<uint16_t>(pack_bf2(y, 0.f) & 0xFFFFu);
+                else
+                    static_cast<float *>(sg.out)[j * sg.ld_out + col] = y;
+            } else if constexpr (OP == 2) {
+                const_cast<float *>(sg.w)[j * sg.ld + col] = y;
+            } else {
+                sg.grad_w[j * sg.ld + col] = e;
+                if constexpr (OP == 4)
+                    const_cast<float *>(sg.w)[j * sg.ld + col] = y;
+            }
+        };
+        if (act && !exact) {
+            const float sc = static_cast<float>(fac[0][c / G]), qt = static_cast<float>(fac[1][c / G]);
+#pragma unroll 8
+            for (int j = ks; j < K; j += S) {
+                const float w = sg.w[j * sg.ld + col];
+                float e = 0.f;
+                if constexpr (TWO) {
+                    const float ei = fmaf(-w, qt, dval(j));
+                    e = OP == 1 ? sc * ei : ei;
+                }
+                put(j, w, w * sc, e);
+            }
+        } else if (act) {
+            const double sc = fac[0][c / G], qt = fac[1][c / G];
+            for (int j = ks; j < K; j += S) {
+                const double w = sg.w[j * sg.ld + col];
+                float e = 0.f;
+                if constexpr (TWO) {
+                    const double ei = static_cast<double>(dval(j)) - w * qt;
+                    e = static_cast<float>(OP == 1 ? sc * ei : ei);
+                }
+                put(j, static_cast<float>(w), static_cast<float>(w * sc), e);
+            }
+        }
+        __syncthreads(); // red and fac are reused by the next block of unit rows
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Transposed rows in column tiles staged whole.  A tile is CT consecutive
 // unit rows (stored columns c0 .. c0 + CT) over the whole unit-row length K
 // (every stored row); a cluster of CL CTAs owns one tile, CTA k staging the
@@ -521,6 +673,14 @@ cudaError_t launch_col_t(const WParams &p, int64_t units, cudaStream_t st)
     return cudaGetLastError();
 }
 
+template <int OP, bool B16>
+cudaError_t launch_colg_t(const WParams &p, int64_t units, cudaStream_t st)
+{
+    const int grid = static_cast<int>(units < 148 * 8 ? units : 148 * 8);
+    k_colg<OP, B16><<<grid, kCta, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
 template <int OP, bool B16, int CT>
 cudaError_t launch_colt_t(const ColtParams &p, int64_t units, int cl, int smem, cudaStream_t st)
 {
@@ -622,6 +782,24 @@ int launch_col(int op, bool b16, const WParams &p, int64_t units, void *stream)
     case 2: return launch_col_t<2, false>(p, units, st);
     case 3: return launch_col_t<3, false>(p, units, st);
     case 4: return launch_col_t<4, false>(p, units, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+int col_group_units(int group)
+{
+    return group >= 64 ? 1 : 64 / group;
+}
+
+int launch_colg(int op, bool b16, const WParams &p, int64_t units, void *stream)
+{
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (op) {
+    case 0: return b16 ? launch_colg_t<0, true>(p, units, st) : launch_colg_t<0, false>(p, units, st);
+    case 1: return b16 ? launch_colg_t<1, true>(p, units, st) : launch_colg_t<1, false>(p, units, st);
+    case 2: return launch_colg_t<2, false>(p, units, st);
+    case 3: return launch_colg_t<3, false>(p, units, st);
+    case 4: return launch_colg_t<4, false>(p, units, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -241,6 +241,11 @@ int launch_row_norms(const RNParams &p, int sms, void *stream);
 // p's unit_start counts tiles of col_tile_rows() rows.
 int launch_col(int op, bool b16, const WParams &p, int64_t units, void *stream);
 int col_tile_rows();
+// Grouped transposed rows (ds_col.cu, ConvTranspose): each segment's
+// `group` = G stored columns per unit row and `nu` = col_group_units(G)
+// unit rows per block; p's unit_start counts blocks.
+int col_group_units(int group);
+int launch_colg(int op, bool b16, const WParams &p, int64_t units, void *stream);
 // Transposed rows in whole column tiles (ds_col.cu): tiles of ct unit rows
 // (32, 64 or 128) over every stored row, a cluster of cl CTAs per tile
 // (bands of ceil(K / cl) stored rows each, loaded as 2-D TMA boxes); p's

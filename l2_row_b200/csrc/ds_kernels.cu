@@ -20,8 +20,6 @@ namespace ds {
 
 namespace {
 
-constexpr float kZero = 0.f;
-
 // ------------------------------------------------------------- unit I/O --
 
 __device__ __forceinline__ float4 quad_f32(const float *row, int u, int cols)

@@ -105,11 +105,6 @@ __device__ __forceinline__ uint32_t peer_addr(const void *local, uint32_t rank)
     return r;
 }
 
-__device__ __forceinline__ void peer_store_f32(uint32_t addr, float v)
-{
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
-}
-
 __device__ __forceinline__ void peer_store_u32(uint32_t addr, uint32_t v)
 {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");

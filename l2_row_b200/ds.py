@@ -54,7 +54,7 @@ class ds_wseg(ct.Structure):
     _fields_ = [("w", ct.c_void_p), ("gain", ct.c_void_p), ("w_eff", ct.c_void_p), ("gy", ct.c_void_p),
                 ("grad_w", ct.c_void_p), ("grad_g", ct.c_void_p), ("rows", ct.c_int64), ("cols", ct.c_int64),
                 ("ld", ct.c_int64), ("ld_out", ct.c_int64), ("radius", ct.c_float), ("gain_scalar", ct.c_int32),
-                ("rnorm", ct.c_void_p), ("transposed", ct.c_int32)]
+                ("rnorm", ct.c_void_p), ("transposed", ct.c_int32), ("tgroup", ct.c_int32)]
 
 
 class ds_aseg(ct.Structure):
@@ -207,7 +207,10 @@ class WSeg:
     (per-row parts, then their sum).  rnorm: fp32 [R] output of
     ds_row_norms / ds_gain_preserve.  transposed: the unit rows are the
     columns of w (GPT-2 Conv1D, stored [in, out] = [C, R]); w, w_eff, gy and
-    grad_w are then given in that stored layout."""
+    grad_w are then given in that stored layout.  tgroup (with transposed):
+    G consecutive stored columns per unit row, for a ConvTranspose weight
+    [in, out, k...] viewed as [in, out * G] (G = the kernel's volume): unit
+    rows R = out, row length C = in * G."""
 
     w: Any
     gain: Any = None
@@ -219,10 +222,14 @@ class WSeg:
     gain_scalar: bool = False
     rnorm: Any = None
     transposed: bool = False
+    tgroup: int = 1
 
     def to_c(self) -> ds_wseg:
         SR, SC = (int(self.w.shape[0]), int(self.w.shape[1]))   # the stored shape
-        R, C = (SC, SR) if self.transposed else (SR, SC)
+        G = int(self.tgroup) if self.transposed else 1
+        if G < 1 or SC % G:
+            raise ValueError("tgroup must be >= 1 and divide the stored columns")
+        R, C = (SC // G, SR * G) if self.transposed else (SR, SC)
         w, ld = _mat(self.w, "w", SR, SC)
         weff, ld_out = _mat(self.w_eff, "w_eff", SR, SC)
         gy, ld_gy = _mat(self.gy, "gy", SR, SC)
@@ -233,7 +240,7 @@ class WSeg:
             raise ValueError("grad_w must share w's leading dimension")
         return ds_wseg(w, _vec(self.gain), weff, gy, gw, _vec(self.grad_g), R, C, ld,
                        ld_out if self.w_eff is not None else ld_gy, float(self.radius), int(bool(self.gain_scalar)),
-                       _vec(self.rnorm), int(bool(self.transposed)))
+                       _vec(self.rnorm), int(bool(self.transposed)), G if self.transposed else 0)
 
 
 @dataclass

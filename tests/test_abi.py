@@ -487,6 +487,26 @@ def test_transposed_validation():
     assert ds.ds_launch_count() == before
 
 
+def test_grouped_transposed_validation():
+    """ConvTranspose rows (transposed with tgroup G): cols a multiple of G,
+    ld and ld_out >= rows * G, 1 <= G <= 256, and no tgroup without
+    transposed; row lengths refuse them."""
+    E = ds
+    before = ds.ds_launch_count()
+    # rows 4 of G = 2 columns each: stored [cols / 2, ld] with ld >= 8
+    ok = dict(transposed=1, tgroup=2, rows=4, cols=8, ld=8, ld_out=8)
+    bad = [dict(ok, tgroup=3),                       # 8 is not a multiple of 3
+           dict(ok, ld=7), dict(ok, ld_out=7),      # < rows * G
+           dict(ok, tgroup=257), dict(ok, tgroup=-1),
+           dict(transposed=0, tgroup=2)]
+    for kw in bad:
+        assert call_w("ds_wn_forward", [wseg(**kw)]) == E.DS_ERR_INVALID_ARG, kw
+        assert call_w("ds_wn_backward", [wseg(**kw)]) == E.DS_ERR_INVALID_ARG, kw
+    arr = (ds.ds_wseg * 1)(wseg(tgroup=2, rnorm=BASE + (5 << 30)))
+    assert ds.lib().ds_row_norms(arr, 1, ct.c_float(1e-6), None) == E.DS_ERR_INVALID_ARG
+    assert ds.ds_launch_count() == before
+
+
 def test_python_segments_map_shapes():
     """The binding's segment builders: a transposed weight gives rows = its
     stored columns; q/k segments count heads from the widths and refuse a
@@ -498,6 +518,11 @@ def test_python_segments_map_shapes():
     assert (c.rows, c.cols, c.ld, c.transposed) == (10, 6, 10, 1)
     c = ds.WSeg(w=w).to_c()
     assert (c.rows, c.cols, c.transposed) == (6, 10, 0)
+    # a ConvTranspose1d weight [in = 6, out = 5, k = 2] viewed as [6, 10]
+    c = ds.WSeg(w=w, transposed=True, tgroup=2).to_c()
+    assert (c.rows, c.cols, c.ld, c.transposed, c.tgroup) == (5, 12, 10, 1, 2)
+    with pytest.raises(ValueError):
+        ds.WSeg(w=w, transposed=True, tgroup=3).to_c()
     q = torch.zeros(3, 4 * 64, dtype=torch.bfloat16)
     k = torch.zeros(3, 2 * 64, dtype=torch.bfloat16)
     pos = torch.zeros(3, dtype=torch.int32)

@@ -164,3 +164,164 @@ def test_extreme_columns(eps):
     ds.ds_row_renorm([ds.WSeg(w=wd, transposed=True)], eps)
     torch.cuda.synchronize()
     gu.check_renorm(_seg_t(w, None, None), wd.t().contiguous(), eps, what="extreme renorm")
+
+
+# ConvTranspose weights [in, out, k...] stored [in, out * G] (G = the kernel's
+# volume): unit row r = the G columns [r G, r G + G) of every stored row.
+# (in, out, G): ConvTranspose2d 3x3, ConvTranspose1d k=4, ConvTranspose3d
+# 3x3x3, a ragged one, a 4x4 decoder layer, the largest G, and G >= 128
+# (one unit row per block).
+GROUPED = [(64, 32, 9), (128, 64, 4), (16, 8, 27), (5, 7, 6), (512, 256, 16), (3, 2, 256), (40, 3, 130)]
+
+
+def _unit_rows(stored: np.ndarray, G: int) -> np.ndarray:
+    """[in, out * G] -> the unit rows [out, in * G] (stored row j's G
+    elements of unit row r at j G .. j G + G - 1)."""
+    K, N = stored.shape
+    return np.ascontiguousarray(stored.reshape(K, N // G, G).transpose(1, 0, 2).reshape(N // G, K * G))
+
+
+def _dev_unit_rows(t: torch.Tensor, G: int) -> torch.Tensor:
+    K, N = t.shape
+    return t.reshape(K, N // G, G).permute(1, 0, 2).reshape(N // G, K * G).contiguous()
+
+
+def _grouped(rng, K, R, G):
+    """Weights drifted per output channel, stored [K, R G]."""
+    units = wl.drifted_rows(rng, R, K * G, 0.02)                     # [R, K G]
+    return np.ascontiguousarray(units.reshape(R, K, G).transpose(1, 0, 2).reshape(K, R * G))
+
+
+def _ld(n: int) -> int:
+    """A leading dimension >= n whose rows start on 16 bytes in fp32 and bf16."""
+    return (n + 7) // 8 * 8
+
+
+def _dev(a: np.ndarray, ld: int, bf16=False):
+    """a (fp32, or bf16 bits) in a [K, ld] device buffer with guard rows;
+    returns (view, buffer, canary)."""
+    K, N = a.shape
+    dt, canary = (torch.bfloat16, gu.CANARY_BF16) if bf16 else (torch.float32, gu.CANARY_F32)
+    v, buf = gu.padded(K, N, ld, dt, canary)
+    v.copy_(gu.dev_bf16(a) if bf16 else gu.dev_f32(a))
+    return v, buf, canary
+
+
+@pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
+def test_grouped_forward(out_dtype):
+    rng = np.random.default_rng(96)
+    for K, R, G in GROUPED:
+        w = _grouped(rng, K, R, G)
+        g = wl.gains(rng, R)
+        ld = _ld(R * G)
+        wd, _, _ = _dev(w, ld)
+        dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+        canary = gu.CANARY_BF16 if out_dtype == "bf16" else gu.CANARY_F32
+        ld_o = ld + 8
+        o, obuf = gu.padded(K, R * G, ld_o, dt, canary)
+        ds.ds_wn_forward([ds.WSeg(w=wd, gain=gu.dev_f32(g), w_eff=o, transposed=True, tgroup=G)], out_dtype, 1e-6)
+        torch.cuda.synchronize()
+        assert gu.guards_intact(obuf, K, R * G, ld_o, canary), (K, R, G)
+        seg = wl.WeightSeg("g", _unit_rows(w, G), g, None)
+        gu.check_forward(seg, _dev_unit_rows(o, G), 1e-6, out_dtype, what=f"grouped fwd [{K},{R}x{G}]")
+
+
+@pytest.mark.parametrize("gy_dtype", ["bf16", "f32"])
+def test_grouped_backward(gy_dtype):
+    rng = np.random.default_rng(97)
+    for K, R, G in GROUPED:
+        w = _grouped(rng, K, R, G)
+        g = wl.gains(rng, R)
+        gy = rng.standard_normal((K, R * G)).astype(np.float32) * np.float32(1e-3)
+        if gy_dtype == "bf16":
+            gy = wl.to_bf16_bits(gy)
+        ld = _ld(R * G)
+        wd, _, _ = _dev(w, ld)
+        gyd, _, _ = _dev(gy, ld, bf16=gy_dtype == "bf16")
+        gw, gwbuf = gu.padded(K, R * G, ld, torch.float32, gu.CANARY_F32)
+        gg = torch.empty(R, dtype=torch.float32, device="cuda")
+        ds.ds_wn_backward([ds.WSeg(w=wd, gain=gu.dev_f32(g), gy=gyd, grad_w=gw, grad_g=gg, transposed=True,
+                                   tgroup=G)], gy_dtype, 1e-6)
+        torch.cuda.synchronize()
+        assert gu.guards_intact(gwbuf, K, R * G, ld, gu.CANARY_F32), (K, R, G)
+        seg = wl.WeightSeg("g", _unit_rows(w, G), g, _unit_rows(gy, G))
+        gu.check_backward(seg, _dev_unit_rows(gw, G), gg, 1e-6, what=f"grouped bwd [{K},{R}x{G}]")
+
+
+def test_grouped_renorm_projections_and_scalar_gain():
+    rng = np.random.default_rng(98)
+    for K, R, G in GROUPED:
+        ld = _ld(R * G)
+        w = _grouped(rng, K, R, G)
+        wd, wbuf, can = _dev(w, ld)
+        ds.ds_row_renorm([ds.WSeg(w=wd, transposed=True, tgroup=G)], 1e-6)
+        torch.cuda.synchronize()
+        assert gu.guards_intact(wbuf, K, R * G, ld, can), (K, R, G)
+        gu.check_renorm(wl.WeightSeg("g", _unit_rows(w, G), None, None), _dev_unit_rows(wd, G), 1e-6,
+                        what=f"grouped renorm [{K},{R}x{G}]")
+        w2 = _grouped(rng, K, R, G)
+        G2 = rng.standard_normal((K, R * G)).astype(np.float32)
+        wd2, _, _ = _dev(w2, ld)
+        Gd, _, _ = _dev(G2, ld)
+        ds.ds_grad_project([ds.WSeg(w=wd2, grad_w=Gd, transposed=True, tgroup=G)], 1e-6)
+        torch.cuda.synchronize()
+        seg2 = wl.WeightSeg("g", _unit_rows(w2, G), None, _unit_rows(G2, G))
+        gu.check_project(seg2, _dev_unit_rows(Gd, G), 1e-6, what=f"grouped project [{K},{R}x{G}]")
+        md, _, _ = _dev(G2, ld)
+        ds.ds_renorm_momentum([ds.WSeg(w=wd2, grad_w=md, transposed=True, tgroup=G)], 1e-6)
+        torch.cuda.synchronize()
+        gu.check_momentum(seg2, _dev_unit_rows(wd2, G), _dev_unit_rows(md, G), 1e-6,
+                          what=f"grouped momentum [{K},{R}x{G}]")
+    # one gain for the whole layer: per-row parts, then their sum
+    K, R, G = 64, 32, 9
+    ld = _ld(R * G)
+    w = _grouped(rng, K, R, G)
+    gy = wl.to_bf16_bits(rng.standard_normal((K, R * G)).astype(np.float32) * np.float32(1e-3))
+    wd, _, _ = _dev(w, ld)
+    gyd, _, _ = _dev(gy, ld, bf16=True)
+    gw, _ = gu.padded(K, R * G, ld, torch.float32, gu.CANARY_F32)
+    gg = torch.empty(R + 1, dtype=torch.float32, device="cuda")
+    gs = torch.full((1,), 0.75, dtype=torch.float32, device="cuda")
+    ds.ds_wn_backward([ds.WSeg(w=wd, gain=gs, gy=gyd, grad_w=gw, grad_g=gg, transposed=True, tgroup=G,
+                               gain_scalar=True)], "bf16", 1e-6)
+    torch.cuda.synchronize()
+    seg = wl.WeightSeg("g", _unit_rows(w, G), np.full(R, 0.75, np.float32), _unit_rows(gy, G))
+    gu.check_backward(seg, _dev_unit_rows(gw, G), gg[:R], 1e-6, what="grouped, scalar gain")
+    h = gu.host_f32(gg)
+    assert abs(float(h[R]) - float(np.sum(h[:R], dtype=np.float64))) <= np.spacing(np.float32(abs(h[R])))
+
+
+@pytest.mark.parametrize("eps", [1e-6, 0.0])
+def test_grouped_extreme_channels(eps):
+    """ConvTranspose channels whose fp32 sums overflow (|w| ~ 1e25) or, at
+    eps = 0, fall below 2^-100 (|w| ~ 1e-30) take the double pass; the other
+    blocks keep fp32.  Against the oracle."""
+    rng = np.random.default_rng(99)
+    K, R, G = 64, 32, 9
+    ld = _ld(R * G)
+    w = _grouped(rng, K, R, G)
+    w[:, 2 * G:3 * G] *= np.float32(1e27)          # channel 2
+    w[:, 20 * G:21 * G] *= np.float32(1e-28)       # channel 20, another block
+    g = wl.gains(rng, R)
+    for out_dtype in ("f32", "bf16"):
+        wd, _, _ = _dev(w, ld)
+        dt = torch.bfloat16 if out_dtype == "bf16" else torch.float32
+        o = torch.empty(K, ld, dtype=dt, device="cuda")[:, :R * G]
+        ds.ds_wn_forward([ds.WSeg(w=wd, gain=gu.dev_f32(g), w_eff=o, transposed=True, tgroup=G)], out_dtype, eps)
+        torch.cuda.synchronize()
+        gu.check_forward(wl.WeightSeg("g", _unit_rows(w, G), g, None), _dev_unit_rows(o, G), eps, out_dtype,
+                         what=f"grouped extreme fwd {out_dtype}")
+    gy = wl.to_bf16_bits(rng.standard_normal((K, R * G)).astype(np.float32) * np.float32(1e-3))
+    wd, _, _ = _dev(w, ld)
+    gyd, _, _ = _dev(gy, ld, bf16=True)
+    gw, _ = gu.padded(K, R * G, ld, torch.float32, gu.CANARY_F32)
+    gg = torch.empty(R, dtype=torch.float32, device="cuda")
+    ds.ds_wn_backward([ds.WSeg(w=wd, gain=gu.dev_f32(g), gy=gyd, grad_w=gw, grad_g=gg, transposed=True, tgroup=G)],
+                      "bf16", eps)
+    torch.cuda.synchronize()
+    gu.check_backward(wl.WeightSeg("g", _unit_rows(w, G), g, _unit_rows(gy, G)), _dev_unit_rows(gw, G), gg, eps,
+                      what="grouped extreme bwd")
+    ds.ds_row_renorm([ds.WSeg(w=wd, transposed=True, tgroup=G)], eps)
+    torch.cuda.synchronize()
+    gu.check_renorm(wl.WeightSeg("g", _unit_rows(w, G), None, None), _dev_unit_rows(wd, G), eps,
+                    what="grouped extreme renorm")
