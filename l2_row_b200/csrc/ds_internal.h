@@ -54,8 +54,11 @@ constexpr int kTileSlotMaxBytes = 65536;       // largest CTA-path slot of the a
 constexpr int kTileSlotMaxWeightBytes = 114688;
 constexpr int kMaxTileSlots = 13;         // 13 x 16 KB = 208 KB of the 227 KB per CTA
 constexpr int kTileMaxRowsPerSlot = 64;
-// Two-pass path: pipeline stages (the chunk size is per operation).
-constexpr int kStages = 4;
+// Two-pass path: pipeline stages (the chunk size is per operation).  Three
+// stages let four CTAs share an SM where four stages let three; on rows of
+// 262,144 columns that took the forward 107 -> 97 us, slerp 384 -> 326 and
+// l2 150 -> 127 (two stages: 114, 334, 121).
+constexpr int kStages = 3;
 
 // Rows split over a cluster of `ncta` CTAs (staged cluster classes): CTA k
 // stages units [k * per, min(nu, (k + 1) * per)) of every row, per =
