@@ -575,11 +575,15 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         // gradient / momentum) where the operation reads one
         const int eb = 4 + (cop == 1 ? esize : (cop == 3 || cop == 4) ? 4 : 0);
         std::vector<int> ct_of(static_cast<size_t>(nseg), 0), cl_of(static_cast<size_t>(nseg), 0);
-        auto grouped = [&](int i) { return segs[i].transposed && segs[i].tgroup > 1; };
+        // G stored columns per unit row: the tiles take G = 1 and powers of
+        // two up to 32 (a tile then holds whole unit rows); other G, and
+        // grouped rows too tall for the tiles, take the grouped kernel
+        auto gsize = [&](int i) { return segs[i].transposed && segs[i].tgroup > 1 ? segs[i].tgroup : 1; };
+        auto tile_group = [&](int g) { return g == 1 || (g <= 32 && (g & (g - 1)) == 0); };
         for (int i = 0; i < nseg; ++i) {
-            if (!segs[i].transposed || segs[i].rows == 0 || grouped(i))
+            if (!segs[i].transposed || segs[i].rows == 0 || !tile_group(gsize(i)))
                 continue;
-            const int64_t K = segs[i].cols;
+            const int64_t K = segs[i].cols / gsize(i);   // stored rows
             for (const int budget : ds::kColTileBudgets) {
                 for (const int ct : {128, 64, 32}) {
                     for (const int cl : {1, 2, 4, 8})
@@ -622,18 +626,20 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
                     return DS_OK;
                 };
                 for (int i = 0; i < nseg; ++i) {
-                    if (!segs[i].transposed || segs[i].rows == 0 || grouped(i) || ct_of[i] != ct ||
-                        (ct && cl_of[i] != cl))
+                    if (!segs[i].transposed || segs[i].rows == 0 || ct_of[i] != ct || (ct && cl_of[i] != cl) ||
+                        (!ct && gsize(i) > 1))
                         continue;
                     if (n == (ct ? ds::col_tile_segments() : ds::kSegPerLaunch))
                         if (ds_status st = flush())
                             return st;
                     const int tile = ct ? ct : ds::col_tile_rows();
+                    const int64_t G = gsize(i);
                     tp.seg[n] = make(i, 0, segs[i].rows);
+                    tp.seg[n].group = static_cast<int32_t>(G);
                     tp.unit_start[n] = units;
-                    units += (segs[i].rows + tile - 1) / tile;
+                    units += (segs[i].rows * G + tile - 1) / tile;   // tiles of stored columns
                     if (ct)
-                        smem = std::max(smem, ds::col_tile_smem(ct, cl, (segs[i].cols + cl - 1) / cl, eb));
+                        smem = std::max(smem, ds::col_tile_smem(ct, cl, (segs[i].cols / G + cl - 1) / cl, eb));
                     ++n;
                 }
                 if (ds_status st = flush())
@@ -661,7 +667,7 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
             return DS_OK;
         };
         for (int i = 0; i < nseg; ++i) {
-            if (!grouped(i) || segs[i].rows == 0)
+            if (gsize(i) == 1 || ct_of[i] != 0 || segs[i].rows == 0)
                 continue;
             if (n == ds::kSegPerLaunch)
                 if (ds_status st = flush_g())

@@ -405,9 +405,13 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
     const int64_t unit = blockIdx.x / ncta;
     const int si = find_segment(p, unit);
     const WSegK &sg = p.seg[si];
-    const int64_t c0 = (unit - p.unit_start[si]) * CT;          // first unit row of the tile (a stored column)
-    const int ncols = static_cast<int>(sg.rows - c0 < CT ? sg.rows - c0 : CT);
-    const int K = sg.cols;
+    // G stored columns per unit row (ConvTranspose; 1 for Conv1D; a power
+    // of two <= 32, so a tile holds whole unit rows)
+    const int G = sg.group > 1 ? sg.group : 1;
+    const int64_t NC = sg.rows * G;                              // stored columns
+    const int64_t c0 = (unit - p.unit_start[si]) * CT;          // first stored column of the tile
+    const int ncols = static_cast<int>(NC - c0 < CT ? NC - c0 : CT);
+    const int K = sg.cols / G;
     const int band = (K + static_cast<int>(ncta) - 1) / static_cast<int>(ncta);
     const int k0 = min(K, static_cast<int>(rank) * band), nk = min(K, k0 + band) - k0;
     const bool d_bf16 = OP == 1 && B16;
@@ -531,14 +535,36 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
             }
         }
     }
+    // per column S (and D), identical in every CTA; with G > 1 each column
+    // then takes its unit row's sums: the G columns added in order
+    auto unit_sums = [&](double &Sc, double &Dc) {
+        if (G == 1)
+            return;
+        if (threadIdx.x < CT) {
+            fac[0][threadIdx.x] = Sc;
+            fac[1][threadIdx.x] = Dc;
+        }
+        __syncthreads();
+        if (threadIdx.x < CT) {
+            const int b = threadIdx.x / G * G;
+            Sc = 0.0;
+            Dc = 0.0;
+            for (int m = 0; m < G; ++m) {
+                Sc += fac[0][b + m];
+                Dc += fac[1][b + m];
+            }
+        }
+        __syncthreads();
+    };
     cluster_wait();   // every peer has started (arrival at kernel start)
     double S, D;
     cluster_sums(S, D);
+    unit_sums(S, D);
     // A column whose fp32 sum overflowed (or, at eps = 0, fell below
     // 2^-100) takes the tile through an exact pass: the band summed again
     // in double and a second exchange, then double arithmetic in pass 2.
     // S is the same in every CTA, so every CTA takes the same branch.
-    const bool need = threadIdx.x < CT && c0 + threadIdx.x < sg.rows &&
+    const bool need = threadIdx.x < CT && c0 + threadIdx.x < NC &&
                       (!(S <= static_cast<double>(FLT_MAX)) || (p.eps == 0.f && S < 0x1p-100));
     const bool exact = __syncthreads_or(need) != 0;
     if (exact) {
@@ -573,11 +599,12 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
             }
         }
         cluster_sums(S, D);
+        unit_sums(S, D);
     }
     if (threadIdx.x < CT) {
         const int c = threadIdx.x;
-        const int64_t r = c0 + c;
-        if (r < sg.rows) {
+        const int64_t r = (c0 + c) / G;   // the unit row of this column
+        if (c0 + c < NC) {
             S += static_cast<double>(p.eps);
             const double n = sqrt(S);
             const double g = (OP <= 1 && sg.gain) ? static_cast<double>(__ldg(sg.gain + r * sg.gain_stride)) : 1.0;
@@ -585,7 +612,7 @@ __global__ void __launch_bounds__(kCta) k_colt(const __grid_constant__ ColtParam
             if constexpr (TWO)
                 fac[1][c] = D / S;
             if constexpr (OP == 1) {
-                if (sg.gain && rank == 0 && ok)
+                if (sg.gain && rank == 0 && ok && (c0 + c) % G == 0)
                     sg.grad_g[r] = static_cast<float>(static_cast<double>(sg.radius) * D / n);
             }
         } else {
@@ -813,17 +840,18 @@ int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &w, in
     const bool two = op == 1 || op == 3 || op == 4;
     for (int i = 0; i < w.nseg; ++i) {
         const WSegK &sg = w.seg[i];
-        const int64_t K = sg.cols, band = (K + cl - 1) / cl;
+        const int64_t G = sg.group > 1 ? sg.group : 1;
+        const int64_t K = sg.cols / G, N = sg.rows * G, band = (K + cl - 1) / cl;
         const int bh = col_tile_box_rows(band);
         p.seg[i] = sg;
         p.unit_start[i] = w.unit_start[i];
         p.box_h[i] = bh;
-        if (!encode_map(&p.tmw[i], sg.w, false, K, sg.rows, sg.ld, ct, bh))
+        if (!encode_map(&p.tmw[i], sg.w, false, K, N, sg.ld, ct, bh))
             return cudaErrorInvalidValue;
         if (two) {
             const bool d16 = op == 1 && b16;
             const int64_t ld_d = op == 1 ? sg.ld_out : sg.ld;
-            if (!encode_map(&p.tmd[i], sg.gy, d16, K, sg.rows, ld_d, ct, bh))
+            if (!encode_map(&p.tmd[i], sg.gy, d16, K, N, ld_d, ct, bh))
                 return cudaErrorInvalidValue;
         }
     }

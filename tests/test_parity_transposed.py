@@ -169,9 +169,12 @@ def test_extreme_columns(eps):
 # ConvTranspose weights [in, out, k...] stored [in, out * G] (G = the kernel's
 # volume): unit row r = the G columns [r G, r G + G) of every stored row.
 # (in, out, G): ConvTranspose2d 3x3, ConvTranspose1d k=4, ConvTranspose3d
-# 3x3x3, a ragged one, a 4x4 decoder layer, the largest G, and G >= 128
-# (one unit row per block).
-GROUPED = [(64, 32, 9), (128, 64, 4), (16, 8, 27), (5, 7, 6), (512, 256, 16), (3, 2, 256), (40, 3, 130)]
+# 3x3x3, a ragged one, a 4x4 decoder layer, the largest G, G >= 64 (one unit
+# row per block), ConvTranspose3d 2x2x2 with a ragged out, and a 2x2 layer too
+# tall for the column tiles.  Powers of two up to 32 take the column tiles
+# (whole unit rows per tile), the rest the grouped kernel.
+GROUPED = [(64, 32, 9), (128, 64, 4), (16, 8, 27), (5, 7, 6), (512, 256, 16), (3, 2, 256), (40, 3, 130),
+           (96, 13, 8), (14000, 6, 4)]
 
 
 def _unit_rows(stored: np.ndarray, G: int) -> np.ndarray:
@@ -292,12 +295,14 @@ def test_grouped_renorm_projections_and_scalar_gain():
 
 
 @pytest.mark.parametrize("eps", [1e-6, 0.0])
-def test_grouped_extreme_channels(eps):
+@pytest.mark.parametrize("G", [9, 16])
+def test_grouped_extreme_channels(eps, G):
     """ConvTranspose channels whose fp32 sums overflow (|w| ~ 1e25) or, at
     eps = 0, fall below 2^-100 (|w| ~ 1e-30) take the double pass; the other
-    blocks keep fp32.  Against the oracle."""
+    blocks keep fp32 (G = 9: the grouped kernel; G = 16: column tiles of whole
+    unit rows).  Against the oracle."""
     rng = np.random.default_rng(99)
-    K, R, G = 64, 32, 9
+    K, R = 64, 32
     ld = _ld(R * G)
     w = _grouped(rng, K, R, G)
     w[:, 2 * G:3 * G] *= np.float32(1e27)          # channel 2
