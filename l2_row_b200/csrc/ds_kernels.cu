@@ -4,9 +4,10 @@
 // bounded-wait self-test).
 //
 //   * stream  : a cluster of 8 CTAs per row, each streaming its slice
-//               through a 4-stage shared-memory ring filled by bulk (TMA)
-//               copies, once per pass (the re-reads hit L2).  Rows of any
-//               length; partial sums meet through distributed shared memory.
+//               through a kStages-deep shared-memory ring filled by bulk
+//               (TMA) copies, once per pass (most re-reads hit L2).  Rows of
+//               any length; partial sums meet through distributed shared
+//               memory.
 // Operations (sources cited in include/ds.h):
 //   wn_forward, wn_backward, row_renorm : DragonScale unit rows with gains
 //   grad_project, renorm_momentum       : DragonScale "Optimizer" (rescale)
