@@ -575,6 +575,9 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
         // gradient / momentum) where the operation reads one
         const int eb = 4 + (cop == 1 ? esize : (cop == 3 || cop == 4) ? 4 : 0);
         std::vector<int> ct_of(static_cast<size_t>(nseg), 0), cl_of(static_cast<size_t>(nseg), 0);
+        // Per segment: the first budget that holds some tile shape, and in it
+        // the smallest cluster, then the widest tile (fewer CTAs meeting at
+        // each tile's barrier measured faster than wider tiles).
         // G stored columns per unit row: the tiles take G = 1 and powers of
         // two up to 32 (a tile then holds whole unit rows); other G, and
         // grouped rows too tall for the tiles, take the grouped kernel
@@ -585,8 +588,8 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
                 continue;
             const int64_t K = segs[i].cols / gsize(i);   // stored rows
             for (const int budget : ds::kColTileBudgets) {
-                for (const int ct : {128, 64, 32}) {
-                    for (const int cl : {1, 2, 4, 8})
+                for (const int cl : {1, 2, 4, 8}) {
+                    for (const int ct : {128, 64, 32})
                         if (ds::col_tile_smem(ct, cl, (K + cl - 1) / cl, eb) <= budget) {
                             ct_of[i] = ct;
                             cl_of[i] = cl;
