@@ -1,6 +1,6 @@
 """The benchmark harness end to end on the GPU: one short run of the default
-step with the extra report of every other workload, and one of the
-reference arm's line format, checked for the keys the JSON line promises."""
+step with the extra report of every other workload, checked for the keys
+the JSON line promises."""
 from __future__ import annotations
 
 import json

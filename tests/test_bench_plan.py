@@ -69,3 +69,23 @@ def test_extras_cover_every_other_workload():
     """After the default step the bench reports every other workload."""
     assert set(bench.EXTRA_CONFIGS) == set(bench.WORKLOADS) - {"step"}
     assert len(bench.EXTRA_CONFIGS) == len(set(bench.EXTRA_CONFIGS))
+
+
+def test_reference_arm_line():
+    """bench.py --impl reference (the float64 oracle on the host cores) prints
+    one JSON line with the reference arm's keys; no GPU is touched."""
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "1"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s" and d["value"] > 0
+    assert d["dtype"] == "f64" and d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
