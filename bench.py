@@ -920,9 +920,16 @@ def cpu_baseline(step: Step, min_seconds: float = 10.0, max_reps: int = 20) -> d
         total += dt
         nbytes += b
         reps += 1
+    # the same oracle on one thread, over the first 1/16 of every segment's
+    # and of the activation rows (about a second)
+    s1, a1 = oracle_sample(step.wg["model"], step.ag["x"], 1.0 / 16)
+    dt1, b1 = time_oracle_step(s1, a1, 1)
     return {"value": round(nbytes / total / 1e9, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
             "sample": f"the whole step (all six calls on every weight segment and all activation rows, "
-                      f"{nbytes / reps / 1e6:.0f} MB algorithmic) x {reps}, {total:.1f} s wall"}
+                      f"{nbytes / reps / 1e6:.0f} MB algorithmic) x {reps}, {total:.1f} s wall",
+            "single_thread": {"value": round(b1 / dt1 / 1e9, 3), "unit": "GB/s", "cores": 1,
+                              "sample": f"the first 1/16 of every segment's rows and of the activation rows "
+                                        f"({b1 / 1e6:.0f} MB algorithmic) x 1, {dt1:.1f} s wall"}}
 
 
 def run_reference(args, rank: int, world: int) -> None:
