@@ -589,8 +589,8 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
             const int64_t K = segs[i].cols / gsize(i);   // stored rows
             for (const int budget : ds::kColTileBudgets) {
                 for (const int cl : {1, 2, 4, 8}) {
-                    for (const int ct : {128, 64, 32})
-                        if (ds::col_tile_smem(ct, cl, (K + cl - 1) / cl, eb) <= budget) {
+                    for (const int ct : {128, 64, 32, 16})
+                        if (ct >= gsize(i) && ds::col_tile_smem(ct, cl, (K + cl - 1) / cl, eb) <= budget) {
                             ct_of[i] = ct;
                             cl_of[i] = cl;
                             break;
@@ -602,7 +602,7 @@ ds_status run_weight(WOp wop, const ds_wseg *segs, int nseg, ds_dtype dt, float 
                     break;
             }
         }
-        for (const int ct : {128, 64, 32, 0})
+        for (const int ct : {128, 64, 32, 16, 0})
             for (const int cl : {1, 2, 4, 8}) {
                 if (ct == 0 && cl != 1)
                     continue;

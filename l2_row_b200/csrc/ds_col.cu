@@ -733,6 +733,7 @@ template <int OP, bool B16>
 cudaError_t launch_colt_ct(const ColtParams &p, int64_t units, int ct, int cl, int smem, cudaStream_t st)
 {
     switch (ct) {
+    case 16: return launch_colt_t<OP, B16, 16>(p, units, cl, smem, st);
     case 32: return launch_colt_t<OP, B16, 32>(p, units, cl, smem, st);
     case 64: return launch_colt_t<OP, B16, 64>(p, units, cl, smem, st);
     case 128: return launch_colt_t<OP, B16, 128>(p, units, cl, smem, st);
@@ -779,19 +780,25 @@ int col_tile_rows() { return kColTile; }
 
 // Rows per box: the band in as few boxes of at most 256 rows (the TMA box
 // limit) as possible, all of one height, so that no box reaches far into
-// the next band.
-int col_tile_box_rows(int64_t band)
+// the next band.  A tensor copy's shared-memory destination must start on
+// 128 bytes, so the height is a multiple of the rows that fill 128 bytes at
+// the narrowest staged row (CT bf16 elements of a bf16 GY): 4 rows at CT =
+// 16, 2 at CT = 32; every box of w and of the second input then starts on
+// 128 bytes.  (Rows a box takes past the band are ignored.)
+int col_tile_box_rows(int64_t band, int ct)
 {
     if (band <= 0)
         return 1;
     const int64_t nbox = (band + 255) / 256;
-    return static_cast<int>((band + nbox - 1) / nbox);
+    const int64_t m = ct * 2 >= 128 ? 1 : 128 / (ct * 2);
+    const int64_t bh = (band + nbox - 1) / nbox;
+    return static_cast<int>((bh + m - 1) / m * m);
 }
 
 int col_tile_smem(int ct, int cl, int64_t band, int elem_bytes)
 {
     (void)cl;
-    const int64_t bh = col_tile_box_rows(band);
+    const int64_t bh = col_tile_box_rows(band, ct);
     const int64_t rows = band > 0 ? (band + bh - 1) / bh * bh : 0;
     const int64_t tile = rows * ct * elem_bytes;
     const int64_t xch = int64_t(2) * kMaxCluster * ct * 8;
@@ -842,7 +849,7 @@ int launch_colt(int op, bool b16, int ct, int cl, int smem, const WParams &w, in
         const WSegK &sg = w.seg[i];
         const int64_t G = sg.group > 1 ? sg.group : 1;
         const int64_t K = sg.cols / G, N = sg.rows * G, band = (K + cl - 1) / cl;
-        const int bh = col_tile_box_rows(band);
+        const int bh = col_tile_box_rows(band, ct);
         p.seg[i] = sg;
         p.unit_start[i] = w.unit_start[i];
         p.box_h[i] = bh;

@@ -250,7 +250,7 @@ int col_tile_rows();
 int col_group_units(int group);
 int launch_colg(int op, bool b16, const WParams &p, int64_t units, void *stream);
 // Transposed rows in whole column tiles (ds_col.cu): tiles of ct unit rows
-// (32, 64 or 128) over every stored row, a cluster of cl CTAs per tile
+// (16, 32, 64 or 128) over every stored row, a cluster of cl CTAs per tile
 // (bands of ceil(K / cl) stored rows each, loaded as 2-D TMA boxes); p's
 // unit_start counts tiles; at most col_tile_segments() segments.
 // Dynamic shared memory of a launch: col_tile_smem(ct, cl, largest band,

@@ -18,12 +18,14 @@ from tests import gpu_util as gu
 pytestmark = pytest.mark.gpu
 
 # (stored rows = in, stored cols = out): GPT-2 small's Conv1D shapes,
-# GPT-2 XL's MLP pair (c_fc [1600, 6400]: tiles over clusters of 8 with two
-# or three CTAs per SM; c_proj [6400, 1600]: 32-column tiles, one CTA per
-# SM), ragged ones (out not a multiple of 4; one output channel), and one too
-# tall for eight CTAs' shared memory, which takes the column kernel
+# GPT-2 XL's MLP pair ([1600, 6400] and [6400, 1600]: narrow tiles over
+# clusters), ragged ones (out not a multiple of 4; one output channel), bands
+# whose box heights must be rounded so that every TMA box starts on 128 bytes
+# ([13000, 24]: 16-column tiles in boxes of 236 rows; [301, 40]: 32-column
+# tiles, a bf16 GY in two boxes), and one too tall for eight CTAs' shared
+# memory, which takes the column kernel ([30000, 8])
 SHAPES = [(768, 2304), (768, 768), (768, 3072), (3072, 768), (1600, 6400), (6400, 1600), (100, 13), (7, 1),
-          (5, 6), (13000, 24)]
+          (5, 6), (13000, 24), (301, 40), (30000, 8)]
 
 
 def _stored(rng, K, N, ld_pad=0):
